@@ -1,0 +1,378 @@
+#!/usr/bin/env python
+"""Throughput of the ALBERT phoneme-encoder forward pass on B200 (one JSON line).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one whole forward pass (embedding + LN, 128->768 projection, 12
+executions of the shared layer, 768->512 projection) over one synthetic batch:
+by default 256 sequences padded to T=128 with lengths uniform in [16, 128],
+packed by length inside the library.  `value` counts valid tokens per second
+over all ranks; every rank runs its own batch (sequences are independent:
+weak scaling, no collective on the data path).  L2 is flushed (512 MiB write)
+between timed steps; step times are CUDA-event times of the forward alone,
+max over ranks.
+
+`--impl reference` times the fp64 CPU oracle on the host cores instead (each
+step: one sequence of the same workload), rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "encoder tokens/sec (BF16, 1×B200) and % of dense BF16 tensor peak"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------- accounting ----
+
+def flops_per_class(lengths, arch, rows):
+    """Algorithmic FLOPs of one launch of each kernel class.  `rows` = rows the
+    GEMMs process (valid tokens when packed); attention counts valid keys only."""
+    H, E, F, O = arch["hidden"], arch["emb"], arch["ffn"], arch["out_dim"]
+    s2 = float(sum(int(l) ** 2 for l in lengths))
+    return {
+        "gemm_in_proj": 2.0 * rows * E * H,
+        "gemm_qkv": 2.0 * rows * H * 3 * H,
+        "attention": 4.0 * s2 * H,
+        "gemm_out_proj_ln": 2.0 * rows * H * H,
+        "gemm_ffn_up_gelu": 2.0 * rows * H * F,
+        "gemm_ffn_down_ln": 2.0 * rows * F * H,
+        "gemm_final_proj": 2.0 * rows * H * O,
+    }
+
+
+def forward_flops(lengths, arch):
+    n_tok = int(sum(int(l) for l in lengths))
+    f = flops_per_class(lengths, arch, n_tok)
+    per_exec = f["gemm_qkv"] + f["attention"] + f["gemm_out_proj_ln"] + f["gemm_ffn_up_gelu"] + f["gemm_ffn_down_ln"]
+    gemm = f["gemm_in_proj"] + f["gemm_final_proj"] + arch["n_exec"] * (per_exec - f["attention"])
+    return gemm + arch["n_exec"] * f["attention"], gemm
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks -----
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.t is not None:
+                self.t.join(timeout=2)
+
+    def summary(self, t0, t1):
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            rows.append((ts, parts))
+        inside = [p for ts, p in rows if t0 <= ts <= t1] or [p for _, p in rows]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[0]) for p in inside if num(p[0]) is not None]
+        mx = [num(p[1]) for p in inside if num(p[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for p in inside for i in range(4) if p[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(inside)}
+
+
+# -------------------------------------------------------------- oracle arm ---
+
+def oracle_throughput(weights, ids, mask, L, arch, budget_s=None, steps=None, warmup=0):
+    """Time the fp64 CPU oracle, one sequence per step (round robin over the batch)."""
+    import oracle
+    oracle.set_threads(os.cpu_count() or 1)
+    m = oracle.Model(weights, arch)
+    order = list(range(len(L)))
+    tok, secs, done, i = 0, 0.0, 0, 0
+    for _ in range(warmup):
+        b = order[i % len(order)]; i += 1
+        m.encode(ids[b, :L[b]], mask[b, :L[b]])
+    while True:
+        b = order[i % len(order)]; i += 1
+        t0 = time.perf_counter()
+        m.encode(ids[b, :L[b]], mask[b, :L[b]])
+        secs += time.perf_counter() - t0
+        tok += int(L[b])
+        done += 1
+        if steps is not None and done >= steps:
+            break
+        if budget_s is not None and secs >= budget_s:
+            break
+    return tok / secs, done, tok, secs, oracle.num_threads()
+
+
+def run_reference(args):
+    import synth
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = synth.WORKLOADS[args.workload]
+    w = synth.make_weights(seed=1234, bf16=True)
+    ids, mask, L = synth.make_batch(wl)
+    value, done, tok, secs, cores = oracle_throughput(w, ids, mask, L, synth.ARCH, steps=args.steps,
+                                                      warmup=args.warmup)
+    sample = f"{done} whole sequences of the {wl.name} batch ({tok} valid tokens), one per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * secs / max(done, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,0.02) weights rounded to bf16, seeded ids and lengths)",
+        "config": {"workload": wl.name, "batch": wl.B, "seq_len": wl.T, "lengths": wl.describe()},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm ----
+
+def run_gpu(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    import transformer_encoder_albert_b200 as tea
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            raise SystemExit("--gpus N > 1 needs torchrun with N processes")
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return float(t.item())
+
+    arch = synth.ARCH
+    wl = synth.WORKLOADS[args.workload]
+    w = synth.make_weights(seed=1234, bf16=True)
+    ids, mask, L = synth.make_batch(wl, seed=wl.seed + 1000 * rank)
+    n_tok = int(L.sum())
+    ids_d = torch.as_tensor(ids).cuda()
+    mask_d = torch.as_tensor(mask).cuda()
+    enc = tea.Encoder(w, arch, dtype="bf16", max_tokens=wl.B * wl.T, pack=not args.padded)
+    out = torch.empty(wl.B, wl.T, arch["out_dim"], device="cuda", dtype=torch.bfloat16)
+    stream = torch.cuda.current_stream()
+    rows = n_tok if not args.padded else wl.B * wl.T
+    per_launch = flops_per_class(L, arch, rows)
+    fwd_flops, gemm_flops = forward_flops(L, arch)
+
+    # which kernel dominates: a short all-class profile before the timed region
+    enc.profile(None)
+    for _ in range(3):
+        enc.forward(ids_d, mask_d, out)
+    prof0 = enc.profile_read()
+    enc.profile([])
+    enc.profile_reset()
+    dominant = max(prof0, key=lambda k: prof0[k][1])
+
+    for _ in range(args.warmup):
+        enc.forward(ids_d, mask_d, out)
+    if enc.status() != 0:
+        raise SystemExit(f"device status {enc.status()}")
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+
+    gpu_id = getattr(torch.cuda.get_device_properties(local), "pci_bus_id", None) or str(local)
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.5)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    enc.profile([dominant])  # only the dominant class is timed live
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for k in range(args.steps):
+        flush.zero_()
+        starts[k].record(stream)
+        enc.forward(ids_d, mask_d, out)
+        ends[k].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    sampler.stop()
+    st = enc.status()
+    if st != 0:
+        raise SystemExit(f"device status {tea.STATUS_NAMES.get(st, st)}")
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    dom = enc.profile_read()[dominant]
+    enc.profile([])
+    enc.profile_reset()
+    total_ms = max_over_ranks(sum(step_ms))
+    tokens_all = sum_over_ranks(float(n_tok * args.steps))
+    value = tokens_all / (total_ms / 1000.0)
+    ms_per_step = total_ms / args.steps
+
+    # per-kernel breakdown: a profiled replay of a few steps (all classes)
+    enc.profile(None)
+    n_prof = min(args.steps, 10)
+    for _ in range(n_prof):
+        flush.zero_()
+        enc.forward(ids_d, mask_d, out)
+    prof = enc.profile_read()
+    enc.profile([])
+    gemm_classes = [c for c in prof if c.startswith("gemm_")]
+    gemm_ms = sum(prof[c][1] for c in gemm_classes) / n_prof
+    breakdown = {c: {"launches_per_step": prof[c][0] / n_prof, "ms_per_step": prof[c][1] / n_prof}
+                 for c in prof if prof[c][0]}
+
+    # end to end through the public C call with host buffers
+    ids_h = torch.as_tensor(ids).pin_memory()
+    mask_h = torch.as_tensor(mask).pin_memory()
+    out_h = torch.empty(wl.B, wl.T, arch["out_dim"], dtype=torch.bfloat16).pin_memory()
+    n_e2e = args.steps
+    e_s = torch.cuda.Event(enable_timing=True)
+    e_e = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e_s.record(stream)
+    for _ in range(n_e2e):
+        rc = enc.forward_host(ids_h, mask_h, out_h)
+        if rc != 0:
+            raise SystemExit(f"forward_host status {rc}")
+    e_e.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e_s.elapsed_time(e_e))
+    e2e_value = sum_over_ranks(float(n_tok * n_e2e)) / (e2e_ms / 1000.0)
+
+    peaks, peaks_src = load_peaks()
+    peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    dom_ms = dom[1] / max(dom[0], 1)
+    achieved = per_launch.get(dominant, 0.0) / (dom_ms / 1000.0) / 1e12
+    roofline = {"kernel": dominant, "bound": "tensor", "achieved": achieved, "peak": peak_sus,
+                "unit": "TFLOP/s", "frac": achieved / peak_sus, "traffic": None,
+                "peak_source": f"{peaks_src} bf16_tflops_sustained (kernel timed inside back-to-back forwards)",
+                "launches_timed": dom[0], "avg_launch_ms": dom_ms,
+                "flops_per_launch": per_launch.get(dominant, 0.0)}
+    clocks = sampler.summary(t_wall0, t_wall1)
+    launches = enc.launches_per_forward(True)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02) weights rounded to bf16, seeded ids and lengths)",
+        "config": {"workload": wl.name + ("_padded" if args.padded else "_packed"), "batch": wl.B,
+                   "seq_len": wl.T, "lengths": wl.describe(), "valid_tokens_per_step_per_gpu": n_tok,
+                   "pack": not args.padded, "parallelism": f"replicas x{world}",
+                   "l2": "flushed between timed steps (512 MiB write)"},
+        "tensor_peak_frac": {"whole_encoder": fwd_flops / (ms_per_step / 1000.0) / 1e12 / peak_sus,
+                             "gemm_path": gemm_flops / (gemm_ms / 1000.0) / 1e12 / peak_sus,
+                             "peak_tflops": peak_sus, "peak_source": peaks_src},
+        "roofline": roofline,
+        "kernels": breakdown,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(ids_h.numel() * 8 + mask_h.numel()),
+                "d2h_bytes_per_step": int(out_h.numel() * 2), "api": "albert_forward_host"},
+        "gpu_launches": launches * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, done, tok, secs, cores = oracle_throughput(w, ids, mask, L, arch, budget_s=args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"{done} whole sequences of the same batch ({tok} valid tokens, "
+                                          f"{secs:.1f} s of fp64 CPU work)"}
+    enc.close()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="b256_T128")
+    ap.add_argument("--padded", action="store_true", help="run the GEMMs on all B*T padded rows")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

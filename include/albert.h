@@ -1,0 +1,189 @@
+/*
+ * albert.h -- C ABI of the B200 (sm_100a) forward pass of Kokoro's ALBERT
+ * phoneme encoder.
+ *
+ * What the library computes ("ALBERT: How Kokoro's Phoneme Encoder Works, and
+ * Where CKE Has Reached It", section "Inside One Real ALBERT Layer", steps 1-6
+ * and the paragraph after them):
+ *   E  = LN_128(word[id] + pos[t] + type[0])            (three-table embedding)
+ *   X  = E W_in^T + b_in                                 (128 -> 768)
+ *   repeat n_exec times with ONE shared weight set:
+ *     [Q|K|V] = X [Wq;Wk;Wv]^T + b
+ *     C  = per head h (64 columns each): softmax(Q_h K_h^T / 8 + mask) V_h
+ *     X1 = LN(X + C Wo^T + bo)
+ *     X  = LN(X1 + GELU_tanh(X1 W1^T + b1) W2^T + b2)
+ *   Y  = X W_out^T + b_out                               (768 -> 512)
+ * The mask is a key-padding mask: slot u of sequence b takes part only if
+ * u < L_b ("How Kokoro TTS Works and Where CKE Stands", section "What ALBERT
+ * does here": softmax(QK^T/sqrt(d) + mask) V).  Positions are slot indices
+ * 0..T-1 (right padding); token type 0.
+ *
+ * Conventions (from "How Kokoro TTS Works and Where CKE Stands", sections on
+ * checked kernels and the compiler side: integer status, validate before
+ * writing, caller-owned memory planned up front):
+ *   - every call returns an int status, ALBERT_OK (0) on success;
+ *   - host-detected errors return before anything is enqueued, so `out` is
+ *     untouched;
+ *   - device-detected errors (bad id, bad mask, bad sequence lengths, an
+ *     expired bounded wait) are recorded in a device status word; every later
+ *     kernel of the same forward then exits without writing, so `out` is left
+ *     as it was.  albert_get_status() reports that word;
+ *   - all memory the forward pass needs is allocated by albert_create();
+ *     albert_forward() and albert_forward_varlen() allocate nothing.
+ *
+ * All device pointers are CUDA device addresses on the device that was current
+ * when the handle was created.  `stream` is a cudaStream_t passed as void*
+ * (NULL = legacy default stream).  A handle may be used from one stream at a
+ * time; two forwards that overlap on different streams race on its workspace.
+ */
+#ifndef ALBERT_B200_H
+#define ALBERT_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---- */
+#define ALBERT_OK           0
+#define ALBERT_ERR_NULL     1  /* a required pointer is NULL                        */
+#define ALBERT_ERR_CONFIG   2  /* unsupported albert_config                         */
+#define ALBERT_ERR_SHAPE    3  /* B, T, nseq, max_len or token count out of range   */
+#define ALBERT_ERR_ID       4  /* device: a valid slot holds an id outside [0,vocab) */
+#define ALBERT_ERR_MASK     5  /* device: a mask row is not a non-empty 1..1 0..0 prefix */
+#define ALBERT_ERR_SEQLENS  6  /* device: cu_seqlens not 0-based / lengths outside [1, max_pos] */
+#define ALBERT_ERR_CUDA     7  /* a CUDA runtime call failed                        */
+#define ALBERT_ERR_TIMEOUT  8  /* device: a bounded wait inside a kernel expired    */
+#define ALBERT_ERR_ALLOC    9  /* device memory allocation failed in albert_create  */
+
+/* ---- precision of the whole path ---- */
+#define ALBERT_BF16 0  /* bf16 weights and activations, fp32 accumulation and norms */
+#define ALBERT_FP32 1  /* fp32 everywhere (SIMT kernels; small workloads)          */
+
+/* Architecture and capacity.  The kernels support exactly: emb 128, hidden 768,
+ * heads 12 (64 wide), ffn 2048, max_pos <= 512, out_dim 512 or 0 (0 = return the
+ * [.., 768] hidden states), n_groups 1 (one fully shared layer).  n_exec >= 0
+ * is free.  max_tokens is the workspace capacity in rows: albert_forward needs
+ * B*T <= max_tokens, albert_forward_varlen needs total tokens <= max_tokens. */
+typedef struct {
+    int vocab;       /* 178 for Kokoro                                  */
+    int emb;         /* E = 128                                         */
+    int hidden;      /* H = 768                                         */
+    int heads;       /* 12                                              */
+    int ffn;         /* 2048                                            */
+    int n_exec;      /* executions of the shared layer, 12 for Kokoro   */
+    int n_groups;    /* distinct layer weight sets; must be 1           */
+    int max_pos;     /* rows of the position table, <= 512              */
+    int n_types;     /* rows of the token-type table (type 0 is used)   */
+    int out_dim;     /* 512, or 0 for no final projection               */
+    int dtype;       /* ALBERT_BF16 or ALBERT_FP32                      */
+    int max_tokens;  /* workspace capacity in rows (>= 1)               */
+    int pack;        /* albert_forward: 1 = pack valid tokens by length
+                        (the GEMMs run on sum(L_b) rows), 0 = run on all B*T
+                        padded rows                                     */
+    float ln_eps;    /* LayerNorm epsilon, 1e-12 for Kokoro             */
+} albert_config;
+
+/* Parameters: DEVICE pointers to fp32 tensors in PyTorch layouts ([out, in] for
+ * linears).  albert_create copies them (converting to bf16 for ALBERT_BF16), so
+ * the caller may free them afterwards.  w_out/b_out may be NULL if out_dim == 0. */
+typedef struct {
+    const float *word;      /* [vocab, emb]     */
+    const float *pos;       /* [max_pos, emb]   */
+    const float *type;      /* [n_types, emb]   */
+    const float *emb_ln_g;  /* [emb]            */
+    const float *emb_ln_b;  /* [emb]            */
+    const float *w_in;      /* [hidden, emb]    */
+    const float *b_in;      /* [hidden]         */
+    const float *wq, *bq;   /* [hidden, hidden], [hidden] */
+    const float *wk, *bk;
+    const float *wv, *bv;
+    const float *wo, *bo;
+    const float *ln1_g, *ln1_b;  /* [hidden]    */
+    const float *w1, *b1;   /* [ffn, hidden], [ffn]       */
+    const float *w2, *b2;   /* [hidden, ffn], [hidden]    */
+    const float *ln2_g, *ln2_b;
+    const float *w_out, *b_out;  /* [out_dim, hidden], [out_dim] */
+} albert_weights;
+
+typedef struct albert_handle albert_handle;
+
+/* Validate cfg, copy/pack the weights, allocate the workspace for max_tokens
+ * rows and build the TMA descriptors.  Synchronous.  On success *out receives
+ * the handle; on failure *out is NULL and nothing stays allocated. */
+int albert_create(const albert_weights *w, const albert_config *cfg, albert_handle **out);
+
+/* Padded batch.  ids: [B, T] int64 (device); mask: [B, T] uint8 (device),
+ * 1 = token, each row a non-empty prefix of ones; out: [B, T, D] (device),
+ * D = out_dim or hidden, bf16 for ALBERT_BF16 and fp32 for ALBERT_FP32.
+ * Rows at padding slots are written as zeros.  Ids at padding slots are not
+ * read for the result and may hold anything.  Asynchronous on `stream`.
+ * Host errors: NULL pointers, B < 1, T < 1, T > max_pos, B*T > max_tokens. */
+int albert_forward(albert_handle *h, const int64_t *ids, const uint8_t *mask, int B, int T,
+                   void *out, void *stream);
+
+/* Packed variable-length batch.  ids: [N_tok] int64 (device), the sequences
+ * back to back; cu_seqlens: [nseq+1] int32 (device), cu_seqlens[0] = 0,
+ * sequence s = rows cu_seqlens[s] .. cu_seqlens[s+1]-1, each length in
+ * [1, max_pos] and N_tok = cu_seqlens[nseq] <= max_tokens (checked on the
+ * device); out: [N_tok, D] (device).  max_len bounds every length (host check
+ * max_len <= max_pos; the device checks each length against it).
+ * Asynchronous on `stream`. */
+int albert_forward_varlen(albert_handle *h, const int64_t *ids, const int32_t *cu_seqlens,
+                          int nseq, int max_len, void *out, void *stream);
+
+/* Convenience path with HOST buffers: copies ids/mask (pinned or pageable) to
+ * the handle's device staging area, runs albert_forward, copies the result
+ * back to out_host and synchronizes `stream`.  Returns the device status. */
+int albert_forward_host(albert_handle *h, const int64_t *ids_host, const uint8_t *mask_host,
+                        int B, int T, void *out_host, void *stream);
+
+/* Synchronize `stream` and return the status recorded by the last forward on
+ * this handle (ALBERT_OK, ALBERT_ERR_ID, _MASK, _SEQLENS, _SHAPE or _TIMEOUT). */
+int albert_get_status(albert_handle *h, void *stream);
+
+/* Free everything the handle owns.  NULL is ignored. */
+void albert_destroy(albert_handle *h);
+
+/* Number of kernel launches one forward of this handle enqueues for a batch
+ * with the given shape (used to report launches per step). */
+int albert_launches_per_forward(const albert_handle *h, int padded_api);
+
+/* ---- per-kernel timing (optional) ----
+ * albert_profile_enable(h, class_mask): for every kernel class whose bit is set
+ * in class_mask (-1 = all, 0 = off), each forward records a CUDA event before
+ * and after each launch of that class on the forward's stream.  albert_profile_read synchronizes the
+ * last recorded stream and adds, per kernel class, the launch count and the
+ * summed milliseconds since the last reset.  Classes are numbered
+ * 0..albert_profile_classes()-1 and named by albert_profile_name(). */
+int albert_profile_enable(albert_handle *h, int class_mask);
+int albert_profile_reset(albert_handle *h);
+int albert_profile_classes(void);
+const char *albert_profile_name(int cls);
+int albert_profile_read(albert_handle *h, int *launches, double *ms);
+
+/* ---- single-kernel entry points (parity tests of one kernel) ----
+ * These run one kernel of the path in isolation, synchronously, and return its
+ * status.  They allocate and free temporary device memory. */
+
+/* Y = epilogue(A W^T + bias) with the tcgen05 GEMM.  A: [M, K] bf16, W: [N, K]
+ * bf16, bias: [N] fp32 (device).  epi: 0 = bias -> bf16 Y[M, N];
+ * 1 = tanh-GELU(+bias) -> bf16; 2 = LN(A W^T + bias + R; g, b, eps) -> bf16,
+ * with R: [M, N] bf16 and N == 768; 3 = bias -> bf16 rows scattered to
+ * row_dst[r] (row_dst[r] < 0 skips the row).  K % 64 == 0, N % 256 == 0. */
+int albert_test_gemm(const void *A, const void *W, const float *bias, const void *R,
+                     const float *ln_g, const float *ln_b, float eps, const int32_t *row_dst,
+                     void *Y, int M, int N, int K, int epi, void *stream);
+
+/* Masked bidirectional attention on a packed [N_tok, 3*768] bf16 QKV buffer
+ * (Q | K | V, head h = columns 64h..64h+63 of each); cu_seqlens as in
+ * albert_forward_varlen; ctx: [N_tok, 768] bf16.  dtype ALBERT_FP32 runs the
+ * fp32 kernel on fp32 buffers instead. */
+int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, int max_len,
+                          void *ctx, int dtype, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ALBERT_B200_H */

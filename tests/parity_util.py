@@ -1,0 +1,58 @@
+"""Helpers shared by the parity tests: tolerances and oracle sampling.
+
+Tolerances (stated for the encoder output over valid tokens):
+  bf16 path: max |gpu - oracle| <= 3e-2 and per-token cosine >= 0.999;
+  fp32 path: ||gpu - oracle||_inf / ||oracle||_inf <= 1e-4.
+"""
+import numpy as np
+
+import oracle
+import synth
+
+BF16_MAX_ABS = 3e-2
+BF16_MIN_COS = 0.999
+FP32_REL = 1e-4
+
+
+def per_token_cosine(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    a = a.astype(np.float64)
+    b = b.astype(np.float64)
+    return (a * b).sum(-1) / (np.linalg.norm(a, axis=-1) * np.linalg.norm(b, axis=-1) + 1e-300)
+
+
+def check_bf16(gpu: np.ndarray, ref: np.ndarray, what: str = ""):
+    err = float(np.max(np.abs(gpu.astype(np.float64) - ref)))
+    cos = float(np.min(per_token_cosine(gpu, ref)))
+    assert np.all(np.isfinite(gpu)), f"{what}: non-finite output"
+    assert err <= BF16_MAX_ABS, f"{what}: max abs err {err:.3e} > {BF16_MAX_ABS}"
+    assert cos >= BF16_MIN_COS, f"{what}: min per-token cosine {cos:.6f} < {BF16_MIN_COS}"
+    return err, cos
+
+
+def check_fp32(gpu: np.ndarray, ref: np.ndarray, what: str = ""):
+    rel = float(np.max(np.abs(gpu.astype(np.float64) - ref)) / np.max(np.abs(ref)))
+    assert np.all(np.isfinite(gpu)), f"{what}: non-finite output"
+    assert rel <= FP32_REL, f"{what}: relative error {rel:.3e} > {FP32_REL}"
+    return rel
+
+
+def sample_sequences(L: np.ndarray, k: int, seed: int = 0) -> list:
+    """The longest and shortest sequence plus k-2 others drawn with a seed."""
+    L = np.asarray(L)
+    idx = {int(np.argmax(L)), int(np.argmin(L))}
+    rng = np.random.default_rng(seed)
+    rest = [i for i in range(len(L)) if i not in idx]
+    rng.shuffle(rest)
+    idx.update(rest[: max(0, k - len(idx))])
+    return sorted(idx)
+
+
+def oracle_rows(weights: dict, ids: np.ndarray, mask: np.ndarray, L: np.ndarray, seqs, n_exec=None,
+                out_dim=None) -> dict:
+    """Oracle outputs of the valid rows of the chosen sequences (each alone, unpadded)."""
+    m = oracle.Model(weights, synth.ARCH, n_exec=n_exec, out_dim=out_dim)
+    out = {}
+    for b in seqs:
+        n = int(L[b])
+        out[b] = m.encode(ids[b, :n], mask[b, :n])
+    return out

@@ -1,0 +1,76 @@
+"""CPU checks of the boundary: the library builds, loads and exports every
+function include/albert.h declares; the Python binding's structs and status
+codes agree with the header.  No compute call is made (no GPU here)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import transformer_encoder_albert_b200 as tea
+from transformer_encoder_albert_b200 import build as tea_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "albert.h")
+
+
+def _header():
+    with open(HEADER) as f:
+        return f.read()
+
+
+def _declared_functions():
+    text = re.sub(r"/\*.*?\*/", "", _header(), flags=re.S)
+    return sorted(set(re.findall(r"\b(albert_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    tea_build.build()
+    return C.CDLL(tea.LIB_PATH)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = _declared_functions()
+    assert "albert_create" in names and "albert_forward" in names and "albert_destroy" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(tea.EXPORTS)
+
+
+def test_status_codes_match_header():
+    codes = dict((m[0], int(m[1])) for m in re.findall(r"#define (ALBERT_(?:OK|ERR_\w+))\s+(\d+)", _header()))
+    for code, name in tea.STATUS_NAMES.items():
+        assert codes[name] == code
+
+
+def test_config_struct_matches_header_field_order():
+    text = _header()
+    body = re.search(r"typedef struct \{(.*?)\} albert_config;", text, re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = re.findall(r"\b(\w+)\s*;", body)
+    assert fields == [f for f, _ in tea.albert_config._fields_]
+    assert C.sizeof(tea.albert_config) == 14 * 4
+
+
+def test_weights_struct_matches_header_field_order():
+    body = re.search(r"typedef struct \{(.*?)\} albert_weights;", _header(), re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = re.findall(r"\*\s*(\w+)", body)
+    assert tuple(fields) == tea.WEIGHT_FIELDS
+
+
+def test_library_is_built_for_sm100a_only():
+    assert "arch=compute_100a,code=sm_100a" in " ".join(tea_build.FLAGS)
+
+
+def test_host_side_rejections_need_no_gpu(lib):
+    """Null pointers are rejected before any CUDA call."""
+    lib.albert_create.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p]
+    assert lib.albert_create(None, None, None) == 1
+    h = C.c_void_p()
+    assert lib.albert_create(None, None, C.byref(h)) == 1 and h.value is None
+    lib.albert_forward.argtypes = [C.c_void_p] * 3 + [C.c_int, C.c_int, C.c_void_p, C.c_void_p]
+    assert lib.albert_forward(None, None, None, 1, 1, None, None) == 1
+    lib.albert_destroy.argtypes = [C.c_void_p]
+    lib.albert_destroy(None)

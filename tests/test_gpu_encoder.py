@@ -1,0 +1,232 @@
+"""Whole-encoder parity on the GPU, through the C ABI, against the fp64 oracle.
+
+Every workload of the suite runs at its full size on the GPU; the oracle
+recomputes a seeded sample of whole sequences (sequences are independent, so
+a sample of sequences is a sample of outputs), always including the longest
+and the shortest.  Padding rows must be exactly zero.  Error paths must leave
+the output byte-identical to its sentinel fill.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+import transformer_encoder_albert_b200 as tea
+from parity_util import check_bf16, check_fp32, oracle_rows, sample_sequences
+
+pytestmark = pytest.mark.gpu
+A = synth.ARCH
+
+
+@pytest.fixture(scope="module")
+def w_bf16():
+    return synth.make_weights(seed=1234, bf16=True)
+
+
+@pytest.fixture(scope="module")
+def w_fp32():
+    return synth.make_weights(seed=1234, bf16=False)
+
+
+def _t(a, dtype=None):
+    return torch.as_tensor(a).to("cuda") if dtype is None else torch.as_tensor(a).to("cuda", dtype)
+
+
+def _run(weights, wl, dtype="bf16", pack=True, n_exec=None, out_dim=None, max_tokens=None):
+    ids, mask, L = synth.make_batch(wl)
+    enc = tea.Encoder(weights, A, dtype=dtype, max_tokens=max_tokens or wl.B * wl.T, pack=pack,
+                      n_exec=n_exec, out_dim=wl.out_dim if out_dim is None else out_dim)
+    out = enc.forward(_t(ids), _t(mask))
+    st = enc.status()
+    enc.close()
+    assert st == 0, tea.STATUS_NAMES[st]
+    return ids, mask, L, out.float().cpu().numpy()
+
+
+def _compare(weights, wl, got, ids, mask, L, seqs, fp32=False, n_exec=None, out_dim=None):
+    ref = oracle_rows(weights, ids, mask, L, seqs, n_exec=n_exec,
+                      out_dim=wl.out_dim if out_dim is None else out_dim)
+    for b in seqs:
+        n = int(L[b])
+        if fp32:
+            check_fp32(got[b, :n], ref[b], f"{wl.name} seq {b}")
+        else:
+            check_bf16(got[b, :n], ref[b], f"{wl.name} seq {b} (L={n})")
+    for b in range(len(L)):
+        assert np.all(got[b, int(L[b]):] == 0.0), f"padding rows of seq {b} not zero"
+
+
+def test_tiny_fp32_T36(w_fp32):
+    wl = synth.WORKLOADS["tiny_fp32_T36"]
+    ids, mask, L, got = _run(w_fp32, wl, dtype="fp32")
+    _compare(w_fp32, wl, got, ids, mask, L, [0], fp32=True)
+
+
+@pytest.mark.parametrize("pack", [True, False])
+def test_b8_T128_all_sequences(w_bf16, pack):
+    wl = synth.WORKLOADS["b8_T128"]
+    ids, mask, L, got = _run(w_bf16, wl, pack=pack)
+    _compare(w_bf16, wl, got, ids, mask, L, list(range(wl.B)))
+
+
+def test_b64_T128_normal_lengths(w_bf16):
+    wl = synth.WORKLOADS["b64_T128_normal"]
+    ids, mask, L, got = _run(w_bf16, wl)
+    _compare(w_bf16, wl, got, ids, mask, L, sample_sequences(L, 6, seed=2))
+
+
+def test_b32_T512_long(w_bf16):
+    wl = synth.WORKLOADS["b32_T512_long"]
+    ids, mask, L, got = _run(w_bf16, wl)
+    _compare(w_bf16, wl, got, ids, mask, L, sample_sequences(L, 2, seed=3))
+
+
+@pytest.mark.parametrize("pack", [True, False])
+def test_b256_T128_throughput_config(w_bf16, pack):
+    wl = synth.WORKLOADS["b256_T128"]
+    ids, mask, L, got = _run(w_bf16, wl, pack=pack)
+    _compare(w_bf16, wl, got, ids, mask, L, sample_sequences(L, 4, seed=4))
+
+
+def test_b1_T64_latency(w_bf16):
+    wl = synth.WORKLOADS["b1_T64_latency"]
+    ids, mask, L, got = _run(w_bf16, wl)
+    _compare(w_bf16, wl, got, ids, mask, L, [0])
+
+
+@pytest.mark.parametrize("n_exec", [0, 1, 2])
+def test_stage_checkpoints_hidden_states(w_bf16, n_exec):
+    """Connected checkpoints: the [T, 768] states after the embedding + input
+    projection (n_exec=0) and after one and two shared-layer executions."""
+    wl = synth.Workload("stages", 4, 96, "uniform", lo=5, hi=96, seed=77)
+    ids, mask, L, got = _run(w_bf16, wl, n_exec=n_exec, out_dim=0)
+    _compare(w_bf16, wl, got, ids, mask, L, list(range(wl.B)), n_exec=n_exec, out_dim=0)
+
+
+def test_random_layer_norm_affine_catches_swaps():
+    w = synth.make_weights(seed=99, bf16=True, ln_affine="random")
+    wl = synth.Workload("affine", 3, 64, "uniform", lo=10, hi=64, seed=78)
+    ids, mask, L, got = _run(w, wl, n_exec=3)
+    _compare(w, wl, got, ids, mask, L, list(range(wl.B)), n_exec=3)
+
+
+def test_fp32_small_padded_batch(w_fp32):
+    wl = synth.Workload("fp32b", 3, 40, "uniform", lo=2, hi=40, seed=79, dtype="fp32", out_dim=512)
+    ids, mask, L, got = _run(w_fp32, wl, dtype="fp32", n_exec=3)
+    _compare(w_fp32, wl, got, ids, mask, L, list(range(wl.B)), fp32=True, n_exec=3)
+
+
+def test_varlen_equals_padded_api(w_bf16):
+    wl = synth.WORKLOADS["b64_T128_normal"]
+    ids, mask, L = synth.make_batch(wl)
+    enc = tea.Encoder(w_bf16, A, max_tokens=wl.B * wl.T)
+    padded = enc.forward(_t(ids), _t(mask)).float().cpu().numpy()
+    packed_ids = np.concatenate([ids[b, :L[b]] for b in range(wl.B)])
+    cu = np.concatenate([[0], np.cumsum(L)]).astype(np.int32)
+    out = enc.forward_varlen(_t(packed_ids), _t(cu), int(L.max())).float().cpu().numpy()
+    assert enc.status() == 0
+    enc.close()
+    for b in range(wl.B):
+        np.testing.assert_array_equal(out[cu[b]:cu[b + 1]], padded[b, :L[b]])
+
+
+def test_repeat_calls_are_deterministic_and_stateless(w_bf16):
+    """A second request with another shape does not change the first one's result."""
+    wl1, wl2 = synth.WORKLOADS["b8_T128"], synth.WORKLOADS["b1_T64_latency"]
+    enc = tea.Encoder(w_bf16, A, max_tokens=4096)
+    i1, m1, _ = synth.make_batch(wl1)
+    i2, m2, _ = synth.make_batch(wl2)
+    a = enc.forward(_t(i1), _t(m1)).clone()
+    enc.forward(_t(i2), _t(m2))
+    b = enc.forward(_t(i1), _t(m1))
+    assert enc.status() == 0
+    assert torch.equal(a, b)
+    enc.close()
+
+
+def test_forward_host_buffers_match_device_path(w_bf16):
+    wl = synth.WORKLOADS["b8_T128"]
+    ids, mask, L = synth.make_batch(wl)
+    enc = tea.Encoder(w_bf16, A, max_tokens=wl.B * wl.T)
+    dev = enc.forward(_t(ids), _t(mask)).cpu()
+    ids_h = torch.as_tensor(ids).pin_memory()
+    mask_h = torch.as_tensor(mask).pin_memory()
+    out_h = torch.empty(wl.B, wl.T, 512, dtype=torch.bfloat16).pin_memory()
+    assert enc.forward_host(ids_h, mask_h, out_h) == 0
+    assert torch.equal(dev, out_h)
+    enc.close()
+
+
+# ------------------------------------------------------------ error paths ----
+
+def _sentinel(shape):
+    return torch.full((*shape, 512), 3.25, device="cuda", dtype=torch.bfloat16)
+
+
+def test_invalid_id_leaves_output_untouched(w_bf16):
+    wl = synth.WORKLOADS["b8_T128"]
+    ids, mask, L = synth.make_batch(wl)
+    enc = tea.Encoder(w_bf16, A, max_tokens=wl.B * wl.T)
+    good = enc.forward(_t(ids), _t(mask)).clone()
+    for bad in (178, -1, 10**12):
+        ids_bad = ids.copy()
+        ids_bad[3, int(L[3]) // 2] = bad
+        out = _sentinel(ids.shape)
+        tea.albert_forward(enc.h, _t(ids_bad), _t(mask), out)
+        assert enc.status() == 4  # ALBERT_ERR_ID
+        assert torch.all(out == 3.25)
+    # an invalid id in a padding slot is ignored
+    ids_pad = ids.copy()
+    ids_pad[0, -1] = 999 if L[0] < wl.T else 0
+    out = enc.forward(_t(ids_pad), _t(mask))
+    assert enc.status() == 0
+    if L[0] < wl.T:
+        assert torch.equal(out[0], good[0])
+    # and the next valid call reproduces the earlier result
+    assert torch.equal(enc.forward(_t(ids), _t(mask)), good)
+    enc.close()
+
+
+def test_bad_masks_are_rejected(w_bf16):
+    wl = synth.WORKLOADS["b8_T128"]
+    ids, mask, L = synth.make_batch(wl)
+    enc = tea.Encoder(w_bf16, A, max_tokens=wl.B * wl.T)
+    holes = mask.copy()
+    holes[2, 1] = 0  # not a prefix
+    empty = mask.copy()
+    empty[5, :] = 0  # empty sequence
+    late = mask.copy()
+    late[1, -1] = 1 if L[1] < wl.T - 1 else late[1, -1]
+    cases = [holes, empty] + ([late] if L[1] < wl.T - 1 else [])
+    for m in cases:
+        out = _sentinel(ids.shape)
+        tea.albert_forward(enc.h, _t(ids), _t(m), out)
+        assert enc.status() == 5  # ALBERT_ERR_MASK
+        assert torch.all(out == 3.25)
+    enc.close()
+
+
+def test_host_shape_errors(w_bf16):
+    enc = tea.Encoder(w_bf16, A, max_tokens=1000)
+    ids = torch.zeros(2, 513, dtype=torch.int64, device="cuda")
+    mask = torch.ones(2, 513, dtype=torch.uint8, device="cuda")
+    out = _sentinel((2, 513))
+    with pytest.raises(tea.AlbertError) as e:
+        tea.albert_forward(enc.h, ids, mask, out)
+    assert e.value.code == 3
+    ids = torch.zeros(8, 128, dtype=torch.int64, device="cuda")  # 1024 > 1000 rows
+    with pytest.raises(tea.AlbertError) as e:
+        tea.albert_forward(enc.h, ids, torch.ones_like(ids, dtype=torch.uint8), _sentinel((8, 128)))
+    assert e.value.code == 3
+    enc.close()
+
+
+def test_varlen_rejections(w_bf16):
+    enc = tea.Encoder(w_bf16, A, max_tokens=300)
+    ids = torch.zeros(400, dtype=torch.int64, device="cuda")
+    out = torch.full((400, 512), 3.25, device="cuda", dtype=torch.bfloat16)
+    for cu, code in (([0, 10, 10, 20], 6), ([1, 10, 20], 6), ([0, 128, 256, 384], 3), ([0, 100, 250], 6)):
+        tea.albert_forward_varlen(enc.h, ids, _t(np.array(cu, np.int32)), 128, out)
+        assert enc.status() == code, cu
+        assert torch.all(out == 3.25)
+    enc.close()

@@ -1,0 +1,139 @@
+"""Single-kernel parity on the GPU, through the library's C ABI.
+
+Each kernel runs alone on seeded inputs, over sizes that span several tiles
+plus a ragged tail, and is compared with the oracle's stage functions (fp64)
+on the same bf16-representable inputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import transformer_encoder_albert_b200 as tea
+
+pytestmark = pytest.mark.gpu
+
+
+def _bf16_t(a):
+    return torch.tensor(synth.bf16_round(np.asarray(a, np.float32)), dtype=torch.float32).to("cuda").to(torch.bfloat16)
+
+
+def _np(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def _close(got, ref, rel=8e-3, what=""):
+    """bf16 output: error bounded by output rounding (2^-8 relative) plus an
+    accumulation term proportional to the row scale."""
+    scale = np.max(np.abs(ref))
+    err = np.abs(got - ref)
+    bound = rel * np.abs(ref) + 2e-3 * scale
+    bad = err > bound
+    assert not bad.any(), f"{what}: {bad.sum()} elements off, worst {err.max():.3e} (scale {scale:.3e})"
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 64), (300, 768, 128), (129, 2304, 768), (700, 2048, 768), (257, 512, 768)])
+def test_gemm_bias(M, N, K):
+    r = np.random.default_rng(M + N + K)
+    A, W, b = r.normal(0, 1, (M, K)), r.normal(0, 0.05, (N, K)), r.normal(0, 0.1, N)
+    At, Wt = _bf16_t(A), _bf16_t(W)
+    Y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+    assert tea.test_gemm(At, Wt, torch.tensor(b, dtype=torch.float32, device="cuda"), Y, 0) == 0
+    ref = oracle.linear(_np(At), _np(Wt), np.float32(b).astype(np.float64))
+    _close(_np(Y), ref, what="bias")
+
+
+@pytest.mark.parametrize("M", [5, 200, 640])
+def test_gemm_gelu(M):
+    r = np.random.default_rng(M)
+    N, K = 2048, 768
+    A, W, b = r.normal(0, 1, (M, K)), r.normal(0, 0.05, (N, K)), r.normal(0, 0.1, N)
+    At, Wt = _bf16_t(A), _bf16_t(W)
+    Y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+    assert tea.test_gemm(At, Wt, torch.tensor(b, dtype=torch.float32, device="cuda"), Y, 1) == 0
+    ref = oracle.gelu(oracle.linear(_np(At), _np(Wt), np.float32(b).astype(np.float64)))
+    _close(_np(Y), ref, what="gelu")
+
+
+@pytest.mark.parametrize("M,K", [(3, 768), (130, 768), (513, 2048), (1000, 768)])
+def test_gemm_residual_layer_norm(M, K):
+    r = np.random.default_rng(M * 7 + K)
+    N = 768
+    A, W, b = r.normal(0, 1, (M, K)), r.normal(0, 0.05, (N, K)), r.normal(0, 0.1, N)
+    R = r.normal(0.3, 1.0, (M, N))
+    g, beta = 1 + r.normal(0, 0.1, N), r.normal(0, 0.1, N)
+    At, Wt, Rt = _bf16_t(A), _bf16_t(W), _bf16_t(R)
+    Y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+    f = lambda a: torch.tensor(a, dtype=torch.float32, device="cuda")
+    assert tea.test_gemm(At, Wt, f(b), Y, 2, R=Rt, ln_g=f(g), ln_b=f(beta), eps=1e-12) == 0
+    z = oracle.linear(_np(At), _np(Wt), np.float32(b).astype(np.float64)) + _np(Rt)
+    ref = oracle.layer_norm(z, np.float32(g).astype(np.float64), np.float32(beta).astype(np.float64), 1e-12)
+    _close(_np(Y), ref, what="ln")
+
+
+def test_gemm_scatter_rows():
+    r = np.random.default_rng(9)
+    M, N, K = 333, 512, 768
+    A, W, b = r.normal(0, 1, (M, K)), r.normal(0, 0.05, (N, K)), r.normal(0, 0.1, N)
+    At, Wt = _bf16_t(A), _bf16_t(W)
+    dst = r.permutation(M + 50)[:M].astype(np.int32)
+    dst[::7] = -1
+    Y = torch.full((M + 50, N), 7.0, device="cuda", dtype=torch.bfloat16)
+    assert tea.test_gemm(At, Wt, torch.tensor(b, dtype=torch.float32, device="cuda"), Y, 3,
+                         row_dst=torch.tensor(dst, device="cuda")) == 0
+    ref = oracle.linear(_np(At), _np(Wt), np.float32(b).astype(np.float64))
+    got = _np(Y)
+    keep = dst >= 0
+    _close(got[dst[keep]], ref[keep], what="scatter")
+    untouched = np.setdiff1d(np.arange(M + 50), dst[keep])
+    assert np.all(got[untouched] == 7.0)
+
+
+def _attention_case(lengths, fp32=False, seed=0):
+    r = np.random.default_rng(seed)
+    n = int(sum(lengths))
+    qkv = r.normal(0, 1.0, (n, 3 * 768))
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    if fp32:
+        q_dev = torch.tensor(qkv, dtype=torch.float32, device="cuda")
+        ctx = torch.empty(n, 768, device="cuda", dtype=torch.float32)
+    else:
+        q_dev = _bf16_t(qkv)
+        ctx = torch.empty(n, 768, device="cuda", dtype=torch.bfloat16)
+    assert tea.test_attention(q_dev, torch.tensor(cu, device="cuda"), max(lengths), ctx, fp32=fp32) == 0
+    q64 = _np(q_dev)
+    got = _np(ctx)
+    for s, L in enumerate(lengths):
+        rows = slice(cu[s], cu[s + 1])
+        x = q64[rows]
+        ref = oracle.attention(x[:, :768], x[:, 768:1536], x[:, 1536:], np.ones(L, np.uint8), 12)
+        if fp32:
+            assert np.max(np.abs(got[rows] - ref)) <= 1e-5 * max(1.0, np.max(np.abs(ref)))
+        else:
+            _close(got[rows], ref, rel=2e-2, what=f"attention L={L}")
+
+
+def test_attention_bf16_ragged_lengths():
+    _attention_case([1, 2, 7, 16, 63, 64, 65, 100, 127, 128, 129, 200])
+
+
+def test_attention_bf16_long_sequences():
+    _attention_case([256, 300, 511, 512], seed=1)
+
+
+def test_attention_fp32_ragged_lengths():
+    _attention_case([1, 5, 36, 40, 129], fp32=True, seed=2)
+
+
+def test_attention_identical_keys_give_mean_of_values():
+    L = 50
+    r = np.random.default_rng(3)
+    qkv = r.normal(0, 1, (L, 3 * 768))
+    qkv[:, 768:1536] = qkv[0, 768:1536]
+    q_dev = _bf16_t(qkv)
+    ctx = torch.empty(L, 768, device="cuda", dtype=torch.bfloat16)
+    cu = torch.tensor([0, L], dtype=torch.int32, device="cuda")
+    assert tea.test_attention(q_dev, cu, L, ctx) == 0
+    v = _np(q_dev)[:, 1536:]
+    _close(_np(ctx), np.tile(v.mean(0), (L, 1)), rel=2e-2, what="identical keys")

@@ -1,0 +1,253 @@
+"""B200 (sm_100a) forward pass of Kokoro's ALBERT phoneme encoder behind a C ABI.
+
+The library ``libalbert_b200.so`` (built from ``csrc/`` by ``build.py``) does all
+the work; this module only marshals arguments: it builds the C structs, passes
+torch tensors' device pointers and the current CUDA stream, and turns non-zero
+status codes into exceptions.  Nothing here computes any step of the encoder,
+and there is no CPU fallback: if the library or a GPU is missing, calls fail.
+
+The C functions are exposed under their own names (``albert_create``,
+``albert_forward``, ``albert_forward_varlen``, ``albert_forward_host``,
+``albert_get_status``, ``albert_destroy``) plus the ``Encoder`` convenience class.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libalbert_b200.so")
+
+ALBERT_OK = 0
+ALBERT_BF16, ALBERT_FP32 = 0, 1
+STATUS_NAMES = {
+    0: "ALBERT_OK", 1: "ALBERT_ERR_NULL", 2: "ALBERT_ERR_CONFIG", 3: "ALBERT_ERR_SHAPE",
+    4: "ALBERT_ERR_ID", 5: "ALBERT_ERR_MASK", 6: "ALBERT_ERR_SEQLENS", 7: "ALBERT_ERR_CUDA",
+    8: "ALBERT_ERR_TIMEOUT", 9: "ALBERT_ERR_ALLOC",
+}
+
+WEIGHT_FIELDS = (
+    "word", "pos", "type", "emb_ln_g", "emb_ln_b", "w_in", "b_in",
+    "wq", "bq", "wk", "bk", "wv", "bv", "wo", "bo", "ln1_g", "ln1_b",
+    "w1", "b1", "w2", "b2", "ln2_g", "ln2_b", "w_out", "b_out",
+)
+
+EXPORTS = (
+    "albert_create", "albert_forward", "albert_forward_varlen", "albert_forward_host",
+    "albert_get_status", "albert_destroy", "albert_launches_per_forward",
+    "albert_profile_enable", "albert_profile_reset", "albert_profile_classes",
+    "albert_profile_name", "albert_profile_read", "albert_test_gemm", "albert_test_attention",
+)
+
+
+class AlbertError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS_NAMES.get(code, code)}")
+
+
+class albert_config(C.Structure):
+    _fields_ = [(n, C.c_int) for n in ("vocab", "emb", "hidden", "heads", "ffn", "n_exec", "n_groups",
+                                       "max_pos", "n_types", "out_dim", "dtype", "max_tokens", "pack")] \
+        + [("ln_eps", C.c_float)]
+
+
+class albert_weights(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in WEIGHT_FIELDS]
+
+
+_lib = None
+
+
+def lib() -> C.CDLL:
+    """Load the CUDA library; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m transformer_encoder_albert_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        vp, i = C.c_void_p, C.c_int
+        L.albert_create.argtypes = [C.POINTER(albert_weights), C.POINTER(albert_config), C.POINTER(vp)]
+        L.albert_forward.argtypes = [vp, vp, vp, i, i, vp, vp]
+        L.albert_forward_varlen.argtypes = [vp, vp, vp, i, i, vp, vp]
+        L.albert_forward_host.argtypes = [vp, vp, vp, i, i, vp, vp]
+        L.albert_get_status.argtypes = [vp, vp]
+        L.albert_destroy.argtypes = [vp]
+        L.albert_destroy.restype = None
+        L.albert_launches_per_forward.argtypes = [vp, i]
+        L.albert_profile_enable.argtypes = [vp, i]
+        L.albert_profile_reset.argtypes = [vp]
+        L.albert_profile_classes.argtypes = []
+        L.albert_profile_name.argtypes = [i]
+        L.albert_profile_name.restype = C.c_char_p
+        L.albert_profile_read.argtypes = [vp, C.POINTER(C.c_int), C.POINTER(C.c_double)]
+        L.albert_test_gemm.argtypes = [vp, vp, vp, vp, vp, vp, C.c_float, vp, vp, i, i, i, i, vp]
+        L.albert_test_attention.argtypes = [vp, vp, i, i, vp, i, vp]
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != ALBERT_OK:
+        raise AlbertError(rc, where)
+
+
+def _stream_ptr(stream=None) -> int:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else int(t.data_ptr())
+
+
+def make_config(arch: dict, dtype: str = "bf16", max_tokens: int = 4096, pack: bool = True,
+                n_exec: int | None = None, out_dim: int | None = None) -> albert_config:
+    return albert_config(
+        vocab=arch["vocab"], emb=arch["emb"], hidden=arch["hidden"], heads=arch["heads"],
+        ffn=arch["ffn"], n_exec=arch["n_exec"] if n_exec is None else n_exec, n_groups=1,
+        max_pos=arch["max_pos"], n_types=arch["n_types"],
+        out_dim=arch["out_dim"] if out_dim is None else out_dim,
+        dtype=ALBERT_BF16 if dtype == "bf16" else ALBERT_FP32, max_tokens=max_tokens,
+        pack=1 if pack else 0, ln_eps=arch["ln_eps"])
+
+
+# ---------------------------------------------------------------- C names --
+
+def albert_create(weights: dict, cfg: albert_config) -> int:
+    """weights: name -> CUDA float32 tensor (contiguous).  Returns the handle."""
+    import torch
+    dev = {}
+    for k in WEIGHT_FIELDS:
+        t = weights.get(k)
+        if t is None:
+            dev[k] = None
+            continue
+        if not torch.is_tensor(t):
+            t = torch.as_tensor(t)
+        dev[k] = t.to(device="cuda", dtype=torch.float32).contiguous()
+    w = albert_weights(*[_ptr(dev[k]) for k in WEIGHT_FIELDS])
+    h = C.c_void_p()
+    _check(lib().albert_create(C.byref(w), C.byref(cfg), C.byref(h)), "albert_create")
+    return h.value
+
+
+def albert_forward(h: int, ids, mask, out, stream=None) -> None:
+    B, T = ids.shape
+    _check(lib().albert_forward(h, _ptr(ids), _ptr(mask), B, T, _ptr(out), _stream_ptr(stream)),
+           "albert_forward")
+
+
+def albert_forward_varlen(h: int, ids, cu_seqlens, max_len: int, out, stream=None) -> None:
+    nseq = cu_seqlens.numel() - 1
+    _check(lib().albert_forward_varlen(h, _ptr(ids), _ptr(cu_seqlens), nseq, int(max_len), _ptr(out),
+                                       _stream_ptr(stream)), "albert_forward_varlen")
+
+
+def albert_forward_host(h: int, ids_host, mask_host, out_host, stream=None) -> int:
+    B, T = ids_host.shape
+    return lib().albert_forward_host(h, _ptr(ids_host), _ptr(mask_host), B, T, _ptr(out_host),
+                                     _stream_ptr(stream))
+
+
+def albert_get_status(h: int, stream=None) -> int:
+    return lib().albert_get_status(h, _stream_ptr(stream))
+
+
+def albert_destroy(h: int) -> None:
+    lib().albert_destroy(h)
+
+
+# --------------------------------------------------------- convenience class --
+
+class Encoder:
+    """Owns one library handle.  Outputs are bf16 (dtype "bf16") or fp32 tensors."""
+
+    def __init__(self, weights: dict, arch: dict, dtype: str = "bf16", max_tokens: int = 4096,
+                 pack: bool = True, n_exec: int | None = None, out_dim: int | None = None):
+        self.cfg = make_config(arch, dtype, max_tokens, pack, n_exec, out_dim)
+        self.dtype = dtype
+        self.out_dim = self.cfg.out_dim if self.cfg.out_dim > 0 else self.cfg.hidden
+        self.h = albert_create(weights, self.cfg)
+
+    def _out(self, shape):
+        import torch
+        dt = torch.bfloat16 if self.dtype == "bf16" else torch.float32
+        return torch.empty(*shape, self.out_dim, device="cuda", dtype=dt)
+
+    def forward(self, ids, mask, out=None, stream=None):
+        if out is None:
+            out = self._out(ids.shape)
+        albert_forward(self.h, ids, mask, out, stream)
+        return out
+
+    def forward_varlen(self, ids, cu_seqlens, max_len, out=None, stream=None):
+        if out is None:
+            out = self._out((ids.shape[0],))
+        albert_forward_varlen(self.h, ids, cu_seqlens, max_len, out, stream)
+        return out
+
+    def forward_host(self, ids_host, mask_host, out_host, stream=None) -> int:
+        return albert_forward_host(self.h, ids_host, mask_host, out_host, stream)
+
+    def status(self, stream=None) -> int:
+        return albert_get_status(self.h, stream)
+
+    def launches_per_forward(self, padded_api: bool = True) -> int:
+        return lib().albert_launches_per_forward(self.h, 1 if padded_api else 0)
+
+    def profile(self, classes=None) -> None:
+        """Time launches of the named kernel classes (None = all, [] = off)."""
+        if classes is None:
+            mask = -1
+        else:
+            names = profile_class_names()
+            mask = 0
+            for c in classes:
+                mask |= 1 << names.index(c)
+        _check(lib().albert_profile_enable(self.h, mask), "albert_profile_enable")
+
+    def profile_reset(self) -> None:
+        _check(lib().albert_profile_reset(self.h), "albert_profile_reset")
+
+    def profile_read(self) -> dict:
+        n = lib().albert_profile_classes()
+        launches = (C.c_int * n)()
+        ms = (C.c_double * n)()
+        _check(lib().albert_profile_read(self.h, launches, ms), "albert_profile_read")
+        return {lib().albert_profile_name(i).decode(): (launches[i], ms[i]) for i in range(n)}
+
+    def close(self) -> None:
+        if self.h:
+            albert_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def profile_class_names() -> list:
+    n = lib().albert_profile_classes()
+    return [lib().albert_profile_name(i).decode() for i in range(n)]
+
+
+def test_gemm(A, W, bias, Y, epi: int, R=None, ln_g=None, ln_b=None, eps: float = 1e-12,
+              row_dst=None, stream=None) -> int:
+    """Run the tcgen05 GEMM alone (single-kernel parity tests)."""
+    M, K = A.shape
+    N = W.shape[0]
+    return lib().albert_test_gemm(_ptr(A), _ptr(W), _ptr(bias), _ptr(R), _ptr(ln_g), _ptr(ln_b),
+                                  float(eps), _ptr(row_dst), _ptr(Y), M, N, K, epi,
+                                  _stream_ptr(stream))
+
+
+def test_attention(qkv, cu_seqlens, max_len: int, ctx, fp32: bool = False, stream=None) -> int:
+    """Run the attention kernel alone (single-kernel parity tests)."""
+    return lib().albert_test_attention(_ptr(qkv), _ptr(cu_seqlens), cu_seqlens.numel() - 1,
+                                       int(max_len), _ptr(ctx), ALBERT_FP32 if fp32 else ALBERT_BF16,
+                                       _stream_ptr(stream))

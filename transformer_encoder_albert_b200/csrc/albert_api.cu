@@ -1,0 +1,597 @@
+// albert_api.cu -- the C ABI (include/albert.h): weights, workspace, TMA
+// descriptors and the launch schedule of one forward pass.
+//
+// Schedule of one forward ("ALBERT: How Kokoro's Phoneme Encoder Works",
+// section "Inside One Real ALBERT Layer" and the paragraph after it):
+//   prep (mask / lengths -> packed row offsets) -> embed+LN -> GEMM 128->768
+//   -> n_exec x [ GEMM Q|K|V -> attention -> GEMM Wo + residual + LN
+//                 -> GEMM W1 + GELU -> GEMM W2 + residual + LN ]
+//   -> GEMM 768->512 scattered to [B, T, 512] -> zero padding rows.
+// The shared layer's weights exist once in device memory and every execution
+// reads the same copy, which stays resident in L2 across executions.
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "albert.h"
+#include "kernels.h"
+
+using namespace albert;
+
+namespace {
+
+enum ProfClass {
+    kProfPrep = 0, kProfEmbed, kProfGemmIn, kProfGemmQKV, kProfAttention, kProfGemmWoLN,
+    kProfGemmW1Gelu, kProfGemmW2LN, kProfGemmOut, kProfOutput, kProfLayerNorm, kProfClasses
+};
+const char *kProfNames[kProfClasses] = {
+    "prep", "embed_ln", "gemm_in_proj", "gemm_qkv", "attention", "gemm_out_proj_ln",
+    "gemm_ffn_up_gelu", "gemm_ffn_down_ln", "gemm_final_proj", "output_rows", "layer_norm_f32"};
+
+constexpr int kEventPool = 16384;
+
+}  // namespace
+
+struct albert_handle {
+    albert_config cfg{};
+    int device = 0, num_sms = 0;
+    int rows_cap = 0;   // workspace rows (multiple of 128)
+    int seq_cap = 0;    // sequences
+    std::vector<void *> allocs;
+
+    // parameters
+    float *word = nullptr, *pos = nullptr, *type = nullptr, *emb_g = nullptr, *emb_b = nullptr;
+    float *b_in = nullptr, *bqkv = nullptr, *bo = nullptr, *ln1_g = nullptr, *ln1_b = nullptr;
+    float *b1 = nullptr, *b2 = nullptr, *ln2_g = nullptr, *ln2_b = nullptr, *b_out = nullptr;
+    void *w_in = nullptr, *wqkv = nullptr, *wo = nullptr, *w1 = nullptr, *w2 = nullptr, *w_out = nullptr;
+    void *wblock = nullptr;
+    size_t wblock_bytes = 0;
+
+    // workspace
+    void *E = nullptr, *X = nullptr, *QKV = nullptr, *C = nullptr, *X1 = nullptr, *H = nullptr, *Z = nullptr;
+    float *scratch = nullptr;
+    int *seq_start = nullptr, *seq_len = nullptr, *row_dst = nullptr, *n_rows = nullptr, *status = nullptr;
+    int grid_ln = 0;
+
+    // host-buffer staging
+    int64_t *st_ids = nullptr;
+    uint8_t *st_mask = nullptr;
+    void *st_out = nullptr;
+
+    // TMA descriptors (bf16)
+    CUtensorMap tm_E, tm_X, tm_C, tm_X1, tm_H;
+    CUtensorMap tm_win, tm_wqkv, tm_wo, tm_w1, tm_w2, tm_wout;
+
+    // per-kernel timing
+    unsigned prof_mask = 0;  // classes whose launches are timed
+    std::vector<cudaEvent_t> ev;
+    std::vector<int> ev_cls;
+    int ev_used = 0;
+    int prof_launches[kProfClasses] = {};
+    double prof_ms[kProfClasses] = {};
+};
+
+namespace {
+
+#define TRY(x)                                                     \
+    do {                                                           \
+        cudaError_t e_ = (x);                                      \
+        if (e_ != cudaSuccess) {                                   \
+            if (getenv("ALBERT_DEBUG"))                            \
+                fprintf(stderr, "albert: %s failed: %s (%s:%d)\n", #x, \
+                        cudaGetErrorString(e_), __FILE__, __LINE__); \
+            return ALBERT_ERR_CUDA;                                \
+        }                                                          \
+    } while (0)
+
+int dev_alloc(albert_handle *h, void **p, size_t bytes) {
+    if (bytes == 0) bytes = 16;
+    if (cudaMalloc(p, bytes) != cudaSuccess) {
+        *p = nullptr;
+        return ALBERT_ERR_ALLOC;
+    }
+    h->allocs.push_back(*p);
+    return ALBERT_OK;
+}
+
+size_t elem_bytes(const albert_handle *h) { return h->cfg.dtype == ALBERT_FP32 ? 4 : 2; }
+int out_width(const albert_handle *h) { return h->cfg.out_dim > 0 ? h->cfg.out_dim : kHidden; }
+
+int check_config(const albert_config *c) {
+    if (c->emb != kEmb || c->hidden != kHidden || c->heads != kHeads || c->ffn != kFfn) return ALBERT_ERR_CONFIG;
+    if (c->n_groups != 1 || c->n_exec < 0) return ALBERT_ERR_CONFIG;
+    if (c->max_pos < 1 || c->max_pos > kMaxPos || c->vocab < 1 || c->n_types < 1) return ALBERT_ERR_CONFIG;
+    if (c->out_dim != 0 && c->out_dim != 512) return ALBERT_ERR_CONFIG;
+    if (c->dtype != ALBERT_BF16 && c->dtype != ALBERT_FP32) return ALBERT_ERR_CONFIG;
+    if (c->max_tokens < 1 || c->max_tokens > (1 << 24)) return ALBERT_ERR_CONFIG;
+    if (c->pack != 0 && c->pack != 1) return ALBERT_ERR_CONFIG;
+    if (!(c->ln_eps >= 0.f)) return ALBERT_ERR_CONFIG;
+    return ALBERT_OK;
+}
+
+// ---- per-kernel timing ----
+int prof_harvest(albert_handle *h) {
+    if (h->ev_used == 0) return ALBERT_OK;
+    TRY(cudaEventSynchronize(h->ev[h->ev_used - 1]));
+    for (int i = 0; i + 1 < h->ev_used; i += 2) {
+        float ms = 0.f;
+        TRY(cudaEventElapsedTime(&ms, h->ev[i], h->ev[i + 1]));
+        h->prof_ms[h->ev_cls[i]] += ms;
+        h->prof_launches[h->ev_cls[i]] += 1;
+    }
+    h->ev_used = 0;
+    return ALBERT_OK;
+}
+
+struct Launch {
+    albert_handle *h;
+    cudaStream_t s;
+    int cls = -1;
+    int begin(int c) {
+        cls = c;
+        if (!(h->prof_mask >> c & 1u)) return ALBERT_OK;
+        if (h->ev_used + 2 > kEventPool) {
+            int rc = prof_harvest(h);
+            if (rc) return rc;
+        }
+        h->ev_cls[h->ev_used] = c;
+        TRY(cudaEventRecord(h->ev[h->ev_used++], s));
+        return ALBERT_OK;
+    }
+    int end(cudaError_t launched) {
+        if (launched != cudaSuccess) {
+            if (getenv("ALBERT_DEBUG"))
+                fprintf(stderr, "albert: launch of %s failed: %s\n", kProfNames[cls], cudaGetErrorString(launched));
+            return ALBERT_ERR_CUDA;
+        }
+        if (!(h->prof_mask >> cls & 1u)) return ALBERT_OK;
+        h->ev_cls[h->ev_used] = cls;
+        TRY(cudaEventRecord(h->ev[h->ev_used++], s));
+        return ALBERT_OK;
+    }
+};
+
+#define LAUNCH(L, cls, call)               \
+    do {                                   \
+        int rc_ = (L).begin(cls);          \
+        if (rc_) return rc_;               \
+        rc_ = (L).end(call);               \
+        if (rc_) return rc_;               \
+    } while (0)
+
+GemmArgs gemm_args(albert_handle *h, int N, int K, const float *bias, void *out, int ld_out) {
+    GemmArgs a{};
+    a.N = N;
+    a.K = K;
+    a.rows_cap = h->rows_cap;
+    a.n_rows = h->n_rows;
+    a.bias = bias;
+    a.out = static_cast<bf16 *>(out);
+    a.ld_out = ld_out;
+    a.scratch = h->scratch;
+    a.row_dst = h->row_dst;
+    a.status = h->status;
+    a.eps = h->cfg.ln_eps;
+    return a;
+}
+
+int gemm_bf16(Launch &L, int cls, int epi, const CUtensorMap &A, const CUtensorMap &B, const GemmArgs &a) {
+    const int grid = gemm_grid(epi, a.rows_cap, a.N, L.h->num_sms);
+    if (epi == kEpiLN && grid > L.h->grid_ln) return ALBERT_ERR_CONFIG;
+    LAUNCH(L, cls, launch_gemm(epi, A, B, a, grid, L.s));
+    return ALBERT_OK;
+}
+
+GemmF32Args f32_args(albert_handle *h, const void *A, const void *W, const float *bias, void *out,
+                     int ld_out, int N, int K) {
+    GemmF32Args a{};
+    a.A = static_cast<const float *>(A);
+    a.W = static_cast<const float *>(W);
+    a.bias = bias;
+    a.out = static_cast<float *>(out);
+    a.ld_out = ld_out;
+    a.N = N;
+    a.K = K;
+    a.rows_cap = h->rows_cap;
+    a.n_rows = h->n_rows;
+    a.row_dst = h->row_dst;
+    a.status = h->status;
+    return a;
+}
+
+// Everything after the prep kernel; `padded_api` selects zero-filled padding rows.
+int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, int nseq, int T,
+               int max_len, void *out, int padded_api) {
+    const albert_config &c = h->cfg;
+    const bool bf = c.dtype == ALBERT_BF16;
+    EmbedArgs ea{};
+    ea.ids = ids;
+    ea.ids_padded = ids_padded;
+    ea.T = T;
+    ea.seq_start = h->seq_start;
+    ea.seq_len = h->seq_len;
+    ea.nseq = nseq;
+    ea.n_rows = h->n_rows;
+    ea.rows_cap = h->rows_cap;
+    ea.word = h->word;
+    ea.pos = h->pos;
+    ea.type = h->type;
+    ea.g = h->emb_g;
+    ea.b = h->emb_b;
+    ea.eps = c.ln_eps;
+    ea.vocab = c.vocab;
+    ea.E = h->E;
+    ea.out_f32 = bf ? 0 : 1;
+    ea.row_dst = h->row_dst;
+    ea.dst_padded = padded_api;
+    ea.status = h->status;
+    LAUNCH(L, kProfEmbed, launch_embed(ea, L.s));
+
+    const int D = out_width(h);
+    if (bf) {
+        int rc;
+        if ((rc = gemm_bf16(L, kProfGemmIn, kEpiBias, h->tm_E, h->tm_win, gemm_args(h, kHidden, kEmb, h->b_in, h->X, kHidden)))) return rc;
+        for (int l = 0; l < c.n_exec; ++l) {
+            if ((rc = gemm_bf16(L, kProfGemmQKV, kEpiBias, h->tm_X, h->tm_wqkv, gemm_args(h, kQKV, kHidden, h->bqkv, h->QKV, kQKV)))) return rc;
+            LAUNCH(L, kProfAttention, launch_attention_bf16(static_cast<bf16 *>(h->QKV), static_cast<bf16 *>(h->C), h->seq_start,
+                                                           h->seq_len, nseq, max_len, h->status, L.s));
+            GemmArgs a = gemm_args(h, kHidden, kHidden, h->bo, h->X1, kHidden);
+            a.resid = static_cast<bf16 *>(h->X);
+            a.ld_resid = kHidden;
+            a.ln_g = h->ln1_g;
+            a.ln_b = h->ln1_b;
+            if ((rc = gemm_bf16(L, kProfGemmWoLN, kEpiLN, h->tm_C, h->tm_wo, a))) return rc;
+            if ((rc = gemm_bf16(L, kProfGemmW1Gelu, kEpiGelu, h->tm_X1, h->tm_w1, gemm_args(h, kFfn, kHidden, h->b1, h->H, kFfn)))) return rc;
+            a = gemm_args(h, kHidden, kFfn, h->b2, h->X, kHidden);
+            a.resid = static_cast<bf16 *>(h->X1);
+            a.ld_resid = kHidden;
+            a.ln_g = h->ln2_g;
+            a.ln_b = h->ln2_b;
+            if ((rc = gemm_bf16(L, kProfGemmW2LN, kEpiLN, h->tm_H, h->tm_w2, a))) return rc;
+        }
+        if (c.out_dim > 0) {
+            if ((rc = gemm_bf16(L, kProfGemmOut, kEpiScatter, h->tm_X, h->tm_wout, gemm_args(h, c.out_dim, kHidden, h->b_out, out, c.out_dim)))) return rc;
+        } else {
+            LAUNCH(L, kProfOutput, launch_scatter_rows(h->X, out, kHidden, 2, h->rows_cap, h->n_rows, h->row_dst, h->status, L.s));
+        }
+    } else {
+        LAUNCH(L, kProfGemmIn, launch_gemm_f32(kF32Bias, f32_args(h, h->E, h->w_in, h->b_in, h->X, kHidden, kHidden, kEmb), L.s));
+        for (int l = 0; l < c.n_exec; ++l) {
+            LAUNCH(L, kProfGemmQKV, launch_gemm_f32(kF32Bias, f32_args(h, h->X, h->wqkv, h->bqkv, h->QKV, kQKV, kQKV, kHidden), L.s));
+            LAUNCH(L, kProfAttention, launch_attention_f32(static_cast<float *>(h->QKV), static_cast<float *>(h->C), h->seq_start,
+                                                          h->seq_len, nseq, max_len, h->status, L.s));
+            GemmF32Args a = f32_args(h, h->C, h->wo, h->bo, h->Z, kHidden, kHidden, kHidden);
+            a.resid = static_cast<float *>(h->X);
+            LAUNCH(L, kProfGemmWoLN, launch_gemm_f32(kF32Resid, a, L.s));
+            LAUNCH(L, kProfLayerNorm, launch_layer_norm_f32(static_cast<float *>(h->Z), static_cast<float *>(h->X1), h->ln1_g, h->ln1_b,
+                                                           c.ln_eps, h->rows_cap, h->n_rows, h->status, L.s));
+            LAUNCH(L, kProfGemmW1Gelu, launch_gemm_f32(kF32Gelu, f32_args(h, h->X1, h->w1, h->b1, h->H, kFfn, kFfn, kHidden), L.s));
+            a = f32_args(h, h->H, h->w2, h->b2, h->Z, kHidden, kHidden, kFfn);
+            a.resid = static_cast<float *>(h->X1);
+            LAUNCH(L, kProfGemmW2LN, launch_gemm_f32(kF32Resid, a, L.s));
+            LAUNCH(L, kProfLayerNorm, launch_layer_norm_f32(static_cast<float *>(h->Z), static_cast<float *>(h->X), h->ln2_g, h->ln2_b,
+                                                           c.ln_eps, h->rows_cap, h->n_rows, h->status, L.s));
+        }
+        if (c.out_dim > 0) {
+            LAUNCH(L, kProfGemmOut, launch_gemm_f32(kF32Scatter, f32_args(h, h->X, h->w_out, h->b_out, out, c.out_dim, c.out_dim, kHidden), L.s));
+        } else {
+            LAUNCH(L, kProfOutput, launch_scatter_rows(h->X, out, kHidden, 4, h->rows_cap, h->n_rows, h->row_dst, h->status, L.s));
+        }
+    }
+    if (padded_api)
+        LAUNCH(L, kProfOutput, launch_zero_pad(out, nseq, T, D, (int)elem_bytes(h), h->seq_len, h->status, L.s));
+    return ALBERT_OK;
+}
+
+int copy_param(float *dst, const float *src, size_t n, cudaStream_t s) {
+    if (!src) return ALBERT_ERR_NULL;
+    TRY(cudaMemcpyAsync(dst, src, n * sizeof(float), cudaMemcpyDeviceToDevice, s));
+    return ALBERT_OK;
+}
+
+int copy_matrix(albert_handle *h, void *dst, const float *src, size_t n, cudaStream_t s) {
+    if (!src) return ALBERT_ERR_NULL;
+    if (h->cfg.dtype == ALBERT_BF16) {
+        TRY(launch_f32_to_bf16(src, static_cast<bf16 *>(dst), n, s));
+    } else {
+        TRY(cudaMemcpyAsync(dst, src, n * sizeof(float), cudaMemcpyDeviceToDevice, s));
+    }
+    return ALBERT_OK;
+}
+
+int create_impl(albert_handle *h, const albert_weights *w) {
+    const albert_config &c = h->cfg;
+    TRY(cudaGetDevice(&h->device));
+    TRY(cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device));
+    h->rows_cap = (c.max_tokens + 127) / 128 * 128;
+    h->seq_cap = c.max_tokens;
+    const size_t R = h->rows_cap;
+    const bool bf = c.dtype == ALBERT_BF16;
+    const size_t eb = elem_bytes(h);
+    int rc;
+    cudaStream_t s = nullptr;
+    TRY(cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking));
+    struct StreamGuard { cudaStream_t s; ~StreamGuard() { cudaStreamDestroy(s); } } guard{s};
+
+    // ---- small fp32 parameters: one block ----
+    const size_t V = c.vocab, P = c.max_pos, NT = c.n_types, O = c.out_dim;
+    const size_t n_small = V * kEmb + P * kEmb + NT * kEmb + 2 * kEmb + kHidden + kQKV + kHidden + 2 * kHidden +
+                           kFfn + kHidden + 2 * kHidden + O;
+    float *small = nullptr;
+    if ((rc = dev_alloc(h, (void **)&small, n_small * sizeof(float)))) return rc;
+    float *q = small;
+    auto take = [&](size_t n) { float *r = q; q += n; return r; };
+    h->word = take(V * kEmb); h->pos = take(P * kEmb); h->type = take(NT * kEmb);
+    h->emb_g = take(kEmb); h->emb_b = take(kEmb); h->b_in = take(kHidden); h->bqkv = take(kQKV);
+    h->bo = take(kHidden); h->ln1_g = take(kHidden); h->ln1_b = take(kHidden); h->b1 = take(kFfn);
+    h->b2 = take(kHidden); h->ln2_g = take(kHidden); h->ln2_b = take(kHidden); h->b_out = take(O);
+    if ((rc = copy_param(h->word, w->word, V * kEmb, s))) return rc;
+    if ((rc = copy_param(h->pos, w->pos, P * kEmb, s))) return rc;
+    if ((rc = copy_param(h->type, w->type, NT * kEmb, s))) return rc;
+    if ((rc = copy_param(h->emb_g, w->emb_ln_g, kEmb, s))) return rc;
+    if ((rc = copy_param(h->emb_b, w->emb_ln_b, kEmb, s))) return rc;
+    if ((rc = copy_param(h->b_in, w->b_in, kHidden, s))) return rc;
+    if ((rc = copy_param(h->bqkv, w->bq, kHidden, s))) return rc;
+    if ((rc = copy_param(h->bqkv + kHidden, w->bk, kHidden, s))) return rc;
+    if ((rc = copy_param(h->bqkv + 2 * kHidden, w->bv, kHidden, s))) return rc;
+    if ((rc = copy_param(h->bo, w->bo, kHidden, s))) return rc;
+    if ((rc = copy_param(h->ln1_g, w->ln1_g, kHidden, s))) return rc;
+    if ((rc = copy_param(h->ln1_b, w->ln1_b, kHidden, s))) return rc;
+    if ((rc = copy_param(h->b1, w->b1, kFfn, s))) return rc;
+    if ((rc = copy_param(h->b2, w->b2, kHidden, s))) return rc;
+    if ((rc = copy_param(h->ln2_g, w->ln2_g, kHidden, s))) return rc;
+    if ((rc = copy_param(h->ln2_b, w->ln2_b, kHidden, s))) return rc;
+    if (O && (rc = copy_param(h->b_out, w->b_out, O, s))) return rc;
+
+    // ---- matrices: one contiguous block (bf16 or fp32), 256-byte aligned pieces ----
+    const size_t n_win = (size_t)kHidden * kEmb, n_qkv = (size_t)kQKV * kHidden, n_wo = (size_t)kHidden * kHidden;
+    const size_t n_w1 = (size_t)kFfn * kHidden, n_w2 = (size_t)kHidden * kFfn, n_out = O * kHidden;
+    auto al = [](size_t b) { return (b + 255) / 256 * 256; };
+    size_t off_win = 0, off_qkv = off_win + al(n_win * eb), off_wo = off_qkv + al(n_qkv * eb);
+    size_t off_w1 = off_wo + al(n_wo * eb), off_w2 = off_w1 + al(n_w1 * eb), off_out = off_w2 + al(n_w2 * eb);
+    h->wblock_bytes = off_out + al(n_out * eb);
+    if ((rc = dev_alloc(h, &h->wblock, h->wblock_bytes))) return rc;
+    uint8_t *wb = static_cast<uint8_t *>(h->wblock);
+    h->w_in = wb + off_win; h->wqkv = wb + off_qkv; h->wo = wb + off_wo;
+    h->w1 = wb + off_w1; h->w2 = wb + off_w2; h->w_out = wb + off_out;
+    if ((rc = copy_matrix(h, h->w_in, w->w_in, n_win, s))) return rc;
+    if ((rc = copy_matrix(h, h->wqkv, w->wq, n_wo, s))) return rc;
+    if ((rc = copy_matrix(h, static_cast<uint8_t *>(h->wqkv) + n_wo * eb, w->wk, n_wo, s))) return rc;
+    if ((rc = copy_matrix(h, static_cast<uint8_t *>(h->wqkv) + 2 * n_wo * eb, w->wv, n_wo, s))) return rc;
+    if ((rc = copy_matrix(h, h->wo, w->wo, n_wo, s))) return rc;
+    if ((rc = copy_matrix(h, h->w1, w->w1, n_w1, s))) return rc;
+    if ((rc = copy_matrix(h, h->w2, w->w2, n_w2, s))) return rc;
+    if (O && (rc = copy_matrix(h, h->w_out, w->w_out, n_out, s))) return rc;
+
+    // ---- workspace ----
+    if ((rc = dev_alloc(h, &h->E, R * kEmb * eb))) return rc;
+    if ((rc = dev_alloc(h, &h->X, R * kHidden * eb))) return rc;
+    if ((rc = dev_alloc(h, &h->QKV, R * kQKV * eb))) return rc;
+    if ((rc = dev_alloc(h, &h->C, R * kHidden * eb))) return rc;
+    if ((rc = dev_alloc(h, &h->X1, R * kHidden * eb))) return rc;
+    if ((rc = dev_alloc(h, &h->H, R * kFfn * eb))) return rc;
+    if (bf) {
+        h->grid_ln = gemm_grid(kEpiLN, h->rows_cap, kHidden, h->num_sms);
+        if ((rc = dev_alloc(h, (void **)&h->scratch, gemm_ln_scratch_floats(h->grid_ln) * sizeof(float)))) return rc;
+    } else {
+        if ((rc = dev_alloc(h, &h->Z, R * kHidden * eb))) return rc;
+    }
+    if ((rc = dev_alloc(h, (void **)&h->seq_start, (h->seq_cap + 1) * sizeof(int)))) return rc;
+    if ((rc = dev_alloc(h, (void **)&h->seq_len, (h->seq_cap + 1) * sizeof(int)))) return rc;
+    if ((rc = dev_alloc(h, (void **)&h->row_dst, R * sizeof(int)))) return rc;
+    if ((rc = dev_alloc(h, (void **)&h->n_rows, 2 * sizeof(int)))) return rc;
+    h->status = h->n_rows + 1;
+    if ((rc = dev_alloc(h, (void **)&h->st_ids, (size_t)c.max_tokens * sizeof(int64_t)))) return rc;
+    if ((rc = dev_alloc(h, (void **)&h->st_mask, (size_t)c.max_tokens))) return rc;
+    if ((rc = dev_alloc(h, &h->st_out, (size_t)c.max_tokens * out_width(h) * eb))) return rc;
+    // Deterministic contents for rows a forward never writes.
+    for (void *p : {h->E, h->X, h->QKV, h->C, h->X1, h->H}) {
+        size_t bytes = (p == h->E ? kEmb : p == h->QKV ? kQKV : p == h->H ? kFfn : kHidden) * R * eb;
+        TRY(cudaMemsetAsync(p, 0, bytes, s));
+    }
+    TRY(cudaMemsetAsync(h->n_rows, 0, 2 * sizeof(int), s));
+
+    // ---- TMA descriptors ----
+    if (bf) {
+        if (make_tmap_bf16(&h->tm_E, h->E, R, kEmb, gemm::BM) || make_tmap_bf16(&h->tm_X, h->X, R, kHidden, gemm::BM) ||
+            make_tmap_bf16(&h->tm_C, h->C, R, kHidden, gemm::BM) || make_tmap_bf16(&h->tm_X1, h->X1, R, kHidden, gemm::BM) ||
+            make_tmap_bf16(&h->tm_H, h->H, R, kFfn, gemm::BM) ||
+            make_tmap_bf16(&h->tm_win, h->w_in, kHidden, kEmb, gemm::BN) ||
+            make_tmap_bf16(&h->tm_wqkv, h->wqkv, kQKV, kHidden, gemm::BN) ||
+            make_tmap_bf16(&h->tm_wo, h->wo, kHidden, kHidden, gemm::BN) ||
+            make_tmap_bf16(&h->tm_w1, h->w1, kFfn, kHidden, gemm::BN) ||
+            make_tmap_bf16(&h->tm_w2, h->w2, kHidden, kFfn, gemm::BN) ||
+            (O && make_tmap_bf16(&h->tm_wout, h->w_out, O, kHidden, gemm::BN)))
+            return ALBERT_ERR_CUDA;
+    }
+    TRY(cudaStreamSynchronize(s));
+    return ALBERT_OK;
+}
+
+void free_all(albert_handle *h) {
+    for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
+    h->ev.clear();
+    for (void *p : h->allocs) cudaFree(p);
+    h->allocs.clear();
+}
+
+int forward_padded(albert_handle *h, const int64_t *ids, const uint8_t *mask, int B, int T, void *out,
+                   cudaStream_t s) {
+    Launch L{h, s};
+    LAUNCH(L, kProfPrep, launch_prep_padded(mask, B, T, h->cfg.pack, h->cfg.max_tokens, h->seq_start, h->seq_len,
+                                            h->n_rows, h->status, s));
+    return run_layers(h, L, ids, 1, B, T, T, out, 1);
+}
+
+}  // namespace
+
+extern "C" {
+
+int albert_create(const albert_weights *w, const albert_config *cfg, albert_handle **out) {
+    if (!out) return ALBERT_ERR_NULL;
+    *out = nullptr;
+    if (!w || !cfg) return ALBERT_ERR_NULL;
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    albert_handle *h = new (std::nothrow) albert_handle();
+    if (!h) return ALBERT_ERR_ALLOC;
+    h->cfg = *cfg;
+    rc = create_impl(h, w);
+    if (rc) {
+        free_all(h);
+        delete h;
+        return rc;
+    }
+    *out = h;
+    return ALBERT_OK;
+}
+
+int albert_forward(albert_handle *h, const int64_t *ids, const uint8_t *mask, int B, int T, void *out,
+                   void *stream) {
+    if (!h || !ids || !mask || !out) return ALBERT_ERR_NULL;
+    if (B < 1 || T < 1 || T > h->cfg.max_pos || (long long)B * T > h->cfg.max_tokens) return ALBERT_ERR_SHAPE;
+    return forward_padded(h, ids, mask, B, T, out, static_cast<cudaStream_t>(stream));
+}
+
+int albert_forward_varlen(albert_handle *h, const int64_t *ids, const int32_t *cu_seqlens, int nseq,
+                          int max_len, void *out, void *stream) {
+    if (!h || !ids || !cu_seqlens || !out) return ALBERT_ERR_NULL;
+    if (nseq < 1 || nseq > h->seq_cap || max_len < 1 || max_len > h->cfg.max_pos) return ALBERT_ERR_SHAPE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Launch L{h, s};
+    LAUNCH(L, kProfPrep, launch_prep_varlen(cu_seqlens, nseq, max_len, h->cfg.max_tokens, h->seq_start, h->seq_len,
+                                            h->n_rows, h->status, s));
+    return run_layers(h, L, ids, 0, nseq, 0, max_len, out, 0);
+}
+
+int albert_forward_host(albert_handle *h, const int64_t *ids_host, const uint8_t *mask_host, int B, int T,
+                        void *out_host, void *stream) {
+    if (!h || !ids_host || !mask_host || !out_host) return ALBERT_ERR_NULL;
+    if (B < 1 || T < 1 || T > h->cfg.max_pos || (long long)B * T > h->cfg.max_tokens) return ALBERT_ERR_SHAPE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t n = (size_t)B * T;
+    TRY(cudaMemcpyAsync(h->st_ids, ids_host, n * sizeof(int64_t), cudaMemcpyHostToDevice, s));
+    TRY(cudaMemcpyAsync(h->st_mask, mask_host, n, cudaMemcpyHostToDevice, s));
+    int rc = forward_padded(h, h->st_ids, h->st_mask, B, T, h->st_out, s);
+    if (rc) return rc;
+    TRY(cudaMemcpyAsync(out_host, h->st_out, n * out_width(h) * elem_bytes(h), cudaMemcpyDeviceToHost, s));
+    return albert_get_status(h, stream);
+}
+
+int albert_get_status(albert_handle *h, void *stream) {
+    if (!h) return ALBERT_ERR_NULL;
+    TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    int st = 0;
+    TRY(cudaMemcpy(&st, h->status, sizeof(int), cudaMemcpyDeviceToHost));
+    return st;
+}
+
+void albert_destroy(albert_handle *h) {
+    if (!h) return;
+    cudaDeviceSynchronize();
+    free_all(h);
+    delete h;
+}
+
+int albert_launches_per_forward(const albert_handle *h, int padded_api) {
+    if (!h) return -1;
+    const int per_layer = h->cfg.dtype == ALBERT_BF16 ? 5 : 7;
+    return 1 /*prep*/ + 1 /*embed*/ + 1 /*in proj*/ + per_layer * h->cfg.n_exec + 1 /*final or scatter*/ +
+           (padded_api ? 1 : 0);
+}
+
+int albert_profile_enable(albert_handle *h, int class_mask) {
+    if (!h) return ALBERT_ERR_NULL;
+    if (class_mask && h->ev.empty()) {
+        h->ev.resize(kEventPool);
+        h->ev_cls.assign(kEventPool, 0);
+        for (auto &e : h->ev) TRY(cudaEventCreate(&e));
+    }
+    h->prof_mask = (unsigned)class_mask & ((1u << kProfClasses) - 1u);
+    return ALBERT_OK;
+}
+
+int albert_profile_reset(albert_handle *h) {
+    if (!h) return ALBERT_ERR_NULL;
+    int rc = prof_harvest(h);
+    for (int i = 0; i < kProfClasses; ++i) { h->prof_launches[i] = 0; h->prof_ms[i] = 0.0; }
+    return rc;
+}
+
+int albert_profile_classes(void) { return kProfClasses; }
+
+const char *albert_profile_name(int cls) { return (cls >= 0 && cls < kProfClasses) ? kProfNames[cls] : ""; }
+
+int albert_profile_read(albert_handle *h, int *launches, double *ms) {
+    if (!h || !launches || !ms) return ALBERT_ERR_NULL;
+    int rc = prof_harvest(h);
+    for (int i = 0; i < kProfClasses; ++i) { launches[i] = h->prof_launches[i]; ms[i] = h->prof_ms[i]; }
+    return rc;
+}
+
+// ------------------------------------------------------ single-kernel entries --
+int albert_test_gemm(const void *A, const void *W, const float *bias, const void *R, const float *ln_g,
+                     const float *ln_b, float eps, const int32_t *row_dst, void *Y, int M, int N, int K,
+                     int epi, void *stream) {
+    if (!A || !W || !bias || !Y) return ALBERT_ERR_NULL;
+    if (M < 1 || N < gemm::BN || N % gemm::BN || K < gemm::BK || K % gemm::BK) return ALBERT_ERR_SHAPE;
+    if (epi < 0 || epi > 3) return ALBERT_ERR_CONFIG;
+    if (epi == kEpiLN && (!R || !ln_g || !ln_b || N != gemm::LN_N)) return ALBERT_ERR_CONFIG;
+    if (epi == kEpiScatter && !row_dst) return ALBERT_ERR_NULL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int dev = 0, sms = 0;
+    TRY(cudaGetDevice(&dev));
+    TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    const int rows_cap = (M + gemm::BM - 1) / gemm::BM * gemm::BM;
+    const int grid = gemm_grid(epi, rows_cap, N, sms);
+    CUtensorMap ta, tb;
+    if (make_tmap_bf16(&ta, A, M, K, gemm::BM) || make_tmap_bf16(&tb, W, N, K, gemm::BN)) return ALBERT_ERR_CUDA;
+    int *ints = nullptr;
+    float *scratch = nullptr;
+    TRY(cudaMalloc(&ints, 2 * sizeof(int)));
+    if (epi == kEpiLN && cudaMalloc(&scratch, gemm_ln_scratch_floats(grid) * sizeof(float)) != cudaSuccess) {
+        cudaFree(ints);
+        return ALBERT_ERR_ALLOC;
+    }
+    const int host_ints[2] = {M, 0};
+    cudaError_t e = cudaMemcpyAsync(ints, host_ints, sizeof(host_ints), cudaMemcpyHostToDevice, s);
+    GemmArgs a{};
+    a.N = N; a.K = K; a.rows_cap = rows_cap; a.n_rows = ints; a.bias = bias;
+    a.resid = static_cast<const bf16 *>(R); a.ld_resid = N; a.ln_g = ln_g; a.ln_b = ln_b; a.eps = eps;
+    a.out = static_cast<bf16 *>(Y); a.ld_out = N; a.scratch = scratch; a.row_dst = row_dst; a.status = ints + 1;
+    if (e == cudaSuccess) e = launch_gemm(epi, ta, tb, a, grid, s);
+    int st = 0;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&st, ints + 1, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    cudaFree(ints);
+    if (scratch) cudaFree(scratch);
+    return e == cudaSuccess ? st : ALBERT_ERR_CUDA;
+}
+
+int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, int max_len, void *ctx, int dtype,
+                          void *stream) {
+    if (!qkv || !cu_seqlens || !ctx) return ALBERT_ERR_NULL;
+    if (nseq < 1 || max_len < 1 || max_len > kMaxPos) return ALBERT_ERR_SHAPE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int *ints = nullptr;
+    TRY(cudaMalloc(&ints, (2 * (size_t)nseq + 4) * sizeof(int)));
+    int *seq_start = ints, *seq_len = ints + nseq + 1, *n_rows = seq_len + nseq + 1, *status = n_rows + 1;
+    cudaError_t e = launch_prep_varlen(cu_seqlens, nseq, max_len, 1 << 30, seq_start, seq_len, n_rows, status, s);
+    if (e == cudaSuccess) {
+        if (dtype == ALBERT_FP32)
+            e = launch_attention_f32(static_cast<const float *>(qkv), static_cast<float *>(ctx), seq_start, seq_len, nseq,
+                                     max_len, status, s);
+        else
+            e = launch_attention_bf16(static_cast<const bf16 *>(qkv), static_cast<bf16 *>(ctx), seq_start, seq_len, nseq,
+                                      max_len, status, s);
+    }
+    int st = 0;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&st, status, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    cudaFree(ints);
+    return e == cudaSuccess ? st : ALBERT_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,274 @@
+// attention.cu -- bidirectional multi-head attention with a key-padding mask.
+//
+// Per sequence b and head h ("ALBERT: How Kokoro's Phoneme Encoder Works",
+// section "Inside One Real ALBERT Layer", step 4; "How Kokoro TTS Works and
+// Where CKE Stands", section "What ALBERT does here"):
+//     C_h = softmax(Q_h K_h^T / sqrt(64) + mask) V_h,
+// where key u of sequence b takes part iff u < L_b (additive -inf mask) and
+// every query attends to keys on both sides.  Q, K, V live in one packed
+// [rows, 3*768] buffer (Q | K | V); head h is the 64-column slice 64h..64h+63
+// of each; the context goes to [rows, 768] with the same head layout.
+//
+// bf16 kernel: one CTA per (sequence, head, 128-query tile), 8 warps x 16
+// query rows.  The head's whole K and V (L_b <= 512 rows of 64 bf16) are
+// staged once in shared memory; each warp runs an online (max-subtracted)
+// softmax over 64-key blocks with mma.sync m16n8k16 (bf16 in, fp32 accumulate),
+// keeping P in registers between the two products.
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace albert {
+namespace {
+
+constexpr int QT = 128;      // query rows per CTA
+constexpr int KBLK = 64;     // keys per online-softmax block
+constexpr int LDS = 72;      // shared row stride in bf16 (144 B): conflict-free ldmatrix
+constexpr int ATT_THREADS = 256;
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const bf16 *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const bf16 *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__global__ void __launch_bounds__(ATT_THREADS)
+attn_bf16_kernel(const bf16 *__restrict__ qkv, bf16 *__restrict__ ctx, const int *__restrict__ seq_start,
+                 const int *__restrict__ seq_len, const int *__restrict__ status) {
+    if (*reinterpret_cast<const volatile int *>(status) != 0) return;
+    const int b = blockIdx.z, h = blockIdx.y, q0 = blockIdx.x * QT;
+    const int L = seq_len[b];
+    if (q0 >= L) return;
+    const int start = seq_start[b];
+    const int Lpad = (L + KBLK - 1) / KBLK * KBLK;
+
+    extern __shared__ uint4 smem4[];
+    bf16 *sQ = reinterpret_cast<bf16 *>(smem4);
+    bf16 *sK = sQ + QT * LDS;
+    bf16 *sV = sK + Lpad * LDS;
+
+    const uint4 zero = make_uint4(0, 0, 0, 0);
+    for (int i = threadIdx.x; i < Lpad * 8; i += ATT_THREADS) {
+        const int u = i >> 3, c = i & 7;
+        uint4 kv = zero, vv = zero;
+        if (u < L) {
+            const bf16 *row = qkv + (size_t)(start + u) * kQKV + h * kHeadDim + c * 8;
+            kv = __ldg(reinterpret_cast<const uint4 *>(row + kHidden));
+            vv = __ldg(reinterpret_cast<const uint4 *>(row + 2 * kHidden));
+        }
+        *reinterpret_cast<uint4 *>(sK + u * LDS + c * 8) = kv;
+        *reinterpret_cast<uint4 *>(sV + u * LDS + c * 8) = vv;
+    }
+    for (int i = threadIdx.x; i < QT * 8; i += ATT_THREADS) {
+        const int t = i >> 3, c = i & 7;
+        uint4 qv = zero;
+        if (q0 + t < L)
+            qv = __ldg(reinterpret_cast<const uint4 *>(qkv + (size_t)(start + q0 + t) * kQKV + h * kHeadDim + c * 8));
+        *reinterpret_cast<uint4 *>(sQ + t * LDS + c * 8) = qv;
+    }
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qw = q0 + warp * 16;
+    if (qw >= L) return;
+    const int g = lane >> 2, tig = lane & 3;
+
+    uint32_t qf[4][4];
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+        ldsm_x4(qf[ks], sQ + (warp * 16 + (lane & 15)) * LDS + ks * 16 + (lane >> 4) * 8);
+
+    // scores are kept in log2 units: s * (1/8) * log2(e)
+    const float sl2 = 0.125f * 1.4426950408889634f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float o[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+
+    const int j8 = lane >> 3, r8 = lane & 7;
+    for (int kb = 0; kb < Lpad; kb += KBLK) {
+        float s[8][4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t kf[4];
+                ldsm_x4(kf, sK + (kb + np * 16 + (j8 >> 1) * 8 + r8) * LDS + ks * 16 + (j8 & 1) * 8);
+                mma_bf16_16816(s[2 * np], qf[ks], kf[0], kf[1]);
+                mma_bf16_16816(s[2 * np + 1], qf[ks], kf[2], kf[3]);
+            }
+        }
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            const int key = kb + nt * 8 + tig * 2;
+            s[nt][0] = key < L ? s[nt][0] * sl2 : -INFINITY;
+            s[nt][1] = key + 1 < L ? s[nt][1] * sl2 : -INFINITY;
+            s[nt][2] = key < L ? s[nt][2] * sl2 : -INFINITY;
+            s[nt][3] = key + 1 < L ? s[nt][3] * sl2 : -INFINITY;
+            mx0 = fmaxf(mx0, fmaxf(s[nt][0], s[nt][1]));
+            mx1 = fmaxf(mx1, fmaxf(s[nt][2], s[nt][3]));
+        }
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: block holds a valid key
+        const float a0 = ex2_approx(m0 - mn0), a1 = ex2_approx(m1 - mn1);
+        m0 = mn0;
+        m1 = mn1;
+        float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            s[nt][0] = ex2_approx(s[nt][0] - mn0);
+            s[nt][1] = ex2_approx(s[nt][1] - mn0);
+            s[nt][2] = ex2_approx(s[nt][2] - mn1);
+            s[nt][3] = ex2_approx(s[nt][3] - mn1);
+            rs0 += s[nt][0] + s[nt][1];
+            rs1 += s[nt][2] + s[nt][3];
+        }
+        l0 = l0 * a0 + rs0;
+        l1 = l1 * a1 + rs1;
+#pragma unroll
+        for (int nd = 0; nd < 8; ++nd) {
+            o[nd][0] *= a0; o[nd][1] *= a0;
+            o[nd][2] *= a1; o[nd][3] *= a1;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t pa[4];
+            pa[0] = pack_bf16x2(s[2 * j][0], s[2 * j][1]);
+            pa[1] = pack_bf16x2(s[2 * j][2], s[2 * j][3]);
+            pa[2] = pack_bf16x2(s[2 * j + 1][0], s[2 * j + 1][1]);
+            pa[3] = pack_bf16x2(s[2 * j + 1][2], s[2 * j + 1][3]);
+#pragma unroll
+            for (int dp = 0; dp < 4; ++dp) {
+                uint32_t vf[4];
+                ldsm_x4_t(vf, sV + (kb + j * 16 + (j8 & 1) * 8 + r8) * LDS + dp * 16 + (j8 >> 1) * 8);
+                mma_bf16_16816(o[2 * dp], pa, vf[0], vf[1]);
+                mma_bf16_16816(o[2 * dp + 1], pa, vf[2], vf[3]);
+            }
+        }
+    }
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    const float i0 = 1.f / l0, i1 = 1.f / l1;
+    const int t0 = qw + g, t1 = qw + g + 8;
+#pragma unroll
+    for (int nd = 0; nd < 8; ++nd) {
+        const int col = h * kHeadDim + nd * 8 + tig * 2;
+        if (t0 < L)
+            *reinterpret_cast<uint32_t *>(ctx + (size_t)(start + t0) * kHidden + col) =
+                pack_bf16x2(o[nd][0] * i0, o[nd][1] * i0);
+        if (t1 < L)
+            *reinterpret_cast<uint32_t *>(ctx + (size_t)(start + t1) * kHidden + col) =
+                pack_bf16x2(o[nd][2] * i1, o[nd][3] * i1);
+    }
+}
+
+// fp32 kernel: one warp per query row; scores of the row in shared memory.
+constexpr int F32_ROWS = 8;
+__global__ void __launch_bounds__(32 * F32_ROWS)
+attn_f32_kernel(const float *__restrict__ qkv, float *__restrict__ ctx, const int *__restrict__ seq_start,
+                const int *__restrict__ seq_len, const int *__restrict__ status, int max_len) {
+    if (*reinterpret_cast<const volatile int *>(status) != 0) return;
+    const int b = blockIdx.z, h = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * F32_ROWS + warp;
+    const int L = seq_len[b];
+    if (t >= L) return;
+    const int start = seq_start[b];
+    extern __shared__ float fsm[];
+    float *sc = fsm + warp * max_len;
+    float *qs = fsm + F32_ROWS * max_len + warp * kHeadDim;
+    const float *qrow = qkv + (size_t)(start + t) * kQKV + h * kHeadDim;
+    qs[lane] = qrow[lane];
+    qs[lane + 32] = qrow[lane + 32];
+    __syncwarp();
+    const float scale = 0.125f;
+    float mx = -INFINITY;
+    for (int u = lane; u < L; u += 32) {
+        const float *k = qkv + (size_t)(start + u) * kQKV + kHidden + h * kHeadDim;
+        float d = 0.f;
+        for (int i = 0; i < kHeadDim; ++i) d = fmaf(qs[i], k[i], d);
+        d *= scale;
+        sc[u] = d;
+        mx = fmaxf(mx, d);
+    }
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float den = 0.f;
+    for (int u = lane; u < L; u += 32) {
+        const float e = expf(sc[u] - mx);
+        sc[u] = e;
+        den += e;
+    }
+    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    __syncwarp();
+    const float inv = 1.f / den;
+    float a0 = 0.f, a1 = 0.f;
+    for (int u = 0; u < L; ++u) {
+        const float *v = qkv + (size_t)(start + u) * kQKV + 2 * kHidden + h * kHeadDim;
+        a0 = fmaf(sc[u], v[lane], a0);
+        a1 = fmaf(sc[u], v[lane + 32], a1);
+    }
+    float *crow = ctx + (size_t)(start + t) * kHidden + h * kHeadDim;
+    crow[lane] = a0 * inv;
+    crow[lane + 32] = a1 * inv;
+}
+
+}  // namespace
+
+static size_t attn_bf16_smem(int max_len) {
+    const int lpad = (max_len + KBLK - 1) / KBLK * KBLK;
+    return (size_t)(QT + 2 * lpad) * LDS * sizeof(bf16);
+}
+
+cudaError_t launch_attention_bf16(const bf16 *qkv, bf16 *ctx, const int *seq_start,
+                                  const int *seq_len, int nseq, int max_len, const int *status,
+                                  cudaStream_t s) {
+    if (nseq <= 0) return cudaSuccess;
+    const size_t smem = attn_bf16_smem(max_len);
+    static size_t configured = 0;
+    if (smem > configured) {
+        cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)attn_bf16_smem(kMaxPos));
+        if (e != cudaSuccess) return e;
+        configured = attn_bf16_smem(kMaxPos);
+    }
+    dim3 grid((max_len + QT - 1) / QT, kHeads, nseq);
+    attn_bf16_kernel<<<grid, ATT_THREADS, smem, s>>>(qkv, ctx, seq_start, seq_len, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attention_f32(const float *qkv, float *ctx, const int *seq_start,
+                                 const int *seq_len, int nseq, int max_len, const int *status,
+                                 cudaStream_t s) {
+    if (nseq <= 0) return cudaSuccess;
+    const size_t smem = (size_t)F32_ROWS * (max_len + kHeadDim) * sizeof(float);
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)((size_t)F32_ROWS * (kMaxPos + kHeadDim) * sizeof(float)));
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    dim3 grid((max_len + F32_ROWS - 1) / F32_ROWS, kHeads, nseq);
+    attn_f32_kernel<<<grid, 32 * F32_ROWS, smem, s>>>(qkv, ctx, seq_start, seq_len, status, max_len);
+    return cudaGetLastError();
+}
+
+}  // namespace albert

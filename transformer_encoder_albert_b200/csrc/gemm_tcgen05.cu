@@ -1,0 +1,436 @@
+// gemm_tcgen05.cu -- persistent BF16 GEMM for sm_100a: Y = epi(A W^T + bias).
+//
+// The dense contractions of the encoder (the 128->768 input projection, the
+// fused Q|K|V projection, the attention output projection, both FFN matrices
+// and the 768->512 final projection; "ALBERT: How Kokoro's Phoneme Encoder
+// Works", section "Inside One Real ALBERT Layer", steps 2-6) all run here.
+// A linear layer is y_j = b_j + sum_i x_i W_{j,i} with W stored [out, in]
+// ("Qwen3-TTS and Kokoro", section A), i.e. both operands are K-major.
+//
+// Design (one CTA per SM, persistent over work units):
+//   warp 0      : TMA producer, 4-stage ring of {A 128x64, B 256x64} bf16 tiles
+//                 (128-byte swizzle, no multicast);
+//   warp 1      : TMEM allocator + single-thread tcgen05.mma issuer into two
+//                 128x256 fp32 accumulators (512 TMEM columns), so the epilogue
+//                 of one tile overlaps the main loop of the next;
+//   warps 2..9  : epilogue, 2 warps per TMEM lane quadrant (column halves);
+//                 tcgen05.ld -> bias (+ tanh-GELU | + residual, LayerNorm) ->
+//                 bf16 stores.
+// LayerNorm epilogue (post-LN steps 5 and 6): a work unit is a full 128x768
+// row block (3 sub-tiles of 256 columns).  Each thread owns one row half;
+// it keeps exact running (mean, M2) statistics per 32-column chunk (Chan's
+// merge), parks the fp32 pre-norm row in a per-CTA scratch slot that stays
+// L2-resident, exchanges statistics with the partner warp through shared
+// memory, then normalizes from the scratch slot.
+// Every wait is bounded (%globaltimer); on expiry the CTA records
+// ALBERT_ERR_TIMEOUT, drains its in-flight copies and MMAs, frees TMEM and exits.
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace albert {
+namespace {
+
+using namespace gemm;
+
+struct Smem {
+    uint8_t *a, *b;
+    uint64_t *full, *empty, *tfull, *tempty, *drain;
+    uint32_t *tmem_slot;
+    volatile int *abort_flag;
+    int *misc;               // [0] n_rows, [1] status at entry
+    volatile int *pair_flag; // [4 quadrants][2 halves]
+    float2 *stats;           // [2 buffers][2 halves][BM]
+};
+
+__device__ __forceinline__ Smem carve(uint8_t *raw) {
+    Smem s;
+    uint8_t *p = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    s.a = p;
+    s.b = p + STAGES * A_BYTES;
+    uint8_t *ctrl = s.b + STAGES * B_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl);
+    s.full = bars;
+    s.empty = bars + STAGES;
+    s.tfull = bars + 2 * STAGES;
+    s.tempty = bars + 2 * STAGES + 2;
+    s.drain = bars + 2 * STAGES + 4;
+    uint32_t *u = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
+    s.tmem_slot = u;
+    s.abort_flag = reinterpret_cast<volatile int *>(u + 1);
+    s.misc = reinterpret_cast<int *>(u + 2);
+    s.pair_flag = reinterpret_cast<volatile int *>(u + 4);
+    s.stats = reinterpret_cast<float2 *>(ctrl + 1024);
+    return s;
+}
+
+// Wait on the partner warp's flag (bounded); only lane 0 polls.
+__device__ __forceinline__ bool wait_flag(volatile int *flag, int target, volatile int *abort_flag) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) {
+        const unsigned long long t0 = globaltimer_ns();
+        while (*flag < target) {
+            if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                ok = false;
+                break;
+            }
+        }
+    }
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    __threadfence_block();
+    __syncwarp();
+    return ok;
+}
+
+__device__ __forceinline__ void store_bf16x32(bf16 *dst, const float (&v)[32]) {
+    uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 w;
+        w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+        w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+        w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+        w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+        d[q] = w;
+    }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(THREADS, 1)
+gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const GemmArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem sm = carve(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        sm.misc[0] = *reinterpret_cast<const volatile int *>(p.n_rows);
+        sm.misc[1] = *reinterpret_cast<const volatile int *>(p.status);
+        *sm.abort_flag = 0;
+        for (int i = 0; i < 8; ++i) sm.pair_flag[i] = 0;
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(smem_u32(&sm.full[i]), 1);
+            mbar_init(smem_u32(&sm.empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&sm.tfull[i]), 1);
+            mbar_init(smem_u32(&sm.tempty[i]), EPI_WARPS);
+        }
+        mbar_init(smem_u32(sm.drain), 1);
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    __syncthreads();
+    // An earlier kernel of this forward failed, or the row count is out of range.
+    if (sm.misc[1] != 0 || sm.misc[0] < 0 || sm.misc[0] > p.rows_cap) return;
+
+    if (warp == 1) {
+        tmem_alloc(smem_u32(sm.tmem_slot), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *sm.tmem_slot;
+
+    const int n_rows = sm.misc[0];
+    const int m_blocks = (n_rows + BM - 1) / BM;
+    const int n_sub = p.N / BN;
+    const int units = (EPI == kEpiLN) ? m_blocks : m_blocks * n_sub;
+    const int subs = (EPI == kEpiLN) ? n_sub : 1;
+    const int kblocks = p.K / BK;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer --
+        if (lane == 0) {
+            const uint64_t keep = policy_evict_last();  // weights: reused by every CTA
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                const int m = (EPI == kEpiLN) ? u : u / n_sub;
+                const int n0 = (EPI == kEpiLN) ? 0 : u % n_sub;
+                for (int s = 0; s < subs && ok; ++s) {
+                    for (int kb = 0; kb < kblocks; ++kb) {
+                        if (!mbar_wait(smem_u32(&sm.empty[stage]), phase ^ 1, sm.abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t fb = smem_u32(&sm.full[stage]);
+                        mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
+                        tma_load_2d(smem_u32(sm.a + stage * A_BYTES), &tmA, fb, kb * BK, m * BM);
+                        tma_load_2d_hint(smem_u32(sm.b + stage * B_BYTES), &tmB, fb, kb * BK,
+                                         (n0 + s) * BN, keep);
+                        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    }
+                }
+            }
+            if (!ok) {
+                // Drain: every stage whose load may still be in flight completes
+                // its transaction count before the CTA's shared memory goes away.
+                for (int i = 0; i < STAGES; ++i) {
+                    if (--stage < 0) { stage = STAGES - 1; phase ^= 1; }
+                    mbar_wait_drain(smem_u32(&sm.full[stage]), phase);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // -------------------------------------------------------- MMA issuer --
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(BM, BN);
+            int stage = 0, acc = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                for (int s = 0; s < subs && ok; ++s) {
+                    const int ab = acc & 1;
+                    const uint32_t aph = (acc >> 1) & 1;
+                    if (!mbar_wait(smem_u32(&sm.tempty[ab]), aph ^ 1, sm.abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d = tmem_base + ab * BN;
+                    for (int kb = 0; kb < kblocks; ++kb) {
+                        if (!mbar_wait(smem_u32(&sm.full[stage]), phase, sm.abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t a0 = smem_u32(sm.a + stage * A_BYTES);
+                        const uint32_t b0 = smem_u32(sm.b + stage * B_BYTES);
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k)
+                            umma_bf16(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32),
+                                      idesc, (kb | k) != 0);
+                        umma_commit(smem_u32(&sm.empty[stage]));
+                        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    }
+                    if (!ok) break;
+                    umma_commit(smem_u32(&sm.tfull[ab]));
+                    ++acc;
+                }
+            }
+            // All MMAs issued by this thread complete before TMEM is released.
+            umma_commit(smem_u32(sm.drain));
+            mbar_wait_drain(smem_u32(sm.drain), 0);
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue --
+        const int ew = warp - 2;            // 0..7
+        const int quad = warp & 3;          // TMEM lanes 32*quad .. 32*quad+31
+        const int half = ew >> 2;           // column half of a 256-wide sub-tile
+        const int r_local = quad * 32 + lane;
+        int acc = 0, it = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++it) {
+            const int m = (EPI == kEpiLN) ? u : u / n_sub;
+            const int n0 = (EPI == kEpiLN) ? 0 : u % n_sub;
+            const int row = m * BM + r_local;
+            const bool row_ok = row < n_rows;
+            float mean = 0.f, m2 = 0.f, cnt = 0.f;
+            float *slot = (EPI == kEpiLN) ? p.scratch + (size_t)blockIdx.x * BM * p.N : nullptr;
+            int dst = row;
+            if (EPI == kEpiScatter) dst = row_ok ? __ldg(p.row_dst + row) : -1;
+
+            for (int s = 0; s < subs; ++s) {
+                const int ab = acc & 1;
+                const uint32_t aph = (acc >> 1) & 1;
+                bool got = mbar_wait(smem_u32(&sm.tfull[ab]), aph, sm.abort_flag);
+                got = __all_sync(0xffffffffu, got);
+                if (!got) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + ab * BN + half * 128;
+                const int ncol0 = (n0 + s) * BN + half * 128;  // first output column
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + c * 32, r);
+                    tmem_ld_wait();
+                    if (c == 3) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(smem_u32(&sm.tempty[ab]));
+                    }
+                    const int col0 = ncol0 + c * 32;
+                    float v[32];
+                    const float4 *bias4 = reinterpret_cast<const float4 *>(p.bias + col0);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 bb = __ldg(bias4 + q);
+                        v[4 * q + 0] = __uint_as_float(r[4 * q + 0]) + bb.x;
+                        v[4 * q + 1] = __uint_as_float(r[4 * q + 1]) + bb.y;
+                        v[4 * q + 2] = __uint_as_float(r[4 * q + 2]) + bb.z;
+                        v[4 * q + 3] = __uint_as_float(r[4 * q + 3]) + bb.w;
+                    }
+                    if (EPI == kEpiBias) {
+                        if (row_ok) store_bf16x32(p.out + (size_t)row * p.ld_out + col0, v);
+                    } else if (EPI == kEpiGelu) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = gelu_tanh_fast(v[j]);
+                        if (row_ok) store_bf16x32(p.out + (size_t)row * p.ld_out + col0, v);
+                    } else if (EPI == kEpiScatter) {
+                        if (dst >= 0) store_bf16x32(p.out + (size_t)dst * p.ld_out + col0, v);
+                    } else {
+                        // residual
+                        if (row_ok) {
+                            const uint4 *rr = reinterpret_cast<const uint4 *>(p.resid + (size_t)row * p.ld_resid + col0);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const uint4 w = __ldg(rr + q);
+                                float2 f;
+                                f = unpack_bf16x2(w.x); v[8 * q + 0] += f.x; v[8 * q + 1] += f.y;
+                                f = unpack_bf16x2(w.y); v[8 * q + 2] += f.x; v[8 * q + 3] += f.y;
+                                f = unpack_bf16x2(w.z); v[8 * q + 4] += f.x; v[8 * q + 5] += f.y;
+                                f = unpack_bf16x2(w.w); v[8 * q + 6] += f.x; v[8 * q + 7] += f.y;
+                            }
+                        }
+                        // exact chunk statistics, merged into the running ones
+                        float cs = 0.f;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) cs += v[j];
+                        const float cm = cs * (1.0f / 32.0f);
+                        float cq = 0.f;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) { const float d = v[j] - cm; cq = fmaf(d, d, cq); }
+                        if (cnt == 0.f) {
+                            mean = cm; m2 = cq;
+                        } else {
+                            const float nn = cnt + 32.f, d = cm - mean;
+                            mean = fmaf(d, 32.f / nn, mean);
+                            m2 += cq + d * d * (cnt * 32.f / nn);
+                        }
+                        cnt += 32.f;
+                        // park the pre-norm values: layout [col/4][BM][4] (coalesced per warp)
+                        float4 *sl = reinterpret_cast<float4 *>(slot);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            sl[(size_t)(col0 / 4 + q) * BM + r_local] =
+                                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    }
+                }
+                ++acc;
+            }
+            if (!ok) break;
+
+            if (EPI == kEpiLN) {
+                // combine the two column halves of each row (partner warp = other half)
+                float2 *st = sm.stats + (size_t)((it & 1) * 2 + half) * BM;
+                st[r_local] = make_float2(mean, m2);
+                __syncwarp();
+                __threadfence_block();
+                if (lane == 0) sm.pair_flag[quad * 2 + half] = it + 1;
+                if (!wait_flag(&sm.pair_flag[quad * 2 + (half ^ 1)], it + 1, sm.abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const float2 o = sm.stats[(size_t)((it & 1) * 2 + (half ^ 1)) * BM + r_local];
+                const float nh = cnt;  // both halves hold the same count
+                const float d = o.x - mean;
+                const float mu = mean + 0.5f * d;
+                const float var = (m2 + o.y + d * d * (nh * 0.5f)) / (2.f * nh);
+                const float rstd = rsqrtf(var + p.eps);
+                if (row_ok) {
+                    const float4 *sl = reinterpret_cast<const float4 *>(slot);
+#pragma unroll 1
+                    for (int s = 0; s < subs; ++s) {
+#pragma unroll 1
+                        for (int c = 0; c < 4; ++c) {
+                            const int col0 = s * BN + half * 128 + c * 32;
+                            float v[32];
+                            const float4 *g4 = reinterpret_cast<const float4 *>(p.ln_g + col0);
+                            const float4 *b4 = reinterpret_cast<const float4 *>(p.ln_b + col0);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const float4 z = sl[(size_t)(col0 / 4 + q) * BM + r_local];
+                                const float4 g = __ldg(g4 + q), bb = __ldg(b4 + q);
+                                v[4 * q + 0] = fmaf((z.x - mu) * rstd, g.x, bb.x);
+                                v[4 * q + 1] = fmaf((z.y - mu) * rstd, g.y, bb.y);
+                                v[4 * q + 2] = fmaf((z.z - mu) * rstd, g.z, bb.z);
+                                v[4 * q + 3] = fmaf((z.w - mu) * rstd, g.w, bb.w);
+                            }
+                            store_bf16x32(p.out + (size_t)row * p.ld_out + col0, v);
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+    if (threadIdx.x == 0 && *sm.abort_flag) set_status(p.status, kStatusTimeout);
+}
+
+}  // namespace
+
+int gemm_grid(int epi, int rows_cap, int N, int num_sms) {
+    const int m_blocks = (rows_cap + BM - 1) / BM;
+    const int units = (epi == kEpiLN) ? m_blocks : m_blocks * (N / BN);
+    return units < num_sms ? (units > 0 ? units : 1) : num_sms;
+}
+
+template <int EPI>
+static cudaError_t launch_one(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmArgs &a,
+                              int grid, cudaStream_t s) {
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_bf16_kernel<EPI>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    gemm_bf16_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmB, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                        const GemmArgs &a, int grid, cudaStream_t s) {
+    switch (epi) {
+        case kEpiBias: return launch_one<kEpiBias>(tmA, tmB, a, grid, s);
+        case kEpiGelu: return launch_one<kEpiGelu>(tmA, tmB, a, grid, s);
+        case kEpiLN: return launch_one<kEpiLN>(tmA, tmB, a, grid, s);
+        case kEpiScatter: return launch_one<kEpiScatter>(tmA, tmB, a, grid, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+// ------------------------------------------------------------ tensor maps --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+int make_tmap_bf16(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return -1;
+    if ((reinterpret_cast<uintptr_t>(base) & 15) || (cols * 2) % 16) return -2;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? 0 : -3;
+}
+
+}  // namespace albert

@@ -1,0 +1,247 @@
+// prep_embed.cu -- batch preparation, the three-table embedding + LayerNorm, and
+// the output-side kernels (padding rows, row scatter).
+//
+// Embedding ("ALBERT: How Kokoro's Phoneme Encoder Works", section "Inside One
+// Real ALBERT Layer", step 1; section "1. Factorized embedding" for the table
+// sizes): e = word[id] + pos[t] + type[0], E = LN_128(e; gamma, beta, eps).
+// Checked-input convention ("How Kokoro TTS Works and Where CKE Stands":
+// invalid ids and arena rejection are detected before any output is written;
+// a failed check stops downstream work): these kernels record an error in
+// the device status word and every later kernel of the forward returns
+// without writing.
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace albert {
+namespace {
+
+constexpr int PREP_THREADS = 1024;
+
+// Block-wide exclusive scan of rows[b] (b < n) into start[b]; returns the total.
+__device__ int block_exclusive_scan(const int *rows, int n, int *start, int *sh) {
+    const int tid = threadIdx.x;
+    const int chunk = (n + PREP_THREADS - 1) / PREP_THREADS;
+    const int lo = min(n, tid * chunk), hi = min(n, lo + chunk);
+    int local = 0;
+    for (int i = lo; i < hi; ++i) local += rows[i];
+    sh[tid] = local;
+    __syncthreads();
+    for (int off = 1; off < PREP_THREADS; off <<= 1) {
+        const int v = tid >= off ? sh[tid - off] : 0;
+        __syncthreads();
+        sh[tid] += v;
+        __syncthreads();
+    }
+    int run = sh[tid] - local;  // exclusive prefix of this thread's chunk
+    for (int i = lo; i < hi; ++i) {
+        const int v = rows[i];  // rows and start may be the same array
+        start[i] = run;
+        run += v;
+    }
+    const int total = sh[PREP_THREADS - 1];
+    __syncthreads();
+    return total;
+}
+
+// Padded batch: mask[B, T] must hold, per row, a non-empty prefix of non-zero
+// bytes followed only by zeros.  L_b = prefix length.  Packed mode gives
+// sequence b L_b rows, padded mode T rows.
+__global__ void __launch_bounds__(PREP_THREADS)
+prep_padded_kernel(const uint8_t *__restrict__ mask, int B, int T, int pack, int rows_cap,
+                   int *seq_start, int *seq_len, int *n_rows, int *status) {
+    __shared__ int sh[PREP_THREADS];
+    __shared__ int bad;
+    if (threadIdx.x == 0) { *status = 0; bad = 0; }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int b = warp; b < B; b += PREP_THREADS / 32) {
+        const uint8_t *m = mask + (size_t)b * T;
+        int first_zero = T, last_one = -1;
+        for (int t = lane; t < T; t += 32) {
+            const bool on = m[t] != 0;
+            if (!on) first_zero = min(first_zero, t);
+            else last_one = max(last_one, t);
+        }
+        for (int o = 16; o; o >>= 1) {
+            first_zero = min(first_zero, __shfl_xor_sync(0xffffffffu, first_zero, o));
+            last_one = max(last_one, __shfl_xor_sync(0xffffffffu, last_one, o));
+        }
+        const bool ok = first_zero >= 1 && last_one < first_zero;
+        if (lane == 0) {
+            seq_len[b] = ok ? first_zero : 0;
+            if (!ok) bad = 1;
+        }
+    }
+    __syncthreads();
+    if (bad) {
+        if (threadIdx.x == 0) { set_status(status, kStatusMask); *n_rows = 0; }
+        return;
+    }
+    // rows per sequence, reusing seq_start as the input of the scan
+    for (int b = threadIdx.x; b < B; b += PREP_THREADS) seq_start[b] = pack ? seq_len[b] : T;
+    __syncthreads();
+    const int total = block_exclusive_scan(seq_start, B, seq_start, sh);
+    if (threadIdx.x == 0) {
+        *n_rows = total;
+        if (total > rows_cap) set_status(status, kStatusShape);
+    }
+}
+
+// Packed batch: cu[0] == 0, 1 <= cu[s+1]-cu[s] <= max_len, cu[nseq] <= rows_cap.
+__global__ void __launch_bounds__(PREP_THREADS)
+prep_varlen_kernel(const int32_t *__restrict__ cu, int nseq, int max_len, int rows_cap,
+                   int *seq_start, int *seq_len, int *n_rows, int *status) {
+    __shared__ int bad;
+    if (threadIdx.x == 0) { *status = 0; bad = 0; }
+    __syncthreads();
+    for (int s = threadIdx.x; s < nseq; s += PREP_THREADS) {
+        const int a = cu[s], e = cu[s + 1];
+        const int len = e - a;
+        seq_start[s] = a;
+        seq_len[s] = len;
+        if (len < 1 || len > max_len || (s == 0 && a != 0)) bad = 1;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int total = cu[nseq];
+        if (bad) {
+            set_status(status, kStatusSeqlens);
+            *n_rows = 0;
+        } else if (total > rows_cap) {
+            set_status(status, kStatusShape);
+            *n_rows = 0;
+        } else {
+            *n_rows = total;
+        }
+    }
+}
+
+// One warp per row: gather the three table rows, LayerNorm over 128 (two-pass,
+// fp32), write E (bf16 or fp32) and the row's destination in the output.
+__global__ void __launch_bounds__(256)
+embed_ln_kernel(const EmbedArgs a) {
+    if (*reinterpret_cast<const volatile int *>(a.status) != 0) return;
+    const int n_rows = *a.n_rows;
+    const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (r >= n_rows) return;
+    // sequence of row r: last b with seq_start[b] <= r
+    int lo = 0, hi = a.nseq - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(a.seq_start + mid) <= r) lo = mid; else hi = mid - 1;
+    }
+    const int b = lo;
+    const int t = r - __ldg(a.seq_start + b);
+    const bool valid = t < __ldg(a.seq_len + b);
+    long long id = a.ids_padded ? a.ids[(size_t)b * a.T + t] : a.ids[r];
+    if (id < 0 || id >= a.vocab) {
+        if (valid) set_status(a.status, kStatusId);
+        id = 0;  // padding slot: any id; its row never reaches a valid output
+    }
+    const float4 w = __ldg(reinterpret_cast<const float4 *>(a.word + id * kEmb) + lane);
+    const float4 ps = __ldg(reinterpret_cast<const float4 *>(a.pos + (size_t)t * kEmb) + lane);
+    const float4 ty = __ldg(reinterpret_cast<const float4 *>(a.type) + lane);
+    float x[4] = {w.x + ps.x + ty.x, w.y + ps.y + ty.y, w.z + ps.z + ty.z, w.w + ps.w + ty.w};
+    float s = x[0] + x[1] + x[2] + x[3];
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float mu = s * (1.0f / kEmb);
+    float q = 0.f;
+    for (int i = 0; i < 4; ++i) { const float d = x[i] - mu; q = fmaf(d, d, q); }
+    for (int o = 16; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    const float rstd = rsqrtf(q * (1.0f / kEmb) + a.eps);
+    const float4 g = __ldg(reinterpret_cast<const float4 *>(a.g) + lane);
+    const float4 bb = __ldg(reinterpret_cast<const float4 *>(a.b) + lane);
+    const float y0 = fmaf((x[0] - mu) * rstd, g.x, bb.x), y1 = fmaf((x[1] - mu) * rstd, g.y, bb.y);
+    const float y2 = fmaf((x[2] - mu) * rstd, g.z, bb.z), y3 = fmaf((x[3] - mu) * rstd, g.w, bb.w);
+    if (a.out_f32) {
+        reinterpret_cast<float4 *>(static_cast<float *>(a.E) + (size_t)r * kEmb)[lane] = make_float4(y0, y1, y2, y3);
+    } else {
+        uint2 u;
+        u.x = pack_bf16x2(y0, y1);
+        u.y = pack_bf16x2(y2, y3);
+        reinterpret_cast<uint2 *>(static_cast<bf16 *>(a.E) + (size_t)r * kEmb)[lane] = u;
+    }
+    if (lane == 0) a.row_dst[r] = valid ? (a.dst_padded ? b * a.T + t : r) : -1;
+}
+
+__global__ void zero_pad_kernel(uint4 *out, int B, int T, int chunks_per_row, const int *seq_len,
+                                const int *status) {
+    if (*reinterpret_cast<const volatile int *>(status) != 0) return;
+    const size_t n = (size_t)B * T * chunks_per_row;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const size_t row = i / chunks_per_row;
+        const int b = (int)(row / T), t = (int)(row % T);
+        if (t >= __ldg(seq_len + b)) out[i] = make_uint4(0, 0, 0, 0);
+    }
+}
+
+__global__ void scatter_rows_kernel(const uint4 *X, uint4 *out, int chunks_per_row, int rows_cap,
+                                    const int *n_rows, const int *row_dst, const int *status) {
+    if (*reinterpret_cast<const volatile int *>(status) != 0) return;
+    const int rows = *n_rows;
+    const size_t n = (size_t)rows * chunks_per_row;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const int r = (int)(i / chunks_per_row), c = (int)(i % chunks_per_row);
+        const int d = __ldg(row_dst + r);
+        if (d >= 0) out[(size_t)d * chunks_per_row + c] = X[i];
+    }
+}
+
+__global__ void f32_to_bf16_kernel(const float *src, bf16 *dst, size_t n) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        dst[i] = __float2bfloat16_rn(src[i]);
+}
+
+}  // namespace
+
+cudaError_t launch_prep_padded(const uint8_t *mask, int B, int T, int pack, int rows_cap,
+                               int *seq_start, int *seq_len, int *n_rows, int *status,
+                               cudaStream_t s) {
+    prep_padded_kernel<<<1, PREP_THREADS, 0, s>>>(mask, B, T, pack, rows_cap, seq_start, seq_len, n_rows, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prep_varlen(const int32_t *cu, int nseq, int max_len, int rows_cap,
+                               int *seq_start, int *seq_len, int *n_rows, int *status,
+                               cudaStream_t s) {
+    prep_varlen_kernel<<<1, PREP_THREADS, 0, s>>>(cu, nseq, max_len, rows_cap, seq_start, seq_len, n_rows, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_embed(const EmbedArgs &a, cudaStream_t s) {
+    const int blocks = (a.rows_cap + 7) / 8;
+    embed_ln_kernel<<<blocks, 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+static int grid_for(size_t n, int threads) {
+    size_t b = (n + threads - 1) / threads;
+    if (b > 148 * 16) b = 148 * 16;
+    return b < 1 ? 1 : (int)b;
+}
+
+cudaError_t launch_zero_pad(void *out, int B, int T, int D, int elem_bytes, const int *seq_len,
+                            const int *status, cudaStream_t s) {
+    const int cpr = D * elem_bytes / 16;
+    const size_t n = (size_t)B * T * cpr;
+    zero_pad_kernel<<<grid_for(n, 256), 256, 0, s>>>(static_cast<uint4 *>(out), B, T, cpr, seq_len, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_rows(const void *X, void *out, int D, int elem_bytes, int rows_cap,
+                                const int *n_rows, const int *row_dst, const int *status,
+                                cudaStream_t s) {
+    const int cpr = D * elem_bytes / 16;
+    const size_t n = (size_t)rows_cap * cpr;
+    scatter_rows_kernel<<<grid_for(n, 256), 256, 0, s>>>(static_cast<const uint4 *>(X), static_cast<uint4 *>(out),
+                                                         cpr, rows_cap, n_rows, row_dst, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_f32_to_bf16(const float *src, bf16 *dst, size_t n, cudaStream_t s) {
+    f32_to_bf16_kernel<<<grid_for(n, 256), 256, 0, s>>>(src, dst, n);
+    return cudaGetLastError();
+}
+
+}  // namespace albert
