@@ -183,6 +183,32 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
 int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, int max_len,
                           void *ctx, int dtype, void *stream);
 
+/* ---- residual + LayerNorm GEMM without any device allocation ----
+ * The pages have no counterpart of this entry point; it exists for callers
+ * that must not allocate device memory while running -- a real-time audio
+ * thread that cannot absorb cudaMalloc's device-wide synchronization and
+ * latency, or a runtime that lays out all device memory before its first
+ * request.  It computes Y = LN(A W^T + bias + R; ln_g, ln_b, eps) exactly like
+ * albert_test_gemm with epi = 2, but its scratch (fp32 row slots of the
+ * LayerNorm epilogue, a row-count word and the status word) lives in a
+ * file-scope __device__ array of 6 MiB inside the library instead of memory
+ * the call allocates; it calls no cudaMalloc/cudaFree.
+ *   A: [M, K] bf16, W: [768, K] bf16, bias/ln_g/ln_b: [768] fp32,
+ *   R: [M, 768] bf16, Y: [M, 768] bf16, all device pointers the caller owns.
+ *   Limits: 1 <= M <= 2048 (the array holds 16 row blocks of 128), K % 64 == 0;
+ *   anything else returns ALBERT_ERR_SHAPE before any work is enqueued.
+ * The array is reserved on every device where the library's module holding it
+ * is loaded and stays until the process exits.  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress) with that device
+ * current; make that first call before any stream capture.  Every call shares
+ * the one array (its status word is reset by each call, the row slots are
+ * fully rewritten before they are read), so calls that overlap on the GPU --
+ * on different streams or from different threads -- race and must be
+ * serialized by the caller.  Synchronous: returns the kernel's status. */
+int albert_gemm_residual_ln_noalloc(const void *A, const void *W, const float *bias, const void *R,
+                                    const float *ln_g, const float *ln_b, float eps, void *Y, int M,
+                                    int K, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -37,6 +37,7 @@ EXPORTS = (
     "albert_get_status", "albert_destroy", "albert_launches_per_forward",
     "albert_profile_enable", "albert_profile_reset", "albert_profile_classes",
     "albert_profile_name", "albert_profile_read", "albert_test_gemm", "albert_test_attention",
+    "albert_gemm_residual_ln_noalloc",
 )
 
 
@@ -84,6 +85,7 @@ def lib() -> C.CDLL:
         L.albert_profile_read.argtypes = [vp, C.POINTER(C.c_int), C.POINTER(C.c_double)]
         L.albert_test_gemm.argtypes = [vp, vp, vp, vp, vp, vp, C.c_float, vp, vp, i, i, i, i, vp]
         L.albert_test_attention.argtypes = [vp, vp, i, i, vp, i, vp]
+        L.albert_gemm_residual_ln_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, C.c_float, vp, i, i, vp]
         _lib = L
     return _lib
 
@@ -251,3 +253,12 @@ def test_attention(qkv, cu_seqlens, max_len: int, ctx, fp32: bool = False, strea
     return lib().albert_test_attention(_ptr(qkv), _ptr(cu_seqlens), cu_seqlens.numel() - 1,
                                        int(max_len), _ptr(ctx), ALBERT_FP32 if fp32 else ALBERT_BF16,
                                        _stream_ptr(stream))
+
+
+def gemm_residual_ln_noalloc(A, W, bias, R, ln_g, ln_b, Y, eps: float = 1e-12, stream=None) -> int:
+    """Y = LN(A W^T + bias + R) through the entry point that allocates no device
+    memory (static scratch inside the library; M <= 2048)."""
+    M, K = A.shape
+    return lib().albert_gemm_residual_ln_noalloc(_ptr(A), _ptr(W), _ptr(bias), _ptr(R), _ptr(ln_g),
+                                                 _ptr(ln_b), float(eps), _ptr(Y), M, K,
+                                                 _stream_ptr(stream))
