@@ -131,6 +131,25 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(inside)}
 
 
+def nvidia_smi_id(torch, local: int) -> str:
+    """nvidia-smi --id for the CUDA device `local`: its UUID, else its index."""
+    try:
+        uu = torch.cuda.get_device_properties(local).uuid
+        raw = getattr(uu, "bytes", None)
+        if raw is not None and len(raw) == 16:
+            h = bytes(raw).hex()
+            return f"GPU-{h[:8]}-{h[8:12]}-{h[12:16]}-{h[16:20]}-{h[20:]}"
+        u = str(uu)
+        if u and not u.startswith("<"):
+            return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        pass
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        return vis.split(",")[local].strip()
+    return str(local)
+
+
 # -------------------------------------------------------------- oracle arm ---
 
 def oracle_throughput(weights, ids, mask, L, arch, budget_s=None, steps=None, warmup=0):
@@ -250,8 +269,7 @@ def run_gpu(args):
         raise SystemExit(f"device status {enc.status()}")
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
 
-    gpu_id = getattr(torch.cuda.get_device_properties(local), "pci_bus_id", None) or str(local)
-    sampler = ClockSampler(gpu_id)
+    sampler = ClockSampler(nvidia_smi_id(torch, local))
     sampler.start()
     time.sleep(0.5)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]

@@ -63,6 +63,7 @@ struct albert_handle {
     // TMA descriptors (bf16)
     CUtensorMap tm_E, tm_X, tm_C, tm_X1, tm_H;
     CUtensorMap tm_win, tm_wqkv, tm_wo, tm_w1, tm_w2, tm_wout;
+    CUtensorMap t32_X, t32_QKV, t32_X1, t32_H;  // 32x32-box maps: epilogue stores / residual loads
 
     // per-kernel timing
     unsigned prof_mask = 0;  // classes whose launches are timed
@@ -177,10 +178,11 @@ GemmArgs gemm_args(albert_handle *h, int N, int K, const float *bias, void *out,
     return a;
 }
 
-int gemm_bf16(Launch &L, int cls, int epi, const CUtensorMap &A, const CUtensorMap &B, const GemmArgs &a) {
+int gemm_bf16(Launch &L, int cls, int epi, const CUtensorMap &A, const CUtensorMap &B, const CUtensorMap &Out,
+              const CUtensorMap &Res, const GemmArgs &a) {
     const int grid = gemm_grid(epi, a.rows_cap, a.N, L.h->num_sms);
     if (epi == kEpiLN && grid > L.h->grid_ln) return ALBERT_ERR_CONFIG;
-    LAUNCH(L, cls, launch_gemm(epi, A, B, a, grid, L.s));
+    LAUNCH(L, cls, launch_gemm(epi, A, B, Out, Res, a, grid, L.s));
     return ALBERT_OK;
 }
 
@@ -232,9 +234,9 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
     const int D = out_width(h);
     if (bf) {
         int rc;
-        if ((rc = gemm_bf16(L, kProfGemmIn, kEpiBias, h->tm_E, h->tm_win, gemm_args(h, kHidden, kEmb, h->b_in, h->X, kHidden)))) return rc;
+        if ((rc = gemm_bf16(L, kProfGemmIn, kEpiBias, h->tm_E, h->tm_win, h->t32_X, h->t32_X, gemm_args(h, kHidden, kEmb, h->b_in, h->X, kHidden)))) return rc;
         for (int l = 0; l < c.n_exec; ++l) {
-            if ((rc = gemm_bf16(L, kProfGemmQKV, kEpiBias, h->tm_X, h->tm_wqkv, gemm_args(h, kQKV, kHidden, h->bqkv, h->QKV, kQKV)))) return rc;
+            if ((rc = gemm_bf16(L, kProfGemmQKV, kEpiBias, h->tm_X, h->tm_wqkv, h->t32_QKV, h->t32_QKV, gemm_args(h, kQKV, kHidden, h->bqkv, h->QKV, kQKV)))) return rc;
             LAUNCH(L, kProfAttention, launch_attention_bf16(static_cast<bf16 *>(h->QKV), static_cast<bf16 *>(h->C), h->seq_start,
                                                            h->seq_len, nseq, max_len, h->status, L.s));
             GemmArgs a = gemm_args(h, kHidden, kHidden, h->bo, h->X1, kHidden);
@@ -242,17 +244,17 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
             a.ld_resid = kHidden;
             a.ln_g = h->ln1_g;
             a.ln_b = h->ln1_b;
-            if ((rc = gemm_bf16(L, kProfGemmWoLN, kEpiLN, h->tm_C, h->tm_wo, a))) return rc;
-            if ((rc = gemm_bf16(L, kProfGemmW1Gelu, kEpiGelu, h->tm_X1, h->tm_w1, gemm_args(h, kFfn, kHidden, h->b1, h->H, kFfn)))) return rc;
+            if ((rc = gemm_bf16(L, kProfGemmWoLN, kEpiLN, h->tm_C, h->tm_wo, h->t32_X1, h->t32_X, a))) return rc;
+            if ((rc = gemm_bf16(L, kProfGemmW1Gelu, kEpiGelu, h->tm_X1, h->tm_w1, h->t32_H, h->t32_H, gemm_args(h, kFfn, kHidden, h->b1, h->H, kFfn)))) return rc;
             a = gemm_args(h, kHidden, kFfn, h->b2, h->X, kHidden);
             a.resid = static_cast<bf16 *>(h->X1);
             a.ld_resid = kHidden;
             a.ln_g = h->ln2_g;
             a.ln_b = h->ln2_b;
-            if ((rc = gemm_bf16(L, kProfGemmW2LN, kEpiLN, h->tm_H, h->tm_w2, a))) return rc;
+            if ((rc = gemm_bf16(L, kProfGemmW2LN, kEpiLN, h->tm_H, h->tm_w2, h->t32_X, h->t32_X1, a))) return rc;
         }
         if (c.out_dim > 0) {
-            if ((rc = gemm_bf16(L, kProfGemmOut, kEpiScatter, h->tm_X, h->tm_wout, gemm_args(h, c.out_dim, kHidden, h->b_out, out, c.out_dim)))) return rc;
+            if ((rc = gemm_bf16(L, kProfGemmOut, kEpiScatter, h->tm_X, h->tm_wout, h->t32_X, h->t32_X, gemm_args(h, c.out_dim, kHidden, h->b_out, out, c.out_dim)))) return rc;
         } else {
             LAUNCH(L, kProfOutput, launch_scatter_rows(h->X, out, kHidden, 2, h->rows_cap, h->n_rows, h->row_dst, h->status, L.s));
         }
@@ -403,7 +405,9 @@ int create_impl(albert_handle *h, const albert_weights *w) {
             make_tmap_bf16(&h->tm_wo, h->wo, kHidden, kHidden, gemm::BN) ||
             make_tmap_bf16(&h->tm_w1, h->w1, kFfn, kHidden, gemm::BN) ||
             make_tmap_bf16(&h->tm_w2, h->w2, kHidden, kFfn, gemm::BN) ||
-            (O && make_tmap_bf16(&h->tm_wout, h->w_out, O, kHidden, gemm::BN)))
+            (O && make_tmap_bf16(&h->tm_wout, h->w_out, O, kHidden, gemm::BN)) ||
+            make_tmap_bf16_tile32(&h->t32_X, h->X, R, kHidden) || make_tmap_bf16_tile32(&h->t32_QKV, h->QKV, R, kQKV) ||
+            make_tmap_bf16_tile32(&h->t32_X1, h->X1, R, kHidden) || make_tmap_bf16_tile32(&h->t32_H, h->H, R, kFfn))
             return ALBERT_ERR_CUDA;
     }
     TRY(cudaStreamSynchronize(s));
@@ -546,8 +550,15 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
     TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
     const int rows_cap = (M + gemm::BM - 1) / gemm::BM * gemm::BM;
     const int grid = gemm_grid(epi, rows_cap, N, sms);
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, to, tr;
     if (make_tmap_bf16(&ta, A, M, K, gemm::BM) || make_tmap_bf16(&tb, W, N, K, gemm::BN)) return ALBERT_ERR_CUDA;
+    if (epi != kEpiScatter && make_tmap_bf16_tile32(&to, Y, M, N)) return ALBERT_ERR_CUDA;
+    if (epi == kEpiScatter) to = ta;
+    if (epi == kEpiLN) {
+        if (make_tmap_bf16_tile32(&tr, R, M, N)) return ALBERT_ERR_CUDA;
+    } else {
+        tr = to;
+    }
     int *ints = nullptr;
     float *scratch = nullptr;
     TRY(cudaMalloc(&ints, 2 * sizeof(int)));
@@ -561,7 +572,7 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
     a.N = N; a.K = K; a.rows_cap = rows_cap; a.n_rows = ints; a.bias = bias;
     a.resid = static_cast<const bf16 *>(R); a.ld_resid = N; a.ln_g = ln_g; a.ln_b = ln_b; a.eps = eps;
     a.out = static_cast<bf16 *>(Y); a.ld_out = N; a.scratch = scratch; a.row_dst = row_dst; a.status = ints + 1;
-    if (e == cudaSuccess) e = launch_gemm(epi, ta, tb, a, grid, s);
+    if (e == cudaSuccess) e = launch_gemm(epi, ta, tb, to, tr, a, grid, s);
     int st = 0;
     if (e == cudaSuccess) e = cudaMemcpyAsync(&st, ints + 1, sizeof(int), cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);

@@ -15,13 +15,17 @@
 //                 of one tile overlaps the main loop of the next;
 //   warps 2..9  : epilogue, 2 warps per TMEM lane quadrant (column halves);
 //                 tcgen05.ld -> bias (+ tanh-GELU | + residual, LayerNorm) ->
-//                 bf16 stores.
+//                 bf16 32x32 tile in a swizzled shared staging buffer -> TMA
+//                 bulk tensor store (coalesced, asynchronous; one-row-per-lane
+//                 global stores would contend with the tensor core's
+//                 shared-memory operand reads in the unified L1/shared array).
 // LayerNorm epilogue (post-LN steps 5 and 6): a work unit is a full 128x768
 // row block (3 sub-tiles of 256 columns).  Each thread owns one row half;
 // it keeps exact running (mean, M2) statistics per 32-column chunk (Chan's
 // merge), parks the fp32 pre-norm row in a per-CTA scratch slot that stays
 // L2-resident, exchanges statistics with the partner warp through shared
-// memory, then normalizes from the scratch slot.
+// memory, then normalizes from the scratch slot.  Its residual tiles arrive
+// by TMA into the same staging buffer, prefetched one 32-column chunk ahead.
 // Every wait is bounded (%globaltimer); on expiry the CTA records
 // ALBERT_ERR_TIMEOUT, drains its in-flight copies and MMAs, frees TMEM and exits.
 #include "kernels.h"
@@ -33,8 +37,8 @@ namespace {
 using namespace gemm;
 
 struct Smem {
-    uint8_t *a, *b;
-    uint64_t *full, *empty, *tfull, *tempty, *drain;
+    uint8_t *a, *b, *stg;    // stg: one 2 KB 32x32 bf16 staging tile per epilogue warp
+    uint64_t *full, *empty, *tfull, *tempty, *drain, *rbar;
     uint32_t *tmem_slot;
     volatile int *abort_flag;
     int *misc;               // [0] n_rows, [1] status at entry
@@ -47,14 +51,16 @@ __device__ __forceinline__ Smem carve(uint8_t *raw) {
     uint8_t *p = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
     s.a = p;
     s.b = p + STAGES * A_BYTES;
-    uint8_t *ctrl = s.b + STAGES * B_BYTES;
+    s.stg = s.b + STAGES * B_BYTES;
+    uint8_t *ctrl = s.stg + EPI_WARPS * STG_BYTES;
     uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl);
     s.full = bars;
     s.empty = bars + STAGES;
     s.tfull = bars + 2 * STAGES;
     s.tempty = bars + 2 * STAGES + 2;
     s.drain = bars + 2 * STAGES + 4;
-    uint32_t *u = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
+    s.rbar = bars + 2 * STAGES + 5;
+    uint32_t *u = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5 + EPI_WARPS);
     s.tmem_slot = u;
     s.abort_flag = reinterpret_cast<volatile int *>(u + 1);
     s.misc = reinterpret_cast<int *>(u + 2);
@@ -95,9 +101,50 @@ __device__ __forceinline__ void store_bf16x32(bf16 *dst, const float (&v)[32]) {
     }
 }
 
+// Byte offset of 16-byte chunk q of row r in a 32x32 bf16 tile (64-byte rows)
+// stored with the TMA 64-byte swizzle: chunk index XOR ((r >> 1) & 3).  A warp
+// writing one chunk per lane (lane = row) hits 32 distinct banks per 8 lanes.
+__device__ __forceinline__ uint32_t stg_off(int r, int q) {
+    return (uint32_t)(r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t a, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a) : "memory");
+    return v;
+}
+
+// Write this lane's 32 values (its row of the warp's 32x32 tile) as bf16 into
+// the staging tile, then one lane stores the tile to global memory by TMA.
+// The previous store from the same tile must have finished reading it.
+__device__ __forceinline__ void stage_and_store(uint32_t stg, const float (&v)[32], const CUtensorMap *tm,
+                                                int x, int y, int lane) {
+    if (lane == 0) bulk_wait_read0();
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 w;
+        w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+        w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+        w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+        w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+        st_shared_v4(stg + stg_off(lane, q), w);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(tm, stg, x, y);
+        bulk_commit();
+    }
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmRes,
                  const GemmArgs p) {
     extern __shared__ uint8_t smem_raw[];
     Smem sm = carve(smem_raw);
@@ -117,11 +164,14 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             mbar_init(smem_u32(&sm.tempty[i]), EPI_WARPS);
         }
         mbar_init(smem_u32(sm.drain), 1);
+        for (int i = 0; i < EPI_WARPS; ++i) mbar_init(smem_u32(&sm.rbar[i]), 1);
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
+        if (EPI != kEpiScatter) prefetch_tmap(&tmOut);
+        if (EPI == kEpiLN) prefetch_tmap(&tmRes);
     }
     __syncthreads();
     // An earlier kernel of this forward failed, or the row count is out of range.
@@ -224,13 +274,28 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int quad = warp & 3;          // TMEM lanes 32*quad .. 32*quad+31
         const int half = ew >> 2;           // column half of a 256-wide sub-tile
         const int r_local = quad * 32 + lane;
+        const uint32_t stg = smem_u32(sm.stg + ew * STG_BYTES);
+        const uint32_t rbar = smem_u32(&sm.rbar[ew]);
+        uint32_t rph = 0;
+        bool res_pending = false;
+        // residual chunk c (0..4*subs-1) of unit u -> TMA load into the staging tile
+        auto res_issue = [&](int u, int c) {
+            if (lane == 0) {
+                bulk_wait_read0();  // an earlier output store may still read the tile
+                mbar_arrive_expect_tx(rbar, STG_BYTES);
+                tma_load_2d(stg, &tmRes, rbar, (c >> 2) * BN + half * 128 + (c & 3) * 32, u * BM + quad * 32);
+            }
+            res_pending = true;
+        };
         int acc = 0, it = 0;
         bool ok = true;
+        if (EPI == kEpiLN && (int)blockIdx.x < units) res_issue(blockIdx.x, 0);
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++it) {
             const int m = (EPI == kEpiLN) ? u : u / n_sub;
             const int n0 = (EPI == kEpiLN) ? 0 : u % n_sub;
             const int row = m * BM + r_local;
             const bool row_ok = row < n_rows;
+            const int tile_row = m * BM + quad * 32;
             float mean = 0.f, m2 = 0.f, cnt = 0.f;
             float *slot = (EPI == kEpiLN) ? p.scratch + (size_t)blockIdx.x * BM * p.N : nullptr;
             int dst = row;
@@ -249,6 +314,16 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 for (int c = 0; c < 4; ++c) {
                     uint32_t r[32];
                     tmem_ld32(tbase + c * 32, r);
+                    uint4 rr[4];
+                    if (EPI == kEpiLN) {
+                        bool rok = mbar_wait(rbar, rph, sm.abort_flag);
+                        rok = __all_sync(0xffffffffu, rok);
+                        if (!rok) { ok = false; tmem_ld_wait(); break; }
+                        rph ^= 1;
+                        res_pending = false;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) rr[q] = ld_shared_v4(stg + stg_off(lane, q));
+                    }
                     tmem_ld_wait();
                     if (c == 3) {
                         tc_fence_before();
@@ -267,27 +342,26 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         v[4 * q + 3] = __uint_as_float(r[4 * q + 3]) + bb.w;
                     }
                     if (EPI == kEpiBias) {
-                        if (row_ok) store_bf16x32(p.out + (size_t)row * p.ld_out + col0, v);
+                        stage_and_store(stg, v, &tmOut, col0, tile_row, lane);
                     } else if (EPI == kEpiGelu) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[j] = gelu_tanh_fast(v[j]);
-                        if (row_ok) store_bf16x32(p.out + (size_t)row * p.ld_out + col0, v);
+                        stage_and_store(stg, v, &tmOut, col0, tile_row, lane);
                     } else if (EPI == kEpiScatter) {
                         if (dst >= 0) store_bf16x32(p.out + (size_t)dst * p.ld_out + col0, v);
                     } else {
-                        // residual
-                        if (row_ok) {
-                            const uint4 *rr = reinterpret_cast<const uint4 *>(p.resid + (size_t)row * p.ld_resid + col0);
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const uint4 w = __ldg(rr + q);
-                                float2 f;
-                                f = unpack_bf16x2(w.x); v[8 * q + 0] += f.x; v[8 * q + 1] += f.y;
-                                f = unpack_bf16x2(w.y); v[8 * q + 2] += f.x; v[8 * q + 3] += f.y;
-                                f = unpack_bf16x2(w.z); v[8 * q + 4] += f.x; v[8 * q + 5] += f.y;
-                                f = unpack_bf16x2(w.w); v[8 * q + 6] += f.x; v[8 * q + 7] += f.y;
-                            }
+                        for (int q = 0; q < 4; ++q) {
+                            float2 f;
+                            f = unpack_bf16x2(rr[q].x); v[8 * q + 0] += f.x; v[8 * q + 1] += f.y;
+                            f = unpack_bf16x2(rr[q].y); v[8 * q + 2] += f.x; v[8 * q + 3] += f.y;
+                            f = unpack_bf16x2(rr[q].z); v[8 * q + 4] += f.x; v[8 * q + 5] += f.y;
+                            f = unpack_bf16x2(rr[q].w); v[8 * q + 6] += f.x; v[8 * q + 7] += f.y;
                         }
+                        // the staging tile has been read: prefetch the next residual chunk
+                        __syncwarp();
+                        const int cn = s * 4 + c + 1;
+                        if (cn < 4 * subs) res_issue(u, cn);
                         // exact chunk statistics, merged into the running ones
                         float cs = 0.f;
 #pragma unroll
@@ -305,13 +379,15 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         }
                         cnt += 32.f;
                         // park the pre-norm values: layout [col/4][BM][4] (coalesced per warp)
+                        const int lcol0 = s * BN + half * 128 + c * 32;
                         float4 *sl = reinterpret_cast<float4 *>(slot);
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
-                            sl[(size_t)(col0 / 4 + q) * BM + r_local] =
+                            sl[(size_t)(lcol0 / 4 + q) * BM + r_local] =
                                 make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
                     }
                 }
+                if (!ok) break;
                 ++acc;
             }
             if (!ok) break;
@@ -333,31 +409,35 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const float mu = mean + 0.5f * d;
                 const float var = (m2 + o.y + d * d * (nh * 0.5f)) / (2.f * nh);
                 const float rstd = rsqrtf(var + p.eps);
-                if (row_ok) {
-                    const float4 *sl = reinterpret_cast<const float4 *>(slot);
+                const float4 *sl = reinterpret_cast<const float4 *>(slot);
 #pragma unroll 1
-                    for (int s = 0; s < subs; ++s) {
+                for (int s = 0; s < subs; ++s) {
 #pragma unroll 1
-                        for (int c = 0; c < 4; ++c) {
-                            const int col0 = s * BN + half * 128 + c * 32;
-                            float v[32];
-                            const float4 *g4 = reinterpret_cast<const float4 *>(p.ln_g + col0);
-                            const float4 *b4 = reinterpret_cast<const float4 *>(p.ln_b + col0);
+                    for (int c = 0; c < 4; ++c) {
+                        const int col0 = s * BN + half * 128 + c * 32;
+                        float v[32];
+                        const float4 *g4 = reinterpret_cast<const float4 *>(p.ln_g + col0);
+                        const float4 *b4 = reinterpret_cast<const float4 *>(p.ln_b + col0);
 #pragma unroll
-                            for (int q = 0; q < 8; ++q) {
-                                const float4 z = sl[(size_t)(col0 / 4 + q) * BM + r_local];
-                                const float4 g = __ldg(g4 + q), bb = __ldg(b4 + q);
-                                v[4 * q + 0] = fmaf((z.x - mu) * rstd, g.x, bb.x);
-                                v[4 * q + 1] = fmaf((z.y - mu) * rstd, g.y, bb.y);
-                                v[4 * q + 2] = fmaf((z.z - mu) * rstd, g.z, bb.z);
-                                v[4 * q + 3] = fmaf((z.w - mu) * rstd, g.w, bb.w);
-                            }
-                            store_bf16x32(p.out + (size_t)row * p.ld_out + col0, v);
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 z = sl[(size_t)(col0 / 4 + q) * BM + r_local];
+                            const float4 g = __ldg(g4 + q), bb = __ldg(b4 + q);
+                            v[4 * q + 0] = fmaf((z.x - mu) * rstd, g.x, bb.x);
+                            v[4 * q + 1] = fmaf((z.y - mu) * rstd, g.y, bb.y);
+                            v[4 * q + 2] = fmaf((z.z - mu) * rstd, g.z, bb.z);
+                            v[4 * q + 3] = fmaf((z.w - mu) * rstd, g.w, bb.w);
                         }
+                        stage_and_store(stg, v, &tmOut, col0, tile_row, lane);
                     }
                 }
+                // first residual chunk of this CTA's next unit
+                if (u + (int)gridDim.x < units) res_issue(u + gridDim.x, 0);
             }
         }
+        // outstanding copies finish before the CTA's shared memory goes away
+        if (lane == 0) bulk_wait0();
+        if (res_pending && lane == 0) mbar_wait_drain(rbar, rph);
+        __syncwarp();
     }
 
     __syncthreads();
@@ -377,8 +457,8 @@ int gemm_grid(int epi, int rows_cap, int N, int num_sms) {
 }
 
 template <int EPI>
-static cudaError_t launch_one(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmArgs &a,
-                              int grid, cudaStream_t s) {
+static cudaError_t launch_one(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
+                              const CUtensorMap &tmRes, const GemmArgs &a, int grid, cudaStream_t s) {
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(gemm_bf16_kernel<EPI>,
@@ -386,17 +466,17 @@ static cudaError_t launch_one(const CUtensorMap &tmA, const CUtensorMap &tmB, co
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    gemm_bf16_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmB, a);
+    gemm_bf16_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmB, tmOut, tmRes, a);
     return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                        const GemmArgs &a, int grid, cudaStream_t s) {
+cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
+                        const CUtensorMap &tmRes, const GemmArgs &a, int grid, cudaStream_t s) {
     switch (epi) {
-        case kEpiBias: return launch_one<kEpiBias>(tmA, tmB, a, grid, s);
-        case kEpiGelu: return launch_one<kEpiGelu>(tmA, tmB, a, grid, s);
-        case kEpiLN: return launch_one<kEpiLN>(tmA, tmB, a, grid, s);
-        case kEpiScatter: return launch_one<kEpiScatter>(tmA, tmB, a, grid, s);
+        case kEpiBias: return launch_one<kEpiBias>(tmA, tmB, tmOut, tmRes, a, grid, s);
+        case kEpiGelu: return launch_one<kEpiGelu>(tmA, tmB, tmOut, tmRes, a, grid, s);
+        case kEpiLN: return launch_one<kEpiLN>(tmA, tmB, tmOut, tmRes, a, grid, s);
+        case kEpiScatter: return launch_one<kEpiScatter>(tmA, tmB, tmOut, tmRes, a, grid, s);
     }
     return cudaErrorInvalidValue;
 }
@@ -419,18 +499,27 @@ static EncodeTiledFn encode_fn() {
     return fn;
 }
 
-int make_tmap_bf16(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+static int encode_bf16(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                       uint32_t box_rows, CUtensorMapSwizzle swz) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return -1;
     if ((reinterpret_cast<uintptr_t>(base) & 15) || (cols * 2) % 16) return -2;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t es[2] = {1, 1};
     CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
-                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? 0 : -3;
+}
+
+int make_tmap_bf16(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    return encode_bf16(tm, base, rows, cols, BK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+int make_tmap_bf16_tile32(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols) {
+    return encode_bf16(tm, base, rows, cols, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 }  // namespace albert

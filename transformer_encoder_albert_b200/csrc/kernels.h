@@ -25,7 +25,8 @@ constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 32 * (2 + EPI_WARPS);
 constexpr int TMEM_COLS = 512;
 constexpr int LN_N = 768;  // the LayerNorm epilogue normalizes rows of this width
-constexpr int SMEM_BYTES = 2048 + STAGES * (A_BYTES + B_BYTES) + 1024 + 2 * 2 * BM * 8;
+constexpr int STG_BYTES = 32 * 32 * 2;  // one 32x32 bf16 epilogue staging tile per epilogue warp
+constexpr int SMEM_BYTES = 2048 + STAGES * (A_BYTES + B_BYTES) + EPI_WARPS * STG_BYTES + 1024 + 2 * 2 * BM * 8;
 }  // namespace gemm
 
 struct GemmArgs {
@@ -48,14 +49,19 @@ struct GemmArgs {
 // box and the 128-byte swizzle.  Returns 0 on success.
 int make_tmap_bf16(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols,
                    uint32_t box_rows);
+// Map of a bf16 row-major [rows, cols] tensor with a 32x32 box and the 64-byte
+// swizzle: the epilogue's output stores and residual loads.
+int make_tmap_bf16_tile32(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols);
 
 // Grid the GEMM uses for this many rows (persistent: <= number of SMs).
 int gemm_grid(int epi, int rows_cap, int N, int num_sms);
 // Scratch floats the LN epilogue needs for a grid of this size.
 inline size_t gemm_ln_scratch_floats(int grid) { return (size_t)grid * gemm::BM * gemm::LN_N; }
 
-cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                        const GemmArgs &args, int grid, cudaStream_t s);
+// tmOut: tile32 map of the output (unused by the scatter epilogue); tmRes: tile32
+// map of the residual (LayerNorm epilogue only; pass any valid map otherwise).
+cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
+                        const CUtensorMap &tmRes, const GemmArgs &args, int grid, cudaStream_t s);
 
 // ---------------------------------------------------------------- attention --
 // Masked bidirectional attention, bf16 tensor-core kernel (mma.sync m16n8k16).

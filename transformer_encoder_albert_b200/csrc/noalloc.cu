@@ -77,8 +77,10 @@ extern "C" int albert_gemm_residual_ln_noalloc(const void *A, const void *W, con
     const int N = gemm::LN_N;
     const int rows_cap = (M + gemm::BM - 1) / gemm::BM * gemm::BM;
     const int grid = rows_cap / gemm::BM;  // one CTA per row block: <= kNoAllocSlots scratch slots
-    CUtensorMap ta, tb;
-    if (make_tmap_bf16(&ta, A, M, K, gemm::BM) || make_tmap_bf16(&tb, W, N, K, gemm::BN)) return ALBERT_ERR_CUDA;
+    CUtensorMap ta, tb, to, tr;
+    if (make_tmap_bf16(&ta, A, M, K, gemm::BM) || make_tmap_bf16(&tb, W, N, K, gemm::BN) ||
+        make_tmap_bf16_tile32(&to, Y, M, N) || make_tmap_bf16_tile32(&tr, R, M, N))
+        return ALBERT_ERR_CUDA;
 
     reset_words_kernel<<<1, 1, 0, s>>>(words, M);
     if (cudaGetLastError() != cudaSuccess) return ALBERT_ERR_CUDA;
@@ -97,7 +99,7 @@ extern "C" int albert_gemm_residual_ln_noalloc(const void *A, const void *W, con
     a.ld_out = N;
     a.scratch = scratch;
     a.status = words + 1;
-    if (launch_gemm(kEpiLN, ta, tb, a, grid, s) != cudaSuccess) return ALBERT_ERR_CUDA;
+    if (launch_gemm(kEpiLN, ta, tb, to, tr, a, grid, s) != cudaSuccess) return ALBERT_ERR_CUDA;
     int st = 0;
     if (cudaMemcpyAsync(&st, words + 1, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return ALBERT_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return ALBERT_ERR_CUDA;
