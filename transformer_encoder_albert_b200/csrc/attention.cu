@@ -9,21 +9,21 @@
 // [rows, 3*768] buffer (Q | K | V); head h is the 64-column slice 64h..64h+63
 // of each; the context goes to [rows, 768] with the same head layout.
 //
-// bf16 kernel: one CTA per (sequence, head, 128-query tile), 8 warps x 16
-// query rows.  The head's whole K and V (L_b <= 512 rows of 64 bf16) are
-// staged once in shared memory; each warp runs an online (max-subtracted)
-// softmax over 64-key blocks with mma.sync m16n8k16 (bf16 in, fp32 accumulate),
-// keeping P in registers between the two products.
+// bf16 kernel: one CTA per (sequence, head, query tile of 16 rows per warp;
+// 4 warps for T <= 128, 8 warps above).  The head's whole K and V (L_b <= 512
+// rows of 64 bf16) are staged in shared memory by cp.async, one commit group
+// per 64-key block, so the first block's math overlaps the later blocks'
+// loads; each warp runs an online (max-subtracted) softmax over the 64-key
+// blocks with mma.sync m16n8k16 (bf16 in, fp32 accumulate), keeping P in
+// registers between the two products.
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
 namespace albert {
 namespace {
 
-constexpr int QT = 128;      // query rows per CTA
 constexpr int KBLK = 64;     // keys per online-softmax block
 constexpr int LDS = 72;      // shared row stride in bf16 (144 B): conflict-free ldmatrix
-constexpr int ATT_THREADS = 256;
 
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const bf16 *p) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -41,62 +41,83 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// 16-byte global -> shared copy; src_bytes = 0 writes zeros and reads nothing.
+__device__ __forceinline__ void cp_async16(bf16 *dst, const bf16 *src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most n of this thread's cp.async groups are still pending (n <= 7).
+__device__ __forceinline__ void cp_async_wait_pending(int n) {
+    switch (n) {
+        case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+        case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+        case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+        case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+        case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+        case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+        case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
+        default: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
+    }
+}
 
-__global__ void __launch_bounds__(ATT_THREADS)
+template <int NW>
+__global__ void __launch_bounds__(NW * 32)
 attn_bf16_kernel(const bf16 *__restrict__ qkv, bf16 *__restrict__ ctx, const int *__restrict__ seq_start,
                  const int *__restrict__ seq_len, const int *__restrict__ status) {
+    constexpr int QT = 16 * NW, NT = 32 * NW;
     if (*reinterpret_cast<const volatile int *>(status) != 0) return;
     const int b = blockIdx.z, h = blockIdx.y, q0 = blockIdx.x * QT;
     const int L = seq_len[b];
     if (q0 >= L) return;
     const int start = seq_start[b];
-    const int Lpad = (L + KBLK - 1) / KBLK * KBLK;
+    const int nkb = (L + KBLK - 1) / KBLK;
 
     extern __shared__ uint4 smem4[];
     bf16 *sQ = reinterpret_cast<bf16 *>(smem4);
     bf16 *sK = sQ + QT * LDS;
-    bf16 *sV = sK + Lpad * LDS;
+    bf16 *sV = sK + nkb * KBLK * LDS;
+    const bf16 *base = qkv + (size_t)start * kQKV + h * kHeadDim;
 
-    const uint4 zero = make_uint4(0, 0, 0, 0);
-    for (int i = threadIdx.x; i < Lpad * 8; i += ATT_THREADS) {
-        const int u = i >> 3, c = i & 7;
-        uint4 kv = zero, vv = zero;
-        if (u < L) {
-            const bf16 *row = qkv + (size_t)(start + u) * kQKV + h * kHeadDim + c * 8;
-            kv = __ldg(reinterpret_cast<const uint4 *>(row + kHidden));
-            vv = __ldg(reinterpret_cast<const uint4 *>(row + 2 * kHidden));
+    // group 0: the query tile and key/value block 0; group j: key/value block j
+    for (int j = 0; j < nkb; ++j) {
+        if (j == 0) {
+            for (int i = threadIdx.x; i < QT * 8; i += NT) {
+                const int t = i >> 3, c = i & 7, row = q0 + t;
+                cp_async16(sQ + t * LDS + c * 8, base + (size_t)min(row, L - 1) * kQKV + c * 8, row < L ? 16 : 0);
+            }
         }
-        *reinterpret_cast<uint4 *>(sK + u * LDS + c * 8) = kv;
-        *reinterpret_cast<uint4 *>(sV + u * LDS + c * 8) = vv;
+        for (int i = threadIdx.x; i < 2 * KBLK * 8; i += NT) {
+            const int which = i >> 9, r = (i >> 3) & (KBLK - 1), c = i & 7, u = j * KBLK + r;
+            const bf16 *src = base + (size_t)min(u, L - 1) * kQKV + (1 + which) * kHidden + c * 8;
+            cp_async16((which ? sV : sK) + u * LDS + c * 8, src, u < L ? 16 : 0);
+        }
+        cp_async_commit();
     }
-    for (int i = threadIdx.x; i < QT * 8; i += ATT_THREADS) {
-        const int t = i >> 3, c = i & 7;
-        uint4 qv = zero;
-        if (q0 + t < L)
-            qv = __ldg(reinterpret_cast<const uint4 *>(qkv + (size_t)(start + q0 + t) * kQKV + h * kHeadDim + c * 8));
-        *reinterpret_cast<uint4 *>(sQ + t * LDS + c * 8) = qv;
-    }
-    __syncthreads();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qw = q0 + warp * 16;
-    if (qw >= L) return;
+    const bool active = qw < L;
     const int g = lane >> 2, tig = lane & 3;
-
-    uint32_t qf[4][4];
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks)
-        ldsm_x4(qf[ks], sQ + (warp * 16 + (lane & 15)) * LDS + ks * 16 + (lane >> 4) * 8);
-
+    const int j8 = lane >> 3, r8 = lane & 7;
     // scores are kept in log2 units: s * (1/8) * log2(e)
     const float sl2 = 0.125f * 1.4426950408889634f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     float o[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    uint32_t qf[4][4];
 
-    const int j8 = lane >> 3, r8 = lane & 7;
-    for (int kb = 0; kb < Lpad; kb += KBLK) {
+    for (int j = 0; j < nkb; ++j) {
+        cp_async_wait_pending(nkb - 1 - j);
+        __syncthreads();
+        if (!active) continue;
+        if (j == 0) {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                ldsm_x4(qf[ks], sQ + (warp * 16 + (lane & 15)) * LDS + ks * 16 + (lane >> 4) * 8);
+        }
+        const int kb = j * KBLK;
         float s[8][4];
 #pragma unroll
         for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
@@ -147,21 +168,22 @@ attn_bf16_kernel(const bf16 *__restrict__ qkv, bf16 *__restrict__ ctx, const int
             o[nd][2] *= a1; o[nd][3] *= a1;
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int jj = 0; jj < 4; ++jj) {
             uint32_t pa[4];
-            pa[0] = pack_bf16x2(s[2 * j][0], s[2 * j][1]);
-            pa[1] = pack_bf16x2(s[2 * j][2], s[2 * j][3]);
-            pa[2] = pack_bf16x2(s[2 * j + 1][0], s[2 * j + 1][1]);
-            pa[3] = pack_bf16x2(s[2 * j + 1][2], s[2 * j + 1][3]);
+            pa[0] = pack_bf16x2(s[2 * jj][0], s[2 * jj][1]);
+            pa[1] = pack_bf16x2(s[2 * jj][2], s[2 * jj][3]);
+            pa[2] = pack_bf16x2(s[2 * jj + 1][0], s[2 * jj + 1][1]);
+            pa[3] = pack_bf16x2(s[2 * jj + 1][2], s[2 * jj + 1][3]);
 #pragma unroll
             for (int dp = 0; dp < 4; ++dp) {
                 uint32_t vf[4];
-                ldsm_x4_t(vf, sV + (kb + j * 16 + (j8 & 1) * 8 + r8) * LDS + dp * 16 + (j8 >> 1) * 8);
+                ldsm_x4_t(vf, sV + (kb + jj * 16 + (j8 & 1) * 8 + r8) * LDS + dp * 16 + (j8 >> 1) * 8);
                 mma_bf16_16816(o[2 * dp], pa, vf[0], vf[1]);
                 mma_bf16_16816(o[2 * dp + 1], pa, vf[2], vf[3]);
             }
         }
     }
+    if (!active) return;
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
@@ -232,26 +254,33 @@ attn_f32_kernel(const float *__restrict__ qkv, float *__restrict__ ctx, const in
 
 }  // namespace
 
-static size_t attn_bf16_smem(int max_len) {
+static size_t attn_bf16_smem(int max_len, int qt) {
     const int lpad = (max_len + KBLK - 1) / KBLK * KBLK;
-    return (size_t)(QT + 2 * lpad) * LDS * sizeof(bf16);
+    return (size_t)(qt + 2 * lpad) * LDS * sizeof(bf16);
+}
+
+template <int NW>
+static cudaError_t launch_attn_nw(const bf16 *qkv, bf16 *ctx, const int *seq_start, const int *seq_len, int nseq,
+                                  int max_len, const int *status, cudaStream_t s) {
+    constexpr int QT = 16 * NW;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)attn_bf16_smem(kMaxPos, QT));
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    dim3 grid((max_len + QT - 1) / QT, kHeads, nseq);
+    attn_bf16_kernel<NW><<<grid, NW * 32, attn_bf16_smem(max_len, QT), s>>>(qkv, ctx, seq_start, seq_len, status);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_attention_bf16(const bf16 *qkv, bf16 *ctx, const int *seq_start,
                                   const int *seq_len, int nseq, int max_len, const int *status,
                                   cudaStream_t s) {
     if (nseq <= 0) return cudaSuccess;
-    const size_t smem = attn_bf16_smem(max_len);
-    static size_t configured = 0;
-    if (smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)attn_bf16_smem(kMaxPos));
-        if (e != cudaSuccess) return e;
-        configured = attn_bf16_smem(kMaxPos);
-    }
-    dim3 grid((max_len + QT - 1) / QT, kHeads, nseq);
-    attn_bf16_kernel<<<grid, ATT_THREADS, smem, s>>>(qkv, ctx, seq_start, seq_len, status);
-    return cudaGetLastError();
+    if (max_len <= 128) return launch_attn_nw<4>(qkv, ctx, seq_start, seq_len, nseq, max_len, status, s);
+    return launch_attn_nw<8>(qkv, ctx, seq_start, seq_len, nseq, max_len, status, s);
 }
 
 cudaError_t launch_attention_f32(const float *qkv, float *ctx, const int *seq_start,
