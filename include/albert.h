@@ -189,22 +189,24 @@ int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, 
  * thread that cannot absorb cudaMalloc's device-wide synchronization and
  * latency, or a runtime that lays out all device memory before its first
  * request.  It computes Y = LN(A W^T + bias + R; ln_g, ln_b, eps) exactly like
- * albert_test_gemm with epi = 2, but its scratch (fp32 row slots of the
- * LayerNorm epilogue, a row-count word and the status word) lives in a
- * file-scope __device__ array of 6 MiB inside the library instead of memory
- * the call allocates; it calls no cudaMalloc/cudaFree.
+ * albert_test_gemm with epi = 2, but its scratch (the per-row LayerNorm
+ * statistics and epoch flags its column tiles exchange, a row-count word and
+ * the status word) lives in file-scope __device__ arrays of about 195 KiB
+ * inside the library instead of memory the call allocates; it calls no
+ * cudaMalloc/cudaFree.
  *   A: [M, K] bf16, W: [768, K] bf16, bias/ln_g/ln_b: [768] fp32,
  *   R: [M, 768] bf16, Y: [M, 768] bf16, all device pointers the caller owns.
- *   Limits: 1 <= M <= 2048 (the array holds 16 row blocks of 128), K % 64 == 0;
+ *   Limits: 1 <= M <= 8192 (the size the arrays hold), K % 64 == 0;
  *   anything else returns ALBERT_ERR_SHAPE before any work is enqueued.
- * The array is reserved on every device where the library's module holding it
- * is loaded and stays until the process exits.  The first call on a device
- * looks up the array's device address (cudaGetSymbolAddress) with that device
+ * The arrays are reserved on every device where the library's module holding
+ * them is loaded and stay until the process exits.  The first call on a device
+ * looks up their device addresses (cudaGetSymbolAddress) with that device
  * current; make that first call before any stream capture.  Every call shares
- * the one array (its status word is reset by each call, the row slots are
- * fully rewritten before they are read), so calls that overlap on the GPU --
- * on different streams or from different threads -- race and must be
- * serialized by the caller.  Synchronous: returns the kernel's status. */
+ * the same arrays (the status word is reset by each call; statistics are
+ * rewritten before they are read and flags carry a per-call epoch, so nothing
+ * else needs clearing), so calls that overlap on the GPU -- on different
+ * streams or from different threads -- race and must be serialized by the
+ * caller.  Synchronous: returns the kernel's status. */
 int albert_gemm_residual_ln_noalloc(const void *A, const void *W, const float *bias, const void *R,
                                     const float *ln_g, const float *ln_b, float eps, void *Y, int M,
                                     int K, void *stream);

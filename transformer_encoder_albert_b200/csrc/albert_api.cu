@@ -51,9 +51,10 @@ struct albert_handle {
 
     // workspace
     void *E = nullptr, *X = nullptr, *QKV = nullptr, *C = nullptr, *X1 = nullptr, *H = nullptr, *Z = nullptr;
-    float *scratch = nullptr;
+    float2 *ln_stats = nullptr;  // per-row (mean, M2) of each 256-column tile
+    int *ln_flags = nullptr;     // epoch flags of the LayerNorm GEMM's cross-CTA exchange
+    int ln_epoch = 0;            // last epoch handed to a LayerNorm GEMM launch
     int *seq_start = nullptr, *seq_len = nullptr, *row_dst = nullptr, *n_rows = nullptr, *status = nullptr;
-    int grid_ln = 0;
 
     // host-buffer staging
     int64_t *st_ids = nullptr;
@@ -171,7 +172,8 @@ GemmArgs gemm_args(albert_handle *h, int N, int K, const float *bias, void *out,
     a.bias = bias;
     a.out = static_cast<bf16 *>(out);
     a.ld_out = ld_out;
-    a.scratch = h->scratch;
+    a.ln_stats = h->ln_stats;
+    a.ln_flags = h->ln_flags;
     a.row_dst = h->row_dst;
     a.status = h->status;
     a.eps = h->cfg.ln_eps;
@@ -179,9 +181,12 @@ GemmArgs gemm_args(albert_handle *h, int N, int K, const float *bias, void *out,
 }
 
 int gemm_bf16(Launch &L, int cls, int epi, const CUtensorMap &A, const CUtensorMap &B, const CUtensorMap &Out,
-              const CUtensorMap &Res, const GemmArgs &a) {
+              const CUtensorMap &Res, GemmArgs a) {
     const int grid = gemm_grid(epi, a.rows_cap, a.N, L.h->num_sms);
-    if (epi == kEpiLN && grid > L.h->grid_ln) return ALBERT_ERR_CONFIG;
+    if (epi == kEpiLN) {
+        if (a.N != gemm::LN_N) return ALBERT_ERR_CONFIG;
+        a.epoch = ++L.h->ln_epoch;
+    }
     LAUNCH(L, cls, launch_gemm(epi, A, B, Out, Res, a, grid, L.s));
     return ALBERT_OK;
 }
@@ -375,8 +380,9 @@ int create_impl(albert_handle *h, const albert_weights *w) {
     if ((rc = dev_alloc(h, &h->X1, R * kHidden * eb))) return rc;
     if ((rc = dev_alloc(h, &h->H, R * kFfn * eb))) return rc;
     if (bf) {
-        h->grid_ln = gemm_grid(kEpiLN, h->rows_cap, kHidden, h->num_sms);
-        if ((rc = dev_alloc(h, (void **)&h->scratch, gemm_ln_scratch_floats(h->grid_ln) * sizeof(float)))) return rc;
+        if ((rc = dev_alloc(h, (void **)&h->ln_stats, gemm_ln_stats_count(h->rows_cap) * sizeof(float2)))) return rc;
+        if ((rc = dev_alloc(h, (void **)&h->ln_flags, gemm_ln_flags_count(h->rows_cap) * sizeof(int)))) return rc;
+        TRY(cudaMemsetAsync(h->ln_flags, 0, gemm_ln_flags_count(h->rows_cap) * sizeof(int), s));
     } else {
         if ((rc = dev_alloc(h, &h->Z, R * kHidden * eb))) return rc;
     }
@@ -560,24 +566,30 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
         tr = to;
     }
     int *ints = nullptr;
-    float *scratch = nullptr;
+    float2 *stats = nullptr;
+    int *flags = nullptr;
     TRY(cudaMalloc(&ints, 2 * sizeof(int)));
-    if (epi == kEpiLN && cudaMalloc(&scratch, gemm_ln_scratch_floats(grid) * sizeof(float)) != cudaSuccess) {
+    if (epi == kEpiLN && (cudaMalloc(&stats, gemm_ln_stats_count(rows_cap) * sizeof(float2)) != cudaSuccess ||
+                          cudaMalloc(&flags, gemm_ln_flags_count(rows_cap) * sizeof(int)) != cudaSuccess)) {
         cudaFree(ints);
+        cudaFree(stats);
         return ALBERT_ERR_ALLOC;
     }
     const int host_ints[2] = {M, 0};
     cudaError_t e = cudaMemcpyAsync(ints, host_ints, sizeof(host_ints), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && flags) e = cudaMemsetAsync(flags, 0, gemm_ln_flags_count(rows_cap) * sizeof(int), s);
     GemmArgs a{};
     a.N = N; a.K = K; a.rows_cap = rows_cap; a.n_rows = ints; a.bias = bias;
     a.resid = static_cast<const bf16 *>(R); a.ld_resid = N; a.ln_g = ln_g; a.ln_b = ln_b; a.eps = eps;
-    a.out = static_cast<bf16 *>(Y); a.ld_out = N; a.scratch = scratch; a.row_dst = row_dst; a.status = ints + 1;
+    a.out = static_cast<bf16 *>(Y); a.ld_out = N; a.ln_stats = stats; a.ln_flags = flags; a.epoch = 1;
+    a.row_dst = row_dst; a.status = ints + 1;
     if (e == cudaSuccess) e = launch_gemm(epi, ta, tb, to, tr, a, grid, s);
     int st = 0;
     if (e == cudaSuccess) e = cudaMemcpyAsync(&st, ints + 1, sizeof(int), cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     cudaFree(ints);
-    if (scratch) cudaFree(scratch);
+    if (stats) cudaFree(stats);
+    if (flags) cudaFree(flags);
     return e == cudaSuccess ? st : ALBERT_ERR_CUDA;
 }
 

@@ -7,7 +7,7 @@
 // A linear layer is y_j = b_j + sum_i x_i W_{j,i} with W stored [out, in]
 // ("Qwen3-TTS and Kokoro", section A), i.e. both operands are K-major.
 //
-// Design (one CTA per SM, persistent over work units):
+// Design (one CTA per SM, persistent over 128x256 output tiles):
 //   warp 0      : TMA producer, 4-stage ring of {A 128x64, B 256x64} bf16 tiles
 //                 (128-byte swizzle, no multicast);
 //   warp 1      : TMEM allocator + single-thread tcgen05.mma issuer into two
@@ -19,13 +19,16 @@
 //                 bulk tensor store (coalesced, asynchronous; one-row-per-lane
 //                 global stores would contend with the tensor core's
 //                 shared-memory operand reads in the unified L1/shared array).
-// LayerNorm epilogue (post-LN steps 5 and 6): a work unit is a full 128x768
-// row block (3 sub-tiles of 256 columns).  Each thread owns one row half;
-// it keeps exact running (mean, M2) statistics per 32-column chunk (Chan's
-// merge), parks the fp32 pre-norm row in a per-CTA scratch slot that stays
-// L2-resident, exchanges statistics with the partner warp through shared
-// memory, then normalizes from the scratch slot.  Its residual tiles arrive
-// by TMA into the same staging buffer, prefetched one 32-column chunk ahead.
+// LayerNorm epilogue (post-LN steps 5 and 6, rows of 768 = 3 tiles of 256):
+// each tile's epilogue adds bias and residual (residual tiles arrive by TMA,
+// one 32-column chunk ahead), writes the fp32 pre-norm sum back into its TMEM
+// accumulator, and keeps exact per-row (mean, M2) statistics (Chan's merge of
+// 32-column chunks, then of the two column halves through shared memory).
+// The three tiles of a row block run on three CTAs at the same time: each
+// publishes its per-row statistics to a small global buffer with a release
+// flag tagged by the launch's epoch and acquires the other two, then
+// normalizes its 256 columns straight from TMEM.  The cross-CTA waits need
+// every CTA resident, so this variant is launched cooperatively.
 // Every wait is bounded (%globaltimer); on expiry the CTA records
 // ALBERT_ERR_TIMEOUT, drains its in-flight copies and MMAs, frees TMEM and exits.
 #include "kernels.h"
@@ -88,6 +91,26 @@ __device__ __forceinline__ bool wait_flag(volatile int *flag, int target, volati
     return ok;
 }
 
+// Wait (bounded, lane 0 polls) until another CTA has published `epoch` at *flag.
+__device__ __forceinline__ bool wait_epoch(const int *flag, int epoch, volatile int *abort_flag) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) {
+        if (ld_acquire_gpu(flag) != epoch) {
+            const unsigned long long t0 = globaltimer_ns();
+            while (ld_acquire_gpu(flag) != epoch) {
+                if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
+                    *abort_flag = 1;
+                    ok = false;
+                    break;
+                }
+            }
+        }
+    }
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    __syncwarp();
+    return ok;
+}
+
 __device__ __forceinline__ void store_bf16x32(bf16 *dst, const float (&v)[32]) {
     uint4 *d = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
@@ -141,6 +164,13 @@ __device__ __forceinline__ void stage_and_store(uint32_t stg, const float (&v)[3
     }
 }
 
+// Chan's merge: (mean, m2) over cnt values absorbs a group (cm, cq) of cn values.
+__device__ __forceinline__ void chan_merge(float &mean, float &m2, float cnt, float cm, float cq, float cn) {
+    const float nn = cnt + cn, d = cm - mean;
+    mean = fmaf(d, cn / nn, mean);
+    m2 += cq + d * d * (cnt * cn / nn);
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -189,39 +219,35 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const int n_rows = sm.misc[0];
     const int m_blocks = (n_rows + BM - 1) / BM;
     const int n_sub = p.N / BN;
-    const int units = (EPI == kEpiLN) ? m_blocks : m_blocks * n_sub;
-    const int subs = (EPI == kEpiLN) ? n_sub : 1;
+    const int units = m_blocks * n_sub;  // unit u = tile (u / n_sub, u % n_sub), row-block major
     const int kblocks = p.K / BK;
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer --
         if (lane == 0) {
             const uint64_t keep = policy_evict_last();  // weights: reused by every CTA
-            int stage = 0;
+            int stage = 0, issued = 0;
             uint32_t phase = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-                const int m = (EPI == kEpiLN) ? u : u / n_sub;
-                const int n0 = (EPI == kEpiLN) ? 0 : u % n_sub;
-                for (int s = 0; s < subs && ok; ++s) {
-                    for (int kb = 0; kb < kblocks; ++kb) {
-                        if (!mbar_wait(smem_u32(&sm.empty[stage]), phase ^ 1, sm.abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        const uint32_t fb = smem_u32(&sm.full[stage]);
-                        mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
-                        tma_load_2d(smem_u32(sm.a + stage * A_BYTES), &tmA, fb, kb * BK, m * BM);
-                        tma_load_2d_hint(smem_u32(sm.b + stage * B_BYTES), &tmB, fb, kb * BK,
-                                         (n0 + s) * BN, keep);
-                        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                const int m = u / n_sub, n = u % n_sub;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(smem_u32(&sm.empty[stage]), phase ^ 1, sm.abort_flag)) {
+                        ok = false;
+                        break;
                     }
+                    const uint32_t fb = smem_u32(&sm.full[stage]);
+                    mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
+                    tma_load_2d(smem_u32(sm.a + stage * A_BYTES), &tmA, fb, kb * BK, m * BM);
+                    tma_load_2d_hint(smem_u32(sm.b + stage * B_BYTES), &tmB, fb, kb * BK, n * BN, keep);
+                    ++issued;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
             }
             if (!ok) {
                 // Drain: every stage whose load may still be in flight completes
                 // its transaction count before the CTA's shared memory goes away.
-                for (int i = 0; i < STAGES; ++i) {
+                for (int i = 0; i < STAGES && i < issued; ++i) {
                     if (--stage < 0) { stage = STAGES - 1; phase ^= 1; }
                     mbar_wait_drain(smem_u32(&sm.full[stage]), phase);
                 }
@@ -235,34 +261,29 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             uint32_t phase = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-                for (int s = 0; s < subs && ok; ++s) {
-                    const int ab = acc & 1;
-                    const uint32_t aph = (acc >> 1) & 1;
-                    if (!mbar_wait(smem_u32(&sm.tempty[ab]), aph ^ 1, sm.abort_flag)) {
+                const int ab = acc & 1;
+                const uint32_t aph = (acc >> 1) & 1;
+                if (!mbar_wait(smem_u32(&sm.tempty[ab]), aph ^ 1, sm.abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + ab * BN;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(smem_u32(&sm.full[stage]), phase, sm.abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t d = tmem_base + ab * BN;
-                    for (int kb = 0; kb < kblocks; ++kb) {
-                        if (!mbar_wait(smem_u32(&sm.full[stage]), phase, sm.abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t a0 = smem_u32(sm.a + stage * A_BYTES);
-                        const uint32_t b0 = smem_u32(sm.b + stage * B_BYTES);
+                    const uint32_t a0 = smem_u32(sm.a + stage * A_BYTES);
+                    const uint32_t b0 = smem_u32(sm.b + stage * B_BYTES);
 #pragma unroll
-                        for (int k = 0; k < BK / 16; ++k)
-                            umma_bf16(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32),
-                                      idesc, (kb | k) != 0);
-                        umma_commit(smem_u32(&sm.empty[stage]));
-                        if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                    }
-                    if (!ok) break;
-                    umma_commit(smem_u32(&sm.tfull[ab]));
-                    ++acc;
+                    for (int k = 0; k < BK / 16; ++k)
+                        umma_bf16(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), idesc,
+                                  (kb | k) != 0);
+                    umma_commit(smem_u32(&sm.empty[stage]));
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
+                if (!ok) break;
+                umma_commit(smem_u32(&sm.tfull[ab]));
+                ++acc;
             }
             // All MMAs issued by this thread complete before TMEM is released.
             umma_commit(smem_u32(sm.drain));
@@ -272,18 +293,19 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         // ---------------------------------------------------------- epilogue --
         const int ew = warp - 2;            // 0..7
         const int quad = warp & 3;          // TMEM lanes 32*quad .. 32*quad+31
-        const int half = ew >> 2;           // column half of a 256-wide sub-tile
+        const int half = ew >> 2;           // column half of the 256-wide tile
         const int r_local = quad * 32 + lane;
         const uint32_t stg = smem_u32(sm.stg + ew * STG_BYTES);
         const uint32_t rbar = smem_u32(&sm.rbar[ew]);
         uint32_t rph = 0;
         bool res_pending = false;
-        // residual chunk c (0..4*subs-1) of unit u -> TMA load into the staging tile
+        // residual chunk c (0..3) of unit u -> TMA load into this warp's staging tile
         auto res_issue = [&](int u, int c) {
             if (lane == 0) {
                 bulk_wait_read0();  // an earlier output store may still read the tile
                 mbar_arrive_expect_tx(rbar, STG_BYTES);
-                tma_load_2d(stg, &tmRes, rbar, (c >> 2) * BN + half * 128 + (c & 3) * 32, u * BM + quad * 32);
+                tma_load_2d(stg, &tmRes, rbar, (u % n_sub) * BN + half * 128 + c * 32,
+                            (u / n_sub) * BM + quad * 32);
             }
             res_pending = true;
         };
@@ -291,109 +313,94 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         bool ok = true;
         if (EPI == kEpiLN && (int)blockIdx.x < units) res_issue(blockIdx.x, 0);
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++it) {
-            const int m = (EPI == kEpiLN) ? u : u / n_sub;
-            const int n0 = (EPI == kEpiLN) ? 0 : u % n_sub;
+            const int m = u / n_sub, n = u % n_sub;
             const int row = m * BM + r_local;
             const bool row_ok = row < n_rows;
             const int tile_row = m * BM + quad * 32;
-            float mean = 0.f, m2 = 0.f, cnt = 0.f;
-            float *slot = (EPI == kEpiLN) ? p.scratch + (size_t)blockIdx.x * BM * p.N : nullptr;
             int dst = row;
             if (EPI == kEpiScatter) dst = row_ok ? __ldg(p.row_dst + row) : -1;
 
-            for (int s = 0; s < subs; ++s) {
-                const int ab = acc & 1;
-                const uint32_t aph = (acc >> 1) & 1;
-                bool got = mbar_wait(smem_u32(&sm.tfull[ab]), aph, sm.abort_flag);
-                got = __all_sync(0xffffffffu, got);
-                if (!got) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + ab * BN + half * 128;
-                const int ncol0 = (n0 + s) * BN + half * 128;  // first output column
+            const int ab = acc & 1;
+            const uint32_t aph = (acc >> 1) & 1;
+            bool got = mbar_wait(smem_u32(&sm.tfull[ab]), aph, sm.abort_flag);
+            got = __all_sync(0xffffffffu, got);
+            if (!got) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + ab * BN + half * 128;
+            const int ncol0 = n * BN + half * 128;  // first output column of this warp
+            float mean = 0.f, m2 = 0.f;
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tbase + c * 32, r);
-                    uint4 rr[4];
-                    if (EPI == kEpiLN) {
-                        bool rok = mbar_wait(rbar, rph, sm.abort_flag);
-                        rok = __all_sync(0xffffffffu, rok);
-                        if (!rok) { ok = false; tmem_ld_wait(); break; }
-                        rph ^= 1;
-                        res_pending = false;
+            for (int c = 0; c < 4; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tbase + c * 32, r);
+                uint4 rr[4];
+                if (EPI == kEpiLN) {
+                    bool rok = mbar_wait(rbar, rph, sm.abort_flag);
+                    rok = __all_sync(0xffffffffu, rok);
+                    if (!rok) { ok = false; tmem_ld_wait(); break; }
+                    rph ^= 1;
+                    res_pending = false;
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) rr[q] = ld_shared_v4(stg + stg_off(lane, q));
-                    }
-                    tmem_ld_wait();
-                    if (c == 3) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(smem_u32(&sm.tempty[ab]));
-                    }
-                    const int col0 = ncol0 + c * 32;
-                    float v[32];
-                    const float4 *bias4 = reinterpret_cast<const float4 *>(p.bias + col0);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 bb = __ldg(bias4 + q);
-                        v[4 * q + 0] = __uint_as_float(r[4 * q + 0]) + bb.x;
-                        v[4 * q + 1] = __uint_as_float(r[4 * q + 1]) + bb.y;
-                        v[4 * q + 2] = __uint_as_float(r[4 * q + 2]) + bb.z;
-                        v[4 * q + 3] = __uint_as_float(r[4 * q + 3]) + bb.w;
-                    }
-                    if (EPI == kEpiBias) {
-                        stage_and_store(stg, v, &tmOut, col0, tile_row, lane);
-                    } else if (EPI == kEpiGelu) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = gelu_tanh_fast(v[j]);
-                        stage_and_store(stg, v, &tmOut, col0, tile_row, lane);
-                    } else if (EPI == kEpiScatter) {
-                        if (dst >= 0) store_bf16x32(p.out + (size_t)dst * p.ld_out + col0, v);
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            float2 f;
-                            f = unpack_bf16x2(rr[q].x); v[8 * q + 0] += f.x; v[8 * q + 1] += f.y;
-                            f = unpack_bf16x2(rr[q].y); v[8 * q + 2] += f.x; v[8 * q + 3] += f.y;
-                            f = unpack_bf16x2(rr[q].z); v[8 * q + 4] += f.x; v[8 * q + 5] += f.y;
-                            f = unpack_bf16x2(rr[q].w); v[8 * q + 6] += f.x; v[8 * q + 7] += f.y;
-                        }
-                        // the staging tile has been read: prefetch the next residual chunk
-                        __syncwarp();
-                        const int cn = s * 4 + c + 1;
-                        if (cn < 4 * subs) res_issue(u, cn);
-                        // exact chunk statistics, merged into the running ones
-                        float cs = 0.f;
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) cs += v[j];
-                        const float cm = cs * (1.0f / 32.0f);
-                        float cq = 0.f;
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) { const float d = v[j] - cm; cq = fmaf(d, d, cq); }
-                        if (cnt == 0.f) {
-                            mean = cm; m2 = cq;
-                        } else {
-                            const float nn = cnt + 32.f, d = cm - mean;
-                            mean = fmaf(d, 32.f / nn, mean);
-                            m2 += cq + d * d * (cnt * 32.f / nn);
-                        }
-                        cnt += 32.f;
-                        // park the pre-norm values: layout [col/4][BM][4] (coalesced per warp)
-                        const int lcol0 = s * BN + half * 128 + c * 32;
-                        float4 *sl = reinterpret_cast<float4 *>(slot);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            sl[(size_t)(lcol0 / 4 + q) * BM + r_local] =
-                                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                    }
+                    for (int q = 0; q < 4; ++q) rr[q] = ld_shared_v4(stg + stg_off(lane, q));
                 }
-                if (!ok) break;
-                ++acc;
+                tmem_ld_wait();
+                if (EPI != kEpiLN && c == 3) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&sm.tempty[ab]));
+                }
+                const int col0 = ncol0 + c * 32;
+                float v[32];
+                const float4 *bias4 = reinterpret_cast<const float4 *>(p.bias + col0);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 bb = __ldg(bias4 + q);
+                    v[4 * q + 0] = __uint_as_float(r[4 * q + 0]) + bb.x;
+                    v[4 * q + 1] = __uint_as_float(r[4 * q + 1]) + bb.y;
+                    v[4 * q + 2] = __uint_as_float(r[4 * q + 2]) + bb.z;
+                    v[4 * q + 3] = __uint_as_float(r[4 * q + 3]) + bb.w;
+                }
+                if (EPI == kEpiBias) {
+                    stage_and_store(stg, v, &tmOut, col0, tile_row, lane);
+                } else if (EPI == kEpiGelu) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = gelu_tanh_fast(v[j]);
+                    stage_and_store(stg, v, &tmOut, col0, tile_row, lane);
+                } else if (EPI == kEpiScatter) {
+                    if (dst >= 0) store_bf16x32(p.out + (size_t)dst * p.ld_out + col0, v);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float2 f;
+                        f = unpack_bf16x2(rr[q].x); v[8 * q + 0] += f.x; v[8 * q + 1] += f.y;
+                        f = unpack_bf16x2(rr[q].y); v[8 * q + 2] += f.x; v[8 * q + 3] += f.y;
+                        f = unpack_bf16x2(rr[q].z); v[8 * q + 4] += f.x; v[8 * q + 5] += f.y;
+                        f = unpack_bf16x2(rr[q].w); v[8 * q + 6] += f.x; v[8 * q + 7] += f.y;
+                    }
+                    // the staging tile has been read: prefetch the next residual chunk
+                    __syncwarp();
+                    if (c < 3) res_issue(u, c + 1);
+                    // exact chunk statistics, merged into the running ones
+                    float cs = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) cs += v[j];
+                    const float cm = cs * (1.0f / 32.0f);
+                    float cq = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) { const float d = v[j] - cm; cq = fmaf(d, d, cq); }
+                    if (c == 0) { mean = cm; m2 = cq; }
+                    else chan_merge(mean, m2, 32.f * c, cm, cq, 32.f);
+                    // keep the fp32 pre-norm sum in TMEM, over the accumulator
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(v[j]);
+                    tmem_st32(tbase + c * 32, r);
+                }
             }
             if (!ok) break;
 
             if (EPI == kEpiLN) {
-                // combine the two column halves of each row (partner warp = other half)
+                tmem_st_wait();
+                // 1. the two column halves of each row (partner warp = other half)
                 float2 *st = sm.stats + (size_t)((it & 1) * 2 + half) * BM;
                 st[r_local] = make_float2(mean, m2);
                 __syncwarp();
@@ -404,35 +411,66 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     break;
                 }
                 const float2 o = sm.stats[(size_t)((it & 1) * 2 + (half ^ 1)) * BM + r_local];
-                const float nh = cnt;  // both halves hold the same count
-                const float d = o.x - mean;
-                const float mu = mean + 0.5f * d;
-                const float var = (m2 + o.y + d * d * (nh * 0.5f)) / (2.f * nh);
-                const float rstd = rsqrtf(var + p.eps);
-                const float4 *sl = reinterpret_cast<const float4 *>(slot);
-#pragma unroll 1
-                for (int s = 0; s < subs; ++s) {
-#pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        const int col0 = s * BN + half * 128 + c * 32;
-                        float v[32];
-                        const float4 *g4 = reinterpret_cast<const float4 *>(p.ln_g + col0);
-                        const float4 *b4 = reinterpret_cast<const float4 *>(p.ln_b + col0);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const float4 z = sl[(size_t)(col0 / 4 + q) * BM + r_local];
-                            const float4 g = __ldg(g4 + q), bb = __ldg(b4 + q);
-                            v[4 * q + 0] = fmaf((z.x - mu) * rstd, g.x, bb.x);
-                            v[4 * q + 1] = fmaf((z.y - mu) * rstd, g.y, bb.y);
-                            v[4 * q + 2] = fmaf((z.z - mu) * rstd, g.z, bb.z);
-                            v[4 * q + 3] = fmaf((z.w - mu) * rstd, g.w, bb.w);
-                        }
-                        stage_and_store(stg, v, &tmOut, col0, tile_row, lane);
+                // the row over this tile's 256 columns (same result in both halves:
+                // merge in column order)
+                float tmean = half == 0 ? mean : o.x, tm2 = half == 0 ? m2 : o.y;
+                chan_merge(tmean, tm2, 128.f, half == 0 ? o.x : mean, half == 0 ? o.y : m2, 128.f);
+                // 2. publish, then gather the other tiles of the row block
+                float2 *gst = p.ln_stats + (size_t)row * n_sub;
+                int *flags = p.ln_flags + ((size_t)m * 4 + quad) * n_sub;
+                if (half == 0) {
+                    gst[n] = make_float2(tmean, tm2);
+                    __syncwarp();
+                    if (lane == 0) {
+                        __threadfence();
+                        st_release_gpu(flags + n, p.epoch);
                     }
+                }
+                float rmean = 0.f, rm2 = 0.f, rcnt = 0.f;
+                for (int k = 0; k < n_sub; ++k) {
+                    float2 pk;
+                    if (k == n) {
+                        pk = make_float2(tmean, tm2);
+                    } else {
+                        if (!wait_epoch(flags + k, p.epoch, sm.abort_flag)) { ok = false; break; }
+                        pk = __ldcg(gst + k);
+                    }
+                    if (k == 0) { rmean = pk.x; rm2 = pk.y; }
+                    else chan_merge(rmean, rm2, rcnt, pk.x, pk.y, (float)BN);
+                    rcnt += (float)BN;
+                }
+                if (!ok) break;
+                const float mu = rmean;
+                const float rstd = rsqrtf(rm2 / rcnt + p.eps);
+                // 3. normalize this warp's 128 columns from TMEM
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + c * 32, r);
+                    tmem_ld_wait();
+                    if (c == 3) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(smem_u32(&sm.tempty[ab]));
+                    }
+                    const int col0 = ncol0 + c * 32;
+                    float v[32];
+                    const float4 *g4 = reinterpret_cast<const float4 *>(p.ln_g + col0);
+                    const float4 *b4 = reinterpret_cast<const float4 *>(p.ln_b + col0);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 g = __ldg(g4 + q), bb = __ldg(b4 + q);
+                        v[4 * q + 0] = fmaf((__uint_as_float(r[4 * q + 0]) - mu) * rstd, g.x, bb.x);
+                        v[4 * q + 1] = fmaf((__uint_as_float(r[4 * q + 1]) - mu) * rstd, g.y, bb.y);
+                        v[4 * q + 2] = fmaf((__uint_as_float(r[4 * q + 2]) - mu) * rstd, g.z, bb.z);
+                        v[4 * q + 3] = fmaf((__uint_as_float(r[4 * q + 3]) - mu) * rstd, g.w, bb.w);
+                    }
+                    stage_and_store(stg, v, &tmOut, col0, tile_row, lane);
                 }
                 // first residual chunk of this CTA's next unit
                 if (u + (int)gridDim.x < units) res_issue(u + gridDim.x, 0);
             }
+            ++acc;
         }
         // outstanding copies finish before the CTA's shared memory goes away
         if (lane == 0) bulk_wait0();
@@ -451,8 +489,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 }  // namespace
 
 int gemm_grid(int epi, int rows_cap, int N, int num_sms) {
-    const int m_blocks = (rows_cap + BM - 1) / BM;
-    const int units = (epi == kEpiLN) ? m_blocks : m_blocks * (N / BN);
+    (void)epi;
+    const int units = ((rows_cap + BM - 1) / BM) * (N / BN);
     return units < num_sms ? (units > 0 ? units : 1) : num_sms;
 }
 
@@ -465,6 +503,20 @@ static cudaError_t launch_one(const CUtensorMap &tmA, const CUtensorMap &tmB, co
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
         configured = true;
+    }
+    if (EPI == kEpiLN) {
+        // CTAs of a row block wait for one another: all must be resident.
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(THREADS);
+        cfg.dynamicSmemBytes = SMEM_BYTES;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, gemm_bf16_kernel<EPI>, tmA, tmB, tmOut, tmRes, a);
     }
     gemm_bf16_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmB, tmOut, tmRes, a);
     return cudaGetLastError();

@@ -40,7 +40,9 @@ struct GemmArgs {
     float eps;
     bf16 *out;                 // [rows, ld_out] (scatter: destination rows)
     int ld_out;
-    float *scratch;            // LN: grid * BM * N floats
+    float2 *ln_stats;          // LN: per-row (mean, M2) of each 256-column tile, [rows_cap][N/256]
+    int *ln_flags;             // LN: per (row block, lane quadrant, column tile) epoch flags
+    int epoch;                 // LN: value this launch writes to ln_flags (> every earlier one)
     const int *row_dst;        // scatter: destination row or -1
     int *status;               // device status word
 };
@@ -55,8 +57,11 @@ int make_tmap_bf16_tile32(CUtensorMap *tm, const void *base, uint64_t rows, uint
 
 // Grid the GEMM uses for this many rows (persistent: <= number of SMs).
 int gemm_grid(int epi, int rows_cap, int N, int num_sms);
-// Scratch floats the LN epilogue needs for a grid of this size.
-inline size_t gemm_ln_scratch_floats(int grid) { return (size_t)grid * gemm::BM * gemm::LN_N; }
+// Cross-tile LayerNorm buffers for rows_cap rows of width LN_N.
+inline size_t gemm_ln_stats_count(int rows_cap) { return (size_t)rows_cap * (gemm::LN_N / gemm::BN); }
+inline size_t gemm_ln_flags_count(int rows_cap) {
+    return (size_t)((rows_cap + gemm::BM - 1) / gemm::BM) * 4 * (gemm::LN_N / gemm::BN);
+}
 
 // tmOut: tile32 map of the output (unused by the scatter epilogue); tmRes: tile32
 // map of the residual (LayerNorm epilogue only; pass any valid map otherwise).
