@@ -171,7 +171,8 @@ int albert_profile_read(albert_handle *h, int *launches, double *ms);
  * bf16, bias: [N] fp32 (device).  epi: 0 = bias -> bf16 Y[M, N];
  * 1 = tanh-GELU(+bias) -> bf16; 2 = LN(A W^T + bias + R; g, b, eps) -> bf16,
  * with R: [M, N] bf16 and N == 768; 3 = bias -> bf16 rows scattered to
- * row_dst[r] (row_dst[r] < 0 skips the row).  K % 64 == 0, N % 256 == 0. */
+ * row_dst[r] (row_dst[r] < 0 skips the row).  K % 64 == 0, N % 256 == 0;
+ * bias and ln_g 16-byte aligned (else ALBERT_ERR_CONFIG). */
 int albert_test_gemm(const void *A, const void *W, const float *bias, const void *R,
                      const float *ln_g, const float *ln_b, float eps, const int32_t *row_dst,
                      void *Y, int M, int N, int K, int epi, void *stream);
@@ -188,23 +189,25 @@ int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, 
  * that must not allocate device memory while running -- a real-time audio
  * thread that cannot absorb cudaMalloc's device-wide synchronization and
  * latency, or a runtime that lays out all device memory before its first
- * request.  It computes Y = LN(A W^T + bias + R; ln_g, ln_b, eps) exactly like
- * albert_test_gemm with epi = 2, but its scratch (the per-row LayerNorm
- * statistics and epoch flags its column tiles exchange, a row-count word and
- * the status word) lives in file-scope __device__ arrays of about 195 KiB
- * inside the library instead of memory the call allocates; it calls no
+ * request.  It computes Y = LN(A W^T + bias + R; ln_g, ln_b, eps) with the
+ * same two kernels as albert_test_gemm with epi = 2 (the GEMM whose epilogue
+ * forms the pre-norm row, then the row normalization), but their scratch
+ * (z * ln_g as bf16, per-row partial statistics, a row-count word and the
+ * status word) lives in file-scope __device__ arrays of about 3.1 MiB inside
+ * the library instead of memory the call allocates; it calls no
  * cudaMalloc/cudaFree.
  *   A: [M, K] bf16, W: [768, K] bf16, bias/ln_g/ln_b: [768] fp32,
  *   R: [M, 768] bf16, Y: [M, 768] bf16, all device pointers the caller owns.
- *   Limits: 1 <= M <= 8192 (the size the arrays hold), K % 64 == 0;
- *   anything else returns ALBERT_ERR_SHAPE before any work is enqueued.
+ *   Limits: 1 <= M <= 2048 (the rows the arrays hold), K % 64 == 0;
+ *   anything else returns ALBERT_ERR_SHAPE before any work is enqueued;
+ *   bias and ln_g must be 16-byte aligned (else ALBERT_ERR_CONFIG).
  * The arrays are reserved on every device where the library's module holding
  * them is loaded and stay until the process exits.  The first call on a device
  * looks up their device addresses (cudaGetSymbolAddress) with that device
  * current; make that first call before any stream capture.  Every call shares
- * the same arrays (the status word is reset by each call; statistics are
- * rewritten before they are read and flags carry a per-call epoch, so nothing
- * else needs clearing), so calls that overlap on the GPU -- on different
+ * the same arrays (the status word is reset by each call; the intermediates
+ * are rewritten before they are read, so nothing else needs clearing), so
+ * calls that overlap on the GPU -- on different
  * streams or from different threads -- race and must be serialized by the
  * caller.  Synchronous: returns the kernel's status. */
 int albert_gemm_residual_ln_noalloc(const void *A, const void *W, const float *bias, const void *R,

@@ -3,6 +3,11 @@
 Tolerances (stated for the encoder output over valid tokens):
   bf16 path: max |gpu - oracle| <= 3e-2 and per-token cosine >= 0.999;
   fp32 path: ||gpu - oracle||_inf / ||oracle||_inf <= 1e-4.
+Hidden-state checkpoints (the [T, 768] LayerNorm outputs, unit variance, |x| up
+to ~5) get the same cosine bar and an elementwise bar of 3e-2 + 2^-7 |ref|:
+one bf16 ulp of the value on top of the output bar, for the extra bf16
+rounding of z * gamma that the deferred LayerNorm carries to its consumer
+(a half-ulp at |x| in [4, 8) is already 0.0156).
 """
 import numpy as np
 
@@ -20,11 +25,16 @@ def per_token_cosine(a: np.ndarray, b: np.ndarray) -> np.ndarray:
     return (a * b).sum(-1) / (np.linalg.norm(a, axis=-1) * np.linalg.norm(b, axis=-1) + 1e-300)
 
 
-def check_bf16(gpu: np.ndarray, ref: np.ndarray, what: str = ""):
-    err = float(np.max(np.abs(gpu.astype(np.float64) - ref)))
+def check_bf16(gpu: np.ndarray, ref: np.ndarray, what: str = "", checkpoint: bool = False):
+    diff = np.abs(gpu.astype(np.float64) - ref)
+    err = float(np.max(diff))
     cos = float(np.min(per_token_cosine(gpu, ref)))
     assert np.all(np.isfinite(gpu)), f"{what}: non-finite output"
-    assert err <= BF16_MAX_ABS, f"{what}: max abs err {err:.3e} > {BF16_MAX_ABS}"
+    if checkpoint:
+        excess = float(np.max(diff - (BF16_MAX_ABS + 2.0 ** -7 * np.abs(ref))))
+        assert excess <= 0, f"{what}: checkpoint error {err:.3e} exceeds 3e-2 + 2^-7|ref| by {excess:.3e}"
+    else:
+        assert err <= BF16_MAX_ABS, f"{what}: max abs err {err:.3e} > {BF16_MAX_ABS}"
     assert cos >= BF16_MIN_COS, f"{what}: min per-token cosine {cos:.6f} < {BF16_MIN_COS}"
     return err, cos
 

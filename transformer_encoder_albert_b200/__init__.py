@@ -257,7 +257,7 @@ def test_attention(qkv, cu_seqlens, max_len: int, ctx, fp32: bool = False, strea
 
 def gemm_residual_ln_noalloc(A, W, bias, R, ln_g, ln_b, Y, eps: float = 1e-12, stream=None) -> int:
     """Y = LN(A W^T + bias + R) through the entry point that allocates no device
-    memory (static scratch inside the library; M <= 8192)."""
+    memory (static scratch inside the library; M <= 2048)."""
     M, K = A.shape
     return lib().albert_gemm_residual_ln_noalloc(_ptr(A), _ptr(W), _ptr(bias), _ptr(R), _ptr(ln_g),
                                                  _ptr(ln_b), float(eps), _ptr(Y), M, K,

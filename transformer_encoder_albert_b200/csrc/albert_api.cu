@@ -50,10 +50,16 @@ struct albert_handle {
     size_t wblock_bytes = 0;
 
     // workspace
+    // bf16: X = input projection output, X1 = z1 * gamma1, Z = z2 * gamma2 (z1, z2:
+    // the pre-norm rows of the two LayerNorms, normalized by their consumers);
+    // fp32: X, X1 = LayerNorm outputs, Z = pre-norm rows.
     void *E = nullptr, *X = nullptr, *QKV = nullptr, *C = nullptr, *X1 = nullptr, *H = nullptr, *Z = nullptr;
-    float2 *ln_stats = nullptr;  // per-row (mean, M2) of each 256-column tile
-    int *ln_flags = nullptr;     // epoch flags of the LayerNorm GEMM's cross-CTA exchange
-    int ln_epoch = 0;            // last epoch handed to a LayerNorm GEMM launch
+    float2 *st1 = nullptr, *st2 = nullptr;  // partial (mean, M2) of z1 / z2, [rows][6]
+    // folded LayerNorm constants: s = W gamma, c = W beta + b, and biases plus the
+    // beta of a rebuilt residual
+    float *fold = nullptr;
+    float *s_qkv = nullptr, *c_qkv = nullptr, *s_1 = nullptr, *c_1 = nullptr, *s_out = nullptr, *c_out = nullptr;
+    float *bias_o2 = nullptr, *bias_21 = nullptr;
     int *seq_start = nullptr, *seq_len = nullptr, *row_dst = nullptr, *n_rows = nullptr, *status = nullptr;
 
     // host-buffer staging
@@ -62,9 +68,9 @@ struct albert_handle {
     void *st_out = nullptr;
 
     // TMA descriptors (bf16)
-    CUtensorMap tm_E, tm_X, tm_C, tm_X1, tm_H;
+    CUtensorMap tm_E, tm_X, tm_C, tm_X1, tm_H, tm_Z;
     CUtensorMap tm_win, tm_wqkv, tm_wo, tm_w1, tm_w2, tm_wout;
-    CUtensorMap t32_X, t32_QKV, t32_X1, t32_H;  // 32x32-box maps: epilogue stores / residual loads
+    CUtensorMap t32_X, t32_QKV, t32_X1, t32_H, t32_Z;  // 32x32-box maps: epilogue stores / residual loads
 
     // per-kernel timing
     unsigned prof_mask = 0;  // classes whose launches are timed
@@ -172,8 +178,6 @@ GemmArgs gemm_args(albert_handle *h, int N, int K, const float *bias, void *out,
     a.bias = bias;
     a.out = static_cast<bf16 *>(out);
     a.ld_out = ld_out;
-    a.ln_stats = h->ln_stats;
-    a.ln_flags = h->ln_flags;
     a.row_dst = h->row_dst;
     a.status = h->status;
     a.eps = h->cfg.ln_eps;
@@ -183,10 +187,8 @@ GemmArgs gemm_args(albert_handle *h, int N, int K, const float *bias, void *out,
 int gemm_bf16(Launch &L, int cls, int epi, const CUtensorMap &A, const CUtensorMap &B, const CUtensorMap &Out,
               const CUtensorMap &Res, GemmArgs a) {
     const int grid = gemm_grid(epi, a.rows_cap, a.N, L.h->num_sms);
-    if (epi == kEpiLN) {
-        if (a.N != gemm::LN_N) return ALBERT_ERR_CONFIG;
-        a.epoch = ++L.h->ln_epoch;
-    }
+    if (epi == kEpiResStats && a.N != gemm::LN_N) return ALBERT_ERR_CONFIG;
+    if (!gemm_vectors_aligned(a)) return ALBERT_ERR_CONFIG;
     LAUNCH(L, cls, launch_gemm(epi, A, B, Out, Res, a, grid, L.s));
     return ALBERT_OK;
 }
@@ -212,6 +214,7 @@ GemmF32Args f32_args(albert_handle *h, const void *A, const void *W, const float
 int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, int nseq, int T,
                int max_len, void *out, int padded_api) {
     const albert_config &c = h->cfg;
+    const int out_rows = padded_api ? nseq * T : c.max_tokens;
     const bool bf = c.dtype == ALBERT_BF16;
     EmbedArgs ea{};
     ea.ids = ids;
@@ -239,29 +242,61 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
     const int D = out_width(h);
     if (bf) {
         int rc;
-        if ((rc = gemm_bf16(L, kProfGemmIn, kEpiBias, h->tm_E, h->tm_win, h->t32_X, h->t32_X, gemm_args(h, kHidden, kEmb, h->b_in, h->X, kHidden)))) return rc;
+        if ((rc = gemm_bf16(L, kProfGemmIn, kEpiBias, h->tm_E, h->tm_win, h->t32_X, h->t32_X,
+                            gemm_args(h, kHidden, kEmb, h->b_in, nullptr, 0))))
+            return rc;
         for (int l = 0; l < c.n_exec; ++l) {
-            if ((rc = gemm_bf16(L, kProfGemmQKV, kEpiBias, h->tm_X, h->tm_wqkv, h->t32_QKV, h->t32_QKV, gemm_args(h, kQKV, kHidden, h->bqkv, h->QKV, kQKV)))) return rc;
+            // Q|K|V from the layer input: X for the first execution, else LN2(z2) folded
+            if (l == 0) {
+                rc = gemm_bf16(L, kProfGemmQKV, kEpiBias, h->tm_X, h->tm_wqkv, h->t32_QKV, h->t32_QKV,
+                               gemm_args(h, kQKV, kHidden, h->bqkv, nullptr, 0));
+            } else {
+                GemmArgs a = gemm_args(h, kQKV, kHidden, h->c_qkv, nullptr, 0);
+                a.fold_s = h->s_qkv;
+                a.in_stats = h->st2;
+                rc = gemm_bf16(L, kProfGemmQKV, kEpiLnIn, h->tm_Z, h->tm_wqkv, h->t32_QKV, h->t32_QKV, a);
+            }
+            if (rc) return rc;
             LAUNCH(L, kProfAttention, launch_attention_bf16(static_cast<bf16 *>(h->QKV), static_cast<bf16 *>(h->C), h->seq_start,
                                                            h->seq_len, nseq, max_len, h->status, L.s));
-            GemmArgs a = gemm_args(h, kHidden, kHidden, h->bo, h->X1, kHidden);
-            a.resid = static_cast<bf16 *>(h->X);
-            a.ld_resid = kHidden;
-            a.ln_g = h->ln1_g;
-            a.ln_b = h->ln1_b;
-            if ((rc = gemm_bf16(L, kProfGemmWoLN, kEpiLN, h->tm_C, h->tm_wo, h->t32_X1, h->t32_X, a))) return rc;
-            if ((rc = gemm_bf16(L, kProfGemmW1Gelu, kEpiGelu, h->tm_X1, h->tm_w1, h->t32_H, h->t32_H, gemm_args(h, kFfn, kHidden, h->b1, h->H, kFfn)))) return rc;
-            a = gemm_args(h, kHidden, kFfn, h->b2, h->X, kHidden);
-            a.resid = static_cast<bf16 *>(h->X1);
-            a.ld_resid = kHidden;
-            a.ln_g = h->ln2_g;
-            a.ln_b = h->ln2_b;
-            if ((rc = gemm_bf16(L, kProfGemmW2LN, kEpiLN, h->tm_H, h->tm_w2, h->t32_X, h->t32_X1, a))) return rc;
+            // z1 = C Wo^T + bo + layer input -> X1 = z1 * gamma1, st1
+            GemmArgs a = gemm_args(h, kHidden, kHidden, l == 0 ? h->bo : h->bias_o2, nullptr, 0);
+            a.res_stats = l == 0 ? nullptr : h->st2;
+            a.res_g = h->ln2_g;
+            a.out_g = h->ln1_g;
+            a.out_stats = h->st1;
+            if ((rc = gemm_bf16(L, kProfGemmWoLN, kEpiResStats, h->tm_C, h->tm_wo, h->t32_X1, l == 0 ? h->t32_X : h->t32_Z, a)))
+                return rc;
+            // H = GELU(LN1(z1) W1^T + b1)
+            a = gemm_args(h, kFfn, kHidden, h->c_1, nullptr, 0);
+            a.fold_s = h->s_1;
+            a.in_stats = h->st1;
+            if ((rc = gemm_bf16(L, kProfGemmW1Gelu, kEpiLnInGelu, h->tm_X1, h->tm_w1, h->t32_H, h->t32_H, a))) return rc;
+            // z2 = H W2^T + b2 + LN1(z1) -> Z = z2 * gamma2, st2
+            a = gemm_args(h, kHidden, kFfn, h->bias_21, nullptr, 0);
+            a.res_stats = h->st1;
+            a.res_g = h->ln1_g;
+            a.out_g = h->ln2_g;
+            a.out_stats = h->st2;
+            if ((rc = gemm_bf16(L, kProfGemmW2LN, kEpiResStats, h->tm_H, h->tm_w2, h->t32_Z, h->t32_X1, a))) return rc;
         }
         if (c.out_dim > 0) {
-            if ((rc = gemm_bf16(L, kProfGemmOut, kEpiScatter, h->tm_X, h->tm_wout, h->t32_X, h->t32_X, gemm_args(h, c.out_dim, kHidden, h->b_out, out, c.out_dim)))) return rc;
-        } else {
+            if (c.n_exec == 0) {
+                rc = gemm_bf16(L, kProfGemmOut, kEpiScatter, h->tm_X, h->tm_wout, h->t32_X, h->t32_X,
+                               gemm_args(h, c.out_dim, kHidden, h->b_out, out, c.out_dim));
+            } else {
+                GemmArgs a = gemm_args(h, c.out_dim, kHidden, h->c_out, out, c.out_dim);
+                a.fold_s = h->s_out;
+                a.in_stats = h->st2;
+                rc = gemm_bf16(L, kProfGemmOut, kEpiLnInScatter, h->tm_Z, h->tm_wout, h->t32_X, h->t32_X, a);
+            }
+            if (rc) return rc;
+        } else if (c.n_exec == 0) {
             LAUNCH(L, kProfOutput, launch_scatter_rows(h->X, out, kHidden, 2, h->rows_cap, h->n_rows, h->row_dst, h->status, L.s));
+        } else {
+            LAUNCH(L, kProfOutput, launch_ln_rows(static_cast<bf16 *>(h->Z), h->st2, h->ln2_g, h->ln2_b, c.ln_eps,
+                                                  static_cast<bf16 *>(out), h->row_dst, out_rows, h->rows_cap, h->n_rows,
+                                                  h->status, L.s));
         }
     } else {
         LAUNCH(L, kProfGemmIn, launch_gemm_f32(kF32Bias, f32_args(h, h->E, h->w_in, h->b_in, h->X, kHidden, kHidden, kEmb), L.s));
@@ -324,12 +359,14 @@ int create_impl(albert_handle *h, const albert_weights *w) {
 
     // ---- small fp32 parameters: one block ----
     const size_t V = c.vocab, P = c.max_pos, NT = c.n_types, O = c.out_dim;
-    const size_t n_small = V * kEmb + P * kEmb + NT * kEmb + 2 * kEmb + kHidden + kQKV + kHidden + 2 * kHidden +
-                           kFfn + kHidden + 2 * kHidden + O;
+    auto sl = [](size_t n) { return (n + 63) / 64 * 64; };
+    const size_t n_small = sl(V * kEmb) + sl(P * kEmb) + sl(NT * kEmb) + 2 * sl(kEmb) + sl(kHidden) + sl(kQKV) +
+                           sl(kHidden) + 2 * sl(kHidden) + sl(kFfn) + sl(kHidden) + 2 * sl(kHidden) + sl(O);
     float *small = nullptr;
     if ((rc = dev_alloc(h, (void **)&small, n_small * sizeof(float)))) return rc;
     float *q = small;
-    auto take = [&](size_t n) { float *r = q; q += n; return r; };
+    // slices start on 256-byte boundaries (kernels read several of them as float4)
+    auto take = [&](size_t n) { float *r = q; q += (n + 63) / 64 * 64; return r; };
     h->word = take(V * kEmb); h->pos = take(P * kEmb); h->type = take(NT * kEmb);
     h->emb_g = take(kEmb); h->emb_b = take(kEmb); h->b_in = take(kHidden); h->bqkv = take(kQKV);
     h->bo = take(kHidden); h->ln1_g = take(kHidden); h->ln1_b = take(kHidden); h->b1 = take(kFfn);
@@ -379,12 +416,27 @@ int create_impl(albert_handle *h, const albert_weights *w) {
     if ((rc = dev_alloc(h, &h->C, R * kHidden * eb))) return rc;
     if ((rc = dev_alloc(h, &h->X1, R * kHidden * eb))) return rc;
     if ((rc = dev_alloc(h, &h->H, R * kFfn * eb))) return rc;
+    if ((rc = dev_alloc(h, &h->Z, R * kHidden * eb))) return rc;
     if (bf) {
-        if ((rc = dev_alloc(h, (void **)&h->ln_stats, gemm_ln_stats_count(h->rows_cap) * sizeof(float2)))) return rc;
-        if ((rc = dev_alloc(h, (void **)&h->ln_flags, gemm_ln_flags_count(h->rows_cap) * sizeof(int)))) return rc;
-        TRY(cudaMemsetAsync(h->ln_flags, 0, gemm_ln_flags_count(h->rows_cap) * sizeof(int), s));
-    } else {
-        if ((rc = dev_alloc(h, &h->Z, R * kHidden * eb))) return rc;
+        const size_t nst = R * gemm::LN_PARTS;
+        if ((rc = dev_alloc(h, (void **)&h->st1, nst * sizeof(float2)))) return rc;
+        if ((rc = dev_alloc(h, (void **)&h->st2, nst * sizeof(float2)))) return rc;
+        TRY(cudaMemsetAsync(h->st1, 0, nst * sizeof(float2), s));
+        TRY(cudaMemsetAsync(h->st2, 0, nst * sizeof(float2), s));
+        // every vector starts on a 256-byte boundary: the epilogues read them as float4
+        auto seg = [](size_t n) { return (n + 63) / 64 * 64; };
+        const size_t nf = 2 * seg(kQKV) + 2 * seg(kFfn) + 2 * seg(O) + 2 * seg(kHidden);
+        if ((rc = dev_alloc(h, (void **)&h->fold, nf * sizeof(float)))) return rc;
+        float *f = h->fold;
+        h->s_qkv = f; f += seg(kQKV); h->c_qkv = f; f += seg(kQKV);
+        h->s_1 = f; f += seg(kFfn); h->c_1 = f; f += seg(kFfn);
+        h->s_out = f; f += seg(O); h->c_out = f; f += seg(O);
+        h->bias_o2 = f; f += seg(kHidden); h->bias_21 = f;
+        TRY(launch_fold_ln(static_cast<const bf16 *>(h->wqkv), kQKV, kHidden, h->ln2_g, h->ln2_b, h->bqkv, h->s_qkv, h->c_qkv, s));
+        TRY(launch_fold_ln(static_cast<const bf16 *>(h->w1), kFfn, kHidden, h->ln1_g, h->ln1_b, h->b1, h->s_1, h->c_1, s));
+        if (O) TRY(launch_fold_ln(static_cast<const bf16 *>(h->w_out), (int)O, kHidden, h->ln2_g, h->ln2_b, h->b_out, h->s_out, h->c_out, s));
+        TRY(launch_vec_add(h->bo, h->ln2_b, h->bias_o2, kHidden, s));
+        TRY(launch_vec_add(h->b2, h->ln1_b, h->bias_21, kHidden, s));
     }
     if ((rc = dev_alloc(h, (void **)&h->seq_start, (h->seq_cap + 1) * sizeof(int)))) return rc;
     if ((rc = dev_alloc(h, (void **)&h->seq_len, (h->seq_cap + 1) * sizeof(int)))) return rc;
@@ -395,7 +447,7 @@ int create_impl(albert_handle *h, const albert_weights *w) {
     if ((rc = dev_alloc(h, (void **)&h->st_mask, (size_t)c.max_tokens))) return rc;
     if ((rc = dev_alloc(h, &h->st_out, (size_t)c.max_tokens * out_width(h) * eb))) return rc;
     // Deterministic contents for rows a forward never writes.
-    for (void *p : {h->E, h->X, h->QKV, h->C, h->X1, h->H}) {
+    for (void *p : {h->E, h->X, h->QKV, h->C, h->X1, h->H, h->Z}) {
         size_t bytes = (p == h->E ? kEmb : p == h->QKV ? kQKV : p == h->H ? kFfn : kHidden) * R * eb;
         TRY(cudaMemsetAsync(p, 0, bytes, s));
     }
@@ -405,7 +457,7 @@ int create_impl(albert_handle *h, const albert_weights *w) {
     if (bf) {
         if (make_tmap_bf16(&h->tm_E, h->E, R, kEmb, gemm::BM) || make_tmap_bf16(&h->tm_X, h->X, R, kHidden, gemm::BM) ||
             make_tmap_bf16(&h->tm_C, h->C, R, kHidden, gemm::BM) || make_tmap_bf16(&h->tm_X1, h->X1, R, kHidden, gemm::BM) ||
-            make_tmap_bf16(&h->tm_H, h->H, R, kFfn, gemm::BM) ||
+            make_tmap_bf16(&h->tm_H, h->H, R, kFfn, gemm::BM) || make_tmap_bf16(&h->tm_Z, h->Z, R, kHidden, gemm::BM) ||
             make_tmap_bf16(&h->tm_win, h->w_in, kHidden, kEmb, gemm::BN) ||
             make_tmap_bf16(&h->tm_wqkv, h->wqkv, kQKV, kHidden, gemm::BN) ||
             make_tmap_bf16(&h->tm_wo, h->wo, kHidden, kHidden, gemm::BN) ||
@@ -413,7 +465,8 @@ int create_impl(albert_handle *h, const albert_weights *w) {
             make_tmap_bf16(&h->tm_w2, h->w2, kHidden, kFfn, gemm::BN) ||
             (O && make_tmap_bf16(&h->tm_wout, h->w_out, O, kHidden, gemm::BN)) ||
             make_tmap_bf16_tile32(&h->t32_X, h->X, R, kHidden) || make_tmap_bf16_tile32(&h->t32_QKV, h->QKV, R, kQKV) ||
-            make_tmap_bf16_tile32(&h->t32_X1, h->X1, R, kHidden) || make_tmap_bf16_tile32(&h->t32_H, h->H, R, kFfn))
+            make_tmap_bf16_tile32(&h->t32_X1, h->X1, R, kHidden) || make_tmap_bf16_tile32(&h->t32_H, h->H, R, kFfn) ||
+            make_tmap_bf16_tile32(&h->t32_Z, h->Z, R, kHidden))
             return ALBERT_ERR_CUDA;
     }
     TRY(cudaStreamSynchronize(s));
@@ -548,48 +601,50 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
     if (!A || !W || !bias || !Y) return ALBERT_ERR_NULL;
     if (M < 1 || N < gemm::BN || N % gemm::BN || K < gemm::BK || K % gemm::BK) return ALBERT_ERR_SHAPE;
     if (epi < 0 || epi > 3) return ALBERT_ERR_CONFIG;
-    if (epi == kEpiLN && (!R || !ln_g || !ln_b || N != gemm::LN_N)) return ALBERT_ERR_CONFIG;
-    if (epi == kEpiScatter && !row_dst) return ALBERT_ERR_NULL;
+    if (epi == 2 && (!R || !ln_g || !ln_b || N != gemm::LN_N)) return ALBERT_ERR_CONFIG;
+    if (epi == 3 && !row_dst) return ALBERT_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(bias) | reinterpret_cast<uintptr_t>(ln_g)) & 15) return ALBERT_ERR_CONFIG;
+    const int kepi = epi == 0 ? kEpiBias : epi == 1 ? kEpiGelu : epi == 2 ? kEpiResStats : kEpiScatter;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int dev = 0, sms = 0;
     TRY(cudaGetDevice(&dev));
     TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
     const int rows_cap = (M + gemm::BM - 1) / gemm::BM * gemm::BM;
-    const int grid = gemm_grid(epi, rows_cap, N, sms);
-    CUtensorMap ta, tb, to, tr;
-    if (make_tmap_bf16(&ta, A, M, K, gemm::BM) || make_tmap_bf16(&tb, W, N, K, gemm::BN)) return ALBERT_ERR_CUDA;
-    if (epi != kEpiScatter && make_tmap_bf16_tile32(&to, Y, M, N)) return ALBERT_ERR_CUDA;
-    if (epi == kEpiScatter) to = ta;
-    if (epi == kEpiLN) {
-        if (make_tmap_bf16_tile32(&tr, R, M, N)) return ALBERT_ERR_CUDA;
-    } else {
-        tr = to;
-    }
+    const int grid = gemm_grid(kepi, rows_cap, N, sms);
+    // epi 2 writes z * gamma and row statistics to temporaries, then normalizes them into Y
     int *ints = nullptr;
+    void *zg = nullptr;
     float2 *stats = nullptr;
-    int *flags = nullptr;
     TRY(cudaMalloc(&ints, 2 * sizeof(int)));
-    if (epi == kEpiLN && (cudaMalloc(&stats, gemm_ln_stats_count(rows_cap) * sizeof(float2)) != cudaSuccess ||
-                          cudaMalloc(&flags, gemm_ln_flags_count(rows_cap) * sizeof(int)) != cudaSuccess)) {
+    if (epi == 2 && (cudaMalloc(&zg, (size_t)rows_cap * N * 2) != cudaSuccess ||
+                     cudaMalloc(&stats, (size_t)rows_cap * gemm::LN_PARTS * sizeof(float2)) != cudaSuccess)) {
         cudaFree(ints);
-        cudaFree(stats);
+        cudaFree(zg);
         return ALBERT_ERR_ALLOC;
     }
+    CUtensorMap ta, tb, to, tr;
+    int bad = make_tmap_bf16(&ta, A, M, K, gemm::BM) || make_tmap_bf16(&tb, W, N, K, gemm::BN);
+    if (epi == 2) bad = bad || make_tmap_bf16_tile32(&to, zg, rows_cap, N) || make_tmap_bf16_tile32(&tr, R, M, N);
+    else if (epi != 3) bad = bad || make_tmap_bf16_tile32(&to, Y, M, N);
+    if (epi == 3) to = ta;
+    if (epi != 2) tr = to;
+    cudaError_t e = bad ? cudaErrorInvalidValue : cudaSuccess;
     const int host_ints[2] = {M, 0};
-    cudaError_t e = cudaMemcpyAsync(ints, host_ints, sizeof(host_ints), cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess && flags) e = cudaMemsetAsync(flags, 0, gemm_ln_flags_count(rows_cap) * sizeof(int), s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ints, host_ints, sizeof(host_ints), cudaMemcpyHostToDevice, s);
     GemmArgs a{};
-    a.N = N; a.K = K; a.rows_cap = rows_cap; a.n_rows = ints; a.bias = bias;
-    a.resid = static_cast<const bf16 *>(R); a.ld_resid = N; a.ln_g = ln_g; a.ln_b = ln_b; a.eps = eps;
-    a.out = static_cast<bf16 *>(Y); a.ld_out = N; a.ln_stats = stats; a.ln_flags = flags; a.epoch = 1;
+    a.N = N; a.K = K; a.rows_cap = rows_cap; a.n_rows = ints; a.bias = bias; a.eps = eps;
+    a.out_g = ln_g; a.out_stats = stats; a.out = static_cast<bf16 *>(Y); a.ld_out = N;
     a.row_dst = row_dst; a.status = ints + 1;
-    if (e == cudaSuccess) e = launch_gemm(epi, ta, tb, to, tr, a, grid, s);
+    if (e == cudaSuccess) e = launch_gemm(kepi, ta, tb, to, tr, a, grid, s);
+    if (e == cudaSuccess && epi == 2)
+        e = launch_ln_rows(static_cast<const bf16 *>(zg), stats, ln_g, ln_b, eps, static_cast<bf16 *>(Y), nullptr, M,
+                           rows_cap, ints, ints + 1, s);
     int st = 0;
     if (e == cudaSuccess) e = cudaMemcpyAsync(&st, ints + 1, sizeof(int), cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     cudaFree(ints);
+    if (zg) cudaFree(zg);
     if (stats) cudaFree(stats);
-    if (flags) cudaFree(flags);
     return e == cudaSuccess ? st : ALBERT_ERR_CUDA;
 }
 

@@ -14,23 +14,27 @@
 //                 128x256 fp32 accumulators (512 TMEM columns), so the epilogue
 //                 of one tile overlaps the main loop of the next;
 //   warps 2..9  : epilogue, 2 warps per TMEM lane quadrant (column halves);
-//                 tcgen05.ld -> bias (+ tanh-GELU | + residual, LayerNorm) ->
-//                 bf16 32x32 tile in a swizzled shared staging buffer -> TMA
-//                 bulk tensor store (coalesced, asynchronous; one-row-per-lane
-//                 global stores would contend with the tensor core's
-//                 shared-memory operand reads in the unified L1/shared array).
-// LayerNorm epilogue (post-LN steps 5 and 6, rows of 768 = 3 tiles of 256):
-// each tile's epilogue adds bias and residual (residual tiles arrive by TMA,
-// one 32-column chunk ahead), writes the fp32 pre-norm sum back into its TMEM
-// accumulator, and keeps exact per-row (mean, M2) statistics (Chan's merge of
-// 32-column chunks, then of the two column halves through shared memory).
-// The three tiles of a row block run on three CTAs at the same time: each
-// publishes its per-row statistics to a small global buffer with a release
-// flag tagged by the launch's epoch and acquires the other two, then
-// normalizes its 256 columns straight from TMEM.  The cross-CTA waits need
-// every CTA resident, so this variant is launched cooperatively.
-// Every wait is bounded (%globaltimer); on expiry the CTA records
-// ALBERT_ERR_TIMEOUT, drains its in-flight copies and MMAs, frees TMEM and exits.
+//                 tcgen05.ld -> epilogue math -> bf16 32x32 tile in a swizzled
+//                 shared staging buffer -> TMA bulk tensor store (coalesced,
+//                 asynchronous; one-row-per-lane global stores would contend
+//                 with the tensor core's shared-memory operand reads in the
+//                 unified L1/shared array).
+//
+// Post-LN LayerNorms (steps 5 and 6) are deferred to the consumers of their
+// output, so every epilogue is a single pass with no cross-CTA dependency:
+//   * the GEMM that forms the pre-norm row z = acc + bias + residual writes
+//     z * gamma (bf16) and, per row and 128-column slice, exact (mean, M2)
+//     statistics of z (two-pass inside each 32-column chunk, Chan's merge
+//     across chunks);
+//   * a GEMM that reads z * gamma as its A operand merges the six partial
+//     statistics of its row into (mu, rstd) and applies
+//     LN(z) W^T = rstd * (z*gamma) W^T - rstd * mu * (W gamma) + W beta;
+//   * a GEMM whose residual is LN(z) rebuilds it from the z*gamma tile as
+//     rstd * (z*gamma) - rstd * mu * gamma + beta.
+// Residual tiles arrive by TMA into a second per-warp staging tile, one
+// 32-column chunk ahead.  Every wait is bounded (%globaltimer); on expiry the
+// CTA records ALBERT_ERR_TIMEOUT, drains its in-flight copies and MMAs, frees
+// TMEM and exits.
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
@@ -40,13 +44,13 @@ namespace {
 using namespace gemm;
 
 struct Smem {
-    uint8_t *a, *b, *stg;    // stg: one 2 KB 32x32 bf16 staging tile per epilogue warp
+    uint8_t *a, *b;
+    uint8_t *stg;            // one 2 KB output staging tile per epilogue warp
+    uint8_t *rstg;           // one 2 KB residual staging tile per epilogue warp
     uint64_t *full, *empty, *tfull, *tempty, *drain, *rbar;
     uint32_t *tmem_slot;
     volatile int *abort_flag;
     int *misc;               // [0] n_rows, [1] status at entry
-    volatile int *pair_flag; // [4 quadrants][2 halves]
-    float2 *stats;           // [2 buffers][2 halves][BM]
 };
 
 __device__ __forceinline__ Smem carve(uint8_t *raw) {
@@ -55,7 +59,8 @@ __device__ __forceinline__ Smem carve(uint8_t *raw) {
     s.a = p;
     s.b = p + STAGES * A_BYTES;
     s.stg = s.b + STAGES * B_BYTES;
-    uint8_t *ctrl = s.stg + EPI_WARPS * STG_BYTES;
+    s.rstg = s.stg + EPI_WARPS * STG_BYTES;
+    uint8_t *ctrl = s.rstg + EPI_WARPS * STG_BYTES;
     uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl);
     s.full = bars;
     s.empty = bars + STAGES;
@@ -67,48 +72,7 @@ __device__ __forceinline__ Smem carve(uint8_t *raw) {
     s.tmem_slot = u;
     s.abort_flag = reinterpret_cast<volatile int *>(u + 1);
     s.misc = reinterpret_cast<int *>(u + 2);
-    s.pair_flag = reinterpret_cast<volatile int *>(u + 4);
-    s.stats = reinterpret_cast<float2 *>(ctrl + 1024);
     return s;
-}
-
-// Wait on the partner warp's flag (bounded); only lane 0 polls.
-__device__ __forceinline__ bool wait_flag(volatile int *flag, int target, volatile int *abort_flag) {
-    bool ok = true;
-    if ((threadIdx.x & 31) == 0) {
-        const unsigned long long t0 = globaltimer_ns();
-        while (*flag < target) {
-            if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
-                *abort_flag = 1;
-                ok = false;
-                break;
-            }
-        }
-    }
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    __threadfence_block();
-    __syncwarp();
-    return ok;
-}
-
-// Wait (bounded, lane 0 polls) until another CTA has published `epoch` at *flag.
-__device__ __forceinline__ bool wait_epoch(const int *flag, int epoch, volatile int *abort_flag) {
-    bool ok = true;
-    if ((threadIdx.x & 31) == 0) {
-        if (ld_acquire_gpu(flag) != epoch) {
-            const unsigned long long t0 = globaltimer_ns();
-            while (ld_acquire_gpu(flag) != epoch) {
-                if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
-                    *abort_flag = 1;
-                    ok = false;
-                    break;
-                }
-            }
-        }
-    }
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    __syncwarp();
-    return ok;
 }
 
 __device__ __forceinline__ void store_bf16x32(bf16 *dst, const float (&v)[32]) {
@@ -171,11 +135,34 @@ __device__ __forceinline__ void chan_merge(float &mean, float &m2, float cnt, fl
     m2 += cq + d * d * (cnt * cn / nn);
 }
 
+// Mean and 1/sqrt(var + eps) of a 768-wide row from its six 128-column partials.
+__device__ __forceinline__ void row_stats(const float2 *part, float eps, float &mu, float &rstd) {
+    float2 q[LN_PARTS];
+#pragma unroll
+    for (int i = 0; i < LN_PARTS; ++i) q[i] = __ldg(part + i);
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < LN_PARTS; ++i) m += q[i].x;
+    m *= (1.0f / LN_PARTS);
+    float m2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < LN_PARTS; ++i) {
+        const float d = q[i].x - m;
+        m2 += q[i].y + (float)(LN_N / LN_PARTS) * d * d;
+    }
+    mu = m;
+    rstd = rsqrtf(m2 * (1.0f / LN_N) + eps);
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmRes,
                  const GemmArgs p) {
+    constexpr bool kLnIn = EPI == kEpiLnIn || EPI == kEpiLnInGelu || EPI == kEpiLnInScatter;
+    constexpr bool kGelu = EPI == kEpiGelu || EPI == kEpiLnInGelu;
+    constexpr bool kScatter = EPI == kEpiScatter || EPI == kEpiLnInScatter;
+    constexpr bool kRes = EPI == kEpiResStats;
     extern __shared__ uint8_t smem_raw[];
     Smem sm = carve(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -184,7 +171,6 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         sm.misc[0] = *reinterpret_cast<const volatile int *>(p.n_rows);
         sm.misc[1] = *reinterpret_cast<const volatile int *>(p.status);
         *sm.abort_flag = 0;
-        for (int i = 0; i < 8; ++i) sm.pair_flag[i] = 0;
         for (int i = 0; i < STAGES; ++i) {
             mbar_init(smem_u32(&sm.full[i]), 1);
             mbar_init(smem_u32(&sm.empty[i]), 1);
@@ -200,8 +186,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
-        if (EPI != kEpiScatter) prefetch_tmap(&tmOut);
-        if (EPI == kEpiLN) prefetch_tmap(&tmRes);
+        if (!kScatter) prefetch_tmap(&tmOut);
+        if (kRes) prefetch_tmap(&tmRes);
     }
     __syncthreads();
     // An earlier kernel of this forward failed, or the row count is out of range.
@@ -296,29 +282,35 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int half = ew >> 2;           // column half of the 256-wide tile
         const int r_local = quad * 32 + lane;
         const uint32_t stg = smem_u32(sm.stg + ew * STG_BYTES);
+        const uint32_t rstg = smem_u32(sm.rstg + ew * STG_BYTES);
         const uint32_t rbar = smem_u32(&sm.rbar[ew]);
+        const bool res_ln = kRes && p.res_stats != nullptr;
         uint32_t rph = 0;
         bool res_pending = false;
-        // residual chunk c (0..3) of unit u -> TMA load into this warp's staging tile
+        // residual chunk c (0..3) of unit u -> TMA load into this warp's residual tile
         auto res_issue = [&](int u, int c) {
             if (lane == 0) {
-                bulk_wait_read0();  // an earlier output store may still read the tile
                 mbar_arrive_expect_tx(rbar, STG_BYTES);
-                tma_load_2d(stg, &tmRes, rbar, (u % n_sub) * BN + half * 128 + c * 32,
+                tma_load_2d(rstg, &tmRes, rbar, (u % n_sub) * BN + half * 128 + c * 32,
                             (u / n_sub) * BM + quad * 32);
             }
             res_pending = true;
         };
-        int acc = 0, it = 0;
+        int acc = 0;
         bool ok = true;
-        if (EPI == kEpiLN && (int)blockIdx.x < units) res_issue(blockIdx.x, 0);
-        for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++it) {
+        if (kRes && (int)blockIdx.x < units) res_issue(blockIdx.x, 0);
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             const int m = u / n_sub, n = u % n_sub;
-            const int row = m * BM + r_local;
+            const int row = m * BM + r_local;  // < rows_cap
             const bool row_ok = row < n_rows;
             const int tile_row = m * BM + quad * 32;
             int dst = row;
-            if (EPI == kEpiScatter) dst = row_ok ? __ldg(p.row_dst + row) : -1;
+            if (kScatter) dst = row_ok ? __ldg(p.row_dst + row) : -1;
+            float mu = 0.f, rstd = 1.f;        // LayerNorm of the A operand
+            if (kLnIn) row_stats(p.in_stats + (size_t)row * LN_PARTS, p.eps, mu, rstd);
+            float rmu = 0.f, rrstd = 1.f;      // LayerNorm of the residual
+            if (res_ln) row_stats(p.res_stats + (size_t)row * LN_PARTS, p.eps, rmu, rrstd);
+            const float nmu = -rstd * mu, rnmu = -rrstd * rmu;
 
             const int ab = acc & 1;
             const uint32_t aph = (acc >> 1) & 1;
@@ -334,17 +326,17 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 uint32_t r[32];
                 tmem_ld32(tbase + c * 32, r);
                 uint4 rr[4];
-                if (EPI == kEpiLN) {
+                if (kRes) {
                     bool rok = mbar_wait(rbar, rph, sm.abort_flag);
                     rok = __all_sync(0xffffffffu, rok);
                     if (!rok) { ok = false; tmem_ld_wait(); break; }
                     rph ^= 1;
                     res_pending = false;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) rr[q] = ld_shared_v4(stg + stg_off(lane, q));
+                    for (int q = 0; q < 4; ++q) rr[q] = ld_shared_v4(rstg + stg_off(lane, q));
                 }
                 tmem_ld_wait();
-                if (EPI != kEpiLN && c == 3) {
+                if (c == 3) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_u32(&sm.tempty[ab]));
@@ -352,35 +344,60 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const int col0 = ncol0 + c * 32;
                 float v[32];
                 const float4 *bias4 = reinterpret_cast<const float4 *>(p.bias + col0);
+                if (kLnIn) {
+                    const float4 *s4 = reinterpret_cast<const float4 *>(p.fold_s + col0);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 bb = __ldg(bias4 + q);
-                    v[4 * q + 0] = __uint_as_float(r[4 * q + 0]) + bb.x;
-                    v[4 * q + 1] = __uint_as_float(r[4 * q + 1]) + bb.y;
-                    v[4 * q + 2] = __uint_as_float(r[4 * q + 2]) + bb.z;
-                    v[4 * q + 3] = __uint_as_float(r[4 * q + 3]) + bb.w;
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 bb = __ldg(bias4 + q), ss = __ldg(s4 + q);
+                        v[4 * q + 0] = fmaf(rstd, __uint_as_float(r[4 * q + 0]), fmaf(nmu, ss.x, bb.x));
+                        v[4 * q + 1] = fmaf(rstd, __uint_as_float(r[4 * q + 1]), fmaf(nmu, ss.y, bb.y));
+                        v[4 * q + 2] = fmaf(rstd, __uint_as_float(r[4 * q + 2]), fmaf(nmu, ss.z, bb.z));
+                        v[4 * q + 3] = fmaf(rstd, __uint_as_float(r[4 * q + 3]), fmaf(nmu, ss.w, bb.w));
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 bb = __ldg(bias4 + q);
+                        v[4 * q + 0] = __uint_as_float(r[4 * q + 0]) + bb.x;
+                        v[4 * q + 1] = __uint_as_float(r[4 * q + 1]) + bb.y;
+                        v[4 * q + 2] = __uint_as_float(r[4 * q + 2]) + bb.z;
+                        v[4 * q + 3] = __uint_as_float(r[4 * q + 3]) + bb.w;
+                    }
                 }
-                if (EPI == kEpiBias) {
-                    stage_and_store(stg, v, &tmOut, col0, tile_row, lane);
-                } else if (EPI == kEpiGelu) {
+                if (kGelu) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] = gelu_tanh_fast(v[j]);
-                    stage_and_store(stg, v, &tmOut, col0, tile_row, lane);
-                } else if (EPI == kEpiScatter) {
-                    if (dst >= 0) store_bf16x32(p.out + (size_t)dst * p.ld_out + col0, v);
-                } else {
+                }
+                if (kRes) {
+                    // residual: plain, or rebuilt LayerNorm output (its beta is folded into bias)
+                    float x[32];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         float2 f;
-                        f = unpack_bf16x2(rr[q].x); v[8 * q + 0] += f.x; v[8 * q + 1] += f.y;
-                        f = unpack_bf16x2(rr[q].y); v[8 * q + 2] += f.x; v[8 * q + 3] += f.y;
-                        f = unpack_bf16x2(rr[q].z); v[8 * q + 4] += f.x; v[8 * q + 5] += f.y;
-                        f = unpack_bf16x2(rr[q].w); v[8 * q + 6] += f.x; v[8 * q + 7] += f.y;
+                        f = unpack_bf16x2(rr[q].x); x[8 * q + 0] = f.x; x[8 * q + 1] = f.y;
+                        f = unpack_bf16x2(rr[q].y); x[8 * q + 2] = f.x; x[8 * q + 3] = f.y;
+                        f = unpack_bf16x2(rr[q].z); x[8 * q + 4] = f.x; x[8 * q + 5] = f.y;
+                        f = unpack_bf16x2(rr[q].w); x[8 * q + 6] = f.x; x[8 * q + 7] = f.y;
                     }
-                    // the staging tile has been read: prefetch the next residual chunk
+                    // the residual tile has been read: prefetch the next chunk
                     __syncwarp();
                     if (c < 3) res_issue(u, c + 1);
-                    // exact chunk statistics, merged into the running ones
+                    else if (u + (int)gridDim.x < units) res_issue(u + gridDim.x, 0);
+                    if (res_ln) {
+                        const float4 *rg4 = reinterpret_cast<const float4 *>(p.res_g + col0);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 g = __ldg(rg4 + q);
+                            v[4 * q + 0] += fmaf(rrstd, x[4 * q + 0], rnmu * g.x);
+                            v[4 * q + 1] += fmaf(rrstd, x[4 * q + 1], rnmu * g.y);
+                            v[4 * q + 2] += fmaf(rrstd, x[4 * q + 2], rnmu * g.z);
+                            v[4 * q + 3] += fmaf(rrstd, x[4 * q + 3], rnmu * g.w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] += x[j];
+                    }
+                    // exact chunk statistics of z, merged into the running ones
                     float cs = 0.f;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) cs += v[j];
@@ -390,86 +407,22 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     for (int j = 0; j < 32; ++j) { const float d = v[j] - cm; cq = fmaf(d, d, cq); }
                     if (c == 0) { mean = cm; m2 = cq; }
                     else chan_merge(mean, m2, 32.f * c, cm, cq, 32.f);
-                    // keep the fp32 pre-norm sum in TMEM, over the accumulator
+                    // output z * gamma of the LayerNorm that will normalize z
+                    const float4 *og4 = reinterpret_cast<const float4 *>(p.out_g + col0);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(v[j]);
-                    tmem_st32(tbase + c * 32, r);
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 g = __ldg(og4 + q);
+                        v[4 * q + 0] *= g.x; v[4 * q + 1] *= g.y; v[4 * q + 2] *= g.z; v[4 * q + 3] *= g.w;
+                    }
+                }
+                if (kScatter) {
+                    if (dst >= 0) store_bf16x32(p.out + (size_t)dst * p.ld_out + col0, v);
+                } else {
+                    stage_and_store(stg, v, &tmOut, col0, tile_row, lane);
                 }
             }
             if (!ok) break;
-
-            if (EPI == kEpiLN) {
-                tmem_st_wait();
-                // 1. the two column halves of each row (partner warp = other half)
-                float2 *st = sm.stats + (size_t)((it & 1) * 2 + half) * BM;
-                st[r_local] = make_float2(mean, m2);
-                __syncwarp();
-                __threadfence_block();
-                if (lane == 0) sm.pair_flag[quad * 2 + half] = it + 1;
-                if (!wait_flag(&sm.pair_flag[quad * 2 + (half ^ 1)], it + 1, sm.abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                const float2 o = sm.stats[(size_t)((it & 1) * 2 + (half ^ 1)) * BM + r_local];
-                // the row over this tile's 256 columns (same result in both halves:
-                // merge in column order)
-                float tmean = half == 0 ? mean : o.x, tm2 = half == 0 ? m2 : o.y;
-                chan_merge(tmean, tm2, 128.f, half == 0 ? o.x : mean, half == 0 ? o.y : m2, 128.f);
-                // 2. publish, then gather the other tiles of the row block
-                float2 *gst = p.ln_stats + (size_t)row * n_sub;
-                int *flags = p.ln_flags + ((size_t)m * 4 + quad) * n_sub;
-                if (half == 0) {
-                    gst[n] = make_float2(tmean, tm2);
-                    __syncwarp();
-                    if (lane == 0) {
-                        __threadfence();
-                        st_release_gpu(flags + n, p.epoch);
-                    }
-                }
-                float rmean = 0.f, rm2 = 0.f, rcnt = 0.f;
-                for (int k = 0; k < n_sub; ++k) {
-                    float2 pk;
-                    if (k == n) {
-                        pk = make_float2(tmean, tm2);
-                    } else {
-                        if (!wait_epoch(flags + k, p.epoch, sm.abort_flag)) { ok = false; break; }
-                        pk = __ldcg(gst + k);
-                    }
-                    if (k == 0) { rmean = pk.x; rm2 = pk.y; }
-                    else chan_merge(rmean, rm2, rcnt, pk.x, pk.y, (float)BN);
-                    rcnt += (float)BN;
-                }
-                if (!ok) break;
-                const float mu = rmean;
-                const float rstd = rsqrtf(rm2 / rcnt + p.eps);
-                // 3. normalize this warp's 128 columns from TMEM
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tbase + c * 32, r);
-                    tmem_ld_wait();
-                    if (c == 3) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(smem_u32(&sm.tempty[ab]));
-                    }
-                    const int col0 = ncol0 + c * 32;
-                    float v[32];
-                    const float4 *g4 = reinterpret_cast<const float4 *>(p.ln_g + col0);
-                    const float4 *b4 = reinterpret_cast<const float4 *>(p.ln_b + col0);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 g = __ldg(g4 + q), bb = __ldg(b4 + q);
-                        v[4 * q + 0] = fmaf((__uint_as_float(r[4 * q + 0]) - mu) * rstd, g.x, bb.x);
-                        v[4 * q + 1] = fmaf((__uint_as_float(r[4 * q + 1]) - mu) * rstd, g.y, bb.y);
-                        v[4 * q + 2] = fmaf((__uint_as_float(r[4 * q + 2]) - mu) * rstd, g.z, bb.z);
-                        v[4 * q + 3] = fmaf((__uint_as_float(r[4 * q + 3]) - mu) * rstd, g.w, bb.w);
-                    }
-                    stage_and_store(stg, v, &tmOut, col0, tile_row, lane);
-                }
-                // first residual chunk of this CTA's next unit
-                if (u + (int)gridDim.x < units) res_issue(u + gridDim.x, 0);
-            }
+            if (kRes) p.out_stats[(size_t)row * LN_PARTS + n * 2 + half] = make_float2(mean, m2);
             ++acc;
         }
         // outstanding copies finish before the CTA's shared memory goes away
@@ -504,20 +457,6 @@ static cudaError_t launch_one(const CUtensorMap &tmA, const CUtensorMap &tmB, co
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    if (EPI == kEpiLN) {
-        // CTAs of a row block wait for one another: all must be resident.
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(grid);
-        cfg.blockDim = dim3(THREADS);
-        cfg.dynamicSmemBytes = SMEM_BYTES;
-        cfg.stream = s;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeCooperative;
-        attr[0].val.cooperative = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, gemm_bf16_kernel<EPI>, tmA, tmB, tmOut, tmRes, a);
-    }
     gemm_bf16_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmB, tmOut, tmRes, a);
     return cudaGetLastError();
 }
@@ -527,8 +466,11 @@ cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB,
     switch (epi) {
         case kEpiBias: return launch_one<kEpiBias>(tmA, tmB, tmOut, tmRes, a, grid, s);
         case kEpiGelu: return launch_one<kEpiGelu>(tmA, tmB, tmOut, tmRes, a, grid, s);
-        case kEpiLN: return launch_one<kEpiLN>(tmA, tmB, tmOut, tmRes, a, grid, s);
+        case kEpiResStats: return launch_one<kEpiResStats>(tmA, tmB, tmOut, tmRes, a, grid, s);
         case kEpiScatter: return launch_one<kEpiScatter>(tmA, tmB, tmOut, tmRes, a, grid, s);
+        case kEpiLnIn: return launch_one<kEpiLnIn>(tmA, tmB, tmOut, tmRes, a, grid, s);
+        case kEpiLnInGelu: return launch_one<kEpiLnInGelu>(tmA, tmB, tmOut, tmRes, a, grid, s);
+        case kEpiLnInScatter: return launch_one<kEpiLnInScatter>(tmA, tmB, tmOut, tmRes, a, grid, s);
     }
     return cudaErrorInvalidValue;
 }

@@ -15,7 +15,21 @@ constexpr int kQKV = 3 * kHidden;
 constexpr int kMaxPos = 512;
 
 // ------------------------------------------------------------- tcgen05 GEMM --
-enum GemmEpi : int { kEpiBias = 0, kEpiGelu = 1, kEpiLN = 2, kEpiScatter = 3 };
+// Epilogues.  "LN input" operands hold z * gamma of a row z that a LayerNorm
+// (width 768) still has to normalize; its per-row statistics come as six
+// partial (mean, M2) pairs over 128-column slices, [rows][6] float2.  Since
+// LN(z) W^T = rstd * (z*gamma) W^T - rstd * mu * (W gamma) + W beta, a GEMM on
+// z*gamma applies the LayerNorm in its epilogue with fold_s = W gamma and
+// bias = W beta + b.
+enum GemmEpi : int {
+    kEpiBias = 0,         // Y = acc + bias
+    kEpiGelu = 1,         // Y = GELU_tanh(acc + bias)
+    kEpiResStats = 2,     // z = acc + bias + residual; Y = z * out_g; out_stats = partial stats of z
+    kEpiScatter = 3,      // Y[row_dst[r]] = acc + bias (row_dst[r] < 0: skipped)
+    kEpiLnIn = 4,         // Y = rstd * acc - rstd * mu * fold_s + bias
+    kEpiLnInGelu = 5,     // Y = GELU_tanh(rstd * acc - rstd * mu * fold_s + bias)
+    kEpiLnInScatter = 6,  // Y[row_dst[r]] = rstd * acc - rstd * mu * fold_s + bias
+};
 
 namespace gemm {
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
@@ -24,9 +38,11 @@ constexpr int B_BYTES = BN * BK * 2;
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 32 * (2 + EPI_WARPS);
 constexpr int TMEM_COLS = 512;
-constexpr int LN_N = 768;  // the LayerNorm epilogue normalizes rows of this width
-constexpr int STG_BYTES = 32 * 32 * 2;  // one 32x32 bf16 epilogue staging tile per epilogue warp
-constexpr int SMEM_BYTES = 2048 + STAGES * (A_BYTES + B_BYTES) + EPI_WARPS * STG_BYTES + 1024 + 2 * 2 * BM * 8;
+constexpr int LN_N = 768;     // LayerNorm row width
+constexpr int LN_PARTS = 6;   // partial statistics per row (128 columns each)
+constexpr int STG_BYTES = 32 * 32 * 2;  // one 32x32 bf16 staging tile
+// stages + per-warp output staging + per-warp residual staging + control, 1 KiB aligned
+constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES) + 2 * EPI_WARPS * STG_BYTES + 1024;
 }  // namespace gemm
 
 struct GemmArgs {
@@ -34,15 +50,19 @@ struct GemmArgs {
     int rows_cap;              // rows of the A / out buffers (multiple of 128)
     const int *n_rows;         // device: rows that hold data (<= rows_cap)
     const float *bias;         // [N]
-    const bf16 *resid;         // LN: [rows, N]
-    int ld_resid;
-    const float *ln_g, *ln_b;  // LN: [N]
+    // kEpiLnIn*: statistics of the LayerNorm input held (times gamma) in A
+    const float2 *in_stats;    // [rows][6]
+    const float *fold_s;       // [N] = W gamma
+    // kEpiResStats: residual tile (tmRes) is plain (res_stats == nullptr) or a
+    // LayerNorm input z*gamma with statistics res_stats, rebuilt as
+    // rstd * r - rstd * mu * res_g + (its beta, folded into bias)
+    const float2 *res_stats;   // [rows][6] or nullptr
+    const float *res_g;        // [N]
+    const float *out_g;        // [N]: Y = z * out_g
+    float2 *out_stats;         // [rows][6]: partial (mean, M2) of z per 128 columns
     float eps;
-    bf16 *out;                 // [rows, ld_out] (scatter: destination rows)
+    bf16 *out;                 // scatter epilogues: [*, ld_out] destination rows
     int ld_out;
-    float2 *ln_stats;          // LN: per-row (mean, M2) of each 256-column tile, [rows_cap][N/256]
-    int *ln_flags;             // LN: per (row block, lane quadrant, column tile) epoch flags
-    int epoch;                 // LN: value this launch writes to ln_flags (> every earlier one)
     const int *row_dst;        // scatter: destination row or -1
     int *status;               // device status word
 };
@@ -57,14 +77,15 @@ int make_tmap_bf16_tile32(CUtensorMap *tm, const void *base, uint64_t rows, uint
 
 // Grid the GEMM uses for this many rows (persistent: <= number of SMs).
 int gemm_grid(int epi, int rows_cap, int N, int num_sms);
-// Cross-tile LayerNorm buffers for rows_cap rows of width LN_N.
-inline size_t gemm_ln_stats_count(int rows_cap) { return (size_t)rows_cap * (gemm::LN_N / gemm::BN); }
-inline size_t gemm_ln_flags_count(int rows_cap) {
-    return (size_t)((rows_cap + gemm::BM - 1) / gemm::BM) * 4 * (gemm::LN_N / gemm::BN);
+
+// The epilogue reads its per-column vectors as float4: each must be 16-byte aligned.
+inline bool gemm_vectors_aligned(const GemmArgs &a) {
+    auto ok = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+    return ok(a.bias) && ok(a.fold_s) && ok(a.res_g) && ok(a.out_g);
 }
 
-// tmOut: tile32 map of the output (unused by the scatter epilogue); tmRes: tile32
-// map of the residual (LayerNorm epilogue only; pass any valid map otherwise).
+// tmOut: tile32 map of the output (unused by the scatter epilogues); tmRes: tile32
+// map of the residual (kEpiResStats only; pass any valid map otherwise).
 cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
                         const CUtensorMap &tmRes, const GemmArgs &args, int grid, cudaStream_t s);
 
@@ -112,6 +133,19 @@ cudaError_t launch_zero_pad(void *out, int B, int T, int D, int elem_bytes, cons
 cudaError_t launch_scatter_rows(const void *X, void *out, int D, int elem_bytes, int rows_cap,
                                 const int *n_rows, const int *row_dst, const int *status,
                                 cudaStream_t s);
+
+// Folded LayerNorm constants of a linear layer W [N, K] (bf16) that consumes
+// LN(z) = (z - mu) * rstd * gamma + beta:  s = W gamma,  c = W beta + b.
+cudaError_t launch_fold_ln(const bf16 *W, int N, int K, const float *gamma, const float *beta,
+                           const float *b, float *s_out, float *c_out, cudaStream_t s);
+// out[row_dst[r]] = LN(z) = rstd * zg - rstd * mu * gamma + beta for r < n_rows
+// (zg = z * gamma, [rows, 768] bf16; stats [rows][6]); row_dst == nullptr: out[r].
+// out_rows bounds row_dst (a larger destination is recorded as ALBERT_ERR_SHAPE).
+cudaError_t launch_ln_rows(const bf16 *zg, const float2 *stats, const float *gamma, const float *beta,
+                           float eps, bf16 *out, const int *row_dst, int out_rows, int rows_cap,
+                           const int *n_rows, int *status, cudaStream_t s);
+// out[i] = a[i] + b[i]
+cudaError_t launch_vec_add(const float *a, const float *b, float *out, int n, cudaStream_t s);
 
 // fp32 -> bf16 conversion of a parameter block.
 cudaError_t launch_f32_to_bf16(const float *src, bf16 *dst, size_t n, cudaStream_t s);
