@@ -200,6 +200,37 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------- multi-rank ----
+
+def rank_batch_seed(base_seed: int, rank: int) -> int:
+    """Each rank encodes its own batch of the workload (weak scaling)."""
+    return base_seed + 1000 * rank
+
+
+def max_over_ranks(x: float, dist=None, device="cpu") -> float:
+    """Max of a per-rank float over all ranks (the job's time is its slowest rank's)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, dist=None, device="cpu") -> float:
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def job_throughput(local_tokens: float, local_ms: float, dist=None, device="cpu") -> float:
+    """All ranks' tokens divided by the slowest rank's time (tokens/s)."""
+    return sum_over_ranks(local_tokens, dist, device) / (max_over_ranks(local_ms, dist, device) / 1000.0)
+
+
 # ---------------------------------------------------------------- GPU arm ----
 
 def run_gpu(args):
@@ -226,24 +257,14 @@ def run_gpu(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    def sum_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        return float(t.item())
+    dev = torch.device("cuda", local)
+    max_r = lambda x: max_over_ranks(x, dist, dev)
+    sum_r = lambda x: sum_over_ranks(x, dist, dev)
 
     arch = synth.ARCH
     wl = synth.WORKLOADS[args.workload]
     w = synth.make_weights(seed=1234, bf16=True)
-    ids, mask, L = synth.make_batch(wl, seed=wl.seed + 1000 * rank)
+    ids, mask, L = synth.make_batch(wl, seed=rank_batch_seed(wl.seed, rank))
     n_tok = int(L.sum())
     ids_d = torch.as_tensor(ids).cuda()
     mask_d = torch.as_tensor(mask).cuda()
@@ -294,8 +315,8 @@ def run_gpu(args):
     dom = enc.profile_read()[dominant]
     enc.profile([])
     enc.profile_reset()
-    total_ms = max_over_ranks(sum(step_ms))
-    tokens_all = sum_over_ranks(float(n_tok * args.steps))
+    total_ms = max_r(sum(step_ms))
+    tokens_all = sum_r(float(n_tok * args.steps))
     value = tokens_all / (total_ms / 1000.0)
     ms_per_step = total_ms / args.steps
 
@@ -328,8 +349,8 @@ def run_gpu(args):
             raise SystemExit(f"forward_host status {rc}")
     e_e.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e_s.elapsed_time(e_e))
-    e2e_value = sum_over_ranks(float(n_tok * n_e2e)) / (e2e_ms / 1000.0)
+    e2e_ms = max_r(e_s.elapsed_time(e_e))
+    e2e_value = sum_r(float(n_tok * n_e2e)) / (e2e_ms / 1000.0)
 
     peaks, peaks_src = load_peaks()
     peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
