@@ -15,10 +15,11 @@
 //                 of one tile overlaps the main loop of the next;
 //   warps 2..9  : epilogue, 2 warps per TMEM lane quadrant (column halves);
 //                 tcgen05.ld -> epilogue math -> bf16 32x32 tile in a swizzled
-//                 shared staging buffer -> TMA bulk tensor store (coalesced,
-//                 asynchronous; one-row-per-lane global stores would contend
-//                 with the tensor core's shared-memory operand reads in the
-//                 unified L1/shared array).
+//                 shared staging buffer (two, used alternately, when the
+//                 epilogue has no residual) -> TMA bulk tensor store
+//                 (coalesced, asynchronous; one-row-per-lane global stores
+//                 would contend with the tensor core's shared-memory operand
+//                 reads in the unified L1/shared array).
 //
 // Post-LN LayerNorms (steps 5 and 6) are deferred to the consumers of their
 // output, so every epilogue is a single pass with no cross-CTA dependency:
@@ -106,10 +107,15 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
 
 // Write this lane's 32 values (its row of the warp's 32x32 tile) as bf16 into
 // the staging tile, then one lane stores the tile to global memory by TMA.
-// The previous store from the same tile must have finished reading it.
+// The previous store from the same tile must have finished reading it: with
+// two tiles used alternately (double_buffered) that store is the one before
+// the most recent.
 __device__ __forceinline__ void stage_and_store(uint32_t stg, const float (&v)[32], const CUtensorMap *tm,
-                                                int x, int y, int lane) {
-    if (lane == 0) bulk_wait_read0();
+                                                int x, int y, int lane, bool double_buffered) {
+    if (lane == 0) {
+        if (double_buffered) bulk_wait_read1();
+        else bulk_wait_read0();
+    }
     __syncwarp();
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -417,8 +423,11 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 }
                 if (kScatter) {
                     if (dst >= 0) store_bf16x32(p.out + (size_t)dst * p.ld_out + col0, v);
+                } else if (kRes) {
+                    stage_and_store(stg, v, &tmOut, col0, tile_row, lane, false);
                 } else {
-                    stage_and_store(stg, v, &tmOut, col0, tile_row, lane);
+                    // the residual tile is free here: alternate the two staging tiles
+                    stage_and_store((c & 1) ? rstg : stg, v, &tmOut, col0, tile_row, lane, true);
                 }
             }
             if (!ok) break;
