@@ -90,7 +90,7 @@ def test_gemm_scatter_rows():
     assert np.all(got[untouched] == 7.0)
 
 
-def _attention_case(lengths, fp32=False, seed=0):
+def _attention_case(lengths, fp32=False, seed=0, legacy=False):
     r = np.random.default_rng(seed)
     n = int(sum(lengths))
     qkv = r.normal(0, 1.0, (n, 3 * 768))
@@ -101,7 +101,8 @@ def _attention_case(lengths, fp32=False, seed=0):
     else:
         q_dev = _bf16_t(qkv)
         ctx = torch.empty(n, 768, device="cuda", dtype=torch.bfloat16)
-    assert tea.test_attention(q_dev, torch.tensor(cu, device="cuda"), max(lengths), ctx, fp32=fp32) == 0
+    assert tea.test_attention(q_dev, torch.tensor(cu, device="cuda"), max(lengths), ctx, fp32=fp32,
+                              legacy=legacy) == 0
     q64 = _np(q_dev)
     got = _np(ctx)
     for s, L in enumerate(lengths):
@@ -118,6 +119,15 @@ def test_attention_bf16_ragged_lengths():
     _attention_case([1, 2, 7, 16, 63, 64, 65, 100, 127, 128, 129, 200])
 
 
+def test_attention_tcgen05_short_sequences():
+    """max_len <= 128 runs the tcgen05 kernel: every length 1..128 class."""
+    _attention_case([1, 2, 3, 15, 16, 17, 31, 32, 33, 63, 64, 65, 96, 127, 128, 40, 5], seed=7)
+
+
+def test_attention_mma_sync_kernel_short_sequences():
+    _attention_case([1, 16, 33, 64, 100, 128], seed=8, legacy=True)
+
+
 def test_attention_bf16_long_sequences():
     _attention_case([256, 300, 511, 512], seed=1)
 
@@ -126,8 +136,8 @@ def test_attention_fp32_ragged_lengths():
     _attention_case([1, 5, 36, 40, 129], fp32=True, seed=2)
 
 
-def test_attention_identical_keys_give_mean_of_values():
-    L = 50
+@pytest.mark.parametrize("L", [50, 128, 300])
+def test_attention_identical_keys_give_mean_of_values(L):
     r = np.random.default_rng(3)
     qkv = r.normal(0, 1, (L, 3 * 768))
     qkv[:, 768:1536] = qkv[0, 768:1536]

@@ -248,11 +248,13 @@ def test_gemm(A, W, bias, Y, epi: int, R=None, ln_g=None, ln_b=None, eps: float 
                                   _stream_ptr(stream))
 
 
-def test_attention(qkv, cu_seqlens, max_len: int, ctx, fp32: bool = False, stream=None) -> int:
-    """Run the attention kernel alone (single-kernel parity tests)."""
+def test_attention(qkv, cu_seqlens, max_len: int, ctx, fp32: bool = False, legacy: bool = False,
+                   stream=None) -> int:
+    """Run the attention kernel alone (single-kernel parity tests); legacy forces
+    the mma.sync kernel for bf16."""
+    mode = ALBERT_FP32 if fp32 else (2 if legacy else ALBERT_BF16)
     return lib().albert_test_attention(_ptr(qkv), _ptr(cu_seqlens), cu_seqlens.numel() - 1,
-                                       int(max_len), _ptr(ctx), ALBERT_FP32 if fp32 else ALBERT_BF16,
-                                       _stream_ptr(stream))
+                                       int(max_len), _ptr(ctx), mode, _stream_ptr(stream))
 
 
 def gemm_residual_ln_noalloc(A, W, bias, R, ln_g, ln_b, Y, eps: float = 1e-12, stream=None) -> int:

@@ -68,7 +68,7 @@ struct albert_handle {
     void *st_out = nullptr;
 
     // TMA descriptors (bf16)
-    CUtensorMap tm_E, tm_X, tm_C, tm_X1, tm_H, tm_Z;
+    CUtensorMap tm_E, tm_X, tm_C, tm_X1, tm_H, tm_Z, tm_QKV, tm_QKV64;
     CUtensorMap tm_win, tm_wqkv, tm_wo, tm_w1, tm_w2, tm_wout;
     CUtensorMap t32_X, t32_QKV, t32_X1, t32_H, t32_Z;  // 32x32-box maps: epilogue stores / residual loads
 
@@ -257,8 +257,13 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
                 rc = gemm_bf16(L, kProfGemmQKV, kEpiLnIn, h->tm_Z, h->tm_wqkv, h->t32_QKV, h->t32_QKV, a);
             }
             if (rc) return rc;
-            LAUNCH(L, kProfAttention, launch_attention_bf16(static_cast<bf16 *>(h->QKV), static_cast<bf16 *>(h->C), h->seq_start,
-                                                           h->seq_len, nseq, max_len, h->status, L.s));
+            if (max_len <= kAttnTcMaxLen) {
+                LAUNCH(L, kProfAttention, launch_attention_tc(h->tm_QKV, h->tm_QKV64, static_cast<bf16 *>(h->C), h->seq_start,
+                                                             h->seq_len, nseq, h->status, h->num_sms, L.s));
+            } else {
+                LAUNCH(L, kProfAttention, launch_attention_bf16(static_cast<bf16 *>(h->QKV), static_cast<bf16 *>(h->C),
+                                                               h->seq_start, h->seq_len, nseq, max_len, h->status, L.s));
+            }
             // z1 = C Wo^T + bo + layer input -> X1 = z1 * gamma1, st1
             GemmArgs a = gemm_args(h, kHidden, kHidden, l == 0 ? h->bo : h->bias_o2, nullptr, 0);
             a.res_stats = l == 0 ? nullptr : h->st2;
@@ -458,6 +463,7 @@ int create_impl(albert_handle *h, const albert_weights *w) {
         if (make_tmap_bf16(&h->tm_E, h->E, R, kEmb, gemm::BM) || make_tmap_bf16(&h->tm_X, h->X, R, kHidden, gemm::BM) ||
             make_tmap_bf16(&h->tm_C, h->C, R, kHidden, gemm::BM) || make_tmap_bf16(&h->tm_X1, h->X1, R, kHidden, gemm::BM) ||
             make_tmap_bf16(&h->tm_H, h->H, R, kFfn, gemm::BM) || make_tmap_bf16(&h->tm_Z, h->Z, R, kHidden, gemm::BM) ||
+            make_tmap_bf16(&h->tm_QKV, h->QKV, R, kQKV, 128) || make_tmap_bf16(&h->tm_QKV64, h->QKV, R, kQKV, 64) ||
             make_tmap_bf16(&h->tm_win, h->w_in, kHidden, kEmb, gemm::BN) ||
             make_tmap_bf16(&h->tm_wqkv, h->wqkv, kQKV, kHidden, gemm::BN) ||
             make_tmap_bf16(&h->tm_wo, h->wo, kHidden, kHidden, gemm::BN) ||
@@ -652,18 +658,31 @@ int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, 
                           void *stream) {
     if (!qkv || !cu_seqlens || !ctx) return ALBERT_ERR_NULL;
     if (nseq < 1 || max_len < 1 || max_len > kMaxPos) return ALBERT_ERR_SHAPE;
+    if (dtype < 0 || dtype > 2) return ALBERT_ERR_CONFIG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int dev = 0, sms = 0;
+    TRY(cudaGetDevice(&dev));
+    TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    int n_tok = 0;
+    TRY(cudaMemcpy(&n_tok, cu_seqlens + nseq, sizeof(int), cudaMemcpyDeviceToHost));
+    if (n_tok < 1) return ALBERT_ERR_SHAPE;
     int *ints = nullptr;
     TRY(cudaMalloc(&ints, (2 * (size_t)nseq + 4) * sizeof(int)));
     int *seq_start = ints, *seq_len = ints + nseq + 1, *n_rows = seq_len + nseq + 1, *status = n_rows + 1;
     cudaError_t e = launch_prep_varlen(cu_seqlens, nseq, max_len, 1 << 30, seq_start, seq_len, n_rows, status, s);
     if (e == cudaSuccess) {
-        if (dtype == ALBERT_FP32)
+        if (dtype == ALBERT_FP32) {
             e = launch_attention_f32(static_cast<const float *>(qkv), static_cast<float *>(ctx), seq_start, seq_len, nseq,
                                      max_len, status, s);
-        else
+        } else if (dtype == ALBERT_BF16 && max_len <= kAttnTcMaxLen) {
+            CUtensorMap tm, tm64;
+            if (make_tmap_bf16(&tm, qkv, (uint64_t)n_tok, kQKV, 128) || make_tmap_bf16(&tm64, qkv, (uint64_t)n_tok, kQKV, 64))
+                e = cudaErrorInvalidValue;
+            else e = launch_attention_tc(tm, tm64, static_cast<bf16 *>(ctx), seq_start, seq_len, nseq, status, sms, s);
+        } else {
             e = launch_attention_bf16(static_cast<const bf16 *>(qkv), static_cast<bf16 *>(ctx), seq_start, seq_len, nseq,
                                       max_len, status, s);
+        }
     }
     int st = 0;
     if (e == cudaSuccess) e = cudaMemcpyAsync(&st, status, sizeof(int), cudaMemcpyDeviceToHost, s);

@@ -1,0 +1,320 @@
+// attention_tc.cu -- masked bidirectional attention on the 5th-generation tensor
+// cores (tcgen05) for sequences of at most 128 tokens.
+//
+// Per sequence b and head h ("ALBERT: How Kokoro's Phoneme Encoder Works",
+// section "Inside One Real ALBERT Layer", step 4; "How Kokoro TTS Works and
+// Where CKE Stands", section "What ALBERT does here"):
+//     C_h = softmax(Q_h K_h^T / sqrt(64) + mask) V_h,
+// key u of sequence b takes part iff u < L_b, every query sees both sides.
+//
+// One work item = (sequence, head), all L_b <= 128 queries and keys at once:
+//   warp 0      : TMA producer: the head's Q, K and V tiles (128 or 64 rows x
+//                 64, 128-byte swizzle) from the packed [rows, 3*768] buffer
+//                 into a ring of four shared stages;
+//   warp 1      : tcgen05.mma issuer, an event loop that issues whichever is
+//                 ready: S = Q K^T (M=128, N=128 or 64, K=64) into TMEM, or
+//                 O = P V (M=128, N=64, K = L rounded up to 16) with P read from
+//                 TMEM and V from shared memory as an MN-major operand;
+//   warps 2..9  : two groups of 4 warps, one per TMEM buffer: each thread owns
+//                 one query row, reads its scores from TMEM, applies the mask and
+//                 a max-subtracted softmax in registers (no cross-thread
+//                 reductions), writes P as packed bf16 back into TMEM over the
+//                 scores it has read, then scales its row of O by 1/sum and
+//                 stores it.
+// Scores/P and O are double-buffered in TMEM, loads run up to four items ahead,
+// so item i's softmax overlaps item i+1's products and later items' loads.
+// Every wait is bounded (%globaltimer).
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace albert {
+namespace {
+
+constexpr int TROWS = 128;                     // query rows / keys per item
+constexpr int TILE = TROWS * 128;              // 128 rows x 64 bf16 = 16 KB
+constexpr int STAGE = 3 * TILE;                // Q, K, V
+constexpr int NSTAGE = 4;
+constexpr int ATC_THREADS = 32 * 10;
+constexpr int ATC_SMEM = 1024 + NSTAGE * STAGE + 512;
+constexpr uint32_t TM_S = 0, TM_O = 256;       // TMEM columns: S/P[s] at 128 s, O[s] at 256 + 64 s
+
+struct AttSmem {
+    uint8_t *stage;
+    uint64_t *ld_full, *ld_empty;              // [NSTAGE]
+    uint64_t *s_full, *s_empty, *p_full, *o_full, *o_empty;  // [2]
+    uint64_t *drain;
+    uint32_t *tmem_slot;
+    volatile int *abort_flag;
+    int *misc;
+};
+
+__device__ __forceinline__ AttSmem att_carve(uint8_t *raw) {
+    AttSmem s;
+    uint8_t *p = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    s.stage = p;
+    uint64_t *b = reinterpret_cast<uint64_t *>(p + NSTAGE * STAGE);
+    s.ld_full = b;
+    s.ld_empty = b + NSTAGE;
+    s.s_full = b + 2 * NSTAGE;
+    s.s_empty = s.s_full + 2;
+    s.p_full = s.s_full + 4;
+    s.o_full = s.s_full + 6;
+    s.o_empty = s.s_full + 8;
+    s.drain = s.s_full + 10;
+    uint32_t *u = reinterpret_cast<uint32_t *>(s.drain + 1);
+    s.tmem_slot = u;
+    s.abort_flag = reinterpret_cast<volatile int *>(u + 1);
+    s.misc = reinterpret_cast<int *>(u + 2);
+    return s;
+}
+
+__global__ void __launch_bounds__(ATC_THREADS, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmQKV64,
+               bf16 *__restrict__ ctx, const int *__restrict__ seq_start, const int *__restrict__ seq_len, int nseq,
+               int *status) {
+    extern __shared__ uint8_t smem_raw[];
+    AttSmem sm = att_carve(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        sm.misc[0] = *reinterpret_cast<const volatile int *>(status);
+        *sm.abort_flag = 0;
+        for (int i = 0; i < NSTAGE; ++i) {
+            mbar_init(smem_u32(&sm.ld_full[i]), 1);
+            mbar_init(smem_u32(&sm.ld_empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&sm.s_full[i]), 1);
+            mbar_init(smem_u32(&sm.s_empty[i]), 1);
+            mbar_init(smem_u32(&sm.p_full[i]), 4);
+            mbar_init(smem_u32(&sm.o_full[i]), 1);
+            mbar_init(smem_u32(&sm.o_empty[i]), 4);
+        }
+        mbar_init(smem_u32(sm.drain), 1);
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmQKV);
+        prefetch_tmap(&tmQKV64);
+    }
+    __syncthreads();
+    if (sm.misc[0] != 0) return;  // an earlier kernel of this forward failed
+    if (warp == 1) {
+        tmem_alloc(smem_u32(sm.tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *sm.tmem_slot;
+    const int total = nseq * kHeads;  // item id = b * 12 + h
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer --
+        if (lane == 0) {
+            int i = 0, issued = 0;
+            bool ok = true;
+            for (int id = blockIdx.x; id < total && ok; id += gridDim.x, ++i) {
+                const int st = i % NSTAGE;
+                const uint32_t ph = (i / NSTAGE) & 1;
+                if (!mbar_wait(smem_u32(&sm.ld_empty[st]), ph ^ 1, sm.abort_flag)) { ok = false; break; }
+                const int b = id / kHeads, h = id % kHeads;
+                const int start = __ldg(seq_start + b);
+                // sequences of at most 64 tokens move 64-row tiles
+                const bool short_seq = __ldg(seq_len + b) <= 64;
+                const CUtensorMap *tm = short_seq ? &tmQKV64 : &tmQKV;
+                const uint32_t dst = smem_u32(sm.stage + st * STAGE);
+                const uint32_t fb = smem_u32(&sm.ld_full[st]);
+                mbar_arrive_expect_tx(fb, short_seq ? 3 * TILE / 2 : 3 * TILE);
+                tma_load_2d(dst, tm, fb, h * kHeadDim, start);
+                tma_load_2d(dst + TILE, tm, fb, kHidden + h * kHeadDim, start);
+                tma_load_2d(dst + 2 * TILE, tm, fb, 2 * kHidden + h * kHeadDim, start);
+                ++issued;
+            }
+            if (!ok) {
+                for (int k = 0; k < NSTAGE && k < issued; ++k) {
+                    const int j = issued - 1 - k;
+                    mbar_wait_drain(smem_u32(&sm.ld_full[j % NSTAGE]), (j / NSTAGE) & 1);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // -------------------------------------------------------- MMA issuer --
+        // Issues S(next) and O(next) products as soon as each is ready, so an
+        // output product never queues behind the next item's loads.
+        if (lane == 0) {
+            const uint32_t idesc_s128 = idesc_bf16_f32(TROWS, TROWS);
+            const uint32_t idesc_s64 = idesc_bf16_f32(TROWS, 64);
+            const uint32_t idesc_o = idesc_bf16_f32(TROWS, kHeadDim) | (1u << 16);  // B (= V) MN-major
+            int n_items = 0;
+            for (int id = blockIdx.x; id < total; id += gridDim.x) ++n_items;
+            int ns = 0, no = 0;  // next S product, next O product
+            unsigned long long t_idle = 0;
+            while (no < n_items) {
+                bool progress = false;
+                if (no < ns) {
+                    const int tb = no & 1, st = no % NSTAGE;
+                    const uint32_t ph = (no >> 1) & 1;
+                    if (mbar_try_wait(smem_u32(&sm.p_full[tb]), ph) && mbar_try_wait(smem_u32(&sm.o_empty[tb]), ph ^ 1)) {
+                        tc_fence_after();
+                        const int L = __ldg(seq_len + (blockIdx.x + no * gridDim.x) / kHeads);
+                        const int ksteps = (L + 15) >> 4;
+                        const uint32_t vbase = smem_u32(sm.stage + st * STAGE + 2 * TILE);
+                        for (int kk = 0; kk < ksteps; ++kk) {
+                            // P: 16 keys = 8 packed TMEM columns; V: 16 keys = 16 rows of 128 B
+                            umma_bf16_ts(tmem_base + TM_O + tb * kHeadDim, tmem_base + TM_S + tb * TROWS + kk * 8,
+                                         sw128_kmajor_desc(vbase + kk * 2048), idesc_o, kk != 0);
+                        }
+                        umma_commit(smem_u32(&sm.o_full[tb]));
+                        umma_commit(smem_u32(&sm.s_empty[tb]));   // P consumed: S buffer free
+                        umma_commit(smem_u32(&sm.ld_empty[st]));  // Q, K, V consumed: stage free
+                        ++no;
+                        progress = true;
+                    }
+                }
+                if (ns < n_items && ns < no + 2) {
+                    const int tb = ns & 1, st = ns % NSTAGE;
+                    const uint32_t ph = (ns >> 1) & 1;
+                    if (mbar_try_wait(smem_u32(&sm.ld_full[st]), (ns / NSTAGE) & 1) &&
+                        mbar_try_wait(smem_u32(&sm.s_empty[tb]), ph ^ 1)) {
+                        tc_fence_after();
+                        const int L = __ldg(seq_len + (blockIdx.x + ns * gridDim.x) / kHeads);
+                        const uint32_t q = smem_u32(sm.stage + st * STAGE), k = q + TILE;
+#pragma unroll
+                        for (int kk = 0; kk < kHeadDim / 16; ++kk)
+                            umma_bf16(tmem_base + TM_S + tb * TROWS, sw128_kmajor_desc(q + kk * 32),
+                                      sw128_kmajor_desc(k + kk * 32), L <= 64 ? idesc_s64 : idesc_s128, kk != 0);
+                        umma_commit(smem_u32(&sm.s_full[tb]));
+                        ++ns;
+                        progress = true;
+                    }
+                }
+                if (progress) {
+                    t_idle = 0;
+                } else {
+                    if (*sm.abort_flag) break;
+                    const unsigned long long now = globaltimer_ns();
+                    if (t_idle == 0) t_idle = now;
+                    else if (now - t_idle > kWaitLimitNs) { *sm.abort_flag = 1; break; }
+                }
+            }
+            umma_commit(smem_u32(sm.drain));
+            mbar_wait_drain(smem_u32(sm.drain), 0);
+        }
+    } else {
+        // ------------------------------------------- softmax + output warps --
+        const int g = (warp - 2) >> 2;   // TMEM buffer this group serves
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;  // query row within the item
+        const float sl2 = 0.125f * 1.4426950408889634f;
+        const uint32_t trow = tmem_base + ((uint32_t)(quad * 32) << 16);
+        const uint32_t srow = trow + TM_S + g * TROWS;
+        int i = 0;
+        for (int id = blockIdx.x; id < total; id += gridDim.x, ++i) {
+            if ((i & 1) != g) continue;
+            const uint32_t ph = (i >> 1) & 1;
+            const int b = id / kHeads, h = id % kHeads;
+            const int L = __ldg(seq_len + b), start = __ldg(seq_start + b);
+            const int nch = (L + 31) >> 5;  // 32-key chunks holding valid keys
+            bool got = mbar_wait(smem_u32(&sm.s_full[g]), ph, sm.abort_flag);
+            got = __all_sync(0xffffffffu, got);
+            if (!got) break;
+            tc_fence_after();
+            // pass 1: row maximum over the valid keys (two 32-key chunks per TMEM wait)
+            float m = -INFINITY;
+#pragma unroll 1
+            for (int c = 0; c < nch; c += 2) {
+                uint32_t v[2][32];
+                tmem_ld32(srow + c * 32, v[0]);
+                if (c + 1 < nch) tmem_ld32(srow + (c + 1) * 32, v[1]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    if (c + e >= nch) continue;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if ((c + e) * 32 + j < L) m = fmaxf(m, __uint_as_float(v[e][j]));
+                }
+            }
+            // pass 2: P = exp(scale * (s - max)) packed as bf16 pairs; chunk c goes to
+            // columns 16c..16c+15 of the same buffer, which hold scores already read
+            const float ms = m * sl2;
+            float l = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < nch; c += 2) {
+                uint32_t v[2][32];
+                tmem_ld32(srow + c * 32, v[0]);
+                if (c + 1 < nch) tmem_ld32(srow + (c + 1) * 32, v[1]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int cc = c + e;
+                    if (cc >= nch) continue;
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int k0 = cc * 32 + 2 * j;
+                        const float p0 = k0 < L ? ex2_approx(fmaf(__uint_as_float(v[e][2 * j]), sl2, -ms)) : 0.f;
+                        const float p1 = k0 + 1 < L ? ex2_approx(fmaf(__uint_as_float(v[e][2 * j + 1]), sl2, -ms)) : 0.f;
+                        l += p0 + p1;
+                        pk[j] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(srow + cc * 16, pk);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[g]));
+            got = mbar_wait(smem_u32(&sm.o_full[g]), ph, sm.abort_flag);
+            got = __all_sync(0xffffffffu, got);
+            if (!got) break;
+            tc_fence_after();
+            uint32_t o[2][32];
+            tmem_ld32(trow + TM_O + g * kHeadDim, o[0]);
+            tmem_ld32(trow + TM_O + g * kHeadDim + 32, o[1]);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.o_empty[g]));
+            if (r < L) {
+                const float inv = 1.f / l;
+                uint4 *dst = reinterpret_cast<uint4 *>(ctx + (size_t)(start + r) * kHidden + h * kHeadDim);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const uint32_t *x = o[q >> 2] + (q & 3) * 8;
+                    dst[q] = make_uint4(pack_bf16x2(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv),
+                                        pack_bf16x2(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv),
+                                        pack_bf16x2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv),
+                                        pack_bf16x2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv));
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+    if (threadIdx.x == 0 && *sm.abort_flag) set_status(status, kStatusTimeout);
+}
+
+}  // namespace
+
+cudaError_t launch_attention_tc(const CUtensorMap &tmQKV, const CUtensorMap &tmQKV64, bf16 *ctx, const int *seq_start,
+                                const int *seq_len, int nseq, int *status, int num_sms, cudaStream_t s) {
+    if (nseq <= 0) return cudaSuccess;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATC_SMEM);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    const int total = nseq * kHeads;
+    const int grid = total < num_sms ? total : num_sms;
+    attn_tc_kernel<<<grid, ATC_THREADS, ATC_SMEM, s>>>(tmQKV, tmQKV64, ctx, seq_start, seq_len, nseq, status);
+    return cudaGetLastError();
+}
+
+}  // namespace albert

@@ -94,6 +94,12 @@ cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB,
 cudaError_t launch_attention_bf16(const bf16 *qkv, bf16 *ctx, const int *seq_start,
                                   const int *seq_len, int nseq, int max_len,
                                   const int *status, cudaStream_t s);
+// Same operation on tcgen05 for max_len <= 128 (one item = one (sequence, head));
+// tmQKV / tmQKV64: bf16 maps of the packed [rows, 3*768] buffer with a {64, 128} /
+// {64, 64} box and the 128-byte swizzle.
+constexpr int kAttnTcMaxLen = 128;
+cudaError_t launch_attention_tc(const CUtensorMap &tmQKV, const CUtensorMap &tmQKV64, bf16 *ctx, const int *seq_start,
+                                const int *seq_len, int nseq, int *status, int num_sms, cudaStream_t s);
 cudaError_t launch_attention_f32(const float *qkv, float *ctx, const int *seq_start,
                                  const int *seq_len, int nseq, int max_len,
                                  const int *status, cudaStream_t s);
