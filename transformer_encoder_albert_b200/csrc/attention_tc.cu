@@ -155,7 +155,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                 if (no < ns) {
                     const int tb = no & 1, st = no % NSTAGE;
                     const uint32_t ph = (no >> 1) & 1;
-                    if (mbar_try_wait(smem_u32(&sm.p_full[tb]), ph) && mbar_try_wait(smem_u32(&sm.o_empty[tb]), ph ^ 1)) {
+                    if (mbar_test(smem_u32(&sm.p_full[tb]), ph) && mbar_test(smem_u32(&sm.o_empty[tb]), ph ^ 1)) {
                         tc_fence_after();
                         const int L = __ldg(seq_len + (blockIdx.x + no * gridDim.x) / kHeads);
                         const int ksteps = (L + 15) >> 4;
@@ -175,8 +175,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                 if (ns < n_items && ns < no + 2) {
                     const int tb = ns & 1, st = ns % NSTAGE;
                     const uint32_t ph = (ns >> 1) & 1;
-                    if (mbar_try_wait(smem_u32(&sm.ld_full[st]), (ns / NSTAGE) & 1) &&
-                        mbar_try_wait(smem_u32(&sm.s_empty[tb]), ph ^ 1)) {
+                    if (mbar_test(smem_u32(&sm.ld_full[st]), (ns / NSTAGE) & 1) &&
+                        mbar_test(smem_u32(&sm.s_empty[tb]), ph ^ 1)) {
                         tc_fence_after();
                         const int L = __ldg(seq_len + (blockIdx.x + ns * gridDim.x) / kHeads);
                         const uint32_t q = smem_u32(sm.stage + st * STAGE), k = q + TILE;

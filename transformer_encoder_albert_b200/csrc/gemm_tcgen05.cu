@@ -142,10 +142,7 @@ __device__ __forceinline__ void chan_merge(float &mean, float &m2, float cnt, fl
 }
 
 // Mean and 1/sqrt(var + eps) of a 768-wide row from its six 128-column partials.
-__device__ __forceinline__ void row_stats(const float2 *part, float eps, float &mu, float &rstd) {
-    float2 q[LN_PARTS];
-#pragma unroll
-    for (int i = 0; i < LN_PARTS; ++i) q[i] = __ldg(part + i);
+__device__ __forceinline__ void row_stats_merge(const float2 (&q)[LN_PARTS], float eps, float &mu, float &rstd) {
     float m = 0.f;
 #pragma unroll
     for (int i = 0; i < LN_PARTS; ++i) m += q[i].x;
@@ -305,6 +302,17 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         int acc = 0;
         bool ok = true;
         if (kRes && (int)blockIdx.x < units) res_issue(blockIdx.x, 0);
+        // row statistics of the next unit are fetched while the current one runs
+        float2 qin[LN_PARTS], qres[LN_PARTS];
+        auto fetch_stats = [&](int u) {
+            const size_t row = (size_t)(u / n_sub) * BM + r_local;
+#pragma unroll
+            for (int i = 0; i < LN_PARTS; ++i) {
+                if (kLnIn) qin[i] = __ldg(p.in_stats + row * LN_PARTS + i);
+                if (res_ln) qres[i] = __ldg(p.res_stats + row * LN_PARTS + i);
+            }
+        };
+        if ((kLnIn || res_ln) && (int)blockIdx.x < units) fetch_stats(blockIdx.x);
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             const int m = u / n_sub, n = u % n_sub;
             const int row = m * BM + r_local;  // < rows_cap
@@ -313,9 +321,10 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             int dst = row;
             if (kScatter) dst = row_ok ? __ldg(p.row_dst + row) : -1;
             float mu = 0.f, rstd = 1.f;        // LayerNorm of the A operand
-            if (kLnIn) row_stats(p.in_stats + (size_t)row * LN_PARTS, p.eps, mu, rstd);
+            if (kLnIn) row_stats_merge(qin, p.eps, mu, rstd);
             float rmu = 0.f, rrstd = 1.f;      // LayerNorm of the residual
-            if (res_ln) row_stats(p.res_stats + (size_t)row * LN_PARTS, p.eps, rmu, rrstd);
+            if (res_ln) row_stats_merge(qres, p.eps, rmu, rrstd);
+            if ((kLnIn || res_ln) && u + (int)gridDim.x < units) fetch_stats(u + gridDim.x);
             const float nmu = -rstd * mu, rnmu = -rrstd * rmu;
 
             const int ab = acc & 1;
@@ -327,10 +336,11 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + ab * BN + half * 128;
             const int ncol0 = n * BN + half * 128;  // first output column of this warp
             float mean = 0.f, m2 = 0.f;
-#pragma unroll 1
+            // chunk c + 1 loads from TMEM while chunk c is processed
+            uint32_t r[2][32];
+            tmem_ld32(tbase, r[0]);
+#pragma unroll
             for (int c = 0; c < 4; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tbase + c * 32, r);
                 uint4 rr[4];
                 if (kRes) {
                     bool rok = mbar_wait(rbar, rph, sm.abort_flag);
@@ -342,11 +352,14 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     for (int q = 0; q < 4; ++q) rr[q] = ld_shared_v4(rstg + stg_off(lane, q));
                 }
                 tmem_ld_wait();
-                if (c == 3) {
+                if (c < 3) {
+                    tmem_ld32(tbase + (c + 1) * 32, r[(c + 1) & 1]);
+                } else {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_u32(&sm.tempty[ab]));
                 }
+                const uint32_t *rc = r[c & 1];
                 const int col0 = ncol0 + c * 32;
                 float v[32];
                 const float4 *bias4 = reinterpret_cast<const float4 *>(p.bias + col0);
@@ -355,19 +368,19 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const float4 bb = __ldg(bias4 + q), ss = __ldg(s4 + q);
-                        v[4 * q + 0] = fmaf(rstd, __uint_as_float(r[4 * q + 0]), fmaf(nmu, ss.x, bb.x));
-                        v[4 * q + 1] = fmaf(rstd, __uint_as_float(r[4 * q + 1]), fmaf(nmu, ss.y, bb.y));
-                        v[4 * q + 2] = fmaf(rstd, __uint_as_float(r[4 * q + 2]), fmaf(nmu, ss.z, bb.z));
-                        v[4 * q + 3] = fmaf(rstd, __uint_as_float(r[4 * q + 3]), fmaf(nmu, ss.w, bb.w));
+                        v[4 * q + 0] = fmaf(rstd, __uint_as_float(rc[4 * q + 0]), fmaf(nmu, ss.x, bb.x));
+                        v[4 * q + 1] = fmaf(rstd, __uint_as_float(rc[4 * q + 1]), fmaf(nmu, ss.y, bb.y));
+                        v[4 * q + 2] = fmaf(rstd, __uint_as_float(rc[4 * q + 2]), fmaf(nmu, ss.z, bb.z));
+                        v[4 * q + 3] = fmaf(rstd, __uint_as_float(rc[4 * q + 3]), fmaf(nmu, ss.w, bb.w));
                     }
                 } else {
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const float4 bb = __ldg(bias4 + q);
-                        v[4 * q + 0] = __uint_as_float(r[4 * q + 0]) + bb.x;
-                        v[4 * q + 1] = __uint_as_float(r[4 * q + 1]) + bb.y;
-                        v[4 * q + 2] = __uint_as_float(r[4 * q + 2]) + bb.z;
-                        v[4 * q + 3] = __uint_as_float(r[4 * q + 3]) + bb.w;
+                        v[4 * q + 0] = __uint_as_float(rc[4 * q + 0]) + bb.x;
+                        v[4 * q + 1] = __uint_as_float(rc[4 * q + 1]) + bb.y;
+                        v[4 * q + 2] = __uint_as_float(rc[4 * q + 2]) + bb.z;
+                        v[4 * q + 3] = __uint_as_float(rc[4 * q + 3]) + bb.w;
                     }
                 }
                 if (kGelu) {
