@@ -275,6 +275,18 @@ def run_gpu(args):
     per_launch = flops_per_class(L, arch, rows)
     fwd_flops, gemm_flops = forward_flops(L, arch)
 
+    if args.ncu_forwards:
+        # untimed forwards only, for a profiler's launch list or kernel capture
+        for _ in range(args.ncu_forwards):
+            enc.forward(ids_d, mask_d, out)
+        torch.cuda.synchronize()
+        st = enc.status()
+        enc.close()
+        if st != 0:
+            raise SystemExit(f"device status {st}")
+        print(json.dumps({"ncu_forwards": args.ncu_forwards, "workload": wl.name, "tokens": n_tok}))
+        return 0
+
     # which kernel dominates: a short all-class profile before the timed region
     enc.profile(None)
     for _ in range(3):
@@ -405,6 +417,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ncu-forwards", type=int, default=0,
+                    help="run this many untimed forwards and exit (for ncu captures); no JSON metric line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -172,7 +172,12 @@ int albert_profile_read(albert_handle *h, int *launches, double *ms);
  * 1 = tanh-GELU(+bias) -> bf16; 2 = LN(A W^T + bias + R; g, b, eps) -> bf16,
  * with R: [M, N] bf16 and N == 768; 3 = bias -> bf16 rows scattered to
  * row_dst[r] (row_dst[r] < 0 skips the row).  K % 64 == 0, N % 256 == 0;
- * bias and ln_g 16-byte aligned (else ALBERT_ERR_CONFIG). */
+ * bias and ln_g 16-byte aligned (else ALBERT_ERR_CONFIG).  Adding
+ * ALBERT_GEMM_SINGLE_CTA or ALBERT_GEMM_CTA_PAIR to epi forces that kernel
+ * variant (one CTA per 128x256 tile, or a two-CTA cluster per 256x256 tile);
+ * by default the pair is used whenever M > 128, as in albert_forward. */
+#define ALBERT_GEMM_SINGLE_CTA 16
+#define ALBERT_GEMM_CTA_PAIR 32
 int albert_test_gemm(const void *A, const void *W, const float *bias, const void *R,
                      const float *ln_g, const float *ln_b, float eps, const int32_t *row_dst,
                      void *Y, int M, int N, int K, int epi, void *stream);

@@ -33,31 +33,37 @@ def _close(got, ref, rel=8e-3, what=""):
     assert not bad.any(), f"{what}: {bad.sum()} elements off, worst {err.max():.3e} (scale {scale:.3e})"
 
 
+VARIANTS = ["single", "pair"]
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("M,N,K", [(1, 256, 64), (300, 768, 128), (129, 2304, 768), (700, 2048, 768), (257, 512, 768)])
-def test_gemm_bias(M, N, K):
+def test_gemm_bias(M, N, K, variant):
     r = np.random.default_rng(M + N + K)
     A, W, b = r.normal(0, 1, (M, K)), r.normal(0, 0.05, (N, K)), r.normal(0, 0.1, N)
     At, Wt = _bf16_t(A), _bf16_t(W)
     Y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
-    assert tea.test_gemm(At, Wt, torch.tensor(b, dtype=torch.float32, device="cuda"), Y, 0) == 0
+    assert tea.test_gemm(At, Wt, torch.tensor(b, dtype=torch.float32, device="cuda"), Y, 0, variant=variant) == 0
     ref = oracle.linear(_np(At), _np(Wt), np.float32(b).astype(np.float64))
     _close(_np(Y), ref, what="bias")
 
 
+@pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("M", [5, 200, 640])
-def test_gemm_gelu(M):
+def test_gemm_gelu(M, variant):
     r = np.random.default_rng(M)
     N, K = 2048, 768
     A, W, b = r.normal(0, 1, (M, K)), r.normal(0, 0.05, (N, K)), r.normal(0, 0.1, N)
     At, Wt = _bf16_t(A), _bf16_t(W)
     Y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
-    assert tea.test_gemm(At, Wt, torch.tensor(b, dtype=torch.float32, device="cuda"), Y, 1) == 0
+    assert tea.test_gemm(At, Wt, torch.tensor(b, dtype=torch.float32, device="cuda"), Y, 1, variant=variant) == 0
     ref = oracle.gelu(oracle.linear(_np(At), _np(Wt), np.float32(b).astype(np.float64)))
     _close(_np(Y), ref, what="gelu")
 
 
+@pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("M,K", [(3, 768), (130, 768), (513, 2048), (1000, 768)])
-def test_gemm_residual_layer_norm(M, K):
+def test_gemm_residual_layer_norm(M, K, variant):
     r = np.random.default_rng(M * 7 + K)
     N = 768
     A, W, b = r.normal(0, 1, (M, K)), r.normal(0, 0.05, (N, K)), r.normal(0, 0.1, N)
@@ -66,13 +72,14 @@ def test_gemm_residual_layer_norm(M, K):
     At, Wt, Rt = _bf16_t(A), _bf16_t(W), _bf16_t(R)
     Y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
     f = lambda a: torch.tensor(a, dtype=torch.float32, device="cuda")
-    assert tea.test_gemm(At, Wt, f(b), Y, 2, R=Rt, ln_g=f(g), ln_b=f(beta), eps=1e-12) == 0
+    assert tea.test_gemm(At, Wt, f(b), Y, 2, R=Rt, ln_g=f(g), ln_b=f(beta), eps=1e-12, variant=variant) == 0
     z = oracle.linear(_np(At), _np(Wt), np.float32(b).astype(np.float64)) + _np(Rt)
     ref = oracle.layer_norm(z, np.float32(g).astype(np.float64), np.float32(beta).astype(np.float64), 1e-12)
     _close(_np(Y), ref, what="ln")
 
 
-def test_gemm_scatter_rows():
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_gemm_scatter_rows(variant):
     r = np.random.default_rng(9)
     M, N, K = 333, 512, 768
     A, W, b = r.normal(0, 1, (M, K)), r.normal(0, 0.05, (N, K)), r.normal(0, 0.1, N)
@@ -81,7 +88,7 @@ def test_gemm_scatter_rows():
     dst[::7] = -1
     Y = torch.full((M + 50, N), 7.0, device="cuda", dtype=torch.bfloat16)
     assert tea.test_gemm(At, Wt, torch.tensor(b, dtype=torch.float32, device="cuda"), Y, 3,
-                         row_dst=torch.tensor(dst, device="cuda")) == 0
+                         row_dst=torch.tensor(dst, device="cuda"), variant=variant) == 0
     ref = oracle.linear(_np(At), _np(Wt), np.float32(b).astype(np.float64))
     got = _np(Y)
     keep = dst >= 0

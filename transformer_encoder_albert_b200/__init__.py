@@ -238,14 +238,18 @@ def profile_class_names() -> list:
     return [lib().albert_profile_name(i).decode() for i in range(n)]
 
 
+GEMM_VARIANTS = {"auto": 0, "single": 16, "pair": 32}
+
+
 def test_gemm(A, W, bias, Y, epi: int, R=None, ln_g=None, ln_b=None, eps: float = 1e-12,
-              row_dst=None, stream=None) -> int:
-    """Run the tcgen05 GEMM alone (single-kernel parity tests)."""
+              row_dst=None, stream=None, variant: str = "auto") -> int:
+    """Run the tcgen05 GEMM alone (single-kernel parity tests).  variant picks
+    the one-CTA or the CTA-pair kernel ("auto": the pair when M > 128)."""
     M, K = A.shape
     N = W.shape[0]
     return lib().albert_test_gemm(_ptr(A), _ptr(W), _ptr(bias), _ptr(R), _ptr(ln_g), _ptr(ln_b),
-                                  float(eps), _ptr(row_dst), _ptr(Y), M, N, K, epi,
-                                  _stream_ptr(stream))
+                                  float(eps), _ptr(row_dst), _ptr(Y), M, N, K,
+                                  epi | GEMM_VARIANTS[variant], _stream_ptr(stream))
 
 
 def test_attention(qkv, cu_seqlens, max_len: int, ctx, fp32: bool = False, legacy: bool = False,

@@ -464,12 +464,12 @@ int create_impl(albert_handle *h, const albert_weights *w) {
             make_tmap_bf16(&h->tm_C, h->C, R, kHidden, gemm::BM) || make_tmap_bf16(&h->tm_X1, h->X1, R, kHidden, gemm::BM) ||
             make_tmap_bf16(&h->tm_H, h->H, R, kFfn, gemm::BM) || make_tmap_bf16(&h->tm_Z, h->Z, R, kHidden, gemm::BM) ||
             make_tmap_bf16(&h->tm_QKV, h->QKV, R, kQKV, 128) || make_tmap_bf16(&h->tm_QKV64, h->QKV, R, kQKV, 64) ||
-            make_tmap_bf16(&h->tm_win, h->w_in, kHidden, kEmb, gemm::BN) ||
-            make_tmap_bf16(&h->tm_wqkv, h->wqkv, kQKV, kHidden, gemm::BN) ||
-            make_tmap_bf16(&h->tm_wo, h->wo, kHidden, kHidden, gemm::BN) ||
-            make_tmap_bf16(&h->tm_w1, h->w1, kFfn, kHidden, gemm::BN) ||
-            make_tmap_bf16(&h->tm_w2, h->w2, kHidden, kFfn, gemm::BN) ||
-            (O && make_tmap_bf16(&h->tm_wout, h->w_out, O, kHidden, gemm::BN)) ||
+            make_tmap_bf16(&h->tm_win, h->w_in, kHidden, kEmb, gemm::B_BOX) ||
+            make_tmap_bf16(&h->tm_wqkv, h->wqkv, kQKV, kHidden, gemm::B_BOX) ||
+            make_tmap_bf16(&h->tm_wo, h->wo, kHidden, kHidden, gemm::B_BOX) ||
+            make_tmap_bf16(&h->tm_w1, h->w1, kFfn, kHidden, gemm::B_BOX) ||
+            make_tmap_bf16(&h->tm_w2, h->w2, kHidden, kFfn, gemm::B_BOX) ||
+            (O && make_tmap_bf16(&h->tm_wout, h->w_out, O, kHidden, gemm::B_BOX)) ||
             make_tmap_bf16_tile32(&h->t32_X, h->X, R, kHidden) || make_tmap_bf16_tile32(&h->t32_QKV, h->QKV, R, kQKV) ||
             make_tmap_bf16_tile32(&h->t32_X1, h->X1, R, kHidden) || make_tmap_bf16_tile32(&h->t32_H, h->H, R, kFfn) ||
             make_tmap_bf16_tile32(&h->t32_Z, h->Z, R, kHidden))
@@ -606,6 +606,9 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
                      int epi, void *stream) {
     if (!A || !W || !bias || !Y) return ALBERT_ERR_NULL;
     if (M < 1 || N < gemm::BN || N % gemm::BN || K < gemm::BK || K % gemm::BK) return ALBERT_ERR_SHAPE;
+    const int variant = (epi & ALBERT_GEMM_SINGLE_CTA) ? kGemmSingle : (epi & ALBERT_GEMM_CTA_PAIR) ? kGemmPair : kGemmAuto;
+    if ((epi & ALBERT_GEMM_SINGLE_CTA) && (epi & ALBERT_GEMM_CTA_PAIR)) return ALBERT_ERR_CONFIG;
+    epi &= ~(ALBERT_GEMM_SINGLE_CTA | ALBERT_GEMM_CTA_PAIR);
     if (epi < 0 || epi > 3) return ALBERT_ERR_CONFIG;
     if (epi == 2 && (!R || !ln_g || !ln_b || N != gemm::LN_N)) return ALBERT_ERR_CONFIG;
     if (epi == 3 && !row_dst) return ALBERT_ERR_NULL;
@@ -616,7 +619,7 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
     TRY(cudaGetDevice(&dev));
     TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
     const int rows_cap = (M + gemm::BM - 1) / gemm::BM * gemm::BM;
-    const int grid = gemm_grid(kepi, rows_cap, N, sms);
+    const int grid = gemm_grid(kepi, rows_cap, N, sms, variant);
     // epi 2 writes z * gamma and row statistics to temporaries, then normalizes them into Y
     int *ints = nullptr;
     void *zg = nullptr;
@@ -629,7 +632,7 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
         return ALBERT_ERR_ALLOC;
     }
     CUtensorMap ta, tb, to, tr;
-    int bad = make_tmap_bf16(&ta, A, M, K, gemm::BM) || make_tmap_bf16(&tb, W, N, K, gemm::BN);
+    int bad = make_tmap_bf16(&ta, A, M, K, gemm::BM) || make_tmap_bf16(&tb, W, N, K, gemm::B_BOX);
     if (epi == 2) bad = bad || make_tmap_bf16_tile32(&to, zg, rows_cap, N) || make_tmap_bf16_tile32(&tr, R, M, N);
     else if (epi != 3) bad = bad || make_tmap_bf16_tile32(&to, Y, M, N);
     if (epi == 3) to = ta;
@@ -641,7 +644,7 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
     a.N = N; a.K = K; a.rows_cap = rows_cap; a.n_rows = ints; a.bias = bias; a.eps = eps;
     a.out_g = ln_g; a.out_stats = stats; a.out = static_cast<bf16 *>(Y); a.ld_out = N;
     a.row_dst = row_dst; a.status = ints + 1;
-    if (e == cudaSuccess) e = launch_gemm(kepi, ta, tb, to, tr, a, grid, s);
+    if (e == cudaSuccess) e = launch_gemm(kepi, ta, tb, to, tr, a, grid, s, variant);
     if (e == cudaSuccess && epi == 2)
         e = launch_ln_rows(static_cast<const bf16 *>(zg), stats, ln_g, ln_b, eps, static_cast<bf16 *>(Y), nullptr, M,
                            rows_cap, ints, ints + 1, s);

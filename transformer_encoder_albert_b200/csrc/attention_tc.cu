@@ -12,18 +12,24 @@
 //                 64, 128-byte swizzle) from the packed [rows, 3*768] buffer
 //                 into a ring of four shared stages;
 //   warp 1      : tcgen05.mma issuer, an event loop that issues whichever is
-//                 ready: S = Q K^T (M=128, N=128 or 64, K=64) into TMEM, or
-//                 O = P V (M=128, N=64, K = L rounded up to 16) with P read from
-//                 TMEM and V from shared memory as an MN-major operand;
-//   warps 2..9  : two groups of 4 warps, one per TMEM buffer: each thread owns
-//                 one query row, reads its scores from TMEM, applies the mask and
-//                 a max-subtracted softmax in registers (no cross-thread
-//                 reductions), writes P as packed bf16 back into TMEM over the
-//                 scores it has read, then scales its row of O by 1/sum and
-//                 stores it.
-// Scores/P and O are double-buffered in TMEM, loads run up to four items ahead,
-// so item i's softmax overlaps item i+1's products and later items' loads.
-// Every wait is bounded (%globaltimer).
+//                 ready: S = Q K^T (M=128, N=128 or 64, K=64) into a TMEM
+//                 buffer, or O = P V (M=128, N=64, K = L rounded up to 16) with
+//                 P read from TMEM and V from shared memory as an MN-major
+//                 operand;
+//   warps 2..9  : two softmax groups of 4 warps (items alternate between
+//                 them): each thread owns one query row, reads its scores from
+//                 TMEM, applies the mask and a max-subtracted softmax in
+//                 registers (no cross-thread reductions), writes P as packed
+//                 bf16 back into TMEM over scores it has read and 1/sum into
+//                 shared memory, and moves on to its next item;
+//   warps 10..13: output group: per item, reads its rows of O from TMEM once
+//                 O = P V is complete, scales them by 1/sum and stores them.
+// TMEM holds four 128-column item buffers: S fills a buffer, P is packed into
+// its first 64 columns and O lands in the last 64 (scores already consumed),
+// so four items are in flight between the S product and the output, and a
+// softmax group finds its next scores ready when it finishes an item.  A warp
+// whose 32 query rows all lie past the sequence's end skips its softmax and
+// output.  Every wait is bounded (%globaltimer).
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
@@ -33,34 +39,36 @@ namespace {
 constexpr int TROWS = 128;                     // query rows / keys per item
 constexpr int TILE = TROWS * 128;              // 128 rows x 64 bf16 = 16 KB
 constexpr int STAGE = 3 * TILE;                // Q, K, V
-constexpr int NSTAGE = 4;
-constexpr int ATC_THREADS = 32 * 10;
-constexpr int ATC_SMEM = 1024 + NSTAGE * STAGE + 512;
-constexpr uint32_t TM_S = 0, TM_O = 256;       // TMEM columns: S/P[s] at 128 s, O[s] at 256 + 64 s
+constexpr int NSTAGE = 4;                      // shared-memory stages
+constexpr int NBUF = 4;                        // TMEM item buffers (128 columns each)
+constexpr int ATC_THREADS = 32 * 14;
+constexpr int ATC_SMEM = 1024 + NSTAGE * STAGE + 512 + NBUF * TROWS * 4;
+constexpr uint32_t TM_O = 64;                  // O's first column within an item buffer
 
 struct AttSmem {
     uint8_t *stage;
     uint64_t *ld_full, *ld_empty;              // [NSTAGE]
-    uint64_t *s_full, *s_empty, *p_full, *o_full, *o_empty;  // [2]
+    uint64_t *s_full, *p_full, *o_full, *o_empty;  // [NBUF]
     uint64_t *drain;
     uint32_t *tmem_slot;
     volatile int *abort_flag;
     int *misc;
+    float *inv_sum;                            // [NBUF][TROWS]
 };
 
 __device__ __forceinline__ AttSmem att_carve(uint8_t *raw) {
     AttSmem s;
     uint8_t *p = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
     s.stage = p;
-    uint64_t *b = reinterpret_cast<uint64_t *>(p + NSTAGE * STAGE);
+    s.inv_sum = reinterpret_cast<float *>(p + NSTAGE * STAGE);
+    uint64_t *b = reinterpret_cast<uint64_t *>(p + NSTAGE * STAGE + NBUF * TROWS * 4);
     s.ld_full = b;
     s.ld_empty = b + NSTAGE;
     s.s_full = b + 2 * NSTAGE;
-    s.s_empty = s.s_full + 2;
-    s.p_full = s.s_full + 4;
-    s.o_full = s.s_full + 6;
-    s.o_empty = s.s_full + 8;
-    s.drain = s.s_full + 10;
+    s.p_full = s.s_full + NBUF;
+    s.o_full = s.s_full + 2 * NBUF;
+    s.o_empty = s.s_full + 3 * NBUF;
+    s.drain = s.s_full + 4 * NBUF;
     uint32_t *u = reinterpret_cast<uint32_t *>(s.drain + 1);
     s.tmem_slot = u;
     s.abort_flag = reinterpret_cast<volatile int *>(u + 1);
@@ -83,9 +91,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
             mbar_init(smem_u32(&sm.ld_full[i]), 1);
             mbar_init(smem_u32(&sm.ld_empty[i]), 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NBUF; ++i) {
             mbar_init(smem_u32(&sm.s_full[i]), 1);
-            mbar_init(smem_u32(&sm.s_empty[i]), 1);
             mbar_init(smem_u32(&sm.p_full[i]), 4);
             mbar_init(smem_u32(&sm.o_full[i]), 1);
             mbar_init(smem_u32(&sm.o_empty[i]), 4);
@@ -100,7 +107,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     __syncthreads();
     if (sm.misc[0] != 0) return;  // an earlier kernel of this forward failed
     if (warp == 1) {
-        tmem_alloc(smem_u32(sm.tmem_slot), 512);
+        tmem_alloc(smem_u32(sm.tmem_slot), NBUF * TROWS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -153,36 +160,35 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
             while (no < n_items) {
                 bool progress = false;
                 if (no < ns) {
-                    const int tb = no & 1, st = no % NSTAGE;
-                    const uint32_t ph = (no >> 1) & 1;
-                    if (mbar_test(smem_u32(&sm.p_full[tb]), ph) && mbar_test(smem_u32(&sm.o_empty[tb]), ph ^ 1)) {
+                    const int tb = no % NBUF, st = no % NSTAGE;
+                    if (mbar_test(smem_u32(&sm.p_full[tb]), (no / NBUF) & 1)) {
                         tc_fence_after();
                         const int L = __ldg(seq_len + (blockIdx.x + no * gridDim.x) / kHeads);
                         const int ksteps = (L + 15) >> 4;
                         const uint32_t vbase = smem_u32(sm.stage + st * STAGE + 2 * TILE);
+                        const uint32_t buf = tmem_base + tb * TROWS;
                         for (int kk = 0; kk < ksteps; ++kk) {
                             // P: 16 keys = 8 packed TMEM columns; V: 16 keys = 16 rows of 128 B
-                            umma_bf16_ts(tmem_base + TM_O + tb * kHeadDim, tmem_base + TM_S + tb * TROWS + kk * 8,
-                                         sw128_kmajor_desc(vbase + kk * 2048), idesc_o, kk != 0);
+                            umma_bf16_ts(buf + TM_O, buf + kk * 8, sw128_kmajor_desc(vbase + kk * 2048), idesc_o,
+                                         kk != 0);
                         }
                         umma_commit(smem_u32(&sm.o_full[tb]));
-                        umma_commit(smem_u32(&sm.s_empty[tb]));   // P consumed: S buffer free
                         umma_commit(smem_u32(&sm.ld_empty[st]));  // Q, K, V consumed: stage free
                         ++no;
                         progress = true;
                     }
                 }
-                if (ns < n_items && ns < no + 2) {
-                    const int tb = ns & 1, st = ns % NSTAGE;
-                    const uint32_t ph = (ns >> 1) & 1;
+                if (ns < n_items && ns < no + NBUF) {
+                    const int tb = ns % NBUF, st = ns % NSTAGE;
+                    // the buffer is free once the output group has read item ns - NBUF
                     if (mbar_test(smem_u32(&sm.ld_full[st]), (ns / NSTAGE) & 1) &&
-                        mbar_test(smem_u32(&sm.s_empty[tb]), ph ^ 1)) {
+                        mbar_test(smem_u32(&sm.o_empty[tb]), ((ns / NBUF) & 1) ^ 1)) {
                         tc_fence_after();
                         const int L = __ldg(seq_len + (blockIdx.x + ns * gridDim.x) / kHeads);
                         const uint32_t q = smem_u32(sm.stage + st * STAGE), k = q + TILE;
 #pragma unroll
                         for (int kk = 0; kk < kHeadDim / 16; ++kk)
-                            umma_bf16(tmem_base + TM_S + tb * TROWS, sw128_kmajor_desc(q + kk * 32),
+                            umma_bf16(tmem_base + tb * TROWS, sw128_kmajor_desc(q + kk * 32),
                                       sw128_kmajor_desc(k + kk * 32), L <= 64 ? idesc_s64 : idesc_s128, kk != 0);
                         umma_commit(smem_u32(&sm.s_full[tb]));
                         ++ns;
@@ -201,84 +207,107 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
             umma_commit(smem_u32(sm.drain));
             mbar_wait_drain(smem_u32(sm.drain), 0);
         }
-    } else {
-        // ------------------------------------------- softmax + output warps --
-        const int g = (warp - 2) >> 2;   // TMEM buffer this group serves
+    } else if (warp < 10) {
+        // ------------------------------------------------------ softmax warps --
+        const int g = (warp - 2) >> 2;   // items i with i % 2 == g
         const int quad = warp & 3;
         const int r = quad * 32 + lane;  // query row within the item
         const float sl2 = 0.125f * 1.4426950408889634f;
         const uint32_t trow = tmem_base + ((uint32_t)(quad * 32) << 16);
-        const uint32_t srow = trow + TM_S + g * TROWS;
         int i = 0;
         for (int id = blockIdx.x; id < total; id += gridDim.x, ++i) {
             if ((i & 1) != g) continue;
-            const uint32_t ph = (i >> 1) & 1;
-            const int b = id / kHeads, h = id % kHeads;
-            const int L = __ldg(seq_len + b), start = __ldg(seq_start + b);
+            const int tb = i % NBUF;
+            const uint32_t ph = (i / NBUF) & 1;
+            const uint32_t srow = trow + tb * TROWS;
+            const int L = __ldg(seq_len + id / kHeads);
             const int nch = (L + 31) >> 5;  // 32-key chunks holding valid keys
-            bool got = mbar_wait(smem_u32(&sm.s_full[g]), ph, sm.abort_flag);
+            const bool live = quad * 32 < L;  // some row of this warp is a real query
+            bool got = mbar_wait(smem_u32(&sm.s_full[tb]), ph, sm.abort_flag);
             got = __all_sync(0xffffffffu, got);
             if (!got) break;
             tc_fence_after();
-            // pass 1: row maximum over the valid keys (two 32-key chunks per TMEM wait)
-            float m = -INFINITY;
+            if (live) {
+                // pass 1: row maximum over the valid keys (two 32-key chunks per TMEM wait)
+                float m = -INFINITY;
 #pragma unroll 1
-            for (int c = 0; c < nch; c += 2) {
-                uint32_t v[2][32];
-                tmem_ld32(srow + c * 32, v[0]);
-                if (c + 1 < nch) tmem_ld32(srow + (c + 1) * 32, v[1]);
-                tmem_ld_wait();
+                for (int c = 0; c < nch; c += 2) {
+                    uint32_t v[2][32];
+                    tmem_ld32(srow + c * 32, v[0]);
+                    if (c + 1 < nch) tmem_ld32(srow + (c + 1) * 32, v[1]);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    if (c + e >= nch) continue;
+                    for (int e = 0; e < 2; ++e) {
+                        if (c + e >= nch) continue;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if ((c + e) * 32 + j < L) m = fmaxf(m, __uint_as_float(v[e][j]));
-                }
-            }
-            // pass 2: P = exp(scale * (s - max)) packed as bf16 pairs; chunk c goes to
-            // columns 16c..16c+15 of the same buffer, which hold scores already read
-            const float ms = m * sl2;
-            float l = 0.f;
-#pragma unroll 1
-            for (int c = 0; c < nch; c += 2) {
-                uint32_t v[2][32];
-                tmem_ld32(srow + c * 32, v[0]);
-                if (c + 1 < nch) tmem_ld32(srow + (c + 1) * 32, v[1]);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int cc = c + e;
-                    if (cc >= nch) continue;
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int k0 = cc * 32 + 2 * j;
-                        const float p0 = k0 < L ? ex2_approx(fmaf(__uint_as_float(v[e][2 * j]), sl2, -ms)) : 0.f;
-                        const float p1 = k0 + 1 < L ? ex2_approx(fmaf(__uint_as_float(v[e][2 * j + 1]), sl2, -ms)) : 0.f;
-                        l += p0 + p1;
-                        pk[j] = pack_bf16x2(p0, p1);
+                        for (int j = 0; j < 32; ++j)
+                            if ((c + e) * 32 + j < L) m = fmaxf(m, __uint_as_float(v[e][j]));
                     }
-                    tmem_st16(srow + cc * 16, pk);
                 }
+                // pass 2: P = exp(scale * (s - max)) packed as bf16 pairs; chunk c goes to
+                // columns 16c..16c+15 of the same buffer, which hold scores already read
+                const float ms = m * sl2;
+                float l = 0.f;
+#pragma unroll 1
+                for (int c = 0; c < nch; c += 2) {
+                    uint32_t v[2][32];
+                    tmem_ld32(srow + c * 32, v[0]);
+                    if (c + 1 < nch) tmem_ld32(srow + (c + 1) * 32, v[1]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int cc = c + e;
+                        if (cc >= nch) continue;
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int k0 = cc * 32 + 2 * j;
+                            const float p0 = k0 < L ? ex2_approx(fmaf(__uint_as_float(v[e][2 * j]), sl2, -ms)) : 0.f;
+                            const float p1 = k0 + 1 < L ? ex2_approx(fmaf(__uint_as_float(v[e][2 * j + 1]), sl2, -ms)) : 0.f;
+                            l += p0 + p1;
+                            pk[j] = pack_bf16x2(p0, p1);
+                        }
+                        tmem_st16(srow + cc * 16, pk);
+                    }
+                }
+                // read by the output group after it has waited on p_full
+                sm.inv_sum[tb * TROWS + r] = 1.f / l;
+                tmem_st_wait();
             }
-            tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[g]));
-            got = mbar_wait(smem_u32(&sm.o_full[g]), ph, sm.abort_flag);
+            if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[tb]));
+        }
+    } else {
+        // ------------------------------------------------------- output warps --
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;  // query row within the item
+        const uint32_t trow = tmem_base + ((uint32_t)(quad * 32) << 16);
+        int i = 0;
+        for (int id = blockIdx.x; id < total; id += gridDim.x, ++i) {
+            const int tb = i % NBUF;
+            const uint32_t ph = (i / NBUF) & 1;
+            const int b = id / kHeads, h = id % kHeads;
+            const int L = __ldg(seq_len + b), start = __ldg(seq_start + b);
+            const bool live = quad * 32 < L;
+            // p_full (complete before O is) makes the softmax's 1/sum visible here
+            bool got = mbar_wait(smem_u32(&sm.o_full[tb]), ph, sm.abort_flag) &&
+                       mbar_wait(smem_u32(&sm.p_full[tb]), ph, sm.abort_flag);
             got = __all_sync(0xffffffffu, got);
             if (!got) break;
             tc_fence_after();
             uint32_t o[2][32];
-            tmem_ld32(trow + TM_O + g * kHeadDim, o[0]);
-            tmem_ld32(trow + TM_O + g * kHeadDim + 32, o[1]);
-            tmem_ld_wait();
+            float inv = 0.f;
+            if (live) {
+                tmem_ld32(trow + tb * TROWS + TM_O, o[0]);
+                tmem_ld32(trow + tb * TROWS + TM_O + 32, o[1]);
+                inv = sm.inv_sum[tb * TROWS + r];
+                tmem_ld_wait();
+            }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm.o_empty[g]));
+            if (lane == 0) mbar_arrive(smem_u32(&sm.o_empty[tb]));
             if (r < L) {
-                const float inv = 1.f / l;
                 uint4 *dst = reinterpret_cast<uint4 *>(ctx + (size_t)(start + r) * kHidden + h * kHeadDim);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
@@ -295,7 +324,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, 512);
+        tmem_dealloc(tmem_base, NBUF * TROWS);
     }
     if (threadIdx.x == 0 && *sm.abort_flag) set_status(status, kStatusTimeout);
 }

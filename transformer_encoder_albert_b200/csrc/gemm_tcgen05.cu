@@ -44,49 +44,68 @@ namespace {
 
 using namespace gemm;
 
+// Shared-memory plan of one kernel instance: {A, B} pipeline stages, then 2 KB
+// staging tiles per epilogue warp (output, residual or second output, and for
+// the residual epilogue a second output tile, paid for with one stage), then
+// barriers; 1 KiB slack for the 1 KiB alignment of the stages.
+template <int EPI, bool PAIR>
+struct Plan {
+    static constexpr bool kRes = EPI == kEpiResStats;
+    static constexpr int NST = (PAIR ? PAIR_STAGES : STAGES) - (kRes ? 1 : 0);
+    static constexpr int BSTAGE = PAIR ? B_HALF_BYTES : B_BYTES;
+    static constexpr int NSTG = kRes ? 3 : 2;
+    static constexpr int SMEM = 1024 + NST * (A_BYTES + BSTAGE) + NSTG * EPI_WARPS * STG_BYTES + 1024;
+    static_assert(SMEM <= 232448, "shared memory per CTA");
+};
+
 struct Smem {
     uint8_t *a, *b;
-    uint8_t *stg;            // one 2 KB output staging tile per epilogue warp
-    uint8_t *rstg;           // one 2 KB residual staging tile per epilogue warp
+    uint8_t *stg;            // 2 KB output staging tile per epilogue warp
+    uint8_t *rstg;           // 2 KB residual (or second output) staging tile per epilogue warp
+    uint8_t *stg2;           // residual epilogue: second 2 KB output staging tile per warp
     uint64_t *full, *empty, *tfull, *tempty, *drain, *rbar;
     uint32_t *tmem_slot;
     volatile int *abort_flag;
     int *misc;               // [0] n_rows, [1] status at entry
 };
 
+template <int EPI, bool PAIR>
 __device__ __forceinline__ Smem carve(uint8_t *raw) {
+    using P = Plan<EPI, PAIR>;
+    constexpr int NST = P::NST;
     Smem s;
     uint8_t *p = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
     s.a = p;
-    s.b = p + STAGES * A_BYTES;
-    s.stg = s.b + STAGES * B_BYTES;
+    s.b = p + NST * A_BYTES;
+    s.stg = s.b + NST * P::BSTAGE;
     s.rstg = s.stg + EPI_WARPS * STG_BYTES;
-    uint8_t *ctrl = s.rstg + EPI_WARPS * STG_BYTES;
+    s.stg2 = s.rstg + EPI_WARPS * STG_BYTES;
+    uint8_t *ctrl = s.stg + P::NSTG * EPI_WARPS * STG_BYTES;
     uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl);
     s.full = bars;
-    s.empty = bars + STAGES;
-    s.tfull = bars + 2 * STAGES;
-    s.tempty = bars + 2 * STAGES + 2;
-    s.drain = bars + 2 * STAGES + 4;
-    s.rbar = bars + 2 * STAGES + 5;
-    uint32_t *u = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5 + EPI_WARPS);
+    s.empty = bars + NST;
+    s.tfull = bars + 2 * NST;
+    s.tempty = bars + 2 * NST + 2;
+    s.drain = bars + 2 * NST + 4;
+    s.rbar = bars + 2 * NST + 5;
+    uint32_t *u = reinterpret_cast<uint32_t *>(bars + 2 * NST + 5 + EPI_WARPS);
     s.tmem_slot = u;
     s.abort_flag = reinterpret_cast<volatile int *>(u + 1);
     s.misc = reinterpret_cast<int *>(u + 2);
     return s;
 }
 
-__device__ __forceinline__ void store_bf16x32(bf16 *dst, const float (&v)[32]) {
+// 32 values held as 16 fp32 pairs -> 4 x 16 bytes of bf16.
+__device__ __forceinline__ uint32_t pack_pair(uint64_t v) {
+    const float2 f = f2_split(v);
+    return pack_bf16x2(f.x, f.y);
+}
+
+__device__ __forceinline__ void store_bf16x32(bf16 *dst, const uint64_t (&v)[16]) {
     uint4 *d = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint4 w;
-        w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-        w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-        w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-        w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-        d[q] = w;
-    }
+    for (int q = 0; q < 4; ++q)
+        d[q] = make_uint4(pack_pair(v[4 * q]), pack_pair(v[4 * q + 1]), pack_pair(v[4 * q + 2]), pack_pair(v[4 * q + 3]));
 }
 
 // Byte offset of 16-byte chunk q of row r in a 32x32 bf16 tile (64-byte rows)
@@ -110,22 +129,19 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
 // The previous store from the same tile must have finished reading it: with
 // two tiles used alternately (double_buffered) that store is the one before
 // the most recent.
-__device__ __forceinline__ void stage_and_store(uint32_t stg, const float (&v)[32], const CUtensorMap *tm,
+__device__ __forceinline__ void stage_and_store(uint32_t stg, const uint64_t (&v)[16], const CUtensorMap *tm,
                                                 int x, int y, int lane, bool double_buffered) {
+    uint4 w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        w[q] = make_uint4(pack_pair(v[4 * q]), pack_pair(v[4 * q + 1]), pack_pair(v[4 * q + 2]), pack_pair(v[4 * q + 3]));
     if (lane == 0) {
         if (double_buffered) bulk_wait_read1();
         else bulk_wait_read0();
     }
     __syncwarp();
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint4 w;
-        w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-        w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-        w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-        w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-        st_shared_v4(stg + stg_off(lane, q), w);
-    }
+    for (int q = 0; q < 4; ++q) st_shared_v4(stg + stg_off(lane, q), w[q]);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
@@ -157,7 +173,7 @@ __device__ __forceinline__ void row_stats_merge(const float2 (&q)[LN_PARTS], flo
     rstd = rsqrtf(m2 * (1.0f / LN_N) + eps);
 }
 
-template <int EPI>
+template <int EPI, bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmRes,
@@ -166,21 +182,29 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     constexpr bool kGelu = EPI == kEpiGelu || EPI == kEpiLnInGelu;
     constexpr bool kScatter = EPI == kEpiScatter || EPI == kEpiLnInScatter;
     constexpr bool kRes = EPI == kEpiResStats;
+    constexpr int NST = Plan<EPI, PAIR>::NST;
+    constexpr int BSTAGE = Plan<EPI, PAIR>::BSTAGE;
+    constexpr int UM = PAIR ? 2 * BM : BM;  // rows of A (and D) per unit
     extern __shared__ uint8_t smem_raw[];
-    Smem sm = carve(smem_raw);
+    Smem sm = carve<EPI, PAIR>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // A pair works on one unit at a time; rank 0 issues the MMAs for both CTAs.
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0;
+    const int slot = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int nslots = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
     if (threadIdx.x == 0) {
         sm.misc[0] = *reinterpret_cast<const volatile int *>(p.n_rows);
         sm.misc[1] = *reinterpret_cast<const volatile int *>(p.status);
         *sm.abort_flag = 0;
-        for (int i = 0; i < STAGES; ++i) {
+        for (int i = 0; i < NST; ++i) {
             mbar_init(smem_u32(&sm.full[i]), 1);
             mbar_init(smem_u32(&sm.empty[i]), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&sm.tfull[i]), 1);
-            mbar_init(smem_u32(&sm.tempty[i]), EPI_WARPS);
+            // the pair's accumulator is released by the epilogues of both CTAs
+            mbar_init(smem_u32(&sm.tempty[i]), PAIR ? 2 * EPI_WARPS : EPI_WARPS);
         }
         mbar_init(smem_u32(sm.drain), 1);
         for (int i = 0; i < EPI_WARPS; ++i) mbar_init(smem_u32(&sm.rbar[i]), 1);
@@ -192,21 +216,27 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         if (!kScatter) prefetch_tmap(&tmOut);
         if (kRes) prefetch_tmap(&tmRes);
     }
-    __syncthreads();
-    // An earlier kernel of this forward failed, or the row count is out of range.
-    if (sm.misc[1] != 0 || sm.misc[0] < 0 || sm.misc[0] > p.rows_cap) return;
-
     if (warp == 1) {
-        tmem_alloc(smem_u32(sm.tmem_slot), TMEM_COLS);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(smem_u32(sm.tmem_slot), TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(sm.tmem_slot), TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    // barrier initialisation (and, for a pair, the peer's) is visible before any use
+    if (PAIR) cluster_sync();
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *sm.tmem_slot;
 
-    const int n_rows = sm.misc[0];
-    const int m_blocks = (n_rows + BM - 1) / BM;
+    // An earlier kernel of this forward failed, or the row count is out of range:
+    // no units (every role still reaches the teardown, which a pair shares).
+    const bool skip = sm.misc[1] != 0 || sm.misc[0] < 0 || sm.misc[0] > p.rows_cap;
+    const int n_rows = skip ? 0 : sm.misc[0];
+    const int m_blocks = (n_rows + UM - 1) / UM;
     const int n_sub = p.N / BN;
     const int units = m_blocks * n_sub;  // unit u = tile (u / n_sub, u % n_sub), row-block major
     const int kblocks = p.K / BK;
@@ -218,7 +248,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             int stage = 0, issued = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            for (int u = slot; u < units && ok; u += nslots) {
                 const int m = u / n_sub, n = u % n_sub;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(smem_u32(&sm.empty[stage]), phase ^ 1, sm.abort_flag)) {
@@ -226,33 +256,46 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         break;
                     }
                     const uint32_t fb = smem_u32(&sm.full[stage]);
-                    mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
-                    tma_load_2d(smem_u32(sm.a + stage * A_BYTES), &tmA, fb, kb * BK, m * BM);
-                    tma_load_2d_hint(smem_u32(sm.b + stage * B_BYTES), &tmB, fb, kb * BK, n * BN, keep);
+                    const uint32_t a_dst = smem_u32(sm.a + stage * A_BYTES);
+                    const uint32_t b_dst = smem_u32(sm.b + stage * BSTAGE);
+                    if (PAIR) {
+                        // both CTAs' copies count on rank 0's barrier, which expects them all
+                        const uint32_t fb0 = mapa_shared(fb, 0);
+                        if (rank == 0) mbar_arrive_expect_tx(fb, 2 * (A_BYTES + B_HALF_BYTES));
+                        tma_load_2d_pair(a_dst, &tmA, fb0, kb * BK, m * UM + (int)rank * BM);
+                        tma_load_2d_pair_hint(b_dst, &tmB, fb0, kb * BK, n * BN + (int)rank * B_BOX, keep);
+                    } else {
+                        mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
+                        tma_load_2d(a_dst, &tmA, fb, kb * BK, m * BM);
+                        tma_load_2d_hint(b_dst, &tmB, fb, kb * BK, n * BN, keep);
+                        tma_load_2d_hint(b_dst + B_HALF_BYTES, &tmB, fb, kb * BK, n * BN + B_BOX, keep);
+                    }
                     ++issued;
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    if (++stage == NST) { stage = 0; phase ^= 1; }
                 }
             }
-            if (!ok) {
+            if (!ok && (!PAIR || rank == 0)) {
                 // Drain: every stage whose load may still be in flight completes
                 // its transaction count before the CTA's shared memory goes away.
-                for (int i = 0; i < STAGES && i < issued; ++i) {
-                    if (--stage < 0) { stage = STAGES - 1; phase ^= 1; }
+                // (A pair's rank 1 counts its copies on rank 0's barriers; rank 0
+                // drains them before the pair's closing cluster barrier.)
+                for (int i = 0; i < NST && i < issued; ++i) {
+                    if (--stage < 0) { stage = NST - 1; phase ^= 1; }
                     mbar_wait_drain(smem_u32(&sm.full[stage]), phase);
                 }
             }
         }
     } else if (warp == 1) {
         // -------------------------------------------------------- MMA issuer --
-        if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(BM, BN);
+        if (lane == 0 && rank == 0) {
+            const uint32_t idesc = idesc_bf16_f32(UM, BN);
             int stage = 0, acc = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            for (int u = slot; u < units && ok; u += nslots) {
                 const int ab = acc & 1;
                 const uint32_t aph = (acc >> 1) & 1;
-                if (!mbar_wait(smem_u32(&sm.tempty[ab]), aph ^ 1, sm.abort_flag)) break;
+                if (!mbar_wait<PAIR>(smem_u32(&sm.tempty[ab]), aph ^ 1, sm.abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + ab * BN;
                 for (int kb = 0; kb < kblocks; ++kb) {
@@ -262,20 +305,29 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(sm.a + stage * A_BYTES);
-                    const uint32_t b0 = smem_u32(sm.b + stage * B_BYTES);
+                    const uint32_t b0 = smem_u32(sm.b + stage * BSTAGE);
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k)
-                        umma_bf16(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), idesc,
-                                  (kb | k) != 0);
-                    umma_commit(smem_u32(&sm.empty[stage]));
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    for (int k = 0; k < BK / 16; ++k) {
+                        if (PAIR)
+                            umma_bf16_pair(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), idesc,
+                                           (kb | k) != 0);
+                        else
+                            umma_bf16(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), idesc,
+                                      (kb | k) != 0);
+                    }
+                    // the stage is free in both CTAs once these MMAs have read it
+                    if (PAIR) umma_commit_pair(smem_u32(&sm.empty[stage]), 3);
+                    else umma_commit(smem_u32(&sm.empty[stage]));
+                    if (++stage == NST) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
-                umma_commit(smem_u32(&sm.tfull[ab]));
+                if (PAIR) umma_commit_pair(smem_u32(&sm.tfull[ab]), 3);
+                else umma_commit(smem_u32(&sm.tfull[ab]));
                 ++acc;
             }
             // All MMAs issued by this thread complete before TMEM is released.
-            umma_commit(smem_u32(sm.drain));
+            if (PAIR) umma_commit_pair(smem_u32(sm.drain), 1);
+            else umma_commit(smem_u32(sm.drain));
             mbar_wait_drain(smem_u32(sm.drain), 0);
         }
     } else {
@@ -284,8 +336,10 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int quad = warp & 3;          // TMEM lanes 32*quad .. 32*quad+31
         const int half = ew >> 2;           // column half of the 256-wide tile
         const int r_local = quad * 32 + lane;
+        const int row_off = (int)rank * BM;  // this CTA's rows within a unit
         const uint32_t stg = smem_u32(sm.stg + ew * STG_BYTES);
         const uint32_t rstg = smem_u32(sm.rstg + ew * STG_BYTES);
+        const uint32_t stg2 = smem_u32(sm.stg2 + ew * STG_BYTES);  // kRes only
         const uint32_t rbar = smem_u32(&sm.rbar[ew]);
         const bool res_ln = kRes && p.res_stats != nullptr;
         uint32_t rph = 0;
@@ -295,36 +349,38 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             if (lane == 0) {
                 mbar_arrive_expect_tx(rbar, STG_BYTES);
                 tma_load_2d(rstg, &tmRes, rbar, (u % n_sub) * BN + half * 128 + c * 32,
-                            (u / n_sub) * BM + quad * 32);
+                            (u / n_sub) * UM + row_off + quad * 32);
             }
             res_pending = true;
         };
         int acc = 0;
         bool ok = true;
-        if (kRes && (int)blockIdx.x < units) res_issue(blockIdx.x, 0);
+        if (kRes && slot < units) res_issue(slot, 0);
         // row statistics of the next unit are fetched while the current one runs
         float2 qin[LN_PARTS], qres[LN_PARTS];
+        // (rows past rows_cap, reachable in a pair's last unit, read as zeros)
         auto fetch_stats = [&](int u) {
-            const size_t row = (size_t)(u / n_sub) * BM + r_local;
+            const int row = (u / n_sub) * UM + row_off + r_local;
+            const bool in = row < p.rows_cap;
 #pragma unroll
             for (int i = 0; i < LN_PARTS; ++i) {
-                if (kLnIn) qin[i] = __ldg(p.in_stats + row * LN_PARTS + i);
-                if (res_ln) qres[i] = __ldg(p.res_stats + row * LN_PARTS + i);
+                if (kLnIn) qin[i] = in ? __ldg(p.in_stats + (size_t)row * LN_PARTS + i) : make_float2(0.f, 0.f);
+                if (res_ln) qres[i] = in ? __ldg(p.res_stats + (size_t)row * LN_PARTS + i) : make_float2(0.f, 0.f);
             }
         };
-        if ((kLnIn || res_ln) && (int)blockIdx.x < units) fetch_stats(blockIdx.x);
-        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        if ((kLnIn || res_ln) && slot < units) fetch_stats(slot);
+        for (int u = slot; u < units && ok; u += nslots) {
             const int m = u / n_sub, n = u % n_sub;
-            const int row = m * BM + r_local;  // < rows_cap
+            const int row = m * UM + row_off + r_local;
             const bool row_ok = row < n_rows;
-            const int tile_row = m * BM + quad * 32;
+            const int tile_row = m * UM + row_off + quad * 32;
             int dst = row;
             if (kScatter) dst = row_ok ? __ldg(p.row_dst + row) : -1;
             float mu = 0.f, rstd = 1.f;        // LayerNorm of the A operand
             if (kLnIn) row_stats_merge(qin, p.eps, mu, rstd);
             float rmu = 0.f, rrstd = 1.f;      // LayerNorm of the residual
             if (res_ln) row_stats_merge(qres, p.eps, rmu, rrstd);
-            if ((kLnIn || res_ln) && u + (int)gridDim.x < units) fetch_stats(u + gridDim.x);
+            if ((kLnIn || res_ln) && u + nslots < units) fetch_stats(u + nslots);
             const float nmu = -rstd * mu, rnmu = -rrstd * rmu;
 
             const int ab = acc & 1;
@@ -357,73 +413,80 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 } else {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&sm.tempty[ab]));
+                    if (lane == 0) {
+                        if (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&sm.tempty[ab]), 0));
+                        else mbar_arrive(smem_u32(&sm.tempty[ab]));
+                    }
                 }
                 const uint32_t *rc = r[c & 1];
                 const int col0 = ncol0 + c * 32;
-                float v[32];
+                uint64_t v[16];  // columns col0 + 2j, col0 + 2j + 1
                 const float4 *bias4 = reinterpret_cast<const float4 *>(p.bias + col0);
                 if (kLnIn) {
                     const float4 *s4 = reinterpret_cast<const float4 *>(p.fold_s + col0);
+                    const uint64_t rstd2 = f2_make(rstd, rstd), nmu2 = f2_make(nmu, nmu);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const float4 bb = __ldg(bias4 + q), ss = __ldg(s4 + q);
-                        v[4 * q + 0] = fmaf(rstd, __uint_as_float(rc[4 * q + 0]), fmaf(nmu, ss.x, bb.x));
-                        v[4 * q + 1] = fmaf(rstd, __uint_as_float(rc[4 * q + 1]), fmaf(nmu, ss.y, bb.y));
-                        v[4 * q + 2] = fmaf(rstd, __uint_as_float(rc[4 * q + 2]), fmaf(nmu, ss.z, bb.z));
-                        v[4 * q + 3] = fmaf(rstd, __uint_as_float(rc[4 * q + 3]), fmaf(nmu, ss.w, bb.w));
+                        v[2 * q] = f2_fma(rstd2, f2_make_u(rc[4 * q], rc[4 * q + 1]),
+                                          f2_fma(nmu2, f2_make(ss.x, ss.y), f2_make(bb.x, bb.y)));
+                        v[2 * q + 1] = f2_fma(rstd2, f2_make_u(rc[4 * q + 2], rc[4 * q + 3]),
+                                              f2_fma(nmu2, f2_make(ss.z, ss.w), f2_make(bb.z, bb.w)));
                     }
                 } else {
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const float4 bb = __ldg(bias4 + q);
-                        v[4 * q + 0] = __uint_as_float(rc[4 * q + 0]) + bb.x;
-                        v[4 * q + 1] = __uint_as_float(rc[4 * q + 1]) + bb.y;
-                        v[4 * q + 2] = __uint_as_float(rc[4 * q + 2]) + bb.z;
-                        v[4 * q + 3] = __uint_as_float(rc[4 * q + 3]) + bb.w;
+                        v[2 * q] = f2_add(f2_make_u(rc[4 * q], rc[4 * q + 1]), f2_make(bb.x, bb.y));
+                        v[2 * q + 1] = f2_add(f2_make_u(rc[4 * q + 2], rc[4 * q + 3]), f2_make(bb.z, bb.w));
                     }
                 }
                 if (kGelu) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = gelu_tanh_fast(v[j]);
+                    for (int j = 0; j < 16; ++j) v[j] = gelu_tanh_f2(v[j]);
                 }
                 if (kRes) {
-                    // residual: plain, or rebuilt LayerNorm output (its beta is folded into bias)
-                    float x[32];
+                    // residual: plain, or rebuilt LayerNorm output (its beta is folded into bias);
+                    // bf16 -> fp32 is the high half of a 32-bit word
+                    uint64_t x[16];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        float2 f;
-                        f = unpack_bf16x2(rr[q].x); x[8 * q + 0] = f.x; x[8 * q + 1] = f.y;
-                        f = unpack_bf16x2(rr[q].y); x[8 * q + 2] = f.x; x[8 * q + 3] = f.y;
-                        f = unpack_bf16x2(rr[q].z); x[8 * q + 4] = f.x; x[8 * q + 5] = f.y;
-                        f = unpack_bf16x2(rr[q].w); x[8 * q + 6] = f.x; x[8 * q + 7] = f.y;
+                        const uint32_t w4[4] = {rr[q].x, rr[q].y, rr[q].z, rr[q].w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) x[4 * q + e] = f2_make_u(w4[e] << 16, w4[e] & 0xffff0000u);
                     }
                     // the residual tile has been read: prefetch the next chunk
                     __syncwarp();
                     if (c < 3) res_issue(u, c + 1);
-                    else if (u + (int)gridDim.x < units) res_issue(u + gridDim.x, 0);
+                    else if (u + nslots < units) res_issue(u + nslots, 0);
                     if (res_ln) {
                         const float4 *rg4 = reinterpret_cast<const float4 *>(p.res_g + col0);
+                        const uint64_t rrstd2 = f2_make(rrstd, rrstd), rnmu2 = f2_make(rnmu, rnmu);
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
                             const float4 g = __ldg(rg4 + q);
-                            v[4 * q + 0] += fmaf(rrstd, x[4 * q + 0], rnmu * g.x);
-                            v[4 * q + 1] += fmaf(rrstd, x[4 * q + 1], rnmu * g.y);
-                            v[4 * q + 2] += fmaf(rrstd, x[4 * q + 2], rnmu * g.z);
-                            v[4 * q + 3] += fmaf(rrstd, x[4 * q + 3], rnmu * g.w);
+                            v[2 * q] = f2_fma(rrstd2, x[2 * q], f2_fma(rnmu2, f2_make(g.x, g.y), v[2 * q]));
+                            v[2 * q + 1] = f2_fma(rrstd2, x[2 * q + 1], f2_fma(rnmu2, f2_make(g.z, g.w), v[2 * q + 1]));
                         }
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] += x[j];
+                        for (int j = 0; j < 16; ++j) v[j] = f2_add(v[j], x[j]);
                     }
                     // exact chunk statistics of z, merged into the running ones
-                    float cs = 0.f;
+                    uint64_t s2 = v[0];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) cs += v[j];
-                    const float cm = cs * (1.0f / 32.0f);
-                    float cq = 0.f;
+                    for (int j = 1; j < 16; ++j) s2 = f2_add(s2, v[j]);
+                    const float2 sf = f2_split(s2);
+                    const float cm = (sf.x + sf.y) * (1.0f / 32.0f);
+                    const uint64_t ncm2 = f2_make(-cm, -cm);
+                    uint64_t q2 = f2_make(0.f, 0.f);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) { const float d = v[j] - cm; cq = fmaf(d, d, cq); }
+                    for (int j = 0; j < 16; ++j) {
+                        const uint64_t d = f2_add(v[j], ncm2);
+                        q2 = f2_fma(d, d, q2);
+                    }
+                    const float2 qf = f2_split(q2);
+                    const float cq = qf.x + qf.y;
                     if (c == 0) { mean = cm; m2 = cq; }
                     else chan_merge(mean, m2, 32.f * c, cm, cq, 32.f);
                     // output z * gamma of the LayerNorm that will normalize z
@@ -431,20 +494,21 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const float4 g = __ldg(og4 + q);
-                        v[4 * q + 0] *= g.x; v[4 * q + 1] *= g.y; v[4 * q + 2] *= g.z; v[4 * q + 3] *= g.w;
+                        v[2 * q] = f2_mul(v[2 * q], f2_make(g.x, g.y));
+                        v[2 * q + 1] = f2_mul(v[2 * q + 1], f2_make(g.z, g.w));
                     }
                 }
                 if (kScatter) {
                     if (dst >= 0) store_bf16x32(p.out + (size_t)dst * p.ld_out + col0, v);
                 } else if (kRes) {
-                    stage_and_store(stg, v, &tmOut, col0, tile_row, lane, false);
+                    stage_and_store((c & 1) ? stg2 : stg, v, &tmOut, col0, tile_row, lane, true);
                 } else {
                     // the residual tile is free here: alternate the two staging tiles
                     stage_and_store((c & 1) ? rstg : stg, v, &tmOut, col0, tile_row, lane, true);
                 }
             }
             if (!ok) break;
-            if (kRes) p.out_stats[(size_t)row * LN_PARTS + n * 2 + half] = make_float2(mean, m2);
+            if (kRes && row < p.rows_cap) p.out_stats[(size_t)row * LN_PARTS + n * 2 + half] = make_float2(mean, m2);
             ++acc;
         }
         // outstanding copies finish before the CTA's shared memory goes away
@@ -453,46 +517,117 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         __syncwarp();
     }
 
-    __syncthreads();
+    // A pair's CTAs leave together: rank 1's shared memory and tensor memory are
+    // operands of rank 0's MMAs, and its epilogue arrives on rank 0's barriers.
+    tc_fence_before();
+    if (PAIR) cluster_sync();
+    else __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        if (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+        else tmem_dealloc(tmem_base, TMEM_COLS);
     }
     if (threadIdx.x == 0 && *sm.abort_flag) set_status(p.status, kStatusTimeout);
 }
 
 }  // namespace
 
-int gemm_grid(int epi, int rows_cap, int N, int num_sms) {
+bool gemm_use_pair(int rows_cap, int variant) {
+    if (variant == kGemmPair) return true;
+    if (variant == kGemmSingle) return false;
+    return rows_cap > BM;
+}
+
+template <int EPI, bool PAIR>
+static cudaError_t configure(int smem) {
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_bf16_kernel<EPI, PAIR>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    return cudaSuccess;
+}
+
+// Clusters of two GEMM CTAs that fit on the device at once (every epilogue
+// instance has the same footprint), per device.
+static int pair_clusters(int num_sms) {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return num_sms / 2;
+    if (cached[dev] > 0) return cached[dev];
+    int n = 0;
+    if (configure<kEpiBias, true>(Plan<kEpiBias, true>::SMEM) == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2 * (num_sms / 2));
+        cfg.blockDim = dim3(THREADS);
+        cfg.dynamicSmemBytes = Plan<kEpiBias, true>::SMEM;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_bf16_kernel<kEpiBias, true>, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();
+    if (n <= 0 || n > num_sms / 2) n = num_sms / 2;
+    cached[dev] = n;
+    return n;
+}
+
+int gemm_grid(int epi, int rows_cap, int N, int num_sms, int variant) {
     (void)epi;
+    if (gemm_use_pair(rows_cap, variant)) {
+        const int units = ((rows_cap + 2 * BM - 1) / (2 * BM)) * (N / BN);
+        const int clusters = pair_clusters(num_sms);
+        return 2 * (units < clusters ? (units > 0 ? units : 1) : clusters);
+    }
     const int units = ((rows_cap + BM - 1) / BM) * (N / BN);
     return units < num_sms ? (units > 0 ? units : 1) : num_sms;
 }
 
 template <int EPI>
 static cudaError_t launch_one(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
-                              const CUtensorMap &tmRes, const GemmArgs &a, int grid, cudaStream_t s) {
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_bf16_kernel<EPI>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+                              const CUtensorMap &tmRes, const GemmArgs &a, int grid, cudaStream_t s, bool pair) {
+    if (!pair) {
+        constexpr int smem = Plan<EPI, false>::SMEM;
+        cudaError_t e = configure<EPI, false>(smem);
         if (e != cudaSuccess) return e;
-        configured = true;
+        gemm_bf16_kernel<EPI, false><<<grid, THREADS, smem, s>>>(tmA, tmB, tmOut, tmRes, a);
+        return cudaGetLastError();
     }
-    gemm_bf16_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmB, tmOut, tmRes, a);
-    return cudaGetLastError();
+    if (grid < 2 || grid % 2) return cudaErrorInvalidConfiguration;
+    cudaError_t e = configure<EPI, true>(Plan<EPI, true>::SMEM);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = Plan<EPI, true>::SMEM;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_bf16_kernel<EPI, true>, tmA, tmB, tmOut, tmRes, a);
 }
 
 cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
-                        const CUtensorMap &tmRes, const GemmArgs &a, int grid, cudaStream_t s) {
+                        const CUtensorMap &tmRes, const GemmArgs &a, int grid, cudaStream_t s, int variant) {
+    const bool pair = gemm_use_pair(a.rows_cap, variant);
     switch (epi) {
-        case kEpiBias: return launch_one<kEpiBias>(tmA, tmB, tmOut, tmRes, a, grid, s);
-        case kEpiGelu: return launch_one<kEpiGelu>(tmA, tmB, tmOut, tmRes, a, grid, s);
-        case kEpiResStats: return launch_one<kEpiResStats>(tmA, tmB, tmOut, tmRes, a, grid, s);
-        case kEpiScatter: return launch_one<kEpiScatter>(tmA, tmB, tmOut, tmRes, a, grid, s);
-        case kEpiLnIn: return launch_one<kEpiLnIn>(tmA, tmB, tmOut, tmRes, a, grid, s);
-        case kEpiLnInGelu: return launch_one<kEpiLnInGelu>(tmA, tmB, tmOut, tmRes, a, grid, s);
-        case kEpiLnInScatter: return launch_one<kEpiLnInScatter>(tmA, tmB, tmOut, tmRes, a, grid, s);
+        case kEpiBias: return launch_one<kEpiBias>(tmA, tmB, tmOut, tmRes, a, grid, s, pair);
+        case kEpiGelu: return launch_one<kEpiGelu>(tmA, tmB, tmOut, tmRes, a, grid, s, pair);
+        case kEpiResStats: return launch_one<kEpiResStats>(tmA, tmB, tmOut, tmRes, a, grid, s, pair);
+        case kEpiScatter: return launch_one<kEpiScatter>(tmA, tmB, tmOut, tmRes, a, grid, s, pair);
+        case kEpiLnIn: return launch_one<kEpiLnIn>(tmA, tmB, tmOut, tmRes, a, grid, s, pair);
+        case kEpiLnInGelu: return launch_one<kEpiLnInGelu>(tmA, tmB, tmOut, tmRes, a, grid, s, pair);
+        case kEpiLnInScatter: return launch_one<kEpiLnInScatter>(tmA, tmB, tmOut, tmRes, a, grid, s, pair);
     }
     return cudaErrorInvalidValue;
 }

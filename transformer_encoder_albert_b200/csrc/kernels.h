@@ -32,17 +32,20 @@ enum GemmEpi : int {
 };
 
 namespace gemm {
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int STAGES = 4;       // one CTA per tile: {A 128x64, B 256x64} per stage
+constexpr int PAIR_STAGES = 6;  // CTA pair per 256x256 tile: {A 128x64, B 128x64} per CTA and stage
+constexpr int B_BOX = 128;      // rows of B per TMA box (weight tensor maps)
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
+constexpr int B_HALF_BYTES = B_BOX * BK * 2;
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 32 * (2 + EPI_WARPS);
 constexpr int TMEM_COLS = 512;
 constexpr int LN_N = 768;     // LayerNorm row width
 constexpr int LN_PARTS = 6;   // partial statistics per row (128 columns each)
 constexpr int STG_BYTES = 32 * 32 * 2;  // one 32x32 bf16 staging tile
-// stages + per-warp output staging + per-warp residual staging + control, 1 KiB aligned
-constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES) + 2 * EPI_WARPS * STG_BYTES + 1024;
+
 }  // namespace gemm
 
 struct GemmArgs {
@@ -68,15 +71,23 @@ struct GemmArgs {
 };
 
 // Encode a 2-D bf16 row-major [rows, cols] tensor map with a {64, box_rows}
-// box and the 128-byte swizzle.  Returns 0 on success.
+// box and the 128-byte swizzle (box_rows = BM for A operands, B_BOX for
+// weights).  Returns 0 on success.
 int make_tmap_bf16(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols,
                    uint32_t box_rows);
 // Map of a bf16 row-major [rows, cols] tensor with a 32x32 box and the 64-byte
 // swizzle: the epilogue's output stores and residual loads.
 int make_tmap_bf16_tile32(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols);
 
-// Grid the GEMM uses for this many rows (persistent: <= number of SMs).
-int gemm_grid(int epi, int rows_cap, int N, int num_sms);
+// Kernel variant: one CTA per 128x256 tile, or a CTA pair (cluster of 2,
+// tcgen05.mma cta_group::2) per 256x256 tile.  Auto takes the pair whenever
+// the A buffer holds more than one 128-row block.
+enum GemmVariant { kGemmAuto = 0, kGemmSingle = 1, kGemmPair = 2 };
+bool gemm_use_pair(int rows_cap, int variant);
+
+// Grid (CTAs) the GEMM uses for this many rows: persistent, at most one CTA per
+// SM, and for the pair variant an even count within the co-resident clusters.
+int gemm_grid(int epi, int rows_cap, int N, int num_sms, int variant = kGemmAuto);
 
 // The epilogue reads its per-column vectors as float4: each must be 16-byte aligned.
 inline bool gemm_vectors_aligned(const GemmArgs &a) {
@@ -87,7 +98,8 @@ inline bool gemm_vectors_aligned(const GemmArgs &a) {
 // tmOut: tile32 map of the output (unused by the scatter epilogues); tmRes: tile32
 // map of the residual (kEpiResStats only; pass any valid map otherwise).
 cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
-                        const CUtensorMap &tmRes, const GemmArgs &args, int grid, cudaStream_t s);
+                        const CUtensorMap &tmRes, const GemmArgs &args, int grid, cudaStream_t s,
+                        int variant = kGemmAuto);
 
 // ---------------------------------------------------------------- attention --
 // Masked bidirectional attention, bf16 tensor-core kernel (mma.sync m16n8k16).

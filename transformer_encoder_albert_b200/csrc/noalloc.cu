@@ -89,7 +89,7 @@ extern "C" int albert_gemm_residual_ln_noalloc(const void *A, const void *W, con
     const int rows_cap = (M + gemm::BM - 1) / gemm::BM * gemm::BM;
     const int grid = gemm_grid(kEpiResStats, rows_cap, N, sms);
     CUtensorMap ta, tb, to, tr;
-    if (make_tmap_bf16(&ta, A, M, K, gemm::BM) || make_tmap_bf16(&tb, W, N, K, gemm::BN) ||
+    if (make_tmap_bf16(&ta, A, M, K, gemm::BM) || make_tmap_bf16(&tb, W, N, K, gemm::B_BOX) ||
         make_tmap_bf16_tile32(&to, zg, rows_cap, N) || make_tmap_bf16_tile32(&tr, R, M, N))
         return ALBERT_ERR_CUDA;
 
