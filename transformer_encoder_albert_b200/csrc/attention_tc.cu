@@ -8,9 +8,12 @@
 // key u of sequence b takes part iff u < L_b, every query sees both sides.
 //
 // One work item = (sequence, head), all L_b <= 128 queries and keys at once:
-//   warp 0      : TMA producer: the head's Q, K and V tiles (128 or 64 rows x
-//                 64, 128-byte swizzle) from the packed [rows, 3*768] buffer
-//                 into a ring of four shared stages;
+//   warp 0      : TMA producer, an event loop over two rings of shared
+//                 stages: the head's Q and K tiles (128 or 64 rows x 64,
+//                 128-byte swizzle) from the packed [rows, 3*768] buffer into
+//                 one, its V tile into the other.  A Q/K stage is free again
+//                 as soon as the S product has read it, so Q/K loads run well
+//                 ahead; a V stage lives until the O product;
 //   warp 1      : tcgen05.mma issuer, an event loop that issues whichever is
 //                 ready: S = Q K^T (M=128, N=128 or 64, K=64) into a TMEM
 //                 buffer, or O = P V (M=128, N=64, K = L rounded up to 16) with
@@ -38,33 +41,38 @@ namespace {
 
 constexpr int TROWS = 128;                     // query rows / keys per item
 constexpr int TILE = TROWS * 128;              // 128 rows x 64 bf16 = 16 KB
-constexpr int STAGE = 3 * TILE;                // Q, K, V
-constexpr int NSTAGE = 4;                      // shared-memory stages
+constexpr int NQK = 4;                         // Q/K stages (2 tiles each)
+constexpr int NV = 4;                          // V stages (1 tile each)
 constexpr int NBUF = 4;                        // TMEM item buffers (128 columns each)
 constexpr int ATC_THREADS = 32 * 14;
-constexpr int ATC_SMEM = 1024 + NSTAGE * STAGE + 512 + NBUF * TROWS * 4;
+constexpr int ATC_SMEM = 1024 + (2 * NQK + NV) * TILE + NBUF * TROWS * 4 + 512;
 constexpr uint32_t TM_O = 64;                  // O's first column within an item buffer
 
 struct AttSmem {
-    uint8_t *stage;
-    uint64_t *ld_full, *ld_empty;              // [NSTAGE]
+    uint8_t *qk, *v;                           // [NQK][Q tile, K tile], [NV][V tile]
+    uint64_t *qk_full, *qk_empty;              // [NQK]
+    uint64_t *v_full, *v_empty;                // [NV]
     uint64_t *s_full, *p_full, *o_full, *o_empty;  // [NBUF]
     uint64_t *drain;
     uint32_t *tmem_slot;
     volatile int *abort_flag;
     int *misc;
+    int *qk_len, *v_len;                       // length of the item a stage holds
     float *inv_sum;                            // [NBUF][TROWS]
 };
 
 __device__ __forceinline__ AttSmem att_carve(uint8_t *raw) {
     AttSmem s;
     uint8_t *p = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
-    s.stage = p;
-    s.inv_sum = reinterpret_cast<float *>(p + NSTAGE * STAGE);
-    uint64_t *b = reinterpret_cast<uint64_t *>(p + NSTAGE * STAGE + NBUF * TROWS * 4);
-    s.ld_full = b;
-    s.ld_empty = b + NSTAGE;
-    s.s_full = b + 2 * NSTAGE;
+    s.qk = p;
+    s.v = p + 2 * NQK * TILE;
+    s.inv_sum = reinterpret_cast<float *>(s.v + NV * TILE);
+    uint64_t *b = reinterpret_cast<uint64_t *>(s.v + NV * TILE + NBUF * TROWS * 4);
+    s.qk_full = b;
+    s.qk_empty = b + NQK;
+    s.v_full = b + 2 * NQK;
+    s.v_empty = b + 2 * NQK + NV;
+    s.s_full = b + 2 * NQK + 2 * NV;
     s.p_full = s.s_full + NBUF;
     s.o_full = s.s_full + 2 * NBUF;
     s.o_empty = s.s_full + 3 * NBUF;
@@ -73,6 +81,8 @@ __device__ __forceinline__ AttSmem att_carve(uint8_t *raw) {
     s.tmem_slot = u;
     s.abort_flag = reinterpret_cast<volatile int *>(u + 1);
     s.misc = reinterpret_cast<int *>(u + 2);
+    s.qk_len = s.misc + 2;
+    s.v_len = s.qk_len + NQK;
     return s;
 }
 
@@ -87,9 +97,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     if (threadIdx.x == 0) {
         sm.misc[0] = *reinterpret_cast<const volatile int *>(status);
         *sm.abort_flag = 0;
-        for (int i = 0; i < NSTAGE; ++i) {
-            mbar_init(smem_u32(&sm.ld_full[i]), 1);
-            mbar_init(smem_u32(&sm.ld_empty[i]), 1);
+        for (int i = 0; i < NQK; ++i) {
+            mbar_init(smem_u32(&sm.qk_full[i]), 1);
+            mbar_init(smem_u32(&sm.qk_empty[i]), 1);
+        }
+        for (int i = 0; i < NV; ++i) {
+            mbar_init(smem_u32(&sm.v_full[i]), 1);
+            mbar_init(smem_u32(&sm.v_empty[i]), 1);
         }
         for (int i = 0; i < NBUF; ++i) {
             mbar_init(smem_u32(&sm.s_full[i]), 1);
@@ -116,33 +130,64 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     const uint32_t tmem_base = *sm.tmem_slot;
     const int total = nseq * kHeads;  // item id = b * 12 + h
 
+    int n_items = 0;  // items of this CTA: id = blockIdx.x + j * gridDim.x
+    for (int id = blockIdx.x; id < total; id += gridDim.x) ++n_items;
+
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer --
+        // Event loop: Q/K of item nq into its ring, V of item nv (< nq) into its
+        // ring, whichever has a free stage.
         if (lane == 0) {
-            int i = 0, issued = 0;
-            bool ok = true;
-            for (int id = blockIdx.x; id < total && ok; id += gridDim.x, ++i) {
-                const int st = i % NSTAGE;
-                const uint32_t ph = (i / NSTAGE) & 1;
-                if (!mbar_wait(smem_u32(&sm.ld_empty[st]), ph ^ 1, sm.abort_flag)) { ok = false; break; }
-                const int b = id / kHeads, h = id % kHeads;
-                const int start = __ldg(seq_start + b);
-                // sequences of at most 64 tokens move 64-row tiles
-                const bool short_seq = __ldg(seq_len + b) <= 64;
-                const CUtensorMap *tm = short_seq ? &tmQKV64 : &tmQKV;
-                const uint32_t dst = smem_u32(sm.stage + st * STAGE);
-                const uint32_t fb = smem_u32(&sm.ld_full[st]);
-                mbar_arrive_expect_tx(fb, short_seq ? 3 * TILE / 2 : 3 * TILE);
-                tma_load_2d(dst, tm, fb, h * kHeadDim, start);
-                tma_load_2d(dst + TILE, tm, fb, kHidden + h * kHeadDim, start);
-                tma_load_2d(dst + 2 * TILE, tm, fb, 2 * kHidden + h * kHeadDim, start);
-                ++issued;
-            }
-            if (!ok) {
-                for (int k = 0; k < NSTAGE && k < issued; ++k) {
-                    const int j = issued - 1 - k;
-                    mbar_wait_drain(smem_u32(&sm.ld_full[j % NSTAGE]), (j / NSTAGE) & 1);
+            int nq = 0, nv = 0;
+            unsigned long long t_idle = 0;
+            while (nv < n_items) {
+                bool progress = false;
+                if (nq < n_items) {
+                    const int st = nq % NQK;
+                    if (mbar_test(smem_u32(&sm.qk_empty[st]), ((nq / NQK) & 1) ^ 1)) {
+                        const int id = blockIdx.x + nq * gridDim.x, b = id / kHeads, h = id % kHeads;
+                        const int start = __ldg(seq_start + b), L = __ldg(seq_len + b);
+                        sm.qk_len[st] = L;  // read by the issuer once the stage is full
+                        // sequences of at most 64 tokens move 64-row tiles
+                        const CUtensorMap *tm = L <= 64 ? &tmQKV64 : &tmQKV;
+                        const uint32_t dst = smem_u32(sm.qk + st * 2 * TILE);
+                        const uint32_t fb = smem_u32(&sm.qk_full[st]);
+                        mbar_arrive_expect_tx(fb, L <= 64 ? TILE : 2 * TILE);
+                        tma_load_2d(dst, tm, fb, h * kHeadDim, start);
+                        tma_load_2d(dst + TILE, tm, fb, kHidden + h * kHeadDim, start);
+                        ++nq;
+                        progress = true;
+                    }
                 }
+                if (nv < nq) {
+                    const int st = nv % NV;
+                    if (mbar_test(smem_u32(&sm.v_empty[st]), ((nv / NV) & 1) ^ 1)) {
+                        const int id = blockIdx.x + nv * gridDim.x, b = id / kHeads, h = id % kHeads;
+                        const int start = __ldg(seq_start + b), L = __ldg(seq_len + b);
+                        sm.v_len[st] = L;
+                        const CUtensorMap *tm = L <= 64 ? &tmQKV64 : &tmQKV;
+                        const uint32_t fb = smem_u32(&sm.v_full[st]);
+                        mbar_arrive_expect_tx(fb, L <= 64 ? TILE / 2 : TILE);
+                        tma_load_2d(smem_u32(sm.v + st * TILE), tm, fb, 2 * kHidden + h * kHeadDim, start);
+                        ++nv;
+                        progress = true;
+                    }
+                }
+                if (progress) {
+                    t_idle = 0;
+                } else {
+                    if (*sm.abort_flag) break;
+                    const unsigned long long now = globaltimer_ns();
+                    if (t_idle == 0) t_idle = now;
+                    else if (now - t_idle > kWaitLimitNs) { *sm.abort_flag = 1; break; }
+                }
+            }
+            if (*sm.abort_flag) {
+                // loads still in flight complete before the CTA's shared memory goes away
+                for (int j = nq > NQK ? nq - NQK : 0; j < nq; ++j)
+                    mbar_wait_drain(smem_u32(&sm.qk_full[j % NQK]), (j / NQK) & 1);
+                for (int j = nv > NV ? nv - NV : 0; j < nv; ++j)
+                    mbar_wait_drain(smem_u32(&sm.v_full[j % NV]), (j / NV) & 1);
             }
         }
     } else if (warp == 1) {
@@ -153,19 +198,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
             const uint32_t idesc_s128 = idesc_bf16_f32(TROWS, TROWS);
             const uint32_t idesc_s64 = idesc_bf16_f32(TROWS, 64);
             const uint32_t idesc_o = idesc_bf16_f32(TROWS, kHeadDim) | (1u << 16);  // B (= V) MN-major
-            int n_items = 0;
-            for (int id = blockIdx.x; id < total; id += gridDim.x) ++n_items;
             int ns = 0, no = 0;  // next S product, next O product
             unsigned long long t_idle = 0;
             while (no < n_items) {
                 bool progress = false;
                 if (no < ns) {
-                    const int tb = no % NBUF, st = no % NSTAGE;
-                    if (mbar_test(smem_u32(&sm.p_full[tb]), (no / NBUF) & 1)) {
+                    const int tb = no % NBUF, st = no % NV;
+                    if (mbar_test(smem_u32(&sm.p_full[tb]), (no / NBUF) & 1) &&
+                        mbar_test(smem_u32(&sm.v_full[st]), (no / NV) & 1)) {
                         tc_fence_after();
-                        const int L = __ldg(seq_len + (blockIdx.x + no * gridDim.x) / kHeads);
+                        const int L = sm.v_len[st];
                         const int ksteps = (L + 15) >> 4;
-                        const uint32_t vbase = smem_u32(sm.stage + st * STAGE + 2 * TILE);
+                        const uint32_t vbase = smem_u32(sm.v + st * TILE);
                         const uint32_t buf = tmem_base + tb * TROWS;
                         for (int kk = 0; kk < ksteps; ++kk) {
                             // P: 16 keys = 8 packed TMEM columns; V: 16 keys = 16 rows of 128 B
@@ -173,24 +217,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                                          kk != 0);
                         }
                         umma_commit(smem_u32(&sm.o_full[tb]));
-                        umma_commit(smem_u32(&sm.ld_empty[st]));  // Q, K, V consumed: stage free
+                        umma_commit(smem_u32(&sm.v_empty[st]));  // V consumed: stage free
                         ++no;
                         progress = true;
                     }
                 }
                 if (ns < n_items && ns < no + NBUF) {
-                    const int tb = ns % NBUF, st = ns % NSTAGE;
+                    const int tb = ns % NBUF, st = ns % NQK;
                     // the buffer is free once the output group has read item ns - NBUF
-                    if (mbar_test(smem_u32(&sm.ld_full[st]), (ns / NSTAGE) & 1) &&
+                    if (mbar_test(smem_u32(&sm.qk_full[st]), (ns / NQK) & 1) &&
                         mbar_test(smem_u32(&sm.o_empty[tb]), ((ns / NBUF) & 1) ^ 1)) {
                         tc_fence_after();
-                        const int L = __ldg(seq_len + (blockIdx.x + ns * gridDim.x) / kHeads);
-                        const uint32_t q = smem_u32(sm.stage + st * STAGE), k = q + TILE;
+                        const int L = sm.qk_len[st];
+                        const uint32_t q = smem_u32(sm.qk + st * 2 * TILE), k = q + TILE;
 #pragma unroll
                         for (int kk = 0; kk < kHeadDim / 16; ++kk)
                             umma_bf16(tmem_base + tb * TROWS, sw128_kmajor_desc(q + kk * 32),
                                       sw128_kmajor_desc(k + kk * 32), L <= 64 ? idesc_s64 : idesc_s128, kk != 0);
                         umma_commit(smem_u32(&sm.s_full[tb]));
+                        umma_commit(smem_u32(&sm.qk_empty[st]));  // Q, K consumed: stage free
                         ++ns;
                         progress = true;
                     }
@@ -230,9 +275,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
             if (live) {
                 // pass 1: row maximum over the valid keys (two 32-key chunks per TMEM wait)
                 float m = -INFINITY;
+                uint32_t v[2][32];
 #pragma unroll 1
                 for (int c = 0; c < nch; c += 2) {
-                    uint32_t v[2][32];
                     tmem_ld32(srow + c * 32, v[0]);
                     if (c + 1 < nch) tmem_ld32(srow + (c + 1) * 32, v[1]);
                     tmem_ld_wait();
@@ -250,10 +295,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                 float l = 0.f;
 #pragma unroll 1
                 for (int c = 0; c < nch; c += 2) {
-                    uint32_t v[2][32];
-                    tmem_ld32(srow + c * 32, v[0]);
-                    if (c + 1 < nch) tmem_ld32(srow + (c + 1) * 32, v[1]);
-                    tmem_ld_wait();
+                    if (nch > 2) {  // up to 64 keys the row is still in registers
+                        tmem_ld32(srow + c * 32, v[0]);
+                        if (c + 1 < nch) tmem_ld32(srow + (c + 1) * 32, v[1]);
+                        tmem_ld_wait();
+                    }
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int cc = c + e;
