@@ -140,6 +140,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
         if (lane == 0) {
             int nq = 0, nv = 0;
             unsigned long long t_idle = 0;
+            unsigned polls = 0;
             while (nv < n_items) {
                 bool progress = false;
                 if (nq < n_items) {
@@ -175,7 +176,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                 }
                 if (progress) {
                     t_idle = 0;
-                } else {
+                } else if ((++polls & 255) == 0) {  // the timer read is slow: not on every poll
                     if (*sm.abort_flag) break;
                     const unsigned long long now = globaltimer_ns();
                     if (t_idle == 0) t_idle = now;
@@ -200,6 +201,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
             const uint32_t idesc_o = idesc_bf16_f32(TROWS, kHeadDim) | (1u << 16);  // B (= V) MN-major
             int ns = 0, no = 0;  // next S product, next O product
             unsigned long long t_idle = 0;
+            unsigned polls = 0;
             while (no < n_items) {
                 bool progress = false;
                 if (no < ns) {
@@ -242,7 +244,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                 }
                 if (progress) {
                     t_idle = 0;
-                } else {
+                } else if ((++polls & 255) == 0) {  // the timer read is slow: not on every poll
                     if (*sm.abort_flag) break;
                     const unsigned long long now = globaltimer_ns();
                     if (t_idle == 0) t_idle = now;
@@ -274,7 +276,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
             tc_fence_after();
             if (live) {
                 // pass 1: row maximum over the valid keys (two 32-key chunks per TMEM wait)
-                float m = -INFINITY;
+                // (four independent max / sum chains: a single chain is latency-bound)
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
                 uint32_t v[2][32];
 #pragma unroll 1
                 for (int c = 0; c < nch; c += 2) {
@@ -283,16 +286,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                     tmem_ld_wait();
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
+                        const int base = (c + e) * 32;
                         if (c + e >= nch) continue;
+                        if (base + 32 <= L) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if ((c + e) * 32 + j < L) m = fmaxf(m, __uint_as_float(v[e][j]));
+                            for (int j = 0; j < 32; ++j) mx[j & 3] = fmaxf(mx[j & 3], __uint_as_float(v[e][j]));
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (base + j < L) mx[j & 3] = fmaxf(mx[j & 3], __uint_as_float(v[e][j]));
+                        }
                     }
                 }
+                const float m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
                 // pass 2: P = exp(scale * (s - max)) packed as bf16 pairs; chunk c goes to
                 // columns 16c..16c+15 of the same buffer, which hold scores already read
-                const float ms = m * sl2;
-                float l = 0.f;
+                const uint64_t sl2x2 = f2_make(sl2, sl2), nms2 = f2_make(-m * sl2, -m * sl2);
+                uint64_t lsum[2] = {f2_make(0.f, 0.f), f2_make(0.f, 0.f)};
 #pragma unroll 1
                 for (int c = 0; c < nch; c += 2) {
                     if (nch > 2) {  // up to 64 keys the row is still in registers
@@ -304,20 +314,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                     for (int e = 0; e < 2; ++e) {
                         const int cc = c + e;
                         if (cc >= nch) continue;
+                        const bool full = cc * 32 + 32 <= L;
                         uint32_t pk[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int k0 = cc * 32 + 2 * j;
-                            const float p0 = k0 < L ? ex2_approx(fmaf(__uint_as_float(v[e][2 * j]), sl2, -ms)) : 0.f;
-                            const float p1 = k0 + 1 < L ? ex2_approx(fmaf(__uint_as_float(v[e][2 * j + 1]), sl2, -ms)) : 0.f;
-                            l += p0 + p1;
+                            const float2 x = f2_split(f2_fma(f2_make_u(v[e][2 * j], v[e][2 * j + 1]), sl2x2, nms2));
+                            float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+                            if (!full) {
+                                p0 = k0 < L ? p0 : 0.f;
+                                p1 = k0 + 1 < L ? p1 : 0.f;
+                            }
+                            lsum[j & 1] = f2_add(lsum[j & 1], f2_make(p0, p1));
                             pk[j] = pack_bf16x2(p0, p1);
                         }
                         tmem_st16(srow + cc * 16, pk);
                     }
                 }
+                const float2 ls = f2_split(f2_add(lsum[0], lsum[1]));
                 // read by the output group after it has waited on p_full
-                sm.inv_sum[tb * TROWS + r] = 1.f / l;
+                sm.inv_sum[tb * TROWS + r] = 1.f / (ls.x + ls.y);
                 tmem_st_wait();
             }
             tc_fence_before();
