@@ -51,10 +51,15 @@ using namespace gemm;
 template <int EPI, bool PAIR>
 struct Plan {
     static constexpr bool kRes = EPI == kEpiResStats;
-    static constexpr int NST = (PAIR ? PAIR_STAGES : STAGES) - (kRes ? 1 : 0);
+    static constexpr bool kLnIn = EPI == kEpiLnIn || EPI == kEpiLnInGelu || EPI == kEpiLnInScatter;
+    static constexpr int NST = PAIR ? PAIR_STAGES - 1 : STAGES - 1;
     static constexpr int BSTAGE = PAIR ? B_HALF_BYTES : B_BYTES;
     static constexpr int NSTG = kRes ? 3 : 2;
-    static constexpr int SMEM = 1024 + NST * (A_BYTES + BSTAGE) + NSTG * EPI_WARPS * STG_BYTES + 1024;
+    // per-column vectors of a unit: bias, then W gamma (LayerNorm input) or
+    // out_g and res_g (residual epilogue); two buffers (this unit, the next)
+    static constexpr int NVEC = kLnIn ? 2 : (kRes ? 3 : 1);
+    static constexpr int VEC_BYTES = 2 * NVEC * BN * 4;
+    static constexpr int SMEM = 1024 + NST * (A_BYTES + BSTAGE) + NSTG * EPI_WARPS * STG_BYTES + VEC_BYTES + 1024;
     static_assert(SMEM <= 232448, "shared memory per CTA");
 };
 
@@ -63,6 +68,8 @@ struct Smem {
     uint8_t *stg;            // 2 KB output staging tile per epilogue warp
     uint8_t *rstg;           // 2 KB residual (or second output) staging tile per epilogue warp
     uint8_t *stg2;           // residual epilogue: second 2 KB output staging tile per warp
+    float *vec;              // [2][NVEC][BN] per-column vectors of this unit and the next
+    uint64_t *vec_full;      // [2]: a unit's vectors are in shared memory
     uint64_t *full, *empty, *tfull, *tempty, *drain, *rbar;
     uint32_t *tmem_slot;
     volatile int *abort_flag;
@@ -80,7 +87,8 @@ __device__ __forceinline__ Smem carve(uint8_t *raw) {
     s.stg = s.b + NST * P::BSTAGE;
     s.rstg = s.stg + EPI_WARPS * STG_BYTES;
     s.stg2 = s.rstg + EPI_WARPS * STG_BYTES;
-    uint8_t *ctrl = s.stg + P::NSTG * EPI_WARPS * STG_BYTES;
+    s.vec = reinterpret_cast<float *>(s.stg + P::NSTG * EPI_WARPS * STG_BYTES);
+    uint8_t *ctrl = reinterpret_cast<uint8_t *>(s.vec) + P::VEC_BYTES;
     uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl);
     s.full = bars;
     s.empty = bars + NST;
@@ -88,7 +96,8 @@ __device__ __forceinline__ Smem carve(uint8_t *raw) {
     s.tempty = bars + 2 * NST + 2;
     s.drain = bars + 2 * NST + 4;
     s.rbar = bars + 2 * NST + 5;
-    uint32_t *u = reinterpret_cast<uint32_t *>(bars + 2 * NST + 5 + EPI_WARPS);
+    s.vec_full = bars + 2 * NST + 5 + EPI_WARPS;
+    uint32_t *u = reinterpret_cast<uint32_t *>(bars + 2 * NST + 5 + EPI_WARPS + 2);
     s.tmem_slot = u;
     s.abort_flag = reinterpret_cast<volatile int *>(u + 1);
     s.misc = reinterpret_cast<int *>(u + 2);
@@ -208,6 +217,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         mbar_init(smem_u32(sm.drain), 1);
         for (int i = 0; i < EPI_WARPS; ++i) mbar_init(smem_u32(&sm.rbar[i]), 1);
+        // every epilogue thread arrives once it has stored its columns
+        for (int i = 0; i < 2; ++i) mbar_init(smem_u32(&sm.vec_full[i]), 32 * EPI_WARPS);
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -369,6 +380,34 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             }
         };
         if ((kLnIn || res_ln) && slot < units) fetch_stats(slot);
+        // The per-column vectors of each unit are staged in shared memory: every
+        // epilogue thread loads one column of each a unit ahead (registers),
+        // stores it at the end of the current unit, and arrives on vec_full.
+        // (Read from global memory inside the chunk loop, these uniform loads
+        // stalled every chunk on their latency.)
+        constexpr int NVEC = Plan<EPI, PAIR>::NVEC;
+        const int et = ew * 32 + lane;  // 0..255: the column this thread stages
+        float vreg[NVEC];
+        auto vec_load = [&](int un) {
+            const int col = (un % n_sub) * BN + et;
+            vreg[0] = __ldg(p.bias + col);
+            if (kLnIn) vreg[1] = __ldg(p.fold_s + col);
+            if (kRes) {
+                vreg[1] = __ldg(p.out_g + col);
+                vreg[NVEC - 1] = res_ln ? __ldg(p.res_g + col) : 0.f;
+            }
+        };
+        auto vec_store = [&](int b) {
+#pragma unroll
+            for (int i = 0; i < NVEC; ++i) sm.vec[(b * NVEC + i) * BN + et] = vreg[i];
+            mbar_arrive(smem_u32(&sm.vec_full[b]));
+        };
+        if (slot < units) {
+            vec_load(slot);
+            vec_store(0);
+            if (slot + nslots < units) vec_load(slot + nslots);
+        }
+        int j = 0;  // unit iteration of this CTA
         for (int u = slot; u < units && ok; u += nslots) {
             const int m = u / n_sub, n = u % n_sub;
             const int row = m * UM + row_off + r_local;
@@ -385,10 +424,15 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
             const int ab = acc & 1;
             const uint32_t aph = (acc >> 1) & 1;
-            bool got = mbar_wait(smem_u32(&sm.tfull[ab]), aph, sm.abort_flag);
+            const int vb = j & 1;
+            bool got = mbar_wait(smem_u32(&sm.vec_full[vb]), (j >> 1) & 1, sm.abort_flag) &&
+                       mbar_wait(smem_u32(&sm.tfull[ab]), aph, sm.abort_flag);
             got = __all_sync(0xffffffffu, got);
             if (!got) { ok = false; break; }
             tc_fence_after();
+            const float *vbias = sm.vec + (vb * NVEC) * BN + half * 128;
+            const float *vsec = vbias + BN;                 // W gamma or out_g
+            const float *vres = sm.vec + (vb * NVEC + NVEC - 1) * BN + half * 128;  // res_g
             const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + ab * BN + half * 128;
             const int ncol0 = n * BN + half * 128;  // first output column of this warp
             float mean = 0.f, m2 = 0.f;
@@ -421,13 +465,13 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const uint32_t *rc = r[c & 1];
                 const int col0 = ncol0 + c * 32;
                 uint64_t v[16];  // columns col0 + 2j, col0 + 2j + 1
-                const float4 *bias4 = reinterpret_cast<const float4 *>(p.bias + col0);
+                const float4 *bias4 = reinterpret_cast<const float4 *>(vbias + c * 32);
                 if (kLnIn) {
-                    const float4 *s4 = reinterpret_cast<const float4 *>(p.fold_s + col0);
+                    const float4 *s4 = reinterpret_cast<const float4 *>(vsec + c * 32);
                     const uint64_t rstd2 = f2_make(rstd, rstd), nmu2 = f2_make(nmu, nmu);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const float4 bb = __ldg(bias4 + q), ss = __ldg(s4 + q);
+                        const float4 bb = bias4[q], ss = s4[q];
                         v[2 * q] = f2_fma(rstd2, f2_make_u(rc[4 * q], rc[4 * q + 1]),
                                           f2_fma(nmu2, f2_make(ss.x, ss.y), f2_make(bb.x, bb.y)));
                         v[2 * q + 1] = f2_fma(rstd2, f2_make_u(rc[4 * q + 2], rc[4 * q + 3]),
@@ -436,7 +480,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 } else {
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const float4 bb = __ldg(bias4 + q);
+                        const float4 bb = bias4[q];
                         v[2 * q] = f2_add(f2_make_u(rc[4 * q], rc[4 * q + 1]), f2_make(bb.x, bb.y));
                         v[2 * q + 1] = f2_add(f2_make_u(rc[4 * q + 2], rc[4 * q + 3]), f2_make(bb.z, bb.w));
                     }
@@ -460,11 +504,11 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     if (c < 3) res_issue(u, c + 1);
                     else if (u + nslots < units) res_issue(u + nslots, 0);
                     if (res_ln) {
-                        const float4 *rg4 = reinterpret_cast<const float4 *>(p.res_g + col0);
+                        const float4 *rg4 = reinterpret_cast<const float4 *>(vres + c * 32);
                         const uint64_t rrstd2 = f2_make(rrstd, rrstd), rnmu2 = f2_make(rnmu, rnmu);
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
-                            const float4 g = __ldg(rg4 + q);
+                            const float4 g = rg4[q];
                             v[2 * q] = f2_fma(rrstd2, x[2 * q], f2_fma(rnmu2, f2_make(g.x, g.y), v[2 * q]));
                             v[2 * q + 1] = f2_fma(rrstd2, x[2 * q + 1], f2_fma(rnmu2, f2_make(g.z, g.w), v[2 * q + 1]));
                         }
@@ -490,10 +534,10 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     if (c == 0) { mean = cm; m2 = cq; }
                     else chan_merge(mean, m2, 32.f * c, cm, cq, 32.f);
                     // output z * gamma of the LayerNorm that will normalize z
-                    const float4 *og4 = reinterpret_cast<const float4 *>(p.out_g + col0);
+                    const float4 *og4 = reinterpret_cast<const float4 *>(vsec + c * 32);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const float4 g = __ldg(og4 + q);
+                        const float4 g = og4[q];
                         v[2 * q] = f2_mul(v[2 * q], f2_make(g.x, g.y));
                         v[2 * q + 1] = f2_mul(v[2 * q + 1], f2_make(g.z, g.w));
                     }
@@ -510,6 +554,13 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             if (!ok) break;
             if (kRes && row < p.rows_cap) p.out_stats[(size_t)row * LN_PARTS + n * 2 + half] = make_float2(mean, m2);
             ++acc;
+            // the next unit's vectors: buffer (j + 1) & 1 was last read in unit j - 1,
+            // which every epilogue thread finished before arriving for unit j
+            if (u + nslots < units) {
+                vec_store((j + 1) & 1);
+                if (u + 2 * nslots < units) vec_load(u + 2 * nslots);
+            }
+            ++j;
         }
         // outstanding copies finish before the CTA's shared memory goes away
         if (lane == 0) bulk_wait0();

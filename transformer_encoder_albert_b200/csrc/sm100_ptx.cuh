@@ -209,6 +209,11 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
     return p;
 }
 
+// Bring the 128-byte line holding p into L1 (no register result, no wait).
+__device__ __forceinline__ void prefetch_l1(const void *p) {
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
