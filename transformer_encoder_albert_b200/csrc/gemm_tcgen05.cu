@@ -127,6 +127,11 @@ __device__ __forceinline__ uint32_t stg_off(int r, int q) {
 __device__ __forceinline__ void st_shared_v4(uint32_t a, uint4 v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a) : "memory");
+    return v;
+}
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
     uint4 v;
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a) : "memory");
@@ -306,7 +311,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             for (int u = slot; u < units && ok; u += nslots) {
                 const int ab = acc & 1;
                 const uint32_t aph = (acc >> 1) & 1;
-                if (!mbar_wait<PAIR>(smem_u32(&sm.tempty[ab]), aph ^ 1, sm.abort_flag)) break;
+                if (!mbar_wait(smem_u32(&sm.tempty[ab]), aph ^ 1, sm.abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + ab * BN;
                 for (int kb = 0; kb < kblocks; ++kb) {
@@ -430,9 +435,10 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             got = __all_sync(0xffffffffu, got);
             if (!got) { ok = false; break; }
             tc_fence_after();
-            const float *vbias = sm.vec + (vb * NVEC) * BN + half * 128;
-            const float *vsec = vbias + BN;                 // W gamma or out_g
-            const float *vres = sm.vec + (vb * NVEC + NVEC - 1) * BN + half * 128;  // res_g
+            // shared addresses of this warp's 128 columns of each vector
+            const uint32_t vbias = smem_u32(sm.vec + (vb * NVEC) * BN + half * 128);
+            const uint32_t vsec = vbias + BN * 4;           // W gamma or out_g
+            const uint32_t vres = smem_u32(sm.vec + (vb * NVEC + NVEC - 1) * BN + half * 128);  // res_g
             const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + ab * BN + half * 128;
             const int ncol0 = n * BN + half * 128;  // first output column of this warp
             float mean = 0.f, m2 = 0.f;
@@ -465,13 +471,13 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const uint32_t *rc = r[c & 1];
                 const int col0 = ncol0 + c * 32;
                 uint64_t v[16];  // columns col0 + 2j, col0 + 2j + 1
-                const float4 *bias4 = reinterpret_cast<const float4 *>(vbias + c * 32);
+                const uint32_t bias4 = vbias + c * 128;  // 32 floats per chunk
                 if (kLnIn) {
-                    const float4 *s4 = reinterpret_cast<const float4 *>(vsec + c * 32);
+                    const uint32_t s4 = vsec + c * 128;
                     const uint64_t rstd2 = f2_make(rstd, rstd), nmu2 = f2_make(nmu, nmu);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const float4 bb = bias4[q], ss = s4[q];
+                        const float4 bb = ld_shared_f4(bias4 + q * 16), ss = ld_shared_f4(s4 + q * 16);
                         v[2 * q] = f2_fma(rstd2, f2_make_u(rc[4 * q], rc[4 * q + 1]),
                                           f2_fma(nmu2, f2_make(ss.x, ss.y), f2_make(bb.x, bb.y)));
                         v[2 * q + 1] = f2_fma(rstd2, f2_make_u(rc[4 * q + 2], rc[4 * q + 3]),
@@ -480,7 +486,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 } else {
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const float4 bb = bias4[q];
+                        const float4 bb = ld_shared_f4(bias4 + q * 16);
                         v[2 * q] = f2_add(f2_make_u(rc[4 * q], rc[4 * q + 1]), f2_make(bb.x, bb.y));
                         v[2 * q + 1] = f2_add(f2_make_u(rc[4 * q + 2], rc[4 * q + 3]), f2_make(bb.z, bb.w));
                     }
@@ -504,11 +510,11 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     if (c < 3) res_issue(u, c + 1);
                     else if (u + nslots < units) res_issue(u + nslots, 0);
                     if (res_ln) {
-                        const float4 *rg4 = reinterpret_cast<const float4 *>(vres + c * 32);
+                        const uint32_t rg4 = vres + c * 128;
                         const uint64_t rrstd2 = f2_make(rrstd, rrstd), rnmu2 = f2_make(rnmu, rnmu);
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
-                            const float4 g = rg4[q];
+                            const float4 g = ld_shared_f4(rg4 + q * 16);
                             v[2 * q] = f2_fma(rrstd2, x[2 * q], f2_fma(rnmu2, f2_make(g.x, g.y), v[2 * q]));
                             v[2 * q + 1] = f2_fma(rrstd2, x[2 * q + 1], f2_fma(rnmu2, f2_make(g.z, g.w), v[2 * q + 1]));
                         }
@@ -516,28 +522,29 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
                         for (int j = 0; j < 16; ++j) v[j] = f2_add(v[j], x[j]);
                     }
-                    // exact chunk statistics of z, merged into the running ones
-                    uint64_t s2 = v[0];
+                    // exact chunk statistics of z (four independent chains each),
+                    // merged into the running ones
+                    uint64_t s4[4] = {v[0], v[1], v[2], v[3]};
 #pragma unroll
-                    for (int j = 1; j < 16; ++j) s2 = f2_add(s2, v[j]);
-                    const float2 sf = f2_split(s2);
+                    for (int j = 4; j < 16; ++j) s4[j & 3] = f2_add(s4[j & 3], v[j]);
+                    const float2 sf = f2_split(f2_add(f2_add(s4[0], s4[1]), f2_add(s4[2], s4[3])));
                     const float cm = (sf.x + sf.y) * (1.0f / 32.0f);
                     const uint64_t ncm2 = f2_make(-cm, -cm);
-                    uint64_t q2 = f2_make(0.f, 0.f);
+                    uint64_t q4[4];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const uint64_t d = f2_add(v[j], ncm2);
-                        q2 = f2_fma(d, d, q2);
+                        q4[j & 3] = j < 4 ? f2_mul(d, d) : f2_fma(d, d, q4[j & 3]);
                     }
-                    const float2 qf = f2_split(q2);
+                    const float2 qf = f2_split(f2_add(f2_add(q4[0], q4[1]), f2_add(q4[2], q4[3])));
                     const float cq = qf.x + qf.y;
                     if (c == 0) { mean = cm; m2 = cq; }
                     else chan_merge(mean, m2, 32.f * c, cm, cq, 32.f);
                     // output z * gamma of the LayerNorm that will normalize z
-                    const float4 *og4 = reinterpret_cast<const float4 *>(vsec + c * 32);
+                    const uint32_t og4 = vsec + c * 128;
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const float4 g = og4[q];
+                        const float4 g = ld_shared_f4(og4 + q * 16);
                         v[2 * q] = f2_mul(v[2 * q], f2_make(g.x, g.y));
                         v[2 * q + 1] = f2_mul(v[2 * q + 1], f2_make(g.z, g.w));
                     }

@@ -137,9 +137,11 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Arrive (release at cluster scope) on an mbarrier given by shared::cluster address.
+// Arrive on an mbarrier given by shared::cluster address (possibly the peer
+// CTA's), default semantics.  Used to hand tensor memory back to the MMA
+// issuer, with tcgen05.fence::before_thread_sync ahead of it.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 
 // ----------------------------------------------------------------------- TMA --
