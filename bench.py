@@ -60,6 +60,43 @@ def forward_flops(lengths, arch):
     return gemm + arch["n_exec"] * f["attention"], gemm
 
 
+# DRAM traffic per launch of a kernel class, from an ncu capture summarised in
+# profiles/.  A line there records the digest of the kernel's sources at capture
+# time; the figure is reported only while the sources are unchanged.
+TRAFFIC_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
+                            "dram_traffic_b256_T128_packed.txt")
+CLASS_SOURCES = {
+    "gemm": ["gemm_tcgen05.cu", "sm100_ptx.cuh", "kernels.h"],
+    "attention": ["attention_tc.cu", "sm100_ptx.cuh", "kernels.h"],
+}
+
+
+def sources_digest(cls: str) -> str:
+    import hashlib
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "transformer_encoder_albert_b200", "csrc")
+    h = hashlib.sha256()
+    for f in CLASS_SOURCES["gemm" if cls.startswith("gemm_") else "attention"]:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(cls: str, workload: str):
+    """(bytes per launch, note) for a class, or (None, reason)."""
+    try:
+        lines = open(TRAFFIC_FILE).read().splitlines()
+    except OSError:
+        return None, "no ncu capture summarised"
+    want = sources_digest(cls)
+    for ln in lines:
+        kv = dict(x.split("=", 1) for x in ln.split() if "=" in x)
+        if kv.get("class") == cls and kv.get("workload") == workload:
+            if kv.get("sources") != want:
+                return None, "kernel changed since the ncu capture"
+            return float(kv["dram_bytes_per_launch"]), "ncu capture, " + os.path.basename(TRAFFIC_FILE)
+    return None, "class not in the ncu capture"
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -368,8 +405,10 @@ def run_gpu(args):
     peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     dom_ms = dom[1] / max(dom[0], 1)
     achieved = per_launch.get(dominant, 0.0) / (dom_ms / 1000.0) / 1e12
+    traffic, traffic_note = load_traffic(dominant, wl.name + ("_padded" if args.padded else "_packed"))
     roofline = {"kernel": dominant, "bound": "tensor", "achieved": achieved, "peak": peak_sus,
-                "unit": "TFLOP/s", "frac": achieved / peak_sus, "traffic": None,
+                "unit": "TFLOP/s", "frac": achieved / peak_sus, "traffic": traffic,
+                "traffic_source": traffic_note,
                 "peak_source": f"{peaks_src} bf16_tflops_sustained (kernel timed inside back-to-back forwards)",
                 "launches_timed": dom[0], "avg_launch_ms": dom_ms,
                 "flops_per_launch": per_launch.get(dominant, 0.0)}
