@@ -139,6 +139,24 @@ int albert_forward_varlen(albert_handle *h, const int64_t *ids, const int32_t *c
 int albert_forward_host(albert_handle *h, const int64_t *ids_host, const uint8_t *mask_host,
                         int B, int T, void *out_host, void *stream);
 
+/* Pipelined path with HOST buffers for a sequence of batches (throughput
+ * serving).  Each call enqueues one batch on `stream`: copies of ids/mask to one
+ * of two device staging slots, the forward, and the copy of its output back to
+ * out_host on a stream the handle owns, so that a batch's output copy overlaps
+ * the next batch's forward.  The call does not wait for its own batch; it first
+ * waits for the batch issued two calls earlier (same slot) to reach the host and
+ * returns that batch's status (ALBERT_OK when there was none), or a host-side
+ * error.  Host buffers of a batch must stay valid, and out_host unread, until it
+ * has been waited for (pinned host memory for the copies to overlap).  The first
+ * call allocates the second staging slot (max_tokens rows).  Do not mix with
+ * albert_forward_host on the same handle while batches are in flight. */
+int albert_forward_host_async(albert_handle *h, const int64_t *ids_host, const uint8_t *mask_host,
+                              int B, int T, void *out_host, void *stream);
+
+/* Wait for every batch of albert_forward_host_async still in flight; returns
+ * the first non-OK status among them (ALBERT_OK if none). */
+int albert_forward_host_wait(albert_handle *h);
+
 /* Synchronize `stream` and return the status recorded by the last forward on
  * this handle (ALBERT_OK, ALBERT_ERR_ID, _MASK, _SEQLENS, _SHAPE or _TIMEOUT). */
 int albert_get_status(albert_handle *h, void *stream);

@@ -158,6 +158,44 @@ def test_forward_host_buffers_match_device_path(w_bf16):
     enc.close()
 
 
+def test_forward_host_async_pipeline_matches_device_path(w_bf16):
+    """Five batches of different lengths through the pipelined host path (two in
+    flight, output copies overlapping the next forward) equal the device path."""
+    wl = synth.WORKLOADS["b8_T128"]
+    enc = tea.Encoder(w_bf16, A, max_tokens=wl.B * wl.T)
+    batches, outs, refs = [], [], []
+    for k in range(5):
+        ids, mask, L = synth.make_batch(wl, seed=100 + k)
+        refs.append(enc.forward(_t(ids), _t(mask)).cpu())
+        batches.append((torch.as_tensor(ids).pin_memory(), torch.as_tensor(mask).pin_memory()))
+        outs.append(torch.full((wl.B, wl.T, 512), 7.0, dtype=torch.bfloat16).pin_memory())
+    for k in range(5):
+        assert enc.forward_host_async(batches[k][0], batches[k][1], outs[k]) == 0
+    assert enc.forward_host_wait() == 0
+    for k in range(5):
+        assert torch.equal(refs[k], outs[k]), f"batch {k}"
+    enc.close()
+
+
+def test_forward_host_async_reports_a_bad_batch_when_reaped(w_bf16):
+    wl = synth.WORKLOADS["b8_T128"]
+    enc = tea.Encoder(w_bf16, A, max_tokens=wl.B * wl.T)
+    ids, mask, L = synth.make_batch(wl)
+    ref = enc.forward(_t(ids), _t(mask)).cpu()
+    bad = ids.copy()
+    bad[2, int(L[2]) // 2] = 178
+    pin = lambda a: torch.as_tensor(a).pin_memory()
+    outs = [torch.zeros(wl.B, wl.T, 512, dtype=torch.bfloat16).pin_memory() for _ in range(4)]
+    seq = [ids, bad, ids, ids]
+    rcs = [enc.forward_host_async(pin(seq[k]), pin(mask), outs[k]) for k in range(4)]
+    # call k returns the status of batch k - 2: the bad batch 1 surfaces at call 3
+    assert rcs == [0, 0, 0, 4]
+    assert enc.forward_host_wait() == 0
+    for k in (0, 2, 3):
+        assert torch.equal(ref, outs[k]), f"batch {k}"
+    enc.close()
+
+
 # ------------------------------------------------------------ error paths ----
 
 def _sentinel(shape):

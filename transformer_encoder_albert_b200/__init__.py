@@ -34,6 +34,7 @@ WEIGHT_FIELDS = (
 
 EXPORTS = (
     "albert_create", "albert_forward", "albert_forward_varlen", "albert_forward_host",
+    "albert_forward_host_async", "albert_forward_host_wait",
     "albert_get_status", "albert_destroy", "albert_launches_per_forward",
     "albert_profile_enable", "albert_profile_reset", "albert_profile_classes",
     "albert_profile_name", "albert_profile_read", "albert_test_gemm", "albert_test_attention",
@@ -73,6 +74,8 @@ def lib() -> C.CDLL:
         L.albert_forward.argtypes = [vp, vp, vp, i, i, vp, vp]
         L.albert_forward_varlen.argtypes = [vp, vp, vp, i, i, vp, vp]
         L.albert_forward_host.argtypes = [vp, vp, vp, i, i, vp, vp]
+        L.albert_forward_host_async.argtypes = [vp, vp, vp, i, i, vp, vp]
+        L.albert_forward_host_wait.argtypes = [vp]
         L.albert_get_status.argtypes = [vp, vp]
         L.albert_destroy.argtypes = [vp]
         L.albert_destroy.restype = None
@@ -154,6 +157,16 @@ def albert_forward_host(h: int, ids_host, mask_host, out_host, stream=None) -> i
                                      _stream_ptr(stream))
 
 
+def albert_forward_host_async(h: int, ids_host, mask_host, out_host, stream=None) -> int:
+    B, T = ids_host.shape
+    return lib().albert_forward_host_async(h, _ptr(ids_host), _ptr(mask_host), B, T, _ptr(out_host),
+                                           _stream_ptr(stream))
+
+
+def albert_forward_host_wait(h: int) -> int:
+    return lib().albert_forward_host_wait(h)
+
+
 def albert_get_status(h: int, stream=None) -> int:
     return lib().albert_get_status(h, _stream_ptr(stream))
 
@@ -193,6 +206,15 @@ class Encoder:
 
     def forward_host(self, ids_host, mask_host, out_host, stream=None) -> int:
         return albert_forward_host(self.h, ids_host, mask_host, out_host, stream)
+
+    def forward_host_async(self, ids_host, mask_host, out_host, stream=None) -> int:
+        """Enqueue one batch of the pipelined host path; returns the status of the
+        batch issued two calls earlier (its output is then in host memory)."""
+        return albert_forward_host_async(self.h, ids_host, mask_host, out_host, stream)
+
+    def forward_host_wait(self) -> int:
+        """Wait for all pipelined host batches; first non-OK status."""
+        return albert_forward_host_wait(self.h)
 
     def status(self, stream=None) -> int:
         return albert_get_status(self.h, stream)

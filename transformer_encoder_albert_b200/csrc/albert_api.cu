@@ -67,6 +67,20 @@ struct albert_handle {
     uint8_t *st_mask = nullptr;
     void *st_out = nullptr;
 
+    // pipelined host path: two staging slots (slot 0 is the one above), a copy
+    // stream for the outputs, per-slot events and pinned per-batch status words
+    struct Slot {
+        int64_t *ids = nullptr;
+        uint8_t *mask = nullptr;
+        void *out = nullptr;
+        cudaEvent_t d2h_done = nullptr;  // output copied to the host
+        cudaEvent_t fwd_done = nullptr;  // forward (and its status copy) complete
+        bool in_flight = false;
+    } slot[2];
+    cudaStream_t copy_stream = nullptr;
+    int *status_host = nullptr;          // pinned, [2]
+    long long async_issued = 0;
+
     // TMA descriptors (bf16)
     CUtensorMap tm_E, tm_X, tm_C, tm_X1, tm_H, tm_Z, tm_QKV, tm_QKV64;
     CUtensorMap tm_win, tm_wqkv, tm_wo, tm_w1, tm_w2, tm_wout;
@@ -482,6 +496,15 @@ int create_impl(albert_handle *h, const albert_weights *w) {
 void free_all(albert_handle *h) {
     for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
     h->ev.clear();
+    for (auto &sl : h->slot) {
+        if (sl.d2h_done) cudaEventDestroy(sl.d2h_done);
+        if (sl.fwd_done) cudaEventDestroy(sl.fwd_done);
+        sl.d2h_done = sl.fwd_done = nullptr;
+    }
+    if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
+    h->copy_stream = nullptr;
+    if (h->status_host) cudaFreeHost(h->status_host);
+    h->status_host = nullptr;
     for (void *p : h->allocs) cudaFree(p);
     h->allocs.clear();
 }
@@ -547,6 +570,73 @@ int albert_forward_host(albert_handle *h, const int64_t *ids_host, const uint8_t
     if (rc) return rc;
     TRY(cudaMemcpyAsync(out_host, h->st_out, n * out_width(h) * elem_bytes(h), cudaMemcpyDeviceToHost, s));
     return albert_get_status(h, stream);
+}
+
+// Resources of the pipelined host path, made on first use.
+static int async_setup(albert_handle *h) {
+    if (h->copy_stream) return ALBERT_OK;
+    const size_t n = (size_t)h->cfg.max_tokens;
+    int rc;
+    h->slot[0].ids = h->st_ids;
+    h->slot[0].mask = h->st_mask;
+    h->slot[0].out = h->st_out;
+    if ((rc = dev_alloc(h, (void **)&h->slot[1].ids, n * sizeof(int64_t)))) return rc;
+    if ((rc = dev_alloc(h, (void **)&h->slot[1].mask, n))) return rc;
+    if ((rc = dev_alloc(h, &h->slot[1].out, n * out_width(h) * elem_bytes(h)))) return rc;
+    for (auto &sl : h->slot) {
+        TRY(cudaEventCreateWithFlags(&sl.d2h_done, cudaEventDisableTiming));
+        TRY(cudaEventCreateWithFlags(&sl.fwd_done, cudaEventDisableTiming));
+    }
+    TRY(cudaHostAlloc(reinterpret_cast<void **>(&h->status_host), 2 * sizeof(int), cudaHostAllocDefault));
+    TRY(cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking));
+    return ALBERT_OK;
+}
+
+// Wait for the batch in a slot to be complete on the host side; its status.
+static int async_reap(albert_handle *h, int b) {
+    auto &sl = h->slot[b];
+    if (!sl.in_flight) return ALBERT_OK;
+    TRY(cudaEventSynchronize(sl.d2h_done));
+    sl.in_flight = false;
+    return h->status_host[b];
+}
+
+int albert_forward_host_async(albert_handle *h, const int64_t *ids_host, const uint8_t *mask_host, int B, int T,
+                              void *out_host, void *stream) {
+    if (!h || !ids_host || !mask_host || !out_host) return ALBERT_ERR_NULL;
+    if (B < 1 || T < 1 || T > h->cfg.max_pos || (long long)B * T > h->cfg.max_tokens) return ALBERT_ERR_SHAPE;
+    int rc = async_setup(h);
+    if (rc) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int b = (int)(h->async_issued & 1);
+    // the batch two calls back used this slot: its output must have reached the host
+    const int prev = async_reap(h, b);
+    auto &sl = h->slot[b];
+    const size_t n = (size_t)B * T;
+    TRY(cudaMemcpyAsync(sl.ids, ids_host, n * sizeof(int64_t), cudaMemcpyHostToDevice, s));
+    TRY(cudaMemcpyAsync(sl.mask, mask_host, n, cudaMemcpyHostToDevice, s));
+    if ((rc = forward_padded(h, sl.ids, sl.mask, B, T, sl.out, s))) return rc;
+    // this batch's status, before the next forward's prep kernel resets the word
+    TRY(cudaMemcpyAsync(h->status_host + b, h->status, sizeof(int), cudaMemcpyDeviceToHost, s));
+    TRY(cudaEventRecord(sl.fwd_done, s));
+    TRY(cudaStreamWaitEvent(h->copy_stream, sl.fwd_done, 0));
+    TRY(cudaMemcpyAsync(out_host, sl.out, n * out_width(h) * elem_bytes(h), cudaMemcpyDeviceToHost, h->copy_stream));
+    TRY(cudaEventRecord(sl.d2h_done, h->copy_stream));
+    sl.in_flight = true;
+    ++h->async_issued;
+    return prev;
+}
+
+int albert_forward_host_wait(albert_handle *h) {
+    if (!h) return ALBERT_ERR_NULL;
+    if (!h->copy_stream) return ALBERT_OK;
+    const int b0 = (int)(h->async_issued & 1);  // the older batch first
+    int first = ALBERT_OK;
+    for (int i = 0; i < 2; ++i) {
+        const int st = async_reap(h, b0 ^ i);
+        if (first == ALBERT_OK) first = st;
+    }
+    return first;
 }
 
 int albert_get_status(albert_handle *h, void *stream) {
