@@ -195,6 +195,7 @@ GemmArgs gemm_args(albert_handle *h, int N, int K, const float *bias, void *out,
     a.row_dst = h->row_dst;
     a.status = h->status;
     a.eps = h->cfg.ln_eps;
+    a.trigger = 1;  // inside a forward the next launch is one of ours with PDL
     return a;
 }
 
@@ -251,6 +252,7 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
     ea.row_dst = h->row_dst;
     ea.dst_padded = padded_api;
     ea.status = h->status;
+    ea.trigger = bf ? 1 : 0;  // bf16: the input projection (PDL) follows; fp32: a plain launch
     LAUNCH(L, kProfEmbed, launch_embed(ea, L.s));
 
     const int D = out_width(h);
@@ -273,10 +275,11 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
             if (rc) return rc;
             if (max_len <= kAttnTcMaxLen) {
                 LAUNCH(L, kProfAttention, launch_attention_tc(h->tm_QKV, h->tm_QKV64, static_cast<bf16 *>(h->C), h->seq_start,
-                                                             h->seq_len, nseq, h->status, h->num_sms, L.s));
+                                                             h->seq_len, nseq, h->status, h->num_sms, L.s, true));
             } else {
                 LAUNCH(L, kProfAttention, launch_attention_bf16(static_cast<bf16 *>(h->QKV), static_cast<bf16 *>(h->C),
-                                                               h->seq_start, h->seq_len, nseq, max_len, h->status, L.s));
+                                                               h->seq_start, h->seq_len, nseq, max_len, h->status, L.s,
+                                                               true));
             }
             // z1 = C Wo^T + bo + layer input -> X1 = z1 * gamma1, st1
             GemmArgs a = gemm_args(h, kHidden, kHidden, l == 0 ? h->bo : h->bias_o2, nullptr, 0);
@@ -300,11 +303,14 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
             if ((rc = gemm_bf16(L, kProfGemmW2LN, kEpiResStats, h->tm_H, h->tm_w2, h->t32_Z, h->t32_X1, a))) return rc;
         }
         if (c.out_dim > 0) {
+            // the final projection is followed by zero_pad only in the padded API
             if (c.n_exec == 0) {
-                rc = gemm_bf16(L, kProfGemmOut, kEpiScatter, h->tm_X, h->tm_wout, h->t32_X, h->t32_X,
-                               gemm_args(h, c.out_dim, kHidden, h->b_out, out, c.out_dim));
+                GemmArgs a = gemm_args(h, c.out_dim, kHidden, h->b_out, out, c.out_dim);
+                a.trigger = padded_api;
+                rc = gemm_bf16(L, kProfGemmOut, kEpiScatter, h->tm_X, h->tm_wout, h->t32_X, h->t32_X, a);
             } else {
                 GemmArgs a = gemm_args(h, c.out_dim, kHidden, h->c_out, out, c.out_dim);
+                a.trigger = padded_api;
                 a.fold_s = h->s_out;
                 a.in_stats = h->st2;
                 rc = gemm_bf16(L, kProfGemmOut, kEpiLnInScatter, h->tm_Z, h->tm_wout, h->t32_X, h->t32_X, a);
@@ -513,7 +519,7 @@ int forward_padded(albert_handle *h, const int64_t *ids, const uint8_t *mask, in
                    cudaStream_t s) {
     Launch L{h, s};
     LAUNCH(L, kProfPrep, launch_prep_padded(mask, B, T, h->cfg.pack, h->cfg.max_tokens, h->seq_start, h->seq_len,
-                                            h->n_rows, h->status, s));
+                                            h->n_rows, h->status, s, true));
     return run_layers(h, L, ids, 1, B, T, T, out, 1);
 }
 
@@ -554,7 +560,7 @@ int albert_forward_varlen(albert_handle *h, const int64_t *ids, const int32_t *c
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Launch L{h, s};
     LAUNCH(L, kProfPrep, launch_prep_varlen(cu_seqlens, nseq, max_len, h->cfg.max_tokens, h->seq_start, h->seq_len,
-                                            h->n_rows, h->status, s));
+                                            h->n_rows, h->status, s, true));
     return run_layers(h, L, ids, 0, nseq, 0, max_len, out, 0);
 }
 
@@ -734,7 +740,8 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
     a.N = N; a.K = K; a.rows_cap = rows_cap; a.n_rows = ints; a.bias = bias; a.eps = eps;
     a.out_g = ln_g; a.out_stats = stats; a.out = static_cast<bf16 *>(Y); a.ld_out = N;
     a.row_dst = row_dst; a.status = ints + 1;
-    if (e == cudaSuccess) e = launch_gemm(kepi, ta, tb, to, tr, a, grid, s, variant);
+    // follows a copy in the stream: a plain launch
+    if (e == cudaSuccess) e = launch_gemm(kepi, ta, tb, to, tr, a, grid, s, variant, false);
     if (e == cudaSuccess && epi == 2)
         e = launch_ln_rows(static_cast<const bf16 *>(zg), stats, ln_g, ln_b, eps, static_cast<bf16 *>(Y), nullptr, M,
                            rows_cap, ints, ints + 1, s);
@@ -762,7 +769,7 @@ int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, 
     int *ints = nullptr;
     TRY(cudaMalloc(&ints, (2 * (size_t)nseq + 4) * sizeof(int)));
     int *seq_start = ints, *seq_len = ints + nseq + 1, *n_rows = seq_len + nseq + 1, *status = n_rows + 1;
-    cudaError_t e = launch_prep_varlen(cu_seqlens, nseq, max_len, 1 << 30, seq_start, seq_len, n_rows, status, s);
+    cudaError_t e = launch_prep_varlen(cu_seqlens, nseq, max_len, 1 << 30, seq_start, seq_len, n_rows, status, s, false);
     if (e == cudaSuccess) {
         if (dtype == ALBERT_FP32) {
             e = launch_attention_f32(static_cast<const float *>(qkv), static_cast<float *>(ctx), seq_start, seq_len, nseq,
@@ -771,10 +778,11 @@ int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, 
             CUtensorMap tm, tm64;
             if (make_tmap_bf16(&tm, qkv, (uint64_t)n_tok, kQKV, 128) || make_tmap_bf16(&tm64, qkv, (uint64_t)n_tok, kQKV, 64))
                 e = cudaErrorInvalidValue;
-            else e = launch_attention_tc(tm, tm64, static_cast<bf16 *>(ctx), seq_start, seq_len, nseq, status, sms, s);
+            else e = launch_attention_tc(tm, tm64, static_cast<bf16 *>(ctx), seq_start, seq_len, nseq, status, sms, s,
+                                         false);
         } else {
             e = launch_attention_bf16(static_cast<const bf16 *>(qkv), static_cast<bf16 *>(ctx), seq_start, seq_len, nseq,
-                                      max_len, status, s);
+                                      max_len, status, s, false);
         }
     }
     int st = 0;

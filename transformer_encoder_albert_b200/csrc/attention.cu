@@ -64,7 +64,10 @@ __device__ __forceinline__ void cp_async_wait_pending(int n) {
 template <int NW>
 __global__ void __launch_bounds__(NW * 32)
 attn_bf16_kernel(const bf16 *__restrict__ qkv, bf16 *__restrict__ ctx, const int *__restrict__ seq_start,
-                 const int *__restrict__ seq_len, const int *__restrict__ status) {
+                 const int *__restrict__ seq_len, const int *__restrict__ status, int trigger) {
+    if (trigger) griddep_launch_dependents();  // the next kernel may take SMs as this grid frees them
+    griddep_wait();               // the previous kernel has completed
+
     constexpr int QT = 16 * NW, NT = 32 * NW;
     if (*reinterpret_cast<const volatile int *>(status) != 0) return;
     const int b = blockIdx.z, h = blockIdx.y, q0 = blockIdx.x * QT;
@@ -261,7 +264,7 @@ static size_t attn_bf16_smem(int max_len, int qt) {
 
 template <int NW>
 static cudaError_t launch_attn_nw(const bf16 *qkv, bf16 *ctx, const int *seq_start, const int *seq_len, int nseq,
-                                  int max_len, const int *status, cudaStream_t s) {
+                                  int max_len, const int *status, cudaStream_t s, bool trigger) {
     constexpr int QT = 16 * NW;
     static bool configured = false;
     if (!configured) {
@@ -271,16 +274,16 @@ static cudaError_t launch_attn_nw(const bf16 *qkv, bf16 *ctx, const int *seq_sta
         configured = true;
     }
     dim3 grid((max_len + QT - 1) / QT, kHeads, nseq);
-    attn_bf16_kernel<NW><<<grid, NW * 32, attn_bf16_smem(max_len, QT), s>>>(qkv, ctx, seq_start, seq_len, status);
-    return cudaGetLastError();
+    return launch_pdl(attn_bf16_kernel<NW>, grid, dim3(NW * 32), attn_bf16_smem(max_len, QT), s, qkv, ctx, seq_start,
+                      seq_len, status, trigger ? 1 : 0);
 }
 
 cudaError_t launch_attention_bf16(const bf16 *qkv, bf16 *ctx, const int *seq_start,
                                   const int *seq_len, int nseq, int max_len, const int *status,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, bool trigger) {
     if (nseq <= 0) return cudaSuccess;
-    if (max_len <= 128) return launch_attn_nw<4>(qkv, ctx, seq_start, seq_len, nseq, max_len, status, s);
-    return launch_attn_nw<8>(qkv, ctx, seq_start, seq_len, nseq, max_len, status, s);
+    if (max_len <= 128) return launch_attn_nw<4>(qkv, ctx, seq_start, seq_len, nseq, max_len, status, s, trigger);
+    return launch_attn_nw<8>(qkv, ctx, seq_start, seq_len, nseq, max_len, status, s, trigger);
 }
 
 cudaError_t launch_attention_f32(const float *qkv, float *ctx, const int *seq_start,

@@ -89,7 +89,10 @@ __device__ __forceinline__ AttSmem att_carve(uint8_t *raw) {
 __global__ void __launch_bounds__(ATC_THREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmQKV64,
                bf16 *__restrict__ ctx, const int *__restrict__ seq_start, const int *__restrict__ seq_len, int nseq,
-               int *status) {
+               int *status, int trigger) {
+    if (trigger) griddep_launch_dependents();  // the next kernel may take SMs as this grid frees them
+    griddep_wait();               // the previous kernel has completed
+
     extern __shared__ uint8_t smem_raw[];
     AttSmem sm = att_carve(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -394,7 +397,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
 }  // namespace
 
 cudaError_t launch_attention_tc(const CUtensorMap &tmQKV, const CUtensorMap &tmQKV64, bf16 *ctx, const int *seq_start,
-                                const int *seq_len, int nseq, int *status, int num_sms, cudaStream_t s) {
+                                const int *seq_len, int nseq, int *status, int num_sms, cudaStream_t s, bool trigger) {
     if (nseq <= 0) return cudaSuccess;
     static bool configured = false;
     if (!configured) {
@@ -404,8 +407,8 @@ cudaError_t launch_attention_tc(const CUtensorMap &tmQKV, const CUtensorMap &tmQ
     }
     const int total = nseq * kHeads;
     const int grid = total < num_sms ? total : num_sms;
-    attn_tc_kernel<<<grid, ATC_THREADS, ATC_SMEM, s>>>(tmQKV, tmQKV64, ctx, seq_start, seq_len, nseq, status);
-    return cudaGetLastError();
+    return launch_pdl(attn_tc_kernel, dim3(grid), dim3(ATC_THREADS), ATC_SMEM, s, tmQKV, tmQKV64, ctx, seq_start,
+                      seq_len, nseq, status, trigger ? 1 : 0);
 }
 
 }  // namespace albert

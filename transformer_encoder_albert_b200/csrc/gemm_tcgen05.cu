@@ -207,9 +207,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const int slot = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
     const int nslots = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
+    if (p.trigger) griddep_launch_dependents();  // the next kernel may take SMs as this grid frees them
     if (threadIdx.x == 0) {
-        sm.misc[0] = *reinterpret_cast<const volatile int *>(p.n_rows);
-        sm.misc[1] = *reinterpret_cast<const volatile int *>(p.status);
         *sm.abort_flag = 0;
         for (int i = 0; i < NST; ++i) {
             mbar_init(smem_u32(&sm.full[i]), 1);
@@ -240,6 +239,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             tmem_alloc(smem_u32(sm.tmem_slot), TMEM_COLS);
             tmem_relinquish();
         }
+    }
+    // The prologue above overlaps the previous kernel; its results are used from here on.
+    griddep_wait();
+    if (threadIdx.x == 0) {
+        sm.misc[0] = *reinterpret_cast<const volatile int *>(p.n_rows);
+        sm.misc[1] = *reinterpret_cast<const volatile int *>(p.status);
     }
     tc_fence_before();
     // barrier initialisation (and, for a pair, the peer's) is visible before any use
@@ -649,43 +654,50 @@ int gemm_grid(int epi, int rows_cap, int N, int num_sms, int variant) {
 
 template <int EPI>
 static cudaError_t launch_one(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
-                              const CUtensorMap &tmRes, const GemmArgs &a, int grid, cudaStream_t s, bool pair) {
+                              const CUtensorMap &tmRes, const GemmArgs &a, int grid, cudaStream_t s, bool pair,
+                              bool pdl) {
     if (!pair) {
         constexpr int smem = Plan<EPI, false>::SMEM;
         cudaError_t e = configure<EPI, false>(smem);
         if (e != cudaSuccess) return e;
-        gemm_bf16_kernel<EPI, false><<<grid, THREADS, smem, s>>>(tmA, tmB, tmOut, tmRes, a);
-        return cudaGetLastError();
+        if (!pdl) {
+            gemm_bf16_kernel<EPI, false><<<grid, THREADS, smem, s>>>(tmA, tmB, tmOut, tmRes, a);
+            return cudaGetLastError();
+        }
+        return launch_pdl(gemm_bf16_kernel<EPI, false>, dim3(grid), dim3(THREADS), smem, s, tmA, tmB, tmOut, tmRes, a);
     }
     if (grid < 2 || grid % 2) return cudaErrorInvalidConfiguration;
     cudaError_t e = configure<EPI, true>(Plan<EPI, true>::SMEM);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(THREADS);
     cfg.dynamicSmemBytes = Plan<EPI, true>::SMEM;
     cfg.stream = s;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, gemm_bf16_kernel<EPI, true>, tmA, tmB, tmOut, tmRes, a);
 }
 
 cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
-                        const CUtensorMap &tmRes, const GemmArgs &a, int grid, cudaStream_t s, int variant) {
+                        const CUtensorMap &tmRes, const GemmArgs &a, int grid, cudaStream_t s, int variant,
+                        bool pdl) {
     const bool pair = gemm_use_pair(a.rows_cap, variant);
     switch (epi) {
-        case kEpiBias: return launch_one<kEpiBias>(tmA, tmB, tmOut, tmRes, a, grid, s, pair);
-        case kEpiGelu: return launch_one<kEpiGelu>(tmA, tmB, tmOut, tmRes, a, grid, s, pair);
-        case kEpiResStats: return launch_one<kEpiResStats>(tmA, tmB, tmOut, tmRes, a, grid, s, pair);
-        case kEpiScatter: return launch_one<kEpiScatter>(tmA, tmB, tmOut, tmRes, a, grid, s, pair);
-        case kEpiLnIn: return launch_one<kEpiLnIn>(tmA, tmB, tmOut, tmRes, a, grid, s, pair);
-        case kEpiLnInGelu: return launch_one<kEpiLnInGelu>(tmA, tmB, tmOut, tmRes, a, grid, s, pair);
-        case kEpiLnInScatter: return launch_one<kEpiLnInScatter>(tmA, tmB, tmOut, tmRes, a, grid, s, pair);
+        case kEpiBias: return launch_one<kEpiBias>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+        case kEpiGelu: return launch_one<kEpiGelu>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+        case kEpiResStats: return launch_one<kEpiResStats>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+        case kEpiScatter: return launch_one<kEpiScatter>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+        case kEpiLnIn: return launch_one<kEpiLnIn>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+        case kEpiLnInGelu: return launch_one<kEpiLnInGelu>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+        case kEpiLnInScatter: return launch_one<kEpiLnInScatter>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
     }
     return cudaErrorInvalidValue;
 }

@@ -9,6 +9,27 @@ namespace albert {
 
 using bf16 = __nv_bfloat16;
 
+// Launch with programmatic stream serialization: the kernel may begin while
+// the previous kernel in the stream runs; it must call griddep_wait() before
+// using that kernel's results (every kernel launched this way does).  Used only
+// where the previous operation in the stream is one of this library's kernels:
+// a kernel that follows a copy or an event is launched plainly.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Fixed architecture of the kernels.
 constexpr int kEmb = 128, kHidden = 768, kHeads = 12, kHeadDim = 64, kFfn = 2048;
 constexpr int kQKV = 3 * kHidden;
@@ -68,6 +89,8 @@ struct GemmArgs {
     int ld_out;
     const int *row_dst;        // scatter: destination row or -1
     int *status;               // device status word
+    int trigger;               // the next kernel in the stream is one of ours, launched with PDL:
+                               // let it start early (0 for a last kernel, or before a copy)
 };
 
 // Encode a 2-D bf16 row-major [rows, cols] tensor map with a {64, box_rows}
@@ -99,19 +122,21 @@ inline bool gemm_vectors_aligned(const GemmArgs &a) {
 // map of the residual (kEpiResStats only; pass any valid map otherwise).
 cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
                         const CUtensorMap &tmRes, const GemmArgs &args, int grid, cudaStream_t s,
-                        int variant = kGemmAuto);
+                        int variant = kGemmAuto, bool pdl = true);
 
 // ---------------------------------------------------------------- attention --
 // Masked bidirectional attention, bf16 tensor-core kernel (mma.sync m16n8k16).
+// trigger: the next kernel in the stream is one of ours launched with PDL (see GemmArgs).
 cudaError_t launch_attention_bf16(const bf16 *qkv, bf16 *ctx, const int *seq_start,
                                   const int *seq_len, int nseq, int max_len,
-                                  const int *status, cudaStream_t s);
+                                  const int *status, cudaStream_t s, bool trigger);
 // Same operation on tcgen05 for max_len <= 128 (one item = one (sequence, head));
 // tmQKV / tmQKV64: bf16 maps of the packed [rows, 3*768] buffer with a {64, 128} /
 // {64, 64} box and the 128-byte swizzle.
 constexpr int kAttnTcMaxLen = 128;
 cudaError_t launch_attention_tc(const CUtensorMap &tmQKV, const CUtensorMap &tmQKV64, bf16 *ctx, const int *seq_start,
-                                const int *seq_len, int nseq, int *status, int num_sms, cudaStream_t s);
+                                const int *seq_len, int nseq, int *status, int num_sms, cudaStream_t s,
+                                bool trigger);
 cudaError_t launch_attention_f32(const float *qkv, float *ctx, const int *seq_start,
                                  const int *seq_len, int nseq, int max_len,
                                  const int *status, cudaStream_t s);
@@ -120,10 +145,10 @@ cudaError_t launch_attention_f32(const float *qkv, float *ctx, const int *seq_st
 // max_rows: the handle's max_tokens; a larger total sets ALBERT_ERR_SHAPE.
 cudaError_t launch_prep_padded(const uint8_t *mask, int B, int T, int pack, int max_rows,
                                int *seq_start, int *seq_len, int *n_rows, int *status,
-                               cudaStream_t s);
+                               cudaStream_t s, bool trigger);
 cudaError_t launch_prep_varlen(const int32_t *cu, int nseq, int max_len, int max_rows,
                                int *seq_start, int *seq_len, int *n_rows, int *status,
-                               cudaStream_t s);
+                               cudaStream_t s, bool trigger);
 
 struct EmbedArgs {
     const int64_t *ids;
@@ -141,6 +166,7 @@ struct EmbedArgs {
     int *row_dst;       // destination row in `out` (b*T + t or the row itself) or -1
     int dst_padded;
     int *status;
+    int trigger;        // the next launch is one of ours with PDL (see GemmArgs)
 };
 cudaError_t launch_embed(const EmbedArgs &a, cudaStream_t s);
 

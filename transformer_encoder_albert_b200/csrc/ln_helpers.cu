@@ -44,6 +44,10 @@ __global__ void __launch_bounds__(256)
 ln_rows_kernel(const bf16 *__restrict__ zg, const float2 *__restrict__ stats, const float *__restrict__ gamma,
                const float *__restrict__ beta, float eps, bf16 *__restrict__ out, const int *__restrict__ row_dst,
                int out_rows, const int *n_rows, int *status) {
+    // last kernel of a forward: no early trigger, so that whatever follows in the
+    // stream waits for its completion (and, through the chain, the whole forward's)
+    griddep_wait();               // the previous kernel has completed
+
     if (*reinterpret_cast<const volatile int *>(status) != 0) return;
     const int r = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (r >= *n_rows) return;
@@ -102,9 +106,8 @@ cudaError_t launch_fold_ln(const bf16 *W, int N, int K, const float *gamma, cons
 cudaError_t launch_ln_rows(const bf16 *zg, const float2 *stats, const float *gamma, const float *beta, float eps,
                            bf16 *out, const int *row_dst, int out_rows, int rows_cap, const int *n_rows, int *status,
                            cudaStream_t s) {
-    ln_rows_kernel<<<(rows_cap + 7) / 8, 256, 0, s>>>(zg, stats, gamma, beta, eps, out, row_dst, out_rows, n_rows,
-                                                      status);
-    return cudaGetLastError();
+    return launch_pdl(ln_rows_kernel, dim3((rows_cap + 7) / 8), dim3(256), 0, s, zg, stats, gamma, beta, eps, out,
+                      row_dst, out_rows, n_rows, status);
 }
 
 cudaError_t launch_vec_add(const float *a, const float *b, float *out, int n, cudaStream_t s) {

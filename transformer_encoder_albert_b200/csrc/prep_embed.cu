@@ -48,7 +48,10 @@ __device__ int block_exclusive_scan(const int *rows, int n, int *start, int *sh)
 // sequence b L_b rows, padded mode T rows.
 __global__ void __launch_bounds__(PREP_THREADS)
 prep_padded_kernel(const uint8_t *__restrict__ mask, int B, int T, int pack, int rows_cap,
-                   int *seq_start, int *seq_len, int *n_rows, int *status) {
+                   int *seq_start, int *seq_len, int *n_rows, int *status, int trigger) {
+    if (trigger) griddep_launch_dependents();  // the next kernel may take SMs as this grid frees them
+    griddep_wait();               // the previous kernel has completed
+
     __shared__ int sh[PREP_THREADS];
     __shared__ int bad;
     if (threadIdx.x == 0) { *status = 0; bad = 0; }
@@ -90,7 +93,10 @@ prep_padded_kernel(const uint8_t *__restrict__ mask, int B, int T, int pack, int
 // Packed batch: cu[0] == 0, 1 <= cu[s+1]-cu[s] <= max_len, cu[nseq] <= rows_cap.
 __global__ void __launch_bounds__(PREP_THREADS)
 prep_varlen_kernel(const int32_t *__restrict__ cu, int nseq, int max_len, int rows_cap,
-                   int *seq_start, int *seq_len, int *n_rows, int *status) {
+                   int *seq_start, int *seq_len, int *n_rows, int *status, int trigger) {
+    if (trigger) griddep_launch_dependents();  // the next kernel may take SMs as this grid frees them
+    griddep_wait();               // the previous kernel has completed
+
     __shared__ int bad;
     if (threadIdx.x == 0) { *status = 0; bad = 0; }
     __syncthreads();
@@ -120,6 +126,9 @@ prep_varlen_kernel(const int32_t *__restrict__ cu, int nseq, int max_len, int ro
 // fp32), write E (bf16 or fp32) and the row's destination in the output.
 __global__ void __launch_bounds__(256)
 embed_ln_kernel(const EmbedArgs a) {
+    if (a.trigger) griddep_launch_dependents();  // the next kernel may take SMs as this grid frees them
+    griddep_wait();               // the previous kernel has completed
+
     if (*reinterpret_cast<const volatile int *>(a.status) != 0) return;
     const int n_rows = *a.n_rows;
     const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -167,6 +176,10 @@ embed_ln_kernel(const EmbedArgs a) {
 
 __global__ void zero_pad_kernel(uint4 *out, int B, int T, int chunks_per_row, const int *seq_len,
                                 const int *status) {
+    // last kernel of a forward: no early trigger, so that whatever follows in the
+    // stream waits for its completion (and, through the chain, the whole forward's)
+    griddep_wait();               // the previous kernel has completed
+
     if (*reinterpret_cast<const volatile int *>(status) != 0) return;
     const size_t n = (size_t)B * T * chunks_per_row;
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
@@ -178,6 +191,10 @@ __global__ void zero_pad_kernel(uint4 *out, int B, int T, int chunks_per_row, co
 
 __global__ void scatter_rows_kernel(const uint4 *X, uint4 *out, int chunks_per_row, int rows_cap,
                                     const int *n_rows, const int *row_dst, const int *status) {
+    // last kernel of a forward: no early trigger, so that whatever follows in the
+    // stream waits for its completion (and, through the chain, the whole forward's)
+    griddep_wait();               // the previous kernel has completed
+
     if (*reinterpret_cast<const volatile int *>(status) != 0) return;
     const int rows = *n_rows;
     const size_t n = (size_t)rows * chunks_per_row;
@@ -197,22 +214,26 @@ __global__ void f32_to_bf16_kernel(const float *src, bf16 *dst, size_t n) {
 
 cudaError_t launch_prep_padded(const uint8_t *mask, int B, int T, int pack, int rows_cap,
                                int *seq_start, int *seq_len, int *n_rows, int *status,
-                               cudaStream_t s) {
-    prep_padded_kernel<<<1, PREP_THREADS, 0, s>>>(mask, B, T, pack, rows_cap, seq_start, seq_len, n_rows, status);
+                               cudaStream_t s, bool trigger) {
+    // The first kernel of a forward: a plain launch, so that it is ordered after
+    // every earlier operation of the stream (copies of the inputs included).
+    prep_padded_kernel<<<1, PREP_THREADS, 0, s>>>(mask, B, T, pack, rows_cap, seq_start, seq_len, n_rows, status,
+                                                  trigger ? 1 : 0);
     return cudaGetLastError();
 }
 
 cudaError_t launch_prep_varlen(const int32_t *cu, int nseq, int max_len, int rows_cap,
                                int *seq_start, int *seq_len, int *n_rows, int *status,
-                               cudaStream_t s) {
-    prep_varlen_kernel<<<1, PREP_THREADS, 0, s>>>(cu, nseq, max_len, rows_cap, seq_start, seq_len, n_rows, status);
+                               cudaStream_t s, bool trigger) {
+    // first kernel of a forward: plain launch (see launch_prep_padded)
+    prep_varlen_kernel<<<1, PREP_THREADS, 0, s>>>(cu, nseq, max_len, rows_cap, seq_start, seq_len, n_rows, status,
+                                                  trigger ? 1 : 0);
     return cudaGetLastError();
 }
 
 cudaError_t launch_embed(const EmbedArgs &a, cudaStream_t s) {
     const int blocks = (a.rows_cap + 7) / 8;
-    embed_ln_kernel<<<blocks, 256, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(embed_ln_kernel, dim3(blocks), dim3(256), 0, s, a);
 }
 
 static int grid_for(size_t n, int threads) {
@@ -225,8 +246,8 @@ cudaError_t launch_zero_pad(void *out, int B, int T, int D, int elem_bytes, cons
                             const int *status, cudaStream_t s) {
     const int cpr = D * elem_bytes / 16;
     const size_t n = (size_t)B * T * cpr;
-    zero_pad_kernel<<<grid_for(n, 256), 256, 0, s>>>(static_cast<uint4 *>(out), B, T, cpr, seq_len, status);
-    return cudaGetLastError();
+    return launch_pdl(zero_pad_kernel, dim3(grid_for(n, 256)), dim3(256), 0, s, static_cast<uint4 *>(out), B, T, cpr,
+                      seq_len, status);
 }
 
 cudaError_t launch_scatter_rows(const void *X, void *out, int D, int elem_bytes, int rows_cap,
@@ -234,9 +255,8 @@ cudaError_t launch_scatter_rows(const void *X, void *out, int D, int elem_bytes,
                                 cudaStream_t s) {
     const int cpr = D * elem_bytes / 16;
     const size_t n = (size_t)rows_cap * cpr;
-    scatter_rows_kernel<<<grid_for(n, 256), 256, 0, s>>>(static_cast<const uint4 *>(X), static_cast<uint4 *>(out),
-                                                         cpr, rows_cap, n_rows, row_dst, status);
-    return cudaGetLastError();
+    return launch_pdl(scatter_rows_kernel, dim3(grid_for(n, 256)), dim3(256), 0, s, static_cast<const uint4 *>(X),
+                      static_cast<uint4 *>(out), cpr, rows_cap, n_rows, row_dst, status);
 }
 
 cudaError_t launch_f32_to_bf16(const float *src, bf16 *dst, size_t n, cudaStream_t s) {

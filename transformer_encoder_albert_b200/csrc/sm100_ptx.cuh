@@ -33,6 +33,18 @@ __device__ __forceinline__ void set_status(int *status, int code) {
     atomicCAS(status, 0, code);
 }
 
+// ---------------------------------------------- programmatic dependent launch --
+// A kernel launched with programmatic stream serialization may start while the
+// previous kernel in the stream is still running.  It lets the next kernel be
+// scheduled (launch_dependents: its CTAs take SMs as this grid frees them and
+// run their prologue), and waits for the previous kernel to complete, with its
+// memory visible (wait), before touching anything that kernel writes or reads.
+// Without that launch attribute both are no-ops.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier --
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
