@@ -239,6 +239,44 @@ def run_reference(args):
 
 # ------------------------------------------------------------- multi-rank ----
 
+def measure_length_regulation(torch, synth, tea, L, flush, peaks, peaks_src, stream, steps):
+    """Length regulation (the step after the encoder) on the same batch: its tokens
+    packed, 50 duration channels, 512-wide bf16 features.  HBM-bound: algorithmic
+    bytes = logits + features read, durations / frame starts / frames written."""
+    import numpy as np
+    n = int(np.sum(L))
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(L)]), dtype=torch.int32, device="cuda")
+    C, D = synth.DURATION_CHANNELS, 512
+    z = torch.tensor(synth.make_duration_logits(n, C), device="cuda")
+    f = torch.tensor(synth.make_features(n, D), device="cuda").to(torch.bfloat16)
+    st, dur, start, cuf, frames = tea.length_regulate(z, f, cu, speed=1.0, max_frames=16 * n)
+    if st != 0:
+        raise SystemExit(f"length regulation status {st}")
+    A = int(cuf[-1].item())
+    ms = []
+    P = tea._ptr
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for k in range(steps + 3):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        tea.lib().albert_length_regulate(P(z), C, 1.0, P(f), D, P(cu), len(L), n, P(dur), P(start), P(cuf),
+                                         P(frames), frames.shape[0], P(status), tea._stream_ptr())
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if k >= 3:
+            ms.append(e0.elapsed_time(e1))
+    t = sum(ms) / len(ms)
+    nbytes = n * C * 4 + n * D * 2 + n * 8 + A * D * 2 + 8 * (len(L) + 1)
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    achieved = nbytes / (t / 1000.0) / 1e9
+    return {"tokens": n, "frames": A, "channels": C, "width": D, "ms": t, "tokens_per_s": n / (t / 1000.0),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                         "bytes_per_launch": nbytes, "peak_source": f"{peaks_src} hbm_gbs"},
+            "launches": 3, "l2": "flushed before each timed launch"}
+
+
 def rank_batch_seed(base_seed: int, rank: int) -> int:
     """Each rank encodes its own batch of the workload (weak scaling)."""
     return base_seed + 1000 * rank
@@ -418,6 +456,7 @@ def run_gpu(args):
 
     peaks, peaks_src = load_peaks()
     peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    lenreg = measure_length_regulation(torch, synth, tea, L, flush, peaks, peaks_src, stream, args.steps)
     dom_ms = dom[1] / max(dom[0], 1)
     achieved = per_launch.get(dominant, 0.0) / (dom_ms / 1000.0) / 1e12
     traffic, traffic_note = load_traffic(dominant, wl.name + ("_padded" if args.padded else "_packed"))
@@ -447,6 +486,7 @@ def run_gpu(args):
                 "d2h_bytes_per_step": int(out_h.numel() * 2),
                 "api": "albert_forward_host_async (output copy of a step overlaps the next forward)",
                 "synchronous_api_value": e2e_sync_value},
+        "length_regulation": lenreg,
         "gpu_launches": launches * args.steps,
         "clocks": clocks,
     }

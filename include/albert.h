@@ -181,6 +181,38 @@ int albert_profile_classes(void);
 const char *albert_profile_name(int cls);
 int albert_profile_read(albert_handle *h, int *launches, double *ms);
 
+/* ---- length regulation (the step after the encoder) ----
+ * "ALBERT: How Kokoro's Phoneme Encoder Works", section "The time axis is where a
+ * circuit becomes difficult": per token, the sigmoid duration channels are summed,
+ * divided by the speed, rounded and clamped to at least one frame; A = sum d[t]
+ * is the number of aligned frames; token features are repeated by the duration
+ * vector ("How Kokoro TTS Works and Where CKE Stands", section "Path one":
+ * durations 2, 1, 3 -> p1 p1 p2 p3 p3 p3).
+ *
+ * For a packed batch of nseq sequences (token rows in cu_seqlens order, n_tok =
+ * cu_seqlens[nseq]), all device pointers, asynchronous on `stream`:
+ *   logits      [n_tok, C] fp32: duration channels (pre-sigmoid);
+ *   feats       [n_tok, D] bf16: token features (the encoder output), 16-byte aligned;
+ *   durations   [n_tok] int32 out: d[t] = max(1, rint(sum_c sigmoid(z[t,c]) / speed)),
+ *               taken in fp64, rint = round half to even;
+ *   frame_start [n_tok] int32 out: first frame of token t (frames of all sequences
+ *               back to back: token t owns frames frame_start[t] .. + d[t] - 1);
+ *   cu_frames   [nseq+1] int32 out: sequence b owns frames cu_frames[b] ..
+ *               cu_frames[b+1]-1, so A_b = cu_frames[b+1] - cu_frames[b];
+ *   frames      [max_frames, D] bf16 out: frame rows, 16-byte aligned;
+ *   status      [1] int32 out: ALBERT_OK, ALBERT_ERR_SEQLENS (cu_seqlens not
+ *               monotone from 0 to n_tok) or ALBERT_ERR_SHAPE (sum of durations
+ *               above max_frames; frames untouched).
+ * Host-side errors (returned at once): NULL pointers, C < 1, D not a positive
+ * multiple of 8, nseq or n_tok < 1 (ALBERT_ERR_SHAPE), speed not finite and
+ * positive or an unaligned feats/frames (ALBERT_ERR_CONFIG).  Allocates nothing.
+ * This step is not part of the pages' encoder; it is the workload their text
+ * names next on Kokoro's path. */
+int albert_length_regulate(const float *logits, int C, float speed, const void *feats, int D,
+                           const int32_t *cu_seqlens, int nseq, int n_tok, int32_t *durations,
+                           int32_t *frame_start, int32_t *cu_frames, void *frames, int max_frames,
+                           int32_t *status, void *stream);
+
 /* ---- single-kernel entry points (parity tests of one kernel) ----
  * These run one kernel of the path in isolation, synchronously, and return its
  * status.  They allocate and free temporary device memory. */

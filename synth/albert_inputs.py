@@ -171,3 +171,22 @@ def make_batch(wl: Workload, vocab: int = ARCH["vocab"], seed: int | None = None
             ids[b, 1:n - 1] = rng.integers(1, vocab, size=n - 2)
         mask[b, :n] = 1
     return ids, mask, L
+
+
+# Length regulation inputs: duration channels per token (pre-sigmoid).  50
+# channels drawn N(-2.9, 1) give sigmoid sums near 3.5, i.e. a few frames per
+# token; the channel count is a parameter of the operation.
+DURATION_CHANNELS = 50
+
+
+def make_duration_logits(n_tok: int, channels: int = DURATION_CHANNELS, seed: int = 7,
+                         mean: float = -2.9, std: float = 1.0) -> np.ndarray:
+    """Seeded fp32 duration logits [n_tok, channels]."""
+    rng = np.random.default_rng(seed)
+    return rng.normal(mean, std, (n_tok, channels)).astype(np.float32)
+
+
+def make_features(n_tok: int, width: int = ARCH["out_dim"], seed: int = 8) -> np.ndarray:
+    """Seeded bf16-representable token features [n_tok, width] (fp32 array)."""
+    rng = np.random.default_rng(seed)
+    return bf16_round(rng.normal(0.0, 1.0, (n_tok, width)).astype(np.float32))

@@ -184,10 +184,11 @@ def test_forward_host_async_reports_a_bad_batch_when_reaped(w_bf16):
     ref = enc.forward(_t(ids), _t(mask)).cpu()
     bad = ids.copy()
     bad[2, int(L[2]) // 2] = 178
-    pin = lambda a: torch.as_tensor(a).pin_memory()
+    # host buffers stay referenced until forward_host_wait (the copies are asynchronous)
+    ids_h = [torch.as_tensor(a).pin_memory() for a in (ids, bad, ids, ids)]
+    mask_h = torch.as_tensor(mask).pin_memory()
     outs = [torch.zeros(wl.B, wl.T, 512, dtype=torch.bfloat16).pin_memory() for _ in range(4)]
-    seq = [ids, bad, ids, ids]
-    rcs = [enc.forward_host_async(pin(seq[k]), pin(mask), outs[k]) for k in range(4)]
+    rcs = [enc.forward_host_async(ids_h[k], mask_h, outs[k]) for k in range(4)]
     # call k returns the status of batch k - 2: the bad batch 1 surfaces at call 3
     assert rcs == [0, 0, 0, 4]
     assert enc.forward_host_wait() == 0

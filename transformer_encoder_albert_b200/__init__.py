@@ -38,7 +38,7 @@ EXPORTS = (
     "albert_get_status", "albert_destroy", "albert_launches_per_forward",
     "albert_profile_enable", "albert_profile_reset", "albert_profile_classes",
     "albert_profile_name", "albert_profile_read", "albert_test_gemm", "albert_test_attention",
-    "albert_gemm_residual_ln_noalloc",
+    "albert_gemm_residual_ln_noalloc", "albert_length_regulate",
 )
 
 
@@ -89,6 +89,7 @@ def lib() -> C.CDLL:
         L.albert_test_gemm.argtypes = [vp, vp, vp, vp, vp, vp, C.c_float, vp, vp, i, i, i, i, vp]
         L.albert_test_attention.argtypes = [vp, vp, i, i, vp, i, vp]
         L.albert_gemm_residual_ln_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, C.c_float, vp, i, i, vp]
+        L.albert_length_regulate.argtypes = [vp, i, C.c_float, vp, i, vp, i, i, vp, vp, vp, vp, i, vp, vp]
         _lib = L
     return _lib
 
@@ -290,3 +291,31 @@ def gemm_residual_ln_noalloc(A, W, bias, R, ln_g, ln_b, Y, eps: float = 1e-12, s
     return lib().albert_gemm_residual_ln_noalloc(_ptr(A), _ptr(W), _ptr(bias), _ptr(R), _ptr(ln_g),
                                                  _ptr(ln_b), float(eps), _ptr(Y), M, K,
                                                  _stream_ptr(stream))
+
+
+def length_regulate(logits, feats, cu_seqlens, speed: float = 1.0, max_frames: int | None = None,
+                    stream=None):
+    """Length regulation of a packed batch on the GPU (albert_length_regulate).
+
+    logits [n_tok, C] fp32, feats [n_tok, D] bf16, cu_seqlens [nseq+1] int32, all on
+    the device.  Returns (status, durations, frame_start, cu_frames, frames) with
+    frames [max_frames, D] (the first cu_frames[-1] rows hold the result)."""
+    import torch
+    n_tok, C = logits.shape
+    D = feats.shape[1]
+    nseq = cu_seqlens.numel() - 1
+    if max_frames is None:
+        max_frames = 64 * n_tok
+    dev = logits.device
+    dur = torch.empty(n_tok, dtype=torch.int32, device=dev)
+    start = torch.empty(n_tok, dtype=torch.int32, device=dev)
+    cu_frames = torch.empty(nseq + 1, dtype=torch.int32, device=dev)
+    frames = torch.empty(max_frames, D, dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    rc = lib().albert_length_regulate(_ptr(logits), C, float(speed), _ptr(feats), D, _ptr(cu_seqlens), nseq, n_tok,
+                                      _ptr(dur), _ptr(start), _ptr(cu_frames), _ptr(frames), max_frames,
+                                      _ptr(status), _stream_ptr(stream))
+    if rc != ALBERT_OK:
+        return rc, None, None, None, None
+    torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+    return int(status.item()), dur, start, cu_frames, frames
