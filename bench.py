@@ -256,13 +256,14 @@ def measure_length_regulation(torch, synth, tea, L, flush, peaks, peaks_src, str
     ms = []
     P = tea._ptr
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    scratch = torch.empty(int(tea.lib().albert_length_regulate_scratch_bytes(n)), dtype=torch.uint8, device="cuda")
     for k in range(steps + 3):
         flush.zero_()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         tea.lib().albert_length_regulate(P(z), C, 1.0, P(f), D, P(cu), len(L), n, P(dur), P(start), P(cuf),
-                                         P(frames), frames.shape[0], P(status), tea._stream_ptr())
+                                         P(frames), frames.shape[0], P(scratch), P(status), tea._stream_ptr())
         e1.record(stream)
         torch.cuda.synchronize()
         if k >= 3:

@@ -200,18 +200,24 @@ int albert_profile_read(albert_handle *h, int *launches, double *ms);
  *   cu_frames   [nseq+1] int32 out: sequence b owns frames cu_frames[b] ..
  *               cu_frames[b+1]-1, so A_b = cu_frames[b+1] - cu_frames[b];
  *   frames      [max_frames, D] bf16 out: frame rows, 16-byte aligned;
+ *   scratch     device workspace of albert_length_regulate_scratch_bytes(n_tok)
+ *               bytes, 8-byte aligned (owned by the caller; one call at a time);
  *   status      [1] int32 out: ALBERT_OK, ALBERT_ERR_SEQLENS (cu_seqlens not
  *               monotone from 0 to n_tok) or ALBERT_ERR_SHAPE (sum of durations
  *               above max_frames; frames untouched).
  * Host-side errors (returned at once): NULL pointers, C < 1, D not a positive
  * multiple of 8, nseq or n_tok < 1 (ALBERT_ERR_SHAPE), speed not finite and
- * positive or an unaligned feats/frames (ALBERT_ERR_CONFIG).  Allocates nothing.
+ * positive or an unaligned feats/frames/scratch (ALBERT_ERR_CONFIG).  Allocates
+ * nothing.
  * This step is not part of the pages' encoder; it is the workload their text
  * names next on Kokoro's path. */
 int albert_length_regulate(const float *logits, int C, float speed, const void *feats, int D,
                            const int32_t *cu_seqlens, int nseq, int n_tok, int32_t *durations,
                            int32_t *frame_start, int32_t *cu_frames, void *frames, int max_frames,
-                           int32_t *status, void *stream);
+                           void *scratch, int32_t *status, void *stream);
+
+/* Bytes of device scratch albert_length_regulate needs for n_tok tokens. */
+size_t albert_length_regulate_scratch_bytes(int n_tok);
 
 /* ---- single-kernel entry points (parity tests of one kernel) ----
  * These run one kernel of the path in isolation, synchronously, and return its

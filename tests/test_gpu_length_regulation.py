@@ -101,9 +101,10 @@ def test_capacity_error_leaves_frames_untouched():
     start = torch.empty(20, dtype=torch.int32, device="cuda")
     cuf = torch.empty(2, dtype=torch.int32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    scratch = torch.empty(int(tea.lib().albert_length_regulate_scratch_bytes(20)), dtype=torch.uint8, device="cuda")
     P = tea._ptr
     rc = tea.lib().albert_length_regulate(P(zt), 50, 1.0, P(ft), 512, P(ct), 1, 20, P(dur), P(start), P(cuf),
-                                          P(frames), A - 1, P(status), tea._stream_ptr())
+                                          P(frames), A - 1, P(scratch), P(status), tea._stream_ptr())
     torch.cuda.synchronize()
     assert rc == 0 and int(status.item()) == 3
     assert torch.all(frames == 5.0)

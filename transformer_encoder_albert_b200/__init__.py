@@ -38,7 +38,7 @@ EXPORTS = (
     "albert_get_status", "albert_destroy", "albert_launches_per_forward",
     "albert_profile_enable", "albert_profile_reset", "albert_profile_classes",
     "albert_profile_name", "albert_profile_read", "albert_test_gemm", "albert_test_attention",
-    "albert_gemm_residual_ln_noalloc", "albert_length_regulate",
+    "albert_gemm_residual_ln_noalloc", "albert_length_regulate", "albert_length_regulate_scratch_bytes",
 )
 
 
@@ -89,7 +89,9 @@ def lib() -> C.CDLL:
         L.albert_test_gemm.argtypes = [vp, vp, vp, vp, vp, vp, C.c_float, vp, vp, i, i, i, i, vp]
         L.albert_test_attention.argtypes = [vp, vp, i, i, vp, i, vp]
         L.albert_gemm_residual_ln_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, C.c_float, vp, i, i, vp]
-        L.albert_length_regulate.argtypes = [vp, i, C.c_float, vp, i, vp, i, i, vp, vp, vp, vp, i, vp, vp]
+        L.albert_length_regulate.argtypes = [vp, i, C.c_float, vp, i, vp, i, i, vp, vp, vp, vp, i, vp, vp, vp]
+        L.albert_length_regulate_scratch_bytes.argtypes = [i]
+        L.albert_length_regulate_scratch_bytes.restype = C.c_size_t
         _lib = L
     return _lib
 
@@ -312,9 +314,10 @@ def length_regulate(logits, feats, cu_seqlens, speed: float = 1.0, max_frames: i
     cu_frames = torch.empty(nseq + 1, dtype=torch.int32, device=dev)
     frames = torch.empty(max_frames, D, dtype=torch.bfloat16, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
+    scratch = torch.empty(int(lib().albert_length_regulate_scratch_bytes(n_tok)), dtype=torch.uint8, device=dev)
     rc = lib().albert_length_regulate(_ptr(logits), C, float(speed), _ptr(feats), D, _ptr(cu_seqlens), nseq, n_tok,
                                       _ptr(dur), _ptr(start), _ptr(cu_frames), _ptr(frames), max_frames,
-                                      _ptr(status), _stream_ptr(stream))
+                                      _ptr(scratch), _ptr(status), _stream_ptr(stream))
     if rc != ALBERT_OK:
         return rc, None, None, None, None
     torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
