@@ -137,6 +137,36 @@ class Model:
         return x
 
 
+LAYER_PARAMS = ("wq", "bq", "wk", "bk", "wv", "bv", "wo", "bo", "ln1_g", "ln1_b",
+                "w1", "b1", "w2", "b2", "ln2_g", "ln2_b")
+
+
+def encode_grouped(weights: dict, arch: dict, ids, mask, n_groups: int, n_exec: int | None = None,
+                   out_dim: int | None = None) -> np.ndarray:
+    """ALBERT with grouped sharing ("ALBERT: How Kokoro's Phoneme Encoder Works",
+    section "2. Cross-layer parameter sharing": several distinct weight sets, each
+    reused over a block of consecutive executions).  The layer parameters hold
+    n_groups stacked sets; execution i uses set floor(i * n_groups / n_exec).
+    One sequence (ids, mask: [T]); returns fp64 [T, out_width], padding rows 0."""
+    n_exec = arch["n_exec"] if n_exec is None else n_exec
+    out_dim = arch["out_dim"] if out_dim is None else out_dim
+    ids = np.asarray(ids)
+    mask = np.asarray(mask, dtype=np.uint8)
+    L = int(mask.sum())
+    # one group: the layer parameters are not stacked
+    sets = [{k: (weights[k][g] if k in LAYER_PARAMS and n_groups > 1 else weights[k]) for k in PARAM_ORDER}
+            for g in range(n_groups)]
+    # embedding, its LayerNorm and the 128 -> 768 projection (no execution, no final projection)
+    x = Model(sets[0], arch, n_exec=0, out_dim=0).encode(ids[:L], mask[:L])
+    for i in range(n_exec):
+        x = Model(sets[i * n_groups // n_exec], arch, n_exec=1, out_dim=0).layer(x, mask[:L])
+    if out_dim > 0:
+        x = linear(x, weights["w_out"], weights["b_out"])
+    out = np.zeros((ids.shape[0], x.shape[1]), np.float64)
+    out[:L] = x
+    return out
+
+
 def linear(x, W, b=None) -> np.ndarray:
     x, W = _f64(x), _f64(W)
     b = None if b is None else _f64(b)

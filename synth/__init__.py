@@ -7,6 +7,7 @@ generators, and rounds values to bf16-representable ones where a workload asks.
 from .albert_inputs import (  # noqa: F401
     ARCH,
     DURATION_CHANNELS,
+    LAYER_PARAMS,
     PARAM_ORDER,
     WORKLOADS,
     Workload,

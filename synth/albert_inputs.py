@@ -84,11 +84,21 @@ def bf16_round(a: np.ndarray) -> np.ndarray:
     return out.reshape(a.shape)
 
 
+# Parameters of the transformer layer; with n_groups > 1 each holds n_groups
+# stacked copies (leading axis = weight group).
+LAYER_PARAMS = ("wq", "bq", "wk", "bk", "wv", "bv", "wo", "bo", "ln1_g", "ln1_b",
+                "w1", "b1", "w2", "b2", "ln2_g", "ln2_b")
+
+
 def make_weights(seed: int = 1234, arch: dict = ARCH, bf16: bool = True,
-                 ln_affine: str = "identity", std: float = 0.02) -> dict:
-    """Draw every parameter in PARAM_ORDER from N(0, std); LN gamma=1, beta=0 by default."""
+                 ln_affine: str = "identity", std: float = 0.02, n_groups: int = 1) -> dict:
+    """Draw every parameter in PARAM_ORDER from N(0, std); LN gamma=1, beta=0 by default.
+    n_groups > 1: the layer parameters get a leading axis of n_groups weight sets."""
     rng = np.random.default_rng(seed)
-    shapes = param_shapes(arch)
+    shapes = dict(param_shapes(arch))
+    if n_groups > 1:
+        for k in LAYER_PARAMS:
+            shapes[k] = (n_groups,) + tuple(shapes[k])
     w = {}
     for name in PARAM_ORDER:
         shp = shapes[name]

@@ -200,24 +200,38 @@ def test_attention_is_bidirectional():
 
 # -------------------------------------------------------- whole encoder ----
 
-def _hf_model(w, n_layers):
+def _hf_model(w, n_layers, n_groups=1):
     from transformers import AlbertConfig, AlbertModel
     cfg = AlbertConfig(vocab_size=A["vocab"], embedding_size=A["emb"], hidden_size=A["hidden"],
-                       num_hidden_layers=n_layers, num_hidden_groups=1,
+                       num_hidden_layers=n_layers, num_hidden_groups=n_groups,
                        num_attention_heads=A["heads"], intermediate_size=A["ffn"],
                        inner_group_num=1, hidden_act="gelu_new", hidden_dropout_prob=0.0,
                        attention_probs_dropout_prob=0.0, max_position_embeddings=A["max_pos"],
                        type_vocab_size=A["n_types"], layer_norm_eps=A["ln_eps"],
                        attn_implementation="eager")
     m = AlbertModel(cfg, add_pooling_layer=False).double().eval()
-    lay = "encoder.albert_layer_groups.0.albert_layers.0."
-    names = {
+    shared = {
         "embeddings.word_embeddings.weight": "word",
         "embeddings.position_embeddings.weight": "pos",
         "embeddings.token_type_embeddings.weight": "type",
         "embeddings.LayerNorm.weight": "emb_ln_g", "embeddings.LayerNorm.bias": "emb_ln_b",
         "encoder.embedding_hidden_mapping_in.weight": "w_in",
         "encoder.embedding_hidden_mapping_in.bias": "b_in",
+    }
+    sd = m.state_dict()
+    with torch.no_grad():
+        for hf, ours in shared.items():
+            sd[hf].copy_(torch.tensor(w[ours], dtype=torch.float64))
+        for g in range(n_groups):
+            lay = f"encoder.albert_layer_groups.{g}.albert_layers.0."
+            for hf, ours in _layer_names(lay).items():
+                src = w[ours][g] if n_groups > 1 else w[ours]
+                sd[hf].copy_(torch.tensor(src, dtype=torch.float64))
+    return m
+
+
+def _layer_names(lay):
+    return {
         lay + "attention.query.weight": "wq", lay + "attention.query.bias": "bq",
         lay + "attention.key.weight": "wk", lay + "attention.key.bias": "bk",
         lay + "attention.value.weight": "wv", lay + "attention.value.bias": "bv",
@@ -227,11 +241,6 @@ def _hf_model(w, n_layers):
         lay + "ffn_output.weight": "w2", lay + "ffn_output.bias": "b2",
         lay + "full_layer_layer_norm.weight": "ln2_g", lay + "full_layer_layer_norm.bias": "ln2_b",
     }
-    sd = m.state_dict()
-    with torch.no_grad():
-        for hf, ours in names.items():
-            sd[hf].copy_(torch.tensor(w[ours], dtype=torch.float64))
-    return m
 
 
 @pytest.mark.parametrize("n_exec", [1, 12])
@@ -256,6 +265,36 @@ def test_encoder_matches_hf_albert_model(n_exec):
                  token_type_ids=torch.zeros_like(torch.tensor(ids))).last_hidden_state.numpy()
     for b in range(B):
         np.testing.assert_allclose(got[b, :L[b]], ref[b, :L[b]], rtol=1e-9, atol=1e-9)
+
+
+@pytest.mark.parametrize("n_groups", [2, 3, 12])
+def test_grouped_sharing_matches_hf_albert_model(n_groups):
+    """Grouped sharing (n_groups weight sets over 12 executions) against
+    transformers' AlbertModel with num_hidden_groups = n_groups."""
+    w = synth.make_weights(seed=23, bf16=False, ln_affine="random", n_groups=n_groups)
+    r = _rng(24)
+    T, L = 18, 15
+    ids = np.zeros(T, np.int64)
+    ids[1:L - 1] = r.integers(1, A["vocab"], L - 2)
+    mask = np.array([1] * L + [0] * (T - L), np.uint8)
+    got = oracle.encode_grouped(w, A, ids, mask, n_groups, n_exec=12, out_dim=0)
+    hf = _hf_model(w, 12, n_groups)
+    with torch.no_grad():
+        ref = hf(input_ids=torch.tensor(ids[None]), attention_mask=torch.tensor(mask[None].astype(np.int64)),
+                 token_type_ids=torch.zeros(1, T, dtype=torch.int64)).last_hidden_state.numpy()[0]
+    np.testing.assert_allclose(got[:L], ref[:L], rtol=1e-9, atol=1e-9)
+    assert np.all(got[L:] == 0)
+
+
+def test_grouped_sharing_with_one_group_is_the_shared_model():
+    w = synth.make_weights(seed=25, bf16=False, ln_affine="random")
+    r = _rng(26)
+    ids = np.zeros(12, np.int64)
+    ids[1:9] = r.integers(1, A["vocab"], 8)
+    mask = np.array([1] * 10 + [0] * 2, np.uint8)
+    a = oracle.encode_grouped(w, A, ids, mask, 1)
+    b = oracle.Model(w, A).encode(ids, mask)
+    np.testing.assert_allclose(a[:10], b[:10], rtol=1e-12, atol=1e-12)
 
 
 def test_one_layer_matches_library_post_ln_transformer_layer():
