@@ -63,9 +63,13 @@ extern "C" {
 
 /* Architecture and capacity.  The kernels support exactly: emb 128, hidden 768,
  * heads 12 (64 wide), ffn 2048, max_pos <= 512, out_dim 512 or 0 (0 = return the
- * [.., 768] hidden states), n_groups 1 (one fully shared layer).  n_exec >= 0
- * is free.  max_tokens is the workspace capacity in rows: albert_forward needs
- * B*T <= max_tokens, albert_forward_varlen needs total tokens <= max_tokens. */
+ * [.., 768] hidden states).  n_exec >= 0 is free.  n_groups: distinct layer weight
+ * sets, 1 <= n_groups <= max(n_exec, 1); execution i uses set
+ * floor(i * n_groups / n_exec), i.e. consecutive blocks of executions share a set
+ * ("ALBERT: How Kokoro's Phoneme Encoder Works", section "2. Cross-layer
+ * parameter sharing"; 1 = one fully shared layer, Kokoro's case).  max_tokens
+ * is the workspace capacity in rows: albert_forward needs B*T <= max_tokens,
+ * albert_forward_varlen needs total tokens <= max_tokens. */
 typedef struct {
     int vocab;       /* 178 for Kokoro                                  */
     int emb;         /* E = 128                                         */
@@ -73,7 +77,7 @@ typedef struct {
     int heads;       /* 12                                              */
     int ffn;         /* 2048                                            */
     int n_exec;      /* executions of the shared layer, 12 for Kokoro   */
-    int n_groups;    /* distinct layer weight sets; must be 1           */
+    int n_groups;    /* distinct layer weight sets (1 = fully shared)   */
     int max_pos;     /* rows of the position table, <= 512              */
     int n_types;     /* rows of the token-type table (type 0 is used)   */
     int out_dim;     /* 512, or 0 for no final projection               */
@@ -87,7 +91,10 @@ typedef struct {
 
 /* Parameters: DEVICE pointers to fp32 tensors in PyTorch layouts ([out, in] for
  * linears).  albert_create copies them (converting to bf16 for ALBERT_BF16), so
- * the caller may free them afterwards.  w_out/b_out may be NULL if out_dim == 0. */
+ * the caller may free them afterwards.  w_out/b_out may be NULL if out_dim == 0.
+ * With n_groups > 1 every layer parameter (wq .. ln2_b) holds n_groups copies
+ * back to back, set g at offset g * (its size); the embedding tables, w_in/b_in
+ * and w_out/b_out are single. */
 typedef struct {
     const float *word;      /* [vocab, emb]     */
     const float *pos;       /* [max_pos, emb]   */

@@ -7,6 +7,8 @@ import re
 
 import pytest
 
+import synth
+
 import transformer_encoder_albert_b200 as tea
 from transformer_encoder_albert_b200 import build as tea_build
 
@@ -74,3 +76,16 @@ def test_host_side_rejections_need_no_gpu(lib):
     assert lib.albert_forward(None, None, None, 1, 1, None, None) == 1
     lib.albert_destroy.argtypes = [C.c_void_p]
     lib.albert_destroy(None)
+
+
+def test_create_rejects_bad_group_counts_before_touching_the_device():
+    """albert_create validates the config on the host first: these return
+    ALBERT_ERR_CONFIG without any CUDA call (the weight pointers are never read)."""
+    import transformer_encoder_albert_b200 as tea
+    lib = tea.lib()
+    dummy = tea.albert_weights(*([C.c_void_p(16)] * len(tea.WEIGHT_FIELDS)))
+    for n_exec, n_groups in ((12, 0), (3, 4), (0, 2), (12, -1)):
+        cfg = tea.make_config(synth.ARCH, n_exec=n_exec, n_groups=n_groups)
+        h = C.c_void_p()
+        assert lib.albert_create(C.byref(dummy), C.byref(cfg), C.byref(h)) == 2  # ALBERT_ERR_CONFIG
+        assert h.value is None

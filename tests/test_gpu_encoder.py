@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 import transformer_encoder_albert_b200 as tea
 from parity_util import check_bf16, check_fp32, oracle_rows, sample_sequences
@@ -109,6 +110,44 @@ def test_random_layer_norm_affine_catches_swaps():
     wl = synth.Workload("affine", 3, 64, "uniform", lo=10, hi=64, seed=78)
     ids, mask, L, got = _run(w, wl, n_exec=3)
     _compare(w, wl, got, ids, mask, L, list(range(wl.B)), n_exec=3)
+
+
+@pytest.mark.parametrize("n_groups,n_exec", [(2, 12), (3, 12), (12, 12), (2, 5)])
+def test_grouped_sharing_matches_oracle(n_groups, n_exec):
+    """n_groups weight sets over n_exec executions (consecutive blocks per set):
+    every sequence of a ragged batch against the grouped oracle."""
+    w = synth.make_weights(seed=41 + n_groups, bf16=True, ln_affine="random", n_groups=n_groups)
+    wl = synth.Workload("grouped", 6, 96, "uniform", lo=5, hi=96, seed=80 + n_groups)
+    ids, mask, L = synth.make_batch(wl)
+    enc = tea.Encoder(w, A, max_tokens=wl.B * wl.T, n_exec=n_exec, n_groups=n_groups)
+    got = enc.forward(_t(ids), _t(mask)).float().cpu().numpy()
+    assert enc.status() == 0
+    enc.close()
+    for b in range(wl.B):
+        n = int(L[b])
+        ref = oracle.encode_grouped(w, A, ids[b, :n], mask[b, :n], n_groups, n_exec=n_exec)
+        check_bf16(got[b, :n], ref, f"grouped G={n_groups} seq {b} (L={n})")
+        assert np.all(got[b, n:] == 0.0)
+
+
+def test_grouped_sharing_fp32(w_fp32):
+    w = synth.make_weights(seed=47, bf16=False, ln_affine="random", n_groups=3)
+    wl = synth.Workload("grouped32", 2, 30, "uniform", lo=4, hi=30, seed=90, dtype="fp32")
+    ids, mask, L = synth.make_batch(wl)
+    enc = tea.Encoder(w, A, dtype="fp32", max_tokens=wl.B * wl.T, n_exec=6, n_groups=3)
+    got = enc.forward(_t(ids), _t(mask)).float().cpu().numpy()
+    assert enc.status() == 0
+    enc.close()
+    for b in range(wl.B):
+        n = int(L[b])
+        ref = oracle.encode_grouped(w, A, ids[b, :n], mask[b, :n], 3, n_exec=6)
+        check_fp32(got[b, :n], ref, f"grouped fp32 seq {b}")
+
+
+def test_grouped_sharing_rejects_more_groups_than_executions():
+    w = synth.make_weights(seed=48, bf16=True, n_groups=4)
+    with pytest.raises(tea.AlbertError):
+        tea.Encoder(w, A, max_tokens=64, n_exec=3, n_groups=4)
 
 
 def test_fp32_small_padded_batch(w_fp32):

@@ -112,10 +112,10 @@ def _ptr(t) -> int | None:
 
 
 def make_config(arch: dict, dtype: str = "bf16", max_tokens: int = 4096, pack: bool = True,
-                n_exec: int | None = None, out_dim: int | None = None) -> albert_config:
+                n_exec: int | None = None, out_dim: int | None = None, n_groups: int = 1) -> albert_config:
     return albert_config(
         vocab=arch["vocab"], emb=arch["emb"], hidden=arch["hidden"], heads=arch["heads"],
-        ffn=arch["ffn"], n_exec=arch["n_exec"] if n_exec is None else n_exec, n_groups=1,
+        ffn=arch["ffn"], n_exec=arch["n_exec"] if n_exec is None else n_exec, n_groups=n_groups,
         max_pos=arch["max_pos"], n_types=arch["n_types"],
         out_dim=arch["out_dim"] if out_dim is None else out_dim,
         dtype=ALBERT_BF16 if dtype == "bf16" else ALBERT_FP32, max_tokens=max_tokens,
@@ -184,8 +184,10 @@ class Encoder:
     """Owns one library handle.  Outputs are bf16 (dtype "bf16") or fp32 tensors."""
 
     def __init__(self, weights: dict, arch: dict, dtype: str = "bf16", max_tokens: int = 4096,
-                 pack: bool = True, n_exec: int | None = None, out_dim: int | None = None):
-        self.cfg = make_config(arch, dtype, max_tokens, pack, n_exec, out_dim)
+                 pack: bool = True, n_exec: int | None = None, out_dim: int | None = None, n_groups: int = 1):
+        """n_groups > 1: the layer parameters of `weights` hold n_groups stacked sets
+        (leading axis), execution i using set i * n_groups // n_exec."""
+        self.cfg = make_config(arch, dtype, max_tokens, pack, n_exec, out_dim, n_groups)
         self.dtype = dtype
         self.out_dim = self.cfg.out_dim if self.cfg.out_dim > 0 else self.cfg.hidden
         self.h = albert_create(weights, self.cfg)

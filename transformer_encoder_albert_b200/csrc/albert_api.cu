@@ -41,13 +41,27 @@ struct albert_handle {
     int seq_cap = 0;    // sequences
     std::vector<void *> allocs;
 
-    // parameters
+    // parameters shared by every execution
     float *word = nullptr, *pos = nullptr, *type = nullptr, *emb_g = nullptr, *emb_b = nullptr;
-    float *b_in = nullptr, *bqkv = nullptr, *bo = nullptr, *ln1_g = nullptr, *ln1_b = nullptr;
-    float *b1 = nullptr, *b2 = nullptr, *ln2_g = nullptr, *ln2_b = nullptr, *b_out = nullptr;
-    void *w_in = nullptr, *wqkv = nullptr, *wo = nullptr, *w1 = nullptr, *w2 = nullptr, *w_out = nullptr;
+    float *b_in = nullptr, *b_out = nullptr;
+    void *w_in = nullptr, *w_out = nullptr;
     void *wblock = nullptr;
     size_t wblock_bytes = 0;
+    // one layer weight set per group; execution l uses group group_of(cfg, l)
+    struct Group {
+        float *bqkv = nullptr, *bo = nullptr, *ln1_g = nullptr, *ln1_b = nullptr;
+        float *b1 = nullptr, *b2 = nullptr, *ln2_g = nullptr, *ln2_b = nullptr;
+        void *wqkv = nullptr, *wo = nullptr, *w1 = nullptr, *w2 = nullptr;
+        CUtensorMap tm_wqkv, tm_wo, tm_w1, tm_w2;
+        float *s_1 = nullptr, *c_1 = nullptr, *bias_21 = nullptr;  // bf16: this group's LN1 folded
+    };
+    std::vector<Group> grp;
+    // bf16, execution l >= 1: its group's Q|K|V and out-projection with the LN2
+    // of execution l-1 (possibly another group) folded in
+    struct Exec {
+        float *s_qkv = nullptr, *c_qkv = nullptr, *bias_o2 = nullptr;
+    };
+    std::vector<Exec> ex;
 
     // workspace
     // bf16: X = input projection output, X1 = z1 * gamma1, Z = z2 * gamma2 (z1, z2:
@@ -55,11 +69,10 @@ struct albert_handle {
     // fp32: X, X1 = LayerNorm outputs, Z = pre-norm rows.
     void *E = nullptr, *X = nullptr, *QKV = nullptr, *C = nullptr, *X1 = nullptr, *H = nullptr, *Z = nullptr;
     float2 *st1 = nullptr, *st2 = nullptr;  // partial (mean, M2) of z1 / z2, [rows][6]
-    // folded LayerNorm constants: s = W gamma, c = W beta + b, and biases plus the
-    // beta of a rebuilt residual
+    // folded LayerNorm constants (s = W gamma, c = W beta + b, biases plus the beta
+    // of a rebuilt residual): per group and per execution above, the final ones here
     float *fold = nullptr;
-    float *s_qkv = nullptr, *c_qkv = nullptr, *s_1 = nullptr, *c_1 = nullptr, *s_out = nullptr, *c_out = nullptr;
-    float *bias_o2 = nullptr, *bias_21 = nullptr;
+    float *s_out = nullptr, *c_out = nullptr;
     int *seq_start = nullptr, *seq_len = nullptr, *row_dst = nullptr, *n_rows = nullptr, *status = nullptr;
 
     // host-buffer staging
@@ -83,7 +96,7 @@ struct albert_handle {
 
     // TMA descriptors (bf16)
     CUtensorMap tm_E, tm_X, tm_C, tm_X1, tm_H, tm_Z, tm_QKV, tm_QKV64;
-    CUtensorMap tm_win, tm_wqkv, tm_wo, tm_w1, tm_w2, tm_wout;
+    CUtensorMap tm_win, tm_wout;
     CUtensorMap t32_X, t32_QKV, t32_X1, t32_H, t32_Z;  // 32x32-box maps: epilogue stores / residual loads
 
     // per-kernel timing
@@ -121,9 +134,15 @@ int dev_alloc(albert_handle *h, void **p, size_t bytes) {
 size_t elem_bytes(const albert_handle *h) { return h->cfg.dtype == ALBERT_FP32 ? 4 : 2; }
 int out_width(const albert_handle *h) { return h->cfg.out_dim > 0 ? h->cfg.out_dim : kHidden; }
 
+// Weight group of execution l: ALBERT's grouped sharing splits the executions
+// into n_groups consecutive runs of equal length (floor(l * n_groups / n_exec)).
+int group_of(const albert_config &c, int l) {
+    return c.n_exec > 0 ? (int)((long long)l * c.n_groups / c.n_exec) : 0;
+}
+
 int check_config(const albert_config *c) {
     if (c->emb != kEmb || c->hidden != kHidden || c->heads != kHeads || c->ffn != kFfn) return ALBERT_ERR_CONFIG;
-    if (c->n_groups != 1 || c->n_exec < 0) return ALBERT_ERR_CONFIG;
+    if (c->n_exec < 0 || c->n_groups < 1 || c->n_groups > (c->n_exec > 0 ? c->n_exec : 1)) return ALBERT_ERR_CONFIG;
     if (c->max_pos < 1 || c->max_pos > kMaxPos || c->vocab < 1 || c->n_types < 1) return ALBERT_ERR_CONFIG;
     if (c->out_dim != 0 && c->out_dim != 512) return ALBERT_ERR_CONFIG;
     if (c->dtype != ALBERT_BF16 && c->dtype != ALBERT_FP32) return ALBERT_ERR_CONFIG;
@@ -262,15 +281,17 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
                             gemm_args(h, kHidden, kEmb, h->b_in, nullptr, 0))))
             return rc;
         for (int l = 0; l < c.n_exec; ++l) {
+            const auto &W = h->grp[group_of(c, l)];                  // this execution's weights
+            const auto &Wp = h->grp[group_of(c, l > 0 ? l - 1 : 0)];  // the previous execution's (its LN2)
             // Q|K|V from the layer input: X for the first execution, else LN2(z2) folded
             if (l == 0) {
-                rc = gemm_bf16(L, kProfGemmQKV, kEpiBias, h->tm_X, h->tm_wqkv, h->t32_QKV, h->t32_QKV,
-                               gemm_args(h, kQKV, kHidden, h->bqkv, nullptr, 0));
+                rc = gemm_bf16(L, kProfGemmQKV, kEpiBias, h->tm_X, W.tm_wqkv, h->t32_QKV, h->t32_QKV,
+                               gemm_args(h, kQKV, kHidden, W.bqkv, nullptr, 0));
             } else {
-                GemmArgs a = gemm_args(h, kQKV, kHidden, h->c_qkv, nullptr, 0);
-                a.fold_s = h->s_qkv;
+                GemmArgs a = gemm_args(h, kQKV, kHidden, h->ex[l].c_qkv, nullptr, 0);
+                a.fold_s = h->ex[l].s_qkv;
                 a.in_stats = h->st2;
-                rc = gemm_bf16(L, kProfGemmQKV, kEpiLnIn, h->tm_Z, h->tm_wqkv, h->t32_QKV, h->t32_QKV, a);
+                rc = gemm_bf16(L, kProfGemmQKV, kEpiLnIn, h->tm_Z, W.tm_wqkv, h->t32_QKV, h->t32_QKV, a);
             }
             if (rc) return rc;
             if (max_len <= kAttnTcMaxLen) {
@@ -282,25 +303,25 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
                                                                true));
             }
             // z1 = C Wo^T + bo + layer input -> X1 = z1 * gamma1, st1
-            GemmArgs a = gemm_args(h, kHidden, kHidden, l == 0 ? h->bo : h->bias_o2, nullptr, 0);
+            GemmArgs a = gemm_args(h, kHidden, kHidden, l == 0 ? W.bo : h->ex[l].bias_o2, nullptr, 0);
             a.res_stats = l == 0 ? nullptr : h->st2;
-            a.res_g = h->ln2_g;
-            a.out_g = h->ln1_g;
+            a.res_g = Wp.ln2_g;
+            a.out_g = W.ln1_g;
             a.out_stats = h->st1;
-            if ((rc = gemm_bf16(L, kProfGemmWoLN, kEpiResStats, h->tm_C, h->tm_wo, h->t32_X1, l == 0 ? h->t32_X : h->t32_Z, a)))
+            if ((rc = gemm_bf16(L, kProfGemmWoLN, kEpiResStats, h->tm_C, W.tm_wo, h->t32_X1, l == 0 ? h->t32_X : h->t32_Z, a)))
                 return rc;
             // H = GELU(LN1(z1) W1^T + b1)
-            a = gemm_args(h, kFfn, kHidden, h->c_1, nullptr, 0);
-            a.fold_s = h->s_1;
+            a = gemm_args(h, kFfn, kHidden, W.c_1, nullptr, 0);
+            a.fold_s = W.s_1;
             a.in_stats = h->st1;
-            if ((rc = gemm_bf16(L, kProfGemmW1Gelu, kEpiLnInGelu, h->tm_X1, h->tm_w1, h->t32_H, h->t32_H, a))) return rc;
+            if ((rc = gemm_bf16(L, kProfGemmW1Gelu, kEpiLnInGelu, h->tm_X1, W.tm_w1, h->t32_H, h->t32_H, a))) return rc;
             // z2 = H W2^T + b2 + LN1(z1) -> Z = z2 * gamma2, st2
-            a = gemm_args(h, kHidden, kFfn, h->bias_21, nullptr, 0);
+            a = gemm_args(h, kHidden, kFfn, W.bias_21, nullptr, 0);
             a.res_stats = h->st1;
-            a.res_g = h->ln1_g;
-            a.out_g = h->ln2_g;
+            a.res_g = W.ln1_g;
+            a.out_g = W.ln2_g;
             a.out_stats = h->st2;
-            if ((rc = gemm_bf16(L, kProfGemmW2LN, kEpiResStats, h->tm_H, h->tm_w2, h->t32_Z, h->t32_X1, a))) return rc;
+            if ((rc = gemm_bf16(L, kProfGemmW2LN, kEpiResStats, h->tm_H, W.tm_w2, h->t32_Z, h->t32_X1, a))) return rc;
         }
         if (c.out_dim > 0) {
             // the final projection is followed by zero_pad only in the padded API
@@ -319,26 +340,28 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
         } else if (c.n_exec == 0) {
             LAUNCH(L, kProfOutput, launch_scatter_rows(h->X, out, kHidden, 2, h->rows_cap, h->n_rows, h->row_dst, h->status, L.s));
         } else {
-            LAUNCH(L, kProfOutput, launch_ln_rows(static_cast<bf16 *>(h->Z), h->st2, h->ln2_g, h->ln2_b, c.ln_eps,
+            const auto &Wl = h->grp[group_of(c, c.n_exec - 1)];
+            LAUNCH(L, kProfOutput, launch_ln_rows(static_cast<bf16 *>(h->Z), h->st2, Wl.ln2_g, Wl.ln2_b, c.ln_eps,
                                                   static_cast<bf16 *>(out), h->row_dst, out_rows, h->rows_cap, h->n_rows,
                                                   h->status, L.s));
         }
     } else {
         LAUNCH(L, kProfGemmIn, launch_gemm_f32(kF32Bias, f32_args(h, h->E, h->w_in, h->b_in, h->X, kHidden, kHidden, kEmb), L.s));
         for (int l = 0; l < c.n_exec; ++l) {
-            LAUNCH(L, kProfGemmQKV, launch_gemm_f32(kF32Bias, f32_args(h, h->X, h->wqkv, h->bqkv, h->QKV, kQKV, kQKV, kHidden), L.s));
+            const auto &W = h->grp[group_of(c, l)];
+            LAUNCH(L, kProfGemmQKV, launch_gemm_f32(kF32Bias, f32_args(h, h->X, W.wqkv, W.bqkv, h->QKV, kQKV, kQKV, kHidden), L.s));
             LAUNCH(L, kProfAttention, launch_attention_f32(static_cast<float *>(h->QKV), static_cast<float *>(h->C), h->seq_start,
                                                           h->seq_len, nseq, max_len, h->status, L.s));
-            GemmF32Args a = f32_args(h, h->C, h->wo, h->bo, h->Z, kHidden, kHidden, kHidden);
+            GemmF32Args a = f32_args(h, h->C, W.wo, W.bo, h->Z, kHidden, kHidden, kHidden);
             a.resid = static_cast<float *>(h->X);
             LAUNCH(L, kProfGemmWoLN, launch_gemm_f32(kF32Resid, a, L.s));
-            LAUNCH(L, kProfLayerNorm, launch_layer_norm_f32(static_cast<float *>(h->Z), static_cast<float *>(h->X1), h->ln1_g, h->ln1_b,
+            LAUNCH(L, kProfLayerNorm, launch_layer_norm_f32(static_cast<float *>(h->Z), static_cast<float *>(h->X1), W.ln1_g, W.ln1_b,
                                                            c.ln_eps, h->rows_cap, h->n_rows, h->status, L.s));
-            LAUNCH(L, kProfGemmW1Gelu, launch_gemm_f32(kF32Gelu, f32_args(h, h->X1, h->w1, h->b1, h->H, kFfn, kFfn, kHidden), L.s));
-            a = f32_args(h, h->H, h->w2, h->b2, h->Z, kHidden, kHidden, kFfn);
+            LAUNCH(L, kProfGemmW1Gelu, launch_gemm_f32(kF32Gelu, f32_args(h, h->X1, W.w1, W.b1, h->H, kFfn, kFfn, kHidden), L.s));
+            a = f32_args(h, h->H, W.w2, W.b2, h->Z, kHidden, kHidden, kFfn);
             a.resid = static_cast<float *>(h->X1);
             LAUNCH(L, kProfGemmW2LN, launch_gemm_f32(kF32Resid, a, L.s));
-            LAUNCH(L, kProfLayerNorm, launch_layer_norm_f32(static_cast<float *>(h->Z), static_cast<float *>(h->X), h->ln2_g, h->ln2_b,
+            LAUNCH(L, kProfLayerNorm, launch_layer_norm_f32(static_cast<float *>(h->Z), static_cast<float *>(h->X), W.ln2_g, W.ln2_b,
                                                            c.ln_eps, h->rows_cap, h->n_rows, h->status, L.s));
         }
         if (c.out_dim > 0) {
@@ -382,57 +405,71 @@ int create_impl(albert_handle *h, const albert_weights *w) {
     TRY(cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking));
     struct StreamGuard { cudaStream_t s; ~StreamGuard() { cudaStreamDestroy(s); } } guard{s};
 
-    // ---- small fp32 parameters: one block ----
-    const size_t V = c.vocab, P = c.max_pos, NT = c.n_types, O = c.out_dim;
+    // ---- small fp32 parameters: one block (shared ones, then per group) ----
+    const size_t V = c.vocab, P = c.max_pos, NT = c.n_types, O = c.out_dim, G = c.n_groups;
     auto sl = [](size_t n) { return (n + 63) / 64 * 64; };
-    const size_t n_small = sl(V * kEmb) + sl(P * kEmb) + sl(NT * kEmb) + 2 * sl(kEmb) + sl(kHidden) + sl(kQKV) +
-                           sl(kHidden) + 2 * sl(kHidden) + sl(kFfn) + sl(kHidden) + 2 * sl(kHidden) + sl(O);
+    const size_t n_group_small = sl(kQKV) + sl(kHidden) + 2 * sl(kHidden) + sl(kFfn) + sl(kHidden) + 2 * sl(kHidden);
+    const size_t n_small = sl(V * kEmb) + sl(P * kEmb) + sl(NT * kEmb) + 2 * sl(kEmb) + sl(kHidden) + sl(O) +
+                           G * n_group_small;
     float *small = nullptr;
     if ((rc = dev_alloc(h, (void **)&small, n_small * sizeof(float)))) return rc;
     float *q = small;
     // slices start on 256-byte boundaries (kernels read several of them as float4)
     auto take = [&](size_t n) { float *r = q; q += (n + 63) / 64 * 64; return r; };
     h->word = take(V * kEmb); h->pos = take(P * kEmb); h->type = take(NT * kEmb);
-    h->emb_g = take(kEmb); h->emb_b = take(kEmb); h->b_in = take(kHidden); h->bqkv = take(kQKV);
-    h->bo = take(kHidden); h->ln1_g = take(kHidden); h->ln1_b = take(kHidden); h->b1 = take(kFfn);
-    h->b2 = take(kHidden); h->ln2_g = take(kHidden); h->ln2_b = take(kHidden); h->b_out = take(O);
+    h->emb_g = take(kEmb); h->emb_b = take(kEmb); h->b_in = take(kHidden); h->b_out = take(O);
     if ((rc = copy_param(h->word, w->word, V * kEmb, s))) return rc;
     if ((rc = copy_param(h->pos, w->pos, P * kEmb, s))) return rc;
     if ((rc = copy_param(h->type, w->type, NT * kEmb, s))) return rc;
     if ((rc = copy_param(h->emb_g, w->emb_ln_g, kEmb, s))) return rc;
     if ((rc = copy_param(h->emb_b, w->emb_ln_b, kEmb, s))) return rc;
     if ((rc = copy_param(h->b_in, w->b_in, kHidden, s))) return rc;
-    if ((rc = copy_param(h->bqkv, w->bq, kHidden, s))) return rc;
-    if ((rc = copy_param(h->bqkv + kHidden, w->bk, kHidden, s))) return rc;
-    if ((rc = copy_param(h->bqkv + 2 * kHidden, w->bv, kHidden, s))) return rc;
-    if ((rc = copy_param(h->bo, w->bo, kHidden, s))) return rc;
-    if ((rc = copy_param(h->ln1_g, w->ln1_g, kHidden, s))) return rc;
-    if ((rc = copy_param(h->ln1_b, w->ln1_b, kHidden, s))) return rc;
-    if ((rc = copy_param(h->b1, w->b1, kFfn, s))) return rc;
-    if ((rc = copy_param(h->b2, w->b2, kHidden, s))) return rc;
-    if ((rc = copy_param(h->ln2_g, w->ln2_g, kHidden, s))) return rc;
-    if ((rc = copy_param(h->ln2_b, w->ln2_b, kHidden, s))) return rc;
     if (O && (rc = copy_param(h->b_out, w->b_out, O, s))) return rc;
+    h->grp.assign(G, albert_handle::Group{});
+    for (size_t g = 0; g < G; ++g) {
+        auto &gp = h->grp[g];
+        gp.bqkv = take(kQKV); gp.bo = take(kHidden); gp.ln1_g = take(kHidden); gp.ln1_b = take(kHidden);
+        gp.b1 = take(kFfn); gp.b2 = take(kHidden); gp.ln2_g = take(kHidden); gp.ln2_b = take(kHidden);
+        // group g's copy of each per-layer tensor follows group g-1's
+        if ((rc = copy_param(gp.bqkv, w->bq + g * kHidden, kHidden, s))) return rc;
+        if ((rc = copy_param(gp.bqkv + kHidden, w->bk + g * kHidden, kHidden, s))) return rc;
+        if ((rc = copy_param(gp.bqkv + 2 * kHidden, w->bv + g * kHidden, kHidden, s))) return rc;
+        if ((rc = copy_param(gp.bo, w->bo + g * kHidden, kHidden, s))) return rc;
+        if ((rc = copy_param(gp.ln1_g, w->ln1_g + g * kHidden, kHidden, s))) return rc;
+        if ((rc = copy_param(gp.ln1_b, w->ln1_b + g * kHidden, kHidden, s))) return rc;
+        if ((rc = copy_param(gp.b1, w->b1 + g * kFfn, kFfn, s))) return rc;
+        if ((rc = copy_param(gp.b2, w->b2 + g * kHidden, kHidden, s))) return rc;
+        if ((rc = copy_param(gp.ln2_g, w->ln2_g + g * kHidden, kHidden, s))) return rc;
+        if ((rc = copy_param(gp.ln2_b, w->ln2_b + g * kHidden, kHidden, s))) return rc;
+    }
 
     // ---- matrices: one contiguous block (bf16 or fp32), 256-byte aligned pieces ----
     const size_t n_win = (size_t)kHidden * kEmb, n_qkv = (size_t)kQKV * kHidden, n_wo = (size_t)kHidden * kHidden;
     const size_t n_w1 = (size_t)kFfn * kHidden, n_w2 = (size_t)kHidden * kFfn, n_out = O * kHidden;
     auto al = [](size_t b) { return (b + 255) / 256 * 256; };
-    size_t off_win = 0, off_qkv = off_win + al(n_win * eb), off_wo = off_qkv + al(n_qkv * eb);
-    size_t off_w1 = off_wo + al(n_wo * eb), off_w2 = off_w1 + al(n_w1 * eb), off_out = off_w2 + al(n_w2 * eb);
+    const size_t group_bytes = al(n_qkv * eb) + al(n_wo * eb) + al(n_w1 * eb) + al(n_w2 * eb);
+    const size_t off_groups = al(n_win * eb), off_out = off_groups + G * group_bytes;
     h->wblock_bytes = off_out + al(n_out * eb);
     if ((rc = dev_alloc(h, &h->wblock, h->wblock_bytes))) return rc;
     uint8_t *wb = static_cast<uint8_t *>(h->wblock);
-    h->w_in = wb + off_win; h->wqkv = wb + off_qkv; h->wo = wb + off_wo;
-    h->w1 = wb + off_w1; h->w2 = wb + off_w2; h->w_out = wb + off_out;
+    h->w_in = wb;
+    h->w_out = wb + off_out;
     if ((rc = copy_matrix(h, h->w_in, w->w_in, n_win, s))) return rc;
-    if ((rc = copy_matrix(h, h->wqkv, w->wq, n_wo, s))) return rc;
-    if ((rc = copy_matrix(h, static_cast<uint8_t *>(h->wqkv) + n_wo * eb, w->wk, n_wo, s))) return rc;
-    if ((rc = copy_matrix(h, static_cast<uint8_t *>(h->wqkv) + 2 * n_wo * eb, w->wv, n_wo, s))) return rc;
-    if ((rc = copy_matrix(h, h->wo, w->wo, n_wo, s))) return rc;
-    if ((rc = copy_matrix(h, h->w1, w->w1, n_w1, s))) return rc;
-    if ((rc = copy_matrix(h, h->w2, w->w2, n_w2, s))) return rc;
     if (O && (rc = copy_matrix(h, h->w_out, w->w_out, n_out, s))) return rc;
+    for (size_t g = 0; g < G; ++g) {
+        auto &gp = h->grp[g];
+        uint8_t *gb = wb + off_groups + g * group_bytes;
+        gp.wqkv = gb;
+        gp.wo = gb + al(n_qkv * eb);
+        gp.w1 = static_cast<uint8_t *>(gp.wo) + al(n_wo * eb);
+        gp.w2 = static_cast<uint8_t *>(gp.w1) + al(n_w1 * eb);
+        if ((rc = copy_matrix(h, gp.wqkv, w->wq + g * n_wo, n_wo, s))) return rc;
+        if ((rc = copy_matrix(h, static_cast<uint8_t *>(gp.wqkv) + n_wo * eb, w->wk + g * n_wo, n_wo, s))) return rc;
+        if ((rc = copy_matrix(h, static_cast<uint8_t *>(gp.wqkv) + 2 * n_wo * eb, w->wv + g * n_wo, n_wo, s))) return rc;
+        if ((rc = copy_matrix(h, gp.wo, w->wo + g * n_wo, n_wo, s))) return rc;
+        if ((rc = copy_matrix(h, gp.w1, w->w1 + g * n_w1, n_w1, s))) return rc;
+        if ((rc = copy_matrix(h, gp.w2, w->w2 + g * n_w2, n_w2, s))) return rc;
+    }
 
     // ---- workspace ----
     if ((rc = dev_alloc(h, &h->E, R * kEmb * eb))) return rc;
@@ -450,18 +487,30 @@ int create_impl(albert_handle *h, const albert_weights *w) {
         TRY(cudaMemsetAsync(h->st2, 0, nst * sizeof(float2), s));
         // every vector starts on a 256-byte boundary: the epilogues read them as float4
         auto seg = [](size_t n) { return (n + 63) / 64 * 64; };
-        const size_t nf = 2 * seg(kQKV) + 2 * seg(kFfn) + 2 * seg(O) + 2 * seg(kHidden);
+        const int NX = c.n_exec;
+        const size_t nf = G * (seg(kFfn) * 2 + seg(kHidden)) + (size_t)NX * (2 * seg(kQKV) + seg(kHidden)) + 2 * seg(O);
         if ((rc = dev_alloc(h, (void **)&h->fold, nf * sizeof(float)))) return rc;
         float *f = h->fold;
-        h->s_qkv = f; f += seg(kQKV); h->c_qkv = f; f += seg(kQKV);
-        h->s_1 = f; f += seg(kFfn); h->c_1 = f; f += seg(kFfn);
-        h->s_out = f; f += seg(O); h->c_out = f; f += seg(O);
-        h->bias_o2 = f; f += seg(kHidden); h->bias_21 = f;
-        TRY(launch_fold_ln(static_cast<const bf16 *>(h->wqkv), kQKV, kHidden, h->ln2_g, h->ln2_b, h->bqkv, h->s_qkv, h->c_qkv, s));
-        TRY(launch_fold_ln(static_cast<const bf16 *>(h->w1), kFfn, kHidden, h->ln1_g, h->ln1_b, h->b1, h->s_1, h->c_1, s));
-        if (O) TRY(launch_fold_ln(static_cast<const bf16 *>(h->w_out), (int)O, kHidden, h->ln2_g, h->ln2_b, h->b_out, h->s_out, h->c_out, s));
-        TRY(launch_vec_add(h->bo, h->ln2_b, h->bias_o2, kHidden, s));
-        TRY(launch_vec_add(h->b2, h->ln1_b, h->bias_21, kHidden, s));
+        for (auto &gp : h->grp) {
+            gp.s_1 = f; f += seg(kFfn); gp.c_1 = f; f += seg(kFfn); gp.bias_21 = f; f += seg(kHidden);
+            TRY(launch_fold_ln(static_cast<const bf16 *>(gp.w1), kFfn, kHidden, gp.ln1_g, gp.ln1_b, gp.b1, gp.s_1, gp.c_1, s));
+            TRY(launch_vec_add(gp.b2, gp.ln1_b, gp.bias_21, kHidden, s));
+        }
+        h->ex.assign(NX, albert_handle::Exec{});
+        for (int l = 1; l < NX; ++l) {
+            auto &e = h->ex[l];
+            const auto &cur = h->grp[group_of(c, l)], &prev = h->grp[group_of(c, l - 1)];
+            e.s_qkv = f; f += seg(kQKV); e.c_qkv = f; f += seg(kQKV); e.bias_o2 = f; f += seg(kHidden);
+            TRY(launch_fold_ln(static_cast<const bf16 *>(cur.wqkv), kQKV, kHidden, prev.ln2_g, prev.ln2_b, cur.bqkv,
+                               e.s_qkv, e.c_qkv, s));
+            TRY(launch_vec_add(cur.bo, prev.ln2_b, e.bias_o2, kHidden, s));
+        }
+        h->s_out = f; f += seg(O); h->c_out = f;
+        if (O && NX > 0) {
+            const auto &last = h->grp[group_of(c, NX - 1)];
+            TRY(launch_fold_ln(static_cast<const bf16 *>(h->w_out), (int)O, kHidden, last.ln2_g, last.ln2_b, h->b_out,
+                               h->s_out, h->c_out, s));
+        }
     }
     if ((rc = dev_alloc(h, (void **)&h->seq_start, (h->seq_cap + 1) * sizeof(int)))) return rc;
     if ((rc = dev_alloc(h, (void **)&h->seq_len, (h->seq_cap + 1) * sizeof(int)))) return rc;
@@ -485,15 +534,17 @@ int create_impl(albert_handle *h, const albert_weights *w) {
             make_tmap_bf16(&h->tm_H, h->H, R, kFfn, gemm::BM) || make_tmap_bf16(&h->tm_Z, h->Z, R, kHidden, gemm::BM) ||
             make_tmap_bf16(&h->tm_QKV, h->QKV, R, kQKV, 128) || make_tmap_bf16(&h->tm_QKV64, h->QKV, R, kQKV, 64) ||
             make_tmap_bf16(&h->tm_win, h->w_in, kHidden, kEmb, gemm::B_BOX) ||
-            make_tmap_bf16(&h->tm_wqkv, h->wqkv, kQKV, kHidden, gemm::B_BOX) ||
-            make_tmap_bf16(&h->tm_wo, h->wo, kHidden, kHidden, gemm::B_BOX) ||
-            make_tmap_bf16(&h->tm_w1, h->w1, kFfn, kHidden, gemm::B_BOX) ||
-            make_tmap_bf16(&h->tm_w2, h->w2, kHidden, kFfn, gemm::B_BOX) ||
             (O && make_tmap_bf16(&h->tm_wout, h->w_out, O, kHidden, gemm::B_BOX)) ||
             make_tmap_bf16_tile32(&h->t32_X, h->X, R, kHidden) || make_tmap_bf16_tile32(&h->t32_QKV, h->QKV, R, kQKV) ||
             make_tmap_bf16_tile32(&h->t32_X1, h->X1, R, kHidden) || make_tmap_bf16_tile32(&h->t32_H, h->H, R, kFfn) ||
             make_tmap_bf16_tile32(&h->t32_Z, h->Z, R, kHidden))
             return ALBERT_ERR_CUDA;
+        for (auto &gp : h->grp)
+            if (make_tmap_bf16(&gp.tm_wqkv, gp.wqkv, kQKV, kHidden, gemm::B_BOX) ||
+                make_tmap_bf16(&gp.tm_wo, gp.wo, kHidden, kHidden, gemm::B_BOX) ||
+                make_tmap_bf16(&gp.tm_w1, gp.w1, kFfn, kHidden, gemm::B_BOX) ||
+                make_tmap_bf16(&gp.tm_w2, gp.w2, kHidden, kFfn, gemm::B_BOX))
+                return ALBERT_ERR_CUDA;
     }
     TRY(cudaStreamSynchronize(s));
     return ALBERT_OK;
