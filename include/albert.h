@@ -86,6 +86,12 @@ typedef struct {
     int pack;        /* albert_forward: 1 = pack valid tokens by length
                         (the GEMMs run on sum(L_b) rows), 0 = run on all B*T
                         padded rows                                     */
+    int out_layout;  /* albert_forward output: 0 = [B, T, D] token-major;
+                        1 = [B, D, T], each sequence's projection transposed
+                        ("ALBERT: How Kokoro's Phoneme Encoder Works", section
+                        "Inside One Real ALBERT Layer": Kokoro projects to
+                        [T, 512] and transposes it).  Padding positions are
+                        0 in both.  albert_forward_varlen needs 0.      */
     float ln_eps;    /* LayerNorm epsilon, 1e-12 for Kokoro             */
 } albert_config;
 

@@ -52,7 +52,7 @@ def test_config_struct_matches_header_field_order():
     body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
     fields = re.findall(r"\b(\w+)\s*;", body)
     assert fields == [f for f, _ in tea.albert_config._fields_]
-    assert C.sizeof(tea.albert_config) == 14 * 4
+    assert C.sizeof(tea.albert_config) == 4 * len(fields)  # 4-byte ints and one float
 
 
 def test_weights_struct_matches_header_field_order():
@@ -78,14 +78,14 @@ def test_host_side_rejections_need_no_gpu(lib):
     lib.albert_destroy(None)
 
 
-def test_create_rejects_bad_group_counts_before_touching_the_device():
+def test_create_rejects_bad_group_counts_and_layouts_before_touching_the_device():
     """albert_create validates the config on the host first: these return
     ALBERT_ERR_CONFIG without any CUDA call (the weight pointers are never read)."""
     import transformer_encoder_albert_b200 as tea
     lib = tea.lib()
     dummy = tea.albert_weights(*([C.c_void_p(16)] * len(tea.WEIGHT_FIELDS)))
-    for n_exec, n_groups in ((12, 0), (3, 4), (0, 2), (12, -1)):
-        cfg = tea.make_config(synth.ARCH, n_exec=n_exec, n_groups=n_groups)
+    for n_exec, n_groups, layout in ((12, 0, 0), (3, 4, 0), (0, 2, 0), (12, -1, 0), (12, 1, 2), (12, 1, -1)):
+        cfg = tea.make_config(synth.ARCH, n_exec=n_exec, n_groups=n_groups, out_layout=layout)
         h = C.c_void_p()
         assert lib.albert_create(C.byref(dummy), C.byref(cfg), C.byref(h)) == 2  # ALBERT_ERR_CONFIG
         assert h.value is None

@@ -150,6 +150,45 @@ def test_grouped_sharing_rejects_more_groups_than_executions():
         tea.Encoder(w, A, max_tokens=64, n_exec=3, n_groups=4)
 
 
+@pytest.mark.parametrize("dtype,out_dim", [("bf16", 512), ("bf16", 0), ("fp32", 512)])
+def test_transposed_output_layout(w_bf16, w_fp32, dtype, out_dim):
+    """out_layout 1 returns [B, D, T]: the token-major output transposed per
+    sequence (same arithmetic, so bit-equal), zeros at padding positions."""
+    w = w_bf16 if dtype == "bf16" else w_fp32
+    wl = synth.WORKLOADS["b8_T128"] if dtype == "bf16" else synth.Workload("t32", 3, 40, "uniform", lo=3, hi=40, seed=91)
+    ids, mask, L = synth.make_batch(wl)
+    n_exec = None if dtype == "bf16" else 2
+    a = tea.Encoder(w, A, dtype=dtype, max_tokens=wl.B * wl.T, n_exec=n_exec, out_dim=out_dim)
+    b = tea.Encoder(w, A, dtype=dtype, max_tokens=wl.B * wl.T, n_exec=n_exec, out_dim=out_dim, out_layout=1)
+    tok = a.forward(_t(ids), _t(mask)).cpu()
+    tr = b.forward(_t(ids), _t(mask)).cpu()
+    assert a.status() == 0 and b.status() == 0
+    D = out_dim or 768
+    assert tuple(tr.shape) == (wl.B, D, wl.T)
+    assert torch.equal(tr, tok.transpose(1, 2))
+    # against the oracle on two sequences
+    ref = oracle_rows(w, ids, mask, L, [0, 1], n_exec=n_exec, out_dim=out_dim)
+    for s in (0, 1):
+        n = int(L[s])
+        got = tr[s, :, :n].float().numpy().T
+        if dtype == "fp32":
+            check_fp32(got, ref[s], f"transposed seq {s}")
+        else:
+            check_bf16(got, ref[s], f"transposed seq {s}", checkpoint=(out_dim == 0))
+    # the host path fills the same [B, D, T] buffer
+    if dtype == "bf16" and out_dim == 512:
+        out_h = torch.empty(wl.B, D, wl.T, dtype=torch.bfloat16).pin_memory()
+        assert b.forward_host(torch.as_tensor(ids).pin_memory(), torch.as_tensor(mask).pin_memory(), out_h) == 0
+        assert torch.equal(out_h, tr)
+    # packed rows have no per-sequence [D, T] form
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(L)]).astype(np.int32), device="cuda")
+    packed = _t(np.concatenate([ids[s, :L[s]] for s in range(wl.B)]))
+    with pytest.raises(tea.AlbertError):
+        b.forward_varlen(packed, cu, int(L.max()))
+    a.close()
+    b.close()
+
+
 def test_fp32_small_padded_batch(w_fp32):
     wl = synth.Workload("fp32b", 3, 40, "uniform", lo=2, hi=40, seed=79, dtype="fp32", out_dim=512)
     ids, mask, L, got = _run(w_fp32, wl, dtype="fp32", n_exec=3)

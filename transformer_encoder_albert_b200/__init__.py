@@ -50,7 +50,8 @@ class AlbertError(RuntimeError):
 
 class albert_config(C.Structure):
     _fields_ = [(n, C.c_int) for n in ("vocab", "emb", "hidden", "heads", "ffn", "n_exec", "n_groups",
-                                       "max_pos", "n_types", "out_dim", "dtype", "max_tokens", "pack")] \
+                                       "max_pos", "n_types", "out_dim", "dtype", "max_tokens", "pack",
+                                       "out_layout")] \
         + [("ln_eps", C.c_float)]
 
 
@@ -112,14 +113,15 @@ def _ptr(t) -> int | None:
 
 
 def make_config(arch: dict, dtype: str = "bf16", max_tokens: int = 4096, pack: bool = True,
-                n_exec: int | None = None, out_dim: int | None = None, n_groups: int = 1) -> albert_config:
+                n_exec: int | None = None, out_dim: int | None = None, n_groups: int = 1,
+                out_layout: int = 0) -> albert_config:
     return albert_config(
         vocab=arch["vocab"], emb=arch["emb"], hidden=arch["hidden"], heads=arch["heads"],
         ffn=arch["ffn"], n_exec=arch["n_exec"] if n_exec is None else n_exec, n_groups=n_groups,
         max_pos=arch["max_pos"], n_types=arch["n_types"],
         out_dim=arch["out_dim"] if out_dim is None else out_dim,
         dtype=ALBERT_BF16 if dtype == "bf16" else ALBERT_FP32, max_tokens=max_tokens,
-        pack=1 if pack else 0, ln_eps=arch["ln_eps"])
+        pack=1 if pack else 0, out_layout=out_layout, ln_eps=arch["ln_eps"])
 
 
 # ---------------------------------------------------------------- C names --
@@ -184,10 +186,13 @@ class Encoder:
     """Owns one library handle.  Outputs are bf16 (dtype "bf16") or fp32 tensors."""
 
     def __init__(self, weights: dict, arch: dict, dtype: str = "bf16", max_tokens: int = 4096,
-                 pack: bool = True, n_exec: int | None = None, out_dim: int | None = None, n_groups: int = 1):
+                 pack: bool = True, n_exec: int | None = None, out_dim: int | None = None, n_groups: int = 1,
+                 out_layout: int = 0):
         """n_groups > 1: the layer parameters of `weights` hold n_groups stacked sets
-        (leading axis), execution i using set i * n_groups // n_exec."""
-        self.cfg = make_config(arch, dtype, max_tokens, pack, n_exec, out_dim, n_groups)
+        (leading axis), execution i using set i * n_groups // n_exec.  out_layout 1:
+        forward() returns [B, D, T] (each sequence's output transposed)."""
+        self.cfg = make_config(arch, dtype, max_tokens, pack, n_exec, out_dim, n_groups, out_layout)
+        self.out_layout = out_layout
         self.dtype = dtype
         self.out_dim = self.cfg.out_dim if self.cfg.out_dim > 0 else self.cfg.hidden
         self.h = albert_create(weights, self.cfg)
@@ -199,7 +204,12 @@ class Encoder:
 
     def forward(self, ids, mask, out=None, stream=None):
         if out is None:
-            out = self._out(ids.shape)
+            if self.out_layout == 1:
+                import torch
+                dt = torch.bfloat16 if self.dtype == "bf16" else torch.float32
+                out = torch.empty(ids.shape[0], self.out_dim, ids.shape[1], device="cuda", dtype=dt)
+            else:
+                out = self._out(ids.shape)
         albert_forward(self.h, ids, mask, out, stream)
         return out
 

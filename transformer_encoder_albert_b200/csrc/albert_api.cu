@@ -75,6 +75,9 @@ struct albert_handle {
     float *s_out = nullptr, *c_out = nullptr;
     int *seq_start = nullptr, *seq_len = nullptr, *row_dst = nullptr, *n_rows = nullptr, *status = nullptr;
 
+    // out_layout 1: token-major staging of the output, transposed per sequence into `out`
+    void *tout = nullptr;
+
     // host-buffer staging
     int64_t *st_ids = nullptr;
     uint8_t *st_mask = nullptr;
@@ -148,6 +151,7 @@ int check_config(const albert_config *c) {
     if (c->dtype != ALBERT_BF16 && c->dtype != ALBERT_FP32) return ALBERT_ERR_CONFIG;
     if (c->max_tokens < 1 || c->max_tokens > (1 << 24)) return ALBERT_ERR_CONFIG;
     if (c->pack != 0 && c->pack != 1) return ALBERT_ERR_CONFIG;
+    if (c->out_layout != 0 && c->out_layout != 1) return ALBERT_ERR_CONFIG;
     if (!(c->ln_eps >= 0.f)) return ALBERT_ERR_CONFIG;
     return ALBERT_OK;
 }
@@ -249,6 +253,10 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
                int max_len, void *out, int padded_api) {
     const albert_config &c = h->cfg;
     const int out_rows = padded_api ? nseq * T : c.max_tokens;
+    // out_layout 1: the final stage writes token-major rows to the staging buffer,
+    // which the last kernel transposes per sequence into the caller's output
+    void *const user_out = out;
+    if (padded_api && c.out_layout == 1) out = h->tout;
     const bool bf = c.dtype == ALBERT_BF16;
     EmbedArgs ea{};
     ea.ids = ids;
@@ -370,7 +378,10 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
             LAUNCH(L, kProfOutput, launch_scatter_rows(h->X, out, kHidden, 4, h->rows_cap, h->n_rows, h->row_dst, h->status, L.s));
         }
     }
-    if (padded_api)
+    if (padded_api && c.out_layout == 1)
+        LAUNCH(L, kProfOutput, launch_transpose_out(h->tout, user_out, nseq, T, D, (int)elem_bytes(h), h->seq_len,
+                                                    h->status, L.s));
+    else if (padded_api)
         LAUNCH(L, kProfOutput, launch_zero_pad(out, nseq, T, D, (int)elem_bytes(h), h->seq_len, h->status, L.s));
     return ALBERT_OK;
 }
@@ -520,6 +531,7 @@ int create_impl(albert_handle *h, const albert_weights *w) {
     if ((rc = dev_alloc(h, (void **)&h->st_ids, (size_t)c.max_tokens * sizeof(int64_t)))) return rc;
     if ((rc = dev_alloc(h, (void **)&h->st_mask, (size_t)c.max_tokens))) return rc;
     if ((rc = dev_alloc(h, &h->st_out, (size_t)c.max_tokens * out_width(h) * eb))) return rc;
+    if (c.out_layout == 1 && (rc = dev_alloc(h, &h->tout, (size_t)c.max_tokens * out_width(h) * eb))) return rc;
     // Deterministic contents for rows a forward never writes.
     for (void *p : {h->E, h->X, h->QKV, h->C, h->X1, h->H, h->Z}) {
         size_t bytes = (p == h->E ? kEmb : p == h->QKV ? kQKV : p == h->H ? kFfn : kHidden) * R * eb;
@@ -608,6 +620,7 @@ int albert_forward_varlen(albert_handle *h, const int64_t *ids, const int32_t *c
                           int max_len, void *out, void *stream) {
     if (!h || !ids || !cu_seqlens || !out) return ALBERT_ERR_NULL;
     if (nseq < 1 || nseq > h->seq_cap || max_len < 1 || max_len > h->cfg.max_pos) return ALBERT_ERR_SHAPE;
+    if (h->cfg.out_layout != 0) return ALBERT_ERR_CONFIG;  // packed rows have no per-sequence [D, T] form
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Launch L{h, s};
     LAUNCH(L, kProfPrep, launch_prep_varlen(cu_seqlens, nseq, max_len, h->cfg.max_tokens, h->seq_start, h->seq_len,

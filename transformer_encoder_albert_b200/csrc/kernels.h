@@ -169,6 +169,10 @@ struct EmbedArgs {
     int trigger;        // the next launch is one of ours with PDL (see GemmArgs)
 };
 cudaError_t launch_embed(const EmbedArgs &a, cudaStream_t s);
+// out[b][d][t] = t < seq_len[b] ? src[(b*T + t)*D + d] : 0 (elem_bytes 2 or 4),
+// the last kernel of a forward with the transposed output layout.
+cudaError_t launch_transpose_out(const void *src, void *out, int B, int T, int D, int elem_bytes,
+                                 const int *seq_len, const int *status, cudaStream_t s);
 
 // out[(b*T + t)] = 0 for padding slots t >= seq_len[b]; D columns of elem_bytes.
 cudaError_t launch_zero_pad(void *out, int B, int T, int D, int elem_bytes, const int *seq_len,

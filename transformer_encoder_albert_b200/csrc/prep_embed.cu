@@ -189,6 +189,30 @@ __global__ void zero_pad_kernel(uint4 *out, int B, int T, int chunks_per_row, co
     }
 }
 
+// Per sequence b: a [T, D] block of token-major rows -> [D, T], through 32x32
+// shared tiles (reads along d, writes along t, both coalesced); padding slots 0.
+template <typename E>
+__global__ void __launch_bounds__(256)
+transpose_out_kernel(const E *__restrict__ src, E *__restrict__ out, int T, int D, const int *__restrict__ seq_len,
+                     const int *status) {
+    // last kernel of a forward: no early trigger
+    griddep_wait();               // the previous kernel has completed
+    if (*reinterpret_cast<const volatile int *>(status) != 0) return;
+    __shared__ E tile[32][33];
+    const int b = blockIdx.z, t0 = blockIdx.x * 32, d0 = blockIdx.y * 32;
+    const int L = __ldg(seq_len + b);
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+    for (int k = ty; k < 32; k += 8) {
+        const int t = t0 + k, d = d0 + tx;
+        tile[k][tx] = (t < L && d < D) ? src[((size_t)b * T + t) * D + d] : E(0);
+    }
+    __syncthreads();
+    for (int k = ty; k < 32; k += 8) {
+        const int d = d0 + k, t = t0 + tx;
+        if (d < D && t < T) out[((size_t)b * D + d) * T + t] = tile[tx][k];
+    }
+}
+
 __global__ void scatter_rows_kernel(const uint4 *X, uint4 *out, int chunks_per_row, int rows_cap,
                                     const int *n_rows, const int *row_dst, const int *status) {
     // last kernel of a forward: no early trigger, so that whatever follows in the
@@ -248,6 +272,16 @@ cudaError_t launch_zero_pad(void *out, int B, int T, int D, int elem_bytes, cons
     const size_t n = (size_t)B * T * cpr;
     return launch_pdl(zero_pad_kernel, dim3(grid_for(n, 256)), dim3(256), 0, s, static_cast<uint4 *>(out), B, T, cpr,
                       seq_len, status);
+}
+
+cudaError_t launch_transpose_out(const void *src, void *out, int B, int T, int D, int elem_bytes,
+                                 const int *seq_len, const int *status, cudaStream_t s) {
+    const dim3 grid((T + 31) / 32, (D + 31) / 32, B);
+    if (elem_bytes == 2)
+        return launch_pdl(transpose_out_kernel<uint16_t>, grid, dim3(256), 0, s, static_cast<const uint16_t *>(src),
+                          static_cast<uint16_t *>(out), T, D, seq_len, status);
+    return launch_pdl(transpose_out_kernel<float>, grid, dim3(256), 0, s, static_cast<const float *>(src),
+                      static_cast<float *>(out), T, D, seq_len, status);
 }
 
 cudaError_t launch_scatter_rows(const void *X, void *out, int D, int elem_bytes, int rows_cap,
