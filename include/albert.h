@@ -189,6 +189,15 @@ int albert_launches_per_forward(const albert_handle *h, int padded_api);
  * summed milliseconds since the last reset.  Classes are numbered
  * 0..albert_profile_classes()-1 and named by albert_profile_name(). */
 int albert_profile_enable(albert_handle *h, int class_mask);
+/* retain = 1: a read keeps the recorded event pairs armed instead of recycling
+ * them.  For a forward captured in a CUDA graph with profiling enabled: every
+ * replay re-records the same events, and a read after each replay adds that
+ * replay's times.  retain = 0 (default) disarms them. */
+int albert_profile_retain(albert_handle *h, int retain);
+/* Time only launch k of each enabled class with k % stride == offset, k counted
+ * per class from this call (default stride 1: every launch).  Fewer event
+ * records between launches keep more of the launch chaining intact. */
+int albert_profile_stride(albert_handle *h, int stride, int offset);
 int albert_profile_reset(albert_handle *h);
 int albert_profile_classes(void);
 const char *albert_profile_name(int cls);

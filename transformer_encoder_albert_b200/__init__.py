@@ -36,7 +36,8 @@ EXPORTS = (
     "albert_create", "albert_forward", "albert_forward_varlen", "albert_forward_host",
     "albert_forward_host_async", "albert_forward_host_wait",
     "albert_get_status", "albert_destroy", "albert_launches_per_forward",
-    "albert_profile_enable", "albert_profile_reset", "albert_profile_classes",
+    "albert_profile_enable", "albert_profile_retain", "albert_profile_stride", "albert_profile_reset",
+    "albert_profile_classes",
     "albert_profile_name", "albert_profile_read", "albert_test_gemm", "albert_test_attention",
     "albert_gemm_residual_ln_noalloc", "albert_length_regulate", "albert_length_regulate_scratch_bytes",
 )
@@ -83,6 +84,8 @@ def lib() -> C.CDLL:
         L.albert_launches_per_forward.argtypes = [vp, i]
         L.albert_profile_enable.argtypes = [vp, i]
         L.albert_profile_reset.argtypes = [vp]
+        L.albert_profile_retain.argtypes = [vp, i]
+        L.albert_profile_stride.argtypes = [vp, i, i]
         L.albert_profile_classes.argtypes = []
         L.albert_profile_name.argtypes = [i]
         L.albert_profile_name.restype = C.c_char_p
@@ -247,6 +250,14 @@ class Encoder:
             for c in classes:
                 mask |= 1 << names.index(c)
         _check(lib().albert_profile_enable(self.h, mask), "albert_profile_enable")
+
+    def profile_retain(self, on: bool) -> None:
+        """Keep recorded event pairs armed across reads (CUDA-graph replays)."""
+        _check(lib().albert_profile_retain(self.h, 1 if on else 0), "albert_profile_retain")
+
+    def profile_stride(self, stride: int, offset: int = 0) -> None:
+        """Time only launch k of each enabled class with k % stride == offset."""
+        _check(lib().albert_profile_stride(self.h, stride, offset), "albert_profile_stride")
 
     def profile_reset(self) -> None:
         _check(lib().albert_profile_reset(self.h), "albert_profile_reset")

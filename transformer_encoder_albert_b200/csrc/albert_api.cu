@@ -104,6 +104,10 @@ struct albert_handle {
 
     // per-kernel timing
     unsigned prof_mask = 0;  // classes whose launches are timed
+    bool prof_retain = false;  // keep recorded pairs armed after a read (graph replays)
+    int prof_stride = 1, prof_offset = 0;  // time launch k of a class iff k % stride == offset
+    int prof_count[kProfClasses] = {};      // launches of each class since the stride was set
+    bool prof_open = false;                 // begin() recorded a start event for this launch
     std::vector<cudaEvent_t> ev;
     std::vector<int> ev_cls;
     int ev_used = 0;
@@ -166,7 +170,7 @@ int prof_harvest(albert_handle *h) {
         h->prof_ms[h->ev_cls[i]] += ms;
         h->prof_launches[h->ev_cls[i]] += 1;
     }
-    h->ev_used = 0;
+    if (!h->prof_retain) h->ev_used = 0;
     return ALBERT_OK;
 }
 
@@ -174,15 +178,28 @@ struct Launch {
     albert_handle *h;
     cudaStream_t s;
     int cls = -1;
+    // Inside stream capture a plain event record only orders captured streams;
+    // an external record becomes a graph node that records the event on replay.
+    cudaError_t record(cudaEvent_t e) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        cudaError_t err = cudaStreamIsCapturing(s, &cs);
+        if (err != cudaSuccess) return err;
+        return cudaEventRecordWithFlags(e, s, cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal
+                                                                                    : cudaEventRecordDefault);
+    }
     int begin(int c) {
         cls = c;
+        h->prof_open = false;
         if (!(h->prof_mask >> c & 1u)) return ALBERT_OK;
+        if (h->prof_count[c]++ % h->prof_stride != h->prof_offset) return ALBERT_OK;
+        h->prof_open = true;
         if (h->ev_used + 2 > kEventPool) {
+            if (h->prof_retain) return ALBERT_ERR_CONFIG;  // armed pairs cannot be recycled
             int rc = prof_harvest(h);
             if (rc) return rc;
         }
         h->ev_cls[h->ev_used] = c;
-        TRY(cudaEventRecord(h->ev[h->ev_used++], s));
+        TRY(record(h->ev[h->ev_used++]));
         return ALBERT_OK;
     }
     int end(cudaError_t launched) {
@@ -191,9 +208,9 @@ struct Launch {
                 fprintf(stderr, "albert: launch of %s failed: %s\n", kProfNames[cls], cudaGetErrorString(launched));
             return ALBERT_ERR_CUDA;
         }
-        if (!(h->prof_mask >> cls & 1u)) return ALBERT_OK;
+        if (!h->prof_open) return ALBERT_OK;
         h->ev_cls[h->ev_used] = cls;
-        TRY(cudaEventRecord(h->ev[h->ev_used++], s));
+        TRY(record(h->ev[h->ev_used++]));
         return ALBERT_OK;
     }
 };
@@ -747,6 +764,22 @@ int albert_profile_reset(albert_handle *h) {
     int rc = prof_harvest(h);
     for (int i = 0; i < kProfClasses; ++i) { h->prof_launches[i] = 0; h->prof_ms[i] = 0.0; }
     return rc;
+}
+
+int albert_profile_stride(albert_handle *h, int stride, int offset) {
+    if (!h) return ALBERT_ERR_NULL;
+    if (stride < 1 || offset < 0 || offset >= stride) return ALBERT_ERR_CONFIG;
+    h->prof_stride = stride;
+    h->prof_offset = offset;
+    for (int &n : h->prof_count) n = 0;
+    return ALBERT_OK;
+}
+
+int albert_profile_retain(albert_handle *h, int on) {
+    if (!h) return ALBERT_ERR_NULL;
+    h->prof_retain = on != 0;
+    if (!h->prof_retain) h->ev_used = 0;
+    return ALBERT_OK;
 }
 
 int albert_profile_classes(void) { return kProfClasses; }
