@@ -60,40 +60,49 @@ def forward_flops(lengths, arch):
     return gemm + arch["n_exec"] * f["attention"], gemm
 
 
-# DRAM traffic per launch of a kernel class, from an ncu capture summarised in
-# profiles/.  A line there records the digest of the kernel's sources at capture
-# time; the figure is reported only while the sources are unchanged.
-TRAFFIC_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
-                            "dram_traffic_b256_T128_packed.txt")
+# DRAM traffic per launch of a kernel class, from ncu captures summarised in
+# profiles/dram_traffic_<workload>.txt.  A line there records the digest of the
+# kernel's sources at capture time; the figure is reported only while the
+# sources are unchanged.
+TRAFFIC_GLOB = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "dram_traffic_*.txt")
 CLASS_SOURCES = {
     "gemm": ["gemm_tcgen05.cu", "sm100_ptx.cuh", "kernels.h"],
-    "attention": ["attention_tc.cu", "sm100_ptx.cuh", "kernels.h"],
+    "attention": ["attention_tc.cu", "sm100_ptx.cuh", "kernels.h"],            # longest sequence <= 128
+    "attention_long": ["attention_tc_long.cu", "sm100_ptx.cuh", "kernels.h"],  # 128 < longest <= 512
 }
 
 
-def sources_digest(cls: str) -> str:
+def source_set(cls: str, seq_len: int = 128) -> str:
+    if cls.startswith("gemm_"):
+        return "gemm"
+    return "attention" if seq_len <= 128 else "attention_long"
+
+
+def sources_digest(cls: str, seq_len: int = 128) -> str:
     import hashlib
     csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "transformer_encoder_albert_b200", "csrc")
     h = hashlib.sha256()
-    for f in CLASS_SOURCES["gemm" if cls.startswith("gemm_") else "attention"]:
+    for f in CLASS_SOURCES[source_set(cls, seq_len)]:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def load_traffic(cls: str, workload: str):
+def load_traffic(cls: str, workload: str, seq_len: int = 128):
     """(bytes per launch, note) for a class, or (None, reason)."""
-    try:
-        lines = open(TRAFFIC_FILE).read().splitlines()
-    except OSError:
+    import glob
+    files = sorted(glob.glob(TRAFFIC_GLOB))
+    if not files:
         return None, "no ncu capture summarised"
-    want = sources_digest(cls)
-    for ln in lines:
-        kv = dict(x.split("=", 1) for x in ln.split() if "=" in x)
-        if kv.get("class") == cls and kv.get("workload") == workload:
-            if kv.get("sources") != want:
-                return None, "kernel changed since the ncu capture"
-            return float(kv["dram_bytes_per_launch"]), "ncu capture, " + os.path.basename(TRAFFIC_FILE)
+    want = sources_digest(cls, seq_len)
+    for path in files:
+        with open(path) as fh:
+            for ln in fh.read().splitlines():
+                kv = dict(x.split("=", 1) for x in ln.split() if "=" in x)
+                if kv.get("class") == cls and kv.get("workload") == workload:
+                    if kv.get("sources") != want:
+                        return None, "kernel changed since the ncu capture"
+                    return float(kv["dram_bytes_per_launch"]), "ncu capture, " + os.path.basename(path)
     return None, "class not in the ncu capture"
 
 
@@ -506,7 +515,7 @@ def run_gpu(args):
     lenreg = measure_length_regulation(torch, synth, tea, L, flush, peaks, peaks_src, stream, args.steps)
     dom_ms = dom[1] / max(dom[0], 1)
     achieved = per_launch.get(dominant, 0.0) / (dom_ms / 1000.0) / 1e12
-    traffic, traffic_note = load_traffic(dominant, wl.name + ("_padded" if args.padded else "_packed"))
+    traffic, traffic_note = load_traffic(dominant, wl.name + ("_padded" if args.padded else "_packed"), wl.T)
     roofline = {"kernel": dominant, "bound": "tensor", "achieved": achieved, "peak": peak_sus,
                 "unit": "TFLOP/s", "frac": achieved / peak_sus, "traffic": traffic,
                 "traffic_source": traffic_note,

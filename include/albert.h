@@ -263,8 +263,10 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
 /* Masked bidirectional attention on a packed [N_tok, 3*768] bf16 QKV buffer
  * (Q | K | V, head h = columns 64h..64h+63 of each); cu_seqlens as in
  * albert_forward_varlen; ctx: [N_tok, 768] bf16.  dtype ALBERT_BF16 runs the
- * kernel the forward pass uses for this max_len (tcgen05 for max_len <= 128,
- * else the mma.sync kernel); 2 forces the mma.sync kernel; ALBERT_FP32 runs the
+ * kernel the forward pass uses for this max_len (tcgen05 with one item per
+ * (sequence, head) for max_len <= 128; tcgen05 with one item per (sequence,
+ * 128-query block, head) and all of its scores in tensor memory for
+ * 128 < max_len <= 512); 2 forces the mma.sync kernel; ALBERT_FP32 runs the
  * fp32 kernel on fp32 buffers. */
 int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, int max_len,
                           void *ctx, int dtype, void *stream);

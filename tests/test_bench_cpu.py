@@ -9,7 +9,7 @@ def test_traffic_reported_only_for_unchanged_sources(tmp_path, monkeypatch):
     f.write_text("# comment\n"
                  f"class=gemm_qkv workload=w sources={digest} dram_bytes_per_launch=123456 launches=24\n"
                  "class=attention workload=w sources=0000000000000000 dram_bytes_per_launch=99 launches=24\n")
-    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    monkeypatch.setattr(bench, "TRAFFIC_GLOB", str(f))
     value, note = bench.load_traffic("gemm_qkv", "w")
     assert value == 123456.0 and "ncu" in note
     value, note = bench.load_traffic("attention", "w")
@@ -21,10 +21,24 @@ def test_traffic_reported_only_for_unchanged_sources(tmp_path, monkeypatch):
 
 
 def test_missing_traffic_file(tmp_path, monkeypatch):
-    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "absent.txt"))
+    monkeypatch.setattr(bench, "TRAFFIC_GLOB", str(tmp_path / "absent_*.txt"))
     assert bench.load_traffic("gemm_qkv", "w")[0] is None
 
 
 def test_gemm_classes_share_a_digest_and_attention_differs():
     assert bench.sources_digest("gemm_qkv") == bench.sources_digest("gemm_out_proj_ln")
     assert bench.sources_digest("gemm_qkv") != bench.sources_digest("attention")
+
+
+def test_long_attention_has_its_own_digest_and_lines(tmp_path, monkeypatch):
+    """Batches with a sequence longer than 128 run the long-sequence attention
+    kernel: its traffic line is keyed by that kernel's sources."""
+    short, long_ = bench.sources_digest("attention", 128), bench.sources_digest("attention", 512)
+    assert short != long_
+    assert bench.sources_digest("gemm_qkv", 512) == bench.sources_digest("gemm_qkv", 128)
+    (tmp_path / "dram_traffic_a.txt").write_text(f"class=attention workload=s sources={short} dram_bytes_per_launch=5\n")
+    (tmp_path / "dram_traffic_b.txt").write_text(f"class=attention workload=l sources={long_} dram_bytes_per_launch=7\n")
+    monkeypatch.setattr(bench, "TRAFFIC_GLOB", str(tmp_path / "dram_traffic_*.txt"))
+    assert bench.load_traffic("attention", "s", 128)[0] == 5.0
+    assert bench.load_traffic("attention", "l", 512)[0] == 7.0
+    assert bench.load_traffic("attention", "l", 128)[0] is None

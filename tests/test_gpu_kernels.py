@@ -136,7 +136,19 @@ def test_attention_mma_sync_kernel_short_sequences():
 
 
 def test_attention_bf16_long_sequences():
+    """129 <= max_len <= 512 runs the tcgen05 kernel with one item per
+    (sequence, 128-query block, head)."""
     _attention_case([256, 300, 511, 512], seed=1)
+
+
+def test_attention_tcgen05_long_kernel_every_block_count():
+    """Lengths around every key-block boundary (1 to 4 blocks of 128, ragged last
+    block and last query block) and short sequences sharing the launch."""
+    _attention_case([129, 1, 130, 255, 256, 257, 64, 383, 384, 385, 2, 447, 448, 449, 511, 512, 128, 200], seed=11)
+
+
+def test_attention_mma_sync_kernel_long_sequences():
+    _attention_case([129, 256, 300, 512], seed=12, legacy=True)
 
 
 def test_attention_fp32_ragged_lengths():

@@ -322,6 +322,9 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
             if (max_len <= kAttnTcMaxLen) {
                 LAUNCH(L, kProfAttention, launch_attention_tc(h->tm_QKV, h->tm_QKV64, static_cast<bf16 *>(h->C), h->seq_start,
                                                              h->seq_len, nseq, h->status, h->num_sms, L.s, true));
+            } else if (max_len <= kAttnTcLongMaxLen) {
+                LAUNCH(L, kProfAttention, launch_attention_tc_long(h->tm_QKV, static_cast<bf16 *>(h->C), h->seq_start,
+                                                                  h->seq_len, nseq, h->status, h->num_sms, L.s, true));
             } else {
                 LAUNCH(L, kProfAttention, launch_attention_bf16(static_cast<bf16 *>(h->QKV), static_cast<bf16 *>(h->C),
                                                                h->seq_start, h->seq_len, nseq, max_len, h->status, L.s,
@@ -871,12 +874,16 @@ int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, 
         if (dtype == ALBERT_FP32) {
             e = launch_attention_f32(static_cast<const float *>(qkv), static_cast<float *>(ctx), seq_start, seq_len, nseq,
                                      max_len, status, s);
-        } else if (dtype == ALBERT_BF16 && max_len <= kAttnTcMaxLen) {
+        } else if (dtype == ALBERT_BF16 && max_len <= kAttnTcLongMaxLen) {
             CUtensorMap tm, tm64;
             if (make_tmap_bf16(&tm, qkv, (uint64_t)n_tok, kQKV, 128) || make_tmap_bf16(&tm64, qkv, (uint64_t)n_tok, kQKV, 64))
                 e = cudaErrorInvalidValue;
-            else e = launch_attention_tc(tm, tm64, static_cast<bf16 *>(ctx), seq_start, seq_len, nseq, status, sms, s,
-                                         false);
+            else if (max_len <= kAttnTcMaxLen)
+                e = launch_attention_tc(tm, tm64, static_cast<bf16 *>(ctx), seq_start, seq_len, nseq, status, sms, s,
+                                        false);
+            else
+                e = launch_attention_tc_long(tm, static_cast<bf16 *>(ctx), seq_start, seq_len, nseq, status, sms, s,
+                                             false);
         } else {
             e = launch_attention_bf16(static_cast<const bf16 *>(qkv), static_cast<bf16 *>(ctx), seq_start, seq_len, nseq,
                                       max_len, status, s, false);

@@ -9,6 +9,10 @@
 // [rows, 3*768] buffer (Q | K | V); head h is the 64-column slice 64h..64h+63
 // of each; the context goes to [rows, 768] with the same head layout.
 //
+// The forward pass runs the tcgen05 kernels (attention_tc.cu, attention_tc_long.cu)
+// for bf16; the bf16 kernel here is an independent mma.sync implementation of
+// the same operation, reachable through albert_test_attention as a cross-check.
+//
 // bf16 kernel: one CTA per (sequence, head, query tile of 16 rows per warp;
 // 4 warps for T <= 128, 8 warps above).  The head's whole K and V (L_b <= 512
 // rows of 64 bf16) are staged in shared memory by cp.async, one commit group

@@ -137,6 +137,12 @@ constexpr int kAttnTcMaxLen = 128;
 cudaError_t launch_attention_tc(const CUtensorMap &tmQKV, const CUtensorMap &tmQKV64, bf16 *ctx, const int *seq_start,
                                 const int *seq_len, int nseq, int *status, int num_sms, cudaStream_t s,
                                 bool trigger);
+// Same operation on tcgen05 for 128 < max_len <= 512 (one item = one (sequence,
+// 128-query block, head), the item's scores against all keys held in TMEM);
+// tmQKV as above.
+constexpr int kAttnTcLongMaxLen = 512;
+cudaError_t launch_attention_tc_long(const CUtensorMap &tmQKV, bf16 *ctx, const int *seq_start, const int *seq_len,
+                                     int nseq, int *status, int num_sms, cudaStream_t s, bool trigger);
 cudaError_t launch_attention_f32(const float *qkv, float *ctx, const int *seq_start,
                                  const int *seq_len, int nseq, int max_len,
                                  const int *status, cudaStream_t s);
