@@ -47,11 +47,16 @@ constexpr int NBUF = 4;                        // TMEM item buffers (128 columns
 constexpr int ATC_THREADS = 32 * 14;
 constexpr int ATC_SMEM = 1024 + (2 * NQK + NV) * TILE + NBUF * TROWS * 4 + 512;
 constexpr uint32_t TM_O = 64;                  // O's first column within an item buffer
+// Item n uses Q/K stage, V stage and TMEM buffer n % 4 alike, so a Q/K stage is
+// free when the S product of the item four back completes (s_full) and a V
+// stage when its O product completes (o_full): no separate release barriers,
+// and two fewer tcgen05.commit per item on the issuing thread.
+static_assert(NQK == NBUF && NV == NBUF, "stages and TMEM buffers share one index");
 
 struct AttSmem {
     uint8_t *qk, *v;                           // [NQK][Q tile, K tile], [NV][V tile]
-    uint64_t *qk_full, *qk_empty;              // [NQK]
-    uint64_t *v_full, *v_empty;                // [NV]
+    uint64_t *qk_full;                         // [NQK]
+    uint64_t *v_full;                          // [NV]
     uint64_t *s_full, *p_full, *o_full, *o_empty;  // [NBUF]
     uint64_t *drain;
     uint32_t *tmem_slot;
@@ -69,9 +74,7 @@ __device__ __forceinline__ AttSmem att_carve(uint8_t *raw) {
     s.inv_sum = reinterpret_cast<float *>(s.v + NV * TILE);
     uint64_t *b = reinterpret_cast<uint64_t *>(s.v + NV * TILE + NBUF * TROWS * 4);
     s.qk_full = b;
-    s.qk_empty = b + NQK;
     s.v_full = b + 2 * NQK;
-    s.v_empty = b + 2 * NQK + NV;
     s.s_full = b + 2 * NQK + 2 * NV;
     s.p_full = s.s_full + NBUF;
     s.o_full = s.s_full + 2 * NBUF;
@@ -100,14 +103,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     if (threadIdx.x == 0) {
         sm.misc[0] = *reinterpret_cast<const volatile int *>(status);
         *sm.abort_flag = 0;
-        for (int i = 0; i < NQK; ++i) {
-            mbar_init(smem_u32(&sm.qk_full[i]), 1);
-            mbar_init(smem_u32(&sm.qk_empty[i]), 1);
-        }
-        for (int i = 0; i < NV; ++i) {
-            mbar_init(smem_u32(&sm.v_full[i]), 1);
-            mbar_init(smem_u32(&sm.v_empty[i]), 1);
-        }
+        for (int i = 0; i < NQK; ++i) mbar_init(smem_u32(&sm.qk_full[i]), 1);
+        for (int i = 0; i < NV; ++i) mbar_init(smem_u32(&sm.v_full[i]), 1);
         for (int i = 0; i < NBUF; ++i) {
             mbar_init(smem_u32(&sm.s_full[i]), 1);
             mbar_init(smem_u32(&sm.p_full[i]), 4);
@@ -148,7 +145,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                 bool progress = false;
                 if (nq < n_items) {
                     const int st = nq % NQK;
-                    if (mbar_test(smem_u32(&sm.qk_empty[st]), ((nq / NQK) & 1) ^ 1)) {
+                    // the stage is free once S of item nq - NQK has completed
+                    if (mbar_test(smem_u32(&sm.s_full[st]), ((nq / NQK) & 1) ^ 1)) {
                         const int id = blockIdx.x + nq * gridDim.x, b = id / kHeads, h = id % kHeads;
                         const int start = __ldg(seq_start + b), L = __ldg(seq_len + b);
                         sm.qk_len[st] = L;  // read by the issuer once the stage is full
@@ -165,7 +163,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                 }
                 if (nv < nq) {
                     const int st = nv % NV;
-                    if (mbar_test(smem_u32(&sm.v_empty[st]), ((nv / NV) & 1) ^ 1)) {
+                    // the stage is free once O of item nv - NV has completed
+                    if (mbar_test(smem_u32(&sm.o_full[st]), ((nv / NV) & 1) ^ 1)) {
                         const int id = blockIdx.x + nv * gridDim.x, b = id / kHeads, h = id % kHeads;
                         const int start = __ldg(seq_start + b), L = __ldg(seq_len + b);
                         sm.v_len[st] = L;
@@ -221,8 +220,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                             umma_bf16_ts(buf + TM_O, buf + kk * 8, sw128_kmajor_desc(vbase + kk * 2048), idesc_o,
                                          kk != 0);
                         }
-                        umma_commit(smem_u32(&sm.o_full[tb]));
-                        umma_commit(smem_u32(&sm.v_empty[st]));  // V consumed: stage free
+                        umma_commit(smem_u32(&sm.o_full[tb]));  // also frees V stage st (== tb)
                         ++no;
                         progress = true;
                     }
@@ -239,8 +237,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                         for (int kk = 0; kk < kHeadDim / 16; ++kk)
                             umma_bf16(tmem_base + tb * TROWS, sw128_kmajor_desc(q + kk * 32),
                                       sw128_kmajor_desc(k + kk * 32), L <= 64 ? idesc_s64 : idesc_s128, kk != 0);
-                        umma_commit(smem_u32(&sm.s_full[tb]));
-                        umma_commit(smem_u32(&sm.qk_empty[st]));  // Q, K consumed: stage free
+                        umma_commit(smem_u32(&sm.s_full[tb]));  // also frees Q/K stage st (== tb)
                         ++ns;
                         progress = true;
                     }
