@@ -97,10 +97,10 @@ def test_gemm_scatter_rows(variant):
     assert np.all(got[untouched] == 7.0)
 
 
-def _attention_case(lengths, fp32=False, seed=0, legacy=False):
+def _attention_case(lengths, fp32=False, seed=0, legacy=False, scale=1.0):
     r = np.random.default_rng(seed)
     n = int(sum(lengths))
-    qkv = r.normal(0, 1.0, (n, 3 * 768))
+    qkv = r.normal(0, scale, (n, 3 * 768))
     cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
     if fp32:
         q_dev = torch.tensor(qkv, dtype=torch.float32, device="cuda")
@@ -145,6 +145,12 @@ def test_attention_tcgen05_long_kernel_every_block_count():
     """Lengths around every key-block boundary (1 to 4 blocks of 128, ragged last
     block and last query block) and short sequences sharing the launch."""
     _attention_case([129, 1, 130, 255, 256, 257, 64, 383, 384, 385, 2, 447, 448, 449, 511, 512, 128, 200], seed=11)
+
+
+def test_attention_tcgen05_long_kernel_peaked_softmax():
+    """Scores with a spread of ~16 (QKV ~ N(0, 4)): most probabilities underflow
+    far below the row maximum, exercising the exponentials' clamp."""
+    _attention_case([500, 129, 384, 257], seed=13, scale=4.0)
 
 
 def test_attention_mma_sync_kernel_long_sequences():
