@@ -10,7 +10,8 @@
 //
 // Three launches on the caller's stream (the second and third chained with
 // programmatic dependent launch), bounded by HBM traffic:
-//   durations : a warp per token, 32 tokens per block; fp64 sigmoid sum over the
+//   durations : a warp per token, 32 tokens (warps) per block, so every token's
+//               loads and fp64 chain are in flight at once; fp64 sigmoid sum over the
 //               channels (the decision is an integer, taken in fp64), rint, floor
 //               of 1; then the block's exclusive prefix (local starts) and sum;
 //   scan      : one block over the block sums; validates cu_seqlens, checks the
@@ -28,13 +29,14 @@
 namespace albert {
 namespace {
 
-constexpr int LR_THREADS = 256;
-constexpr int LR_TOK = 32;           // tokens per block of the durations kernel
+constexpr int LR_THREADS = 256;      // expansion kernel
+constexpr int LR_TOK = 32;           // tokens per block of the durations kernel, one warp each
+constexpr int LR_DUR_THREADS = 32 * LR_TOK;
 constexpr int SCAN_THREADS = 1024;
 
-// Durations of LR_TOK consecutive tokens (warp w takes tokens w, w+8, ...), then
-// their exclusive prefix inside the block (local frame start) and the block sum.
-__global__ void __launch_bounds__(LR_THREADS)
+// Durations of LR_TOK consecutive tokens (warp w takes token w), then their
+// exclusive prefix inside the block (local frame start) and the block sum.
+__global__ void __launch_bounds__(LR_DUR_THREADS)
 lr_durations_kernel(const float *__restrict__ logits, int C, double speed, int n_tok, int *__restrict__ dur,
                     int *__restrict__ local_start, long long *__restrict__ block_sum, int *status) {
     __shared__ int sd[LR_TOK];
@@ -42,7 +44,7 @@ lr_durations_kernel(const float *__restrict__ logits, int C, double speed, int n
     griddep_launch_dependents();  // the scan (launched with PDL) may take SMs as this grid frees them
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int t0 = blockIdx.x * LR_TOK;
-    for (int i = warp; i < LR_TOK; i += LR_THREADS / 32) {
+    for (int i = warp; i < LR_TOK; i += LR_DUR_THREADS / 32) {
         const int t = t0 + i;
         int d = 0;
         if (t < n_tok) {
@@ -200,7 +202,7 @@ extern "C" int albert_length_regulate(const float *logits, int C, float speed, c
     int *local_start = static_cast<int *>(scratch);
     long long *block_sum = reinterpret_cast<long long *>(static_cast<char *>(scratch) + off_sum);
     long long *block_start = reinterpret_cast<long long *>(static_cast<char *>(scratch) + off_start);
-    lr_durations_kernel<<<n_blocks, LR_THREADS, 0, s>>>(logits, C, (double)speed, n_tok, durations, local_start,
+    lr_durations_kernel<<<n_blocks, LR_DUR_THREADS, 0, s>>>(logits, C, (double)speed, n_tok, durations, local_start,
                                                         block_sum, status);
     cudaError_t e = launch_pdl(lr_scan_kernel, dim3(1), dim3(SCAN_THREADS), 0, s, block_sum, n_blocks, local_start,
                                cu_seqlens, nseq, n_tok, max_frames, block_start, cu_frames, status);
