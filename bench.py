@@ -222,6 +222,12 @@ def oracle_throughput(weights, ids, mask, L, arch, budget_s=None, steps=None, wa
     return tok / secs, done, tok, secs, oracle.num_threads()
 
 
+def workload_label(wl, args) -> str:
+    """config.workload of both arms: the workload and whether the GEMMs run on the
+    packed valid rows or on all B*T padded rows."""
+    return wl.name + ("_padded" if args.padded else "_packed")
+
+
 def run_reference(args):
     import synth
     rank = int(os.environ.get("RANK", "0"))
@@ -238,7 +244,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * secs / max(done, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,0.02) weights rounded to bf16, seeded ids and lengths)",
-        "config": {"workload": wl.name, "batch": wl.B, "seq_len": wl.T, "lengths": wl.describe()},
+        "config": {"workload": workload_label(wl, args), "batch": wl.B, "seq_len": wl.T, "lengths": wl.describe()},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -515,7 +521,7 @@ def run_gpu(args):
     lenreg = measure_length_regulation(torch, synth, tea, L, flush, peaks, peaks_src, stream, args.steps)
     dom_ms = dom[1] / max(dom[0], 1)
     achieved = per_launch.get(dominant, 0.0) / (dom_ms / 1000.0) / 1e12
-    traffic, traffic_note = load_traffic(dominant, wl.name + ("_padded" if args.padded else "_packed"), wl.T)
+    traffic, traffic_note = load_traffic(dominant, workload_label(wl, args), wl.T)
     roofline = {"kernel": dominant, "bound": "tensor", "achieved": achieved, "peak": peak_sus,
                 "unit": "TFLOP/s", "frac": achieved / peak_sus, "traffic": traffic,
                 "traffic_source": traffic_note,
@@ -529,7 +535,7 @@ def run_gpu(args):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,0.02) weights rounded to bf16, seeded ids and lengths)",
-        "config": {"workload": wl.name + ("_padded" if args.padded else "_packed"), "batch": wl.B,
+        "config": {"workload": workload_label(wl, args), "batch": wl.B,
                    "seq_len": wl.T, "lengths": wl.describe(), "valid_tokens_per_step_per_gpu": n_tok,
                    "pack": not args.padded, "parallelism": f"replicas x{world}",
                    "launch": "cuda_graph" if args.graph else "stream",
