@@ -177,6 +177,32 @@ int albert_get_status(albert_handle *h, void *stream);
 /* Free everything the handle owns.  NULL is ignored. */
 void albert_destroy(albert_handle *h);
 
+/* ---- bounded waits and their failure path ----
+ * Every wait inside the bf16 kernels (on a TMA copy, a tensor-core product or
+ * another warp's hand-off) is bounded in wall time.  When a wait runs out, the
+ * kernel records ALBERT_ERR_TIMEOUT in the status word, lets its in-flight
+ * copies and products finish, frees its tensor memory and returns; every later
+ * kernel of the forward then skips its work, so `out` is left as it was and
+ * the context stays usable.  (The pages' checked-kernel contract: a failed
+ * check stops downstream work and reports an integer status -- "How Kokoro TTS
+ * Works and Where CKE Stands", sections on checked kernels.)
+ *
+ * albert_set_wait_limit: the limit, in nanoseconds, of the waits of every
+ * kernel of later forwards on this handle; 0 restores the default (2 s).
+ * ns < 0 returns ALBERT_ERR_CONFIG.  A limit shorter than a kernel's normal
+ * waits makes healthy forwards fail with ALBERT_ERR_TIMEOUT. */
+int albert_set_wait_limit(albert_handle *h, long long ns);
+
+/* Failure injection for tests of the path above: on later forwards, the GEMM
+ * launches of the kernel classes set in class_mask (bit i = class i of
+ * albert_profile_name; only the GEMM classes are accepted) run with their TMA
+ * producer withholding every load, so their first wait on an operand tile can
+ * never complete and runs out after the wait limit.  Nothing faults: the
+ * forward reports ALBERT_ERR_TIMEOUT through albert_get_status with `out`
+ * untouched.  0 turns it off.  Returns ALBERT_ERR_CONFIG for other classes, or
+ * for a non-zero mask on an ALBERT_FP32 handle (its kernels have no waits). */
+int albert_test_stall(albert_handle *h, int class_mask);
+
 /* Number of kernel launches one forward of this handle enqueues for a batch
  * with the given shape (used to report launches per step). */
 int albert_launches_per_forward(const albert_handle *h, int padded_api);
@@ -204,12 +230,13 @@ const char *albert_profile_name(int cls);
 int albert_profile_read(albert_handle *h, int *launches, double *ms);
 
 /* ---- length regulation (the step after the encoder) ----
- * "ALBERT: How Kokoro's Phoneme Encoder Works", section "The time axis is where a
+ * "How Kokoro TTS Works and Where CKE Stands", section "The time axis is where a
  * circuit becomes difficult": per token, the sigmoid duration channels are summed,
  * divided by the speed, rounded and clamped to at least one frame; A = sum d[t]
  * is the number of aligned frames; token features are repeated by the duration
- * vector ("How Kokoro TTS Works and Where CKE Stands", section "Path one":
- * durations 2, 1, 3 -> p1 p1 p2 p3 p3 p3).
+ * vector ("Qwen3-TTS and Kokoro: Two Routes from Text to Speech", section "Path
+ * one: Kokoro decides how long each sound lasts": durations 2, 1, 3 ->
+ * p1 p1 p2 p3 p3 p3).
  *
  * For a packed batch of nseq sequences (token rows in cu_seqlens order, n_tok =
  * cu_seqlens[nseq]), all device pointers, asynchronous on `stream`:
@@ -289,14 +316,20 @@ int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, 
  *   anything else returns ALBERT_ERR_SHAPE before any work is enqueued;
  *   bias and ln_g must be 16-byte aligned (else ALBERT_ERR_CONFIG).
  * The arrays are reserved on every device where the library's module holding
- * them is loaded and stay until the process exits.  The first call on a device
- * looks up their device addresses (cudaGetSymbolAddress) with that device
- * current; make that first call before any stream capture.  Every call shares
- * the same arrays (the status word is reset by each call; the intermediates
- * are rewritten before they are read, so nothing else needs clearing), so
- * calls that overlap on the GPU -- on different
- * streams or from different threads -- race and must be serialized by the
- * caller.  Synchronous: returns the kernel's status. */
+ * them is loaded and stay until the process exits.  Every call looks up their
+ * device addresses (cudaGetSymbolAddress) with the caller's device current.
+ * The CUDA runtime loads a library's modules lazily: the first call on a
+ * device loads the modules behind it (the arrays and the two kernels), which
+ * reserves their memory and synchronizes the device once.  The no-allocation
+ * guarantee therefore holds from the second call on: make one warm-up call on
+ * each device at set-up time, before any stream capture and before the thread
+ * that must not allocate starts calling.  Every call shares the same arrays
+ * (the status word is reset by each call; the intermediates are rewritten
+ * before they are read, so nothing else needs clearing), so calls that overlap
+ * on the GPU -- on different streams or from different threads -- race and
+ * must be serialized by the caller.  Synchronous: the call synchronizes its
+ * stream before returning the kernel's status, so holding a host-side lock
+ * around each call is enough to serialize them. */
 int albert_gemm_residual_ln_noalloc(const void *A, const void *W, const float *bias, const void *R,
                                     const float *ln_g, const float *ln_b, float eps, void *Y, int M,
                                     int K, void *stream);

@@ -6,14 +6,14 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's ``cpu_baseline`
 CUDA library.
 
 What it computes (sources, by page and section):
-  * "ALBERT: How Kokoro's Phoneme Encoder Works, and Where CKE Has Reached It",
-    section "The time axis is where a circuit becomes difficult": per token, the
-    sigmoid duration channels are summed, divided by the speed, rounded and
-    clamped to at least one frame; A = sum_t d[t] is the number of aligned
-    frames; token features are repeated according to the duration vector.
-  * "How Kokoro TTS Works and Where CKE Stands", section "Path one: Kokoro
-    decides how long each sound lasts": the worked example (durations 2, 1, 3 ->
-    six positions p1 p1 p2 p3 p3 p3) that pins the expansion order.
+  * "How Kokoro TTS Works and Where CKE Stands", section "The time axis is where
+    a circuit becomes difficult": per token, the sigmoid duration channels are
+    summed, divided by the speed, rounded and clamped to at least one frame;
+    A = sum_t d[t] is the number of aligned frames; token features are repeated
+    according to the duration vector.
+  * "Qwen3-TTS and Kokoro: Two Routes from Text to Speech", section "Path one:
+    Kokoro decides how long each sound lasts": the worked example (durations
+    2, 1, 3 -> six positions p1 p1 p2 p3 p3 p3) that pins the expansion order.
 
 Readings where the pages are silent: "rounded" is round-half-to-even (IEEE
 rint); the number of duration channels C is a parameter; the decision is taken

@@ -154,7 +154,7 @@ WORKLOADS = {
                                 mean=60.0, sd=25.0, seed=102),
     "b32_T512_long": Workload("b32_T512_long", 32, 512, "uniform", lo=256, hi=512, seed=103),
     "b256_T128": Workload("b256_T128", 256, 128, "uniform", lo=16, hi=128, seed=104),
-    "b1_T64_latency": Workload("b1_T64_latency", 1, 64, "full", seed=104),
+    "b1_T64_latency": Workload("b1_T64_latency", 1, 64, "full", seed=105),
 }
 
 

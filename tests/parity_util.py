@@ -46,15 +46,13 @@ def check_fp32(gpu: np.ndarray, ref: np.ndarray, what: str = ""):
     return rel
 
 
-def sample_sequences(L: np.ndarray, k: int, seed: int = 0) -> list:
-    """The longest and shortest sequence plus k-2 others drawn with a seed."""
-    L = np.asarray(L)
-    idx = {int(np.argmax(L)), int(np.argmin(L))}
-    rng = np.random.default_rng(seed)
-    rest = [i for i in range(len(L)) if i not in idx]
-    rng.shuffle(rest)
-    idx.update(rest[: max(0, k - len(idx))])
-    return sorted(idx)
+# (label, sequences, valid tokens, worst error, worst per-token cosine, error kind)
+# of every whole-encoder comparison in this session, printed in the summary
+PARITY_REPORT = []
+
+
+def record_parity(label, n_seq, n_tok, err, cos, kind):
+    PARITY_REPORT.append((label, n_seq, n_tok, err, cos, kind))
 
 
 def oracle_rows(weights: dict, ids: np.ndarray, mask: np.ndarray, L: np.ndarray, seqs, n_exec=None,

@@ -1,9 +1,9 @@
 """Pins of the length-regulation oracle (CPU, no GPU).
 
-The oracle follows "ALBERT: How Kokoro's Phoneme Encoder Works, and Where CKE Has
-Reached It", section "The time axis is where a circuit becomes difficult", and the
-worked example of "How Kokoro TTS Works and Where CKE Stands", section "Path one:
-Kokoro decides how long each sound lasts".  Each pin below is fixed by the pages
+The oracle follows "How Kokoro TTS Works and Where CKE Stands", section "The time
+axis is where a circuit becomes difficult", and the worked example of "Qwen3-TTS and
+Kokoro: Two Routes from Text to Speech", section "Path one: Kokoro decides how long
+each sound lasts".  Each pin below is fixed by the pages
 or by closed forms, not by re-evaluating the oracle's own formula.
 """
 import os

@@ -1,17 +1,20 @@
 """The residual + LayerNorm GEMM entry point that allocates no device memory.
 
 It serves callers that cannot allocate while running (a real-time audio thread,
-a runtime whose device memory is laid out in advance).  Its output must match
-the allocating entry point's (albert_test_gemm, epilogue 2) within the
-single-kernel tolerance, on two calls in a row with different data (the calls
-share one static scratch array), and it must reject M beyond its 2048-row limit
-without writing.  This file is collected last so that a stop-at-first-failure
-run has already run every other test.
+a runtime whose device memory is laid out in advance).  On two calls in a row
+with different shapes and data (the calls share one static scratch array), its
+output must match the fp64 oracle's LN(A W^T + bias + R) within the
+single-kernel tolerance and the allocating entry point (albert_test_gemm,
+epilogue 2) closely; after a warm-up call the two calls must leave the device's
+free memory unchanged; and it must reject M beyond its 2048-row limit without
+writing.  This file is collected last so that a stop-at-first-failure run has
+already run every other test.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 import transformer_encoder_albert_b200 as tea
 
@@ -20,35 +23,72 @@ pytestmark = pytest.mark.gpu
 
 def _case(M, K, seed):
     r = np.random.default_rng(seed)
-    bf = lambda a: torch.tensor(synth.bf16_round(np.asarray(a, np.float32))).cuda().to(torch.bfloat16)
-    f32 = lambda a: torch.tensor(np.asarray(a, np.float32)).cuda()
-    return dict(A=bf(r.normal(0, 1, (M, K))), W=bf(r.normal(0, 0.05, (768, K))),
-                bias=f32(r.normal(0, 0.1, 768)), R=bf(r.normal(0.3, 1.0, (M, 768))),
-                ln_g=f32(1 + r.normal(0, 0.1, 768)), ln_b=f32(r.normal(0, 0.1, 768)))
+    host = dict(A=synth.bf16_round(r.normal(0, 1, (M, K)).astype(np.float32)),
+                W=synth.bf16_round(r.normal(0, 0.05, (768, K)).astype(np.float32)),
+                bias=r.normal(0, 0.1, 768).astype(np.float32),
+                R=synth.bf16_round(r.normal(0.3, 1.0, (M, 768)).astype(np.float32)),
+                ln_g=(1 + r.normal(0, 0.1, 768)).astype(np.float32),
+                ln_b=r.normal(0, 0.1, 768).astype(np.float32))
+    dev = {k: torch.tensor(v).cuda() for k, v in host.items()}
+    for k in ("A", "W", "R"):
+        dev[k] = dev[k].to(torch.bfloat16)
+    return host, dev
 
 
-def _close(got, ref):
-    got, ref = got.float().cpu().numpy(), ref.float().cpu().numpy()
+def _oracle(h):
+    z = oracle.linear(h["A"], h["W"], h["bias"]) + h["R"].astype(np.float64)
+    return oracle.layer_norm(z, h["ln_g"], h["ln_b"], 1e-12)
+
+
+def _within(got, ref, what):
+    """The single-kernel tolerance: two bf16 half-ulps of the value plus an
+    fp32-accumulation allowance."""
     scale = np.max(np.abs(ref))
-    assert np.all(np.abs(got - ref) <= 8e-3 * np.abs(ref) + 2e-3 * scale)
+    bad = np.abs(got - ref) > 8e-3 * np.abs(ref) + 2e-3 * scale
+    assert not np.any(bad), f"{what}: {int(bad.sum())} elements outside tolerance, " \
+                            f"max abs err {float(np.max(np.abs(got - ref))):.3e}"
 
 
-def test_noalloc_matches_allocating_entry_on_two_calls_in_a_row():
-    for M, K, seed in ((1000, 768, 1), (2048, 2048, 2)):
-        c = _case(M, K, seed)
+def test_noalloc_matches_oracle_and_allocating_entry_on_two_calls_in_a_row():
+    # M = 2048 fills the static scratch; M = 300 then takes the CTA-pair kernel
+    # with a partial last 256-row unit on arrays that still hold the first call's rows.
+    cases = [(2048, 2048, 2), (300, 768, 1)]
+    data = [_case(M, K, seed) for M, K, seed in cases]
+    outs = [torch.full((M, 768), 5.0, device="cuda", dtype=torch.bfloat16) for M, _, _ in cases]
+    warm = torch.empty(8, 768, device="cuda", dtype=torch.bfloat16)
+    # warm-up: the first call on a device loads the library's modules
+    d0 = data[1][1]
+    assert tea.gemm_residual_ln_noalloc(d0["A"][:8], d0["W"], d0["bias"], d0["R"][:8], d0["ln_g"], d0["ln_b"],
+                                        warm, eps=1e-12) == 0
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for (host, dev), out in zip(data, outs):
+        assert tea.gemm_residual_ln_noalloc(dev["A"], dev["W"], dev["bias"], dev["R"], dev["ln_g"], dev["ln_b"],
+                                            out, eps=1e-12) == 0
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0, "the calls changed the device's free memory"
+    for (M, K, _), (host, dev), out in zip(cases, data, outs):
+        got = out.float().cpu().numpy()
+        _within(got, _oracle(host), f"M={M} K={K} vs oracle")
         ref = torch.empty(M, 768, device="cuda", dtype=torch.bfloat16)
-        assert tea.test_gemm(c["A"], c["W"], c["bias"], ref, 2, R=c["R"], ln_g=c["ln_g"],
-                             ln_b=c["ln_b"], eps=1e-12) == 0
-        got = torch.full((M, 768), 5.0, device="cuda", dtype=torch.bfloat16)
-        assert tea.gemm_residual_ln_noalloc(c["A"], c["W"], c["bias"], c["R"], c["ln_g"], c["ln_b"],
-                                            got, eps=1e-12) == 0
-        _close(got, ref)
+        assert tea.test_gemm(dev["A"], dev["W"], dev["bias"], ref, 2, R=dev["R"], ln_g=dev["ln_g"],
+                             ln_b=dev["ln_b"], eps=1e-12) == 0
+        _within(got, ref.float().cpu().numpy(), f"M={M} K={K} vs the allocating entry")
 
 
 def test_noalloc_rejects_rows_beyond_its_static_scratch():
-    c = _case(2049, 768, 3)
+    _, c = _case(2049, 768, 3)
     Y = torch.full((2049, 768), 5.0, device="cuda", dtype=torch.bfloat16)
     rc = tea.gemm_residual_ln_noalloc(c["A"], c["W"], c["bias"], c["R"], c["ln_g"], c["ln_b"], Y)
     assert rc == 3  # ALBERT_ERR_SHAPE
     torch.cuda.synchronize()
     assert torch.all(Y == 5.0)
+
+
+def test_noalloc_python_guard_rejects_mismatched_tensors():
+    _, c = _case(64, 768, 4)
+    Y = torch.empty(64, 768, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        tea.gemm_residual_ln_noalloc(c["A"], c["W"][:512], c["bias"], c["R"], c["ln_g"], c["ln_b"], Y)
+    with pytest.raises(ValueError):
+        tea.gemm_residual_ln_noalloc(c["A"], c["W"], c["bias"], c["R"][:32], c["ln_g"], c["ln_b"], Y)

@@ -40,6 +40,7 @@ EXPORTS = (
     "albert_profile_classes",
     "albert_profile_name", "albert_profile_read", "albert_test_gemm", "albert_test_attention",
     "albert_gemm_residual_ln_noalloc", "albert_length_regulate", "albert_length_regulate_scratch_bytes",
+    "albert_set_wait_limit", "albert_test_stall",
 )
 
 
@@ -96,6 +97,8 @@ def lib() -> C.CDLL:
         L.albert_length_regulate.argtypes = [vp, i, C.c_float, vp, i, vp, i, i, vp, vp, vp, vp, i, vp, vp, vp]
         L.albert_length_regulate_scratch_bytes.argtypes = [i]
         L.albert_length_regulate_scratch_bytes.restype = C.c_size_t
+        L.albert_set_wait_limit.argtypes = [vp, C.c_longlong]
+        L.albert_test_stall.argtypes = [vp, i]
         _lib = L
     return _lib
 
@@ -237,6 +240,19 @@ class Encoder:
     def status(self, stream=None) -> int:
         return albert_get_status(self.h, stream)
 
+    def set_wait_limit(self, ns: int) -> None:
+        """Limit (ns) of the kernels' bounded waits on later forwards; 0 = default (2 s)."""
+        _check(lib().albert_set_wait_limit(self.h, int(ns)), "albert_set_wait_limit")
+
+    def test_stall(self, classes=()) -> None:
+        """Failure injection: the GEMM launches of these kernel classes withhold
+        their operand loads on later forwards, so their waits run out ([] = off)."""
+        names = profile_class_names()
+        mask = 0
+        for c in classes:
+            mask |= 1 << names.index(c)
+        _check(lib().albert_test_stall(self.h, mask), "albert_test_stall")
+
     def launches_per_forward(self, padded_api: bool = True) -> int:
         return lib().albert_launches_per_forward(self.h, 1 if padded_api else 0)
 
@@ -311,8 +327,19 @@ def test_attention(qkv, cu_seqlens, max_len: int, ctx, fp32: bool = False, legac
 
 def gemm_residual_ln_noalloc(A, W, bias, R, ln_g, ln_b, Y, eps: float = 1e-12, stream=None) -> int:
     """Y = LN(A W^T + bias + R) through the entry point that allocates no device
-    memory (static scratch inside the library; M <= 2048)."""
+    memory (static scratch inside the library; M <= 2048).  The C side cannot see
+    the tensors' extents, so they are checked here: a mismatched tensor would make
+    the kernels read or write past the caller's buffers."""
+    import torch
     M, K = A.shape
+    N = 768
+    want = {"A": (A, (M, K), torch.bfloat16), "W": (W, (N, K), torch.bfloat16), "R": (R, (M, N), torch.bfloat16),
+            "Y": (Y, (M, N), torch.bfloat16), "bias": (bias, (N,), torch.float32),
+            "ln_g": (ln_g, (N,), torch.float32), "ln_b": (ln_b, (N,), torch.float32)}
+    for name, (t, shape, dt) in want.items():
+        if tuple(t.shape) != shape or t.dtype != dt or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"gemm_residual_ln_noalloc: {name} must be a contiguous CUDA {dt} tensor "
+                             f"of shape {shape}, got {tuple(t.shape)} {t.dtype} on {t.device}")
     return lib().albert_gemm_residual_ln_noalloc(_ptr(A), _ptr(W), _ptr(bias), _ptr(R), _ptr(ln_g),
                                                  _ptr(ln_b), float(eps), _ptr(Y), M, K,
                                                  _stream_ptr(stream))

@@ -102,6 +102,11 @@ struct albert_handle {
     CUtensorMap tm_win, tm_wout;
     CUtensorMap t32_X, t32_QKV, t32_X1, t32_H, t32_Z;  // 32x32-box maps: epilogue stores / residual loads
 
+    // bounded waits inside the kernels: limit (0 = the kernels' default, 2 s) and,
+    // for failure-path tests, kernel classes whose GEMM producer withholds its loads
+    unsigned long long wait_ns = 0;
+    unsigned stall_mask = 0;
+
     // per-kernel timing
     unsigned prof_mask = 0;  // classes whose launches are timed
     bool prof_retain = false;  // keep recorded pairs armed after a read (graph replays)
@@ -236,12 +241,14 @@ GemmArgs gemm_args(albert_handle *h, int N, int K, const float *bias, void *out,
     a.status = h->status;
     a.eps = h->cfg.ln_eps;
     a.trigger = 1;  // inside a forward the next launch is one of ours with PDL
+    a.wait_ns = h->wait_ns;
     return a;
 }
 
 int gemm_bf16(Launch &L, int cls, int epi, const CUtensorMap &A, const CUtensorMap &B, const CUtensorMap &Out,
               const CUtensorMap &Res, GemmArgs a) {
     const int grid = gemm_grid(epi, a.rows_cap, a.N, L.h->num_sms);
+    a.withhold_loads = (L.h->stall_mask >> cls) & 1u;
     if (epi == kEpiResStats && a.N != gemm::LN_N) return ALBERT_ERR_CONFIG;
     if (!gemm_vectors_aligned(a)) return ALBERT_ERR_CONFIG;
     LAUNCH(L, cls, launch_gemm(epi, A, B, Out, Res, a, grid, L.s));
@@ -321,10 +328,12 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
             if (rc) return rc;
             if (max_len <= kAttnTcMaxLen) {
                 LAUNCH(L, kProfAttention, launch_attention_tc(h->tm_QKV, h->tm_QKV64, static_cast<bf16 *>(h->C), h->seq_start,
-                                                             h->seq_len, nseq, h->status, h->num_sms, L.s, true));
+                                                             h->seq_len, nseq, h->status, h->num_sms, L.s, true,
+                                                             h->wait_ns));
             } else if (max_len <= kAttnTcLongMaxLen) {
                 LAUNCH(L, kProfAttention, launch_attention_tc_long(h->tm_QKV, static_cast<bf16 *>(h->C), h->seq_start,
-                                                                  h->seq_len, nseq, h->status, h->num_sms, L.s, true));
+                                                                  h->seq_len, nseq, h->status, h->num_sms, L.s, true,
+                                                                  h->wait_ns));
             } else {
                 LAUNCH(L, kProfAttention, launch_attention_bf16(static_cast<bf16 *>(h->QKV), static_cast<bf16 *>(h->C),
                                                                h->seq_start, h->seq_len, nseq, max_len, h->status, L.s,
@@ -782,6 +791,23 @@ int albert_profile_retain(albert_handle *h, int on) {
     if (!h) return ALBERT_ERR_NULL;
     h->prof_retain = on != 0;
     if (!h->prof_retain) h->ev_used = 0;
+    return ALBERT_OK;
+}
+
+int albert_set_wait_limit(albert_handle *h, long long ns) {
+    if (!h) return ALBERT_ERR_NULL;
+    if (ns < 0) return ALBERT_ERR_CONFIG;
+    h->wait_ns = (unsigned long long)ns;
+    return ALBERT_OK;
+}
+
+int albert_test_stall(albert_handle *h, int class_mask) {
+    if (!h) return ALBERT_ERR_NULL;
+    const unsigned gemm_classes = (1u << kProfGemmIn) | (1u << kProfGemmQKV) | (1u << kProfGemmWoLN) |
+                                  (1u << kProfGemmW1Gelu) | (1u << kProfGemmW2LN) | (1u << kProfGemmOut);
+    if ((unsigned)class_mask & ~gemm_classes) return ALBERT_ERR_CONFIG;
+    if (class_mask && h->cfg.dtype != ALBERT_BF16) return ALBERT_ERR_CONFIG;  // the fp32 kernels never wait
+    h->stall_mask = (unsigned)class_mask;
     return ALBERT_OK;
 }
 

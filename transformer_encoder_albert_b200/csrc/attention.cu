@@ -270,13 +270,10 @@ template <int NW>
 static cudaError_t launch_attn_nw(const bf16 *qkv, bf16 *ctx, const int *seq_start, const int *seq_len, int nseq,
                                   int max_len, const int *status, cudaStream_t s, bool trigger) {
     constexpr int QT = 16 * NW;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)attn_bf16_smem(kMaxPos, QT));
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<unsigned long long> configured{0};
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(attn_bf16_kernel<NW>),
+                                     (int)attn_bf16_smem(kMaxPos, QT), configured);
+    if (e != cudaSuccess) return e;
     dim3 grid((max_len + QT - 1) / QT, kHeads, nseq);
     return launch_pdl(attn_bf16_kernel<NW>, grid, dim3(NW * 32), attn_bf16_smem(max_len, QT), s, qkv, ctx, seq_start,
                       seq_len, status, trigger ? 1 : 0);
@@ -295,13 +292,10 @@ cudaError_t launch_attention_f32(const float *qkv, float *ctx, const int *seq_st
                                  cudaStream_t s) {
     if (nseq <= 0) return cudaSuccess;
     const size_t smem = (size_t)F32_ROWS * (max_len + kHeadDim) * sizeof(float);
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)((size_t)F32_ROWS * (kMaxPos + kHeadDim) * sizeof(float)));
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<unsigned long long> configured{0};
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(attn_f32_kernel),
+                                     (int)((size_t)F32_ROWS * (kMaxPos + kHeadDim) * sizeof(float)), configured);
+    if (e != cudaSuccess) return e;
     dim3 grid((max_len + F32_ROWS - 1) / F32_ROWS, kHeads, nseq);
     attn_f32_kernel<<<grid, 32 * F32_ROWS, smem, s>>>(qkv, ctx, seq_start, seq_len, status, max_len);
     return cudaGetLastError();

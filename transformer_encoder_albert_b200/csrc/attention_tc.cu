@@ -92,7 +92,7 @@ __device__ __forceinline__ AttSmem att_carve(uint8_t *raw) {
 __global__ void __launch_bounds__(ATC_THREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmQKV64,
                bf16 *__restrict__ ctx, const int *__restrict__ seq_start, const int *__restrict__ seq_len, int nseq,
-               int *status, int trigger) {
+               int *status, int trigger, unsigned long long wait_ns) {
     if (trigger) griddep_launch_dependents();  // the next kernel may take SMs as this grid frees them
     griddep_wait();               // the previous kernel has completed
 
@@ -103,6 +103,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     if (threadIdx.x == 0) {
         sm.misc[0] = *reinterpret_cast<const volatile int *>(status);
         *sm.abort_flag = 0;
+        wait_limit_init(wait_ns);
         for (int i = 0; i < NQK; ++i) mbar_init(smem_u32(&sm.qk_full[i]), 1);
         for (int i = 0; i < NV; ++i) mbar_init(smem_u32(&sm.v_full[i]), 1);
         for (int i = 0; i < NBUF; ++i) {
@@ -182,7 +183,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                     if (*sm.abort_flag) break;
                     const unsigned long long now = globaltimer_ns();
                     if (t_idle == 0) t_idle = now;
-                    else if (now - t_idle > kWaitLimitNs) { *sm.abort_flag = 1; break; }
+                    else if (now - t_idle > wait_limit()) { *sm.abort_flag = 1; break; }
                 }
             }
             if (*sm.abort_flag) {
@@ -248,7 +249,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                     if (*sm.abort_flag) break;
                     const unsigned long long now = globaltimer_ns();
                     if (t_idle == 0) t_idle = now;
-                    else if (now - t_idle > kWaitLimitNs) { *sm.abort_flag = 1; break; }
+                    else if (now - t_idle > wait_limit()) { *sm.abort_flag = 1; break; }
                 }
             }
             umma_commit(smem_u32(sm.drain));
@@ -394,18 +395,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
 }  // namespace
 
 cudaError_t launch_attention_tc(const CUtensorMap &tmQKV, const CUtensorMap &tmQKV64, bf16 *ctx, const int *seq_start,
-                                const int *seq_len, int nseq, int *status, int num_sms, cudaStream_t s, bool trigger) {
+                                const int *seq_len, int nseq, int *status, int num_sms, cudaStream_t s, bool trigger,
+                                unsigned long long wait_ns) {
     if (nseq <= 0) return cudaSuccess;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATC_SMEM);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<unsigned long long> configured{0};
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(attn_tc_kernel), ATC_SMEM, configured);
+    if (e != cudaSuccess) return e;
     const int total = nseq * kHeads;
     const int grid = total < num_sms ? total : num_sms;
     return launch_pdl(attn_tc_kernel, dim3(grid), dim3(ATC_THREADS), ATC_SMEM, s, tmQKV, tmQKV64, ctx, seq_start,
-                      seq_len, nseq, status, trigger ? 1 : 0);
+                      seq_len, nseq, status, trigger ? 1 : 0, wait_ns);
 }
 
 }  // namespace albert

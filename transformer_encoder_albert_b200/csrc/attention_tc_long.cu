@@ -121,7 +121,7 @@ __device__ __forceinline__ int key_blocks(int L) { return (L + LQ - 1) / LQ; }
 __global__ void __launch_bounds__(LA_THREADS, 1)
 attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, bf16 *__restrict__ ctx,
                     const int *__restrict__ seq_start, const int *__restrict__ seq_len, int nseq, int *status,
-                    int trigger) {
+                    int trigger, unsigned long long wait_ns) {
     if (trigger) griddep_launch_dependents();  // the next kernel may take SMs as this grid frees them
     griddep_wait();               // the previous kernel has completed
 
@@ -132,6 +132,7 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, bf16 *__restrict_
     if (threadIdx.x == 0) {
         sm.misc[0] = *reinterpret_cast<const volatile int *>(status);
         *sm.abort_flag = 0;
+        wait_limit_init(wait_ns);
         mbar_init(smem_u32(sm.qk_full), 1);
         mbar_init(smem_u32(sm.qk_empty), 1);
         for (int i = 0; i < NVS; ++i) {
@@ -411,19 +412,16 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, bf16 *__restrict_
 }  // namespace
 
 cudaError_t launch_attention_tc_long(const CUtensorMap &tmQKV, bf16 *ctx, const int *seq_start, const int *seq_len,
-                                     int nseq, int *status, int num_sms, cudaStream_t s, bool trigger) {
+                                     int nseq, int *status, int num_sms, cudaStream_t s, bool trigger,
+                                     unsigned long long wait_ns) {
     if (nseq <= 0) return cudaSuccess;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e =
-            cudaFuncSetAttribute(attn_tc_long_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LA_SMEM);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<unsigned long long> configured{0};
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(attn_tc_long_kernel), LA_SMEM, configured);
+    if (e != cudaSuccess) return e;
     const int total = nseq * LKB * kHeads;
     const int grid = total < num_sms ? total : num_sms;
     return launch_pdl(attn_tc_long_kernel, dim3(grid), dim3(LA_THREADS), LA_SMEM, s, tmQKV, ctx, seq_start, seq_len,
-                      nseq, status, trigger ? 1 : 0);
+                      nseq, status, trigger ? 1 : 0, wait_ns);
 }
 
 }  // namespace albert

@@ -7,9 +7,14 @@
 // A linear layer is y_j = b_j + sum_i x_i W_{j,i} with W stored [out, in]
 // ("Qwen3-TTS and Kokoro", section A), i.e. both operands are K-major.
 //
-// Design (one CTA per SM, persistent over 128x256 output tiles):
-//   warp 0      : TMA producer, 4-stage ring of {A 128x64, B 256x64} bf16 tiles
-//                 (128-byte swizzle, no multicast);
+// Design (one CTA per SM, persistent over output tiles; two variants):
+//   * single CTA per 128x256 tile: 3-stage ring of {A 128x64, B 256x64};
+//   * CTA pair (cluster of 2, tcgen05.mma cta_group::2) per 256x256 tile: each
+//     CTA stages its 128 rows of A and 128 rows of B, 5-stage ring of
+//     {A 128x64, B 128x64} per CTA (the pair is used whenever A has more than
+//     one 128-row block).
+//   warp 0      : TMA producer of the ring (bf16 tiles, 128-byte swizzle, no
+//                 multicast);
 //   warp 1      : TMEM allocator + single-thread tcgen05.mma issuer into two
 //                 128x256 fp32 accumulators (512 TMEM columns), so the epilogue
 //                 of one tile overlaps the main loop of the next;
@@ -210,6 +215,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     if (p.trigger) griddep_launch_dependents();  // the next kernel may take SMs as this grid frees them
     if (threadIdx.x == 0) {
         *sm.abort_flag = 0;
+        wait_limit_init(p.wait_ns);
         for (int i = 0; i < NST; ++i) {
             mbar_init(smem_u32(&sm.full[i]), 1);
             mbar_init(smem_u32(&sm.empty[i]), 1);
@@ -269,7 +275,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             int stage = 0, issued = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int u = slot; u < units && ok; u += nslots) {
+            const int units_loaded = p.withhold_loads ? 0 : units;
+            for (int u = slot; u < units_loaded && ok; u += nslots) {
                 const int m = u / n_sub, n = u % n_sub;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(smem_u32(&sm.empty[stage]), phase ^ 1, sm.abort_flag)) {
@@ -601,25 +608,21 @@ bool gemm_use_pair(int rows_cap, int variant) {
     return rows_cap > BM;
 }
 
+// The kernel instance's shared-memory limit, raised once per device.
 template <int EPI, bool PAIR>
 static cudaError_t configure(int smem) {
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_bf16_kernel<EPI, PAIR>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
-    return cudaSuccess;
+    static std::atomic<unsigned long long> configured{0};
+    return ensure_smem_attr(reinterpret_cast<const void *>(gemm_bf16_kernel<EPI, PAIR>), smem, configured);
 }
 
 // Clusters of two GEMM CTAs that fit on the device at once (every epilogue
-// instance has the same footprint), per device.
+// instance has the same footprint), per device ordinal.
 static int pair_clusters(int num_sms) {
-    static int cached[64] = {0};
+    static std::atomic<int> cached[64];  // zero-initialised (static storage)
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return num_sms / 2;
-    if (cached[dev] > 0) return cached[dev];
+    const int known = cached[dev].load(std::memory_order_acquire);
+    if (known > 0) return known;
     int n = 0;
     if (configure<kEpiBias, true>(Plan<kEpiBias, true>::SMEM) == cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
@@ -637,7 +640,7 @@ static int pair_clusters(int num_sms) {
     }
     cudaGetLastError();
     if (n <= 0 || n > num_sms / 2) n = num_sms / 2;
-    cached[dev] = n;
+    cached[dev].store(n, std::memory_order_release);
     return n;
 }
 

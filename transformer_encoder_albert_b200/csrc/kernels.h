@@ -3,11 +3,29 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 
 namespace albert {
 
 using bf16 = __nv_bfloat16;
+
+// Raise a kernel's dynamic shared-memory limit on the current device, once per
+// device: the attribute belongs to the kernel as loaded on one device, so a
+// process that drives several devices sets it on each.  `done` holds one bit
+// per device ordinal (0..63; above that the attribute is set on every call).
+// Two threads making their first call together may both set it, which is
+// harmless; the bit is published only after the attribute is in place.
+inline cudaError_t ensure_smem_attr(const void *func, int bytes, std::atomic<unsigned long long> &done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
 
 // Launch with programmatic stream serialization: the kernel may begin while
 // the previous kernel in the stream runs; it must call griddep_wait() before
@@ -54,6 +72,8 @@ enum GemmEpi : int {
 
 namespace gemm {
 constexpr int BM = 128, BN = 256, BK = 64;
+// The ring uses STAGES - 1 (PAIR_STAGES - 1) stages: one stage's worth of shared
+// memory goes to the epilogue's staging tiles.
 constexpr int STAGES = 4;       // one CTA per tile: {A 128x64, B 256x64} per stage
 constexpr int PAIR_STAGES = 6;  // CTA pair per 256x256 tile: {A 128x64, B 128x64} per CTA and stage
 constexpr int B_BOX = 128;      // rows of B per TMA box (weight tensor maps)
@@ -91,6 +111,9 @@ struct GemmArgs {
     int *status;               // device status word
     int trigger;               // the next kernel in the stream is one of ours, launched with PDL:
                                // let it start early (0 for a last kernel, or before a copy)
+    unsigned long long wait_ns;  // limit of the bounded waits (0 = kWaitLimitNs, 2 s)
+    int withhold_loads;        // fault injection for tests: the TMA producer issues no loads, so
+                               // the MMA issuer's first wait cannot complete and runs out
 };
 
 // Encode a 2-D bf16 row-major [rows, cols] tensor map with a {64, box_rows}
@@ -134,15 +157,17 @@ cudaError_t launch_attention_bf16(const bf16 *qkv, bf16 *ctx, const int *seq_sta
 // tmQKV / tmQKV64: bf16 maps of the packed [rows, 3*768] buffer with a {64, 128} /
 // {64, 64} box and the 128-byte swizzle.
 constexpr int kAttnTcMaxLen = 128;
+// wait_ns: limit of the kernel's bounded waits (0 = kWaitLimitNs, 2 s).
 cudaError_t launch_attention_tc(const CUtensorMap &tmQKV, const CUtensorMap &tmQKV64, bf16 *ctx, const int *seq_start,
                                 const int *seq_len, int nseq, int *status, int num_sms, cudaStream_t s,
-                                bool trigger);
+                                bool trigger, unsigned long long wait_ns = 0);
 // Same operation on tcgen05 for 128 < max_len <= 512 (one item = one (sequence,
 // 128-query block, head), the item's scores against all keys held in TMEM);
 // tmQKV as above.
 constexpr int kAttnTcLongMaxLen = 512;
 cudaError_t launch_attention_tc_long(const CUtensorMap &tmQKV, bf16 *ctx, const int *seq_start, const int *seq_len,
-                                     int nseq, int *status, int num_sms, cudaStream_t s, bool trigger);
+                                     int nseq, int *status, int num_sms, cudaStream_t s, bool trigger,
+                                     unsigned long long wait_ns = 0);
 cudaError_t launch_attention_f32(const float *qkv, float *ctx, const int *seq_start,
                                  const int *seq_len, int nseq, int max_len,
                                  const int *status, cudaStream_t s);

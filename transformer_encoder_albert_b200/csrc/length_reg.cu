@@ -1,12 +1,12 @@
 // length_reg.cu -- length regulation: token durations, frame offsets and the
 // frame-level expansion of the encoder's features.
 //
-// "ALBERT: How Kokoro's Phoneme Encoder Works", section "The time axis is where
+// "How Kokoro TTS Works and Where CKE Stands", section "The time axis is where
 // a circuit becomes difficult": per token the sigmoid duration channels are
 // summed, divided by the speed, rounded and clamped to at least one frame; their
 // sum A is the number of aligned frames; token features are repeated by the
-// duration vector.  "How Kokoro TTS Works and Where CKE Stands", section "Path
-// one": durations 2, 1, 3 -> p1 p1 p2 p3 p3 p3.
+// duration vector.  "Qwen3-TTS and Kokoro: Two Routes from Text to Speech",
+// section "Path one": durations 2, 1, 3 -> p1 p1 p2 p3 p3 p3.
 //
 // Three launches on the caller's stream (the second and third chained with
 // programmatic dependent launch), bounded by HBM traffic:

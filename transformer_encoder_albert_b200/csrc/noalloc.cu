@@ -14,8 +14,6 @@
 // file-scope __device__ arrays instead of memory the call allocates.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "albert.h"
 #include "kernels.h"
 
@@ -32,33 +30,25 @@ static __device__ __align__(256) bf16 g_ln_zg[kNoAllocZg];
 static __device__ __align__(256) float2 g_ln_stats[kNoAllocStats];
 static __device__ __align__(256) int g_ln_words[2];  // [0] rows to process, [1] status
 
-constexpr int kMaxDevices = 128;
-std::mutex g_setup_mu;
-bf16 *g_zg_dev[kMaxDevices] = {};
-float2 *g_stats_dev[kMaxDevices] = {};
-int *g_words_dev[kMaxDevices] = {};
-
 __global__ void reset_words_kernel(int *words, int rows) {
     words[0] = rows;
     words[1] = 0;  // the status word must start at zero on every call
 }
 
-// Device addresses of the static arrays on the current device, looked up once.
-int setup_device(int dev, bf16 **zg, float2 **stats, int **words) {
-    if (dev < 0 || dev >= kMaxDevices) return ALBERT_ERR_CONFIG;
-    std::lock_guard<std::mutex> lock(g_setup_mu);
-    if (!g_zg_dev[dev]) {
-        void *z = nullptr, *st = nullptr, *w = nullptr;
-        if (cudaGetSymbolAddress(&z, g_ln_zg) != cudaSuccess) return ALBERT_ERR_CUDA;
-        if (cudaGetSymbolAddress(&st, g_ln_stats) != cudaSuccess) return ALBERT_ERR_CUDA;
-        if (cudaGetSymbolAddress(&w, g_ln_words) != cudaSuccess) return ALBERT_ERR_CUDA;
-        g_zg_dev[dev] = static_cast<bf16 *>(z);
-        g_stats_dev[dev] = static_cast<float2 *>(st);
-        g_words_dev[dev] = static_cast<int *>(w);
-    }
-    *zg = g_zg_dev[dev];
-    *stats = g_stats_dev[dev];
-    *words = g_words_dev[dev];
+// Device addresses of the static arrays on the current device.  In host code
+// the arrays' names stand for host-side shadows, so their device addresses are
+// looked up with the device current.  The lookup runs on every call: it is
+// cheap and allocates nothing once the library's module is loaded on the
+// device, and a cached address would go stale if the device's primary context
+// were reset and the module loaded again elsewhere.
+int lookup_scratch(bf16 **zg, float2 **stats, int **words) {
+    void *z = nullptr, *st = nullptr, *w = nullptr;
+    if (cudaGetSymbolAddress(&z, g_ln_zg) != cudaSuccess) return ALBERT_ERR_CUDA;
+    if (cudaGetSymbolAddress(&st, g_ln_stats) != cudaSuccess) return ALBERT_ERR_CUDA;
+    if (cudaGetSymbolAddress(&w, g_ln_words) != cudaSuccess) return ALBERT_ERR_CUDA;
+    *zg = static_cast<bf16 *>(z);
+    *stats = static_cast<float2 *>(st);
+    *words = static_cast<int *>(w);
     return ALBERT_OK;
 }
 
@@ -80,7 +70,7 @@ extern "C" int albert_gemm_residual_ln_noalloc(const void *A, const void *W, con
     bf16 *zg = nullptr;
     float2 *stats = nullptr;
     int *words = nullptr;
-    int rc = setup_device(dev, &zg, &stats, &words);
+    int rc = lookup_scratch(&zg, &stats, &words);
     if (rc) return rc;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return ALBERT_ERR_CUDA;
@@ -109,6 +99,8 @@ extern "C" int albert_gemm_residual_ln_noalloc(const void *A, const void *W, con
     if (launch_ln_rows(zg, stats, ln_g, ln_b, eps, static_cast<bf16 *>(Y), nullptr, M, rows_cap, words, words + 1, s) !=
         cudaSuccess)
         return ALBERT_ERR_CUDA;
+    // The call returns only once its kernels are done with the shared arrays:
+    // callers may rely on this to serialize calls with a host-side lock alone.
     int st = 0;
     if (cudaMemcpyAsync(&st, words + 1, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return ALBERT_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return ALBERT_ERR_CUDA;

@@ -15,8 +15,18 @@ constexpr int kStatusMask = 5;
 constexpr int kStatusSeqlens = 6;
 constexpr int kStatusTimeout = 8;
 
-// A bounded wait gives up after this much wall time (ns, %globaltimer).
+// A bounded wait gives up after this much wall time (ns, %globaltimer) unless
+// the kernel was launched with another limit.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+// The limit of this CTA's bounded waits.  A kernel with bounded waits stores the
+// limit it was launched with (wait_limit_init, one thread, before the barrier
+// that publishes its mbarrier initialisation); mbar_wait and the event loops
+// read it.  Draining in-flight copies on the way out keeps the fixed limit:
+// those copies always complete, and the CTA must not exit before they land.
+static __shared__ unsigned long long s_wait_limit_ns;
+__device__ __forceinline__ void wait_limit_init(unsigned long long ns) { s_wait_limit_ns = ns ? ns : kWaitLimitNs; }
+__device__ __forceinline__ unsigned long long wait_limit() { return s_wait_limit_ns; }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -99,8 +109,8 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 }
 
 // Wait for the phase with the given parity to complete.  Gives up (returns
-// false) when *abort becomes non-zero or after kWaitLimitNs, in which case it
-// raises *abort itself so the other roles of the CTA stop waiting too.
+// false) when *abort becomes non-zero or after the CTA's wait limit, in which
+// case it raises *abort itself so the other roles of the CTA stop waiting too.
 template <bool kClusterScope = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort) {
     auto probe = [&]() { return kClusterScope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
@@ -111,7 +121,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
         for (int i = 0; i < 32; ++i)
             if (probe()) return true;
         if (*abort) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > wait_limit()) {
             *abort = 1;
             return false;
         }
