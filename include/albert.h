@@ -183,7 +183,9 @@ void albert_destroy(albert_handle *h);
  * kernel records ALBERT_ERR_TIMEOUT in the status word, lets its in-flight
  * copies and products finish, frees its tensor memory and returns; every later
  * kernel of the forward then skips its work, so `out` is left as it was and
- * the context stays usable.  (The pages' checked-kernel contract: a failed
+ * the context stays usable.  (A wait that runs out inside the kernel that
+ * writes `out` stops that kernel's remaining work; rows it had already
+ * written stay written.)  (The pages' checked-kernel contract: a failed
  * check stops downstream work and reports an integer status -- "How Kokoro TTS
  * Works and Where CKE Stands", sections on checked kernels.)
  *
@@ -195,7 +197,8 @@ int albert_set_wait_limit(albert_handle *h, long long ns);
 
 /* Failure injection for tests of the path above: on later forwards, the GEMM
  * launches of the kernel classes set in class_mask (bit i = class i of
- * albert_profile_name; only the GEMM classes are accepted) run with their TMA
+ * albert_profile_name; only the GEMM classes and the small-batch kernel are
+ * accepted) run with their TMA
  * producer withholding every load, so their first wait on an operand tile can
  * never complete and runs out after the wait limit.  Nothing faults: the
  * forward reports ALBERT_ERR_TIMEOUT through albert_get_status with `out`
@@ -204,8 +207,25 @@ int albert_set_wait_limit(albert_handle *h, long long ns);
 int albert_test_stall(albert_handle *h, int class_mask);
 
 /* Number of kernel launches one forward of this handle enqueues for a batch
- * with the given shape (used to report launches per step). */
+ * of max_tokens rows through the per-layer kernels (padded_api: 1 for
+ * albert_forward, 0 for albert_forward_varlen). */
 int albert_launches_per_forward(const albert_handle *h, int padded_api);
+
+/* Kernel launches the last forward on this handle enqueued (-1 for NULL). */
+int albert_last_forward_launches(const albert_handle *h);
+
+/* Small batches.  When a forward holds at most 128 token rows (B*T <= 128 for
+ * albert_forward, nseq*max_len <= 128 for albert_forward_varlen) and the handle
+ * is bf16 with one weight set (n_groups == 1) and n_exec >= 1, everything after
+ * the embedding runs in ONE persistent kernel: a cooperative grid that walks
+ * the layer's steps as phases separated by grid barriers, with the FFN fused
+ * per 64-wide hidden chunk (GELU(X1 W1^T + b1) kept on chip and multiplied
+ * straight into W2), instead of ~65 per-layer launches ("ALBERT: How Kokoro's
+ * Phoneme Encoder Works", section "Inside One Real ALBERT Layer", steps 2-6,
+ * and "2. Cross-layer parameter sharing").  Same results within the stated
+ * tolerances; deterministic.  enable: 1 (default) uses it when it applies,
+ * 0 always runs the per-layer kernels.  Other values: ALBERT_ERR_CONFIG. */
+int albert_set_small_batch_kernel(albert_handle *h, int enable);
 
 /* ---- per-kernel timing (optional) ----
  * albert_profile_enable(h, class_mask): for every kernel class whose bit is set

@@ -40,7 +40,7 @@ EXPORTS = (
     "albert_profile_classes",
     "albert_profile_name", "albert_profile_read", "albert_test_gemm", "albert_test_attention",
     "albert_gemm_residual_ln_noalloc", "albert_length_regulate", "albert_length_regulate_scratch_bytes",
-    "albert_set_wait_limit", "albert_test_stall",
+    "albert_set_wait_limit", "albert_test_stall", "albert_set_small_batch_kernel", "albert_last_forward_launches",
 )
 
 
@@ -99,6 +99,8 @@ def lib() -> C.CDLL:
         L.albert_length_regulate_scratch_bytes.restype = C.c_size_t
         L.albert_set_wait_limit.argtypes = [vp, C.c_longlong]
         L.albert_test_stall.argtypes = [vp, i]
+        L.albert_set_small_batch_kernel.argtypes = [vp, i]
+        L.albert_last_forward_launches.argtypes = [vp]
         _lib = L
     return _lib
 
@@ -239,6 +241,14 @@ class Encoder:
 
     def status(self, stream=None) -> int:
         return albert_get_status(self.h, stream)
+
+    def set_small_batch_kernel(self, enable: bool) -> None:
+        """Batches of at most 128 token rows: one persistent kernel (True, default)
+        or the per-layer kernels (False)."""
+        _check(lib().albert_set_small_batch_kernel(self.h, 1 if enable else 0), "albert_set_small_batch_kernel")
+
+    def last_forward_launches(self) -> int:
+        return lib().albert_last_forward_launches(self.h)
 
     def set_wait_limit(self, ns: int) -> None:
         """Limit (ns) of the kernels' bounded waits on later forwards; 0 = default (2 s)."""

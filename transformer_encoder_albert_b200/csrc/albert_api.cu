@@ -24,11 +24,12 @@ namespace {
 
 enum ProfClass {
     kProfPrep = 0, kProfEmbed, kProfGemmIn, kProfGemmQKV, kProfAttention, kProfGemmWoLN,
-    kProfGemmW1Gelu, kProfGemmW2LN, kProfGemmOut, kProfOutput, kProfLayerNorm, kProfClasses
+    kProfGemmW1Gelu, kProfGemmW2LN, kProfGemmOut, kProfOutput, kProfLayerNorm, kProfSmall, kProfClasses
 };
 const char *kProfNames[kProfClasses] = {
     "prep", "embed_ln", "gemm_in_proj", "gemm_qkv", "attention", "gemm_out_proj_ln",
-    "gemm_ffn_up_gelu", "gemm_ffn_down_ln", "gemm_final_proj", "output_rows", "layer_norm_f32"};
+    "gemm_ffn_up_gelu", "gemm_ffn_down_ln", "gemm_final_proj", "output_rows", "layer_norm_f32",
+    "small_batch_forward"};
 
 constexpr int kEventPool = 16384;
 
@@ -101,6 +102,17 @@ struct albert_handle {
     CUtensorMap tm_E, tm_X, tm_C, tm_X1, tm_H, tm_Z, tm_QKV, tm_QKV64;
     CUtensorMap tm_win, tm_wout;
     CUtensorMap t32_X, t32_QKV, t32_X1, t32_H, t32_Z;  // 32x32-box maps: epilogue stores / residual loads
+
+    // small batches (at most 128 token rows): the whole forward after the
+    // embedding in one persistent kernel; its own statistics, FFN partial sums,
+    // barrier counter and {64, 64}-box tensor maps
+    bool small_ok = false;       // the handle's configuration allows it
+    bool small_enabled = true;   // albert_set_small_batch_kernel
+    float2 *sst1 = nullptr, *sst2 = nullptr;
+    float *spart = nullptr;
+    int *sbar = nullptr;
+    CUtensorMap sm_E, sm_X, sm_C, sm_X1, sm_Z, sm_win, sm_wqkv, sm_wo, sm_w1, sm_w2, sm_wout;
+    int last_launches = 0;       // kernel launches of the last forward
 
     // bounded waits inside the kernels: limit (0 = the kernels' default, 2 s) and,
     // for failure-path tests, kernel classes whose GEMM producer withholds its loads
@@ -208,6 +220,7 @@ struct Launch {
         return ALBERT_OK;
     }
     int end(cudaError_t launched) {
+        if (launched == cudaSuccess) ++h->last_launches;
         if (launched != cudaSuccess) {
             if (getenv("ALBERT_DEBUG"))
                 fprintf(stderr, "albert: launch of %s failed: %s\n", kProfNames[cls], cudaGetErrorString(launched));
@@ -307,6 +320,37 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
     LAUNCH(L, kProfEmbed, launch_embed(ea, L.s));
 
     const int D = out_width(h);
+    // small batches: everything after the embedding in one kernel
+    const long long row_bound = padded_api ? (long long)nseq * T : (long long)nseq * max_len;
+    if (bf && h->small_ok && h->small_enabled && row_bound <= kSmallMaxRows && max_len <= kAttnTcMaxLen) {
+        const auto &W = h->grp[0];
+        const auto &E1 = h->ex[c.n_exec > 1 ? 1 : 0];
+        SmallFwdArgs s{};
+        s.tmE = h->sm_E; s.tmX = h->sm_X; s.tmC = h->sm_C; s.tmX1 = h->sm_X1; s.tmZ = h->sm_Z;
+        s.tmQKV = h->tm_QKV; s.tmQKV64 = h->tm_QKV64;
+        s.tmWin = h->sm_win; s.tmWqkv = h->sm_wqkv; s.tmWo = h->sm_wo; s.tmW1 = h->sm_w1; s.tmW2 = h->sm_w2;
+        s.tmWout = c.out_dim > 0 ? h->sm_wout : h->sm_wo;  // (unused without a final projection)
+        s.X = static_cast<bf16 *>(h->X); s.QKV = static_cast<bf16 *>(h->QKV); s.C = static_cast<bf16 *>(h->C);
+        s.X1 = static_cast<bf16 *>(h->X1); s.Z = static_cast<bf16 *>(h->Z);
+        s.st1 = h->sst1; s.st2 = h->sst2; s.part = h->spart;
+        s.b_in = h->b_in;
+        s.bqkv0 = W.bqkv; s.bqkv = E1.c_qkv; s.s_qkv = E1.s_qkv;
+        s.bo0 = W.bo; s.bo = E1.bias_o2;
+        s.ln1_g = W.ln1_g; s.s_1 = W.s_1; s.c_1 = W.c_1; s.bias_21 = W.bias_21;
+        s.ln2_g = W.ln2_g; s.ln2_b = W.ln2_b; s.s_out = h->s_out; s.c_out = h->c_out;
+        s.out = static_cast<bf16 *>(out); s.out_dim = c.out_dim; s.row_dst = h->row_dst; s.out_rows = out_rows;
+        s.seq_start = h->seq_start; s.seq_len = h->seq_len; s.nseq = nseq;
+        s.n_rows = h->n_rows; s.status = h->status; s.bar = h->sbar;
+        s.n_exec = c.n_exec; s.eps = c.ln_eps; s.wait_ns = h->wait_ns;
+        s.withhold_loads = (h->stall_mask >> kProfSmall) & 1u;
+        LAUNCH(L, kProfSmall, launch_forward_small(s, small_forward_grid(h->num_sms), L.s));
+        if (padded_api && c.out_layout == 1)
+            LAUNCH(L, kProfOutput, launch_transpose_out(h->tout, user_out, nseq, T, D, (int)elem_bytes(h), h->seq_len,
+                                                        h->status, L.s));
+        else if (padded_api)
+            LAUNCH(L, kProfOutput, launch_zero_pad(out, nseq, T, D, (int)elem_bytes(h), h->seq_len, h->status, L.s));
+        return ALBERT_OK;
+    }
     if (bf) {
         int rc;
         if ((rc = gemm_bf16(L, kProfGemmIn, kEpiBias, h->tm_E, h->tm_win, h->t32_X, h->t32_X,
@@ -586,6 +630,26 @@ int create_impl(albert_handle *h, const albert_weights *w) {
                 make_tmap_bf16(&gp.tm_w1, gp.w1, kFfn, kHidden, gemm::B_BOX) ||
                 make_tmap_bf16(&gp.tm_w2, gp.w2, kHidden, kFfn, gemm::B_BOX))
                 return ALBERT_ERR_CUDA;
+        // the small-batch kernel: one weight set, at least one execution
+        if (c.n_groups == 1 && c.n_exec >= 1) {
+            const auto &gp = h->grp[0];
+            if ((rc = dev_alloc(h, (void **)&h->sst1, kSmallMaxRows * kSmallParts * sizeof(float2)))) return rc;
+            if ((rc = dev_alloc(h, (void **)&h->sst2, kSmallMaxRows * kSmallParts * sizeof(float2)))) return rc;
+            if ((rc = dev_alloc(h, (void **)&h->spart, (size_t)(kFfn / 64) * kSmallMaxRows * kHidden * sizeof(float))))
+                return rc;
+            if ((rc = dev_alloc(h, (void **)&h->sbar, sizeof(int)))) return rc;
+            if (make_tmap_bf16(&h->sm_E, h->E, R, kEmb, 64) || make_tmap_bf16(&h->sm_X, h->X, R, kHidden, 64) ||
+                make_tmap_bf16(&h->sm_C, h->C, R, kHidden, 64) || make_tmap_bf16(&h->sm_X1, h->X1, R, kHidden, 64) ||
+                make_tmap_bf16(&h->sm_Z, h->Z, R, kHidden, 64) ||
+                make_tmap_bf16(&h->sm_win, h->w_in, kHidden, kEmb, 64) ||
+                make_tmap_bf16(&h->sm_wqkv, gp.wqkv, kQKV, kHidden, 64) ||
+                make_tmap_bf16(&h->sm_wo, gp.wo, kHidden, kHidden, 64) ||
+                make_tmap_bf16(&h->sm_w1, gp.w1, kFfn, kHidden, 64) ||
+                make_tmap_bf16(&h->sm_w2, gp.w2, kHidden, kFfn, 64) ||
+                (O && make_tmap_bf16(&h->sm_wout, h->w_out, O, kHidden, 64)))
+                return ALBERT_ERR_CUDA;
+            h->small_ok = true;
+        }
     }
     TRY(cudaStreamSynchronize(s));
     return ALBERT_OK;
@@ -609,6 +673,7 @@ void free_all(albert_handle *h) {
 
 int forward_padded(albert_handle *h, const int64_t *ids, const uint8_t *mask, int B, int T, void *out,
                    cudaStream_t s) {
+    h->last_launches = 0;
     Launch L{h, s};
     LAUNCH(L, kProfPrep, launch_prep_padded(mask, B, T, h->cfg.pack, h->cfg.max_tokens, h->seq_start, h->seq_len,
                                             h->n_rows, h->status, s, true));
@@ -651,6 +716,7 @@ int albert_forward_varlen(albert_handle *h, const int64_t *ids, const int32_t *c
     if (nseq < 1 || nseq > h->seq_cap || max_len < 1 || max_len > h->cfg.max_pos) return ALBERT_ERR_SHAPE;
     if (h->cfg.out_layout != 0) return ALBERT_ERR_CONFIG;  // packed rows have no per-sequence [D, T] form
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    h->last_launches = 0;
     Launch L{h, s};
     LAUNCH(L, kProfPrep, launch_prep_varlen(cu_seqlens, nseq, max_len, h->cfg.max_tokens, h->seq_start, h->seq_len,
                                             h->n_rows, h->status, s, true));
@@ -794,6 +860,15 @@ int albert_profile_retain(albert_handle *h, int on) {
     return ALBERT_OK;
 }
 
+int albert_set_small_batch_kernel(albert_handle *h, int enable) {
+    if (!h) return ALBERT_ERR_NULL;
+    if (enable != 0 && enable != 1) return ALBERT_ERR_CONFIG;
+    h->small_enabled = enable == 1;
+    return ALBERT_OK;
+}
+
+int albert_last_forward_launches(const albert_handle *h) { return h ? h->last_launches : -1; }
+
 int albert_set_wait_limit(albert_handle *h, long long ns) {
     if (!h) return ALBERT_ERR_NULL;
     if (ns < 0) return ALBERT_ERR_CONFIG;
@@ -804,7 +879,8 @@ int albert_set_wait_limit(albert_handle *h, long long ns) {
 int albert_test_stall(albert_handle *h, int class_mask) {
     if (!h) return ALBERT_ERR_NULL;
     const unsigned gemm_classes = (1u << kProfGemmIn) | (1u << kProfGemmQKV) | (1u << kProfGemmWoLN) |
-                                  (1u << kProfGemmW1Gelu) | (1u << kProfGemmW2LN) | (1u << kProfGemmOut);
+                                  (1u << kProfGemmW1Gelu) | (1u << kProfGemmW2LN) | (1u << kProfGemmOut) |
+                                  (1u << kProfSmall);
     if ((unsigned)class_mask & ~gemm_classes) return ALBERT_ERR_CONFIG;
     if (class_mask && h->cfg.dtype != ALBERT_BF16) return ALBERT_ERR_CONFIG;  // the fp32 kernels never wait
     h->stall_mask = (unsigned)class_mask;

@@ -147,6 +147,43 @@ cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB,
                         const CUtensorMap &tmRes, const GemmArgs &args, int grid, cudaStream_t s,
                         int variant = kGemmAuto, bool pdl = true);
 
+// ------------------------------------------------- small-batch whole forward --
+// The whole forward for at most 128 token rows in one cooperative persistent
+// kernel (forward_small.cu).  A-operand maps have {64, 64} boxes with the
+// 128-byte swizzle over the workspace rows; weight maps {64, 64} boxes.
+// Statistics are twelve 64-column (mean, M2) partials per row.
+constexpr int kSmallParts = 12;
+constexpr int kSmallMaxRows = 128;
+struct SmallFwdArgs {
+    CUtensorMap tmE, tmX, tmC, tmX1, tmZ;       // E [rows,128]; X, C, X1 = z1*g1, Z = z2*g2 [rows,768]
+    CUtensorMap tmQKV, tmQKV64;                 // [rows, 2304] with {64,128} / {64,64} boxes
+    CUtensorMap tmWin, tmWqkv, tmWo, tmW1, tmW2, tmWout;
+    bf16 *X, *QKV, *C, *X1, *Z;
+    float2 *st1, *st2;                          // [128][12]
+    float *part;                                // [32][128][768] FFN partial sums
+    const float *b_in;
+    const float *bqkv0, *bqkv, *s_qkv;          // first execution: plain bias; later: folded LN2
+    const float *bo0, *bo;                      // out-proj bias (later executions: + beta2)
+    const float *ln1_g, *s_1, *c_1, *bias_21;   // LN1 gamma; W1 folds; b2 + beta1
+    const float *ln2_g, *ln2_b, *s_out, *c_out;
+    bf16 *out;
+    int out_dim;                                // 512, or 0: the hidden states LN2(z2)
+    const int *row_dst;
+    int out_rows;
+    const int *seq_start, *seq_len;
+    int nseq;
+    const int *n_rows;
+    int *status;
+    int *bar;                                   // grid-barrier counter (zeroed by the launcher)
+    int n_exec;                                 // >= 1
+    float eps;
+    unsigned long long wait_ns;
+    int withhold_loads;                         // fault injection for tests (see GemmArgs)
+};
+int small_forward_grid(int num_sms);
+// Zeroes the barrier counter, then a cooperative launch on stream s.
+cudaError_t launch_forward_small(const SmallFwdArgs &a, int grid, cudaStream_t s);
+
 // ---------------------------------------------------------------- attention --
 // Masked bidirectional attention, bf16 tensor-core kernel (mma.sync m16n8k16).
 // trigger: the next kernel in the stream is one of ours launched with PDL (see GemmArgs).
