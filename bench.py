@@ -59,15 +59,18 @@ def flops_per_class(lengths, arch, rows):
         "gemm_ffn_up_gelu": 2.0 * rows * H * F,
         "gemm_ffn_down_ln": 2.0 * rows * F * H,
         "gemm_final_proj": 2.0 * rows * H * O,
+        # the whole forward after the embedding in one persistent kernel (batches of at most 128 rows)
+        "small_batch_forward": forward_flops(lengths, arch)[0],
     }
 
 
 def forward_flops(lengths, arch):
-    n_tok = int(sum(int(l) for l in lengths))
-    f = flops_per_class(lengths, arch, n_tok)
-    per_exec = f["gemm_qkv"] + f["attention"] + f["gemm_out_proj_ln"] + f["gemm_ffn_up_gelu"] + f["gemm_ffn_down_ln"]
-    gemm = f["gemm_in_proj"] + f["gemm_final_proj"] + arch["n_exec"] * (per_exec - f["attention"])
-    return gemm + arch["n_exec"] * f["attention"], gemm
+    """(whole forward, its GEMMs) in algorithmic FLOPs over the valid tokens."""
+    H, E, F, O = arch["hidden"], arch["emb"], arch["ffn"], arch["out_dim"]
+    n_tok = float(sum(int(l) for l in lengths))
+    s2 = float(sum(int(l) ** 2 for l in lengths))
+    gemm = 2.0 * n_tok * (E * H + arch["n_exec"] * (H * 3 * H + H * H + H * F + F * H) + H * O)
+    return gemm + arch["n_exec"] * 4.0 * s2 * H, gemm
 
 
 # DRAM traffic per launch of a kernel class, from ncu captures summarised in
@@ -354,15 +357,14 @@ def run_gpu(args):
         runs = [("b8_T128", False, False), ("b64_T128_normal", False, False), ("b32_T512_long", False, False),
                 ("b256_T128", False, False), ("b256_T128", True, False), ("b1_T64_latency", False, False),
                 ("b1_T64_latency", False, True)]
-        lines = [measure_workload(args, ctx, name, padded, graph, extras=False) for name, padded, graph in runs]
     else:
-        lines = [measure_workload(args, ctx, args.workload, args.padded, args.graph, extras=True)]
+        runs = [(args.workload, args.padded, args.graph)]
+    for name, padded, graph in runs:
+        line = measure_workload(args, ctx, name, padded, graph, extras=not args.all_configs)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
-    if rank == 0:
-        for line in lines:
-            if line is not None:
-                print(json.dumps(line), flush=True)
     return 0
 
 
@@ -393,7 +395,7 @@ def measure_workload(args, ctx, name, padded, graph_mode, extras):
     n_tok = int(L.sum())
     ids_d = torch.as_tensor(ids).cuda()
     mask_d = torch.as_tensor(mask).cuda()
-    enc = tea.Encoder(w, arch, dtype="bf16", max_tokens=wl.B * wl.T, pack=not padded)
+    enc = tea.Encoder(w, arch, dtype=args.dtype, max_tokens=wl.B * wl.T, pack=not padded)
     out = torch.empty(wl.B, wl.T, arch["out_dim"], device="cuda", dtype=torch.bfloat16)
     stream = torch.cuda.current_stream()
     rows = n_tok if not padded else wl.B * wl.T
@@ -474,6 +476,7 @@ def measure_workload(args, ctx, name, padded, graph_mode, extras):
     if st != 0:
         raise SystemExit(f"device status {tea.STATUS_NAMES.get(st, st)}")
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    launches = enc.last_forward_launches()  # kernels of one timed forward (the captured one for a graph)
     if graph is None:
         dom = enc.profile_read()[dominant]
     enc.profile_retain(False)
@@ -554,26 +557,32 @@ def measure_workload(args, ctx, name, padded, graph_mode, extras):
     peaks, peaks_src = load_peaks()
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     peak_sus = peaks.get("bf16_tflops_sustained")
+    peak_note = f"{peaks_src} bf16_tflops (burst)"
+    fp8_classes = ("gemm_qkv", "gemm_out_proj_ln", "gemm_ffn_up_gelu", "gemm_ffn_down_ln")
+    if args.dtype == "fp8":
+        # E4M3 products: the measured bf16 peak times the nominal dense fp8 / bf16 ratio (2)
+        peak, peak_sus = 2.0 * peak, (2.0 * peak_sus if peak_sus else None)
+        peak_note = f"{peaks_src} bf16_tflops (burst) x 2, the nominal dense E4M3 / bf16 ratio"
     lenreg = (measure_length_regulation(torch, synth, tea, L, flush, peaks, peaks_src, stream, args.steps)
               if extras else None)
     dom_ms = dom[1] / max(dom[0], 1)
     achieved = per_launch.get(dominant, 0.0) / (dom_ms / 1000.0) / 1e12
     traffic, traffic_note = load_traffic(dominant, label, wl.T)
     bound = "tensor"
-    roofline = {"kernel": dominant, "bound": bound, "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                "traffic_source": traffic_note,
-                "peak_source": f"{peaks_src} bf16_tflops (burst: the kernel runs {dom_ms * 1000:.0f} us "
-                               f"inside a {ms_per_step:.3f} ms step)",
+    dom_peak = peak if (args.dtype == "bf16" or dominant in fp8_classes) else peak / 2.0
+    roofline = {"kernel": dominant, "bound": bound, "achieved": achieved, "peak": dom_peak,
+                "unit": "TFLOP/s", "frac": achieved / dom_peak, "traffic": traffic if args.dtype == "bf16" else None,
+                "traffic_source": traffic_note if args.dtype == "bf16" else "no ncu capture of the E4M3 kernels",
+                "peak_source": f"{peak_note} (the kernel runs {dom_ms * 1000:.0f} us inside a {ms_per_step:.3f} ms step)",
                 "frac_of_sustained": (achieved / peak_sus) if peak_sus else None,
                 "launches_timed": dom[0], "launches_timed_note": f"1 of {per_step} per step", "avg_launch_ms": dom_ms,
                 "flops_per_launch": per_launch.get(dominant, 0.0)}
     clocks = sampler.summary(t_wall0, t_wall1)
-    launches = enc.launches_per_forward(True)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if args.dtype == "bf16" else "e4m3 (the four layer GEMMs) + bf16",
         "data": "synthetic (seeded N(0,0.02) weights rounded to bf16, seeded ids and lengths)",
         "config": {"workload": label, "batch": wl.B,
                    "seq_len": wl.T, "lengths": wl.describe(), "valid_tokens_per_step_per_gpu": n_tok,
@@ -583,10 +592,11 @@ def measure_workload(args, ctx, name, padded, graph_mode, extras):
                    "l2": "flushed between timed steps (512 MiB write)"},
         "padded_slot_tokens_per_s": sum_r(float(wl.B * wl.T * args.steps)) / (total_ms / 1000.0),
         "tensor_peak_frac": {"whole_encoder": fwd_flops / (ms_per_step / 1000.0) / 1e12 / peak,
-                             "gemm_path": gemm_flops / (gemm_ms / 1000.0) / 1e12 / peak,
+                             "gemm_path": (gemm_flops / (gemm_ms / 1000.0) / 1e12 / peak) if gemm_ms > 0 else None,
                              "gemm_path_source": "per-class profiled replay (an event pair around every launch "
-                                                 "breaks their chaining: a lower bound)",
-                             "peak_tflops": peak, "peak_source": f"{peaks_src} bf16_tflops (burst)",
+                                                 "breaks their chaining: a lower bound)" if gemm_ms > 0 else
+                                                 "no separate GEMM launches (one persistent kernel)",
+                             "peak_tflops": peak, "peak_source": peak_note,
                              "whole_encoder_of_sustained": (fwd_flops / (ms_per_step / 1000.0) / 1e12 / peak_sus)
                              if peak_sus else None},
         "roofline": roofline,
@@ -625,6 +635,8 @@ def main():
                     help="time replays of the forward captured in a CUDA graph instead of stream launches")
     ap.add_argument("--ncu-forwards", type=int, default=0,
                     help="run this many untimed forwards and exit (for ncu captures); no JSON metric line")
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "fp8"],
+                    help="fp8: the four layer GEMMs on E4M3 operands with per-row scales")
     ap.add_argument("--all-configs", action="store_true",
                     help="one JSON line per workload of the suite (packed and padded b256, b1_T64 stream and graph)")
     args = ap.parse_args()

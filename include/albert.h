@@ -60,6 +60,10 @@ extern "C" {
 /* ---- precision of the whole path ---- */
 #define ALBERT_BF16 0  /* bf16 weights and activations, fp32 accumulation and norms */
 #define ALBERT_FP32 1  /* fp32 everywhere (SIMT kernels; small workloads)          */
+#define ALBERT_FP8  2  /* the four layer GEMMs (Q|K|V, out-proj, FFN up and down)
+                          on E4M3 operands with per-row scales (activations per
+                          token, weights per output channel), everything else as
+                          ALBERT_BF16; see albert_test_quant_e4m3               */
 
 /* Architecture and capacity.  The kernels support exactly: emb 128, hidden 768,
  * heads 12 (64 wide), ffn 2048, max_pos <= 512, out_dim 512 or 0 (0 = return the
@@ -145,6 +149,19 @@ int albert_forward(albert_handle *h, const int64_t *ids, const uint8_t *mask, in
  * Asynchronous on `stream`. */
 int albert_forward_varlen(albert_handle *h, const int64_t *ids, const int32_t *cu_seqlens,
                           int nseq, int max_len, void *out, void *stream);
+
+/* The encoder from its post-embedding-LayerNorm rows instead of ids: emb is
+ * [N_tok, 128] fp32 (device, 16-byte aligned), the rows of the packed
+ * sequences as albert_forward_varlen lays out ids; everything after the
+ * embedding's LayerNorm (the 128 -> 768 projection on) runs as in
+ * albert_forward_varlen, and out is [N_tok, D].  This is the input the pages
+ * evaluate a compiled encoder on ("Kokoro-82M-encoder-hailo10h", section "How
+ * to deploy on Hailo-10H": the encoder takes the [1, 128, 128] LayerNorm output
+ * computed on the CPU; section "Eval results": 16 random N(0,1) inputs of that
+ * shape).
+ * Errors as albert_forward_varlen; out_layout must be 0. */
+int albert_forward_embedded(albert_handle *h, const float *emb, const int32_t *cu_seqlens, int nseq, int max_len,
+                            void *out, void *stream);
 
 /* Convenience path with HOST buffers: copies ids/mask (pinned or pageable) to
  * the handle's device staging area, runs albert_forward, copies the result
@@ -303,9 +320,24 @@ size_t albert_length_regulate_scratch_bytes(int n_tok);
  * by default the pair is used whenever M > 128, as in albert_forward. */
 #define ALBERT_GEMM_SINGLE_CTA 16
 #define ALBERT_GEMM_CTA_PAIR 32
+/* Adding ALBERT_GEMM_E4M3 runs the E4M3 variant: A and W are first quantized
+ * per row as albert_test_quant_e4m3 does (into temporaries), then multiplied
+ * on tcgen05 (kind::f8f6f4) with the epilogue starting from
+ * acc * a_scale[row] * w_scale[col].  Needs K % 256 == 0 and K <= 2048. */
+#define ALBERT_GEMM_E4M3 64
 int albert_test_gemm(const void *A, const void *W, const float *bias, const void *R,
                      const float *ln_g, const float *ln_b, float eps, const int32_t *row_dst,
                      void *Y, int M, int N, int K, int epi, void *stream);
+
+/* Row quantization of the FP8 variant (the reading of "Kokoro-82M-encoder-
+ * hailo10h", section "Eval results", that a quantized encoder is compared with
+ * its full-precision outputs; the scheme is this library's): for each row of
+ * x [rows, K] bf16 (device), amax = max |x|, scale[row] = amax / 448 and
+ * q = E4M3(fp32(x * (448 / amax))) with round to nearest even and saturation
+ * (fp32 divisions and product); a row of zeros gives scale 0 and q 0.
+ * q: [rows, K] bytes (E4M3 codes), scale: [rows] fp32, device.  K % 256 == 0,
+ * 256 <= K <= 2048 (else ALBERT_ERR_SHAPE).  Synchronous. */
+int albert_test_quant_e4m3(const void *x, int rows, int K, void *q, float *scale, void *stream);
 
 /* Masked bidirectional attention on a packed [N_tok, 3*768] bf16 QKV buffer
  * (Q | K | V, head h = columns 64h..64h+63 of each); cu_seqlens as in

@@ -86,7 +86,10 @@ class Sim:
 # ----------------------------------------------------------------- short kernel --
 # One item per (sequence, head), four TMEM buffers, Q/K and V stages with the
 # buffer's index; a stage is released by the S (Q/K) or O (V) completion of the
-# item four back.  Two softmax groups take alternate items.
+# item four back.  Two softmax groups take alternate items.  Two issuing
+# threads: one issues the S products in item order, the other the O products.
+# planted: True reuses a V stage one item early; "s_early" issues S into a
+# buffer without waiting for the output warps to have read its previous O.
 def short_kernel(n_items, seed, planted=False):
     NB = 4
     sim = Sim(seed)
@@ -111,23 +114,24 @@ def short_kernel(n_items, seed, planted=False):
                 nv += 1
             yield
 
-    def mma():
-        ns = no = 0
-        while no < n_items:
-            if no < ns:
-                tb = no % NB
-                if sim.bars[f"p_full{tb}"].test((no // NB) & 1) and sim.bars[f"v_full{tb}"].test((no // NB) & 1):
-                    tag = sim.bars[f"v_full{tb}"].tags[no // NB]
-                    assert tag == ("v", no), ("O product reads a V stage holding", tag, "for item", no)
-                    sim.commit(f"o_full{tb}", ("o", no))
-                    no += 1
-            if ns < n_items and ns < no + NB:
-                tb = ns % NB
-                if sim.bars[f"qk_full{tb}"].test((ns // NB) & 1) and sim.bars[f"o_empty{tb}"].test(((ns // NB) & 1) ^ 1):
-                    assert tmem.get(tb) in (None, ("read", ns - NB)), ("S over a buffer still in use", tmem.get(tb))
-                    tmem[tb] = ("s", ns)
-                    sim.commit(f"s_full{tb}", ("s", ns))
-                    ns += 1
+    def mma_s():
+        for ns in range(n_items):
+            tb = ns % NB
+            yield from sim.wait(f"qk_full{tb}", (ns // NB) & 1, ("qk", ns))
+            if planted != "s_early":
+                yield from sim.wait(f"o_empty{tb}", ((ns // NB) & 1) ^ 1)
+            assert tmem.get(tb) in (None, ("read", ns - NB)), ("S over a buffer still in use", tmem.get(tb))
+            tmem[tb] = ("s", ns)
+            sim.commit(f"s_full{tb}", ("s", ns))
+            yield
+
+    def mma_o():
+        for no in range(n_items):
+            tb = no % NB
+            yield from sim.wait(f"p_full{tb}", (no // NB) & 1, ("p", no))
+            yield from sim.wait(f"v_full{tb}", (no // NB) & 1, ("v", no))
+            assert tmem.get(tb) == ("s", no), ("O product into a buffer holding", tmem.get(tb), "for item", no)
+            sim.commit(f"o_full{tb}", ("o", no))
             yield
 
     def softmax(g):
@@ -148,7 +152,8 @@ def short_kernel(n_items, seed, planted=False):
             if sim.bars[f"o_empty{tb}"].arrived == 0:
                 tmem[tb] = ("read", i)
 
-    sim.run([producer(), mma()] + [softmax(g) for g in range(2) for _ in range(4)] + [output(q) for q in range(4)])
+    sim.run([producer(), mma_s(), mma_o()] + [softmax(g) for g in range(2) for _ in range(4)] +
+            [output(q) for q in range(4)])
 
 
 # ------------------------------------------------------------------ long kernel --
@@ -272,4 +277,5 @@ def test_planted_mistakes_are_caught():
         return False
 
     assert fails(lambda s: short_kernel(12, s, planted=True))
+    assert fails(lambda s: short_kernel(12, s, planted="s_early"))
     assert fails(lambda s: long_kernel([(4, [True] * 4)] * 6, s, planted=True))

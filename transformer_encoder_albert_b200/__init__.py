@@ -19,7 +19,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libalbert_b200.so")
 
 ALBERT_OK = 0
-ALBERT_BF16, ALBERT_FP32 = 0, 1
+ALBERT_BF16, ALBERT_FP32, ALBERT_FP8 = 0, 1, 2
+DTYPES = {"bf16": ALBERT_BF16, "fp32": ALBERT_FP32, "fp8": ALBERT_FP8}
 STATUS_NAMES = {
     0: "ALBERT_OK", 1: "ALBERT_ERR_NULL", 2: "ALBERT_ERR_CONFIG", 3: "ALBERT_ERR_SHAPE",
     4: "ALBERT_ERR_ID", 5: "ALBERT_ERR_MASK", 6: "ALBERT_ERR_SEQLENS", 7: "ALBERT_ERR_CUDA",
@@ -41,6 +42,7 @@ EXPORTS = (
     "albert_profile_name", "albert_profile_read", "albert_test_gemm", "albert_test_attention",
     "albert_gemm_residual_ln_noalloc", "albert_length_regulate", "albert_length_regulate_scratch_bytes",
     "albert_set_wait_limit", "albert_test_stall", "albert_set_small_batch_kernel", "albert_last_forward_launches",
+    "albert_test_quant_e4m3", "albert_forward_embedded",
 )
 
 
@@ -101,6 +103,8 @@ def lib() -> C.CDLL:
         L.albert_test_stall.argtypes = [vp, i]
         L.albert_set_small_batch_kernel.argtypes = [vp, i]
         L.albert_last_forward_launches.argtypes = [vp]
+        L.albert_test_quant_e4m3.argtypes = [vp, i, i, vp, vp, vp]
+        L.albert_forward_embedded.argtypes = [vp, vp, vp, i, i, vp, vp]
         _lib = L
     return _lib
 
@@ -128,7 +132,7 @@ def make_config(arch: dict, dtype: str = "bf16", max_tokens: int = 4096, pack: b
         ffn=arch["ffn"], n_exec=arch["n_exec"] if n_exec is None else n_exec, n_groups=n_groups,
         max_pos=arch["max_pos"], n_types=arch["n_types"],
         out_dim=arch["out_dim"] if out_dim is None else out_dim,
-        dtype=ALBERT_BF16 if dtype == "bf16" else ALBERT_FP32, max_tokens=max_tokens,
+        dtype=DTYPES[dtype], max_tokens=max_tokens,
         pack=1 if pack else 0, out_layout=out_layout, ln_eps=arch["ln_eps"])
 
 
@@ -207,14 +211,14 @@ class Encoder:
 
     def _out(self, shape):
         import torch
-        dt = torch.bfloat16 if self.dtype == "bf16" else torch.float32
+        dt = torch.float32 if self.dtype == "fp32" else torch.bfloat16
         return torch.empty(*shape, self.out_dim, device="cuda", dtype=dt)
 
     def forward(self, ids, mask, out=None, stream=None):
         if out is None:
             if self.out_layout == 1:
                 import torch
-                dt = torch.bfloat16 if self.dtype == "bf16" else torch.float32
+                dt = torch.float32 if self.dtype == "fp32" else torch.bfloat16
                 out = torch.empty(ids.shape[0], self.out_dim, ids.shape[1], device="cuda", dtype=dt)
             else:
                 out = self._out(ids.shape)
@@ -225,6 +229,16 @@ class Encoder:
         if out is None:
             out = self._out((ids.shape[0],))
         albert_forward_varlen(self.h, ids, cu_seqlens, max_len, out, stream)
+        return out
+
+    def forward_embedded(self, emb, cu_seqlens, max_len, out=None, stream=None):
+        """From post-embedding-LayerNorm rows emb [N_tok, 128] fp32 (packed as in
+        forward_varlen) to the encoder output [N_tok, D]."""
+        if out is None:
+            out = self._out((emb.shape[0],))
+        nseq = cu_seqlens.numel() - 1
+        _check(lib().albert_forward_embedded(self.h, _ptr(emb), _ptr(cu_seqlens), nseq, int(max_len), _ptr(out),
+                                             _stream_ptr(stream)), "albert_forward_embedded")
         return out
 
     def forward_host(self, ids_host, mask_host, out_host, stream=None) -> int:
@@ -313,17 +327,30 @@ def profile_class_names() -> list:
 
 
 GEMM_VARIANTS = {"auto": 0, "single": 16, "pair": 32}
+GEMM_E4M3 = 64
 
 
 def test_gemm(A, W, bias, Y, epi: int, R=None, ln_g=None, ln_b=None, eps: float = 1e-12,
-              row_dst=None, stream=None, variant: str = "auto") -> int:
+              row_dst=None, stream=None, variant: str = "auto", e4m3: bool = False) -> int:
     """Run the tcgen05 GEMM alone (single-kernel parity tests).  variant picks
-    the one-CTA or the CTA-pair kernel ("auto": the pair when M > 128)."""
+    the one-CTA or the CTA-pair kernel ("auto": the pair when M > 128); e4m3
+    quantizes both operands per row and runs the E4M3 variant."""
     M, K = A.shape
     N = W.shape[0]
     return lib().albert_test_gemm(_ptr(A), _ptr(W), _ptr(bias), _ptr(R), _ptr(ln_g), _ptr(ln_b),
                                   float(eps), _ptr(row_dst), _ptr(Y), M, N, K,
-                                  epi | GEMM_VARIANTS[variant], _stream_ptr(stream))
+                                  epi | GEMM_VARIANTS[variant] | (GEMM_E4M3 if e4m3 else 0), _stream_ptr(stream))
+
+
+def test_quant_e4m3(x, stream=None):
+    """Row quantization of the E4M3 variant: (codes [rows, K] uint8, scales [rows] fp32)."""
+    import torch
+    rows, K = x.shape
+    q = torch.empty(rows, K, dtype=torch.uint8, device=x.device)
+    s = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _check(lib().albert_test_quant_e4m3(_ptr(x), rows, K, _ptr(q), _ptr(s), _stream_ptr(stream)),
+           "albert_test_quant_e4m3")
+    return q, s
 
 
 def test_attention(qkv, cu_seqlens, max_len: int, ctx, fp32: bool = False, legacy: bool = False,

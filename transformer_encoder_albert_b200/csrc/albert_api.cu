@@ -24,12 +24,12 @@ namespace {
 
 enum ProfClass {
     kProfPrep = 0, kProfEmbed, kProfGemmIn, kProfGemmQKV, kProfAttention, kProfGemmWoLN,
-    kProfGemmW1Gelu, kProfGemmW2LN, kProfGemmOut, kProfOutput, kProfLayerNorm, kProfSmall, kProfClasses
+    kProfGemmW1Gelu, kProfGemmW2LN, kProfGemmOut, kProfOutput, kProfLayerNorm, kProfSmall, kProfQuant, kProfClasses
 };
 const char *kProfNames[kProfClasses] = {
     "prep", "embed_ln", "gemm_in_proj", "gemm_qkv", "attention", "gemm_out_proj_ln",
     "gemm_ffn_up_gelu", "gemm_ffn_down_ln", "gemm_final_proj", "output_rows", "layer_norm_f32",
-    "small_batch_forward"};
+    "small_batch_forward", "quant_e4m3"};
 
 constexpr int kEventPool = 16384;
 
@@ -55,6 +55,10 @@ struct albert_handle {
         void *wqkv = nullptr, *wo = nullptr, *w1 = nullptr, *w2 = nullptr;
         CUtensorMap tm_wqkv, tm_wo, tm_w1, tm_w2;
         float *s_1 = nullptr, *c_1 = nullptr, *bias_21 = nullptr;  // bf16: this group's LN1 folded
+        // ALBERT_FP8: E4M3 copies of the four layer matrices with per-row scales
+        uint8_t *q_wqkv = nullptr, *q_wo = nullptr, *q_w1 = nullptr, *q_w2 = nullptr;
+        float *s_wqkv = nullptr, *s_wo = nullptr, *s_w1 = nullptr, *s_w2 = nullptr;
+        CUtensorMap tq_wqkv, tq_wo, tq_w1, tq_w2;
     };
     std::vector<Group> grp;
     // bf16, execution l >= 1: its group's Q|K|V and out-projection with the LN2
@@ -78,6 +82,12 @@ struct albert_handle {
 
     // out_layout 1: token-major staging of the output, transposed per sequence into `out`
     void *tout = nullptr;
+
+    // ALBERT_FP8: the A operand of the current layer GEMM as E4M3 codes with row
+    // scales (one buffer reused by every GEMM), seen as [rows, 768] and [rows, 2048]
+    uint8_t *qA = nullptr;
+    float *sA = nullptr;
+    CUtensorMap tq_A768, tq_A2048;
 
     // host-buffer staging
     int64_t *st_ids = nullptr;
@@ -169,7 +179,7 @@ int check_config(const albert_config *c) {
     if (c->n_exec < 0 || c->n_groups < 1 || c->n_groups > (c->n_exec > 0 ? c->n_exec : 1)) return ALBERT_ERR_CONFIG;
     if (c->max_pos < 1 || c->max_pos > kMaxPos || c->vocab < 1 || c->n_types < 1) return ALBERT_ERR_CONFIG;
     if (c->out_dim != 0 && c->out_dim != 512) return ALBERT_ERR_CONFIG;
-    if (c->dtype != ALBERT_BF16 && c->dtype != ALBERT_FP32) return ALBERT_ERR_CONFIG;
+    if (c->dtype != ALBERT_BF16 && c->dtype != ALBERT_FP32 && c->dtype != ALBERT_FP8) return ALBERT_ERR_CONFIG;
     if (c->max_tokens < 1 || c->max_tokens > (1 << 24)) return ALBERT_ERR_CONFIG;
     if (c->pack != 0 && c->pack != 1) return ALBERT_ERR_CONFIG;
     if (c->out_layout != 0 && c->out_layout != 1) return ALBERT_ERR_CONFIG;
@@ -287,14 +297,15 @@ GemmF32Args f32_args(albert_handle *h, const void *A, const void *W, const float
 
 // Everything after the prep kernel; `padded_api` selects zero-filled padding rows.
 int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, int nseq, int T,
-               int max_len, void *out, int padded_api) {
+               int max_len, void *out, int padded_api, const float *emb_in = nullptr) {
     const albert_config &c = h->cfg;
     const int out_rows = padded_api ? nseq * T : c.max_tokens;
     // out_layout 1: the final stage writes token-major rows to the staging buffer,
     // which the last kernel transposes per sequence into the caller's output
     void *const user_out = out;
     if (padded_api && c.out_layout == 1) out = h->tout;
-    const bool bf = c.dtype == ALBERT_BF16;
+    const bool bf = c.dtype != ALBERT_FP32;  // bf16 activations (ALBERT_BF16 and ALBERT_FP8)
+    const bool f8 = c.dtype == ALBERT_FP8;
     EmbedArgs ea{};
     ea.ids = ids;
     ea.ids_padded = ids_padded;
@@ -317,6 +328,7 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
     ea.dst_padded = padded_api;
     ea.status = h->status;
     ea.trigger = bf ? 1 : 0;  // bf16: the input projection (PDL) follows; fp32: a plain launch
+    ea.emb_in = emb_in;
     LAUNCH(L, kProfEmbed, launch_embed(ea, L.s));
 
     const int D = out_width(h);
@@ -359,15 +371,30 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
         for (int l = 0; l < c.n_exec; ++l) {
             const auto &W = h->grp[group_of(c, l)];                  // this execution's weights
             const auto &Wp = h->grp[group_of(c, l > 0 ? l - 1 : 0)];  // the previous execution's (its LN2)
+            // ALBERT_FP8: a layer GEMM's A operand is first quantized per row (E4M3 codes
+            // and scales in qA / sA); the GEMM reads the codes and the weights' codes
+            auto e4m3_operand = [&](const void *A, int K, const float *ws, GemmArgs &ga) -> int {
+                LAUNCH(L, kProfQuant, launch_quant_rows_e4m3(static_cast<const bf16 *>(A), K, h->rows_cap, h->n_rows,
+                                                             h->qA, h->sA, h->status, L.s, true, true));
+                ga.e4m3 = 1;
+                ga.a_scale = h->sA;
+                ga.w_scale = ws;
+                return ALBERT_OK;
+            };
             // Q|K|V from the layer input: X for the first execution, else LN2(z2) folded
-            if (l == 0) {
-                rc = gemm_bf16(L, kProfGemmQKV, kEpiBias, h->tm_X, W.tm_wqkv, h->t32_QKV, h->t32_QKV,
-                               gemm_args(h, kQKV, kHidden, W.bqkv, nullptr, 0));
-            } else {
-                GemmArgs a = gemm_args(h, kQKV, kHidden, h->ex[l].c_qkv, nullptr, 0);
-                a.fold_s = h->ex[l].s_qkv;
-                a.in_stats = h->st2;
-                rc = gemm_bf16(L, kProfGemmQKV, kEpiLnIn, h->tm_Z, W.tm_wqkv, h->t32_QKV, h->t32_QKV, a);
+            {
+                GemmArgs a = gemm_args(h, kQKV, kHidden, l == 0 ? W.bqkv : h->ex[l].c_qkv, nullptr, 0);
+                if (l > 0) {
+                    a.fold_s = h->ex[l].s_qkv;
+                    a.in_stats = h->st2;
+                }
+                const int epi = l == 0 ? kEpiBias : kEpiLnIn;
+                if (f8) {
+                    if ((rc = e4m3_operand(l == 0 ? h->X : h->Z, kHidden, W.s_wqkv, a))) return rc;
+                    rc = gemm_bf16(L, kProfGemmQKV, epi, h->tq_A768, W.tq_wqkv, h->t32_QKV, h->t32_QKV, a);
+                } else {
+                    rc = gemm_bf16(L, kProfGemmQKV, epi, l == 0 ? h->tm_X : h->tm_Z, W.tm_wqkv, h->t32_QKV, h->t32_QKV, a);
+                }
             }
             if (rc) return rc;
             if (max_len <= kAttnTcMaxLen) {
@@ -389,20 +416,28 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
             a.res_g = Wp.ln2_g;
             a.out_g = W.ln1_g;
             a.out_stats = h->st1;
-            if ((rc = gemm_bf16(L, kProfGemmWoLN, kEpiResStats, h->tm_C, W.tm_wo, h->t32_X1, l == 0 ? h->t32_X : h->t32_Z, a)))
+            if (f8 && (rc = e4m3_operand(h->C, kHidden, W.s_wo, a))) return rc;
+            if ((rc = gemm_bf16(L, kProfGemmWoLN, kEpiResStats, f8 ? h->tq_A768 : h->tm_C, f8 ? W.tq_wo : W.tm_wo,
+                                h->t32_X1, l == 0 ? h->t32_X : h->t32_Z, a)))
                 return rc;
             // H = GELU(LN1(z1) W1^T + b1)
             a = gemm_args(h, kFfn, kHidden, W.c_1, nullptr, 0);
             a.fold_s = W.s_1;
             a.in_stats = h->st1;
-            if ((rc = gemm_bf16(L, kProfGemmW1Gelu, kEpiLnInGelu, h->tm_X1, W.tm_w1, h->t32_H, h->t32_H, a))) return rc;
+            if (f8 && (rc = e4m3_operand(h->X1, kHidden, W.s_w1, a))) return rc;
+            if ((rc = gemm_bf16(L, kProfGemmW1Gelu, kEpiLnInGelu, f8 ? h->tq_A768 : h->tm_X1, f8 ? W.tq_w1 : W.tm_w1,
+                                h->t32_H, h->t32_H, a)))
+                return rc;
             // z2 = H W2^T + b2 + LN1(z1) -> Z = z2 * gamma2, st2
             a = gemm_args(h, kHidden, kFfn, W.bias_21, nullptr, 0);
             a.res_stats = h->st1;
             a.res_g = W.ln1_g;
             a.out_g = W.ln2_g;
             a.out_stats = h->st2;
-            if ((rc = gemm_bf16(L, kProfGemmW2LN, kEpiResStats, h->tm_H, W.tm_w2, h->t32_Z, h->t32_X1, a))) return rc;
+            if (f8 && (rc = e4m3_operand(h->H, kFfn, W.s_w2, a))) return rc;
+            if ((rc = gemm_bf16(L, kProfGemmW2LN, kEpiResStats, f8 ? h->tq_A2048 : h->tm_H, f8 ? W.tq_w2 : W.tm_w2,
+                                h->t32_Z, h->t32_X1, a)))
+                return rc;
         }
         if (c.out_dim > 0) {
             // the final projection is followed by zero_pad only in the padded API
@@ -467,7 +502,7 @@ int copy_param(float *dst, const float *src, size_t n, cudaStream_t s) {
 
 int copy_matrix(albert_handle *h, void *dst, const float *src, size_t n, cudaStream_t s) {
     if (!src) return ALBERT_ERR_NULL;
-    if (h->cfg.dtype == ALBERT_BF16) {
+    if (h->cfg.dtype != ALBERT_FP32) {
         TRY(launch_f32_to_bf16(src, static_cast<bf16 *>(dst), n, s));
     } else {
         TRY(cudaMemcpyAsync(dst, src, n * sizeof(float), cudaMemcpyDeviceToDevice, s));
@@ -482,7 +517,8 @@ int create_impl(albert_handle *h, const albert_weights *w) {
     h->rows_cap = (c.max_tokens + 127) / 128 * 128;
     h->seq_cap = c.max_tokens;
     const size_t R = h->rows_cap;
-    const bool bf = c.dtype == ALBERT_BF16;
+    const bool bf = c.dtype != ALBERT_FP32;  // bf16 activations (ALBERT_BF16 and ALBERT_FP8)
+    const bool f8 = c.dtype == ALBERT_FP8;
     const size_t eb = elem_bytes(h);
     int rc;
     cudaStream_t s = nullptr;
@@ -575,9 +611,33 @@ int create_impl(albert_handle *h, const albert_weights *w) {
         const size_t nf = G * (seg(kFfn) * 2 + seg(kHidden)) + (size_t)NX * (2 * seg(kQKV) + seg(kHidden)) + 2 * seg(O);
         if ((rc = dev_alloc(h, (void **)&h->fold, nf * sizeof(float)))) return rc;
         float *f = h->fold;
+        if (f8) {
+            // E4M3 copies of the layer matrices (quantized from their bf16 copies) and the
+            // A-operand buffer; the folded LayerNorm constants of these GEMMs are taken
+            // from the E4M3 weights, so that the mean correction matches the product
+            for (auto &gp : h->grp) {
+                struct { uint8_t **q; float **sc; const void *w; int N, K; } mats[4] = {
+                    {&gp.q_wqkv, &gp.s_wqkv, gp.wqkv, kQKV, kHidden}, {&gp.q_wo, &gp.s_wo, gp.wo, kHidden, kHidden},
+                    {&gp.q_w1, &gp.s_w1, gp.w1, kFfn, kHidden}, {&gp.q_w2, &gp.s_w2, gp.w2, kHidden, kFfn}};
+                for (auto &m : mats) {
+                    if ((rc = dev_alloc(h, (void **)m.q, (size_t)m.N * m.K))) return rc;
+                    if ((rc = dev_alloc(h, (void **)m.sc, (size_t)m.N * sizeof(float)))) return rc;
+                    TRY(launch_quant_rows_e4m3(static_cast<const bf16 *>(m.w), m.K, m.N, nullptr, *m.q, *m.sc, nullptr,
+                                               s, false, false));
+                }
+            }
+            if ((rc = dev_alloc(h, (void **)&h->qA, R * kFfn))) return rc;
+            if ((rc = dev_alloc(h, (void **)&h->sA, R * sizeof(float)))) return rc;
+            TRY(cudaMemsetAsync(h->qA, 0, R * kFfn, s));
+            TRY(cudaMemsetAsync(h->sA, 0, R * sizeof(float), s));
+        }
         for (auto &gp : h->grp) {
             gp.s_1 = f; f += seg(kFfn); gp.c_1 = f; f += seg(kFfn); gp.bias_21 = f; f += seg(kHidden);
-            TRY(launch_fold_ln(static_cast<const bf16 *>(gp.w1), kFfn, kHidden, gp.ln1_g, gp.ln1_b, gp.b1, gp.s_1, gp.c_1, s));
+            if (f8)
+                TRY(launch_fold_ln_e4m3(gp.q_w1, gp.s_w1, kFfn, kHidden, gp.ln1_g, gp.ln1_b, gp.b1, gp.s_1, gp.c_1, s));
+            else
+                TRY(launch_fold_ln(static_cast<const bf16 *>(gp.w1), kFfn, kHidden, gp.ln1_g, gp.ln1_b, gp.b1, gp.s_1,
+                                   gp.c_1, s));
             TRY(launch_vec_add(gp.b2, gp.ln1_b, gp.bias_21, kHidden, s));
         }
         h->ex.assign(NX, albert_handle::Exec{});
@@ -585,8 +645,12 @@ int create_impl(albert_handle *h, const albert_weights *w) {
             auto &e = h->ex[l];
             const auto &cur = h->grp[group_of(c, l)], &prev = h->grp[group_of(c, l - 1)];
             e.s_qkv = f; f += seg(kQKV); e.c_qkv = f; f += seg(kQKV); e.bias_o2 = f; f += seg(kHidden);
-            TRY(launch_fold_ln(static_cast<const bf16 *>(cur.wqkv), kQKV, kHidden, prev.ln2_g, prev.ln2_b, cur.bqkv,
-                               e.s_qkv, e.c_qkv, s));
+            if (f8)
+                TRY(launch_fold_ln_e4m3(cur.q_wqkv, cur.s_wqkv, kQKV, kHidden, prev.ln2_g, prev.ln2_b, cur.bqkv,
+                                        e.s_qkv, e.c_qkv, s));
+            else
+                TRY(launch_fold_ln(static_cast<const bf16 *>(cur.wqkv), kQKV, kHidden, prev.ln2_g, prev.ln2_b, cur.bqkv,
+                                   e.s_qkv, e.c_qkv, s));
             TRY(launch_vec_add(cur.bo, prev.ln2_b, e.bias_o2, kHidden, s));
         }
         h->s_out = f; f += seg(O); h->c_out = f;
@@ -630,8 +694,19 @@ int create_impl(albert_handle *h, const albert_weights *w) {
                 make_tmap_bf16(&gp.tm_w1, gp.w1, kFfn, kHidden, gemm::B_BOX) ||
                 make_tmap_bf16(&gp.tm_w2, gp.w2, kHidden, kFfn, gemm::B_BOX))
                 return ALBERT_ERR_CUDA;
-        // the small-batch kernel: one weight set, at least one execution
-        if (c.n_groups == 1 && c.n_exec >= 1) {
+        if (f8) {
+            if (make_tmap_e4m3(&h->tq_A768, h->qA, R, kHidden, gemm::BM) ||
+                make_tmap_e4m3(&h->tq_A2048, h->qA, R, kFfn, gemm::BM))
+                return ALBERT_ERR_CUDA;
+            for (auto &gp : h->grp)
+                if (make_tmap_e4m3(&gp.tq_wqkv, gp.q_wqkv, kQKV, kHidden, gemm::B_BOX) ||
+                    make_tmap_e4m3(&gp.tq_wo, gp.q_wo, kHidden, kHidden, gemm::B_BOX) ||
+                    make_tmap_e4m3(&gp.tq_w1, gp.q_w1, kFfn, kHidden, gemm::B_BOX) ||
+                    make_tmap_e4m3(&gp.tq_w2, gp.q_w2, kHidden, kFfn, gemm::B_BOX))
+                    return ALBERT_ERR_CUDA;
+        }
+        // the small-batch kernel: bf16, one weight set, at least one execution
+        if (!f8 && c.n_groups == 1 && c.n_exec >= 1) {
             const auto &gp = h->grp[0];
             if ((rc = dev_alloc(h, (void **)&h->sst1, kSmallMaxRows * kSmallParts * sizeof(float2)))) return rc;
             if ((rc = dev_alloc(h, (void **)&h->sst2, kSmallMaxRows * kSmallParts * sizeof(float2)))) return rc;
@@ -721,6 +796,20 @@ int albert_forward_varlen(albert_handle *h, const int64_t *ids, const int32_t *c
     LAUNCH(L, kProfPrep, launch_prep_varlen(cu_seqlens, nseq, max_len, h->cfg.max_tokens, h->seq_start, h->seq_len,
                                             h->n_rows, h->status, s, true));
     return run_layers(h, L, ids, 0, nseq, 0, max_len, out, 0);
+}
+
+int albert_forward_embedded(albert_handle *h, const float *emb, const int32_t *cu_seqlens, int nseq, int max_len,
+                            void *out, void *stream) {
+    if (!h || !emb || !cu_seqlens || !out) return ALBERT_ERR_NULL;
+    if (nseq < 1 || nseq > h->seq_cap || max_len < 1 || max_len > h->cfg.max_pos) return ALBERT_ERR_SHAPE;
+    if (h->cfg.out_layout != 0) return ALBERT_ERR_CONFIG;
+    if (reinterpret_cast<uintptr_t>(emb) & 15) return ALBERT_ERR_CONFIG;  // rows are read as float4
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    h->last_launches = 0;
+    Launch L{h, s};
+    LAUNCH(L, kProfPrep, launch_prep_varlen(cu_seqlens, nseq, max_len, h->cfg.max_tokens, h->seq_start, h->seq_len,
+                                            h->n_rows, h->status, s, true));
+    return run_layers(h, L, nullptr, 0, nseq, 0, max_len, out, 0, emb);
 }
 
 int albert_forward_host(albert_handle *h, const int64_t *ids_host, const uint8_t *mask_host, int B, int T,
@@ -821,7 +910,7 @@ void albert_destroy(albert_handle *h) {
 
 int albert_launches_per_forward(const albert_handle *h, int padded_api) {
     if (!h) return -1;
-    const int per_layer = h->cfg.dtype == ALBERT_BF16 ? 5 : 7;
+    const int per_layer = h->cfg.dtype == ALBERT_BF16 ? 5 : h->cfg.dtype == ALBERT_FP8 ? 9 : 7;
     return 1 /*prep*/ + 1 /*embed*/ + 1 /*in proj*/ + per_layer * h->cfg.n_exec + 1 /*final or scatter*/ +
            (padded_api ? 1 : 0);
 }
@@ -882,7 +971,7 @@ int albert_test_stall(albert_handle *h, int class_mask) {
                                   (1u << kProfGemmW1Gelu) | (1u << kProfGemmW2LN) | (1u << kProfGemmOut) |
                                   (1u << kProfSmall);
     if ((unsigned)class_mask & ~gemm_classes) return ALBERT_ERR_CONFIG;
-    if (class_mask && h->cfg.dtype != ALBERT_BF16) return ALBERT_ERR_CONFIG;  // the fp32 kernels never wait
+    if (class_mask && h->cfg.dtype == ALBERT_FP32) return ALBERT_ERR_CONFIG;  // the fp32 kernels never wait
     h->stall_mask = (unsigned)class_mask;
     return ALBERT_OK;
 }
@@ -903,10 +992,12 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
                      const float *ln_b, float eps, const int32_t *row_dst, void *Y, int M, int N, int K,
                      int epi, void *stream) {
     if (!A || !W || !bias || !Y) return ALBERT_ERR_NULL;
+    const bool e4m3 = (epi & ALBERT_GEMM_E4M3) != 0;
     if (M < 1 || N < gemm::BN || N % gemm::BN || K < gemm::BK || K % gemm::BK) return ALBERT_ERR_SHAPE;
+    if (e4m3 && (K % 256 || K > 2048 || N % 8)) return ALBERT_ERR_SHAPE;  // the row quantizer's limits
     const int variant = (epi & ALBERT_GEMM_SINGLE_CTA) ? kGemmSingle : (epi & ALBERT_GEMM_CTA_PAIR) ? kGemmPair : kGemmAuto;
     if ((epi & ALBERT_GEMM_SINGLE_CTA) && (epi & ALBERT_GEMM_CTA_PAIR)) return ALBERT_ERR_CONFIG;
-    epi &= ~(ALBERT_GEMM_SINGLE_CTA | ALBERT_GEMM_CTA_PAIR);
+    epi &= ~(ALBERT_GEMM_SINGLE_CTA | ALBERT_GEMM_CTA_PAIR | ALBERT_GEMM_E4M3);
     if (epi < 0 || epi > 3) return ALBERT_ERR_CONFIG;
     if (epi == 2 && (!R || !ln_g || !ln_b || N != gemm::LN_N)) return ALBERT_ERR_CONFIG;
     if (epi == 3 && !row_dst) return ALBERT_ERR_NULL;
@@ -929,8 +1020,20 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
         cudaFree(zg);
         return ALBERT_ERR_ALLOC;
     }
+    // E4M3: both operands quantized per row into temporaries first
+    uint8_t *qa = nullptr, *qw = nullptr;
+    float *sa = nullptr, *sw = nullptr;
+    if (e4m3) {
+        if (cudaMalloc(&qa, (size_t)rows_cap * K) != cudaSuccess || cudaMalloc(&qw, (size_t)N * K) != cudaSuccess ||
+            cudaMalloc(&sa, (size_t)rows_cap * sizeof(float)) != cudaSuccess ||
+            cudaMalloc(&sw, (size_t)N * sizeof(float)) != cudaSuccess) {
+            cudaFree(ints); cudaFree(zg); cudaFree(stats); cudaFree(qa); cudaFree(qw); cudaFree(sa);
+            return ALBERT_ERR_ALLOC;
+        }
+    }
     CUtensorMap ta, tb, to, tr;
-    int bad = make_tmap_bf16(&ta, A, M, K, gemm::BM) || make_tmap_bf16(&tb, W, N, K, gemm::B_BOX);
+    int bad = e4m3 ? (make_tmap_e4m3(&ta, qa, M, K, gemm::BM) || make_tmap_e4m3(&tb, qw, N, K, gemm::B_BOX))
+                   : (make_tmap_bf16(&ta, A, M, K, gemm::BM) || make_tmap_bf16(&tb, W, N, K, gemm::B_BOX));
     if (epi == 2) bad = bad || make_tmap_bf16_tile32(&to, zg, rows_cap, N) || make_tmap_bf16_tile32(&tr, R, M, N);
     else if (epi != 3) bad = bad || make_tmap_bf16_tile32(&to, Y, M, N);
     if (epi == 3) to = ta;
@@ -942,6 +1045,14 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
     a.N = N; a.K = K; a.rows_cap = rows_cap; a.n_rows = ints; a.bias = bias; a.eps = eps;
     a.out_g = ln_g; a.out_stats = stats; a.out = static_cast<bf16 *>(Y); a.ld_out = N;
     a.row_dst = row_dst; a.status = ints + 1;
+    a.e4m3 = e4m3 ? 1 : 0; a.a_scale = sa; a.w_scale = sw;
+    if (e == cudaSuccess && e4m3) {
+        e = cudaMemsetAsync(sa, 0, (size_t)rows_cap * sizeof(float), s);
+        if (e == cudaSuccess)
+            e = launch_quant_rows_e4m3(static_cast<const bf16 *>(A), K, M, nullptr, qa, sa, nullptr, s, false, false);
+        if (e == cudaSuccess)
+            e = launch_quant_rows_e4m3(static_cast<const bf16 *>(W), K, N, nullptr, qw, sw, nullptr, s, false, false);
+    }
     // follows a copy in the stream: a plain launch
     if (e == cudaSuccess) e = launch_gemm(kepi, ta, tb, to, tr, a, grid, s, variant, false);
     if (e == cudaSuccess && epi == 2)
@@ -953,7 +1064,21 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
     cudaFree(ints);
     if (zg) cudaFree(zg);
     if (stats) cudaFree(stats);
+    if (qa) cudaFree(qa);
+    if (qw) cudaFree(qw);
+    if (sa) cudaFree(sa);
+    if (sw) cudaFree(sw);
     return e == cudaSuccess ? st : ALBERT_ERR_CUDA;
+}
+
+int albert_test_quant_e4m3(const void *x, int rows, int K, void *q, float *scale, void *stream) {
+    if (!x || !q || !scale) return ALBERT_ERR_NULL;
+    if (rows < 1 || K < 256 || K > 2048 || K % 256) return ALBERT_ERR_SHAPE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TRY(launch_quant_rows_e4m3(static_cast<const bf16 *>(x), K, rows, nullptr, static_cast<uint8_t *>(q), scale,
+                               nullptr, s, false, false));
+    TRY(cudaStreamSynchronize(s));
+    return ALBERT_OK;
 }
 
 int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, int max_len, void *ctx, int dtype,

@@ -14,11 +14,14 @@
 //                 one, its V tile into the other.  A Q/K stage is free again
 //                 as soon as the S product has read it, so Q/K loads run well
 //                 ahead; a V stage lives until the O product;
-//   warp 1      : tcgen05.mma issuer, an event loop that issues whichever is
-//                 ready: S = Q K^T (M=128, N=128 or 64, K=64) into a TMEM
-//                 buffer, or O = P V (M=128, N=64, K = L rounded up to 16) with
-//                 P read from TMEM and V from shared memory as an MN-major
-//                 operand;
+//   warp 1      : tcgen05.mma issuer of the score products S = Q K^T (M=128,
+//                 N=128 or 64, K=64) into a TMEM buffer, item after item;
+//   warp 14     : tcgen05.mma issuer of the output products O = P V (M=128,
+//                 N=64, K = L rounded up to 16) with P read from TMEM and V
+//                 from shared memory as an MN-major operand.  Two issuing
+//                 threads: the cost of issuing, committing and polling on one
+//                 thread (about as much per MMA as the MMA itself) no longer
+//                 serializes the two products of successive items;
 //   warps 2..9  : two softmax groups of 4 warps (items alternate between
 //                 them): each thread owns one query row, reads its scores from
 //                 TMEM, applies the mask and a max-subtracted softmax in
@@ -44,7 +47,8 @@ constexpr int TILE = TROWS * 128;              // 128 rows x 64 bf16 = 16 KB
 constexpr int NQK = 4;                         // Q/K stages (2 tiles each)
 constexpr int NV = 4;                          // V stages (1 tile each)
 constexpr int NBUF = 4;                        // TMEM item buffers (128 columns each)
-constexpr int ATC_THREADS = 32 * 14;
+constexpr int ATC_THREADS = 32 * 15;
+constexpr int ATC_O_WARP = 14;                 // issuer of the O = P V products
 constexpr int ATC_SMEM = 1024 + (2 * NQK + NV) * TILE + NBUF * TROWS * 4 + 512;
 constexpr uint32_t TM_O = 64;                  // O's first column within an item buffer
 // Item n uses Q/K stage, V stage and TMEM buffer n % 4 alike, so a Q/K stage is
@@ -58,7 +62,7 @@ struct AttSmem {
     uint64_t *qk_full;                         // [NQK]
     uint64_t *v_full;                          // [NV]
     uint64_t *s_full, *p_full, *o_full, *o_empty;  // [NBUF]
-    uint64_t *drain;
+    uint64_t *drain, *drain_o;                 // each issuer's products complete
     uint32_t *tmem_slot;
     volatile int *abort_flag;
     int *misc;
@@ -80,7 +84,8 @@ __device__ __forceinline__ AttSmem att_carve(uint8_t *raw) {
     s.o_full = s.s_full + 2 * NBUF;
     s.o_empty = s.s_full + 3 * NBUF;
     s.drain = s.s_full + 4 * NBUF;
-    uint32_t *u = reinterpret_cast<uint32_t *>(s.drain + 1);
+    s.drain_o = s.drain + 1;
+    uint32_t *u = reinterpret_cast<uint32_t *>(s.drain + 2);
     s.tmem_slot = u;
     s.abort_flag = reinterpret_cast<volatile int *>(u + 1);
     s.misc = reinterpret_cast<int *>(u + 2);
@@ -113,6 +118,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
             mbar_init(smem_u32(&sm.o_empty[i]), 4);
         }
         mbar_init(smem_u32(sm.drain), 1);
+        mbar_init(smem_u32(sm.drain_o), 1);
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -195,65 +201,53 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
             }
         }
     } else if (warp == 1) {
-        // -------------------------------------------------------- MMA issuer --
-        // Issues S(next) and O(next) products as soon as each is ready, so an
-        // output product never queues behind the next item's loads.
+        // --------------------------------------------- score-product issuer --
+        // S of item n goes into TMEM buffer n % 4 once its Q/K stage is full and
+        // the output group has read O of item n - 4 from that buffer.
         if (lane == 0) {
             const uint32_t idesc_s128 = idesc_bf16_f32(TROWS, TROWS);
             const uint32_t idesc_s64 = idesc_bf16_f32(TROWS, 64);
-            const uint32_t idesc_o = idesc_bf16_f32(TROWS, kHeadDim) | (1u << 16);  // B (= V) MN-major
-            int ns = 0, no = 0;  // next S product, next O product
-            unsigned long long t_idle = 0;
-            unsigned polls = 0;
-            while (no < n_items) {
-                bool progress = false;
-                if (no < ns) {
-                    const int tb = no % NBUF, st = no % NV;
-                    if (mbar_test(smem_u32(&sm.p_full[tb]), (no / NBUF) & 1) &&
-                        mbar_test(smem_u32(&sm.v_full[st]), (no / NV) & 1)) {
-                        tc_fence_after();
-                        const int L = sm.v_len[st];
-                        const int ksteps = (L + 15) >> 4;
-                        const uint32_t vbase = smem_u32(sm.v + st * TILE);
-                        const uint32_t buf = tmem_base + tb * TROWS;
-                        for (int kk = 0; kk < ksteps; ++kk) {
-                            // P: 16 keys = 8 packed TMEM columns; V: 16 keys = 16 rows of 128 B
-                            umma_bf16_ts(buf + TM_O, buf + kk * 8, sw128_kmajor_desc(vbase + kk * 2048), idesc_o,
-                                         kk != 0);
-                        }
-                        umma_commit(smem_u32(&sm.o_full[tb]));  // also frees V stage st (== tb)
-                        ++no;
-                        progress = true;
-                    }
-                }
-                if (ns < n_items && ns < no + NBUF) {
-                    const int tb = ns % NBUF, st = ns % NQK;
-                    // the buffer is free once the output group has read item ns - NBUF
-                    if (mbar_test(smem_u32(&sm.qk_full[st]), (ns / NQK) & 1) &&
-                        mbar_test(smem_u32(&sm.o_empty[tb]), ((ns / NBUF) & 1) ^ 1)) {
-                        tc_fence_after();
-                        const int L = sm.qk_len[st];
-                        const uint32_t q = smem_u32(sm.qk + st * 2 * TILE), k = q + TILE;
+            for (int ns = 0; ns < n_items; ++ns) {
+                const int tb = ns % NBUF, st = ns % NQK;
+                if (!mbar_wait(smem_u32(&sm.qk_full[st]), (ns / NQK) & 1, sm.abort_flag) ||
+                    !mbar_wait(smem_u32(&sm.o_empty[tb]), ((ns / NBUF) & 1) ^ 1, sm.abort_flag))
+                    break;
+                tc_fence_after();
+                const int L = sm.qk_len[st];
+                const uint32_t q = smem_u32(sm.qk + st * 2 * TILE), k = q + TILE;
 #pragma unroll
-                        for (int kk = 0; kk < kHeadDim / 16; ++kk)
-                            umma_bf16(tmem_base + tb * TROWS, sw128_kmajor_desc(q + kk * 32),
-                                      sw128_kmajor_desc(k + kk * 32), L <= 64 ? idesc_s64 : idesc_s128, kk != 0);
-                        umma_commit(smem_u32(&sm.s_full[tb]));  // also frees Q/K stage st (== tb)
-                        ++ns;
-                        progress = true;
-                    }
-                }
-                if (progress) {
-                    t_idle = 0;
-                } else if ((++polls & 255) == 0) {  // the timer read is slow: not on every poll
-                    if (*sm.abort_flag) break;
-                    const unsigned long long now = globaltimer_ns();
-                    if (t_idle == 0) t_idle = now;
-                    else if (now - t_idle > wait_limit()) { *sm.abort_flag = 1; break; }
-                }
+                for (int kk = 0; kk < kHeadDim / 16; ++kk)
+                    umma_bf16(tmem_base + tb * TROWS, sw128_kmajor_desc(q + kk * 32), sw128_kmajor_desc(k + kk * 32),
+                              L <= 64 ? idesc_s64 : idesc_s128, kk != 0);
+                umma_commit(smem_u32(&sm.s_full[tb]));  // also frees Q/K stage st (== tb)
             }
             umma_commit(smem_u32(sm.drain));
             mbar_wait_drain(smem_u32(sm.drain), 0);
+        }
+    } else if (warp == ATC_O_WARP) {
+        // -------------------------------------------- output-product issuer --
+        // O of item n once the softmax has written P over its scores (p_full, which
+        // also means every score of the buffer has been read) and its V stage is full.
+        if (lane == 0) {
+            const uint32_t idesc_o = idesc_bf16_f32(TROWS, kHeadDim) | (1u << 16);  // B (= V) MN-major
+            for (int no = 0; no < n_items; ++no) {
+                const int tb = no % NBUF, st = no % NV;
+                if (!mbar_wait(smem_u32(&sm.p_full[tb]), (no / NBUF) & 1, sm.abort_flag) ||
+                    !mbar_wait(smem_u32(&sm.v_full[st]), (no / NV) & 1, sm.abort_flag))
+                    break;
+                tc_fence_after();
+                const int L = sm.v_len[st];
+                const int ksteps = (L + 15) >> 4;
+                const uint32_t vbase = smem_u32(sm.v + st * TILE);
+                const uint32_t buf = tmem_base + tb * TROWS;
+                for (int kk = 0; kk < ksteps; ++kk) {
+                    // P: 16 keys = 8 packed TMEM columns; V: 16 keys = 16 rows of 128 B
+                    umma_bf16_ts(buf + TM_O, buf + kk * 8, sw128_kmajor_desc(vbase + kk * 2048), idesc_o, kk != 0);
+                }
+                umma_commit(smem_u32(&sm.o_full[tb]));  // also frees V stage st (== tb)
+            }
+            umma_commit(smem_u32(sm.drain_o));
+            mbar_wait_drain(smem_u32(sm.drain_o), 0);
         }
     } else if (warp < 10) {
         // ------------------------------------------------------ softmax warps --

@@ -40,7 +40,10 @@
 // depend on scheduling.
 //
 // Roles inside a CTA (192 threads): warp 0 lane 0 issues TMA loads into a
-// 4-stage ring, warp 1 lane 0 allocates TMEM and issues tcgen05.mma, warps
+// 3-stage ring of 64 KB stages (a stage carries up to four 64-wide K blocks of
+// both operands, so a 64-column tile with K = 768 and at most 64 rows has all
+// of K in flight at once: the phases are bound by load latency, not
+// bandwidth), warp 1 lane 0 allocates TMEM and issues tcgen05.mma, warps
 // 2..5 (one per TMEM lane quadrant, one thread per tile row) run epilogues and
 // the softmax; every warp takes rows of the reduce phase.  Every wait is
 // bounded (mbarriers and the grid barrier alike); on expiry the kernel records
@@ -53,10 +56,10 @@ namespace albert {
 namespace {
 
 constexpr int SB_THREADS = 192;
-constexpr int SB_NS = 4;                      // ring stages
+constexpr int SB_NS = 3;                      // ring stages
 constexpr int SB_BOX = 64 * 64 * 2;           // one {64 cols, 64 rows} bf16 box, 128-byte swizzle: 8 KB
-constexpr int SB_A_BYTES = 2 * SB_BOX;        // A: up to 128 rows
-constexpr int SB_B_BYTES = 4 * SB_BOX;        // B: up to 256 rows
+constexpr int SB_A_BYTES = 4 * SB_BOX;        // A: up to four 64-row K blocks (two of 128 rows)
+constexpr int SB_B_BYTES = 4 * SB_BOX;        // B: up to four 64-row K blocks, or one of 256 rows
 constexpr int SB_H_BYTES = 2 * SB_BOX;        // FFN hidden chunk, 128 rows x 64 bf16
 constexpr int SB_SMEM = 1024 + SB_NS * (SB_A_BYTES + SB_B_BYTES) + SB_H_BYTES + 128 * 4 + 512;
 static_assert(SB_SMEM <= 232448, "shared memory per CTA");
@@ -166,11 +169,12 @@ __device__ __forceinline__ int phase_jobs(int ph, const SmallFwdArgs &p) {
 }
 
 // Loads of one job, in the order the MMA issuer consumes them.  Each load step
-// fills one ring stage: a 64-wide K block of A (a_boxes boxes of 64 rows) and
-// of B (b_boxes boxes of 64 rows); the FFN's second products load B only.
+// fills one ring stage with nk consecutive 64-wide K blocks; K block j holds
+// a_boxes boxes of 64 rows of A at j * a_boxes * 8 KB and b_boxes boxes of 64
+// rows of B at j * b_boxes * 8 KB.  The FFN's second products load B only.
 struct LoadStep {
     const CUtensorMap *ta, *tb;
-    int a_boxes, b_boxes;
+    int a_boxes, b_boxes, nk;
     int ax, ay, bx, by;       // coordinates of the first boxes (x = column, y = row)
 };
 
@@ -221,6 +225,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
     // an earlier kernel of this forward failed (or the row count is out of range): nothing to do
     const bool skip = sm.misc[1] != 0 || M < 1 || M > 128;
     const int a_boxes = M > 64 ? 2 : 1;
+    const int kb_step = M > 64 ? 2 : 4;  // 64-wide K blocks per ring stage in the GEMM phases
     const int n_phases = 1 + 5 * p.n_exec + 1;
 
     int epoch = 0;
@@ -244,12 +249,16 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
                 const int c = s * 64 + 2 * lane;
                 if (ph == kPhReduce) {
                     // z2 = sum of the FFN partials + (b2 + beta1) + rstd1 * x1 - rstd1 * mu1 * gamma1
+                    // every partial's load is issued before the first add (one round trip)
+                    float2 pv[SB_CHUNKS];
+#pragma unroll
+                    for (int j = 0; j < SB_CHUNKS; ++j)
+                        pv[j] = *reinterpret_cast<const float2 *>(p.part + ((size_t)j * 128 + r) * kHidden + c);
                     float ax = 0.f, ay = 0.f;
-#pragma unroll 4
+#pragma unroll
                     for (int j = 0; j < SB_CHUNKS; ++j) {
-                        const float2 v = *reinterpret_cast<const float2 *>(p.part + ((size_t)j * 128 + r) * kHidden + c);
-                        ax += v.x;
-                        ay += v.y;
+                        ax += pv[j].x;
+                        ay += pv[j].y;
                     }
                     float mu1, rstd1;
                     merge_parts(p.st1 + (size_t)r * SB_PARTS, p.eps, mu1, rstd1);
@@ -288,27 +297,26 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
             if (lane == 0) {
                 const uint64_t keep = policy_evict_last();  // weights: read by every execution
                 for (int job = p.withhold_loads ? njobs : blockIdx.x; job < njobs && ok; job += gridDim.x) {
-                    LoadStep st[16];  // at most 12 + 3 (FFN)
+                    LoadStep st[12];  // at most 6 + 3 (FFN)
                     int ns = 0;
                     if (ph == kPhIn) {
-                        for (int kb = 0; kb < kEmb / 64; ++kb)
-                            st[ns++] = {&p.tmE, &p.tmWin, a_boxes, 1, kb * 64, 0, kb * 64, job * 64};
-                    } else if (ph == kPhQKV || ph == kPhOut || ph == kPhFinal) {
-                        const CUtensorMap *ta = ph == kPhOut ? &p.tmC : (ph == kPhQKV && l == 0) ? &p.tmX : &p.tmZ;
-                        const CUtensorMap *tb = ph == kPhQKV ? &p.tmWqkv : ph == kPhOut ? &p.tmWo : &p.tmWout;
-                        for (int kb = 0; kb < kHidden / 64; ++kb)
-                            st[ns++] = {ta, tb, a_boxes, 1, kb * 64, 0, kb * 64, job * 64};
-                    } else if (ph == kPhFfn) {
-                        for (int kb = 0; kb < kHidden / 64; ++kb)
-                            st[ns++] = {&p.tmX1, &p.tmW1, a_boxes, 1, kb * 64, 0, kb * 64, job * 64};
-                        for (int nb = 0; nb < 3; ++nb)
-                            st[ns++] = {nullptr, &p.tmW2, 0, 4, 0, 0, job * 64, nb * 256};
+                        st[ns++] = {&p.tmE, &p.tmWin, a_boxes, 1, kEmb / 64, 0, 0, 0, job * 64};
+                    } else if (ph == kPhQKV || ph == kPhOut || ph == kPhFinal || ph == kPhFfn) {
+                        const CUtensorMap *ta = ph == kPhOut ? &p.tmC : ph == kPhFfn ? &p.tmX1
+                                                : (ph == kPhQKV && l == 0) ? &p.tmX : &p.tmZ;
+                        const CUtensorMap *tb = ph == kPhQKV ? &p.tmWqkv : ph == kPhOut ? &p.tmWo
+                                                : ph == kPhFfn ? &p.tmW1 : &p.tmWout;
+                        for (int kb = 0; kb < kHidden / 64; kb += kb_step)
+                            st[ns++] = {ta, tb, a_boxes, 1, kb_step, kb * 64, 0, kb * 64, job * 64};
+                        if (ph == kPhFfn)
+                            for (int nb = 0; nb < 3; ++nb)
+                                st[ns++] = {nullptr, &p.tmW2, 0, 4, 1, 0, 0, job * 64, nb * 256};
                     } else {  // attention: Q and K of (sequence, head), then V
                         const int b = job / kHeads, h = job % kHeads;
                         const int L = __ldg(p.seq_len + b), start = __ldg(p.seq_start + b);
                         const CUtensorMap *tq = L <= 64 ? &p.tmQKV64 : &p.tmQKV;
-                        st[ns++] = {tq, tq, 1, 1, h * kHeadDim, start, kHidden + h * kHeadDim, start};
-                        st[ns++] = {nullptr, tq, 0, 1, 0, 0, 2 * kHidden + h * kHeadDim, start};
+                        st[ns++] = {tq, tq, 1, 1, 1, h * kHeadDim, start, kHidden + h * kHeadDim, start};
+                        st[ns++] = {nullptr, tq, 0, 1, 1, 0, 0, 2 * kHidden + h * kHeadDim, start};
                     }
                     for (int i = 0; i < ns && ok; ++i, ++ring) {
                         const int s = ring % SB_NS;
@@ -321,15 +329,19 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
                         // attention boxes are 128 rows unless the sequence fits in 64
                         const uint32_t box_bytes = attn && d.tb == &p.tmQKV ? 2 * SB_BOX : SB_BOX;
                         const uint32_t fb = smem_u32(&sm.full[s]);
-                        mbar_arrive_expect_tx(fb, box_bytes * (uint32_t)(d.a_boxes + d.b_boxes));
+                        mbar_arrive_expect_tx(fb, box_bytes * (uint32_t)(d.nk * (d.a_boxes + d.b_boxes)));
                         const uint32_t a_dst = smem_u32(sm.a + s * SB_A_BYTES), b_dst = smem_u32(sm.b + s * SB_B_BYTES);
                         if (attn) {
                             if (d.a_boxes) tma_load_2d(a_dst, d.ta, fb, d.ax, d.ay);
                             tma_load_2d(b_dst, d.tb, fb, d.bx, d.by);
                         } else {
-                            for (int q = 0; q < d.a_boxes; ++q) tma_load_2d(a_dst + q * SB_BOX, d.ta, fb, d.ax, d.ay + 64 * q);
-                            for (int q = 0; q < d.b_boxes; ++q)
-                                tma_load_2d_hint(b_dst + q * SB_BOX, d.tb, fb, d.bx, d.by + 64 * q, keep);
+                            for (int j = 0; j < d.nk; ++j) {
+                                for (int q = 0; q < d.a_boxes; ++q)
+                                    tma_load_2d(a_dst + (j * d.a_boxes + q) * SB_BOX, d.ta, fb, d.ax + 64 * j, d.ay + 64 * q);
+                                for (int q = 0; q < d.b_boxes; ++q)
+                                    tma_load_2d_hint(b_dst + (j * d.b_boxes + q) * SB_BOX, d.tb, fb, d.bx + 64 * j,
+                                                     d.by + 64 * q, keep);
+                            }
                         }
                     }
                 }
@@ -379,17 +391,21 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
                         finish_unit();
                         continue;
                     }
-                    const int kblocks = ph == kPhIn ? kEmb / 64 : kHidden / 64;
+                    // one stage per kb_step K blocks (the in-projection's two in one stage)
+                    const int nsteps = ph == kPhIn ? 1 : (kHidden / 64) / kb_step;
+                    const int nk = ph == kPhIn ? kEmb / 64 : kb_step;
                     if (!wait_acc_free()) { ok = false; break; }
                     const uint32_t idesc = idesc_bf16_f32(128, 64);
-                    for (int kb = 0; kb < kblocks && ok; ++kb) {
+                    for (int stp = 0; stp < nsteps && ok; ++stp) {
                         uint32_t s;
                         if (!wait_stage(s)) { ok = false; break; }
                         const uint32_t a0 = smem_u32(sm.a + s * SB_A_BYTES), b0 = smem_u32(sm.b + s * SB_B_BYTES);
+                        for (int j = 0; j < nk; ++j) {
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_bf16(tmem_base, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), idesc,
-                                      (kb | kk) != 0);
+                            for (int kk = 0; kk < 4; ++kk)
+                                umma_bf16(tmem_base, sw128_kmajor_desc(a0 + j * a_boxes * SB_BOX + kk * 32),
+                                          sw128_kmajor_desc(b0 + j * SB_BOX + kk * 32), idesc, (stp | j | kk) != 0);
+                        }
                         umma_commit(smem_u32(&sm.empty[s]));
                         ++ring;
                     }

@@ -1,0 +1,157 @@
+// fp8.cu -- the FP8 (E4M3) variant's quantization and folded LayerNorm constants.
+//
+// The pages evaluate a quantized build of the encoder against its FP32 outputs
+// ("Kokoro-82M-encoder-hailo10h" model card, section "Eval results": per-sample
+// cosine and MSE on random post-embedding-LayerNorm inputs).  Here both
+// operands of the layer GEMMs are E4M3 with one fp32 scale per row along the
+// reduction dimension (per token for activations, per output channel for
+// weights), so the tcgen05 product (kind::f8f6f4) sums q_x q_w exactly in fp32
+// and the epilogue multiplies by s_x s_w:
+//   amax = max |x|,  s = amax / 448,  q = E4M3(fp32(x * (448 / amax)))
+// (one rounding of the fp32 product to E4M3, to nearest even, saturating; the
+// conversion is written out from the format's definition, so that the code is
+// an exact function of the fp32 value; a row of zeros has s = 0 and q = 0).
+// A row's scale needs the whole row, which the GEMM epilogues that produce the
+// activations do not have (their tiles are 256 columns wide), so activations
+// are quantized by a separate pass per GEMM: one warp per row.
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace albert {
+namespace {
+
+constexpr int Q_WARPS = 8;
+
+// fp32 -> E4M3 byte from the format's definition, one rounding: keep 3 mantissa
+// bits of a normal result (|y| >= 2^-6) with round to nearest, ties to even;
+// below 2^-6 the result is a multiple of 2^-9 (subnormal), rounded the same way;
+// magnitudes at or above 448 saturate to 448; the sign is kept (also on zero).
+__device__ __forceinline__ uint32_t f32_to_e4m3(float y) {
+    const uint32_t u = __float_as_uint(y);
+    const uint32_t sign = (u >> 24) & 0x80u;
+    const float ay = fabsf(y);
+    if (!(ay < 448.0f)) return sign | 0x7Eu;  // 448 = 1.75 * 2^8 (exponent field 15, mantissa 6)
+    const int e = (int)((u >> 23) & 0xFFu) - 127;
+    if (e >= -6) {
+        const uint32_t mant = u & 0x7FFFFFu;
+        uint32_t keep = mant >> 20;            // the 3 kept mantissa bits
+        const uint32_t rest = mant & 0xFFFFFu;  // the 20 dropped ones
+        if (rest > 0x80000u || (rest == 0x80000u && (keep & 1u))) ++keep;
+        uint32_t be = (uint32_t)(e + 7);       // biased E4M3 exponent, 1..15
+        if (keep == 8u) { keep = 0u; ++be; }
+        if (be > 15u || (be == 15u && keep == 7u)) return sign | 0x7Eu;
+        return sign | (be << 3) | keep;
+    }
+    // |y| < 2^-6: m * 2^-9 with m = round(|y| * 2^9) (exact scaling, then ties to even);
+    // m = 8 is the encoding of the smallest normal, 2^-6
+    return sign | (uint32_t)rintf(ay * 512.0f);
+}
+
+__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
+    return (uint16_t)(f32_to_e4m3(lo) | (f32_to_e4m3(hi) << 8));
+}
+
+// x [rows, K] bf16 -> q [rows, K] E4M3, scale [rows] fp32.  K is a multiple of
+// 256 and at most 2048: each lane holds K / 256 runs of 8 consecutive values.
+__global__ void __launch_bounds__(32 * Q_WARPS)
+quant_rows_e4m3_kernel(const bf16 *__restrict__ x, int K, int rows, const int *n_rows, uint8_t *__restrict__ q,
+                       float *__restrict__ scale, const int *status, int trigger) {
+    if (trigger) griddep_launch_dependents();
+    griddep_wait();
+    if (status && *reinterpret_cast<const volatile int *>(status) != 0) return;
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * Q_WARPS + (threadIdx.x >> 5);
+    const int nr = n_rows ? *reinterpret_cast<const volatile int *>(n_rows) : rows;
+    if (row >= nr || row >= rows) return;
+    const int runs = K >> 8;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)row * K);
+    uint4 v[8];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        if (i < runs) {
+            v[i] = src[i * 32 + lane];
+            const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = unpack_bf16x2(w[e]);
+                amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+        }
+    }
+    // non-negative floats order like their bit patterns
+    amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+    const bool nz = amax > 0.f;
+    const float inv = nz ? __fdiv_rn(448.0f, amax) : 0.f;
+    if (lane == 0) scale[row] = nz ? __fdiv_rn(amax, 448.0f) : 0.f;
+    uint2 *dst = reinterpret_cast<uint2 *>(q + (size_t)row * K);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        if (i < runs) {
+            const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+            uint16_t b[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = unpack_bf16x2(w[e]);
+                b[e] = cvt_e4m3x2(__fmul_rn(f.x, inv), __fmul_rn(f.y, inv));
+            }
+            dst[i * 32 + lane] = make_uint2((uint32_t)b[0] | ((uint32_t)b[1] << 16), (uint32_t)b[2] | ((uint32_t)b[3] << 16));
+        }
+    }
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint8_t b) {
+    // sign, 4 exponent bits (bias 7), 3 mantissa bits; no infinities; 0x7f / 0xff are NaN
+    const float sgn = (b & 0x80) ? -1.f : 1.f;
+    const int e = (b >> 3) & 15, m = b & 7;
+    if ((b & 0x7f) == 0x7f) return __int_as_float(0x7fc00000);
+    const float mag = e == 0 ? ldexpf((float)m, -9) : ldexpf((float)(8 + m), e - 10);
+    return sgn * mag;
+}
+
+// Folded LayerNorm constants of an E4M3 weight W_q [N, K] with row scales sw:
+// s_j = sw_j sum_k gamma_k q_jk,  c_j = sw_j sum_k beta_k q_jk + b_j (one warp per j).
+__global__ void fold_ln_e4m3_kernel(const uint8_t *__restrict__ Wq, const float *__restrict__ sw, int N, int K,
+                                    const float *__restrict__ gamma, const float *__restrict__ beta,
+                                    const float *__restrict__ b, float *s_out, float *c_out) {
+    const int j = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (j >= N) return;
+    const uint8_t *w = Wq + (size_t)j * K;
+    float s = 0.f, c = 0.f;
+    for (int k = lane; k < K; k += 32) {
+        const float x = e4m3_to_f32(w[k]);
+        s = fmaf(gamma[k], x, s);
+        c = fmaf(beta[k], x, c);
+    }
+    for (int o = 16; o; o >>= 1) {
+        s += __shfl_xor_sync(0xffffffffu, s, o);
+        c += __shfl_xor_sync(0xffffffffu, c, o);
+    }
+    if (lane == 0) {
+        s_out[j] = s * sw[j];
+        c_out[j] = c * sw[j] + (b ? b[j] : 0.f);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_quant_rows_e4m3(const bf16 *x, int K, int rows, const int *n_rows, uint8_t *q, float *scale,
+                                   const int *status, cudaStream_t s, bool pdl, bool trigger) {
+    if (K < 256 || K > 2048 || K % 256) return cudaErrorInvalidValue;
+    const int blocks = (rows + Q_WARPS - 1) / Q_WARPS;
+    if (blocks < 1) return cudaSuccess;
+    if (!pdl) {
+        quant_rows_e4m3_kernel<<<blocks, 32 * Q_WARPS, 0, s>>>(x, K, rows, n_rows, q, scale, status, trigger ? 1 : 0);
+        return cudaGetLastError();
+    }
+    return launch_pdl(quant_rows_e4m3_kernel, dim3(blocks), dim3(32 * Q_WARPS), 0, s, x, K, rows, n_rows, q, scale,
+                      status, trigger ? 1 : 0);
+}
+
+cudaError_t launch_fold_ln_e4m3(const uint8_t *Wq, const float *sw, int N, int K, const float *gamma,
+                                const float *beta, const float *b, float *s_out, float *c_out, cudaStream_t s) {
+    fold_ln_e4m3_kernel<<<(N + 7) / 8, 256, 0, s>>>(Wq, sw, N, K, gamma, beta, b, s_out, c_out);
+    return cudaGetLastError();
+}
+
+}  // namespace albert

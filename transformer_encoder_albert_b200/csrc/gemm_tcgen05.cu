@@ -53,7 +53,7 @@ using namespace gemm;
 // staging tiles per epilogue warp (output, residual or second output, and for
 // the residual epilogue a second output tile, paid for with one stage), then
 // barriers; 1 KiB slack for the 1 KiB alignment of the stages.
-template <int EPI, bool PAIR>
+template <int EPI, bool PAIR, bool F8 = false>
 struct Plan {
     static constexpr bool kRes = EPI == kEpiResStats;
     static constexpr bool kLnIn = EPI == kEpiLnIn || EPI == kEpiLnInGelu || EPI == kEpiLnInScatter;
@@ -61,8 +61,10 @@ struct Plan {
     static constexpr int BSTAGE = PAIR ? B_HALF_BYTES : B_BYTES;
     static constexpr int NSTG = kRes ? 3 : 2;
     // per-column vectors of a unit: bias, then W gamma (LayerNorm input) or
-    // out_g and res_g (residual epilogue); two buffers (this unit, the next)
-    static constexpr int NVEC = kLnIn ? 2 : (kRes ? 3 : 1);
+    // out_g and res_g (residual epilogue), then for E4M3 operands the weight
+    // row scales; two buffers (this unit, the next)
+    static constexpr int NVEC_BASE = kLnIn ? 2 : (kRes ? 3 : 1);
+    static constexpr int NVEC = NVEC_BASE + (F8 ? 1 : 0);
     static constexpr int VEC_BYTES = 2 * NVEC * BN * 4;
     static constexpr int SMEM = 1024 + NST * (A_BYTES + BSTAGE) + NSTG * EPI_WARPS * STG_BYTES + VEC_BYTES + 1024;
     static_assert(SMEM <= 232448, "shared memory per CTA");
@@ -81,9 +83,9 @@ struct Smem {
     int *misc;               // [0] n_rows, [1] status at entry
 };
 
-template <int EPI, bool PAIR>
+template <int EPI, bool PAIR, bool F8>
 __device__ __forceinline__ Smem carve(uint8_t *raw) {
-    using P = Plan<EPI, PAIR>;
+    using P = Plan<EPI, PAIR, F8>;
     constexpr int NST = P::NST;
     Smem s;
     uint8_t *p = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
@@ -132,14 +134,14 @@ __device__ __forceinline__ uint32_t stg_off(int r, int q) {
 __device__ __forceinline__ void st_shared_v4(uint32_t a, uint4 v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
-__device__ __forceinline__ float4 ld_shared_f4(uint32_t a) {
-    float4 v;
-    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a) : "memory");
-    return v;
-}
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
     uint4 v;
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a) : "memory");
     return v;
 }
 
@@ -192,7 +194,10 @@ __device__ __forceinline__ void row_stats_merge(const float2 (&q)[LN_PARTS], flo
     rstd = rsqrtf(m2 * (1.0f / LN_N) + eps);
 }
 
-template <int EPI, bool PAIR>
+// F8: both operands are E4M3 (tiles of 128 bytes = 128 elements along K, products
+// with tcgen05.mma kind::f8f6f4, K = 32 per instruction) with fp32 row scales:
+// the epilogue starts from acc * a_scale[row] * w_scale[col].
+template <int EPI, bool PAIR, bool F8>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmRes,
@@ -201,11 +206,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     constexpr bool kGelu = EPI == kEpiGelu || EPI == kEpiLnInGelu;
     constexpr bool kScatter = EPI == kEpiScatter || EPI == kEpiLnInScatter;
     constexpr bool kRes = EPI == kEpiResStats;
-    constexpr int NST = Plan<EPI, PAIR>::NST;
-    constexpr int BSTAGE = Plan<EPI, PAIR>::BSTAGE;
+    constexpr int NST = Plan<EPI, PAIR, F8>::NST;
+    constexpr int BSTAGE = Plan<EPI, PAIR, F8>::BSTAGE;
+    constexpr int KB = F8 ? 128 : BK;  // K elements per stage (a 128-byte swizzle row)
     constexpr int UM = PAIR ? 2 * BM : BM;  // rows of A (and D) per unit
     extern __shared__ uint8_t smem_raw[];
-    Smem sm = carve<EPI, PAIR>(smem_raw);
+    Smem sm = carve<EPI, PAIR, F8>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // A pair works on one unit at a time; rank 0 issues the MMAs for both CTAs.
     const uint32_t rank = PAIR ? cluster_ctarank() : 0;
@@ -236,6 +242,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         prefetch_tmap(&tmB);
         if (!kScatter) prefetch_tmap(&tmOut);
         if (kRes) prefetch_tmap(&tmRes);
+
     }
     if (warp == 1) {
         if (PAIR) {
@@ -266,7 +273,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const int m_blocks = (n_rows + UM - 1) / UM;
     const int n_sub = p.N / BN;
     const int units = m_blocks * n_sub;  // unit u = tile (u / n_sub, u % n_sub), row-block major
-    const int kblocks = p.K / BK;
+    const int kblocks = p.K / KB;
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer --
@@ -290,13 +297,13 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         // both CTAs' copies count on rank 0's barrier, which expects them all
                         const uint32_t fb0 = mapa_shared(fb, 0);
                         if (rank == 0) mbar_arrive_expect_tx(fb, 2 * (A_BYTES + B_HALF_BYTES));
-                        tma_load_2d_pair(a_dst, &tmA, fb0, kb * BK, m * UM + (int)rank * BM);
-                        tma_load_2d_pair_hint(b_dst, &tmB, fb0, kb * BK, n * BN + (int)rank * B_BOX, keep);
+                        tma_load_2d_pair(a_dst, &tmA, fb0, kb * KB, m * UM + (int)rank * BM);
+                        tma_load_2d_pair_hint(b_dst, &tmB, fb0, kb * KB, n * BN + (int)rank * B_BOX, keep);
                     } else {
                         mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
-                        tma_load_2d(a_dst, &tmA, fb, kb * BK, m * BM);
-                        tma_load_2d_hint(b_dst, &tmB, fb, kb * BK, n * BN, keep);
-                        tma_load_2d_hint(b_dst + B_HALF_BYTES, &tmB, fb, kb * BK, n * BN + B_BOX, keep);
+                        tma_load_2d(a_dst, &tmA, fb, kb * KB, m * BM);
+                        tma_load_2d_hint(b_dst, &tmB, fb, kb * KB, n * BN, keep);
+                        tma_load_2d_hint(b_dst + B_HALF_BYTES, &tmB, fb, kb * KB, n * BN + B_BOX, keep);
                     }
                     ++issued;
                     if (++stage == NST) { stage = 0; phase ^= 1; }
@@ -316,7 +323,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     } else if (warp == 1) {
         // -------------------------------------------------------- MMA issuer --
         if (lane == 0 && rank == 0) {
-            const uint32_t idesc = idesc_bf16_f32(UM, BN);
+            const uint32_t idesc = F8 ? idesc_e4m3_f32(UM, BN) : idesc_bf16_f32(UM, BN);
             int stage = 0, acc = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -336,7 +343,14 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     const uint32_t b0 = smem_u32(sm.b + stage * BSTAGE);
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
-                        if (PAIR)
+                        // each product consumes 32 bytes of K: 16 bf16 or 32 E4M3 elements
+                        if (PAIR && F8)
+                            umma_e4m3_pair(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), idesc,
+                                           (kb | k) != 0);
+                        else if (F8)
+                            umma_e4m3(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), idesc,
+                                      (kb | k) != 0);
+                        else if (PAIR)
                             umma_bf16_pair(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), idesc,
                                            (kb | k) != 0);
                         else
@@ -366,8 +380,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int r_local = quad * 32 + lane;
         const int row_off = (int)rank * BM;  // this CTA's rows within a unit
         const uint32_t stg = smem_u32(sm.stg + ew * STG_BYTES);
-        const uint32_t rstg = smem_u32(sm.rstg + ew * STG_BYTES);
-        const uint32_t stg2 = smem_u32(sm.stg2 + ew * STG_BYTES);  // kRes only
+        const uint32_t rstg = smem_u32(sm.rstg + ew * STG_BYTES);  // residual tile (kRes) or second output tile
+        const uint32_t stg2 = smem_u32(sm.stg2 + ew * STG_BYTES);  // kRes only: second output tile
         const uint32_t rbar = smem_u32(&sm.rbar[ew]);
         const bool res_ln = kRes && p.res_stats != nullptr;
         uint32_t rph = 0;
@@ -402,7 +416,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         // stores it at the end of the current unit, and arrives on vec_full.
         // (Read from global memory inside the chunk loop, these uniform loads
         // stalled every chunk on their latency.)
-        constexpr int NVEC = Plan<EPI, PAIR>::NVEC;
+        constexpr int NVEC = Plan<EPI, PAIR, F8>::NVEC;
+        constexpr int NVEC_BASE = Plan<EPI, PAIR, F8>::NVEC_BASE;
         const int et = ew * 32 + lane;  // 0..255: the column this thread stages
         float vreg[NVEC];
         auto vec_load = [&](int un) {
@@ -411,8 +426,9 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             if (kLnIn) vreg[1] = __ldg(p.fold_s + col);
             if (kRes) {
                 vreg[1] = __ldg(p.out_g + col);
-                vreg[NVEC - 1] = res_ln ? __ldg(p.res_g + col) : 0.f;
+                vreg[NVEC_BASE - 1] = res_ln ? __ldg(p.res_g + col) : 0.f;
             }
+            if (F8) vreg[NVEC - 1] = __ldg(p.w_scale + col);
         };
         auto vec_store = [&](int b) {
 #pragma unroll
@@ -432,6 +448,9 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             const int tile_row = m * UM + row_off + quad * 32;
             int dst = row;
             if (kScatter) dst = row_ok ? __ldg(p.row_dst + row) : -1;
+            // E4M3 operands: the A row's scale (rows past rows_cap, reachable in a
+            // pair's last unit, are never stored)
+            const float asc = F8 ? (row < p.rows_cap ? __ldg(p.a_scale + row) : 0.f) : 1.f;
             float mu = 0.f, rstd = 1.f;        // LayerNorm of the A operand
             if (kLnIn) row_stats_merge(qin, p.eps, mu, rstd);
             float rmu = 0.f, rrstd = 1.f;      // LayerNorm of the residual
@@ -450,7 +469,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             // shared addresses of this warp's 128 columns of each vector
             const uint32_t vbias = smem_u32(sm.vec + (vb * NVEC) * BN + half * 128);
             const uint32_t vsec = vbias + BN * 4;           // W gamma or out_g
-            const uint32_t vres = smem_u32(sm.vec + (vb * NVEC + NVEC - 1) * BN + half * 128);  // res_g
+            const uint32_t vres = smem_u32(sm.vec + (vb * NVEC + NVEC_BASE - 1) * BN + half * 128);  // res_g
+            const uint32_t vws = smem_u32(sm.vec + (vb * NVEC + NVEC - 1) * BN + half * 128);  // w_scale (F8)
             const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + ab * BN + half * 128;
             const int ncol0 = n * BN + half * 128;  // first output column of this warp
             float mean = 0.f, m2 = 0.f;
@@ -481,6 +501,24 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     }
                 }
                 const uint32_t *rc = r[c & 1];
+                uint32_t rsc[32];
+                if (F8) {
+                    // acc * a_scale[row] * w_scale[col]: the product of the unscaled E4M3 codes
+                    const uint32_t ws4 = vws + c * 128;
+                    const uint64_t a2 = f2_make(asc, asc);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 w = ld_shared_f4(ws4 + q * 16);
+                        const float2 x0 = f2_split(f2_mul(f2_mul(f2_make_u(rc[4 * q], rc[4 * q + 1]), f2_make(w.x, w.y)), a2));
+                        const float2 x1 =
+                            f2_split(f2_mul(f2_mul(f2_make_u(rc[4 * q + 2], rc[4 * q + 3]), f2_make(w.z, w.w)), a2));
+                        rsc[4 * q] = __float_as_uint(x0.x);
+                        rsc[4 * q + 1] = __float_as_uint(x0.y);
+                        rsc[4 * q + 2] = __float_as_uint(x1.x);
+                        rsc[4 * q + 3] = __float_as_uint(x1.y);
+                    }
+                    rc = rsc;
+                }
                 const int col0 = ncol0 + c * 32;
                 uint64_t v[16];  // columns col0 + 2j, col0 + 2j + 1
                 const uint32_t bias4 = vbias + c * 128;  // 32 floats per chunk
@@ -609,10 +647,10 @@ bool gemm_use_pair(int rows_cap, int variant) {
 }
 
 // The kernel instance's shared-memory limit, raised once per device.
-template <int EPI, bool PAIR>
+template <int EPI, bool PAIR, bool F8>
 static cudaError_t configure(int smem) {
     static std::atomic<unsigned long long> configured{0};
-    return ensure_smem_attr(reinterpret_cast<const void *>(gemm_bf16_kernel<EPI, PAIR>), smem, configured);
+    return ensure_smem_attr(reinterpret_cast<const void *>(gemm_bf16_kernel<EPI, PAIR, F8>), smem, configured);
 }
 
 // Clusters of two GEMM CTAs that fit on the device at once (every epilogue
@@ -624,7 +662,7 @@ static int pair_clusters(int num_sms) {
     const int known = cached[dev].load(std::memory_order_acquire);
     if (known > 0) return known;
     int n = 0;
-    if (configure<kEpiBias, true>(Plan<kEpiBias, true>::SMEM) == cudaSuccess) {
+    if (configure<kEpiBias, true, false>(Plan<kEpiBias, true>::SMEM) == cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -636,7 +674,7 @@ static int pair_clusters(int num_sms) {
         cfg.dynamicSmemBytes = Plan<kEpiBias, true>::SMEM;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaOccupancyMaxActiveClusters(&n, gemm_bf16_kernel<kEpiBias, true>, &cfg) != cudaSuccess) n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_bf16_kernel<kEpiBias, true, false>, &cfg) != cudaSuccess) n = 0;
     }
     cudaGetLastError();
     if (n <= 0 || n > num_sms / 2) n = num_sms / 2;
@@ -655,22 +693,23 @@ int gemm_grid(int epi, int rows_cap, int N, int num_sms, int variant) {
     return units < num_sms ? (units > 0 ? units : 1) : num_sms;
 }
 
-template <int EPI>
+template <int EPI, bool F8>
 static cudaError_t launch_one(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
                               const CUtensorMap &tmRes, const GemmArgs &a, int grid, cudaStream_t s, bool pair,
                               bool pdl) {
     if (!pair) {
-        constexpr int smem = Plan<EPI, false>::SMEM;
-        cudaError_t e = configure<EPI, false>(smem);
+        constexpr int smem = Plan<EPI, false, F8>::SMEM;
+        cudaError_t e = configure<EPI, false, F8>(smem);
         if (e != cudaSuccess) return e;
         if (!pdl) {
-            gemm_bf16_kernel<EPI, false><<<grid, THREADS, smem, s>>>(tmA, tmB, tmOut, tmRes, a);
+            gemm_bf16_kernel<EPI, false, F8><<<grid, THREADS, smem, s>>>(tmA, tmB, tmOut, tmRes, a);
             return cudaGetLastError();
         }
-        return launch_pdl(gemm_bf16_kernel<EPI, false>, dim3(grid), dim3(THREADS), smem, s, tmA, tmB, tmOut, tmRes, a);
+        return launch_pdl(gemm_bf16_kernel<EPI, false, F8>, dim3(grid), dim3(THREADS), smem, s, tmA, tmB, tmOut, tmRes,
+                          a);
     }
     if (grid < 2 || grid % 2) return cudaErrorInvalidConfiguration;
-    cudaError_t e = configure<EPI, true>(Plan<EPI, true>::SMEM);
+    cudaError_t e = configure<EPI, true, F8>(Plan<EPI, true, F8>::SMEM);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
@@ -682,25 +721,37 @@ static cudaError_t launch_one(const CUtensorMap &tmA, const CUtensorMap &tmB, co
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(THREADS);
-    cfg.dynamicSmemBytes = Plan<EPI, true>::SMEM;
+    cfg.dynamicSmemBytes = Plan<EPI, true, F8>::SMEM;
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, gemm_bf16_kernel<EPI, true>, tmA, tmB, tmOut, tmRes, a);
+    return cudaLaunchKernelEx(&cfg, gemm_bf16_kernel<EPI, true, F8>, tmA, tmB, tmOut, tmRes, a);
 }
 
 cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
                         const CUtensorMap &tmRes, const GemmArgs &a, int grid, cudaStream_t s, int variant,
                         bool pdl) {
     const bool pair = gemm_use_pair(a.rows_cap, variant);
+    if (a.e4m3) {
+        // the E4M3 variant serves the four layer GEMMs and the single-kernel tests
+        switch (epi) {
+            case kEpiBias: return launch_one<kEpiBias, true>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+            case kEpiGelu: return launch_one<kEpiGelu, true>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+            case kEpiResStats: return launch_one<kEpiResStats, true>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+            case kEpiScatter: return launch_one<kEpiScatter, true>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+            case kEpiLnIn: return launch_one<kEpiLnIn, true>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+            case kEpiLnInGelu: return launch_one<kEpiLnInGelu, true>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+        }
+        return cudaErrorInvalidValue;
+    }
     switch (epi) {
-        case kEpiBias: return launch_one<kEpiBias>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-        case kEpiGelu: return launch_one<kEpiGelu>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-        case kEpiResStats: return launch_one<kEpiResStats>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-        case kEpiScatter: return launch_one<kEpiScatter>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-        case kEpiLnIn: return launch_one<kEpiLnIn>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-        case kEpiLnInGelu: return launch_one<kEpiLnInGelu>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-        case kEpiLnInScatter: return launch_one<kEpiLnInScatter>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+        case kEpiBias: return launch_one<kEpiBias, false>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+        case kEpiGelu: return launch_one<kEpiGelu, false>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+        case kEpiResStats: return launch_one<kEpiResStats, false>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+        case kEpiScatter: return launch_one<kEpiScatter, false>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+        case kEpiLnIn: return launch_one<kEpiLnIn, false>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+        case kEpiLnInGelu: return launch_one<kEpiLnInGelu, false>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+        case kEpiLnInScatter: return launch_one<kEpiLnInScatter, false>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
     }
     return cudaErrorInvalidValue;
 }
@@ -740,6 +791,20 @@ static int encode_bf16(CUtensorMap *tm, const void *base, uint64_t rows, uint64_
 
 int make_tmap_bf16(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
     return encode_bf16(tm, base, rows, cols, BK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+int make_tmap_e4m3(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return -1;
+    if ((reinterpret_cast<uintptr_t>(base) & 15) || cols % 16) return -2;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? 0 : -3;
 }
 
 int make_tmap_bf16_tile32(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols) {

@@ -114,6 +114,11 @@ struct GemmArgs {
     unsigned long long wait_ns;  // limit of the bounded waits (0 = kWaitLimitNs, 2 s)
     int withhold_loads;        // fault injection for tests: the TMA producer issues no loads, so
                                // the MMA issuer's first wait cannot complete and runs out
+    // E4M3 operands (A and W as row-scaled E4M3 codes, maps from make_tmap_e4m3; K a
+    // multiple of 128): the epilogue starts from acc * a_scale[row] * w_scale[col]
+    int e4m3;
+    const float *a_scale;      // [rows_cap]
+    const float *w_scale;      // [N]
 };
 
 // Encode a 2-D bf16 row-major [rows, cols] tensor map with a {64, box_rows}
@@ -121,6 +126,9 @@ struct GemmArgs {
 // weights).  Returns 0 on success.
 int make_tmap_bf16(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols,
                    uint32_t box_rows);
+// Map of an E4M3 (byte) row-major [rows, cols] tensor with a {128, box_rows} box
+// and the 128-byte swizzle: the operands of the E4M3 GEMM variant.
+int make_tmap_e4m3(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 // Map of a bf16 row-major [rows, cols] tensor with a 32x32 box and the 64-byte
 // swizzle: the epilogue's output stores and residual loads.
 int make_tmap_bf16_tile32(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols);
@@ -138,7 +146,7 @@ int gemm_grid(int epi, int rows_cap, int N, int num_sms, int variant = kGemmAuto
 // The epilogue reads its per-column vectors as float4: each must be 16-byte aligned.
 inline bool gemm_vectors_aligned(const GemmArgs &a) {
     auto ok = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
-    return ok(a.bias) && ok(a.fold_s) && ok(a.res_g) && ok(a.out_g);
+    return ok(a.bias) && ok(a.fold_s) && ok(a.res_g) && ok(a.out_g) && ok(a.w_scale);
 }
 
 // tmOut: tile32 map of the output (unused by the scatter epilogues); tmRes: tile32
@@ -235,6 +243,7 @@ struct EmbedArgs {
     int dst_padded;
     int *status;
     int trigger;        // the next launch is one of ours with PDL (see GemmArgs)
+    const float *emb_in;  // non-null: rows [n_rows, 128] fp32 taken as E (no gather, no LayerNorm)
 };
 cudaError_t launch_embed(const EmbedArgs &a, cudaStream_t s);
 // out[b][d][t] = t < seq_len[b] ? src[(b*T + t)*D + d] : 0 (elem_bytes 2 or 4),
@@ -262,6 +271,15 @@ cudaError_t launch_ln_rows(const bf16 *zg, const float2 *stats, const float *gam
                            const int *n_rows, int *status, cudaStream_t s);
 // out[i] = a[i] + b[i]
 cudaError_t launch_vec_add(const float *a, const float *b, float *out, int n, cudaStream_t s);
+
+// ---------------------------------------------------------------- E4M3 path --
+// x [rows, K] bf16 -> q [rows, K] E4M3 and scale [rows] (fp8.cu); rows past *n_rows
+// (if given) are left alone; K a multiple of 256, at most 2048.
+cudaError_t launch_quant_rows_e4m3(const bf16 *x, int K, int rows, const int *n_rows, uint8_t *q, float *scale,
+                                   const int *status, cudaStream_t s, bool pdl, bool trigger);
+// Folded LayerNorm constants of an E4M3 weight with row scales (see launch_fold_ln).
+cudaError_t launch_fold_ln_e4m3(const uint8_t *Wq, const float *sw, int N, int K, const float *gamma,
+                                const float *beta, const float *b, float *s_out, float *c_out, cudaStream_t s);
 
 // fp32 -> bf16 conversion of a parameter block.
 cudaError_t launch_f32_to_bf16(const float *src, bf16 *dst, size_t n, cudaStream_t s);

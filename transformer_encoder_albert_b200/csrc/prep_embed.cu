@@ -143,26 +143,33 @@ embed_ln_kernel(const EmbedArgs a) {
     const int b = lo;
     const int t = r - __ldg(a.seq_start + b);
     const bool valid = t < __ldg(a.seq_len + b);
-    long long id = a.ids_padded ? a.ids[(size_t)b * a.T + t] : a.ids[r];
-    if (id < 0 || id >= a.vocab) {
-        if (valid) set_status(a.status, kStatusId);
-        id = 0;  // padding slot: any id; its row never reaches a valid output
+    float y0, y1, y2, y3;
+    if (a.emb_in) {
+        // the caller supplies the post-LayerNorm embedding rows themselves
+        const float4 e = reinterpret_cast<const float4 *>(a.emb_in + (size_t)r * kEmb)[lane];
+        y0 = e.x; y1 = e.y; y2 = e.z; y3 = e.w;
+    } else {
+        long long id = a.ids_padded ? a.ids[(size_t)b * a.T + t] : a.ids[r];
+        if (id < 0 || id >= a.vocab) {
+            if (valid) set_status(a.status, kStatusId);
+            id = 0;  // padding slot: any id; its row never reaches a valid output
+        }
+        const float4 w = __ldg(reinterpret_cast<const float4 *>(a.word + id * kEmb) + lane);
+        const float4 ps = __ldg(reinterpret_cast<const float4 *>(a.pos + (size_t)t * kEmb) + lane);
+        const float4 ty = __ldg(reinterpret_cast<const float4 *>(a.type) + lane);
+        float x[4] = {w.x + ps.x + ty.x, w.y + ps.y + ty.y, w.z + ps.z + ty.z, w.w + ps.w + ty.w};
+        float s = x[0] + x[1] + x[2] + x[3];
+        for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        const float mu = s * (1.0f / kEmb);
+        float q = 0.f;
+        for (int i = 0; i < 4; ++i) { const float d = x[i] - mu; q = fmaf(d, d, q); }
+        for (int o = 16; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+        const float rstd = rsqrtf(q * (1.0f / kEmb) + a.eps);
+        const float4 g = __ldg(reinterpret_cast<const float4 *>(a.g) + lane);
+        const float4 bb = __ldg(reinterpret_cast<const float4 *>(a.b) + lane);
+        y0 = fmaf((x[0] - mu) * rstd, g.x, bb.x); y1 = fmaf((x[1] - mu) * rstd, g.y, bb.y);
+        y2 = fmaf((x[2] - mu) * rstd, g.z, bb.z); y3 = fmaf((x[3] - mu) * rstd, g.w, bb.w);
     }
-    const float4 w = __ldg(reinterpret_cast<const float4 *>(a.word + id * kEmb) + lane);
-    const float4 ps = __ldg(reinterpret_cast<const float4 *>(a.pos + (size_t)t * kEmb) + lane);
-    const float4 ty = __ldg(reinterpret_cast<const float4 *>(a.type) + lane);
-    float x[4] = {w.x + ps.x + ty.x, w.y + ps.y + ty.y, w.z + ps.z + ty.z, w.w + ps.w + ty.w};
-    float s = x[0] + x[1] + x[2] + x[3];
-    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    const float mu = s * (1.0f / kEmb);
-    float q = 0.f;
-    for (int i = 0; i < 4; ++i) { const float d = x[i] - mu; q = fmaf(d, d, q); }
-    for (int o = 16; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-    const float rstd = rsqrtf(q * (1.0f / kEmb) + a.eps);
-    const float4 g = __ldg(reinterpret_cast<const float4 *>(a.g) + lane);
-    const float4 bb = __ldg(reinterpret_cast<const float4 *>(a.b) + lane);
-    const float y0 = fmaf((x[0] - mu) * rstd, g.x, bb.x), y1 = fmaf((x[1] - mu) * rstd, g.y, bb.y);
-    const float y2 = fmaf((x[2] - mu) * rstd, g.z, bb.z), y3 = fmaf((x[3] - mu) * rstd, g.w, bb.w);
     if (a.out_f32) {
         reinterpret_cast<float4 *>(static_cast<float *>(a.E) + (size_t)r * kEmb)[lane] = make_float4(y0, y1, y2, y3);
     } else {
