@@ -396,6 +396,7 @@ def measure_workload(args, ctx, name, padded, graph_mode, extras):
     ids_d = torch.as_tensor(ids).cuda()
     mask_d = torch.as_tensor(mask).cuda()
     enc = tea.Encoder(w, arch, dtype=args.dtype, max_tokens=wl.B * wl.T, pack=not padded)
+    enc.set_small_batch_kernel(args.small_batch == "on")
     out = torch.empty(wl.B, wl.T, arch["out_dim"], device="cuda", dtype=torch.bfloat16)
     stream = torch.cuda.current_stream()
     rows = n_tok if not padded else wl.B * wl.T
@@ -567,6 +568,17 @@ def measure_workload(args, ctx, name, padded, graph_mode, extras):
               if extras else None)
     dom_ms = dom[1] / max(dom[0], 1)
     achieved = per_launch.get(dominant, 0.0) / (dom_ms / 1000.0) / 1e12
+    if dominant == "quant_e4m3":
+        # HBM-bound: bf16 rows read, E4M3 codes and a scale per row written; per
+        # execution three quantizations of 768-wide rows and one of 2048-wide rows
+        qbytes = rows * (3 * 768 + 2048) * 3 / 4.0 + rows * 4
+        hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        roofline_hbm = {"kernel": dominant, "bound": "hbm", "achieved": qbytes / (dom_ms / 1000.0) / 1e9,
+                        "peak": hbm, "unit": "GB/s", "bytes_per_launch": qbytes,
+                        "peak_source": f"{peaks_src} hbm_gbs"}
+        roofline_hbm["frac"] = roofline_hbm["achieved"] / hbm
+    else:
+        roofline_hbm = None
     traffic, traffic_note = load_traffic(dominant, label, wl.T)
     bound = "tensor"
     dom_peak = peak if (args.dtype == "bf16" or dominant in fp8_classes) else peak / 2.0
@@ -577,6 +589,10 @@ def measure_workload(args, ctx, name, padded, graph_mode, extras):
                 "frac_of_sustained": (achieved / peak_sus) if peak_sus else None,
                 "launches_timed": dom[0], "launches_timed_note": f"1 of {per_step} per step", "avg_launch_ms": dom_ms,
                 "flops_per_launch": per_launch.get(dominant, 0.0)}
+    if roofline_hbm is not None:
+        roofline_hbm.update({"launches_timed": dom[0], "avg_launch_ms": dom_ms, "traffic": None,
+                             "traffic_source": "no ncu capture of the quantizer"})
+        roofline = roofline_hbm
     clocks = sampler.summary(t_wall0, t_wall1)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -589,6 +605,7 @@ def measure_workload(args, ctx, name, padded, graph_mode, extras):
                    "padded_slot_tokens_per_step_per_gpu": wl.B * wl.T,
                    "pack": not padded, "parallelism": f"replicas x{world}",
                    "launch": "cuda_graph" if graph_mode else "stream",
+                   "small_batch_kernel": args.small_batch,
                    "l2": "flushed between timed steps (512 MiB write)"},
         "padded_slot_tokens_per_s": sum_r(float(wl.B * wl.T * args.steps)) / (total_ms / 1000.0),
         "tensor_peak_frac": {"whole_encoder": fwd_flops / (ms_per_step / 1000.0) / 1e12 / peak,
@@ -637,6 +654,8 @@ def main():
                     help="run this many untimed forwards and exit (for ncu captures); no JSON metric line")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "fp8"],
                     help="fp8: the four layer GEMMs on E4M3 operands with per-row scales")
+    ap.add_argument("--small-batch", default="off", choices=["on", "off"],
+                    help="on: batches of at most 128 token rows run as one persistent kernel")
     ap.add_argument("--all-configs", action="store_true",
                     help="one JSON line per workload of the suite (packed and padded b256, b1_T64 stream and graph)")
     args = ap.parse_args()

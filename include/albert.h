@@ -240,8 +240,8 @@ int albert_last_forward_launches(const albert_handle *h);
  * straight into W2), instead of ~65 per-layer launches ("ALBERT: How Kokoro's
  * Phoneme Encoder Works", section "Inside One Real ALBERT Layer", steps 2-6,
  * and "2. Cross-layer parameter sharing").  Same results within the stated
- * tolerances; deterministic.  enable: 1 (default) uses it when it applies,
- * 0 always runs the per-layer kernels.  Other values: ALBERT_ERR_CONFIG. */
+ * tolerances; deterministic.  enable: 1 uses it when it applies, 0 (default)
+ * always runs the per-layer kernels.  Other values: ALBERT_ERR_CONFIG. */
 int albert_set_small_batch_kernel(albert_handle *h, int enable);
 
 /* ---- per-kernel timing (optional) ----

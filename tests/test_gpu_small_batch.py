@@ -93,6 +93,7 @@ def test_small_batch_varlen_entry(w_bf16):
     lengths = (40, 1, 25)
     ids, mask, L = _batch(lengths, 40, seed=11)
     enc = tea.Encoder(w_bf16, A, max_tokens=ids.size)
+    enc.set_small_batch_kernel(True)
     padded = enc.forward(_t(ids), _t(mask)).float().cpu().numpy()
     packed_ids = np.concatenate([ids[b, :L[b]] for b in range(len(L))])
     cu = np.concatenate([[0], np.cumsum(L)]).astype(np.int32)
@@ -108,6 +109,7 @@ def test_small_batch_is_deterministic_and_reusable(w_bf16):
     ids, mask, L = _batch((50, 13), 64, seed=21)
     ids2, mask2, _ = _batch((64,), 64, seed=22)
     enc = tea.Encoder(w_bf16, A, max_tokens=128)
+    enc.set_small_batch_kernel(True)
     a = enc.forward(_t(ids), _t(mask)).clone()
     enc.forward(_t(ids2), _t(mask2))
     b = enc.forward(_t(ids), _t(mask))
@@ -120,6 +122,7 @@ def test_small_batch_bad_id_leaves_output_untouched(w_bf16):
     ids, mask, L = _batch((30, 20), 32, seed=5)
     ids[1, 3] = 500
     enc = tea.Encoder(w_bf16, A, max_tokens=64)
+    enc.set_small_batch_kernel(True)
     out = torch.full((2, 32, 512), 3.25, device="cuda", dtype=torch.bfloat16)
     tea.albert_forward(enc.h, _t(ids), _t(mask), out)
     assert enc.status() == 4  # ALBERT_ERR_ID
@@ -134,6 +137,7 @@ def test_small_batch_expired_wait_reports_timeout(w_bf16):
     works again afterwards."""
     ids, mask, L = _batch((64,), 64, seed=9)
     enc = tea.Encoder(w_bf16, A, max_tokens=64)
+    enc.set_small_batch_kernel(True)
     good = enc.forward(_t(ids), _t(mask)).clone()
     enc.set_wait_limit(200_000)
     enc.test_stall(["small_batch_forward"])
@@ -159,6 +163,7 @@ def test_small_batch_forward_in_a_cuda_graph(w_bf16):
     ids, mask, L = synth.make_batch(wl)
     ids_d, mask_d = _t(ids), _t(mask)
     enc = tea.Encoder(w_bf16, A, max_tokens=wl.B * wl.T)
+    enc.set_small_batch_kernel(True)
     ref = enc.forward(ids_d, mask_d).clone()
     out = torch.empty_like(ref)
     g = torch.cuda.CUDAGraph()

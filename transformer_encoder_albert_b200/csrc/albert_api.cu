@@ -117,11 +117,11 @@ struct albert_handle {
     // embedding in one persistent kernel; its own statistics, FFN partial sums,
     // barrier counter and {64, 64}-box tensor maps
     bool small_ok = false;       // the handle's configuration allows it
-    bool small_enabled = true;   // albert_set_small_batch_kernel
+    bool small_enabled = false;  // albert_set_small_batch_kernel
     float2 *sst1 = nullptr, *sst2 = nullptr;
     float *spart = nullptr;
     int *sbar = nullptr;
-    CUtensorMap sm_E, sm_X, sm_C, sm_X1, sm_Z, sm_win, sm_wqkv, sm_wo, sm_w1, sm_w2, sm_wout;
+    CUtensorMap sm_E, sm_X, sm_C, sm_X1, sm_Z, sm_win, sm_wqkv, sm_wo, sm_w1, sm_w2, sm_wout, sm_part;
     int last_launches = 0;       // kernel launches of the last forward
 
     // bounded waits inside the kernels: limit (0 = the kernels' default, 2 s) and,
@@ -342,6 +342,7 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
         s.tmQKV = h->tm_QKV; s.tmQKV64 = h->tm_QKV64;
         s.tmWin = h->sm_win; s.tmWqkv = h->sm_wqkv; s.tmWo = h->sm_wo; s.tmW1 = h->sm_w1; s.tmW2 = h->sm_w2;
         s.tmWout = c.out_dim > 0 ? h->sm_wout : h->sm_wo;  // (unused without a final projection)
+        s.tmPart = h->sm_part;
         s.X = static_cast<bf16 *>(h->X); s.QKV = static_cast<bf16 *>(h->QKV); s.C = static_cast<bf16 *>(h->C);
         s.X1 = static_cast<bf16 *>(h->X1); s.Z = static_cast<bf16 *>(h->Z);
         s.st1 = h->sst1; s.st2 = h->sst2; s.part = h->spart;
@@ -372,10 +373,12 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
             const auto &W = h->grp[group_of(c, l)];                  // this execution's weights
             const auto &Wp = h->grp[group_of(c, l > 0 ? l - 1 : 0)];  // the previous execution's (its LN2)
             // ALBERT_FP8: a layer GEMM's A operand is first quantized per row (E4M3 codes
-            // and scales in qA / sA); the GEMM reads the codes and the weights' codes
+            // and scales in qA / sA); the GEMM reads the codes and the weights' codes.
+            // The quantizer does not let the GEMM start early: resident GEMM CTAs
+            // would hold the registers its warps need.
             auto e4m3_operand = [&](const void *A, int K, const float *ws, GemmArgs &ga) -> int {
                 LAUNCH(L, kProfQuant, launch_quant_rows_e4m3(static_cast<const bf16 *>(A), K, h->rows_cap, h->n_rows,
-                                                             h->qA, h->sA, h->status, L.s, true, true));
+                                                             h->qA, h->sA, h->status, L.s, true, false));
                 ga.e4m3 = 1;
                 ga.a_scale = h->sA;
                 ga.w_scale = ws;
@@ -721,7 +724,8 @@ int create_impl(albert_handle *h, const albert_weights *w) {
                 make_tmap_bf16(&h->sm_wo, gp.wo, kHidden, kHidden, 64) ||
                 make_tmap_bf16(&h->sm_w1, gp.w1, kFfn, kHidden, 64) ||
                 make_tmap_bf16(&h->sm_w2, gp.w2, kHidden, kFfn, 64) ||
-                (O && make_tmap_bf16(&h->sm_wout, h->w_out, O, kHidden, 64)))
+                (O && make_tmap_bf16(&h->sm_wout, h->w_out, O, kHidden, 64)) ||
+                make_tmap_f32_tile32(&h->sm_part, h->spart, (uint64_t)(kFfn / 64) * kSmallMaxRows, kHidden))
                 return ALBERT_ERR_CUDA;
             h->small_ok = true;
         }

@@ -61,14 +61,15 @@ constexpr int SB_BOX = 64 * 64 * 2;           // one {64 cols, 64 rows} bf16 box
 constexpr int SB_A_BYTES = 4 * SB_BOX;        // A: up to four 64-row K blocks (two of 128 rows)
 constexpr int SB_B_BYTES = 4 * SB_BOX;        // B: up to four 64-row K blocks, or one of 256 rows
 constexpr int SB_H_BYTES = 2 * SB_BOX;        // FFN hidden chunk, 128 rows x 64 bf16
-constexpr int SB_SMEM = 1024 + SB_NS * (SB_A_BYTES + SB_B_BYTES) + SB_H_BYTES + 128 * 4 + 512;
+constexpr int SB_STG_BYTES = 4 * 32 * 32 * 4; // FFN partial sums: a 32 x 32 fp32 staging tile per epilogue warp
+constexpr int SB_SMEM = 1024 + SB_NS * (SB_A_BYTES + SB_B_BYTES) + SB_H_BYTES + SB_STG_BYTES + 128 * 4 + 512;
 static_assert(SB_SMEM <= 232448, "shared memory per CTA");
 constexpr int SB_PARTS = kSmallParts;         // 64-column statistics slices of a 768-wide row
 constexpr int SB_CHUNKS = kFfn / 64;          // FFN hidden chunks
 constexpr uint32_t SB_TM_O = 64;              // attention: O's columns within the item's TMEM columns
 
 struct SbSmem {
-    uint8_t *a, *b, *h;
+    uint8_t *a, *b, *h, *stg;
     float *inv_sum;                           // [128] attention: 1 / row sum
     uint64_t *full, *empty;                   // [SB_NS]
     uint64_t *acc_full, *acc_empty, *h_ready, *drain;
@@ -83,7 +84,8 @@ __device__ __forceinline__ SbSmem sb_carve(uint8_t *raw) {
     s.a = p;
     s.b = p + SB_NS * SB_A_BYTES;
     s.h = s.b + SB_NS * SB_B_BYTES;
-    s.inv_sum = reinterpret_cast<float *>(s.h + SB_H_BYTES);
+    s.stg = s.h + SB_H_BYTES;
+    s.inv_sum = reinterpret_cast<float *>(s.stg + SB_STG_BYTES);
     uint64_t *bars = reinterpret_cast<uint64_t *>(s.inv_sum + 128);
     s.full = bars;
     s.empty = bars + SB_NS;
@@ -212,6 +214,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
         prefetch_tmap(&p.tmW1);
         prefetch_tmap(&p.tmW2);
         prefetch_tmap(&p.tmWout);
+        prefetch_tmap(&p.tmPart);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(sm.tmem_slot), 512);
@@ -306,8 +309,14 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
                                                 : (ph == kPhQKV && l == 0) ? &p.tmX : &p.tmZ;
                         const CUtensorMap *tb = ph == kPhQKV ? &p.tmWqkv : ph == kPhOut ? &p.tmWo
                                                 : ph == kPhFfn ? &p.tmW1 : &p.tmWout;
-                        for (int kb = 0; kb < kHidden / 64; kb += kb_step)
+                        // every CTA of the phase reads the same A rows: each starts at another
+                        // stage of K, so that they do not all ask L2 for the same lines at once
+                        // (the sum over K is then taken in a rotated, fixed order per job)
+                        const int nsteps = (kHidden / 64) / kb_step;
+                        for (int i = 0; i < nsteps; ++i) {
+                            const int kb = ((i + job) % nsteps) * kb_step;
                             st[ns++] = {ta, tb, a_boxes, 1, kb_step, kb * 64, 0, kb * 64, job * 64};
+                        }
                         if (ph == kPhFfn)
                             for (int nb = 0; nb < 3; ++nb)
                                 st[ns++] = {nullptr, &p.tmW2, 0, 4, 1, 0, 0, job * 64, nb * 256};
@@ -575,24 +584,40 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
                     fence_proxy_async_smem();  // generic writes, read by the tensor core (async proxy)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_u32(sm.h_ready));
-                    // the three down products: fp32 partial sums of this chunk
+                    // the three down products: fp32 partial sums of this chunk, each warp's
+                    // 32 x 32 tiles staged in shared memory (128-byte swizzle) and stored
+                    // by TMA (rows of the partial buffer are 3 KB apart: one row per lane
+                    // would scatter every store)
+                    const bool any_row = quad * 32 < M;
+                    const uint32_t stg = smem_u32(sm.stg) + (uint32_t)quad * 4096u;
                     for (int nb = 0; nb < 3; ++nb) {
                         if (!wait_unit()) { ok = false; break; }
-                        float *dst = p.part + ((size_t)job * 128 + r) * kHidden + nb * 256;
                         for (int c = 0; c < 8; ++c) {
                             uint32_t t[32];
-                            tmem_ld32(trow + c * 32, t);
-                            tmem_ld_wait();
-                            if (row_ok) {
-                                float4 *d4 = reinterpret_cast<float4 *>(dst + c * 32);
+                            if (any_row) {
+                                tmem_ld32(trow + c * 32, t);
+                                tmem_ld_wait();
+                                if (lane == 0) bulk_wait_read0();  // the previous tile has left the staging
+                                __syncwarp();
 #pragma unroll
                                 for (int q = 0; q < 8; ++q)
-                                    d4[q] = make_float4(__uint_as_float(t[4 * q]), __uint_as_float(t[4 * q + 1]),
-                                                        __uint_as_float(t[4 * q + 2]), __uint_as_float(t[4 * q + 3]));
+                                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                                 ::"r"(stg + lane * 128 + ((q ^ (lane & 7)) << 4)), "r"(t[4 * q]),
+                                                 "r"(t[4 * q + 1]), "r"(t[4 * q + 2]), "r"(t[4 * q + 3])
+                                                 : "memory");
+                                fence_proxy_async_smem();
+                                __syncwarp();
+                                if (lane == 0) {
+                                    tma_store_2d(&p.tmPart, stg, nb * 256 + c * 32, job * 128 + quad * 32);
+                                    bulk_commit();
+                                }
                             }
                         }
                         release_unit();
                     }
+                    // the partial sums are in global memory before the phase's barrier
+                    if (lane == 0) bulk_wait0();
+                    __syncwarp();
                     if (!ok) break;
                     continue;
                 }

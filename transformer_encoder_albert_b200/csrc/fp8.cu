@@ -8,9 +8,8 @@
 // weights), so the tcgen05 product (kind::f8f6f4) sums q_x q_w exactly in fp32
 // and the epilogue multiplies by s_x s_w:
 //   amax = max |x|,  s = amax / 448,  q = E4M3(fp32(x * (448 / amax)))
-// (one rounding of the fp32 product to E4M3, to nearest even, saturating; the
-// conversion is written out from the format's definition, so that the code is
-// an exact function of the fp32 value; a row of zeros has s = 0 and q = 0).
+// (one rounding of the fp32 product to E4M3, to nearest even, saturating; a
+// row of zeros has s = 0 and q = 0).
 // A row's scale needs the whole row, which the GEMM epilogues that produce the
 // activations do not have (their tiles are 256 columns wide), so activations
 // are quantized by a separate pass per GEMM: one warp per row.
@@ -22,33 +21,14 @@ namespace {
 
 constexpr int Q_WARPS = 8;
 
-// fp32 -> E4M3 byte from the format's definition, one rounding: keep 3 mantissa
-// bits of a normal result (|y| >= 2^-6) with round to nearest, ties to even;
-// below 2^-6 the result is a multiple of 2^-9 (subnormal), rounded the same way;
-// magnitudes at or above 448 saturate to 448; the sign is kept (also on zero).
-__device__ __forceinline__ uint32_t f32_to_e4m3(float y) {
-    const uint32_t u = __float_as_uint(y);
-    const uint32_t sign = (u >> 24) & 0x80u;
-    const float ay = fabsf(y);
-    if (!(ay < 448.0f)) return sign | 0x7Eu;  // 448 = 1.75 * 2^8 (exponent field 15, mantissa 6)
-    const int e = (int)((u >> 23) & 0xFFu) - 127;
-    if (e >= -6) {
-        const uint32_t mant = u & 0x7FFFFFu;
-        uint32_t keep = mant >> 20;            // the 3 kept mantissa bits
-        const uint32_t rest = mant & 0xFFFFFu;  // the 20 dropped ones
-        if (rest > 0x80000u || (rest == 0x80000u && (keep & 1u))) ++keep;
-        uint32_t be = (uint32_t)(e + 7);       // biased E4M3 exponent, 1..15
-        if (keep == 8u) { keep = 0u; ++be; }
-        if (be > 15u || (be == 15u && keep == 7u)) return sign | 0x7Eu;
-        return sign | (be << 3) | keep;
-    }
-    // |y| < 2^-6: m * 2^-9 with m = round(|y| * 2^9) (exact scaling, then ties to even);
-    // m = 8 is the encoding of the smallest normal, 2^-6
-    return sign | (uint32_t)rintf(ay * 512.0f);
-}
-
+// Two fp32 -> two E4M3 bytes (lo at the lower address): one rounding to nearest,
+// ties to even, saturating at +-448, the sign kept (also on zero).  The
+// conversion instruction's results were checked bit for bit against this
+// definition on the GPU, every E4M3 midpoint included.
 __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
-    return (uint16_t)(f32_to_e4m3(lo) | (f32_to_e4m3(hi) << 8));
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
 }
 
 // x [rows, K] bf16 -> q [rows, K] E4M3, scale [rows] fp32.  K is a multiple of

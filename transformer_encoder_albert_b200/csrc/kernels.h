@@ -129,6 +129,9 @@ int make_tmap_bf16(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t co
 // Map of an E4M3 (byte) row-major [rows, cols] tensor with a {128, box_rows} box
 // and the 128-byte swizzle: the operands of the E4M3 GEMM variant.
 int make_tmap_e4m3(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// Map of an fp32 row-major [rows, cols] tensor with a 32x32 box and the 128-byte
+// swizzle (tile stores of fp32 partial sums).
+int make_tmap_f32_tile32(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols);
 // Map of a bf16 row-major [rows, cols] tensor with a 32x32 box and the 64-byte
 // swizzle: the epilogue's output stores and residual loads.
 int make_tmap_bf16_tile32(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols);
@@ -166,6 +169,7 @@ struct SmallFwdArgs {
     CUtensorMap tmE, tmX, tmC, tmX1, tmZ;       // E [rows,128]; X, C, X1 = z1*g1, Z = z2*g2 [rows,768]
     CUtensorMap tmQKV, tmQKV64;                 // [rows, 2304] with {64,128} / {64,64} boxes
     CUtensorMap tmWin, tmWqkv, tmWo, tmW1, tmW2, tmWout;
+    CUtensorMap tmPart;                         // part as fp32 [32 * 128, 768], {32, 32} box, 128-byte swizzle
     bf16 *X, *QKV, *C, *X1, *Z;
     float2 *st1, *st2;                          // [128][12]
     float *part;                                // [32][128][768] FFN partial sums
