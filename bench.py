@@ -654,8 +654,8 @@ def main():
                     help="run this many untimed forwards and exit (for ncu captures); no JSON metric line")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "fp8"],
                     help="fp8: the four layer GEMMs on E4M3 operands with per-row scales")
-    ap.add_argument("--small-batch", default="off", choices=["on", "off"],
-                    help="on: batches of at most 128 token rows run as one persistent kernel")
+    ap.add_argument("--small-batch", default="on", choices=["on", "off"],
+                    help="off: batches of at most 128 token rows also take the per-layer kernels")
     ap.add_argument("--all-configs", action="store_true",
                     help="one JSON line per workload of the suite (packed and padded b256, b1_T64 stream and graph)")
     args = ap.parse_args()

@@ -235,13 +235,13 @@ int albert_last_forward_launches(const albert_handle *h);
  * albert_forward, nseq*max_len <= 128 for albert_forward_varlen) and the handle
  * is bf16 with one weight set (n_groups == 1) and n_exec >= 1, everything after
  * the embedding runs in ONE persistent kernel: a cooperative grid that walks
- * the layer's steps as phases separated by grid barriers, with the FFN fused
- * per 64-wide hidden chunk (GELU(X1 W1^T + b1) kept on chip and multiplied
- * straight into W2), instead of ~65 per-layer launches ("ALBERT: How Kokoro's
+ * the layer's steps as phases separated by grid barriers (Q|K|V, attention,
+ * out-projection, FFN up, FFN down, each over all SMs of the grid, with the
+ * intermediate tiles in L2), instead of ~65 per-layer launches ("ALBERT: How Kokoro's
  * Phoneme Encoder Works", section "Inside One Real ALBERT Layer", steps 2-6,
  * and "2. Cross-layer parameter sharing").  Same results within the stated
- * tolerances; deterministic.  enable: 1 uses it when it applies, 0 (default)
- * always runs the per-layer kernels.  Other values: ALBERT_ERR_CONFIG. */
+ * tolerances; deterministic.  enable: 1 (default) uses it when it applies,
+ * 0 always runs the per-layer kernels.  Other values: ALBERT_ERR_CONFIG. */
 int albert_set_small_batch_kernel(albert_handle *h, int enable);
 
 /* ---- per-kernel timing (optional) ----

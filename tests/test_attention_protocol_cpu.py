@@ -86,10 +86,13 @@ class Sim:
 # ----------------------------------------------------------------- short kernel --
 # One item per (sequence, head), four TMEM buffers, Q/K and V stages with the
 # buffer's index; a stage is released by the S (Q/K) or O (V) completion of the
-# item four back.  Two softmax groups take alternate items.  Two issuing
-# threads: one issues the S products in item order, the other the O products.
-# planted: True reuses a V stage one item early; "s_early" issues S into a
-# buffer without waiting for the output warps to have read its previous O.
+# item four back.  The producer loads Q/K of every item and V of items 0..3; one
+# output warp loads V of item i + 4 once it has seen O of item i complete.  Two
+# softmax groups take alternate items.  Two issuing threads: one issues the S
+# products in item order, the other the O products.
+# planted: True loads V of item i + 4 before O of item i is complete; "s_early"
+# issues S into a buffer without waiting for the output warps to have read its
+# previous O.
 def short_kernel(n_items, seed, planted=False):
     NB = 4
     sim = Sim(seed)
@@ -98,20 +101,19 @@ def short_kernel(n_items, seed, planted=False):
             sim.bar(f"{n}{i}", c)
     tmem = {}  # buffer -> item whose S/P/O it holds
 
+    def load_v(n):
+        if n >= NB:
+            assert sim.bars[f"o_full{n % NB}"].phase > (n - NB) // NB, "V stage reused before O read it"
+        sim.commit(f"v_full{n % NB}", ("v", n))
+
     def producer():
-        nq = nv = 0
-        while nv < n_items:
-            if nq < n_items and sim.bars[f"s_full{nq % NB}"].test(((nq // NB) & 1) ^ 1):
-                if nq >= NB:
-                    assert sim.bars[f"s_full{nq % NB}"].phase > (nq - NB) // NB, "Q/K stage reused before S read it"
-                sim.commit(f"qk_full{nq % NB}", ("qk", nq))
-                nq += 1
-            # planted: the V stage is reused without waiting for the O product of the item four back
-            if nv < nq and (planted or sim.bars[f"o_full{nv % NB}"].test(((nv // NB) & 1) ^ 1)):
-                if nv >= NB:
-                    assert sim.bars[f"o_full{nv % NB}"].phase > (nv - NB) // NB, "V stage reused before O read it"
-                sim.commit(f"v_full{nv % NB}", ("v", nv))
-                nv += 1
+        for nq in range(n_items):
+            yield from sim.wait(f"s_full{nq % NB}", ((nq // NB) & 1) ^ 1)
+            if nq >= NB:
+                assert sim.bars[f"s_full{nq % NB}"].phase > (nq - NB) // NB, "Q/K stage reused before S read it"
+            sim.commit(f"qk_full{nq % NB}", ("qk", nq))
+            if nq < NB:
+                load_v(nq)
             yield
 
     def mma_s():
@@ -145,7 +147,11 @@ def short_kernel(n_items, seed, planted=False):
     def output(q):
         for i in range(n_items):
             tb = i % NB
+            if planted is True and q == 2 and i + NB < n_items:
+                load_v(i + NB)  # the planted mistake: before O of item i is complete
             yield from sim.wait(f"o_full{tb}", (i // NB) & 1, ("o", i))
+            if planted is not True and q == 2 and i + NB < n_items:
+                load_v(i + NB)
             yield from sim.wait(f"p_full{tb}", (i // NB) & 1, ("p", i))
             yield
             sim.bars[f"o_empty{tb}"].arrive(("e", i))

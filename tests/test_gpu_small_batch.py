@@ -1,6 +1,6 @@
 """The small-batch path: at most 128 token rows run as ONE persistent kernel
-after the embedding (phases separated by grid barriers, the FFN fused per
-hidden chunk with the chunk kept on chip).  Parity against the fp64 oracle on
+after the embedding (the layer's steps as phases separated by grid barriers).
+Parity against the fp64 oracle on
 every valid row, agreement with the per-layer kernels, the varlen entry, error
 and timeout paths, determinism and the launch count."""
 import time

@@ -117,11 +117,10 @@ struct albert_handle {
     // embedding in one persistent kernel; its own statistics, FFN partial sums,
     // barrier counter and {64, 64}-box tensor maps
     bool small_ok = false;       // the handle's configuration allows it
-    bool small_enabled = false;  // albert_set_small_batch_kernel
+    bool small_enabled = true;   // albert_set_small_batch_kernel
     float2 *sst1 = nullptr, *sst2 = nullptr;
-    float *spart = nullptr;
     int *sbar = nullptr;
-    CUtensorMap sm_E, sm_X, sm_C, sm_X1, sm_Z, sm_win, sm_wqkv, sm_wo, sm_w1, sm_w2, sm_wout, sm_part;
+    CUtensorMap sm_E, sm_X, sm_C, sm_X1, sm_Z, sm_H, sm_win, sm_wqkv, sm_wo, sm_w1, sm_w2, sm_wout;
     int last_launches = 0;       // kernel launches of the last forward
 
     // bounded waits inside the kernels: limit (0 = the kernels' default, 2 s) and,
@@ -338,14 +337,13 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
         const auto &W = h->grp[0];
         const auto &E1 = h->ex[c.n_exec > 1 ? 1 : 0];
         SmallFwdArgs s{};
-        s.tmE = h->sm_E; s.tmX = h->sm_X; s.tmC = h->sm_C; s.tmX1 = h->sm_X1; s.tmZ = h->sm_Z;
+        s.tmE = h->sm_E; s.tmX = h->sm_X; s.tmC = h->sm_C; s.tmX1 = h->sm_X1; s.tmZ = h->sm_Z; s.tmH = h->sm_H;
         s.tmQKV = h->tm_QKV; s.tmQKV64 = h->tm_QKV64;
         s.tmWin = h->sm_win; s.tmWqkv = h->sm_wqkv; s.tmWo = h->sm_wo; s.tmW1 = h->sm_w1; s.tmW2 = h->sm_w2;
         s.tmWout = c.out_dim > 0 ? h->sm_wout : h->sm_wo;  // (unused without a final projection)
-        s.tmPart = h->sm_part;
         s.X = static_cast<bf16 *>(h->X); s.QKV = static_cast<bf16 *>(h->QKV); s.C = static_cast<bf16 *>(h->C);
-        s.X1 = static_cast<bf16 *>(h->X1); s.Z = static_cast<bf16 *>(h->Z);
-        s.st1 = h->sst1; s.st2 = h->sst2; s.part = h->spart;
+        s.X1 = static_cast<bf16 *>(h->X1); s.Z = static_cast<bf16 *>(h->Z); s.H = static_cast<bf16 *>(h->H);
+        s.st1 = h->sst1; s.st2 = h->sst2;
         s.b_in = h->b_in;
         s.bqkv0 = W.bqkv; s.bqkv = E1.c_qkv; s.s_qkv = E1.s_qkv;
         s.bo0 = W.bo; s.bo = E1.bias_o2;
@@ -713,19 +711,16 @@ int create_impl(albert_handle *h, const albert_weights *w) {
             const auto &gp = h->grp[0];
             if ((rc = dev_alloc(h, (void **)&h->sst1, kSmallMaxRows * kSmallParts * sizeof(float2)))) return rc;
             if ((rc = dev_alloc(h, (void **)&h->sst2, kSmallMaxRows * kSmallParts * sizeof(float2)))) return rc;
-            if ((rc = dev_alloc(h, (void **)&h->spart, (size_t)(kFfn / 64) * kSmallMaxRows * kHidden * sizeof(float))))
-                return rc;
             if ((rc = dev_alloc(h, (void **)&h->sbar, sizeof(int)))) return rc;
             if (make_tmap_bf16(&h->sm_E, h->E, R, kEmb, 64) || make_tmap_bf16(&h->sm_X, h->X, R, kHidden, 64) ||
                 make_tmap_bf16(&h->sm_C, h->C, R, kHidden, 64) || make_tmap_bf16(&h->sm_X1, h->X1, R, kHidden, 64) ||
-                make_tmap_bf16(&h->sm_Z, h->Z, R, kHidden, 64) ||
+                make_tmap_bf16(&h->sm_Z, h->Z, R, kHidden, 64) || make_tmap_bf16(&h->sm_H, h->H, R, kFfn, 64) ||
                 make_tmap_bf16(&h->sm_win, h->w_in, kHidden, kEmb, 64) ||
                 make_tmap_bf16(&h->sm_wqkv, gp.wqkv, kQKV, kHidden, 64) ||
-                make_tmap_bf16(&h->sm_wo, gp.wo, kHidden, kHidden, 64) ||
+                make_tmap_bf16(&h->sm_wo, gp.wo, kHidden, kHidden, 32) ||
                 make_tmap_bf16(&h->sm_w1, gp.w1, kFfn, kHidden, 64) ||
-                make_tmap_bf16(&h->sm_w2, gp.w2, kHidden, kFfn, 64) ||
-                (O && make_tmap_bf16(&h->sm_wout, h->w_out, O, kHidden, 64)) ||
-                make_tmap_f32_tile32(&h->sm_part, h->spart, (uint64_t)(kFfn / 64) * kSmallMaxRows, kHidden))
+                make_tmap_bf16(&h->sm_w2, gp.w2, kHidden, kFfn, 32) ||
+                (O && make_tmap_bf16(&h->sm_wout, h->w_out, O, kHidden, 64)))
                 return ALBERT_ERR_CUDA;
             h->small_ok = true;
         }

@@ -7,13 +7,18 @@
 //     C_h = softmax(Q_h K_h^T / sqrt(64) + mask) V_h,
 // key u of sequence b takes part iff u < L_b, every query sees both sides.
 //
-// One work item = (sequence, head), all L_b <= 128 queries and keys at once:
-//   warp 0      : TMA producer, an event loop over two rings of shared
-//                 stages: the head's Q and K tiles (128 or 64 rows x 64,
-//                 128-byte swizzle) from the packed [rows, 3*768] buffer into
-//                 one, its V tile into the other.  A Q/K stage is free again
-//                 as soon as the S product has read it, so Q/K loads run well
-//                 ahead; a V stage lives until the O product;
+// One work item = (sequence, head), all L_b <= 128 queries and keys at once.
+// The (start, length) of every item of the CTA is read into shared memory
+// once, before the roles start (a global load per item on the issuing
+// threads' path cost about as much as the item itself).
+//   warp 0      : TMA producer of the head's Q and K tiles (128 or 64 rows x
+//                 64, 128-byte swizzle) from the packed [rows, 3*768] buffer
+//                 into a ring of stages; a Q/K stage is free again as soon as
+//                 the S product has read it, so Q/K loads run well ahead.  It
+//                 also loads the V tiles of the first four items; the V tile
+//                 of item n + 4 is loaded by the output group as soon as the O
+//                 product of item n, the last reader of that V stage, is
+//                 complete;
 //   warp 1      : tcgen05.mma issuer of the score products S = Q K^T (M=128,
 //                 N=128 or 64, K=64) into a TMEM buffer, item after item;
 //   warp 14     : tcgen05.mma issuer of the output products O = P V (M=128,
@@ -49,7 +54,8 @@ constexpr int NV = 4;                          // V stages (1 tile each)
 constexpr int NBUF = 4;                        // TMEM item buffers (128 columns each)
 constexpr int ATC_THREADS = 32 * 15;
 constexpr int ATC_O_WARP = 14;                 // issuer of the O = P V products
-constexpr int ATC_SMEM = 1024 + (2 * NQK + NV) * TILE + NBUF * TROWS * 4 + 512;
+constexpr int ATC_ITEM_CAP = 512;              // items whose (start, length) are kept in shared memory
+constexpr int ATC_SMEM = 1024 + (2 * NQK + NV) * TILE + NBUF * TROWS * 4 + ATC_ITEM_CAP * 8 + 512;
 constexpr uint32_t TM_O = 64;                  // O's first column within an item buffer
 // Item n uses Q/K stage, V stage and TMEM buffer n % 4 alike, so a Q/K stage is
 // free when the S product of the item four back completes (s_full) and a V
@@ -68,6 +74,8 @@ struct AttSmem {
     int *misc;
     int *qk_len, *v_len;                       // length of the item a stage holds
     float *inv_sum;                            // [NBUF][TROWS]
+    int2 *item;                                // [ATC_ITEM_CAP] (start, length) of the CTA's items
+    int *n_issued;                             // [0] Q/K, [1] V loads issued (read by the teardown)
 };
 
 __device__ __forceinline__ AttSmem att_carve(uint8_t *raw) {
@@ -76,7 +84,8 @@ __device__ __forceinline__ AttSmem att_carve(uint8_t *raw) {
     s.qk = p;
     s.v = p + 2 * NQK * TILE;
     s.inv_sum = reinterpret_cast<float *>(s.v + NV * TILE);
-    uint64_t *b = reinterpret_cast<uint64_t *>(s.v + NV * TILE + NBUF * TROWS * 4);
+    s.item = reinterpret_cast<int2 *>(s.v + NV * TILE + NBUF * TROWS * 4);
+    uint64_t *b = reinterpret_cast<uint64_t *>(s.item + ATC_ITEM_CAP);
     s.qk_full = b;
     s.v_full = b + 2 * NQK;
     s.s_full = b + 2 * NQK + 2 * NV;
@@ -91,7 +100,26 @@ __device__ __forceinline__ AttSmem att_carve(uint8_t *raw) {
     s.misc = reinterpret_cast<int *>(u + 2);
     s.qk_len = s.misc + 2;
     s.v_len = s.qk_len + NQK;
+    s.n_issued = s.v_len + NV;
     return s;
+}
+
+// (start, length) of the CTA's item j (id = blockIdx.x + j * gridDim.x)
+__device__ __forceinline__ int2 item_info(const AttSmem &sm, int j, const int *seq_start, const int *seq_len) {
+    if (j < ATC_ITEM_CAP) return sm.item[j];
+    const int b = (blockIdx.x + j * gridDim.x) / kHeads;
+    return make_int2(__ldg(seq_start + b), __ldg(seq_len + b));
+}
+
+// TMA load of the V tile of the CTA's item n into V stage n % NV (one thread).
+__device__ __forceinline__ void issue_v(const AttSmem &sm, int n, int2 it, const CUtensorMap *tmQKV,
+                                        const CUtensorMap *tmQKV64) {
+    const int h = (blockIdx.x + n * gridDim.x) % kHeads;
+    const int st = n % NV;
+    sm.v_len[st] = it.y;  // read by the O issuer once the stage is full
+    const uint32_t fb = smem_u32(&sm.v_full[st]);
+    mbar_arrive_expect_tx(fb, it.y <= 64 ? TILE / 2 : TILE);
+    tma_load_2d(smem_u32(sm.v + st * TILE), it.y <= 64 ? tmQKV64 : tmQKV, fb, 2 * kHidden + h * kHeadDim, it.x);
 }
 
 __global__ void __launch_bounds__(ATC_THREADS, 1)
@@ -120,6 +148,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
         mbar_init(smem_u32(sm.drain), 1);
         mbar_init(smem_u32(sm.drain_o), 1);
         fence_mbar_init();
+        sm.n_issued[0] = sm.n_issued[1] = sm.n_issued[2] = 0;
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmQKV);
@@ -127,6 +156,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     }
     __syncthreads();
     if (sm.misc[0] != 0) return;  // an earlier kernel of this forward failed
+    const int total = nseq * kHeads;  // item id = b * 12 + h
+    // items of this CTA: id = blockIdx.x + j * gridDim.x, j < n_items
+    const int n_items = (int)blockIdx.x < total ? (total - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    for (int j = threadIdx.x; j < n_items && j < ATC_ITEM_CAP; j += blockDim.x) {
+        const int b = (blockIdx.x + j * gridDim.x) / kHeads;
+        sm.item[j] = make_int2(__ldg(seq_start + b), __ldg(seq_len + b));
+    }
     if (warp == 1) {
         tmem_alloc(smem_u32(sm.tmem_slot), NBUF * TROWS);
         tmem_relinquish();
@@ -135,69 +171,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *sm.tmem_slot;
-    const int total = nseq * kHeads;  // item id = b * 12 + h
-
-    int n_items = 0;  // items of this CTA: id = blockIdx.x + j * gridDim.x
-    for (int id = blockIdx.x; id < total; id += gridDim.x) ++n_items;
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer --
-        // Event loop: Q/K of item nq into its ring, V of item nv (< nq) into its
-        // ring, whichever has a free stage.
+        // Q/K of item n into stage n % 4 once the S product of item n - 4 has read
+        // it; the V tiles of items 0..3 alongside.
         if (lane == 0) {
-            int nq = 0, nv = 0;
-            unsigned long long t_idle = 0;
-            unsigned polls = 0;
-            while (nv < n_items) {
-                bool progress = false;
-                if (nq < n_items) {
-                    const int st = nq % NQK;
-                    // the stage is free once S of item nq - NQK has completed
-                    if (mbar_test(smem_u32(&sm.s_full[st]), ((nq / NQK) & 1) ^ 1)) {
-                        const int id = blockIdx.x + nq * gridDim.x, b = id / kHeads, h = id % kHeads;
-                        const int start = __ldg(seq_start + b), L = __ldg(seq_len + b);
-                        sm.qk_len[st] = L;  // read by the issuer once the stage is full
-                        // sequences of at most 64 tokens move 64-row tiles
-                        const CUtensorMap *tm = L <= 64 ? &tmQKV64 : &tmQKV;
-                        const uint32_t dst = smem_u32(sm.qk + st * 2 * TILE);
-                        const uint32_t fb = smem_u32(&sm.qk_full[st]);
-                        mbar_arrive_expect_tx(fb, L <= 64 ? TILE : 2 * TILE);
-                        tma_load_2d(dst, tm, fb, h * kHeadDim, start);
-                        tma_load_2d(dst + TILE, tm, fb, kHidden + h * kHeadDim, start);
-                        ++nq;
-                        progress = true;
-                    }
+            int nq = 0;
+            for (; nq < n_items; ++nq) {
+                const int st = nq % NQK;
+                if (!mbar_wait(smem_u32(&sm.s_full[st]), ((nq / NQK) & 1) ^ 1, sm.abort_flag)) break;
+                const int2 it = item_info(sm, nq, seq_start, seq_len);
+                const int h = (blockIdx.x + nq * gridDim.x) % kHeads;
+                sm.qk_len[st] = it.y;  // read by the issuer once the stage is full
+                // sequences of at most 64 tokens move 64-row tiles
+                const CUtensorMap *tm = it.y <= 64 ? &tmQKV64 : &tmQKV;
+                const uint32_t dst = smem_u32(sm.qk + st * 2 * TILE);
+                const uint32_t fb = smem_u32(&sm.qk_full[st]);
+                mbar_arrive_expect_tx(fb, it.y <= 64 ? TILE : 2 * TILE);
+                tma_load_2d(dst, tm, fb, h * kHeadDim, it.x);
+                tma_load_2d(dst + TILE, tm, fb, kHidden + h * kHeadDim, it.x);
+                sm.n_issued[0] = nq + 1;
+                if (nq < NV) {
+                    issue_v(sm, nq, it, &tmQKV, &tmQKV64);
+                    sm.n_issued[1] = nq + 1;
                 }
-                if (nv < nq) {
-                    const int st = nv % NV;
-                    // the stage is free once O of item nv - NV has completed
-                    if (mbar_test(smem_u32(&sm.o_full[st]), ((nv / NV) & 1) ^ 1)) {
-                        const int id = blockIdx.x + nv * gridDim.x, b = id / kHeads, h = id % kHeads;
-                        const int start = __ldg(seq_start + b), L = __ldg(seq_len + b);
-                        sm.v_len[st] = L;
-                        const CUtensorMap *tm = L <= 64 ? &tmQKV64 : &tmQKV;
-                        const uint32_t fb = smem_u32(&sm.v_full[st]);
-                        mbar_arrive_expect_tx(fb, L <= 64 ? TILE / 2 : TILE);
-                        tma_load_2d(smem_u32(sm.v + st * TILE), tm, fb, 2 * kHidden + h * kHeadDim, start);
-                        ++nv;
-                        progress = true;
-                    }
-                }
-                if (progress) {
-                    t_idle = 0;
-                } else if ((++polls & 255) == 0) {  // the timer read is slow: not on every poll
-                    if (*sm.abort_flag) break;
-                    const unsigned long long now = globaltimer_ns();
-                    if (t_idle == 0) t_idle = now;
-                    else if (now - t_idle > wait_limit()) { *sm.abort_flag = 1; break; }
-                }
-            }
-            if (*sm.abort_flag) {
-                // loads still in flight complete before the CTA's shared memory goes away
-                for (int j = nq > NQK ? nq - NQK : 0; j < nq; ++j)
-                    mbar_wait_drain(smem_u32(&sm.qk_full[j % NQK]), (j / NQK) & 1);
-                for (int j = nv > NV ? nv - NV : 0; j < nv; ++j)
-                    mbar_wait_drain(smem_u32(&sm.v_full[j % NV]), (j / NV) & 1);
             }
         }
     } else if (warp == 1) {
@@ -262,7 +260,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
             const int tb = i % NBUF;
             const uint32_t ph = (i / NBUF) & 1;
             const uint32_t srow = trow + tb * TROWS;
-            const int L = __ldg(seq_len + id / kHeads);
+            const int L = item_info(sm, i, seq_start, seq_len).y;
             const int nch = (L + 31) >> 5;  // 32-key chunks holding valid keys
             const bool live = quad * 32 < L;  // some row of this warp is a real query
             bool got = mbar_wait(smem_u32(&sm.s_full[tb]), ph, sm.abort_flag);
@@ -344,8 +342,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
         for (int id = blockIdx.x; id < total; id += gridDim.x, ++i) {
             const int tb = i % NBUF;
             const uint32_t ph = (i / NBUF) & 1;
-            const int b = id / kHeads, h = id % kHeads;
-            const int L = __ldg(seq_len + b), start = __ldg(seq_start + b);
+            const int h = id % kHeads;
+            const int2 it = item_info(sm, i, seq_start, seq_len);
+            const int L = it.y, start = it.x;
             const bool live = quad * 32 < L;
             // p_full (complete before O is) makes the softmax's 1/sum visible here
             bool got = mbar_wait(smem_u32(&sm.o_full[tb]), ph, sm.abort_flag) &&
@@ -353,6 +352,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
             got = __all_sync(0xffffffffu, got);
             if (!got) break;
             tc_fence_after();
+            // O of item i is complete: its V stage takes the V tile of item i + 4
+            if (warp == 10 && lane == 0 && i + NV < n_items) {
+                issue_v(sm, i + NV, item_info(sm, i + NV, seq_start, seq_len), &tmQKV, &tmQKV64);
+                sm.n_issued[2] = i + 1;
+            }
             uint32_t o[2][32];
             float inv = 0.f;
             if (live) {
@@ -379,6 +383,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     }
 
     __syncthreads();
+    if (threadIdx.x == 0 && *sm.abort_flag) {
+        // loads still in flight land before the CTA's shared memory goes away (the
+        // last four issued of each ring; the V tiles issued are items 0..last)
+        const int nq = sm.n_issued[0];
+        for (int j = nq > NQK ? nq - NQK : 0; j < nq; ++j)
+            mbar_wait_drain(smem_u32(&sm.qk_full[j % NQK]), (j / NQK) & 1);
+        const int nv = sm.n_issued[2] > 0 ? NV + sm.n_issued[2] : sm.n_issued[1];
+        for (int j = nv > NV ? nv - NV : 0; j < nv; ++j)
+            mbar_wait_drain(smem_u32(&sm.v_full[j % NV]), (j / NV) & 1);
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, NBUF * TROWS);

@@ -20,35 +20,31 @@
 //   attention   one job per (sequence, head): S = Q K^T on tcgen05 into TMEM,
 //               softmax by one thread per query row, P written back to TMEM
 //               as bf16, O = P V (P from TMEM, V from shared memory);
-//   out-proj    12 jobs: a 64-column tile of z1 = C Wo^T + bo + residual,
+//   out-proj    24 jobs: a 32-column tile of z1 = C Wo^T + bo + residual,
 //               stored as z1 * gamma1 with the tile's per-row (mean, M2);
-//   FFN         32 jobs, the FFN fused per hidden chunk: job j computes
-//               H_j = GELU(LN1(z1) W1[64j..64j+63]^T + b1) (K = 768) into
-//               TMEM, keeps it on chip (bf16, shared memory, in the layout
-//               of a tensor-core A operand) and multiplies it straight into
-//               its partial of the down projection, H_j W2[:, 64j..]^T (three
-//               256-column products), stored as fp32 partial sums;
-//   reduce      per (row, 64-column slice): z2 = sum_j partial_j + b2 + LN1(z1),
-//               stored as z2 * gamma2 with its (mean, M2);
+//   FFN up      32 jobs: a 64-column tile of H = GELU(LN1(z1) W1^T + b1);
+//   FFN down    24 jobs: a 32-column tile of z2 = H W2^T + b2 + LN1(z1)
+//               (all of K = 2048 in one job), stored as z2 * gamma2 with its
+//               per-row (mean, M2);
 //   final       8 jobs: a 64-column tile of Y = LN2(z2) W_out^T + b_out,
 //               scattered to the caller's rows (or LN2(z2) itself).
 // The LayerNorms are applied where their input is consumed, as in the rest of
-// the library: a consumer merges the twelve 64-column (mean, M2) partials of a
-// row and uses LN(z) W^T = rstd (z gamma) W^T - rstd mu (W gamma) + W beta + b
-// with W gamma and W beta + b folded once per weight set.  The partial sums of
-// the down projection are reduced in a fixed order: the result does not
-// depend on scheduling.
+// the library: a consumer merges the twenty-four 32-column (mean, M2) partials
+// of a row and uses LN(z) W^T = rstd (z gamma) W^T - rstd mu (W gamma) + W beta + b
+// with W gamma and W beta + b folded once per weight set.  Every output element
+// is one job's sum over all of K in a fixed order: the result does not depend
+// on scheduling.
 //
 // Roles inside a CTA (192 threads): warp 0 lane 0 issues TMA loads into a
 // 3-stage ring of 64 KB stages (a stage carries up to four 64-wide K blocks of
-// both operands, so a 64-column tile with K = 768 and at most 64 rows has all
-// of K in flight at once: the phases are bound by load latency, not
-// bandwidth), warp 1 lane 0 allocates TMEM and issues tcgen05.mma, warps
-// 2..5 (one per TMEM lane quadrant, one thread per tile row) run epilogues and
-// the softmax; every warp takes rows of the reduce phase.  Every wait is
-// bounded (mbarriers and the grid barrier alike); on expiry the kernel records
-// ALBERT_ERR_TIMEOUT, every CTA leaves at its next grid barrier, and in-flight
-// copies and products are drained before TMEM is freed.
+// both operands, so a tile with K = 768 and at most 64 rows has all of K in
+// flight at once: the phases are bound by load latency, not bandwidth), warp 1
+// lane 0 allocates TMEM and issues tcgen05.mma, warps 2..5 (one per TMEM lane
+// quadrant, one thread per tile row) run epilogues and the softmax; every warp
+// takes rows of the hidden-state output.  Every wait is bounded (mbarriers and
+// the grid barrier alike); on expiry the kernel records ALBERT_ERR_TIMEOUT,
+// every CTA leaves at its next grid barrier, and in-flight copies and products
+// are drained before TMEM is freed.
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
@@ -59,20 +55,17 @@ constexpr int SB_THREADS = 192;
 constexpr int SB_NS = 3;                      // ring stages
 constexpr int SB_BOX = 64 * 64 * 2;           // one {64 cols, 64 rows} bf16 box, 128-byte swizzle: 8 KB
 constexpr int SB_A_BYTES = 4 * SB_BOX;        // A: up to four 64-row K blocks (two of 128 rows)
-constexpr int SB_B_BYTES = 4 * SB_BOX;        // B: up to four 64-row K blocks, or one of 256 rows
-constexpr int SB_H_BYTES = 2 * SB_BOX;        // FFN hidden chunk, 128 rows x 64 bf16
-constexpr int SB_STG_BYTES = 4 * 32 * 32 * 4; // FFN partial sums: a 32 x 32 fp32 staging tile per epilogue warp
-constexpr int SB_SMEM = 1024 + SB_NS * (SB_A_BYTES + SB_B_BYTES) + SB_H_BYTES + SB_STG_BYTES + 128 * 4 + 512;
+constexpr int SB_B_BYTES = 4 * SB_BOX;        // B: up to four K blocks of 64 (or 32) rows
+constexpr int SB_SMEM = 1024 + SB_NS * (SB_A_BYTES + SB_B_BYTES) + 128 * 4 + 512;
 static_assert(SB_SMEM <= 232448, "shared memory per CTA");
-constexpr int SB_PARTS = kSmallParts;         // 64-column statistics slices of a 768-wide row
-constexpr int SB_CHUNKS = kFfn / 64;          // FFN hidden chunks
+constexpr int SB_PARTS = kSmallParts;         // 32-column statistics slices of a 768-wide row
 constexpr uint32_t SB_TM_O = 64;              // attention: O's columns within the item's TMEM columns
 
 struct SbSmem {
-    uint8_t *a, *b, *h, *stg;
+    uint8_t *a, *b;
     float *inv_sum;                           // [128] attention: 1 / row sum
     uint64_t *full, *empty;                   // [SB_NS]
-    uint64_t *acc_full, *acc_empty, *h_ready, *drain;
+    uint64_t *acc_full, *acc_empty, *drain;
     uint32_t *tmem_slot;
     volatile int *abort_flag;
     int *misc;                                // [0] rows, [1] status at entry
@@ -83,17 +76,14 @@ __device__ __forceinline__ SbSmem sb_carve(uint8_t *raw) {
     uint8_t *p = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
     s.a = p;
     s.b = p + SB_NS * SB_A_BYTES;
-    s.h = s.b + SB_NS * SB_B_BYTES;
-    s.stg = s.h + SB_H_BYTES;
-    s.inv_sum = reinterpret_cast<float *>(s.stg + SB_STG_BYTES);
+    s.inv_sum = reinterpret_cast<float *>(s.b + SB_NS * SB_B_BYTES);
     uint64_t *bars = reinterpret_cast<uint64_t *>(s.inv_sum + 128);
     s.full = bars;
     s.empty = bars + SB_NS;
     s.acc_full = bars + 2 * SB_NS;
     s.acc_empty = s.acc_full + 1;
-    s.h_ready = s.acc_full + 2;
-    s.drain = s.acc_full + 3;
-    uint32_t *u = reinterpret_cast<uint32_t *>(s.acc_full + 4);
+    s.drain = s.acc_full + 2;
+    uint32_t *u = reinterpret_cast<uint32_t *>(s.acc_full + 3);
     s.tmem_slot = u;
     s.abort_flag = reinterpret_cast<volatile int *>(u + 1);
     s.misc = reinterpret_cast<int *>(u + 2);
@@ -102,8 +92,8 @@ __device__ __forceinline__ SbSmem sb_carve(uint8_t *raw) {
 
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
-// (mean, rstd) of a 768-wide row from its twelve 64-column (mean, M2) partials
-// (Chan's merge of equal-size groups).
+// (mean, rstd) of a 768-wide row from its twenty-four 32-column (mean, M2)
+// partials (Chan's merge of equal-size groups).
 __device__ __forceinline__ void merge_parts(const float2 *q, float eps, float &mu, float &rstd) {
     float2 v[SB_PARTS];
 #pragma unroll
@@ -116,7 +106,7 @@ __device__ __forceinline__ void merge_parts(const float2 *q, float eps, float &m
 #pragma unroll
     for (int i = 0; i < SB_PARTS; ++i) {
         const float d = v[i].x - m;
-        m2 += v[i].y + 64.0f * d * d;
+        m2 += v[i].y + 32.0f * d * d;
     }
     mu = m;
     rstd = rsqrtf(m2 * (1.0f / kHidden) + eps);
@@ -132,8 +122,9 @@ __device__ bool grid_sync(int *ctr, int &epoch, int *status, volatile int *abort
     if (threadIdx.x == 0) {
         ++epoch;
         if (*abort) set_status(status, kStatusTimeout);
-        __threadfence();
-        atomicAdd(ctr, 1);
+        // release at GPU scope: the CTA's stores (ordered before by the CTA barrier)
+        // are visible to any CTA that acquires the count
+        red_release_gpu_add(ctr, 1);
         const int target = epoch * (int)gridDim.x;
         unsigned long long t0 = 0;
         unsigned polls = 0;
@@ -148,7 +139,8 @@ __device__ bool grid_sync(int *ctr, int &epoch, int *status, volatile int *abort
                 }
             }
         }
-        __threadfence();
+        // this thread issues the CTA's TMA loads: the other CTAs' stores it has
+        // acquired are ordered before them
         fence_proxy_async_global();
     }
     __syncthreads();
@@ -156,29 +148,24 @@ __device__ bool grid_sync(int *ctr, int &epoch, int *status, volatile int *abort
 }
 
 // ---------------------------------------------------------------- phases ----
-enum SbPhase : int { kPhIn = 0, kPhQKV, kPhAttn, kPhOut, kPhFfn, kPhReduce, kPhFinal };
+enum SbPhase : int { kPhIn = 0, kPhQKV, kPhAttn, kPhOut, kPhUp, kPhDown, kPhFinal };
+constexpr int SB_PER_EXEC = 5;  // phases per execution of the shared layer
 
 __device__ __forceinline__ int phase_jobs(int ph, const SmallFwdArgs &p) {
     switch (ph) {
         case kPhIn: return kHidden / 64;
         case kPhQKV: return kQKV / 64;
         case kPhAttn: return p.nseq * kHeads;
-        case kPhOut: return kHidden / 64;
-        case kPhFfn: return SB_CHUNKS;
+        case kPhOut: return kHidden / 32;
+        case kPhUp: return kFfn / 64;
+        case kPhDown: return kHidden / 32;
         case kPhFinal: return p.out_dim > 0 ? p.out_dim / 64 : 0;
     }
     return 0;
 }
-
-// Loads of one job, in the order the MMA issuer consumes them.  Each load step
-// fills one ring stage with nk consecutive 64-wide K blocks; K block j holds
-// a_boxes boxes of 64 rows of A at j * a_boxes * 8 KB and b_boxes boxes of 64
-// rows of B at j * b_boxes * 8 KB.  The FFN's second products load B only.
-struct LoadStep {
-    const CUtensorMap *ta, *tb;
-    int a_boxes, b_boxes, nk;
-    int ax, ay, bx, by;       // coordinates of the first boxes (x = column, y = row)
-};
+// output columns per job of a GEMM phase, and its K
+__device__ __forceinline__ int phase_n(int ph) { return ph == kPhOut || ph == kPhDown ? 32 : 64; }
+__device__ __forceinline__ int phase_k(int ph) { return ph == kPhIn ? kEmb : ph == kPhDown ? kFfn : kHidden; }
 
 __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_constant__ SmallFwdArgs p) {
     extern __shared__ uint8_t smem_raw[];
@@ -194,7 +181,6 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
         }
         mbar_init(smem_u32(sm.acc_full), 1);
         mbar_init(smem_u32(sm.acc_empty), 4);  // one arrive per epilogue warp
-        mbar_init(smem_u32(sm.h_ready), 4);
         mbar_init(smem_u32(sm.drain), 1);
         fence_mbar_init();
         sm.misc[0] = *reinterpret_cast<const volatile int *>(p.n_rows);
@@ -206,6 +192,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
         prefetch_tmap(&p.tmC);
         prefetch_tmap(&p.tmX1);
         prefetch_tmap(&p.tmZ);
+        prefetch_tmap(&p.tmH);
         prefetch_tmap(&p.tmQKV);
         prefetch_tmap(&p.tmQKV64);
         prefetch_tmap(&p.tmWin);
@@ -214,7 +201,6 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
         prefetch_tmap(&p.tmW1);
         prefetch_tmap(&p.tmW2);
         prefetch_tmap(&p.tmWout);
-        prefetch_tmap(&p.tmPart);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(sm.tmem_slot), 512);
@@ -229,128 +215,90 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
     const bool skip = sm.misc[1] != 0 || M < 1 || M > 128;
     const int a_boxes = M > 64 ? 2 : 1;
     const int kb_step = M > 64 ? 2 : 4;  // 64-wide K blocks per ring stage in the GEMM phases
-    const int n_phases = 1 + 5 * p.n_exec + 1;
+    const int n_phases = 1 + SB_PER_EXEC * p.n_exec + 1;
 
     int epoch = 0;
     // ring and accumulator progress, advanced identically by the roles that use them
     uint32_t ring = 0;   // load steps issued (producer) / consumed (MMA issuer)
     uint32_t units = 0;  // accumulations committed (MMA issuer) / read (epilogue)
-    uint32_t hcnt = 0;   // FFN hidden chunks handed over through shared memory
     bool ok = !skip;
 
     for (int phi = 0; phi < n_phases && ok; ++phi) {
-        const int ph = phi == 0 ? kPhIn : phi == n_phases - 1 ? kPhFinal : 1 + (phi - 1) % 5;
-        const int l = phi == 0 ? -1 : (phi - 1) / 5;  // execution of the shared layer
+        const int ph = phi == 0 ? kPhIn : phi == n_phases - 1 ? kPhFinal : 1 + (phi - 1) % SB_PER_EXEC;
+        const int l = phi == 0 ? -1 : (phi - 1) / SB_PER_EXEC;  // execution of the shared layer
         const int njobs = phase_jobs(ph, p);
+        const int N = phase_n(ph);
+        // one ring stage per nk 64-wide K blocks (the in-projection's two in one stage)
+        const int nk = ph == kPhIn ? kEmb / 64 : kb_step;
+        const int nsteps = (phase_k(ph) / 64) / nk;
 
-        if (ph == kPhReduce || (ph == kPhFinal && p.out_dim == 0)) {
-            // ------------------------------------------------ row phases (all warps) --
-            // item = (row, 64-column slice); one warp per item, two columns per lane
-            const int items = M * SB_PARTS;
+        if (ph == kPhFinal && p.out_dim == 0) {
+            // --------------------------- hidden-state output (all warps) --
+            // LN2(z2) = rstd2 * zg - rstd2 * mu2 * gamma2 + beta2; item = (row, 64-column
+            // slice), one warp per item, two columns per lane
+            const int items = M * (kHidden / 64);
             for (int it = blockIdx.x * (SB_THREADS / 32) + warp; it < items; it += gridDim.x * (SB_THREADS / 32)) {
-                const int r = it / SB_PARTS, s = it % SB_PARTS;
-                const int c = s * 64 + 2 * lane;
-                if (ph == kPhReduce) {
-                    // z2 = sum of the FFN partials + (b2 + beta1) + rstd1 * x1 - rstd1 * mu1 * gamma1
-                    // every partial's load is issued before the first add (one round trip)
-                    float2 pv[SB_CHUNKS];
-#pragma unroll
-                    for (int j = 0; j < SB_CHUNKS; ++j)
-                        pv[j] = *reinterpret_cast<const float2 *>(p.part + ((size_t)j * 128 + r) * kHidden + c);
-                    float ax = 0.f, ay = 0.f;
-#pragma unroll
-                    for (int j = 0; j < SB_CHUNKS; ++j) {
-                        ax += pv[j].x;
-                        ay += pv[j].y;
-                    }
-                    float mu1, rstd1;
-                    merge_parts(p.st1 + (size_t)r * SB_PARTS, p.eps, mu1, rstd1);
-                    const float2 x1 = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(p.X1 + (size_t)r * kHidden + c));
-                    const float2 g1 = *reinterpret_cast<const float2 *>(p.ln1_g + c);
-                    const float2 bb = *reinterpret_cast<const float2 *>(p.bias_21 + c);
-                    const float z0 = ax + bb.x + rstd1 * x1.x - rstd1 * mu1 * g1.x;
-                    const float z1 = ay + bb.y + rstd1 * x1.y - rstd1 * mu1 * g1.y;
-                    // exact (mean, M2) of the slice: two passes over the warp's 64 values
-                    float sum = z0 + z1;
-#pragma unroll
-                    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-                    const float mean = sum * (1.0f / 64);
-                    float q = (z0 - mean) * (z0 - mean) + (z1 - mean) * (z1 - mean);
-#pragma unroll
-                    for (int o = 16; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-                    const float2 g2 = *reinterpret_cast<const float2 *>(p.ln2_g + c);
-                    *reinterpret_cast<uint32_t *>(p.Z + (size_t)r * kHidden + c) = pack_bf16x2(z0 * g2.x, z1 * g2.y);
-                    if (lane == 0) p.st2[(size_t)r * SB_PARTS + s] = make_float2(mean, q);
-                } else {
-                    // hidden-state output: LN2(z2) = rstd2 * zg - rstd2 * mu2 * gamma2 + beta2
-                    const int dst = p.row_dst[r];
-                    if (dst < 0) continue;
-                    if (dst >= p.out_rows) { set_status(p.status, kStatusShape); continue; }
-                    float mu2, rstd2;
-                    merge_parts(p.st2 + (size_t)r * SB_PARTS, p.eps, mu2, rstd2);
-                    const float2 zg = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(p.Z + (size_t)r * kHidden + c));
-                    const float2 g2 = *reinterpret_cast<const float2 *>(p.ln2_g + c);
-                    const float2 b2 = *reinterpret_cast<const float2 *>(p.ln2_b + c);
-                    *reinterpret_cast<uint32_t *>(p.out + (size_t)dst * kHidden + c) =
-                        pack_bf16x2(rstd2 * zg.x - rstd2 * mu2 * g2.x + b2.x, rstd2 * zg.y - rstd2 * mu2 * g2.y + b2.y);
-                }
+                const int r = it / (kHidden / 64), c = (it % (kHidden / 64)) * 64 + 2 * lane;
+                const int dst = p.row_dst[r];
+                if (dst < 0) continue;
+                if (dst >= p.out_rows) { set_status(p.status, kStatusShape); continue; }
+                float mu2, rstd2;
+                merge_parts(p.st2 + (size_t)r * SB_PARTS, p.eps, mu2, rstd2);
+                const float2 zg = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(p.Z + (size_t)r * kHidden + c));
+                const float2 g2 = *reinterpret_cast<const float2 *>(p.ln2_g + c);
+                const float2 b2 = *reinterpret_cast<const float2 *>(p.ln2_b + c);
+                *reinterpret_cast<uint32_t *>(p.out + (size_t)dst * kHidden + c) =
+                    pack_bf16x2(rstd2 * zg.x - rstd2 * mu2 * g2.x + b2.x, rstd2 * zg.y - rstd2 * mu2 * g2.y + b2.y);
             }
         } else if (warp == 0) {
             // ------------------------------------------------------------ producer --
             if (lane == 0) {
                 const uint64_t keep = policy_evict_last();  // weights: read by every execution
+                const CUtensorMap *ta = ph == kPhIn ? &p.tmE : ph == kPhOut ? &p.tmC : ph == kPhUp ? &p.tmX1
+                                        : ph == kPhDown ? &p.tmH : (ph == kPhQKV && l == 0) ? &p.tmX : &p.tmZ;
+                const CUtensorMap *tb = ph == kPhIn ? &p.tmWin : ph == kPhQKV ? &p.tmWqkv : ph == kPhOut ? &p.tmWo
+                                        : ph == kPhUp ? &p.tmW1 : ph == kPhDown ? &p.tmW2 : &p.tmWout;
+                // B boxes: N rows x 64 columns (the 32-column phases have maps with 32-row boxes)
+                const uint32_t b_box = (uint32_t)N * 128;
+                // one ring stage; false when its wait ran out
+                auto next_stage = [&](uint32_t &fb, uint32_t &a_dst, uint32_t &b_dst) -> bool {
+                    const int s = ring % SB_NS;
+                    if (!mbar_wait(smem_u32(&sm.empty[s]), ((ring / SB_NS) & 1) ^ 1, sm.abort_flag)) return false;
+                    fb = smem_u32(&sm.full[s]);
+                    a_dst = smem_u32(sm.a + s * SB_A_BYTES);
+                    b_dst = smem_u32(sm.b + s * SB_B_BYTES);
+                    ++ring;
+                    return true;
+                };
                 for (int job = p.withhold_loads ? njobs : blockIdx.x; job < njobs && ok; job += gridDim.x) {
-                    LoadStep st[12];  // at most 6 + 3 (FFN)
-                    int ns = 0;
-                    if (ph == kPhIn) {
-                        st[ns++] = {&p.tmE, &p.tmWin, a_boxes, 1, kEmb / 64, 0, 0, 0, job * 64};
-                    } else if (ph == kPhQKV || ph == kPhOut || ph == kPhFinal || ph == kPhFfn) {
-                        const CUtensorMap *ta = ph == kPhOut ? &p.tmC : ph == kPhFfn ? &p.tmX1
-                                                : (ph == kPhQKV && l == 0) ? &p.tmX : &p.tmZ;
-                        const CUtensorMap *tb = ph == kPhQKV ? &p.tmWqkv : ph == kPhOut ? &p.tmWo
-                                                : ph == kPhFfn ? &p.tmW1 : &p.tmWout;
-                        // every CTA of the phase reads the same A rows: each starts at another
-                        // stage of K, so that they do not all ask L2 for the same lines at once
-                        // (the sum over K is then taken in a rotated, fixed order per job)
-                        const int nsteps = (kHidden / 64) / kb_step;
-                        for (int i = 0; i < nsteps; ++i) {
-                            const int kb = ((i + job) % nsteps) * kb_step;
-                            st[ns++] = {ta, tb, a_boxes, 1, kb_step, kb * 64, 0, kb * 64, job * 64};
-                        }
-                        if (ph == kPhFfn)
-                            for (int nb = 0; nb < 3; ++nb)
-                                st[ns++] = {nullptr, &p.tmW2, 0, 4, 1, 0, 0, job * 64, nb * 256};
-                    } else {  // attention: Q and K of (sequence, head), then V
+                    uint32_t fb, a_dst, b_dst;
+                    if (ph == kPhAttn) {
+                        // Q and K of (sequence, head) in one stage, then V; 128-row boxes
+                        // unless the sequence fits in 64
                         const int b = job / kHeads, h = job % kHeads;
                         const int L = __ldg(p.seq_len + b), start = __ldg(p.seq_start + b);
                         const CUtensorMap *tq = L <= 64 ? &p.tmQKV64 : &p.tmQKV;
-                        st[ns++] = {tq, tq, 1, 1, 1, h * kHeadDim, start, kHidden + h * kHeadDim, start};
-                        st[ns++] = {nullptr, tq, 0, 1, 1, 0, 0, 2 * kHidden + h * kHeadDim, start};
+                        const uint32_t box = L <= 64 ? SB_BOX : 2 * SB_BOX;
+                        if (!next_stage(fb, a_dst, b_dst)) { ok = false; break; }
+                        mbar_arrive_expect_tx(fb, 2 * box);
+                        tma_load_2d(a_dst, tq, fb, h * kHeadDim, start);
+                        tma_load_2d(b_dst, tq, fb, kHidden + h * kHeadDim, start);
+                        if (!next_stage(fb, a_dst, b_dst)) { ok = false; break; }
+                        mbar_arrive_expect_tx(fb, box);
+                        tma_load_2d(b_dst, tq, fb, 2 * kHidden + h * kHeadDim, start);
+                        continue;
                     }
-                    for (int i = 0; i < ns && ok; ++i, ++ring) {
-                        const int s = ring % SB_NS;
-                        if (!mbar_wait(smem_u32(&sm.empty[s]), ((ring / SB_NS) & 1) ^ 1, sm.abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        const LoadStep &d = st[i];
-                        const bool attn = ph == kPhAttn;
-                        // attention boxes are 128 rows unless the sequence fits in 64
-                        const uint32_t box_bytes = attn && d.tb == &p.tmQKV ? 2 * SB_BOX : SB_BOX;
-                        const uint32_t fb = smem_u32(&sm.full[s]);
-                        mbar_arrive_expect_tx(fb, box_bytes * (uint32_t)(d.nk * (d.a_boxes + d.b_boxes)));
-                        const uint32_t a_dst = smem_u32(sm.a + s * SB_A_BYTES), b_dst = smem_u32(sm.b + s * SB_B_BYTES);
-                        if (attn) {
-                            if (d.a_boxes) tma_load_2d(a_dst, d.ta, fb, d.ax, d.ay);
-                            tma_load_2d(b_dst, d.tb, fb, d.bx, d.by);
-                        } else {
-                            for (int j = 0; j < d.nk; ++j) {
-                                for (int q = 0; q < d.a_boxes; ++q)
-                                    tma_load_2d(a_dst + (j * d.a_boxes + q) * SB_BOX, d.ta, fb, d.ax + 64 * j, d.ay + 64 * q);
-                                for (int q = 0; q < d.b_boxes; ++q)
-                                    tma_load_2d_hint(b_dst + (j * d.b_boxes + q) * SB_BOX, d.tb, fb, d.bx + 64 * j,
-                                                     d.by + 64 * q, keep);
-                            }
+                    // every CTA of a phase reads the same A rows: each starts at another
+                    // stage of K, so that they do not all ask L2 for the same lines at
+                    // once (the sum over K is then taken in a rotated, fixed order per job)
+                    for (int i = 0; i < nsteps; ++i) {
+                        const int kb = ((i + job) % nsteps) * nk;
+                        if (!next_stage(fb, a_dst, b_dst)) { ok = false; break; }
+                        mbar_arrive_expect_tx(fb, (uint32_t)nk * ((uint32_t)a_boxes * SB_BOX + b_box));
+                        for (int j = 0; j < nk; ++j) {
+                            for (int q = 0; q < a_boxes; ++q)
+                                tma_load_2d(a_dst + (j * a_boxes + q) * SB_BOX, ta, fb, (kb + j) * 64, 64 * q);
+                            tma_load_2d_hint(b_dst + j * b_box, tb, fb, (kb + j) * 64, job * N, keep);
                         }
                     }
                 }
@@ -400,11 +348,9 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
                         finish_unit();
                         continue;
                     }
-                    // one stage per kb_step K blocks (the in-projection's two in one stage)
-                    const int nsteps = ph == kPhIn ? 1 : (kHidden / 64) / kb_step;
-                    const int nk = ph == kPhIn ? kEmb / 64 : kb_step;
                     if (!wait_acc_free()) { ok = false; break; }
-                    const uint32_t idesc = idesc_bf16_f32(128, 64);
+                    const uint32_t idesc = idesc_bf16_f32(128, N);
+                    const uint32_t b_box = (uint32_t)N * 128;
                     for (int stp = 0; stp < nsteps && ok; ++stp) {
                         uint32_t s;
                         if (!wait_stage(s)) { ok = false; break; }
@@ -413,33 +359,13 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
                                 umma_bf16(tmem_base, sw128_kmajor_desc(a0 + j * a_boxes * SB_BOX + kk * 32),
-                                          sw128_kmajor_desc(b0 + j * SB_BOX + kk * 32), idesc, (stp | j | kk) != 0);
+                                          sw128_kmajor_desc(b0 + j * b_box + kk * 32), idesc, (stp | j | kk) != 0);
                         }
                         umma_commit(smem_u32(&sm.empty[s]));
                         ++ring;
                     }
                     if (!ok) break;
                     finish_unit();
-                    if (ph == kPhFfn) {
-                        // the down projection of this hidden chunk: three 256-column products
-                        // with H (bf16, shared memory) as the A operand, K = 64
-                        if (!mbar_wait(smem_u32(sm.h_ready), hcnt & 1, sm.abort_flag)) { ok = false; break; }
-                        ++hcnt;
-                        const uint32_t hb = smem_u32(sm.h);
-                        const uint32_t idesc2 = idesc_bf16_f32(128, 256);
-                        for (int nb = 0; nb < 3; ++nb) {
-                            uint32_t s;
-                            if (!wait_acc_free() || !wait_stage(s)) { ok = false; break; }
-                            const uint32_t b0 = smem_u32(sm.b + s * SB_B_BYTES);
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                umma_bf16(tmem_base, sw128_kmajor_desc(hb + kk * 32), sw128_kmajor_desc(b0 + kk * 32),
-                                          idesc2, kk != 0);
-                            umma_commit(smem_u32(&sm.empty[s]));
-                            ++ring;
-                            finish_unit();
-                        }
-                    }
                 }
             }
         } else {
@@ -525,18 +451,19 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
                     }
                     continue;
                 }
-                // 64-column tile of a GEMM: this thread's row, columns n0..n0+63
-                const int n0 = job * 64;
+                // an N-column tile of a GEMM (N = 64 or 32): this thread's row, columns n0..n0+N-1
+                const int n0 = job * N;
+                const bool wide = N == 64;
                 uint32_t v[2][32];
                 if (!wait_unit()) { ok = false; break; }
                 tmem_ld32(trow, v[0]);
-                tmem_ld32(trow + 32, v[1]);
+                if (wide) tmem_ld32(trow + 32, v[1]);
                 tmem_ld_wait();
                 release_unit();
-                const bool row_ok = r < M;
+                if (r >= M) continue;
                 float y[64];
 #pragma unroll
-                for (int j = 0; j < 64; ++j) y[j] = __uint_as_float(v[j >> 5][j & 31]);
+                for (int j = 0; j < 64; ++j) y[j] = wide || j < 32 ? __uint_as_float(v[j >> 5][j & 31]) : 0.f;
                 // LayerNorm of the A operand (z * gamma held in A, statistics per row)
                 const float2 *in_st = nullptr;
                 const float *fs = nullptr, *bias = nullptr;
@@ -545,12 +472,14 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
                     bias = l == 0 ? p.bqkv0 : p.bqkv;
                     if (l > 0) { in_st = p.st2; fs = p.s_qkv; }
                 } else if (ph == kPhOut) bias = l == 0 ? p.bo0 : p.bo;
-                else if (ph == kPhFfn) { bias = p.c_1; in_st = p.st1; fs = p.s_1; }
+                else if (ph == kPhUp) { bias = p.c_1; in_st = p.st1; fs = p.s_1; }
+                else if (ph == kPhDown) bias = p.bias_21;
                 else { bias = p.c_out; in_st = p.st2; fs = p.s_out; }  // final
                 float mu = 0.f, rstd = 1.f;
-                if (in_st && row_ok) merge_parts(in_st + (size_t)r * SB_PARTS, p.eps, mu, rstd);
+                if (in_st) merge_parts(in_st + (size_t)r * SB_PARTS, p.eps, mu, rstd);
 #pragma unroll
                 for (int j = 0; j < 64; j += 4) {
+                    if (!wide && j >= 32) break;
                     const float4 bb = __ldg(reinterpret_cast<const float4 *>(bias + n0 + j));
                     if (in_st) {
                         const float4 ss = __ldg(reinterpret_cast<const float4 *>(fs + n0 + j));
@@ -565,81 +494,32 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
                         y[j + 3] += bb.w;
                     }
                 }
-                if (ph == kPhFfn) {
-                    // H chunk = GELU(...) as bf16 into shared memory, the layout TMA
-                    // would give a 128 x 64 tile with the 128-byte swizzle (row r: 128 B,
-                    // 16-byte chunk q at position q ^ (r & 7)), for the down products
+                if (ph == kPhUp) {
 #pragma unroll
                     for (int j = 0; j < 64; ++j) y[j] = gelu_tanh_fast(y[j]);
-                    // the previous chunk's down products have read H (its last unit was waited for)
-                    const uint32_t hrow = smem_u32(sm.h) + r * 128;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint32_t w0 = pack_bf16x2(y[8 * q], y[8 * q + 1]), w1 = pack_bf16x2(y[8 * q + 2], y[8 * q + 3]);
-                        const uint32_t w2 = pack_bf16x2(y[8 * q + 4], y[8 * q + 5]), w3 = pack_bf16x2(y[8 * q + 6], y[8 * q + 7]);
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(hrow + ((q ^ (r & 7)) << 4)),
-                                     "r"(w0), "r"(w1), "r"(w2), "r"(w3)
-                                     : "memory");
-                    }
-                    fence_proxy_async_smem();  // generic writes, read by the tensor core (async proxy)
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(sm.h_ready));
-                    // the three down products: fp32 partial sums of this chunk, each warp's
-                    // 32 x 32 tiles staged in shared memory (128-byte swizzle) and stored
-                    // by TMA (rows of the partial buffer are 3 KB apart: one row per lane
-                    // would scatter every store)
-                    const bool any_row = quad * 32 < M;
-                    const uint32_t stg = smem_u32(sm.stg) + (uint32_t)quad * 4096u;
-                    for (int nb = 0; nb < 3; ++nb) {
-                        if (!wait_unit()) { ok = false; break; }
-                        for (int c = 0; c < 8; ++c) {
-                            uint32_t t[32];
-                            if (any_row) {
-                                tmem_ld32(trow + c * 32, t);
-                                tmem_ld_wait();
-                                if (lane == 0) bulk_wait_read0();  // the previous tile has left the staging
-                                __syncwarp();
-#pragma unroll
-                                for (int q = 0; q < 8; ++q)
-                                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                                                 ::"r"(stg + lane * 128 + ((q ^ (lane & 7)) << 4)), "r"(t[4 * q]),
-                                                 "r"(t[4 * q + 1]), "r"(t[4 * q + 2]), "r"(t[4 * q + 3])
-                                                 : "memory");
-                                fence_proxy_async_smem();
-                                __syncwarp();
-                                if (lane == 0) {
-                                    tma_store_2d(&p.tmPart, stg, nb * 256 + c * 32, job * 128 + quad * 32);
-                                    bulk_commit();
-                                }
-                            }
-                        }
-                        release_unit();
-                    }
-                    // the partial sums are in global memory before the phase's barrier
-                    if (lane == 0) bulk_wait0();
-                    __syncwarp();
-                    if (!ok) break;
-                    continue;
-                }
-                if (!row_ok) continue;
-                if (ph == kPhOut) {
-                    // z1 = acc + bias + residual (the layer input: X plain in the first
-                    // execution, else LN2(z2) rebuilt from z2 * gamma2 and its statistics)
-                    const bf16 *res = (l == 0 ? p.X : p.Z) + (size_t)r * kHidden + n0;
+                } else if (ph == kPhOut || ph == kPhDown) {
+                    // z = acc + bias + residual, stored as z * gamma with its (mean, M2).
+                    // out-proj: the residual is the layer input (X plain in the first
+                    // execution, else LN2(z2) rebuilt from z2 * gamma2); FFN down: LN1(z1)
+                    // rebuilt from z1 * gamma1 (its beta is folded into the bias)
+                    const bool down = ph == kPhDown;
+                    const bf16 *res = (down ? p.X1 : l == 0 ? p.X : p.Z) + (size_t)r * kHidden + n0;
+                    const float *rg = down ? p.ln1_g : p.ln2_g;
+                    const bool plain = !down && l == 0;
                     float rmu = 0.f, rrstd = 1.f;
-                    if (l > 0) merge_parts(p.st2 + (size_t)r * SB_PARTS, p.eps, rmu, rrstd);
+                    if (!plain) merge_parts((down ? p.st1 : p.st2) + (size_t)r * SB_PARTS, p.eps, rmu, rrstd);
 #pragma unroll
-                    for (int j = 0; j < 64; j += 8) {
+                    for (int j = 0; j < 32; j += 8) {
                         const uint4 w = *reinterpret_cast<const uint4 *>(res + j);
                         const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const float2 x = unpack_bf16x2(wv[e]);
-                            if (l == 0) {
+                            if (plain) {
                                 y[j + 2 * e] += x.x;
                                 y[j + 2 * e + 1] += x.y;
                             } else {
-                                const float g0 = __ldg(p.ln2_g + n0 + j + 2 * e), g1 = __ldg(p.ln2_g + n0 + j + 2 * e + 1);
+                                const float g0 = __ldg(rg + n0 + j + 2 * e), g1 = __ldg(rg + n0 + j + 2 * e + 1);
                                 y[j + 2 * e] += rrstd * x.x - rrstd * rmu * g0;
                                 y[j + 2 * e + 1] += rrstd * x.y - rrstd * rmu * g1;
                             }
@@ -647,14 +527,15 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
                     }
                     float sum = 0.f;
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) sum += y[j];
-                    const float mean = sum * (1.0f / 64);
+                    for (int j = 0; j < 32; ++j) sum += y[j];
+                    const float mean = sum * (1.0f / 32);
                     float m2 = 0.f;
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) m2 += (y[j] - mean) * (y[j] - mean);
-                    p.st1[(size_t)r * SB_PARTS + job] = make_float2(mean, m2);
+                    for (int j = 0; j < 32; ++j) m2 += (y[j] - mean) * (y[j] - mean);
+                    (down ? p.st2 : p.st1)[(size_t)r * SB_PARTS + job] = make_float2(mean, m2);
+                    const float *og = down ? p.ln2_g : p.ln1_g;
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) y[j] *= __ldg(p.ln1_g + n0 + j);
+                    for (int j = 0; j < 32; ++j) y[j] *= __ldg(og + n0 + j);
                 }
                 bf16 *dst;
                 if (ph == kPhFinal) {
@@ -663,15 +544,17 @@ __global__ void __launch_bounds__(SB_THREADS, 1) fwd_small_kernel(const __grid_c
                     if (d >= p.out_rows) { set_status(p.status, kStatusShape); continue; }
                     dst = p.out + (size_t)d * p.out_dim + n0;
                 } else {
-                    bf16 *base = ph == kPhIn ? p.X : ph == kPhQKV ? p.QKV : p.X1;
-                    const int ld = ph == kPhQKV ? kQKV : kHidden;
+                    bf16 *base = ph == kPhIn ? p.X : ph == kPhQKV ? p.QKV : ph == kPhOut ? p.X1 : ph == kPhUp ? p.H : p.Z;
+                    const int ld = ph == kPhQKV ? kQKV : ph == kPhUp ? kFfn : kHidden;
                     dst = base + (size_t)r * ld + n0;
                 }
                 uint4 *d4 = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
+                for (int q = 0; q < 8; ++q) {
+                    if (!wide && q >= 4) break;
                     d4[q] = make_uint4(pack_bf16x2(y[8 * q], y[8 * q + 1]), pack_bf16x2(y[8 * q + 2], y[8 * q + 3]),
                                        pack_bf16x2(y[8 * q + 4], y[8 * q + 5]), pack_bf16x2(y[8 * q + 6], y[8 * q + 7]));
+                }
             }
         }
         // a failed wait in any role stops the CTA at this barrier; the others

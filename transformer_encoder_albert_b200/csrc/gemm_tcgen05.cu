@@ -807,20 +807,6 @@ int make_tmap_e4m3(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t co
     return r == CUDA_SUCCESS ? 0 : -3;
 }
 
-int make_tmap_f32_tile32(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return -1;
-    if ((reinterpret_cast<uintptr_t>(base) & 15) || (cols * 4) % 16) return -2;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 4};
-    cuuint32_t box[2] = {32, 32};
-    cuuint32_t es[2] = {1, 1};
-    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, es,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? 0 : -3;
-}
-
 int make_tmap_bf16_tile32(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols) {
     return encode_bf16(tm, base, rows, cols, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }

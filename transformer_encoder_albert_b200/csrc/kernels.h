@@ -129,9 +129,6 @@ int make_tmap_bf16(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t co
 // Map of an E4M3 (byte) row-major [rows, cols] tensor with a {128, box_rows} box
 // and the 128-byte swizzle: the operands of the E4M3 GEMM variant.
 int make_tmap_e4m3(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
-// Map of an fp32 row-major [rows, cols] tensor with a 32x32 box and the 128-byte
-// swizzle (tile stores of fp32 partial sums).
-int make_tmap_f32_tile32(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols);
 // Map of a bf16 row-major [rows, cols] tensor with a 32x32 box and the 64-byte
 // swizzle: the epilogue's output stores and residual loads.
 int make_tmap_bf16_tile32(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols);
@@ -163,16 +160,16 @@ cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB,
 // kernel (forward_small.cu).  A-operand maps have {64, 64} boxes with the
 // 128-byte swizzle over the workspace rows; weight maps {64, 64} boxes.
 // Statistics are twelve 64-column (mean, M2) partials per row.
-constexpr int kSmallParts = 12;
+constexpr int kSmallParts = 24;  // 32-column statistics slices of a small-batch row
 constexpr int kSmallMaxRows = 128;
 struct SmallFwdArgs {
-    CUtensorMap tmE, tmX, tmC, tmX1, tmZ;       // E [rows,128]; X, C, X1 = z1*g1, Z = z2*g2 [rows,768]
+    CUtensorMap tmE, tmX, tmC, tmX1, tmZ, tmH;  // E [rows,128]; X, C, X1 = z1*g1, Z = z2*g2 [rows,768];
+                                                // H [rows,2048]; {64 cols, 64 rows} boxes
     CUtensorMap tmQKV, tmQKV64;                 // [rows, 2304] with {64,128} / {64,64} boxes
-    CUtensorMap tmWin, tmWqkv, tmWo, tmW1, tmW2, tmWout;
-    CUtensorMap tmPart;                         // part as fp32 [32 * 128, 768], {32, 32} box, 128-byte swizzle
-    bf16 *X, *QKV, *C, *X1, *Z;
-    float2 *st1, *st2;                          // [128][12]
-    float *part;                                // [32][128][768] FFN partial sums
+    CUtensorMap tmWin, tmWqkv, tmW1, tmWout;    // {64 cols, 64 rows} boxes
+    CUtensorMap tmWo, tmW2;                     // {64 cols, 32 rows} boxes (32-column jobs)
+    bf16 *X, *QKV, *C, *X1, *Z, *H;
+    float2 *st1, *st2;                          // [128][24]: per-row (mean, M2) of 32-column slices
     const float *b_in;
     const float *bqkv0, *bqkv, *s_qkv;          // first execution: plain bias; later: folded LN2
     const float *bo0, *bo;                      // out-proj bias (later executions: + beta2)
