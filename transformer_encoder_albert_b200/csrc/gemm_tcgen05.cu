@@ -253,6 +253,29 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             tmem_relinquish();
         }
     }
+    // The weights do not depend on the previous kernel: before waiting for it,
+    // the producer starts the B tiles of the first stages of its first unit
+    // (their A tiles follow the wait).  A pair's copies count on rank 0's
+    // barriers, so their initialisation must be visible to both CTAs first.
+    if (PAIR) cluster_sync();
+    else __syncthreads();
+    const int pre = p.withhold_loads ? 0 : (p.K / KB < NST ? p.K / KB : NST);  // stages started early
+    if (warp == 0 && lane == 0 && pre > 0) {
+        const uint64_t keep = policy_evict_last();
+        const int n = slot % (p.N / BN);
+        for (int st = 0; st < pre; ++st) {
+            const uint32_t fb = smem_u32(&sm.full[st]);
+            const uint32_t b_dst = smem_u32(sm.b + st * BSTAGE);
+            if (PAIR) {
+                if (rank == 0) mbar_expect_tx(fb, 2 * B_HALF_BYTES);
+                tma_load_2d_pair_hint(b_dst, &tmB, mapa_shared(fb, 0), st * KB, n * BN + (int)rank * B_BOX, keep);
+            } else {
+                mbar_expect_tx(fb, B_BYTES);
+                tma_load_2d_hint(b_dst, &tmB, fb, st * KB, n * BN, keep);
+                tma_load_2d_hint(b_dst + B_HALF_BYTES, &tmB, fb, st * KB, n * BN + B_BOX, keep);
+            }
+        }
+    }
     // The prologue above overlaps the previous kernel; its results are used from here on.
     griddep_wait();
     if (threadIdx.x == 0) {
@@ -293,7 +316,16 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     const uint32_t fb = smem_u32(&sm.full[stage]);
                     const uint32_t a_dst = smem_u32(sm.a + stage * A_BYTES);
                     const uint32_t b_dst = smem_u32(sm.b + stage * BSTAGE);
-                    if (PAIR) {
+                    if (issued < pre) {
+                        // the first unit's B tiles of this stage are already on their way
+                        if (PAIR) {
+                            if (rank == 0) mbar_arrive_expect_tx(fb, 2 * A_BYTES);
+                            tma_load_2d_pair(a_dst, &tmA, mapa_shared(fb, 0), kb * KB, m * UM + (int)rank * BM);
+                        } else {
+                            mbar_arrive_expect_tx(fb, A_BYTES);
+                            tma_load_2d(a_dst, &tmA, fb, kb * KB, m * BM);
+                        }
+                    } else if (PAIR) {
                         // both CTAs' copies count on rank 0's barrier, which expects them all
                         const uint32_t fb0 = mapa_shared(fb, 0);
                         if (rank == 0) mbar_arrive_expect_tx(fb, 2 * (A_BYTES + B_HALF_BYTES));
@@ -308,6 +340,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     ++issued;
                     if (++stage == NST) { stage = 0; phase ^= 1; }
                 }
+            }
+            if (issued < pre && (!PAIR || rank == 0)) {
+                // no unit to load (few rows, or an earlier kernel failed): the early
+                // weight tiles still land before the CTA's shared memory goes away
+                for (int st = issued; st < pre; ++st) mbar_arrive(smem_u32(&sm.full[st]));
+                for (int st = issued; st < pre; ++st) mbar_wait_drain(smem_u32(&sm.full[st]), 0);
             }
             if (!ok && (!PAIR || rank == 0)) {
                 // Drain: every stage whose load may still be in flight completes
