@@ -82,12 +82,18 @@ CLASS_SOURCES = {
     "gemm": ["gemm_tcgen05.cu", "sm100_ptx.cuh", "kernels.h"],
     "attention": ["attention_tc.cu", "sm100_ptx.cuh", "kernels.h"],            # longest sequence <= 128
     "attention_long": ["attention_tc_long.cu", "sm100_ptx.cuh", "kernels.h"],  # 128 < longest <= 512
+    "quant": ["fp8.cu", "sm100_ptx.cuh", "kernels.h"],
+    "small": ["forward_small.cu", "sm100_ptx.cuh", "kernels.h"],
 }
 
 
 def source_set(cls: str, seq_len: int = 128) -> str:
     if cls.startswith("gemm_"):
         return "gemm"
+    if cls == "quant_e4m3":
+        return "quant"
+    if cls == "small_batch_forward":
+        return "small"
     return "attention" if seq_len <= 128 else "attention_long"
 
 
@@ -569,9 +575,12 @@ def measure_workload(args, ctx, name, padded, graph_mode, extras):
     dom_ms = dom[1] / max(dom[0], 1)
     achieved = per_launch.get(dominant, 0.0) / (dom_ms / 1000.0) / 1e12
     if dominant == "quant_e4m3":
-        # HBM-bound: bf16 rows read, E4M3 codes and a scale per row written; per
-        # execution three quantizations of 768-wide rows and one of 2048-wide rows
-        qbytes = rows * (3 * 768 + 2048) * 3 / 4.0 + rows * 4
+        # HBM-bound: bf16 rows read, E4M3 codes and a scale per row written.  Per
+        # execution the quantized inputs are Q|K|V's, the out-projection's and FFN
+        # up's (768 wide) and FFN down's (2048 wide), in that order; the timed
+        # launch is launch per_step // 2 of each forward
+        k_timed = 2048 if (per_step // 2) % 4 == 3 else 768
+        qbytes = rows * k_timed * 3.0 + rows * 4
         hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         roofline_hbm = {"kernel": dominant, "bound": "hbm", "achieved": qbytes / (dom_ms / 1000.0) / 1e9,
                         "peak": hbm, "unit": "GB/s", "bytes_per_launch": qbytes,
@@ -579,19 +588,19 @@ def measure_workload(args, ctx, name, padded, graph_mode, extras):
         roofline_hbm["frac"] = roofline_hbm["achieved"] / hbm
     else:
         roofline_hbm = None
-    traffic, traffic_note = load_traffic(dominant, label, wl.T)
+    # E4M3 runs have their own capture (workload label + "_e4m3")
+    traffic, traffic_note = load_traffic(dominant, label + ("_e4m3" if args.dtype == "fp8" else ""), wl.T)
     bound = "tensor"
     dom_peak = peak if (args.dtype == "bf16" or dominant in fp8_classes) else peak / 2.0
     roofline = {"kernel": dominant, "bound": bound, "achieved": achieved, "peak": dom_peak,
-                "unit": "TFLOP/s", "frac": achieved / dom_peak, "traffic": traffic if args.dtype == "bf16" else None,
-                "traffic_source": traffic_note if args.dtype == "bf16" else "no ncu capture of the E4M3 kernels",
+                "unit": "TFLOP/s", "frac": achieved / dom_peak, "traffic": traffic, "traffic_source": traffic_note,
                 "peak_source": f"{peak_note} (the kernel runs {dom_ms * 1000:.0f} us inside a {ms_per_step:.3f} ms step)",
                 "frac_of_sustained": (achieved / peak_sus) if peak_sus else None,
                 "launches_timed": dom[0], "launches_timed_note": f"1 of {per_step} per step", "avg_launch_ms": dom_ms,
                 "flops_per_launch": per_launch.get(dominant, 0.0)}
     if roofline_hbm is not None:
-        roofline_hbm.update({"launches_timed": dom[0], "avg_launch_ms": dom_ms, "traffic": None,
-                             "traffic_source": "no ncu capture of the quantizer"})
+        roofline_hbm.update({"launches_timed": dom[0], "avg_launch_ms": dom_ms, "traffic": traffic,
+                             "traffic_source": traffic_note})
         roofline = roofline_hbm
     clocks = sampler.summary(t_wall0, t_wall1)
     line = {

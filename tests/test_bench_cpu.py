@@ -28,6 +28,10 @@ def test_missing_traffic_file(tmp_path, monkeypatch):
 def test_gemm_classes_share_a_digest_and_attention_differs():
     assert bench.sources_digest("gemm_qkv") == bench.sources_digest("gemm_out_proj_ln")
     assert bench.sources_digest("gemm_qkv") != bench.sources_digest("attention")
+    # the quantizer and the small-batch kernel have their own source sets
+    assert bench.source_set("quant_e4m3") == "quant" and bench.source_set("small_batch_forward") == "small"
+    assert bench.sources_digest("quant_e4m3") != bench.sources_digest("small_batch_forward")
+    assert bench.source_set("attention", 512) == "attention_long"
 
 
 def test_long_attention_has_its_own_digest_and_lines(tmp_path, monkeypatch):
