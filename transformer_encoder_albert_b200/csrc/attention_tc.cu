@@ -283,7 +283,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                         if (c + e >= nch) continue;
                         if (base + 32 <= L) {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) mx[j & 3] = fmaxf(mx[j & 3], __uint_as_float(v[e][j]));
+                            for (int j = 0; j < 32; j += 2)
+                                mx[(j >> 1) & 3] = fmax3(mx[(j >> 1) & 3], __uint_as_float(v[e][j]),
+                                                           __uint_as_float(v[e][j + 1]));
                         } else {
 #pragma unroll
                             for (int j = 0; j < 32; ++j)

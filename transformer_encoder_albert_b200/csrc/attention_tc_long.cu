@@ -285,7 +285,9 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, bf16 *__restrict_
                         if (c + e >= nch) continue;
                         if (base + 32 <= Lj) {
 #pragma unroll
-                            for (int t = 0; t < 32; ++t) mx[t & 3] = fmaxf(mx[t & 3], __uint_as_float(v[e][t]));
+                            for (int t = 0; t < 32; t += 2)
+                                mx[(t >> 1) & 3] = fmax3(mx[(t >> 1) & 3], __uint_as_float(v[e][t]),
+                                                           __uint_as_float(v[e][t + 1]));
                         } else {
 #pragma unroll
                             for (int t = 0; t < 32; ++t)
