@@ -555,8 +555,33 @@ def measure_workload(args, ctx, name, padded, graph_mode, extras):
         torch.cuda.synchronize()
         return max_r(e_s.elapsed_time(e_e))
 
+    # the same through the packed host call: only the valid rows' ids travel in and
+    # only the valid rows' outputs travel back
+    packed_h = torch.as_tensor(np.concatenate([ids[b, :L[b]] for b in range(wl.B)])).pin_memory()
+    cu_h = torch.as_tensor(np.concatenate([[0], np.cumsum(L)]).astype(np.int32)).pin_memory()
+    pouts_h = [torch.empty(n_tok, arch["out_dim"], dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+
+    def timed_packed_loop() -> float:
+        e_s = torch.cuda.Event(enable_timing=True)
+        e_e = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e_s.record(stream)
+        for k in range(n_e2e):
+            if enc.forward_varlen_host_async(packed_h, cu_h, int(L.max()), pouts_h[k & 1]) != 0:
+                raise SystemExit("packed host path status")
+        if enc.forward_host_wait() != 0:
+            raise SystemExit("packed host path status")
+        e_e.record(stream)
+        torch.cuda.synchronize()
+        return max_r(e_s.elapsed_time(e_e))
+
     timed_host_loop(True)  # warm-up: allocates the second staging slot
     e2e_ms = timed_host_loop(True)
+    e2e_packed_value = None
+    if not padded and wl.T <= 512:
+        timed_packed_loop()
+        e2e_packed_value = sum_r(float(n_tok * n_e2e)) / (timed_packed_loop() / 1000.0)
     e2e_value = sum_r(float(n_tok * n_e2e)) / (e2e_ms / 1000.0)
     e2e_sync_value = sum_r(float(n_tok * n_e2e)) / (timed_host_loop(False) / 1000.0)
     out_h = outs_h[0]
@@ -630,7 +655,11 @@ def measure_workload(args, ctx, name, padded, graph_mode, extras):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(ids_h.numel() * 8 + mask_h.numel()),
                 "d2h_bytes_per_step": int(out_h.numel() * 2),
                 "api": "albert_forward_host_async (output copy of a step overlaps the next forward)",
-                "synchronous_api_value": e2e_sync_value},
+                "synchronous_api_value": e2e_sync_value,
+                "packed_api_value": e2e_packed_value,
+                "packed_api": ("albert_forward_varlen_host_async (packed ids in, valid rows out: "
+                               f"{int(packed_h.numel() * 8 + cu_h.numel() * 4)} B in, "
+                               f"{int(n_tok * arch['out_dim'] * 2)} B out per step)")},
         "stream_launch_ms_per_step": stream_ms,
         "gpu_launches": launches * args.steps,
         "clocks": clocks,

@@ -183,8 +183,19 @@ int albert_forward_host(albert_handle *h, const int64_t *ids_host, const uint8_t
 int albert_forward_host_async(albert_handle *h, const int64_t *ids_host, const uint8_t *mask_host,
                               int B, int T, void *out_host, void *stream);
 
-/* Wait for every batch of albert_forward_host_async still in flight; returns
- * the first non-OK status among them (ALBERT_OK if none). */
+/* The same pipelined path for a PACKED batch (as albert_forward_varlen): ids_host
+ * [cu_seqlens_host[nseq]] int64, cu_seqlens_host [nseq + 1] int32 on the host,
+ * out_host [cu_seqlens_host[nseq], out_dim] -- only the valid rows travel to the
+ * device and back.  The copy sizes are read from cu_seqlens_host: cu[0] != 0 or a
+ * total outside 1..max_tokens returns ALBERT_ERR_SHAPE before any work; the rest
+ * of the lengths are checked on the device as in albert_forward_varlen.  Shares
+ * the staging slots, ordering and waiting rules of albert_forward_host_async
+ * (the two may be mixed on one handle). */
+int albert_forward_varlen_host_async(albert_handle *h, const int64_t *ids_host, const int32_t *cu_seqlens_host,
+                                     int nseq, int max_len, void *out_host, void *stream);
+
+/* Wait for every batch of albert_forward_host_async / albert_forward_varlen_host_async
+ * still in flight; returns the first non-OK status among them (ALBERT_OK if none). */
 int albert_forward_host_wait(albert_handle *h);
 
 /* Synchronize `stream` and return the status recorded by the last forward on
@@ -315,11 +326,15 @@ size_t albert_length_regulate_scratch_bytes(int n_tok);
  * with R: [M, N] bf16 and N == 768; 3 = bias -> bf16 rows scattered to
  * row_dst[r] (row_dst[r] < 0 skips the row).  K % 64 == 0, N % 256 == 0;
  * bias and ln_g 16-byte aligned (else ALBERT_ERR_CONFIG).  Adding
- * ALBERT_GEMM_SINGLE_CTA or ALBERT_GEMM_CTA_PAIR to epi forces that kernel
- * variant (one CTA per 128x256 tile, or a two-CTA cluster per 256x256 tile);
- * by default the pair is used whenever M > 128, as in albert_forward. */
+ * ALBERT_GEMM_SINGLE_CTA, ALBERT_GEMM_CTA_PAIR or ALBERT_GEMM_NARROW to epi
+ * forces that kernel variant (one CTA per 128x256 tile, a two-CTA cluster per
+ * 256x256 tile, or one CTA per 128x128 tile); by default the choice is
+ * albert_forward's: one CTA for M <= 128, the 128x128 tile when the pair tiles
+ * would leave clusters idle and every 128x128 tile runs at once, else the pair.
+ * More than one of the three: ALBERT_ERR_CONFIG. */
 #define ALBERT_GEMM_SINGLE_CTA 16
 #define ALBERT_GEMM_CTA_PAIR 32
+#define ALBERT_GEMM_NARROW 128
 /* Adding ALBERT_GEMM_E4M3 runs the E4M3 variant: A and W are first quantized
  * per row as albert_test_quant_e4m3 does (into temporaries), then multiplied
  * on tcgen05 (kind::f8f6f4) with the epilogue starting from

@@ -326,6 +326,43 @@ def test_forward_host_async_reports_a_bad_batch_when_reaped(w_bf16):
     enc.close()
 
 
+def test_forward_varlen_host_async_matches_device_path(w_bf16):
+    """Packed batches through the pipelined host path (only valid rows cross the
+    bus), interleaved with padded ones on the same staging slots, equal the device
+    path's rows; host-side shape checks reject a bad cu_seqlens before any work."""
+    wl = synth.WORKLOADS["b8_T128"]
+    enc = tea.Encoder(w_bf16, A, max_tokens=wl.B * wl.T)
+    keep, refs, outs = [], [], []
+    for k in range(4):
+        ids, mask, L = synth.make_batch(wl, seed=200 + k)
+        ref = enc.forward(_t(ids), _t(mask)).cpu()
+        if k % 2:  # a padded batch between packed ones
+            ids_h, mask_h = torch.as_tensor(ids).pin_memory(), torch.as_tensor(mask).pin_memory()
+            out_h = torch.zeros(wl.B, wl.T, 512, dtype=torch.bfloat16).pin_memory()
+            assert enc.forward_host_async(ids_h, mask_h, out_h) == 0
+            keep.append((ids_h, mask_h))
+            refs.append(ref)
+        else:
+            packed = np.concatenate([ids[b, :L[b]] for b in range(wl.B)])
+            cu = np.concatenate([[0], np.cumsum(L)]).astype(np.int32)
+            ids_h, cu_h = torch.as_tensor(packed).pin_memory(), torch.as_tensor(cu).pin_memory()
+            out_h = torch.full((int(cu[-1]), 512), 7.0, dtype=torch.bfloat16).pin_memory()
+            assert enc.forward_varlen_host_async(ids_h, cu_h, int(L.max()), out_h) == 0
+            keep.append((ids_h, cu_h))
+            refs.append(torch.cat([ref[b, :L[b]] for b in range(wl.B)]))
+        outs.append(out_h)
+    assert enc.forward_host_wait() == 0
+    for k in range(4):
+        assert torch.equal(refs[k], outs[k]), f"batch {k}"
+    bad_cu = torch.tensor([1, 5], dtype=torch.int32)
+    assert enc.forward_varlen_host_async(torch.zeros(5, dtype=torch.int64), bad_cu, 5,
+                                         torch.zeros(5, 512, dtype=torch.bfloat16)) == 3  # ALBERT_ERR_SHAPE
+    big_cu = torch.tensor([0, wl.B * wl.T + 1], dtype=torch.int32)
+    assert enc.forward_varlen_host_async(torch.zeros(1, dtype=torch.int64), big_cu, 128,
+                                         torch.zeros(1, 512, dtype=torch.bfloat16)) == 3
+    enc.close()
+
+
 # ------------------------------------------------------------ error paths ----
 
 def _sentinel(shape):

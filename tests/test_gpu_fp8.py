@@ -43,7 +43,7 @@ def _tol(got, ref, what):
     assert not np.any(bad), f"{what}: {int(bad.sum())} outside, max err {float(np.max(np.abs(got - ref))):.3e}"
 
 
-@pytest.mark.parametrize("variant", ["single", "pair"])
+@pytest.mark.parametrize("variant", ["single", "pair", "narrow"])
 @pytest.mark.parametrize("epi", [0, 1, 2, 3])
 def test_e4m3_gemm_against_the_quantized_oracle(epi, variant):
     M, N, K = (300, 768, 768) if epi == 2 else (257, 512, 2048)

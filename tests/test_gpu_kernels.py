@@ -33,7 +33,7 @@ def _close(got, ref, rel=8e-3, what=""):
     assert not bad.any(), f"{what}: {bad.sum()} elements off, worst {err.max():.3e} (scale {scale:.3e})"
 
 
-VARIANTS = ["single", "pair"]
+VARIANTS = ["single", "pair", "narrow"]
 
 
 @pytest.mark.parametrize("variant", VARIANTS)

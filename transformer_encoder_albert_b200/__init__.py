@@ -35,7 +35,7 @@ WEIGHT_FIELDS = (
 
 EXPORTS = (
     "albert_create", "albert_forward", "albert_forward_varlen", "albert_forward_host",
-    "albert_forward_host_async", "albert_forward_host_wait",
+    "albert_forward_host_async", "albert_forward_varlen_host_async", "albert_forward_host_wait",
     "albert_get_status", "albert_destroy", "albert_launches_per_forward",
     "albert_profile_enable", "albert_profile_retain", "albert_profile_stride", "albert_profile_reset",
     "albert_profile_classes",
@@ -80,6 +80,7 @@ def lib() -> C.CDLL:
         L.albert_forward_varlen.argtypes = [vp, vp, vp, i, i, vp, vp]
         L.albert_forward_host.argtypes = [vp, vp, vp, i, i, vp, vp]
         L.albert_forward_host_async.argtypes = [vp, vp, vp, i, i, vp, vp]
+        L.albert_forward_varlen_host_async.argtypes = [vp, vp, vp, i, i, vp, vp]
         L.albert_forward_host_wait.argtypes = [vp]
         L.albert_get_status.argtypes = [vp, vp]
         L.albert_destroy.argtypes = [vp]
@@ -180,6 +181,13 @@ def albert_forward_host_async(h: int, ids_host, mask_host, out_host, stream=None
                                            _stream_ptr(stream))
 
 
+def albert_forward_varlen_host_async(h: int, ids_host, cu_seqlens_host, max_len: int, out_host,
+                                     stream=None) -> int:
+    nseq = cu_seqlens_host.numel() - 1
+    return lib().albert_forward_varlen_host_async(h, _ptr(ids_host), _ptr(cu_seqlens_host), nseq, int(max_len),
+                                                  _ptr(out_host), _stream_ptr(stream))
+
+
 def albert_forward_host_wait(h: int) -> int:
     return lib().albert_forward_host_wait(h)
 
@@ -248,6 +256,11 @@ class Encoder:
         """Enqueue one batch of the pipelined host path; returns the status of the
         batch issued two calls earlier (its output is then in host memory)."""
         return albert_forward_host_async(self.h, ids_host, mask_host, out_host, stream)
+
+    def forward_varlen_host_async(self, ids_host, cu_seqlens_host, max_len: int, out_host, stream=None) -> int:
+        """The pipelined host path for a packed batch: int64 ids [n_tok] and int32
+        cu_seqlens [nseq + 1] in host memory, out_host [n_tok, out_dim]."""
+        return albert_forward_varlen_host_async(self.h, ids_host, cu_seqlens_host, max_len, out_host, stream)
 
     def forward_host_wait(self) -> int:
         """Wait for all pipelined host batches; first non-OK status."""
@@ -326,14 +339,15 @@ def profile_class_names() -> list:
     return [lib().albert_profile_name(i).decode() for i in range(n)]
 
 
-GEMM_VARIANTS = {"auto": 0, "single": 16, "pair": 32}
+GEMM_VARIANTS = {"auto": 0, "single": 16, "pair": 32, "narrow": 128}
 GEMM_E4M3 = 64
 
 
 def test_gemm(A, W, bias, Y, epi: int, R=None, ln_g=None, ln_b=None, eps: float = 1e-12,
               row_dst=None, stream=None, variant: str = "auto", e4m3: bool = False) -> int:
     """Run the tcgen05 GEMM alone (single-kernel parity tests).  variant picks
-    the one-CTA or the CTA-pair kernel ("auto": the pair when M > 128); e4m3
+    the one-CTA 128x256, the CTA-pair 256x256 or the one-CTA 128x128 kernel
+    ("auto": the forward's choice); e4m3
     quantizes both operands per row and runs the E4M3 variant."""
     M, K = A.shape
     N = W.shape[0]

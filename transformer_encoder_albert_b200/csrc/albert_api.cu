@@ -99,6 +99,7 @@ struct albert_handle {
     struct Slot {
         int64_t *ids = nullptr;
         uint8_t *mask = nullptr;
+        int32_t *cu = nullptr;           // cu_seqlens of a packed batch
         void *out = nullptr;
         cudaEvent_t d2h_done = nullptr;  // output copied to the host
         cudaEvent_t fwd_done = nullptr;  // forward (and its status copy) complete
@@ -273,7 +274,7 @@ int gemm_bf16(Launch &L, int cls, int epi, const CUtensorMap &A, const CUtensorM
     a.withhold_loads = (L.h->stall_mask >> cls) & 1u;
     if (epi == kEpiResStats && a.N != gemm::LN_N) return ALBERT_ERR_CONFIG;
     if (!gemm_vectors_aligned(a)) return ALBERT_ERR_CONFIG;
-    LAUNCH(L, cls, launch_gemm(epi, A, B, Out, Res, a, grid, L.s));
+    LAUNCH(L, cls, launch_gemm(epi, A, B, Out, Res, a, grid, L.h->num_sms, L.s));
     return ALBERT_OK;
 }
 
@@ -837,6 +838,7 @@ static int async_setup(albert_handle *h) {
     if ((rc = dev_alloc(h, (void **)&h->slot[1].mask, n))) return rc;
     if ((rc = dev_alloc(h, &h->slot[1].out, n * out_width(h) * elem_bytes(h)))) return rc;
     for (auto &sl : h->slot) {
+        if ((rc = dev_alloc(h, (void **)&sl.cu, ((size_t)h->seq_cap + 1) * sizeof(int32_t)))) return rc;
         TRY(cudaEventCreateWithFlags(&sl.d2h_done, cudaEventDisableTiming));
         TRY(cudaEventCreateWithFlags(&sl.fwd_done, cudaEventDisableTiming));
     }
@@ -874,6 +876,34 @@ int albert_forward_host_async(albert_handle *h, const int64_t *ids_host, const u
     TRY(cudaEventRecord(sl.fwd_done, s));
     TRY(cudaStreamWaitEvent(h->copy_stream, sl.fwd_done, 0));
     TRY(cudaMemcpyAsync(out_host, sl.out, n * out_width(h) * elem_bytes(h), cudaMemcpyDeviceToHost, h->copy_stream));
+    TRY(cudaEventRecord(sl.d2h_done, h->copy_stream));
+    sl.in_flight = true;
+    ++h->async_issued;
+    return prev;
+}
+
+int albert_forward_varlen_host_async(albert_handle *h, const int64_t *ids_host, const int32_t *cu_seqlens_host,
+                                     int nseq, int max_len, void *out_host, void *stream) {
+    if (!h || !ids_host || !cu_seqlens_host || !out_host) return ALBERT_ERR_NULL;
+    if (nseq < 1 || nseq > h->seq_cap || max_len < 1 || max_len > h->cfg.max_pos) return ALBERT_ERR_SHAPE;
+    if (h->cfg.out_layout != 0) return ALBERT_ERR_CONFIG;
+    // the copy sizes come from the host's cu_seqlens; the device checks the rest
+    const long long n_tok = cu_seqlens_host[nseq];
+    if (cu_seqlens_host[0] != 0 || n_tok < 1 || n_tok > h->cfg.max_tokens) return ALBERT_ERR_SHAPE;
+    int rc = async_setup(h);
+    if (rc) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int b = (int)(h->async_issued & 1);
+    const int prev = async_reap(h, b);
+    auto &sl = h->slot[b];
+    TRY(cudaMemcpyAsync(sl.ids, ids_host, (size_t)n_tok * sizeof(int64_t), cudaMemcpyHostToDevice, s));
+    TRY(cudaMemcpyAsync(sl.cu, cu_seqlens_host, ((size_t)nseq + 1) * sizeof(int32_t), cudaMemcpyHostToDevice, s));
+    if ((rc = albert_forward_varlen(h, sl.ids, sl.cu, nseq, max_len, sl.out, s))) return rc;
+    TRY(cudaMemcpyAsync(h->status_host + b, h->status, sizeof(int), cudaMemcpyDeviceToHost, s));
+    TRY(cudaEventRecord(sl.fwd_done, s));
+    TRY(cudaStreamWaitEvent(h->copy_stream, sl.fwd_done, 0));
+    TRY(cudaMemcpyAsync(out_host, sl.out, (size_t)n_tok * out_width(h) * elem_bytes(h), cudaMemcpyDeviceToHost,
+                        h->copy_stream));
     TRY(cudaEventRecord(sl.d2h_done, h->copy_stream));
     sl.in_flight = true;
     ++h->async_issued;
@@ -994,9 +1024,12 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
     const bool e4m3 = (epi & ALBERT_GEMM_E4M3) != 0;
     if (M < 1 || N < gemm::BN || N % gemm::BN || K < gemm::BK || K % gemm::BK) return ALBERT_ERR_SHAPE;
     if (e4m3 && (K % 256 || K > 2048 || N % 8)) return ALBERT_ERR_SHAPE;  // the row quantizer's limits
-    const int variant = (epi & ALBERT_GEMM_SINGLE_CTA) ? kGemmSingle : (epi & ALBERT_GEMM_CTA_PAIR) ? kGemmPair : kGemmAuto;
-    if ((epi & ALBERT_GEMM_SINGLE_CTA) && (epi & ALBERT_GEMM_CTA_PAIR)) return ALBERT_ERR_CONFIG;
-    epi &= ~(ALBERT_GEMM_SINGLE_CTA | ALBERT_GEMM_CTA_PAIR | ALBERT_GEMM_E4M3);
+    const int forced = (epi & ALBERT_GEMM_SINGLE_CTA ? 1 : 0) + (epi & ALBERT_GEMM_CTA_PAIR ? 1 : 0) +
+                       (epi & ALBERT_GEMM_NARROW ? 1 : 0);
+    if (forced > 1) return ALBERT_ERR_CONFIG;
+    const int variant = (epi & ALBERT_GEMM_SINGLE_CTA) ? kGemmSingle : (epi & ALBERT_GEMM_CTA_PAIR) ? kGemmPair
+                        : (epi & ALBERT_GEMM_NARROW) ? kGemmNarrow : kGemmAuto;
+    epi &= ~(ALBERT_GEMM_SINGLE_CTA | ALBERT_GEMM_CTA_PAIR | ALBERT_GEMM_NARROW | ALBERT_GEMM_E4M3);
     if (epi < 0 || epi > 3) return ALBERT_ERR_CONFIG;
     if (epi == 2 && (!R || !ln_g || !ln_b || N != gemm::LN_N)) return ALBERT_ERR_CONFIG;
     if (epi == 3 && !row_dst) return ALBERT_ERR_NULL;
@@ -1053,7 +1086,7 @@ int albert_test_gemm(const void *A, const void *W, const float *bias, const void
             e = launch_quant_rows_e4m3(static_cast<const bf16 *>(W), K, N, nullptr, qw, sw, nullptr, s, false, false);
     }
     // follows a copy in the stream: a plain launch
-    if (e == cudaSuccess) e = launch_gemm(kepi, ta, tb, to, tr, a, grid, s, variant, false);
+    if (e == cudaSuccess) e = launch_gemm(kepi, ta, tb, to, tr, a, grid, sms, s, variant, false);
     if (e == cudaSuccess && epi == 2)
         e = launch_ln_rows(static_cast<const bf16 *>(zg), stats, ln_g, ln_b, eps, static_cast<bf16 *>(Y), nullptr, M,
                            rows_cap, ints, ints + 1, s);

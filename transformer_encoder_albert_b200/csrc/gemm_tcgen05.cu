@@ -7,8 +7,11 @@
 // A linear layer is y_j = b_j + sum_i x_i W_{j,i} with W stored [out, in]
 // ("Qwen3-TTS and Kokoro", section A), i.e. both operands are K-major.
 //
-// Design (one CTA per SM, persistent over output tiles; two variants):
+// Design (one CTA per SM, persistent over output tiles; three variants):
 //   * single CTA per 128x256 tile: 3-stage ring of {A 128x64, B 256x64};
+//   * single CTA per 128x128 tile ("narrow"): 5-stage ring of {A 128x64,
+//     B 128x64}, epilogue on one warp per lane quadrant -- for few rows, where
+//     256x256 pair tiles would leave SMs idle;
 //   * CTA pair (cluster of 2, tcgen05.mma cta_group::2) per 256x256 tile: each
 //     CTA stages its 128 rows of A and 128 rows of B, 5-stage ring of
 //     {A 128x64, B 128x64} per CTA (the pair is used whenever A has more than
@@ -53,19 +56,20 @@ using namespace gemm;
 // staging tiles per epilogue warp (output, residual or second output, and for
 // the residual epilogue a second output tile, paid for with one stage), then
 // barriers; 1 KiB slack for the 1 KiB alignment of the stages.
-template <int EPI, bool PAIR, bool F8 = false>
+template <int EPI, bool PAIR, bool F8 = false, int TBN = BN>
 struct Plan {
     static constexpr bool kRes = EPI == kEpiResStats;
     static constexpr bool kLnIn = EPI == kEpiLnIn || EPI == kEpiLnInGelu || EPI == kEpiLnInScatter;
-    static constexpr int NST = PAIR ? PAIR_STAGES - 1 : STAGES - 1;
-    static constexpr int BSTAGE = PAIR ? B_HALF_BYTES : B_BYTES;
+    // (128-column tiles halve the B stage, which buys two more stages)
+    static constexpr int NST = PAIR ? PAIR_STAGES - 1 : (TBN == 128 ? STAGES + 1 : STAGES - 1);
+    static constexpr int BSTAGE = PAIR ? B_HALF_BYTES : TBN * 128;  // TBN rows of 128 bytes
     static constexpr int NSTG = kRes ? 3 : 2;
     // per-column vectors of a unit: bias, then W gamma (LayerNorm input) or
     // out_g and res_g (residual epilogue), then for E4M3 operands the weight
     // row scales; two buffers (this unit, the next)
     static constexpr int NVEC_BASE = kLnIn ? 2 : (kRes ? 3 : 1);
     static constexpr int NVEC = NVEC_BASE + (F8 ? 1 : 0);
-    static constexpr int VEC_BYTES = 2 * NVEC * BN * 4;
+    static constexpr int VEC_BYTES = 2 * NVEC * TBN * 4;
     static constexpr int SMEM = 1024 + NST * (A_BYTES + BSTAGE) + NSTG * EPI_WARPS * STG_BYTES + VEC_BYTES + 1024;
     static_assert(SMEM <= 232448, "shared memory per CTA");
 };
@@ -75,7 +79,7 @@ struct Smem {
     uint8_t *stg;            // 2 KB output staging tile per epilogue warp
     uint8_t *rstg;           // 2 KB residual (or second output) staging tile per epilogue warp
     uint8_t *stg2;           // residual epilogue: second 2 KB output staging tile per warp
-    float *vec;              // [2][NVEC][BN] per-column vectors of this unit and the next
+    float *vec;              // [2][NVEC][TBN] per-column vectors of this unit and the next
     uint64_t *vec_full;      // [2]: a unit's vectors are in shared memory
     uint64_t *full, *empty, *tfull, *tempty, *drain, *rbar;
     uint32_t *tmem_slot;
@@ -83,9 +87,9 @@ struct Smem {
     int *misc;               // [0] n_rows, [1] status at entry
 };
 
-template <int EPI, bool PAIR, bool F8>
+template <int EPI, bool PAIR, bool F8, int TBN>
 __device__ __forceinline__ Smem carve(uint8_t *raw) {
-    using P = Plan<EPI, PAIR, F8>;
+    using P = Plan<EPI, PAIR, F8, TBN>;
     constexpr int NST = P::NST;
     Smem s;
     uint8_t *p = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
@@ -197,7 +201,7 @@ __device__ __forceinline__ void row_stats_merge(const float2 (&q)[LN_PARTS], flo
 // F8: both operands are E4M3 (tiles of 128 bytes = 128 elements along K, products
 // with tcgen05.mma kind::f8f6f4, K = 32 per instruction) with fp32 row scales:
 // the epilogue starts from acc * a_scale[row] * w_scale[col].
-template <int EPI, bool PAIR, bool F8>
+template <int EPI, bool PAIR, bool F8, int TBN>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmRes,
@@ -206,12 +210,15 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     constexpr bool kGelu = EPI == kEpiGelu || EPI == kEpiLnInGelu;
     constexpr bool kScatter = EPI == kEpiScatter || EPI == kEpiLnInScatter;
     constexpr bool kRes = EPI == kEpiResStats;
-    constexpr int NST = Plan<EPI, PAIR, F8>::NST;
-    constexpr int BSTAGE = Plan<EPI, PAIR, F8>::BSTAGE;
+    constexpr int NST = Plan<EPI, PAIR, F8, TBN>::NST;
+    constexpr int BSTAGE = Plan<EPI, PAIR, F8, TBN>::BSTAGE;
+    static_assert(TBN == 256 || (TBN == 128 && !PAIR), "tile widths: 256, or 128 for one CTA");
+    constexpr int NH = TBN / 128;      // 128-column halves of a tile
+    constexpr int AEW = 4 * NH;        // epilogue warps with columns (one per lane quadrant and half)
     constexpr int KB = F8 ? 128 : BK;  // K elements per stage (a 128-byte swizzle row)
     constexpr int UM = PAIR ? 2 * BM : BM;  // rows of A (and D) per unit
     extern __shared__ uint8_t smem_raw[];
-    Smem sm = carve<EPI, PAIR, F8>(smem_raw);
+    Smem sm = carve<EPI, PAIR, F8, TBN>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // A pair works on one unit at a time; rank 0 issues the MMAs for both CTAs.
     const uint32_t rank = PAIR ? cluster_ctarank() : 0;
@@ -229,12 +236,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&sm.tfull[i]), 1);
             // the pair's accumulator is released by the epilogues of both CTAs
-            mbar_init(smem_u32(&sm.tempty[i]), PAIR ? 2 * EPI_WARPS : EPI_WARPS);
+            mbar_init(smem_u32(&sm.tempty[i]), PAIR ? 2 * AEW : AEW);
         }
         mbar_init(smem_u32(sm.drain), 1);
         for (int i = 0; i < EPI_WARPS; ++i) mbar_init(smem_u32(&sm.rbar[i]), 1);
         // every epilogue thread arrives once it has stored its columns
-        for (int i = 0; i < 2; ++i) mbar_init(smem_u32(&sm.vec_full[i]), 32 * EPI_WARPS);
+        for (int i = 0; i < 2; ++i) mbar_init(smem_u32(&sm.vec_full[i]), 32 * AEW);
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -262,7 +269,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const int pre = p.withhold_loads ? 0 : (p.K / KB < NST ? p.K / KB : NST);  // stages started early
     if (warp == 0 && lane == 0 && pre > 0) {
         const uint64_t keep = policy_evict_last();
-        const int n = slot % (p.N / BN);
+        const int n = slot % (p.N / TBN);
         for (int st = 0; st < pre; ++st) {
             const uint32_t fb = smem_u32(&sm.full[st]);
             const uint32_t b_dst = smem_u32(sm.b + st * BSTAGE);
@@ -270,9 +277,9 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 if (rank == 0) mbar_expect_tx(fb, 2 * B_HALF_BYTES);
                 tma_load_2d_pair_hint(b_dst, &tmB, mapa_shared(fb, 0), st * KB, n * BN + (int)rank * B_BOX, keep);
             } else {
-                mbar_expect_tx(fb, B_BYTES);
-                tma_load_2d_hint(b_dst, &tmB, fb, st * KB, n * BN, keep);
-                tma_load_2d_hint(b_dst + B_HALF_BYTES, &tmB, fb, st * KB, n * BN + B_BOX, keep);
+                mbar_expect_tx(fb, BSTAGE);
+                tma_load_2d_hint(b_dst, &tmB, fb, st * KB, n * TBN, keep);
+                if (TBN == 256) tma_load_2d_hint(b_dst + B_HALF_BYTES, &tmB, fb, st * KB, n * TBN + B_BOX, keep);
             }
         }
     }
@@ -294,7 +301,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const bool skip = sm.misc[1] != 0 || sm.misc[0] < 0 || sm.misc[0] > p.rows_cap;
     const int n_rows = skip ? 0 : sm.misc[0];
     const int m_blocks = (n_rows + UM - 1) / UM;
-    const int n_sub = p.N / BN;
+    const int n_sub = p.N / TBN;
     const int units = m_blocks * n_sub;  // unit u = tile (u / n_sub, u % n_sub), row-block major
     const int kblocks = p.K / KB;
 
@@ -330,12 +337,13 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         const uint32_t fb0 = mapa_shared(fb, 0);
                         if (rank == 0) mbar_arrive_expect_tx(fb, 2 * (A_BYTES + B_HALF_BYTES));
                         tma_load_2d_pair(a_dst, &tmA, fb0, kb * KB, m * UM + (int)rank * BM);
-                        tma_load_2d_pair_hint(b_dst, &tmB, fb0, kb * KB, n * BN + (int)rank * B_BOX, keep);
+                        tma_load_2d_pair_hint(b_dst, &tmB, fb0, kb * KB, n * TBN + (int)rank * B_BOX, keep);
                     } else {
-                        mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
+                        mbar_arrive_expect_tx(fb, A_BYTES + BSTAGE);
                         tma_load_2d(a_dst, &tmA, fb, kb * KB, m * BM);
-                        tma_load_2d_hint(b_dst, &tmB, fb, kb * KB, n * BN, keep);
-                        tma_load_2d_hint(b_dst + B_HALF_BYTES, &tmB, fb, kb * KB, n * BN + B_BOX, keep);
+                        tma_load_2d_hint(b_dst, &tmB, fb, kb * KB, n * TBN, keep);
+                        if (TBN == 256)
+                            tma_load_2d_hint(b_dst + B_HALF_BYTES, &tmB, fb, kb * KB, n * TBN + B_BOX, keep);
                     }
                     ++issued;
                     if (++stage == NST) { stage = 0; phase ^= 1; }
@@ -361,7 +369,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     } else if (warp == 1) {
         // -------------------------------------------------------- MMA issuer --
         if (lane == 0 && rank == 0) {
-            const uint32_t idesc = F8 ? idesc_e4m3_f32(UM, BN) : idesc_bf16_f32(UM, BN);
+            const uint32_t idesc = F8 ? idesc_e4m3_f32(UM, TBN) : idesc_bf16_f32(UM, TBN);
             int stage = 0, acc = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -370,7 +378,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const uint32_t aph = (acc >> 1) & 1;
                 if (!mbar_wait(smem_u32(&sm.tempty[ab]), aph ^ 1, sm.abort_flag)) break;
                 tc_fence_after();
-                const uint32_t d = tmem_base + ab * BN;
+                const uint32_t d = tmem_base + ab * TBN;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(smem_u32(&sm.full[stage]), phase, sm.abort_flag)) {
                         ok = false;
@@ -410,11 +418,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             else umma_commit(smem_u32(sm.drain));
             mbar_wait_drain(smem_u32(sm.drain), 0);
         }
-    } else {
+    } else if (warp - 2 < AEW) {
         // ---------------------------------------------------------- epilogue --
-        const int ew = warp - 2;            // 0..7
+        // (a 128-column tile keeps warps 6..9 idle: one warp per lane quadrant)
+        const int ew = warp - 2;            // 0..AEW-1
         const int quad = warp & 3;          // TMEM lanes 32*quad .. 32*quad+31
-        const int half = ew >> 2;           // column half of the 256-wide tile
+        const int half = ew >> 2;           // 128-column half of the tile
         const int r_local = quad * 32 + lane;
         const int row_off = (int)rank * BM;  // this CTA's rows within a unit
         const uint32_t stg = smem_u32(sm.stg + ew * STG_BYTES);
@@ -428,7 +437,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         auto res_issue = [&](int u, int c) {
             if (lane == 0) {
                 mbar_arrive_expect_tx(rbar, STG_BYTES);
-                tma_load_2d(rstg, &tmRes, rbar, (u % n_sub) * BN + half * 128 + c * 32,
+                tma_load_2d(rstg, &tmRes, rbar, (u % n_sub) * TBN + half * 128 + c * 32,
                             (u / n_sub) * UM + row_off + quad * 32);
             }
             res_pending = true;
@@ -454,12 +463,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         // stores it at the end of the current unit, and arrives on vec_full.
         // (Read from global memory inside the chunk loop, these uniform loads
         // stalled every chunk on their latency.)
-        constexpr int NVEC = Plan<EPI, PAIR, F8>::NVEC;
-        constexpr int NVEC_BASE = Plan<EPI, PAIR, F8>::NVEC_BASE;
-        const int et = ew * 32 + lane;  // 0..255: the column this thread stages
+        constexpr int NVEC = Plan<EPI, PAIR, F8, TBN>::NVEC;
+        constexpr int NVEC_BASE = Plan<EPI, PAIR, F8, TBN>::NVEC_BASE;
+        const int et = ew * 32 + lane;  // 0..TBN-1: the column this thread stages
         float vreg[NVEC];
         auto vec_load = [&](int un) {
-            const int col = (un % n_sub) * BN + et;
+            const int col = (un % n_sub) * TBN + et;
             vreg[0] = __ldg(p.bias + col);
             if (kLnIn) vreg[1] = __ldg(p.fold_s + col);
             if (kRes) {
@@ -470,7 +479,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         };
         auto vec_store = [&](int b) {
 #pragma unroll
-            for (int i = 0; i < NVEC; ++i) sm.vec[(b * NVEC + i) * BN + et] = vreg[i];
+            for (int i = 0; i < NVEC; ++i) sm.vec[(b * NVEC + i) * TBN + et] = vreg[i];
             mbar_arrive(smem_u32(&sm.vec_full[b]));
         };
         if (slot < units) {
@@ -505,12 +514,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             if (!got) { ok = false; break; }
             tc_fence_after();
             // shared addresses of this warp's 128 columns of each vector
-            const uint32_t vbias = smem_u32(sm.vec + (vb * NVEC) * BN + half * 128);
-            const uint32_t vsec = vbias + BN * 4;           // W gamma or out_g
-            const uint32_t vres = smem_u32(sm.vec + (vb * NVEC + NVEC_BASE - 1) * BN + half * 128);  // res_g
-            const uint32_t vws = smem_u32(sm.vec + (vb * NVEC + NVEC - 1) * BN + half * 128);  // w_scale (F8)
-            const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + ab * BN + half * 128;
-            const int ncol0 = n * BN + half * 128;  // first output column of this warp
+            const uint32_t vbias = smem_u32(sm.vec + (vb * NVEC) * TBN + half * 128);
+            const uint32_t vsec = vbias + TBN * 4;          // W gamma or out_g
+            const uint32_t vres = smem_u32(sm.vec + (vb * NVEC + NVEC_BASE - 1) * TBN + half * 128);  // res_g
+            const uint32_t vws = smem_u32(sm.vec + (vb * NVEC + NVEC - 1) * TBN + half * 128);  // w_scale (F8)
+            const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + ab * TBN + half * 128;
+            const int ncol0 = n * TBN + half * 128;  // first output column of this warp
             float mean = 0.f, m2 = 0.f;
             // chunk c + 1 loads from TMEM while chunk c is processed
             uint32_t r[2][32];
@@ -647,7 +656,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 }
             }
             if (!ok) break;
-            if (kRes && row < p.rows_cap) p.out_stats[(size_t)row * LN_PARTS + n * 2 + half] = make_float2(mean, m2);
+            if (kRes && row < p.rows_cap) p.out_stats[(size_t)row * LN_PARTS + n * NH + half] = make_float2(mean, m2);
             ++acc;
             // the next unit's vectors: buffer (j + 1) & 1 was last read in unit j - 1,
             // which every epilogue thread finished before arriving for unit j
@@ -678,17 +687,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
 }  // namespace
 
-bool gemm_use_pair(int rows_cap, int variant) {
-    if (variant == kGemmPair) return true;
-    if (variant == kGemmSingle) return false;
-    return rows_cap > BM;
-}
 
 // The kernel instance's shared-memory limit, raised once per device.
-template <int EPI, bool PAIR, bool F8>
+template <int EPI, bool PAIR, bool F8, int TBN = BN>
 static cudaError_t configure(int smem) {
     static std::atomic<unsigned long long> configured{0};
-    return ensure_smem_attr(reinterpret_cast<const void *>(gemm_bf16_kernel<EPI, PAIR, F8>), smem, configured);
+    return ensure_smem_attr(reinterpret_cast<const void *>(gemm_bf16_kernel<EPI, PAIR, F8, TBN>), smem, configured);
 }
 
 // Clusters of two GEMM CTAs that fit on the device at once (every epilogue
@@ -712,7 +716,7 @@ static int pair_clusters(int num_sms) {
         cfg.dynamicSmemBytes = Plan<kEpiBias, true>::SMEM;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaOccupancyMaxActiveClusters(&n, gemm_bf16_kernel<kEpiBias, true, false>, &cfg) != cudaSuccess) n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_bf16_kernel<kEpiBias, true, false, BN>, &cfg) != cudaSuccess) n = 0;
     }
     cudaGetLastError();
     if (n <= 0 || n > num_sms / 2) n = num_sms / 2;
@@ -720,31 +724,54 @@ static int pair_clusters(int num_sms) {
     return n;
 }
 
+// The kernel a launch takes.  Auto: one CTA per 128x256 tile for a single
+// 128-row block; otherwise the CTA pair per 256x256 tile, unless that leaves
+// clusters idle while 128x128 tiles on one CTA each would all run at once
+// (few rows: the narrower tile halves each unit's main loop and spreads the
+// work over more SMs).
+int gemm_resolve(int rows_cap, int N, int num_sms, int variant) {
+    if (variant != kGemmAuto) return variant;
+    if (rows_cap <= BM) return kGemmSingle;
+    const int pair_units = ((rows_cap + 2 * BM - 1) / (2 * BM)) * (N / BN);
+    const int narrow_units = ((rows_cap + BM - 1) / BM) * (N / 128);
+    if (N % 128 == 0 && pair_units < pair_clusters(num_sms) && narrow_units <= num_sms) return kGemmNarrow;
+    return kGemmPair;
+}
+
 int gemm_grid(int epi, int rows_cap, int N, int num_sms, int variant) {
     (void)epi;
-    if (gemm_use_pair(rows_cap, variant)) {
+    const int v = gemm_resolve(rows_cap, N, num_sms, variant);
+    if (v == kGemmPair) {
         const int units = ((rows_cap + 2 * BM - 1) / (2 * BM)) * (N / BN);
         const int clusters = pair_clusters(num_sms);
         return 2 * (units < clusters ? (units > 0 ? units : 1) : clusters);
     }
-    const int units = ((rows_cap + BM - 1) / BM) * (N / BN);
+    const int units = ((rows_cap + BM - 1) / BM) * (N / (v == kGemmNarrow ? 128 : BN));
     return units < num_sms ? (units > 0 ? units : 1) : num_sms;
+}
+
+template <int EPI, bool F8, int TBN>
+static cudaError_t launch_single(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
+                                 const CUtensorMap &tmRes, const GemmArgs &a, int grid, cudaStream_t s, bool pdl) {
+    constexpr int smem = Plan<EPI, false, F8, TBN>::SMEM;
+    cudaError_t e = configure<EPI, false, F8, TBN>(smem);
+    if (e != cudaSuccess) return e;
+    if (!pdl) {
+        gemm_bf16_kernel<EPI, false, F8, TBN><<<grid, THREADS, smem, s>>>(tmA, tmB, tmOut, tmRes, a);
+        return cudaGetLastError();
+    }
+    return launch_pdl(gemm_bf16_kernel<EPI, false, F8, TBN>, dim3(grid), dim3(THREADS), smem, s, tmA, tmB, tmOut,
+                      tmRes, a);
 }
 
 template <int EPI, bool F8>
 static cudaError_t launch_one(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
-                              const CUtensorMap &tmRes, const GemmArgs &a, int grid, cudaStream_t s, bool pair,
+                              const CUtensorMap &tmRes, const GemmArgs &a, int grid, cudaStream_t s, int v,
                               bool pdl) {
-    if (!pair) {
-        constexpr int smem = Plan<EPI, false, F8>::SMEM;
-        cudaError_t e = configure<EPI, false, F8>(smem);
-        if (e != cudaSuccess) return e;
-        if (!pdl) {
-            gemm_bf16_kernel<EPI, false, F8><<<grid, THREADS, smem, s>>>(tmA, tmB, tmOut, tmRes, a);
-            return cudaGetLastError();
-        }
-        return launch_pdl(gemm_bf16_kernel<EPI, false, F8>, dim3(grid), dim3(THREADS), smem, s, tmA, tmB, tmOut, tmRes,
-                          a);
+    if (v == kGemmSingle) return launch_single<EPI, F8, BN>(tmA, tmB, tmOut, tmRes, a, grid, s, pdl);
+    if (v == kGemmNarrow) {
+        if (a.N % 128) return cudaErrorInvalidValue;
+        return launch_single<EPI, F8, 128>(tmA, tmB, tmOut, tmRes, a, grid, s, pdl);
     }
     if (grid < 2 || grid % 2) return cudaErrorInvalidConfiguration;
     cudaError_t e = configure<EPI, true, F8>(Plan<EPI, true, F8>::SMEM);
@@ -763,33 +790,33 @@ static cudaError_t launch_one(const CUtensorMap &tmA, const CUtensorMap &tmB, co
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, gemm_bf16_kernel<EPI, true, F8>, tmA, tmB, tmOut, tmRes, a);
+    return cudaLaunchKernelEx(&cfg, gemm_bf16_kernel<EPI, true, F8, BN>, tmA, tmB, tmOut, tmRes, a);
 }
 
 cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
-                        const CUtensorMap &tmRes, const GemmArgs &a, int grid, cudaStream_t s, int variant,
-                        bool pdl) {
-    const bool pair = gemm_use_pair(a.rows_cap, variant);
+                        const CUtensorMap &tmRes, const GemmArgs &a, int grid, int num_sms, cudaStream_t s,
+                        int variant, bool pdl) {
+    const int v = gemm_resolve(a.rows_cap, a.N, num_sms, variant);
     if (a.e4m3) {
         // the E4M3 variant serves the four layer GEMMs and the single-kernel tests
         switch (epi) {
-            case kEpiBias: return launch_one<kEpiBias, true>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-            case kEpiGelu: return launch_one<kEpiGelu, true>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-            case kEpiResStats: return launch_one<kEpiResStats, true>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-            case kEpiScatter: return launch_one<kEpiScatter, true>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-            case kEpiLnIn: return launch_one<kEpiLnIn, true>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-            case kEpiLnInGelu: return launch_one<kEpiLnInGelu, true>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+            case kEpiBias: return launch_one<kEpiBias, true>(tmA, tmB, tmOut, tmRes, a, grid, s, v, pdl);
+            case kEpiGelu: return launch_one<kEpiGelu, true>(tmA, tmB, tmOut, tmRes, a, grid, s, v, pdl);
+            case kEpiResStats: return launch_one<kEpiResStats, true>(tmA, tmB, tmOut, tmRes, a, grid, s, v, pdl);
+            case kEpiScatter: return launch_one<kEpiScatter, true>(tmA, tmB, tmOut, tmRes, a, grid, s, v, pdl);
+            case kEpiLnIn: return launch_one<kEpiLnIn, true>(tmA, tmB, tmOut, tmRes, a, grid, s, v, pdl);
+            case kEpiLnInGelu: return launch_one<kEpiLnInGelu, true>(tmA, tmB, tmOut, tmRes, a, grid, s, v, pdl);
         }
         return cudaErrorInvalidValue;
     }
     switch (epi) {
-        case kEpiBias: return launch_one<kEpiBias, false>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-        case kEpiGelu: return launch_one<kEpiGelu, false>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-        case kEpiResStats: return launch_one<kEpiResStats, false>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-        case kEpiScatter: return launch_one<kEpiScatter, false>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-        case kEpiLnIn: return launch_one<kEpiLnIn, false>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-        case kEpiLnInGelu: return launch_one<kEpiLnInGelu, false>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
-        case kEpiLnInScatter: return launch_one<kEpiLnInScatter, false>(tmA, tmB, tmOut, tmRes, a, grid, s, pair, pdl);
+        case kEpiBias: return launch_one<kEpiBias, false>(tmA, tmB, tmOut, tmRes, a, grid, s, v, pdl);
+        case kEpiGelu: return launch_one<kEpiGelu, false>(tmA, tmB, tmOut, tmRes, a, grid, s, v, pdl);
+        case kEpiResStats: return launch_one<kEpiResStats, false>(tmA, tmB, tmOut, tmRes, a, grid, s, v, pdl);
+        case kEpiScatter: return launch_one<kEpiScatter, false>(tmA, tmB, tmOut, tmRes, a, grid, s, v, pdl);
+        case kEpiLnIn: return launch_one<kEpiLnIn, false>(tmA, tmB, tmOut, tmRes, a, grid, s, v, pdl);
+        case kEpiLnInGelu: return launch_one<kEpiLnInGelu, false>(tmA, tmB, tmOut, tmRes, a, grid, s, v, pdl);
+        case kEpiLnInScatter: return launch_one<kEpiLnInScatter, false>(tmA, tmB, tmOut, tmRes, a, grid, s, v, pdl);
     }
     return cudaErrorInvalidValue;
 }

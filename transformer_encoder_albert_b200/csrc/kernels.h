@@ -133,11 +133,13 @@ int make_tmap_e4m3(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t co
 // swizzle: the epilogue's output stores and residual loads.
 int make_tmap_bf16_tile32(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t cols);
 
-// Kernel variant: one CTA per 128x256 tile, or a CTA pair (cluster of 2,
-// tcgen05.mma cta_group::2) per 256x256 tile.  Auto takes the pair whenever
-// the A buffer holds more than one 128-row block.
-enum GemmVariant { kGemmAuto = 0, kGemmSingle = 1, kGemmPair = 2 };
-bool gemm_use_pair(int rows_cap, int variant);
+// Kernel variant: one CTA per 128x256 tile, a CTA pair (cluster of 2,
+// tcgen05.mma cta_group::2) per 256x256 tile, or one CTA per 128x128 tile.
+// Auto (gemm_resolve): the single CTA for one 128-row block; the narrow tile
+// when pairs would leave clusters idle and every narrow tile runs at once;
+// else the pair.
+enum GemmVariant { kGemmAuto = 0, kGemmSingle = 1, kGemmPair = 2, kGemmNarrow = 3 };
+int gemm_resolve(int rows_cap, int N, int num_sms, int variant);
 
 // Grid (CTAs) the GEMM uses for this many rows: persistent, at most one CTA per
 // SM, and for the pair variant an even count within the co-resident clusters.
@@ -151,8 +153,9 @@ inline bool gemm_vectors_aligned(const GemmArgs &a) {
 
 // tmOut: tile32 map of the output (unused by the scatter epilogues); tmRes: tile32
 // map of the residual (kEpiResStats only; pass any valid map otherwise).
+// grid: from gemm_grid with the same rows_cap, N, num_sms and variant.
 cudaError_t launch_gemm(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
-                        const CUtensorMap &tmRes, const GemmArgs &args, int grid, cudaStream_t s,
+                        const CUtensorMap &tmRes, const GemmArgs &args, int grid, int num_sms, cudaStream_t s,
                         int variant = kGemmAuto, bool pdl = true);
 
 // ------------------------------------------------- small-batch whole forward --
