@@ -358,12 +358,25 @@ int albert_test_quant_e4m3(const void *x, int rows, int K, void *q, float *scale
  * (Q | K | V, head h = columns 64h..64h+63 of each); cu_seqlens as in
  * albert_forward_varlen; ctx: [N_tok, 768] bf16.  dtype ALBERT_BF16 runs the
  * kernel the forward pass uses for this max_len (tcgen05 with one item per
- * (sequence, head) for max_len <= 128; tcgen05 with one item per (sequence,
- * 128-query block, head) and all of its scores in tensor memory for
- * 128 < max_len <= 512); 2 forces the mma.sync kernel; ALBERT_FP32 runs the
- * fp32 kernel on fp32 buffers. */
+ * (group, head) for max_len <= 128, a group being one sequence or two of at
+ * most 64 tokens each (albert_test_attention_groups);
+ * tcgen05 with one item per (sequence, 128-query block, head) and all of its
+ * scores in tensor memory for 128 < max_len <= 512); 2 forces the mma.sync
+ * kernel; ALBERT_FP32 runs the fp32 kernel on fp32 buffers. */
 int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, int max_len,
                           void *ctx, int dtype, void *stream);
+
+/* The attention groups the forward pass forms for a packed batch (device
+ * cu_seqlens as in albert_forward_varlen): the sequences of at most 64 tokens
+ * are paired in batch order (1st with 2nd, 3rd with 4th, ...), each pair sharing
+ * one item as its two 64-row halves; longer sequences and an unpaired last short
+ * one have an item each.  groups_out: host, room for nseq int32 quadruples
+ * {start row, length, partner start row, partner length (0: none)}: the pairs
+ * first, then the longer sequences in batch order, then the unpaired short one;
+ * *n_out: the number written.
+ * Synchronous.  Invalid cu_seqlens: ALBERT_ERR_SEQLENS. */
+int albert_test_attention_groups(const int32_t *cu_seqlens, int nseq, int max_len, int32_t *groups_out,
+                                 int *n_out, void *stream);
 
 /* ---- residual + LayerNorm GEMM without any device allocation ----
  * The pages have no counterpart of this entry point; it exists for callers

@@ -131,6 +131,34 @@ def test_attention_tcgen05_short_sequences():
     _attention_case([1, 2, 3, 15, 16, 17, 31, 32, 33, 63, 64, 65, 96, 127, 128, 40, 5], seed=7)
 
 
+def test_attention_tcgen05_paired_sequences():
+    """Sequences of at most 64 tokens share an item two by two (64-row halves):
+    halves of 1, 31, 32, 33, 63 and 64 rows, a pair's second half shorter and
+    longer than 32, longer sequences in between, an odd count (one unpaired), and
+    peaked scores, so that a key leaking from one half into the other would show."""
+    r = np.random.default_rng(21)
+    lengths = [1, 64, 100, 64, 33, 31, 128, 32, 63, 65, 2, 40, 127, 17, 3, 50, 64]
+    lengths += [int(x) for x in r.integers(1, 129, 40)]
+    _attention_case(lengths, seed=22, scale=2.0)
+
+
+@pytest.mark.parametrize("case", ["uniform", "all_short", "boundary"])
+def test_attention_groups_match_definition(case):
+    """The device's grouping (warp ballots) equals the plain definition."""
+    from test_attention_groups_cpu import pair_groups, packed
+    r = np.random.default_rng({"uniform": 1, "all_short": 2, "boundary": 3}[case])
+    if case == "uniform":
+        L = r.integers(16, 129, 256)
+    elif case == "all_short":
+        L = r.integers(1, 65, 301)
+    else:
+        L = r.choice([1, 63, 64, 65, 127, 128], 97)
+    starts, lens = packed(L)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32), device="cuda")
+    got = tea.test_attention_groups(cu, int(max(lens)))
+    assert got == [tuple(map(int, g)) for g in pair_groups(starts, lens)]
+
+
 def test_attention_mma_sync_kernel_short_sequences():
     _attention_case([1, 16, 33, 64, 100, 128], seed=8, legacy=True)
 

@@ -42,7 +42,7 @@ EXPORTS = (
     "albert_profile_name", "albert_profile_read", "albert_test_gemm", "albert_test_attention",
     "albert_gemm_residual_ln_noalloc", "albert_length_regulate", "albert_length_regulate_scratch_bytes",
     "albert_set_wait_limit", "albert_test_stall", "albert_set_small_batch_kernel", "albert_last_forward_launches",
-    "albert_test_quant_e4m3", "albert_forward_embedded",
+    "albert_test_quant_e4m3", "albert_forward_embedded", "albert_test_attention_groups",
 )
 
 
@@ -106,6 +106,7 @@ def lib() -> C.CDLL:
         L.albert_last_forward_launches.argtypes = [vp]
         L.albert_test_quant_e4m3.argtypes = [vp, i, i, vp, vp, vp]
         L.albert_forward_embedded.argtypes = [vp, vp, vp, i, i, vp, vp]
+        L.albert_test_attention_groups.argtypes = [vp, i, i, vp, C.POINTER(C.c_int), vp]
         _lib = L
     return _lib
 
@@ -354,6 +355,18 @@ def test_gemm(A, W, bias, Y, epi: int, R=None, ln_g=None, ln_b=None, eps: float 
     return lib().albert_test_gemm(_ptr(A), _ptr(W), _ptr(bias), _ptr(R), _ptr(ln_g), _ptr(ln_b),
                                   float(eps), _ptr(row_dst), _ptr(Y), M, N, K,
                                   epi | GEMM_VARIANTS[variant] | (GEMM_E4M3 if e4m3 else 0), _stream_ptr(stream))
+
+
+def test_attention_groups(cu_seqlens, max_len: int, stream=None):
+    """The attention groups the forward forms for a packed batch: a list of
+    (start row, length, partner start row, partner length (0: none))."""
+    import numpy as np
+    nseq = cu_seqlens.numel() - 1
+    buf = np.zeros((nseq, 4), dtype=np.int32)
+    n = C.c_int(0)
+    _check(lib().albert_test_attention_groups(_ptr(cu_seqlens), nseq, int(max_len), buf.ctypes.data, C.byref(n),
+                                              _stream_ptr(stream)), "albert_test_attention_groups")
+    return [tuple(int(x) for x in g) for g in buf[:n.value]]
 
 
 def test_quant_e4m3(x, stream=None):

@@ -79,6 +79,8 @@ struct albert_handle {
     float *fold = nullptr;
     float *s_out = nullptr, *c_out = nullptr;
     int *seq_start = nullptr, *seq_len = nullptr, *row_dst = nullptr, *n_rows = nullptr, *status = nullptr;
+    int4 *att_groups = nullptr;  // attention items of sequences <= 128 tokens (one or two sequences each)
+    int *n_att_groups = nullptr;
 
     // out_layout 1: token-major staging of the output, transposed per sequence into `out`
     void *tout = nullptr;
@@ -400,9 +402,9 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
             }
             if (rc) return rc;
             if (max_len <= kAttnTcMaxLen) {
-                LAUNCH(L, kProfAttention, launch_attention_tc(h->tm_QKV, h->tm_QKV64, static_cast<bf16 *>(h->C), h->seq_start,
-                                                             h->seq_len, nseq, h->status, h->num_sms, L.s, true,
-                                                             h->wait_ns));
+                LAUNCH(L, kProfAttention, launch_attention_tc(h->tm_QKV, h->tm_QKV64, static_cast<bf16 *>(h->C),
+                                                             h->att_groups, h->n_att_groups, nseq, h->status,
+                                                             h->num_sms, L.s, true, h->wait_ns));
             } else if (max_len <= kAttnTcLongMaxLen) {
                 LAUNCH(L, kProfAttention, launch_attention_tc_long(h->tm_QKV, static_cast<bf16 *>(h->C), h->seq_start,
                                                                   h->seq_len, nseq, h->status, h->num_sms, L.s, true,
@@ -665,8 +667,10 @@ int create_impl(albert_handle *h, const albert_weights *w) {
     if ((rc = dev_alloc(h, (void **)&h->seq_start, (h->seq_cap + 1) * sizeof(int)))) return rc;
     if ((rc = dev_alloc(h, (void **)&h->seq_len, (h->seq_cap + 1) * sizeof(int)))) return rc;
     if ((rc = dev_alloc(h, (void **)&h->row_dst, R * sizeof(int)))) return rc;
-    if ((rc = dev_alloc(h, (void **)&h->n_rows, 2 * sizeof(int)))) return rc;
+    if ((rc = dev_alloc(h, (void **)&h->n_rows, 4 * sizeof(int)))) return rc;
     h->status = h->n_rows + 1;
+    h->n_att_groups = h->n_rows + 2;
+    if ((rc = dev_alloc(h, (void **)&h->att_groups, (h->seq_cap + 1) * sizeof(int4)))) return rc;
     if ((rc = dev_alloc(h, (void **)&h->st_ids, (size_t)c.max_tokens * sizeof(int64_t)))) return rc;
     if ((rc = dev_alloc(h, (void **)&h->st_mask, (size_t)c.max_tokens))) return rc;
     if ((rc = dev_alloc(h, &h->st_out, (size_t)c.max_tokens * out_width(h) * eb))) return rc;
@@ -676,7 +680,7 @@ int create_impl(albert_handle *h, const albert_weights *w) {
         size_t bytes = (p == h->E ? kEmb : p == h->QKV ? kQKV : p == h->H ? kFfn : kHidden) * R * eb;
         TRY(cudaMemsetAsync(p, 0, bytes, s));
     }
-    TRY(cudaMemsetAsync(h->n_rows, 0, 2 * sizeof(int), s));
+    TRY(cudaMemsetAsync(h->n_rows, 0, 4 * sizeof(int), s));
 
     // ---- TMA descriptors ----
     if (bf) {
@@ -751,7 +755,7 @@ int forward_padded(albert_handle *h, const int64_t *ids, const uint8_t *mask, in
     h->last_launches = 0;
     Launch L{h, s};
     LAUNCH(L, kProfPrep, launch_prep_padded(mask, B, T, h->cfg.pack, h->cfg.max_tokens, h->seq_start, h->seq_len,
-                                            h->n_rows, h->status, s, true));
+                                            h->n_rows, h->status, h->att_groups, h->n_att_groups, s, true));
     return run_layers(h, L, ids, 1, B, T, T, out, 1);
 }
 
@@ -794,7 +798,7 @@ int albert_forward_varlen(albert_handle *h, const int64_t *ids, const int32_t *c
     h->last_launches = 0;
     Launch L{h, s};
     LAUNCH(L, kProfPrep, launch_prep_varlen(cu_seqlens, nseq, max_len, h->cfg.max_tokens, h->seq_start, h->seq_len,
-                                            h->n_rows, h->status, s, true));
+                                            h->n_rows, h->status, h->att_groups, h->n_att_groups, s, true));
     return run_layers(h, L, ids, 0, nseq, 0, max_len, out, 0);
 }
 
@@ -808,7 +812,7 @@ int albert_forward_embedded(albert_handle *h, const float *emb, const int32_t *c
     h->last_launches = 0;
     Launch L{h, s};
     LAUNCH(L, kProfPrep, launch_prep_varlen(cu_seqlens, nseq, max_len, h->cfg.max_tokens, h->seq_start, h->seq_len,
-                                            h->n_rows, h->status, s, true));
+                                            h->n_rows, h->status, h->att_groups, h->n_att_groups, s, true));
     return run_layers(h, L, nullptr, 0, nseq, 0, max_len, out, 0, emb);
 }
 
@@ -1126,9 +1130,12 @@ int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, 
     TRY(cudaMemcpy(&n_tok, cu_seqlens + nseq, sizeof(int), cudaMemcpyDeviceToHost));
     if (n_tok < 1) return ALBERT_ERR_SHAPE;
     int *ints = nullptr;
-    TRY(cudaMalloc(&ints, (2 * (size_t)nseq + 4) * sizeof(int)));
-    int *seq_start = ints, *seq_len = ints + nseq + 1, *n_rows = seq_len + nseq + 1, *status = n_rows + 1;
-    cudaError_t e = launch_prep_varlen(cu_seqlens, nseq, max_len, 1 << 30, seq_start, seq_len, n_rows, status, s, false);
+    TRY(cudaMalloc(&ints, (6 * (size_t)nseq + 12) * sizeof(int)));
+    int4 *groups = reinterpret_cast<int4 *>(ints);  // [nseq], first: 16-byte aligned
+    int *seq_start = ints + 4 * (size_t)nseq, *seq_len = seq_start + nseq + 1, *n_rows = seq_len + nseq + 1;
+    int *status = n_rows + 1, *n_groups = n_rows + 2;
+    cudaError_t e = launch_prep_varlen(cu_seqlens, nseq, max_len, 1 << 30, seq_start, seq_len, n_rows, status, groups,
+                                       n_groups, s, false);
     if (e == cudaSuccess) {
         if (dtype == ALBERT_FP32) {
             e = launch_attention_f32(static_cast<const float *>(qkv), static_cast<float *>(ctx), seq_start, seq_len, nseq,
@@ -1138,7 +1145,7 @@ int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, 
             if (make_tmap_bf16(&tm, qkv, (uint64_t)n_tok, kQKV, 128) || make_tmap_bf16(&tm64, qkv, (uint64_t)n_tok, kQKV, 64))
                 e = cudaErrorInvalidValue;
             else if (max_len <= kAttnTcMaxLen)
-                e = launch_attention_tc(tm, tm64, static_cast<bf16 *>(ctx), seq_start, seq_len, nseq, status, sms, s,
+                e = launch_attention_tc(tm, tm64, static_cast<bf16 *>(ctx), groups, n_groups, nseq, status, sms, s,
                                         false);
             else
                 e = launch_attention_tc_long(tm, static_cast<bf16 *>(ctx), seq_start, seq_len, nseq, status, sms, s,
@@ -1153,6 +1160,32 @@ int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, 
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     cudaFree(ints);
     return e == cudaSuccess ? st : ALBERT_ERR_CUDA;
+}
+
+int albert_test_attention_groups(const int32_t *cu_seqlens, int nseq, int max_len, int32_t *groups_out, int *n_out,
+                                 void *stream) {
+    if (!cu_seqlens || !groups_out || !n_out) return ALBERT_ERR_NULL;
+    if (nseq < 1 || max_len < 1 || max_len > kMaxPos) return ALBERT_ERR_SHAPE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int *ints = nullptr;
+    TRY(cudaMalloc(&ints, (6 * (size_t)nseq + 12) * sizeof(int)));
+    int4 *groups = reinterpret_cast<int4 *>(ints);  // [nseq], first: 16-byte aligned
+    int *seq_start = ints + 4 * (size_t)nseq, *seq_len = seq_start + nseq + 1, *n_rows = seq_len + nseq + 1;
+    int *status = n_rows + 1, *n_groups = n_rows + 2;
+    int host[2] = {0, 0};
+    cudaError_t e = launch_prep_varlen(cu_seqlens, nseq, max_len, 1 << 30, seq_start, seq_len, n_rows, status, groups,
+                                       n_groups, s, false);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(host, status, 2 * sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    const int ng = host[1];
+    if (e == cudaSuccess && host[0] == 0 && ng >= 0 && ng <= nseq)
+        e = cudaMemcpy(groups_out, groups, (size_t)ng * sizeof(int4), cudaMemcpyDeviceToHost);
+    cudaFree(ints);
+    if (e != cudaSuccess) return ALBERT_ERR_CUDA;
+    if (host[0] != 0) return host[0];
+    if (ng < 0 || ng > nseq) return ALBERT_ERR_CUDA;
+    *n_out = ng;
+    return ALBERT_OK;
 }
 
 }  // extern "C"

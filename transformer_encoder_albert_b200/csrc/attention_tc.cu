@@ -7,12 +7,18 @@
 //     C_h = softmax(Q_h K_h^T / sqrt(64) + mask) V_h,
 // key u of sequence b takes part iff u < L_b, every query sees both sides.
 //
-// One work item = (sequence, head), all L_b <= 128 queries and keys at once.
-// The (start, length) of every item of the CTA is read into shared memory
-// once, before the roles start (a global load per item on the issuing
-// threads' path cost about as much as the item itself).
+// One work item = (group, head), all of the group's <= 128 queries and keys at
+// once.  A group is one sequence, or two sequences of at most 64 tokens (paired
+// by the prep kernels) loaded as the two 64-row halves of the item's tiles:
+// queries, keys and values of the first in rows 0..63, of the second in rows
+// 64..127, each query taking only the keys of its own half.  Every softmax warp
+// then has real rows, where a lone short sequence leaves half of them idle.
+// The group entries of every item of the CTA are read into shared memory once,
+// before the roles start (a global load per item on the issuing threads' path
+// cost about as much as the item itself).
 //   warp 0      : TMA producer of the head's Q and K tiles (128 or 64 rows x
-//                 64, 128-byte swizzle) from the packed [rows, 3*768] buffer
+//                 64, or two 64-row halves; 128-byte swizzle) from the packed
+//                 [rows, 3*768] buffer
 //                 into a ring of stages; a Q/K stage is free again as soon as
 //                 the S product has read it, so Q/K loads run well ahead.  It
 //                 also loads the V tiles of the first four items; the V tile
@@ -29,10 +35,11 @@
 //                 serializes the two products of successive items;
 //   warps 2..9  : two softmax groups of 4 warps (items alternate between
 //                 them): each thread owns one query row, reads its scores from
-//                 TMEM, applies the mask and a max-subtracted softmax in
-//                 registers (no cross-thread reductions), writes P as packed
-//                 bf16 back into TMEM over scores it has read and 1/sum into
-//                 shared memory, and moves on to its next item;
+//                 TMEM, applies the mask (keys of the row's own sequence) and
+//                 a max-subtracted softmax in registers (no cross-thread
+//                 reductions), writes P as packed bf16 back into TMEM over
+//                 scores it has read (zeros for every other key of the item)
+//                 and 1/sum into shared memory, and moves on to its next item;
 //   warps 10..13: output group: per item, reads its rows of O from TMEM once
 //                 O = P V is complete, scales them by 1/sum and stores them.
 // TMEM holds four 128-column item buffers: S fills a buffer, P is packed into
@@ -55,7 +62,7 @@ constexpr int NBUF = 4;                        // TMEM item buffers (128 columns
 constexpr int ATC_THREADS = 32 * 15;
 constexpr int ATC_O_WARP = 14;                 // issuer of the O = P V products
 constexpr int ATC_ITEM_CAP = 512;              // items whose (start, length) are kept in shared memory
-constexpr int ATC_SMEM = 1024 + (2 * NQK + NV) * TILE + NBUF * TROWS * 4 + ATC_ITEM_CAP * 8 + 512;
+constexpr int ATC_SMEM = 1024 + (2 * NQK + NV) * TILE + NBUF * TROWS * 4 + ATC_ITEM_CAP * 16 + 512;
 constexpr uint32_t TM_O = 64;                  // O's first column within an item buffer
 // Item n uses Q/K stage, V stage and TMEM buffer n % 4 alike, so a Q/K stage is
 // free when the S product of the item four back completes (s_full) and a V
@@ -74,7 +81,7 @@ struct AttSmem {
     int *misc;
     int *qk_len, *v_len;                       // length of the item a stage holds
     float *inv_sum;                            // [NBUF][TROWS]
-    int2 *item;                                // [ATC_ITEM_CAP] (start, length) of the CTA's items
+    int4 *item;                                // [ATC_ITEM_CAP] group entries of the CTA's items
     int *n_issued;                             // [0] Q/K, [1] V loads issued (read by the teardown)
 };
 
@@ -84,7 +91,7 @@ __device__ __forceinline__ AttSmem att_carve(uint8_t *raw) {
     s.qk = p;
     s.v = p + 2 * NQK * TILE;
     s.inv_sum = reinterpret_cast<float *>(s.v + NV * TILE);
-    s.item = reinterpret_cast<int2 *>(s.v + NV * TILE + NBUF * TROWS * 4);
+    s.item = reinterpret_cast<int4 *>(s.v + NV * TILE + NBUF * TROWS * 4);
     uint64_t *b = reinterpret_cast<uint64_t *>(s.item + ATC_ITEM_CAP);
     s.qk_full = b;
     s.v_full = b + 2 * NQK;
@@ -104,28 +111,45 @@ __device__ __forceinline__ AttSmem att_carve(uint8_t *raw) {
     return s;
 }
 
-// (start, length) of the CTA's item j (id = blockIdx.x + j * gridDim.x)
-__device__ __forceinline__ int2 item_info(const AttSmem &sm, int j, const int *seq_start, const int *seq_len) {
+// Group entry {start, length, partner start, partner length} of the CTA's item j
+// (id = blockIdx.x + j * gridDim.x = group * 12 + head).
+__device__ __forceinline__ int4 item_info(const AttSmem &sm, int j, const int4 *groups) {
     if (j < ATC_ITEM_CAP) return sm.item[j];
-    const int b = (blockIdx.x + j * gridDim.x) / kHeads;
-    return make_int2(__ldg(seq_start + b), __ldg(seq_len + b));
+    return groups[(blockIdx.x + j * gridDim.x) / kHeads];
+}
+__device__ __forceinline__ bool item_pair(int4 it) { return it.w > 0; }
+// rows (and keys) of the item's tiles: a pair fills both 64-row halves
+__device__ __forceinline__ int item_rows(int4 it) { return it.w > 0 ? TROWS : it.y; }
+
+// TMA load of 64 columns (one head) of the item's rows into a 128-row tile: one
+// box, or one 64-row box per half for a pair (the second lands 64 rows = 8 KB in,
+// a multiple of the 1 KB swizzle period).
+__device__ __forceinline__ void load_item_tile(uint32_t dst, int4 it, int col, const CUtensorMap *tmQKV,
+                                               const CUtensorMap *tmQKV64, uint32_t bar) {
+    if (item_pair(it)) {
+        tma_load_2d(dst, tmQKV64, bar, col, it.x);
+        tma_load_2d(dst + TILE / 2, tmQKV64, bar, col, it.z);
+    } else {
+        tma_load_2d(dst, it.y <= 64 ? tmQKV64 : tmQKV, bar, col, it.x);
+    }
 }
 
 // TMA load of the V tile of the CTA's item n into V stage n % NV (one thread).
-__device__ __forceinline__ void issue_v(const AttSmem &sm, int n, int2 it, const CUtensorMap *tmQKV,
+__device__ __forceinline__ void issue_v(const AttSmem &sm, int n, int4 it, const CUtensorMap *tmQKV,
                                         const CUtensorMap *tmQKV64) {
     const int h = (blockIdx.x + n * gridDim.x) % kHeads;
     const int st = n % NV;
-    sm.v_len[st] = it.y;  // read by the O issuer once the stage is full
+    const int rows = item_rows(it);
+    sm.v_len[st] = rows;  // read by the O issuer once the stage is full
     const uint32_t fb = smem_u32(&sm.v_full[st]);
-    mbar_arrive_expect_tx(fb, it.y <= 64 ? TILE / 2 : TILE);
-    tma_load_2d(smem_u32(sm.v + st * TILE), it.y <= 64 ? tmQKV64 : tmQKV, fb, 2 * kHidden + h * kHeadDim, it.x);
+    mbar_arrive_expect_tx(fb, rows <= 64 ? TILE / 2 : TILE);
+    load_item_tile(smem_u32(sm.v + st * TILE), it, 2 * kHidden + h * kHeadDim, tmQKV, tmQKV64, fb);
 }
 
 __global__ void __launch_bounds__(ATC_THREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmQKV64,
-               bf16 *__restrict__ ctx, const int *__restrict__ seq_start, const int *__restrict__ seq_len, int nseq,
-               int *status, int trigger, unsigned long long wait_ns) {
+               bf16 *__restrict__ ctx, const int4 *__restrict__ groups, const int *__restrict__ n_groups,
+               int max_groups, int *status, int trigger, unsigned long long wait_ns) {
     if (trigger) griddep_launch_dependents();  // the next kernel may take SMs as this grid frees them
     griddep_wait();               // the previous kernel has completed
 
@@ -135,6 +159,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
 
     if (threadIdx.x == 0) {
         sm.misc[0] = *reinterpret_cast<const volatile int *>(status);
+        const int ng = *reinterpret_cast<const volatile int *>(n_groups);
+        sm.misc[1] = ng < 0 ? 0 : (ng > max_groups ? max_groups : ng);
         *sm.abort_flag = 0;
         wait_limit_init(wait_ns);
         for (int i = 0; i < NQK; ++i) mbar_init(smem_u32(&sm.qk_full[i]), 1);
@@ -156,13 +182,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
     }
     __syncthreads();
     if (sm.misc[0] != 0) return;  // an earlier kernel of this forward failed
-    const int total = nseq * kHeads;  // item id = b * 12 + h
+    const int total = sm.misc[1] * kHeads;  // item id = group * 12 + h
     // items of this CTA: id = blockIdx.x + j * gridDim.x, j < n_items
     const int n_items = (int)blockIdx.x < total ? (total - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-    for (int j = threadIdx.x; j < n_items && j < ATC_ITEM_CAP; j += blockDim.x) {
-        const int b = (blockIdx.x + j * gridDim.x) / kHeads;
-        sm.item[j] = make_int2(__ldg(seq_start + b), __ldg(seq_len + b));
-    }
+    for (int j = threadIdx.x; j < n_items && j < ATC_ITEM_CAP; j += blockDim.x)
+        sm.item[j] = groups[(blockIdx.x + j * gridDim.x) / kHeads];
     if (warp == 1) {
         tmem_alloc(smem_u32(sm.tmem_slot), NBUF * TROWS);
         tmem_relinquish();
@@ -181,16 +205,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
             for (; nq < n_items; ++nq) {
                 const int st = nq % NQK;
                 if (!mbar_wait(smem_u32(&sm.s_full[st]), ((nq / NQK) & 1) ^ 1, sm.abort_flag)) break;
-                const int2 it = item_info(sm, nq, seq_start, seq_len);
+                const int4 it = item_info(sm, nq, groups);
                 const int h = (blockIdx.x + nq * gridDim.x) % kHeads;
-                sm.qk_len[st] = it.y;  // read by the issuer once the stage is full
-                // sequences of at most 64 tokens move 64-row tiles
-                const CUtensorMap *tm = it.y <= 64 ? &tmQKV64 : &tmQKV;
+                const int rows = item_rows(it);
+                sm.qk_len[st] = rows;  // read by the issuer once the stage is full
+                // a lone sequence of at most 64 tokens moves 64-row tiles
                 const uint32_t dst = smem_u32(sm.qk + st * 2 * TILE);
                 const uint32_t fb = smem_u32(&sm.qk_full[st]);
-                mbar_arrive_expect_tx(fb, it.y <= 64 ? TILE : 2 * TILE);
-                tma_load_2d(dst, tm, fb, h * kHeadDim, it.x);
-                tma_load_2d(dst + TILE, tm, fb, kHidden + h * kHeadDim, it.x);
+                mbar_arrive_expect_tx(fb, rows <= 64 ? TILE : 2 * TILE);
+                load_item_tile(dst, it, h * kHeadDim, &tmQKV, &tmQKV64, fb);
+                load_item_tile(dst + TILE, it, kHidden + h * kHeadDim, &tmQKV, &tmQKV64, fb);
                 sm.n_issued[0] = nq + 1;
                 if (nq < NV) {
                     issue_v(sm, nq, it, &tmQKV, &tmQKV64);
@@ -259,10 +283,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
             if ((i & 1) != g) continue;
             const int tb = i % NBUF;
             const uint32_t ph = (i / NBUF) & 1;
-            const uint32_t srow = trow + tb * TROWS;
-            const int L = item_info(sm, i, seq_start, seq_len).y;
+            const int4 it = item_info(sm, i, groups);
+            // A pair's second sequence holds rows and keys 64..127: its warps read
+            // scores from column 64 and write P from column 32 (keys 64..127), and
+            // otherwise run as for a sequence of their own.
+            const bool pair = item_pair(it), hi = pair && quad >= 2;
+            const int L = hi ? it.w : it.y;  // keys of this warp's sequence
+            const uint32_t srow = trow + tb * TROWS + (hi ? 64u : 0u);
+            const uint32_t prow = trow + tb * TROWS + (hi ? 32u : 0u);
             const int nch = (L + 31) >> 5;  // 32-key chunks holding valid keys
-            const bool live = quad * 32 < L;  // some row of this warp is a real query
+            const bool live = (hi ? quad * 32 - 64 : quad * 32) < L;  // some row of this warp is a real query
             bool got = mbar_wait(smem_u32(&sm.s_full[tb]), ph, sm.abort_flag);
             got = __all_sync(0xffffffffu, got);
             if (!got) break;
@@ -323,7 +353,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
                             lsum[j & 1] = f2_add(lsum[j & 1], f2_make(p0, p1));
                             pk[j] = pack_bf16x2(p0, p1);
                         }
-                        tmem_st16(srow + cc * 16, pk);
+                        tmem_st16(prow + cc * 16, pk);
+                    }
+                }
+                if (pair) {
+                    // the O product reads P for all 128 keys: the other half's keys
+                    // (and those past this sequence's end) get P = 0
+                    uint32_t z[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) z[j] = 0u;
+                    const uint32_t p0row = trow + tb * TROWS;
+                    for (int cc = 0; cc < 4; ++cc) {
+                        const int rel = cc - (hi ? 2 : 0);  // chunk within this warp's half
+                        if (rel < 0 || rel >= nch) tmem_st16(p0row + cc * 16, z);
                     }
                 }
                 const float2 ls = f2_split(f2_add(lsum[0], lsum[1]));
@@ -345,9 +387,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
             const int tb = i % NBUF;
             const uint32_t ph = (i / NBUF) & 1;
             const int h = id % kHeads;
-            const int2 it = item_info(sm, i, seq_start, seq_len);
-            const int L = it.y, start = it.x;
-            const bool live = quad * 32 < L;
+            const int4 it = item_info(sm, i, groups);
+            // this warp's rows belong to the pair's second sequence (rows 64..127) or
+            // to the item's first (or only) one
+            const bool hi = item_pair(it) && quad >= 2;
+            const int start = hi ? it.z : it.x, n_valid = hi ? it.w : it.y;
+            const int rs = hi ? r - 64 : r;  // row within its sequence
+            const bool live = (hi ? quad * 32 - 64 : quad * 32) < n_valid;
             // p_full (complete before O is) makes the softmax's 1/sum visible here
             bool got = mbar_wait(smem_u32(&sm.o_full[tb]), ph, sm.abort_flag) &&
                        mbar_wait(smem_u32(&sm.p_full[tb]), ph, sm.abort_flag);
@@ -356,7 +402,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
             tc_fence_after();
             // O of item i is complete: its V stage takes the V tile of item i + 4
             if (warp == 10 && lane == 0 && i + NV < n_items) {
-                issue_v(sm, i + NV, item_info(sm, i + NV, seq_start, seq_len), &tmQKV, &tmQKV64);
+                issue_v(sm, i + NV, item_info(sm, i + NV, groups), &tmQKV, &tmQKV64);
                 sm.n_issued[2] = i + 1;
             }
             uint32_t o[2][32];
@@ -370,8 +416,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sm.o_empty[tb]));
-            if (r < L) {
-                uint4 *dst = reinterpret_cast<uint4 *>(ctx + (size_t)(start + r) * kHidden + h * kHeadDim);
+            if (rs < n_valid) {
+                uint4 *dst = reinterpret_cast<uint4 *>(ctx + (size_t)(start + rs) * kHidden + h * kHeadDim);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const uint32_t *x = o[q >> 2] + (q & 3) * 8;
@@ -404,17 +450,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant_
 
 }  // namespace
 
-cudaError_t launch_attention_tc(const CUtensorMap &tmQKV, const CUtensorMap &tmQKV64, bf16 *ctx, const int *seq_start,
-                                const int *seq_len, int nseq, int *status, int num_sms, cudaStream_t s, bool trigger,
-                                unsigned long long wait_ns) {
-    if (nseq <= 0) return cudaSuccess;
+cudaError_t launch_attention_tc(const CUtensorMap &tmQKV, const CUtensorMap &tmQKV64, bf16 *ctx, const int4 *groups,
+                                const int *n_groups, int max_groups, int *status, int num_sms, cudaStream_t s,
+                                bool trigger, unsigned long long wait_ns) {
+    if (max_groups <= 0) return cudaSuccess;
     static std::atomic<unsigned long long> configured{0};
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(attn_tc_kernel), ATC_SMEM, configured);
     if (e != cudaSuccess) return e;
-    const int total = nseq * kHeads;
+    // sized for one group per sequence; CTAs past the groups' items have none
+    const int total = max_groups * kHeads;
     const int grid = total < num_sms ? total : num_sms;
-    return launch_pdl(attn_tc_kernel, dim3(grid), dim3(ATC_THREADS), ATC_SMEM, s, tmQKV, tmQKV64, ctx, seq_start,
-                      seq_len, nseq, status, trigger ? 1 : 0, wait_ns);
+    return launch_pdl(attn_tc_kernel, dim3(grid), dim3(ATC_THREADS), ATC_SMEM, s, tmQKV, tmQKV64, ctx, groups,
+                      n_groups, max_groups, status, trigger ? 1 : 0, wait_ns);
 }
 
 }  // namespace albert

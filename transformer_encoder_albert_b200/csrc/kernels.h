@@ -202,13 +202,18 @@ cudaError_t launch_forward_small(const SmallFwdArgs &a, int grid, cudaStream_t s
 cudaError_t launch_attention_bf16(const bf16 *qkv, bf16 *ctx, const int *seq_start,
                                   const int *seq_len, int nseq, int max_len,
                                   const int *status, cudaStream_t s, bool trigger);
-// Same operation on tcgen05 for max_len <= 128 (one item = one (sequence, head));
-// tmQKV / tmQKV64: bf16 maps of the packed [rows, 3*768] buffer with a {64, 128} /
-// {64, 64} box and the 128-byte swizzle.
+// Same operation on tcgen05 for max_len <= 128.  One item = one (group, head); a
+// group is one sequence, or two sequences of at most kAttnHalfRows tokens placed
+// in the two 64-row halves of one 128-row tile (each query attends only to the
+// keys of its own sequence).  groups[g] = {start, length, partner start, partner
+// length (0: no partner)} for g < *n_groups (device; written by the prep
+// kernels), at most max_groups.  tmQKV / tmQKV64: bf16 maps of the packed
+// [rows, 3*768] buffer with a {64, 128} / {64, 64} box and the 128-byte swizzle.
 constexpr int kAttnTcMaxLen = 128;
+constexpr int kAttnHalfRows = 64;
 // wait_ns: limit of the kernel's bounded waits (0 = kWaitLimitNs, 2 s).
-cudaError_t launch_attention_tc(const CUtensorMap &tmQKV, const CUtensorMap &tmQKV64, bf16 *ctx, const int *seq_start,
-                                const int *seq_len, int nseq, int *status, int num_sms, cudaStream_t s,
+cudaError_t launch_attention_tc(const CUtensorMap &tmQKV, const CUtensorMap &tmQKV64, bf16 *ctx, const int4 *groups,
+                                const int *n_groups, int max_groups, int *status, int num_sms, cudaStream_t s,
                                 bool trigger, unsigned long long wait_ns = 0);
 // Same operation on tcgen05 for 128 < max_len <= 512 (one item = one (sequence,
 // 128-query block, head), the item's scores against all keys held in TMEM);
@@ -223,12 +228,14 @@ cudaError_t launch_attention_f32(const float *qkv, float *ctx, const int *seq_st
 
 // ---------------------------------------------------- prep / embed / output --
 // max_rows: the handle's max_tokens; a larger total sets ALBERT_ERR_SHAPE.
+// Besides the per-sequence rows, both build the attention groups of
+// launch_attention_tc (groups: room for one per sequence; n_groups: one int).
 cudaError_t launch_prep_padded(const uint8_t *mask, int B, int T, int pack, int max_rows,
                                int *seq_start, int *seq_len, int *n_rows, int *status,
-                               cudaStream_t s, bool trigger);
+                               int4 *groups, int *n_groups, cudaStream_t s, bool trigger);
 cudaError_t launch_prep_varlen(const int32_t *cu, int nseq, int max_len, int max_rows,
                                int *seq_start, int *seq_len, int *n_rows, int *status,
-                               cudaStream_t s, bool trigger);
+                               int4 *groups, int *n_groups, cudaStream_t s, bool trigger);
 
 struct EmbedArgs {
     const int64_t *ids;

@@ -43,12 +43,50 @@ __device__ int block_exclusive_scan(const int *rows, int n, int *start, int *sh)
     return total;
 }
 
+// Attention groups (launch_attention_tc): the k-th and (k+1)-th sequences of at
+// most 64 tokens (k even, in batch order) share one item, as its two 64-row
+// halves; longer sequences, and a last short one without a partner, have an item
+// each.  groups[g] = {start, length, partner start, partner length} (partner
+// length 0: one sequence): the pairs first, then the longer sequences in batch
+// order, then the unpaired short one.  One warp, 32 sequences per step, ranks
+// from ballots.  Warp 0 only; seq_start / seq_len are final and visible to it.
+__device__ void build_attention_groups(const int *seq_start, const int *seq_len, int n, int4 *groups,
+                                       int *n_groups) {
+    const int lane = threadIdx.x & 31;
+    const unsigned below = (1u << lane) - 1u;
+    int n_short = 0;
+    for (int base = 0; base < n; base += 32) {
+        const int b = base + lane;
+        n_short += __popc(__ballot_sync(0xffffffffu, b < n && seq_len[b] <= kAttnHalfRows));
+    }
+    const int n_pairs = n_short >> 1;
+    const int n_long = n - n_short;
+    int2 *half = reinterpret_cast<int2 *>(groups);  // {start, length} halves of the entries
+    int short_seen = 0, long_seen = 0;
+    for (int base = 0; base < n; base += 32) {
+        const int b = base + lane;
+        const int len = b < n ? seq_len[b] : 0, st = b < n ? seq_start[b] : 0;
+        const bool is_short = b < n && len <= kAttnHalfRows, is_long = b < n && !is_short;
+        const unsigned S = __ballot_sync(0xffffffffu, is_short), Lg = __ballot_sync(0xffffffffu, is_long);
+        if (is_short) {
+            const int k = short_seen + __popc(S & below);
+            if (k < 2 * n_pairs) half[k] = make_int2(st, len);  // entry k / 2, half k % 2
+            else groups[n_pairs + n_long] = make_int4(st, len, 0, 0);
+        } else if (is_long) {
+            groups[n_pairs + long_seen + __popc(Lg & below)] = make_int4(st, len, 0, 0);
+        }
+        short_seen += __popc(S);
+        long_seen += __popc(Lg);
+    }
+    if (lane == 0) *n_groups = n_pairs + n_long + (n_short & 1);
+}
+
 // Padded batch: mask[B, T] must hold, per row, a non-empty prefix of non-zero
 // bytes followed only by zeros.  L_b = prefix length.  Packed mode gives
 // sequence b L_b rows, padded mode T rows.
 __global__ void __launch_bounds__(PREP_THREADS)
 prep_padded_kernel(const uint8_t *__restrict__ mask, int B, int T, int pack, int rows_cap,
-                   int *seq_start, int *seq_len, int *n_rows, int *status, int trigger) {
+                   int *seq_start, int *seq_len, int *n_rows, int *status, int4 *groups, int *n_groups, int trigger) {
     if (trigger) griddep_launch_dependents();  // the next kernel may take SMs as this grid frees them
     griddep_wait();               // the previous kernel has completed
 
@@ -77,23 +115,25 @@ prep_padded_kernel(const uint8_t *__restrict__ mask, int B, int T, int pack, int
     }
     __syncthreads();
     if (bad) {
-        if (threadIdx.x == 0) { set_status(status, kStatusMask); *n_rows = 0; }
+        if (threadIdx.x == 0) { set_status(status, kStatusMask); *n_rows = 0; *n_groups = 0; }
         return;
     }
     // rows per sequence, reusing seq_start as the input of the scan
     for (int b = threadIdx.x; b < B; b += PREP_THREADS) seq_start[b] = pack ? seq_len[b] : T;
     __syncthreads();
-    const int total = block_exclusive_scan(seq_start, B, seq_start, sh);
+    const int total = block_exclusive_scan(seq_start, B, seq_start, sh);  // ends with a block barrier
     if (threadIdx.x == 0) {
         *n_rows = total;
         if (total > rows_cap) set_status(status, kStatusShape);
     }
+    if (warp == 0) build_attention_groups(seq_start, seq_len, B, groups, n_groups);
 }
 
 // Packed batch: cu[0] == 0, 1 <= cu[s+1]-cu[s] <= max_len, cu[nseq] <= rows_cap.
 __global__ void __launch_bounds__(PREP_THREADS)
 prep_varlen_kernel(const int32_t *__restrict__ cu, int nseq, int max_len, int rows_cap,
-                   int *seq_start, int *seq_len, int *n_rows, int *status, int trigger) {
+                   int *seq_start, int *seq_len, int *n_rows, int *status, int4 *groups, int *n_groups,
+                   int trigger) {
     if (trigger) griddep_launch_dependents();  // the next kernel may take SMs as this grid frees them
     griddep_wait();               // the previous kernel has completed
 
@@ -118,6 +158,13 @@ prep_varlen_kernel(const int32_t *__restrict__ cu, int nseq, int max_len, int ro
             *n_rows = 0;
         } else {
             *n_rows = total;
+        }
+    }
+    if (threadIdx.x < 32) {
+        if (bad) {
+            if (threadIdx.x == 0) *n_groups = 0;
+        } else {
+            build_attention_groups(seq_start, seq_len, nseq, groups, n_groups);
         }
     }
 }
@@ -245,20 +292,20 @@ __global__ void f32_to_bf16_kernel(const float *src, bf16 *dst, size_t n) {
 
 cudaError_t launch_prep_padded(const uint8_t *mask, int B, int T, int pack, int rows_cap,
                                int *seq_start, int *seq_len, int *n_rows, int *status,
-                               cudaStream_t s, bool trigger) {
+                               int4 *groups, int *n_groups, cudaStream_t s, bool trigger) {
     // The first kernel of a forward: a plain launch, so that it is ordered after
     // every earlier operation of the stream (copies of the inputs included).
     prep_padded_kernel<<<1, PREP_THREADS, 0, s>>>(mask, B, T, pack, rows_cap, seq_start, seq_len, n_rows, status,
-                                                  trigger ? 1 : 0);
+                                                  groups, n_groups, trigger ? 1 : 0);
     return cudaGetLastError();
 }
 
 cudaError_t launch_prep_varlen(const int32_t *cu, int nseq, int max_len, int rows_cap,
                                int *seq_start, int *seq_len, int *n_rows, int *status,
-                               cudaStream_t s, bool trigger) {
+                               int4 *groups, int *n_groups, cudaStream_t s, bool trigger) {
     // first kernel of a forward: plain launch (see launch_prep_padded)
     prep_varlen_kernel<<<1, PREP_THREADS, 0, s>>>(cu, nseq, max_len, rows_cap, seq_start, seq_len, n_rows, status,
-                                                  trigger ? 1 : 0);
+                                                  groups, n_groups, trigger ? 1 : 0);
     return cudaGetLastError();
 }
 
