@@ -53,6 +53,8 @@ def flops_per_class(lengths, arch, rows):
     s2 = float(sum(int(l) ** 2 for l in lengths))
     return {
         "gemm_in_proj": 2.0 * rows * E * H,
+        # the embedding and the input projection in one kernel (its products are the in-projection's)
+        "embed_proj": 2.0 * rows * E * H,
         "gemm_qkv": 2.0 * rows * H * 3 * H,
         "attention": 4.0 * s2 * H,
         "gemm_out_proj_ln": 2.0 * rows * H * H,
@@ -84,6 +86,7 @@ CLASS_SOURCES = {
     "attention_long": ["attention_tc_long.cu", "sm100_ptx.cuh", "kernels.h"],  # 128 < longest <= 512
     "quant": ["fp8.cu", "sm100_ptx.cuh", "kernels.h"],
     "small": ["forward_small.cu", "sm100_ptx.cuh", "kernels.h"],
+    "embed_proj": ["embed_proj.cu", "sm100_ptx.cuh", "kernels.h"],
 }
 
 
@@ -94,6 +97,8 @@ def source_set(cls: str, seq_len: int = 128) -> str:
         return "quant"
     if cls == "small_batch_forward":
         return "small"
+    if cls == "embed_proj":
+        return "embed_proj"
     return "attention" if seq_len <= 128 else "attention_long"
 
 

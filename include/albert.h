@@ -223,10 +223,10 @@ void albert_destroy(albert_handle *h);
  * waits makes healthy forwards fail with ALBERT_ERR_TIMEOUT. */
 int albert_set_wait_limit(albert_handle *h, long long ns);
 
-/* Failure injection for tests of the path above: on later forwards, the GEMM
+/* Failure injection for tests of the path above: on later forwards, the
  * launches of the kernel classes set in class_mask (bit i = class i of
- * albert_profile_name; only the GEMM classes and the small-batch kernel are
- * accepted) run with their TMA
+ * albert_profile_name; only the GEMM classes, the small-batch kernel and the
+ * embedding + input projection kernel are accepted) run with their TMA
  * producer withholding every load, so their first wait on an operand tile can
  * never complete and runs out after the wait limit.  Nothing faults: the
  * forward reports ALBERT_ERR_TIMEOUT through albert_get_status with `out`
@@ -248,7 +248,7 @@ int albert_last_forward_launches(const albert_handle *h);
  * the embedding runs in ONE persistent kernel: a cooperative grid that walks
  * the layer's steps as phases separated by grid barriers (Q|K|V, attention,
  * out-projection, FFN up, FFN down, each over all SMs of the grid, with the
- * intermediate tiles in L2), instead of ~65 per-layer launches ("ALBERT: How Kokoro's
+ * intermediate tiles in L2), instead of ~64 per-layer launches ("ALBERT: How Kokoro's
  * Phoneme Encoder Works", section "Inside One Real ALBERT Layer", steps 2-6,
  * and "2. Cross-layer parameter sharing").  Same results within the stated
  * tolerances; deterministic.  enable: 1 (default) uses it when it applies,

@@ -256,7 +256,7 @@ def test_expired_wait_reports_timeout_and_leaves_output_untouched(w_bf16):
     good = enc.forward(_t(ids), _t(mask)).clone()
     assert enc.status() == 0
     enc.set_wait_limit(200_000)  # 200 us
-    for cls in ("gemm_in_proj", "gemm_qkv", "gemm_ffn_down_ln", "gemm_final_proj"):
+    for cls in ("embed_proj", "gemm_qkv", "gemm_ffn_down_ln", "gemm_final_proj"):
         enc.test_stall([cls])
         out = _sentinel(ids.shape)
         torch.cuda.synchronize()

@@ -74,7 +74,7 @@ def test_small_batch_kernel_agrees_with_per_layer_kernels(w_bf16):
     ids, mask, L = synth.make_batch(wl)
     small, n_small = _forward(w_bf16, ids, mask, small=True)
     layers, n_layers = _forward(w_bf16, ids, mask, small=False)
-    assert n_small == 4 and n_layers == 65
+    assert n_small == 4 and n_layers == 64
     # two bf16 pipelines with different rounding points: within the output bar of each other
     assert float(np.max(np.abs(small - layers))) <= 3e-2
 

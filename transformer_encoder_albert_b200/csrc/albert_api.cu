@@ -24,12 +24,13 @@ namespace {
 
 enum ProfClass {
     kProfPrep = 0, kProfEmbed, kProfGemmIn, kProfGemmQKV, kProfAttention, kProfGemmWoLN,
-    kProfGemmW1Gelu, kProfGemmW2LN, kProfGemmOut, kProfOutput, kProfLayerNorm, kProfSmall, kProfQuant, kProfClasses
+    kProfGemmW1Gelu, kProfGemmW2LN, kProfGemmOut, kProfOutput, kProfLayerNorm, kProfSmall, kProfQuant,
+    kProfEmbedProj, kProfClasses
 };
 const char *kProfNames[kProfClasses] = {
     "prep", "embed_ln", "gemm_in_proj", "gemm_qkv", "attention", "gemm_out_proj_ln",
     "gemm_ffn_up_gelu", "gemm_ffn_down_ln", "gemm_final_proj", "output_rows", "layer_norm_f32",
-    "small_batch_forward", "quant_e4m3"};
+    "small_batch_forward", "quant_e4m3", "embed_proj"};
 
 constexpr int kEventPool = 16384;
 
@@ -329,14 +330,21 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
     ea.row_dst = h->row_dst;
     ea.dst_padded = padded_api;
     ea.status = h->status;
-    ea.trigger = bf ? 1 : 0;  // bf16: the input projection (PDL) follows; fp32: a plain launch
+    ea.trigger = bf ? 1 : 0;  // bf16: a kernel of ours (PDL) follows; fp32: a plain launch
     ea.emb_in = emb_in;
-    LAUNCH(L, kProfEmbed, launch_embed(ea, L.s));
 
     const int D = out_width(h);
     // small batches: everything after the embedding in one kernel
     const long long row_bound = padded_api ? (long long)nseq * T : (long long)nseq * max_len;
-    if (bf && h->small_ok && h->small_enabled && row_bound <= kSmallMaxRows && max_len <= kAttnTcMaxLen) {
+    const bool small = bf && h->small_ok && h->small_enabled && row_bound <= kSmallMaxRows && max_len <= kAttnTcMaxLen;
+    if (bf && !small) {
+        // larger bf16 batches: the embedding and the input projection in one kernel
+        LAUNCH(L, kProfEmbedProj, launch_embed_proj(h->tm_win, ea, h->b_in, static_cast<bf16 *>(h->X), h->num_sms,
+                                                    L.s, h->wait_ns, (h->stall_mask >> kProfEmbedProj) & 1u));
+    } else {
+        LAUNCH(L, kProfEmbed, launch_embed(ea, L.s));
+    }
+    if (small) {
         const auto &W = h->grp[0];
         const auto &E1 = h->ex[c.n_exec > 1 ? 1 : 0];
         SmallFwdArgs s{};
@@ -367,9 +375,6 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
     }
     if (bf) {
         int rc;
-        if ((rc = gemm_bf16(L, kProfGemmIn, kEpiBias, h->tm_E, h->tm_win, h->t32_X, h->t32_X,
-                            gemm_args(h, kHidden, kEmb, h->b_in, nullptr, 0))))
-            return rc;
         for (int l = 0; l < c.n_exec; ++l) {
             const auto &W = h->grp[group_of(c, l)];                  // this execution's weights
             const auto &Wp = h->grp[group_of(c, l > 0 ? l - 1 : 0)];  // the previous execution's (its LN2)
@@ -1002,7 +1007,7 @@ int albert_test_stall(albert_handle *h, int class_mask) {
     if (!h) return ALBERT_ERR_NULL;
     const unsigned gemm_classes = (1u << kProfGemmIn) | (1u << kProfGemmQKV) | (1u << kProfGemmWoLN) |
                                   (1u << kProfGemmW1Gelu) | (1u << kProfGemmW2LN) | (1u << kProfGemmOut) |
-                                  (1u << kProfSmall);
+                                  (1u << kProfSmall) | (1u << kProfEmbedProj);
     if ((unsigned)class_mask & ~gemm_classes) return ALBERT_ERR_CONFIG;
     if (class_mask && h->cfg.dtype == ALBERT_FP32) return ALBERT_ERR_CONFIG;  // the fp32 kernels never wait
     h->stall_mask = (unsigned)class_mask;

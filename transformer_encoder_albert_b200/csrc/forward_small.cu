@@ -11,7 +11,7 @@
 //   Y  = X W_out^T + b_out  (or the hidden states when out_dim == 0).
 // With at most 128 rows every GEMM is a single 128-row tile, so the per-layer
 // kernels of the large-batch path leave most SMs idle and the forward is the
-// sum of ~65 launch latencies.  Here a cooperative grid of G CTAs (one per SM,
+// sum of ~64 launch latencies.  Here a cooperative grid of G CTAs (one per SM,
 // all resident) runs the forward as a sequence of phases separated by grid
 // barriers; inside a phase each CTA takes jobs round robin:
 //   in-proj     12 jobs: a 64-column tile of X (K = 128);

@@ -257,6 +257,13 @@ struct EmbedArgs {
     const float *emb_in;  // non-null: rows [n_rows, 128] fp32 taken as E (no gather, no LayerNorm)
 };
 cudaError_t launch_embed(const EmbedArgs &a, cudaStream_t s);
+// The embedding and the input projection in one kernel (bf16): X = E W_in^T + b_in
+// with E = the rows launch_embed would write, kept in shared memory (a.E and
+// a.out_f32 unused).  tmWin: W_in [768, 128] bf16 with a {64, 128} box and the
+// 128-byte swizzle; a.rows_cap a multiple of 128; X: [rows_cap, 768] bf16.
+// withhold_w (failure-path tests): W_in is never loaded, so the wait for it runs out.
+cudaError_t launch_embed_proj(const CUtensorMap &tmWin, const EmbedArgs &a, const float *b_in, bf16 *X, int num_sms,
+                              cudaStream_t s, unsigned long long wait_ns = 0, bool withhold_w = false);
 // out[b][d][t] = t < seq_len[b] ? src[(b*T + t)*D + d] : 0 (elem_bytes 2 or 4),
 // the last kernel of a forward with the transposed output layout.
 cudaError_t launch_transpose_out(const void *src, void *out, int B, int T, int D, int elem_bytes,
