@@ -425,7 +425,11 @@ def measure_workload(args, ctx, name, padded, graph_mode, extras):
             raise SystemExit(f"device status {st}")
         return {"ncu_forwards": args.ncu_forwards, "workload": wl.name, "tokens": n_tok}
 
-    # which kernel dominates: a short all-class profile before the timed region
+    # which kernel dominates: a short all-class profile before the timed region, after
+    # one untimed forward (a kernel's first launch loads its module, which the event
+    # pair around that launch would count)
+    enc.forward(ids_d, mask_d, out)
+    torch.cuda.synchronize()
     enc.profile(None)
     for _ in range(3):
         enc.forward(ids_d, mask_d, out)

@@ -393,6 +393,25 @@ def test_invalid_id_leaves_output_untouched(w_bf16):
     enc.close()
 
 
+def test_invalid_id_small_batch_path(w_bf16):
+    """The same rejection on the small-batch path (standalone embedding kernel in
+    front of the persistent forward) as on the fused embedding + projection kernel
+    above."""
+    wl = synth.WORKLOADS["b1_T64_latency"]
+    ids, mask, L = synth.make_batch(wl)
+    enc = tea.Encoder(w_bf16, A, max_tokens=wl.B * wl.T)
+    enc.set_small_batch_kernel(True)
+    good = enc.forward(_t(ids), _t(mask)).clone()
+    ids_bad = ids.copy()
+    ids_bad[0, int(L[0]) // 2] = 178
+    out = _sentinel(ids.shape)
+    tea.albert_forward(enc.h, _t(ids_bad), _t(mask), out)
+    assert enc.status() == 4  # ALBERT_ERR_ID
+    assert torch.all(out == 3.25)
+    assert torch.equal(enc.forward(_t(ids), _t(mask)), good)
+    enc.close()
+
+
 def test_bad_masks_are_rejected(w_bf16):
     wl = synth.WORKLOADS["b8_T128"]
     ids, mask, L = synth.make_batch(wl)
