@@ -1,9 +1,11 @@
 // gemm_tcgen05.cu -- persistent BF16 GEMM for sm_100a: Y = epi(A W^T + bias).
 //
-// The dense contractions of the encoder (the 128->768 input projection, the
-// fused Q|K|V projection, the attention output projection, both FFN matrices
-// and the 768->512 final projection; "ALBERT: How Kokoro's Phoneme Encoder
-// Works", section "Inside One Real ALBERT Layer", steps 2-6) all run here.
+// The dense contractions of the encoder (the fused Q|K|V projection, the
+// attention output projection, both FFN matrices and the 768->512 final
+// projection; "ALBERT: How Kokoro's Phoneme Encoder Works", section "Inside One
+// Real ALBERT Layer", steps 3-6) run here; the 128->768 input projection (step
+// 2) runs inside the embedding kernel (embed_proj.cu) and, through the test
+// entry, here as well.
 // A linear layer is y_j = b_j + sum_i x_i W_{j,i} with W stored [out, in]
 // ("Qwen3-TTS and Kokoro", section A), i.e. both operands are K-major.
 //

@@ -1,5 +1,7 @@
-// prep_embed.cu -- batch preparation, the three-table embedding + LayerNorm, and
-// the output-side kernels (padding rows, row scatter).
+// prep_embed.cu -- batch preparation (rows per sequence, the attention groups),
+// the standalone three-table embedding + LayerNorm (small batches and the fp32
+// path; larger bf16 batches use embed_proj.cu), and the output-side kernels
+// (padding rows, row scatter).
 //
 // Embedding ("ALBERT: How Kokoro's Phoneme Encoder Works", section "Inside One
 // Real ALBERT Layer", step 1; section "1. Factorized embedding" for the table
