@@ -6,10 +6,9 @@
 //     E = LN_128(word[id] + pos[t] + type[0]; gamma, beta, eps)
 //     X = E W_in^T + b_in                         (128 -> 768)
 // Each CTA takes 128-row blocks of the packed rows.  Its eight warps gather and
-// normalize the block's embedding rows (one warp per row, four features per
-// lane, as the standalone embedding kernel does) straight into shared memory, in
-// the 128-byte-swizzled K-major layout the tensor core reads, so E never goes
-// to global memory.  One thread then issues the products against W_in, which
+// normalize the block's embedding rows (sixteen rows per warp, four at a time,
+// four features per lane) straight into shared memory, in the 128-byte-swizzled
+// K-major layout the tensor core reads, so E never goes to global memory.  One thread then issues the products against W_in, which
 // every CTA loads once by TMA (192 KB, resident for all of its blocks) before
 // waiting on the previous kernel: two passes of M=128 x N=256 x K=128 tcgen05
 // products into tensor memory (output columns 0..511, then 512..767), each read
