@@ -93,25 +93,40 @@ embed_proj_kernel(const __grid_constant__ CUtensorMap tmW, const EmbedArgs a, co
 
     for (int rb = blockIdx.x; ok && rb * 128 < n_rows; rb += gridDim.x) {
         // ---- E rows of this block into shared memory: 16 per warp ----
-        // Lane i < 16 resolves row i of the warp (sequence, position, id) with
-        // its own search, so the 16 rows' dependent loads overlap; the rows are
-        // then gathered and normalized four at a time.
+        // The warp finds the sequence of its first row with a 32-way search (one
+        // load per lane and level instead of a chain of dependent loads), then
+        // lane i < 16 takes row i: its sequence is that one plus the sequences
+        // that start within the sixteen rows, counted from the next 16 starts.
         const int r0 = rb * 128 + warp * 16;
+        int b0 = 0;
+        {
+            int lo = 0, n = a.nseq;  // the answer lies in [lo, lo + n)
+            while (n > 1) {
+                const int step = (n + 31) / 32;
+                const int k = lo + lane * step;
+                const bool le = lane * step < n && __ldg(a.seq_start + k) <= r0;
+                const unsigned m = __ballot_sync(0xffffffffu, le);  // lane 0 always (seq_start[lo] <= r0)
+                const int h = 31 - __clz(m);
+                lo += h * step;
+                n = min(step, n - h * step);
+            }
+            b0 = lo;
+        }
+        const int nb = b0 + 1 + (lane & 15);
+        const int next_start = nb < a.nseq ? __ldg(a.seq_start + nb) : 0x7fffffff;
         int my_t = 0, my_dst = -1;
         long long my_id = 0;
         {
             const int r = r0 + (lane & 15);
+            int b = b0;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) b += __shfl_sync(0xffffffffu, next_start, j) <= r ? 1 : 0;
             if (r < n_rows) {
-                int lo = 0, hi = a.nseq - 1;
-                while (lo < hi) {
-                    const int mid = (lo + hi + 1) >> 1;
-                    if (__ldg(a.seq_start + mid) <= r) lo = mid; else hi = mid - 1;
-                }
-                my_t = r - __ldg(a.seq_start + lo);
-                const bool valid = my_t < __ldg(a.seq_len + lo);
-                my_dst = valid ? (a.dst_padded ? lo * a.T + my_t : r) : -1;
+                my_t = r - __ldg(a.seq_start + b);
+                const bool valid = my_t < __ldg(a.seq_len + b);
+                my_dst = valid ? (a.dst_padded ? b * a.T + my_t : r) : -1;
                 if (!a.emb_in) {
-                    my_id = a.ids_padded ? a.ids[(size_t)lo * a.T + my_t] : a.ids[r];
+                    my_id = a.ids_padded ? a.ids[(size_t)b * a.T + my_t] : a.ids[r];
                     if (my_id < 0 || my_id >= a.vocab) {
                         if (valid && lane < 16) set_status(a.status, kStatusId);
                         my_id = 0;  // padding slot: any id; its row never reaches a valid output
@@ -224,28 +239,45 @@ embed_proj_kernel(const __grid_constant__ CUtensorMap tmW, const EmbedArgs a, co
             }
             tc_fence_after();
             // ---- epilogue: + b_in, bf16, rows of X ----
+            // (chunk c + 1's accumulator and bias load while chunk c is processed)
             const int r = rb * 128 + (warp & 3) * 32 + lane;
             const int ncol = pass ? 128 : 256;  // TMEM columns per warp in this pass
-            for (int c = 0; c < ncol; c += 32) {
-                const int tcol = half * ncol + c;
-                const int col = pass * 512 + tcol;
-                uint32_t v[32];
-                tmem_ld32(tmem_base + lanes + tcol, v);
-                tmem_ld_wait();
-                if (r < n_rows) {
-                    uint32_t pk[16];
+            const int nch = ncol / 32;
+            uint32_t v[2][32];
+            float4 bv[2][8];
+            auto fetch = [&](int c, int slot) {
+                const int tcol = half * ncol + c * 32;
+                tmem_ld32(tmem_base + lanes + tcol, v[slot]);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 bb = __ldg(reinterpret_cast<const float4 *>(b_in + col) + q);
-                        pk[2 * q] = pack_bf16x2(__uint_as_float(v[4 * q]) + bb.x, __uint_as_float(v[4 * q + 1]) + bb.y);
-                        pk[2 * q + 1] =
-                            pack_bf16x2(__uint_as_float(v[4 * q + 2]) + bb.z, __uint_as_float(v[4 * q + 3]) + bb.w);
+                for (int q = 0; q < 8; ++q)
+                    bv[slot][q] = __ldg(reinterpret_cast<const float4 *>(b_in + pass * 512 + tcol) + q);
+            };
+            fetch(0, 0);
+#pragma unroll 1
+            for (int c = 0; c < nch; c += 2) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    tmem_ld_wait();
+                    if (c + e + 1 < nch) fetch(c + e + 1, e ^ 1);
+                    const int col = pass * 512 + half * ncol + (c + e) * 32;
+                    if (r < n_rows) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 bb = bv[e][q];
+                            pk[2 * q] = pack_bf16x2(__uint_as_float(v[e][4 * q]) + bb.x,
+                                                    __uint_as_float(v[e][4 * q + 1]) + bb.y);
+                            pk[2 * q + 1] = pack_bf16x2(__uint_as_float(v[e][4 * q + 2]) + bb.z,
+                                                        __uint_as_float(v[e][4 * q + 3]) + bb.w);
+                        }
+                        uint4 *dst = reinterpret_cast<uint4 *>(X + (size_t)r * kHidden + col);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
                     }
-                    uint4 *dst = reinterpret_cast<uint4 *>(X + (size_t)r * kHidden + col);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
                 }
             }
+            tmem_ld_wait();
             // the TMEM columns (next pass) and E (next block) are free once every warp is here
             tc_fence_before();
             __syncthreads();
