@@ -32,6 +32,15 @@ def test_gemm_classes_share_a_digest_and_attention_differs():
     assert bench.source_set("quant_e4m3") == "quant" and bench.source_set("small_batch_forward") == "small"
     assert bench.sources_digest("quant_e4m3") != bench.sources_digest("small_batch_forward")
     assert bench.source_set("attention", 512) == "attention_long"
+    # the fused embedding + input projection kernel is keyed by its own file
+    assert bench.source_set("embed_proj") == "embed_proj"
+    assert bench.sources_digest("embed_proj") not in (bench.sources_digest("gemm_qkv"), bench.sources_digest("attention"))
+
+
+def test_embedding_kernel_counts_the_input_projection_flops():
+    arch = {"hidden": 768, "emb": 128, "ffn": 2048, "out_dim": 512, "n_exec": 12}
+    f = bench.flops_per_class([10, 20], arch, 30)
+    assert f["embed_proj"] == f["gemm_in_proj"] == 2.0 * 30 * 128 * 768
 
 
 def test_long_attention_has_its_own_digest_and_lines(tmp_path, monkeypatch):
