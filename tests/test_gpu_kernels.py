@@ -142,6 +142,31 @@ def test_attention_tcgen05_paired_sequences():
     _attention_case(lengths, seed=22, scale=2.0)
 
 
+def test_attention_tcgen05_item_table_overflow():
+    """More items per CTA than its shared-memory table holds (512): 13,000 sequences
+    of 1..4 tokens pair into 6,500 groups, 78,000 (group, head) items over at most
+    148 CTAs, so items past the table are read from the group array in global
+    memory.  Every row must be finite; a spread sample of sequences (including
+    the last ones, which only the overflow path reaches) is checked against the
+    oracle."""
+    r = np.random.default_rng(31)
+    lengths = [int(x) for x in r.integers(1, 5, 13000)]
+    n = int(sum(lengths))
+    qkv = r.normal(0, 1, (n, 3 * 768))
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    q_dev = _bf16_t(qkv)
+    ctx = torch.empty(n, 768, device="cuda", dtype=torch.bfloat16)
+    assert tea.test_attention(q_dev, torch.tensor(cu, device="cuda"), max(lengths), ctx) == 0
+    got = _np(ctx)
+    assert np.all(np.isfinite(got))
+    q64 = _np(q_dev)
+    for s in list(range(0, 13000, 97)) + list(range(12950, 13000)):
+        rows = slice(cu[s], cu[s + 1])
+        x = q64[rows]
+        ref = oracle.attention(x[:, :768], x[:, 768:1536], x[:, 1536:], np.ones(lengths[s], np.uint8), 12)
+        _close(got[rows], ref, rel=2e-2, what=f"attention seq {s} L={lengths[s]}")
+
+
 @pytest.mark.parametrize("case", ["uniform", "all_short", "boundary"])
 def test_attention_groups_match_definition(case):
     """The device's grouping (warp ballots) equals the plain definition."""
