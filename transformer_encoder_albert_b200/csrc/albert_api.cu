@@ -411,7 +411,7 @@ int run_layers(albert_handle *h, Launch &L, const int64_t *ids, int ids_padded, 
                                                              h->att_groups, h->n_att_groups, nseq, h->status,
                                                              h->num_sms, L.s, true, h->wait_ns));
             } else if (max_len <= kAttnTcLongMaxLen) {
-                LAUNCH(L, kProfAttention, launch_attention_tc_long(h->tm_QKV, static_cast<bf16 *>(h->C), h->seq_start,
+                LAUNCH(L, kProfAttention, launch_attention_tc_long(h->tm_QKV, h->tm_QKV64, static_cast<bf16 *>(h->C), h->seq_start,
                                                                   h->seq_len, nseq, h->status, h->num_sms, L.s, true,
                                                                   h->wait_ns));
             } else {
@@ -1153,7 +1153,7 @@ int albert_test_attention(const void *qkv, const int32_t *cu_seqlens, int nseq, 
                 e = launch_attention_tc(tm, tm64, static_cast<bf16 *>(ctx), groups, n_groups, nseq, status, sms, s,
                                         false);
             else
-                e = launch_attention_tc_long(tm, static_cast<bf16 *>(ctx), seq_start, seq_len, nseq, status, sms, s,
+                e = launch_attention_tc_long(tm, tm64, static_cast<bf16 *>(ctx), seq_start, seq_len, nseq, status, sms, s,
                                              false);
         } else {
             e = launch_attention_bf16(static_cast<const bf16 *>(qkv), static_cast<bf16 *>(ctx), seq_start, seq_len, nseq,

@@ -216,12 +216,12 @@ cudaError_t launch_attention_tc(const CUtensorMap &tmQKV, const CUtensorMap &tmQ
                                 const int *n_groups, int max_groups, int *status, int num_sms, cudaStream_t s,
                                 bool trigger, unsigned long long wait_ns = 0);
 // Same operation on tcgen05 for 128 < max_len <= 512 (one item = one (sequence,
-// 128-query block, head), the item's scores against all keys held in TMEM);
-// tmQKV as above.
+// 128-query block, head); keys in 64-key blocks with a running maximum, two items
+// in flight per CTA); tmQKV as above, tmQKV64 with a {64, 64} box.
 constexpr int kAttnTcLongMaxLen = 512;
-cudaError_t launch_attention_tc_long(const CUtensorMap &tmQKV, bf16 *ctx, const int *seq_start, const int *seq_len,
-                                     int nseq, int *status, int num_sms, cudaStream_t s, bool trigger,
-                                     unsigned long long wait_ns = 0);
+cudaError_t launch_attention_tc_long(const CUtensorMap &tmQKV, const CUtensorMap &tmQKV64, bf16 *ctx,
+                                     const int *seq_start, const int *seq_len, int nseq, int *status, int num_sms,
+                                     cudaStream_t s, bool trigger, unsigned long long wait_ns = 0);
 cudaError_t launch_attention_f32(const float *qkv, float *ctx, const int *seq_start,
                                  const int *seq_len, int nseq, int max_len,
                                  const int *status, cudaStream_t s);
