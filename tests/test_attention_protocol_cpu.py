@@ -14,7 +14,7 @@ would see a false completion.  The checks:
   * a phase never mixes arrivals of two items;
   * tensor memory: no product overwrites columns another role still reads
     (scores of an item stay until its softmax is done, O until the output warps
-    have read it, and O of the long kernel only after block 0's scores are read);
+    have read it; in the long kernel, a score buffer only after its P V is issued);
   * every run finishes (no deadlock).
 A planted protocol mistake (checked below) makes these checks fail, so they are
 not vacuous.
@@ -163,93 +163,131 @@ def short_kernel(n_items, seed, planted=False):
 
 
 # ------------------------------------------------------------------ long kernel --
-# One item per (sequence, 128-query block, head); all of its scores in TMEM
-# (key block j in columns 128j..), O in columns 64..127.  Softmax half w owns
-# key blocks w, w+2 and exchanges row maxima with the other half when both own a
-# block.  S of an item waits until the output warps have read the previous O.
-def long_kernel(items, seed, planted=False):
-    NVS = 2
+# Per slot (the two slots of a CTA share no barrier): items of (sequence, 128-query
+# block, head), keys in 64-key blocks numbered b over the slot's items.  The
+# producer loads Q of item n into buffer n % 2 and the {K, V} tiles of block b into
+# stage b % NKV.  The issuer issues S of blocks b and b + 1 ahead, then per block:
+# P V once the softmax has written P (score buffer b % 2), S of block b + 2 into
+# that buffer (after P V in its issue order), the first P V of an item only after
+# the softmax warps have read the previous item's O.  Every softmax warp waits for
+# every phase of pv_done in order (P V of block b - 1 in a rescale of O, else before
+# its arrival on P of block b; an item's last P V before reading O), so a rescale
+# sees O complete through block b - 1.  That wait also orders the warps' P arrivals
+# block by block, and a
+# warp arrives on the first P of an item only after reading the previous O, so the
+# issuer's o_empty wait is implied by its P wait (the kernel keeps it all the same).
+# planted: "s_early" issues S of block b + 2 before P V of block b; "kv_early"
+# loads a K/V stage without waiting for the P V of the block it held; "lazy_pv"
+# waits on pv_done only before a rescale, so a warp can be two phases behind and
+# take an old phase for the one it wants.
+def long_kernel(items, seed, planted=None):
+    NKV = 4
     sim = Sim(seed)
-    for n, c in (("qk_full", 1), ("qk_empty", 1), ("o_full", 1), ("o_empty", 4)):
+    for i in range(2):
+        sim.bar(f"q_full{i}", 1)
+        sim.bar(f"q_empty{i}", 1)
+        sim.bar(f"s_full{i}", 1)
+        sim.bar(f"p_full{i}", 4)
+    for i in range(NKV):
+        sim.bar(f"kv_full{i}", 1)
+        sim.bar(f"kv_empty{i}", 1)
+    for n, c in (("pv_done", 1), ("o_full", 1), ("o_empty", 4)):
         sim.bar(n, c)
-    for s in range(NVS):
-        sim.bar(f"v_full{s}", 1)
-        sim.bar(f"v_empty{s}", 1)
-    for j in range(4):
-        sim.bar(f"s_full{j}", 1)
-        sim.bar(f"p_full{j}", 4)
-    for q in range(4):
-        sim.bar(f"x{q}", 2)
-    st = {"item": None, "o_read": -1, "s0_read": 0, "p": {}, "xmax": set(), "xsum": set()}
+    blocks = [(n, j) for n, (nkb, _) in enumerate(items) for j in range(nkb)]
+    buf = {0: None, 1: None}   # score buffer -> ("s" | "p" | "pv", block)
+    o = {"item": None, "read": -1}
+    written = {}               # block -> warps that have finished it
 
     def producer():
-        for i, (nkb, _) in enumerate(items):
-            yield from sim.wait("qk_empty", (i & 1) ^ 1)
-            sim.commit("qk_full", ("qk", i))
-            yield from sim.wait(f"v_empty{i % NVS}", ((i // NVS) & 1) ^ 1)
-            sim.commit(f"v_full{i % NVS}", ("v", i))
-
-    def mma():
-        par = 0
-        for i, (nkb, _) in enumerate(items):
-            yield from sim.wait("qk_full", i & 1, ("qk", i))
-            if not planted:
-                yield from sim.wait("o_empty", (i & 1) ^ 1, ("e", i - 1) if i else None)
-                assert st["o_read"] == i - 1
-            st["item"] = i
-            for j in range(nkb):
-                sim.commit(f"s_full{j}", ("s", i))
-            sim.commit("qk_empty", ("qk-free", i))
-            yield from sim.wait(f"v_full{i % NVS}", (i // NVS) & 1, ("v", i))
-            for j in range(nkb):  # O products in block order: block 0 first
-                yield from sim.wait(f"p_full{j}", (par >> j) & 1, ("p", i))
-                assert st["p"].get((i, j)) == 4
-                if j == 0:
-                    assert st["s0_read"] == 4 * (i + 1), "O written over block 0's unread scores"
-            sim.commit("o_full", ("o", i))
-            sim.commit(f"v_empty{i % NVS}", ("v-free", i))
-            par ^= (1 << nkb) - 1
-
-    def softmax(half, quad):
-        par = xpar = 0
-        for i, (nkb, live_q) in enumerate(items):
-            live = live_q[quad]
-            for j in range(half, nkb, 2):
-                yield from sim.wait(f"s_full{j}", (par >> j) & 1, ("s", i))
-                assert st["item"] == i
-            if live and nkb >= 2:
-                st["xmax"].add((i, half, quad))
-                sim.bars[f"x{quad}"].arrive(("x", i))
-                yield from sim.wait(f"x{quad}", xpar, ("x", i))
-                xpar ^= 1
-                assert (i, half ^ 1, quad) in st["xmax"]
-            for j in range(half, nkb, 2):
-                assert st["item"] == i, "scores overwritten during the softmax"
-                yield
-                if j == 0:
-                    st["s0_read"] += 1
-                if j + 2 >= nkb and live:
-                    st["xsum"].add((i, half, quad))
-                st["p"][(i, j)] = st["p"].get((i, j), 0) + 1
-                sim.bars[f"p_full{j}"].arrive(("p", i))
-            par ^= (1 << nkb) - 1
-
-    def output(quad):
-        par = 0
-        for i, (nkb, live_q) in enumerate(items):
-            yield from sim.wait("o_full", i & 1, ("o", i))
-            for j in range(nkb):
-                yield from sim.wait(f"p_full{j}", (par >> j) & 1, ("p", i))
-            par ^= (1 << nkb) - 1
-            if live_q[quad]:
-                assert (i, 0, quad) in st["xsum"] and (nkb < 2 or (i, 1, quad) in st["xsum"])
-            assert st["item"] == i, "O overwritten before the output warps read it"
+        for b, (n, j) in enumerate(blocks):
+            if j == 0:
+                yield from sim.wait(f"q_empty{n & 1}", ((n >> 1) & 1) ^ 1)
+                sim.commit(f"q_full{n & 1}", ("q", n))
+            if planted != "kv_early":
+                yield from sim.wait(f"kv_empty{b % NKV}", ((b // NKV) & 1) ^ 1)
+            if b >= NKV:
+                assert sim.bars[f"kv_empty{b % NKV}"].phase > (b - NKV) // NKV, "K/V stage reused before its P V"
+            sim.commit(f"kv_full{b % NKV}", ("kv", b))
             yield
-            sim.bars["o_empty"].arrive(("e", i))
-            if sim.bars["o_empty"].arrived == 0:
-                st["o_read"] = i
 
-    sim.run([producer(), mma()] + [softmax(h, q) for h in (0, 1) for q in range(4)] + [output(q) for q in range(4)])
+    def issuer():
+        state = {"s": 0}
+
+        def issue_s():
+            b = state["s"]
+            n, j = blocks[b]
+            if j == 0:
+                yield from sim.wait(f"q_full{n & 1}", (n >> 1) & 1, ("q", n))
+            yield from sim.wait(f"kv_full{b % NKV}", (b // NKV) & 1, ("kv", b))
+            prev = buf[b & 1]
+            assert prev is None or prev == ("pv", b - 2), ("S over a score buffer still in use", prev, b)
+            buf[b & 1] = ("s", b)
+            sim.commit(f"s_full{b & 1}", ("s", b))
+            if j == items[n][0] - 1:
+                sim.commit(f"q_empty{n & 1}", ("q-free", n))
+            state["s"] += 1
+
+        for _ in range(2):
+            if state["s"] < len(blocks):
+                yield from issue_s()
+        oph = 0
+        for b, (n, j) in enumerate(blocks):
+            if planted == "s_early" and state["s"] < len(blocks) and state["s"] == b + 2:
+                buf[b & 1] = ("pv", b)  # pretends P V was issued
+                yield from issue_s()
+            yield from sim.wait(f"p_full{b & 1}", (b >> 1) & 1, ("p", b))
+            assert written.get(b) == 4, ("P V before every softmax warp wrote P", b, written.get(b))
+            if j == 0:
+                yield from sim.wait("o_empty", oph ^ 1, ("e", n - 1) if n else None)
+                oph ^= 1
+                assert o["read"] == n - 1, ("O of item", n - 1, "overwritten before it was read")
+                o["item"] = n
+            assert buf[b & 1] == ("s", b)
+            buf[b & 1] = ("pv", b)
+            sim.commit(f"kv_empty{b % NKV}", ("kv-free", b))
+            sim.commit("pv_done", ("pv", b))
+            if j == items[n][0] - 1:
+                sim.commit("o_full", ("o", n))
+            yield
+            if state["s"] < len(blocks):
+                yield from issue_s()
+
+    def softmax(q):
+        pvph = oph = 0
+        b = 0
+        for n, (nkb, live_q) in enumerate(items):
+            live = live_q[q]
+            for j in range(nkb):
+                yield from sim.wait(f"s_full{b & 1}", (b >> 1) & 1, ("s", b))
+                assert buf[b & 1] == ("s", b), ("scores gone during the softmax", buf[b & 1], b)
+                seen = j == 0
+                if live and j > 0 and sim.rnd.random() < 0.3:  # a rescale of O
+                    yield from sim.wait("pv_done", pvph, ("pv", b - 1))
+                    pvph ^= 1
+                    seen = True
+                    done = sim.bars["pv_done"].tags  # O complete through block b - 1
+                    assert o["item"] == n and len(done) >= b and done[b - 1] == ("pv", b - 1), \
+                        ("O rescaled before P V of", b - 1)
+                yield
+                if not seen:  # P V of block b - 1, before this warp's arrival on P of block b
+                    if planted != "lazy_pv":
+                        yield from sim.wait("pv_done", pvph, ("pv", b - 1))
+                    pvph ^= 1
+                written[b] = written.get(b, 0) + 1
+                sim.bars[f"p_full{b & 1}"].arrive(("p", b))
+                b += 1
+            yield from sim.wait("o_full", oph, ("o", n))
+            if planted != "lazy_pv":
+                yield from sim.wait("pv_done", pvph, ("pv", b - 1))  # the item's last P V
+            oph ^= 1
+            pvph ^= 1
+            assert o["item"] == n
+            yield
+            sim.bars["o_empty"].arrive(("e", n))
+            if sim.bars["o_empty"].arrived == 0:
+                o["read"] = n
+
+    sim.run([producer(), issuer()] + [softmax(q) for q in range(4)])
 
 
 def _long_items(rnd):
@@ -257,7 +295,7 @@ def _long_items(rnd):
     for _ in range(rnd.randint(0, 10)):
         L = rnd.choice([rnd.randint(1, 128), rnd.randint(129, 512)])
         qb = rnd.randint(0, (L - 1) // 128)
-        items.append(((L + 127) // 128, [qb * 128 + q * 32 < L for q in range(4)]))
+        items.append(((L + 63) // 64, [qb * 128 + q * 32 < L for q in range(4)]))
     return items
 
 
@@ -272,8 +310,10 @@ def test_long_kernel_protocol(seed):
 
 
 def test_planted_mistakes_are_caught():
-    """Reusing a V stage one item early, or issuing S before the previous O was
-    read, must trip the checks for some schedule."""
+    """Reusing a V stage one item early, issuing S before the previous O was read,
+    S over a score buffer before its P V, reusing a K/V stage before its P V, or
+    waiting on pv_done only before a rescale must trip the checks for some
+    schedule."""
     def fails(fn):
         for seed in range(300):
             try:
@@ -284,4 +324,7 @@ def test_planted_mistakes_are_caught():
 
     assert fails(lambda s: short_kernel(12, s, planted=True))
     assert fails(lambda s: short_kernel(12, s, planted="s_early"))
-    assert fails(lambda s: long_kernel([(4, [True] * 4)] * 6, s, planted=True))
+    assert fails(lambda s: long_kernel([(3, [True] * 4)] * 4, s, planted="s_early"))
+    assert fails(lambda s: long_kernel([(3, [True] * 4)] * 4, s, planted="kv_early"))
+    # waiting on pv_done only before a rescale: a warp can fall two phases behind
+    assert fails(lambda s: long_kernel([(8, [True] * 4)] * 4, s, planted="lazy_pv"))

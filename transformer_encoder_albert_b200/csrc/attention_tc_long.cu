@@ -330,6 +330,11 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_cons
                     break;
                 }
                 tc_fence_after();
+                // every warp observes every phase of pv_done in order: P V of block b - 1
+                // before its arrival on P of block b (in the rescale if there is one), an
+                // item's last P V after o_full.  P V of block b cannot complete before
+                // that arrival, so a parity wait is never more than one phase behind.
+                bool seen = j == 0;
                 if (live) {
                     const int Lj = min(KB, L - j * KB), nch = (Lj + 31) >> 5;
                     // the block's scores stay in registers for both passes
@@ -365,6 +370,8 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_cons
                             ok = false;
                             break;
                         }
+                        pvph ^= 1;
+                        seen = true;
                         tc_fence_after();
                         const float sc = raise ? ex2_approx((m_used - m_new) * sl2) : 1.f;
 #pragma unroll 1
@@ -405,19 +412,26 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_cons
                     l += ls.x + ls.y;
                     tmem_st_wait();
                 }
-                // every P V of the slot completes a phase of pv_done; this count stays in
-                // step whether or not the warp waited (block j's P V completes phase b + 1)
-                if (j > 0) pvph ^= 1;
                 tc_fence_before();
+                if (!seen) {
+                    bool d = mbar_wait(smem_u32(sm.pv_done), pvph, abort_flag);
+                    d = __all_sync(0xffffffffu, d);
+                    if (!d) {
+                        ok = false;
+                        break;
+                    }
+                    pvph ^= 1;
+                }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[b & 1]));
             }
             if (!ok) break;
-            pvph ^= 1;  // the item's last P V
             bool got = mbar_wait(smem_u32(sm.o_full), oph, abort_flag);
+            got = got && mbar_wait(smem_u32(sm.pv_done), pvph, abort_flag);  // the item's last P V
             got = __all_sync(0xffffffffu, got);
             if (!got) break;
             oph ^= 1;
+            pvph ^= 1;
             tc_fence_after();
             // O / l as bf16, read 32 columns at a time (packed as they arrive)
             uint32_t ob[32];
