@@ -45,12 +45,13 @@ class Sim:
     def __init__(self, seed):
         self.rnd = random.Random(seed)
         self.bars, self.pending = {}, []
+        self.done = 0  # products known complete: a commit's arrival covers every earlier one
 
     def bar(self, name, count):
         self.bars[name] = Bar(name, count)
 
-    def commit(self, name, tag):
-        self.pending.append((name, tag))
+    def commit(self, name, tag, upto=0):
+        self.pending.append((name, tag, upto))
 
     def wait(self, name, parity, tag=None):
         b = self.bars[name]
@@ -69,7 +70,8 @@ class Sim:
             if self.pending and (not alive or self.rnd.random() < 0.3):
                 name = self.pending[self.rnd.randrange(len(self.pending))][0]
                 k = min(i for i, p in enumerate(self.pending) if p[0] == name)  # in order per barrier
-                n, t = self.pending.pop(k)
+                n, t, upto = self.pending.pop(k)
+                self.done = max(self.done, upto)
                 self.bars[n].arrive(t)
                 continue
             if not alive:
@@ -169,17 +171,19 @@ def short_kernel(n_items, seed, planted=False):
 # stage b % NKV.  The issuer issues S of blocks b and b + 1 ahead, then per block:
 # P V once the softmax has written P (score buffer b % 2), S of block b + 2 into
 # that buffer (after P V in its issue order), the first P V of an item only after
-# the softmax warps have read the previous item's O.  Every softmax warp waits for
-# every phase of pv_done in order (P V of block b - 1 in a rescale of O, else before
-# its arrival on P of block b; an item's last P V before reading O), so a rescale
-# sees O complete through block b - 1.  That wait also orders the warps' P arrivals
-# block by block, and a
+# the softmax warps have read the previous item's O.  After the slot's last S, one
+# commit with no product stands in for the next.  Products complete in issue
+# order, and a commit's arrival means every product issued before it is complete
+# (Sim.done).  A rescale of O on block b waits for S of block b + 1, which follows
+# P V of block b - 1.  Every softmax warp waits for every phase of s_full in order,
+# so none of these parity waits is two phases off; and P of block b - 2 is
+# complete before any arrival on P of block b (one barrier per score buffer).  A
 # warp arrives on the first P of an item only after reading the previous O, so the
 # issuer's o_empty wait is implied by its P wait (the kernel keeps it all the same).
 # planted: "s_early" issues S of block b + 2 before P V of block b; "kv_early"
-# loads a K/V stage without waiting for the P V of the block it held; "lazy_pv"
-# waits on pv_done only before a rescale, so a warp can be two phases behind and
-# take an old phase for the one it wants.
+# loads a K/V stage without waiting for the P V of the block it held; "rescale_s0"
+# rescales O after S of block b instead of b + 1; "no_sentinel" leaves out the
+# commit after the slot's last S.
 def long_kernel(items, seed, planted=None):
     NKV = 4
     sim = Sim(seed)
@@ -191,12 +195,13 @@ def long_kernel(items, seed, planted=None):
     for i in range(NKV):
         sim.bar(f"kv_full{i}", 1)
         sim.bar(f"kv_empty{i}", 1)
-    for n, c in (("pv_done", 1), ("o_full", 1), ("o_empty", 4)):
+    for n, c in (("o_full", 1), ("o_empty", 4)):
         sim.bar(n, c)
     blocks = [(n, j) for n, (nkb, _) in enumerate(items) for j in range(nkb)]
     buf = {0: None, 1: None}   # score buffer -> ("s" | "p" | "pv", block)
     o = {"item": None, "read": -1}
     written = {}               # block -> warps that have finished it
+    pv_seq = {}                # block -> issue number of its P V
 
     def producer():
         for b, (n, j) in enumerate(blocks):
@@ -211,7 +216,7 @@ def long_kernel(items, seed, planted=None):
             yield
 
     def issuer():
-        state = {"s": 0}
+        state = {"s": 0, "seq": 0, "sentinel": False}
 
         def issue_s():
             b = state["s"]
@@ -222,9 +227,10 @@ def long_kernel(items, seed, planted=None):
             prev = buf[b & 1]
             assert prev is None or prev == ("pv", b - 2), ("S over a score buffer still in use", prev, b)
             buf[b & 1] = ("s", b)
-            sim.commit(f"s_full{b & 1}", ("s", b))
+            state["seq"] += 1
+            sim.commit(f"s_full{b & 1}", ("s", b), state["seq"])
             if j == items[n][0] - 1:
-                sim.commit(f"q_empty{n & 1}", ("q-free", n))
+                sim.commit(f"q_empty{n & 1}", ("q-free", n), state["seq"])
             state["s"] += 1
 
         for _ in range(2):
@@ -244,43 +250,38 @@ def long_kernel(items, seed, planted=None):
                 o["item"] = n
             assert buf[b & 1] == ("s", b)
             buf[b & 1] = ("pv", b)
-            sim.commit(f"kv_empty{b % NKV}", ("kv-free", b))
-            sim.commit("pv_done", ("pv", b))
+            state["seq"] += 1
+            pv_seq[b] = state["seq"]
+            sim.commit(f"kv_empty{b % NKV}", ("kv-free", b), state["seq"])
             if j == items[n][0] - 1:
-                sim.commit("o_full", ("o", n))
+                sim.commit("o_full", ("o", n), state["seq"])
             yield
             if state["s"] < len(blocks):
                 yield from issue_s()
+            elif not state["sentinel"] and planted != "no_sentinel":
+                nb = state["s"]
+                sim.commit(f"s_full{nb & 1}", ("s", nb), state["seq"])
+                state["sentinel"] = True
 
     def softmax(q):
-        pvph = oph = 0
+        oph = 0
         b = 0
         for n, (nkb, live_q) in enumerate(items):
             live = live_q[q]
             for j in range(nkb):
                 yield from sim.wait(f"s_full{b & 1}", (b >> 1) & 1, ("s", b))
                 assert buf[b & 1] == ("s", b), ("scores gone during the softmax", buf[b & 1], b)
-                seen = j == 0
                 if live and j > 0 and sim.rnd.random() < 0.3:  # a rescale of O
-                    yield from sim.wait("pv_done", pvph, ("pv", b - 1))
-                    pvph ^= 1
-                    seen = True
-                    done = sim.bars["pv_done"].tags  # O complete through block b - 1
-                    assert o["item"] == n and len(done) >= b and done[b - 1] == ("pv", b - 1), \
-                        ("O rescaled before P V of", b - 1)
+                    nb = b if planted == "rescale_s0" else b + 1
+                    yield from sim.wait(f"s_full{nb & 1}", (nb >> 1) & 1, ("s", nb))
+                    assert o["item"] == n and sim.done >= pv_seq.get(b - 1, 1 << 30), \
+                        ("O rescaled before P V of", b - 1, "completed")
                 yield
-                if not seen:  # P V of block b - 1, before this warp's arrival on P of block b
-                    if planted != "lazy_pv":
-                        yield from sim.wait("pv_done", pvph, ("pv", b - 1))
-                    pvph ^= 1
                 written[b] = written.get(b, 0) + 1
                 sim.bars[f"p_full{b & 1}"].arrive(("p", b))
                 b += 1
             yield from sim.wait("o_full", oph, ("o", n))
-            if planted != "lazy_pv":
-                yield from sim.wait("pv_done", pvph, ("pv", b - 1))  # the item's last P V
             oph ^= 1
-            pvph ^= 1
             assert o["item"] == n
             yield
             sim.bars["o_empty"].arrive(("e", n))
@@ -311,9 +312,9 @@ def test_long_kernel_protocol(seed):
 
 def test_planted_mistakes_are_caught():
     """Reusing a V stage one item early, issuing S before the previous O was read,
-    S over a score buffer before its P V, reusing a K/V stage before its P V, or
-    waiting on pv_done only before a rescale must trip the checks for some
-    schedule."""
+    S over a score buffer before its P V, reusing a K/V stage before its P V, a
+    rescale of O that waits for the wrong S, or no stand-in commit after a slot's
+    last S must trip the checks for some schedule."""
     def fails(fn):
         for seed in range(300):
             try:
@@ -326,5 +327,6 @@ def test_planted_mistakes_are_caught():
     assert fails(lambda s: short_kernel(12, s, planted="s_early"))
     assert fails(lambda s: long_kernel([(3, [True] * 4)] * 4, s, planted="s_early"))
     assert fails(lambda s: long_kernel([(3, [True] * 4)] * 4, s, planted="kv_early"))
-    # waiting on pv_done only before a rescale: a warp can fall two phases behind
-    assert fails(lambda s: long_kernel([(8, [True] * 4)] * 4, s, planted="lazy_pv"))
+    # a rescale after S of its own block, or no commit after the slot's last S
+    assert fails(lambda s: long_kernel([(8, [True] * 4)] * 4, s, planted="rescale_s0"))
+    assert fails(lambda s: long_kernel([(3, [True] * 4)], s, planted="no_sentinel"))

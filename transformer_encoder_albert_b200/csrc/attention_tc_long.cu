@@ -25,7 +25,10 @@
 // of its own item once the pipeline is full.  P_j is written as packed bf16 over
 // the first 32 columns of its score buffer.  A slot's products run in its
 // thread's issue order, so S_{j+2} cannot overwrite P_j before P_j V_j has read
-// it.  After an item's last block its softmax warps read O, scale it by 1 / l
+// it.  A rescale of O while on block j waits for S_{j+1}: the issuer issues it
+// right after P_{j-1} V_{j-1}, and its completion covers every earlier product
+// of the slot (after the slot's last S, a commit with no product stands in for
+// it).  After an item's last block its softmax warps read O, scale it by 1 / l
 // and store it.  A warp whose 32 query rows all lie past the sequence's end
 // skips the arithmetic but takes part in every barrier.  Every wait is bounded
 // (%globaltimer).
@@ -54,7 +57,7 @@ struct SlotSmem {
     uint64_t *q_full, *q_empty;                // [2]
     uint64_t *kv_full, *kv_empty;              // [NKV]
     uint64_t *s_full, *p_full;                 // [2] per score buffer
-    uint64_t *pv_done, *o_full, *o_empty, *drain;
+    uint64_t *o_full, *o_empty, *drain;
 };
 
 __device__ __forceinline__ SlotSmem slot_carve(uint8_t *raw, int slot, uint64_t **bars_end) {
@@ -62,18 +65,17 @@ __device__ __forceinline__ SlotSmem slot_carve(uint8_t *raw, int slot, uint64_t 
     SlotSmem s;
     s.q = p + slot * SLOT_BYTES;
     s.kv = s.q + 2 * QTILE;
-    uint64_t *b = reinterpret_cast<uint64_t *>(p + 2 * SLOT_BYTES) + slot * (4 + 2 * NKV + 8);
+    uint64_t *b = reinterpret_cast<uint64_t *>(p + 2 * SLOT_BYTES) + slot * (4 + 2 * NKV + 7);
     s.q_full = b;
     s.q_empty = b + 2;
     s.kv_full = b + 4;
     s.kv_empty = b + 4 + NKV;
     s.s_full = b + 4 + 2 * NKV;
     s.p_full = s.s_full + 2;
-    s.pv_done = s.s_full + 4;
-    s.o_full = s.s_full + 5;
-    s.o_empty = s.s_full + 6;
-    s.drain = s.s_full + 7;
-    if (bars_end) *bars_end = reinterpret_cast<uint64_t *>(p + 2 * SLOT_BYTES) + 2 * (4 + 2 * NKV + 8);
+    s.o_full = s.s_full + 4;
+    s.o_empty = s.s_full + 5;
+    s.drain = s.s_full + 6;
+    if (bars_end) *bars_end = reinterpret_cast<uint64_t *>(p + 2 * SLOT_BYTES) + 2 * (4 + 2 * NKV + 7);
     return s;
 }
 
@@ -177,15 +179,14 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_cons
                 mbar_init(smem_u32(&t.q_full[i]), 1);
                 mbar_init(smem_u32(&t.q_empty[i]), 1);
                 mbar_init(smem_u32(&t.s_full[i]), 1);
-                // per score buffer: a warp with no live row may reach block j + 1 before
-                // the others finish block j, never block j + 2 (its S follows P_j V)
+                // per score buffer: a warp may arrive for block j + 1 before the others
+                // finish block j, never for block j + 2 (its S follows P_j V)
                 mbar_init(smem_u32(&t.p_full[i]), 4);  // the slot's four softmax warps
             }
             for (int i = 0; i < NKV; ++i) {
                 mbar_init(smem_u32(&t.kv_full[i]), 1);
                 mbar_init(smem_u32(&t.kv_empty[i]), 1);
             }
-            mbar_init(smem_u32(t.pv_done), 1);
             mbar_init(smem_u32(t.o_full), 1);
             mbar_init(smem_u32(t.o_empty), 4);
             mbar_init(smem_u32(t.drain), 1);
@@ -275,6 +276,7 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_cons
                 return true;
             };
             for (int i = 0; i < 2 && gs.has && ok; ++i) ok = issue_s();
+            bool sentinel = false;  // the commit that stands in for S after the slot's last
             while (ok && gp.has) {
                 ok = mbar_wait(smem_u32(&sm.p_full[gp.b & 1]), (gp.b >> 1) & 1, abort_flag);
                 if (!ok) break;
@@ -296,10 +298,16 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_cons
                                  (gp.j | kk) != 0);
                 }
                 umma_commit(smem_u32(&sm.kv_empty[st]));  // K, V of the block consumed
-                umma_commit(smem_u32(sm.pv_done));
                 if (gp.j == key_blocks(gp.it.L) - 1) umma_commit(smem_u32(sm.o_full));
                 gp.advance(slot, total, seq_start, seq_len);
-                if (gs.has) ok = issue_s();  // into the score buffer P V has just read
+                if (gs.has) {
+                    ok = issue_s();  // into the score buffer P V has just read
+                } else if (!sentinel) {
+                    // no S of block gs.b: its phase of s_full completes once P V of block
+                    // gs.b - 2 has, for a rescale on the slot's last block
+                    umma_commit(smem_u32(&sm.s_full[gs.b & 1]));
+                    sentinel = true;
+                }
             }
             umma_commit(smem_u32(sm.drain));
             mbar_wait_drain(smem_u32(sm.drain), 0);
@@ -311,7 +319,7 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_cons
         const float sl2 = 0.125f * 1.4426950408889634f;
         const uint32_t lanes = (uint32_t)(quad * 32) << 16;
         const uint32_t orow = sbase + lanes + 2 * KB;
-        uint32_t oph = 0, pvph = 0;
+        uint32_t oph = 0;
         int b = 0;  // block counter of the slot (score buffer b & 1)
         SlotCursor cur;
         cur.start();
@@ -330,11 +338,6 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_cons
                     break;
                 }
                 tc_fence_after();
-                // every warp observes every phase of pv_done in order: P V of block b - 1
-                // before its arrival on P of block b (in the rescale if there is one), an
-                // item's last P V after o_full.  P V of block b cannot complete before
-                // that arrival, so a parity wait is never more than one phase behind.
-                bool seen = j == 0;
                 if (live) {
                     const int Lj = min(KB, L - j * KB), nch = (Lj + 31) >> 5;
                     // the block's scores stay in registers for both passes
@@ -360,18 +363,20 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_cons
                     }
                     const float mb = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
                     // raise the running maximum only when this block would exceed it by
-                    // more than 2^8; O and l follow (O needs the slot's P V of block j - 1)
+                    // more than 2^8; O and l follow.  O needs the slot's P V of block b - 1,
+                    // which S of block b + 1 (or the commit after the slot's last S)
+                    // follows in the issuer's order.  This warp has seen that barrier's
+                    // previous phase (block b - 1), and its next needs this warp's arrival
+                    // on P of block b + 1: the parity wait is exact.
                     const bool raise = j == 0 || (mb - m_used) * sl2 > kRescaleLog2;
                     const float m_new = raise ? mb : m_used;
                     if (j > 0 && __any_sync(0xffffffffu, raise)) {
-                        bool d = mbar_wait(smem_u32(sm.pv_done), pvph, abort_flag);
+                        bool d = mbar_wait(smem_u32(&sm.s_full[(b + 1) & 1]), ((b + 1) >> 1) & 1, abort_flag);
                         d = __all_sync(0xffffffffu, d);
                         if (!d) {
                             ok = false;
                             break;
                         }
-                        pvph ^= 1;
-                        seen = true;
                         tc_fence_after();
                         const float sc = raise ? ex2_approx((m_used - m_new) * sl2) : 1.f;
 #pragma unroll 1
@@ -413,25 +418,14 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_cons
                     tmem_st_wait();
                 }
                 tc_fence_before();
-                if (!seen) {
-                    bool d = mbar_wait(smem_u32(sm.pv_done), pvph, abort_flag);
-                    d = __all_sync(0xffffffffu, d);
-                    if (!d) {
-                        ok = false;
-                        break;
-                    }
-                    pvph ^= 1;
-                }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[b & 1]));
             }
             if (!ok) break;
             bool got = mbar_wait(smem_u32(sm.o_full), oph, abort_flag);
-            got = got && mbar_wait(smem_u32(sm.pv_done), pvph, abort_flag);  // the item's last P V
             got = __all_sync(0xffffffffu, got);
             if (!got) break;
             oph ^= 1;
-            pvph ^= 1;
             tc_fence_after();
             // O / l as bf16, read 32 columns at a time (packed as they arrive)
             uint32_t ob[32];
