@@ -97,10 +97,11 @@ def test_gemm_scatter_rows(variant):
     assert np.all(got[untouched] == 7.0)
 
 
-def _attention_case(lengths, fp32=False, seed=0, legacy=False, scale=1.0):
+def _attention_case(lengths, fp32=False, seed=0, legacy=False, scale=1.0, qkv=None):
     r = np.random.default_rng(seed)
     n = int(sum(lengths))
-    qkv = r.normal(0, scale, (n, 3 * 768))
+    if qkv is None:
+        qkv = r.normal(0, scale, (n, 3 * 768))
     cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
     if fp32:
         q_dev = torch.tensor(qkv, dtype=torch.float32, device="cuda")
@@ -204,6 +205,32 @@ def test_attention_tcgen05_long_kernel_peaked_softmax():
     """Scores with a spread of ~16 (QKV ~ N(0, 4)): most probabilities underflow
     far below the row maximum, exercising the exponentials' clamp."""
     _attention_case([500, 129, 384, 257], seed=13, scale=4.0)
+
+
+def _last_key_dominates(lengths, seed):
+    """Q/K/V rows in which, for every head, each query is u + noise and the
+    sequence's last key is 3u (u = +-1 per dimension): its score exceeds every
+    other by about 2^29 in the exponential, so every row raises its running
+    maximum on its last key block."""
+    r = np.random.default_rng(seed)
+    n = int(sum(lengths))
+    qkv = r.normal(0, 1, (n, 3 * 768))
+    u = r.choice([-1.0, 1.0], 768)
+    qkv[:, :768] = u + r.normal(0, 0.25, (n, 768))
+    for end in np.cumsum(lengths):
+        qkv[end - 1, 768:1536] = 3.0 * u
+    return qkv
+
+
+def test_attention_tcgen05_long_kernel_rescale_on_last_block():
+    """Every row rescales O on its last key block.  With one item per slot that
+    block is the slot's last, whose rescale waits for the commit that stands in
+    for the next S; with several items per slot it waits for the next item's
+    first S."""
+    few = [200, 320, 449, 512]              # 156 items over 296 slots
+    _attention_case(few, qkv=_last_key_dominates(few, 31))
+    many = [512] * 30 + [300] * 10 + [129]  # 1,812 items, about six per slot
+    _attention_case(many, qkv=_last_key_dominates(many, 32))
 
 
 def test_attention_mma_sync_kernel_long_sequences():
