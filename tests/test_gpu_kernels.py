@@ -233,6 +233,29 @@ def test_attention_tcgen05_long_kernel_rescale_on_last_block():
     _attention_case(many, qkv=_last_key_dominates(many, 32))
 
 
+def test_attention_tcgen05_long_kernel_item_table_overflow():
+    """More items per CTA than the long kernel's shared-memory table holds (512):
+    3,300 sequences of 129..200 tokens give 79,200 (sequence, query block, head)
+    items, about 535 per CTA over 148, so every CTA takes its last items from the
+    walk over the candidates in global memory.  Every row must be finite; a spread
+    sample of sequences and the last 40 (which only that walk reaches) are checked
+    against the oracle."""
+    r = np.random.default_rng(41)
+    lengths = [int(x) for x in r.integers(129, 201, 3300)]
+    n = int(sum(lengths))
+    g = torch.Generator(device="cuda")
+    g.manual_seed(42)
+    q_dev = torch.randn(n, 3 * 768, generator=g, device="cuda").to(torch.bfloat16)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    ctx = torch.empty(n, 768, device="cuda", dtype=torch.bfloat16)
+    assert tea.test_attention(q_dev, torch.tensor(cu, device="cuda"), max(lengths), ctx) == 0
+    assert bool(torch.isfinite(ctx.float()).all())
+    for s in list(range(0, 3300, 151)) + list(range(3260, 3300)):
+        x = _np(q_dev[cu[s]:cu[s + 1]])
+        ref = oracle.attention(x[:, :768], x[:, 768:1536], x[:, 1536:], np.ones(lengths[s], np.uint8), 12)
+        _close(_np(ctx[cu[s]:cu[s + 1]]), ref, rel=2e-2, what=f"attention seq {s} L={lengths[s]}")
+
+
 def test_attention_mma_sync_kernel_long_sequences():
     _attention_case([129, 256, 300, 512], seed=12, legacy=True)
 

@@ -49,7 +49,8 @@ constexpr int LA_THREADS = 32 * 12;            // producer 0 / 10, issuer 1 / 11
 constexpr uint32_t SLOT_COLS = 192;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int SLOT_BYTES = 2 * QTILE + NKV * 2 * KVTILE;  // 96 KB
-constexpr int LA_SMEM = 1024 + 2 * SLOT_BYTES + 512;
+constexpr int LA_ITEM_CAP = 512;               // items of a CTA kept in shared memory
+constexpr int LA_SMEM = 1024 + 2 * SLOT_BYTES + 512 + LA_ITEM_CAP * 16;
 static_assert(LA_SMEM <= 232448, "shared memory per CTA");
 
 struct SlotSmem {
@@ -60,8 +61,12 @@ struct SlotSmem {
     uint64_t *o_full, *o_empty, *drain;
 };
 
+__device__ __forceinline__ uint8_t *smem_base(uint8_t *raw) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+}
+
 __device__ __forceinline__ SlotSmem slot_carve(uint8_t *raw, int slot, uint64_t **bars_end) {
-    uint8_t *p = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *p = smem_base(raw);
     SlotSmem s;
     s.q = p + slot * SLOT_BYTES;
     s.kv = s.q + 2 * QTILE;
@@ -107,18 +112,46 @@ __device__ __forceinline__ bool next_long_item(int &id, int total, const int *__
 
 __device__ __forceinline__ int key_blocks(int L) { return (L + KB - 1) / KB; }
 
-// The items of one slot: the CTA's items k with k % 2 == slot.
+// The CTA's first LA_ITEM_CAP items (h, qb, L, start), built in shared memory
+// before the roles start: walking the candidates through global memory at every
+// item boundary put a chain of dependent loads on each role's path.  resume is
+// the candidate index of the first item past the table, or -1 if there is none.
+struct ItemTable {
+    const int4 *tab;
+    int n, resume;
+};
+
+// The items of one slot: the CTA's items k with k % 2 == slot, from the table,
+// then (past it) from the candidates in global memory.
 struct SlotCursor {
-    int id, k;
-    __device__ void start() {
-        id = blockIdx.x;
-        k = 0;
+    ItemTable t;
+    int k;      // next table index of this slot
+    int id, c;  // past the table: next candidate id and the CTA item index it would get
+    __device__ void start(int slot, const ItemTable &tb) {
+        t = tb;
+        k = slot;
+        id = -1;
+        c = 0;
     }
     __device__ bool next(int slot, int total, const int *seq_start, const int *seq_len, LongItem &it) {
-        LongItem t;
-        while (next_long_item(id, total, seq_start, seq_len, t)) {
-            if ((k++ & 1) == slot) {
-                it = t;
+        if (k < t.n) {
+            const int4 e = t.tab[k];
+            k += 2;
+            it.h = e.x;
+            it.qb = e.y;
+            it.L = e.z;
+            it.start = e.w;
+            return true;
+        }
+        if (t.resume < 0) return false;
+        if (id < 0) {
+            id = blockIdx.x + t.resume * gridDim.x;
+            c = t.n;
+        }
+        LongItem u;
+        while (next_long_item(id, total, seq_start, seq_len, u)) {
+            if ((c++ & 1) == slot) {
+                it = u;
                 return true;
             }
         }
@@ -134,8 +167,8 @@ struct SlotBlocks {
     LongItem it;
     bool has;
     int j, n, b;
-    __device__ void start(int slot, int total, const int *seq_start, const int *seq_len) {
-        cur.start();
+    __device__ void start(int slot, int total, const int *seq_start, const int *seq_len, const ItemTable &tb) {
+        cur.start(slot, tb);
         has = cur.next(slot, total, seq_start, seq_len, it);
         j = 0;
         n = 0;
@@ -199,6 +232,47 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_cons
     }
     __syncthreads();
     if (misc[0] != 0) return;  // an earlier kernel of this forward failed
+    const int total = nseq * LKB * kHeads;
+    ItemTable items;
+    {
+        // candidates blockIdx.x + c * gridDim.x, c = 0 .. ncand - 1, compacted in order:
+        // per chunk of LA_THREADS candidates, warp ballots, then the warps' counts
+        int4 *tab = reinterpret_cast<int4 *>(smem_base(smem_raw) + 2 * SLOT_BYTES + 512);
+        int *wcount = misc + 4;  // [LA_THREADS / 32]
+        const int ncand = total > (int)blockIdx.x ? (total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+        int found = 0;
+        for (int c0 = 0; c0 < ncand; c0 += LA_THREADS) {
+            const int c = c0 + threadIdx.x;
+            int4 e = make_int4(0, 0, 0, 0);
+            bool valid = false;
+            if (c < ncand) {
+                const int id = blockIdx.x + c * gridDim.x;
+                const int sb = id / (LKB * kHeads), rem = id - sb * (LKB * kHeads);
+                const int qb = rem / kHeads;
+                // lengths are validated against max_len <= 512 before this kernel runs;
+                // the clamp only keeps every tile in bounds regardless
+                const int L = min(__ldg(seq_len + sb), LKB * LQ);
+                valid = qb * LQ < L;
+                if (valid) e = make_int4(rem - qb * kHeads, qb, L, __ldg(seq_start + sb));
+            }
+            const unsigned bal = __ballot_sync(0xffffffffu, valid);
+            if (lane == 0) wcount[warp] = __popc(bal);
+            __syncthreads();
+            int before = found, chunk = 0;
+            for (int w = 0; w < LA_THREADS / 32; ++w) {
+                before += w < warp ? wcount[w] : 0;
+                chunk += wcount[w];
+            }
+            const int rank = before + __popc(bal & ((1u << lane) - 1));
+            if (valid && rank < LA_ITEM_CAP) tab[rank] = e;
+            if (valid && rank == LA_ITEM_CAP) misc[2] = c;
+            found += chunk;
+            __syncthreads();  // wcount is rewritten by the next chunk
+        }
+        items.tab = tab;
+        items.n = min(found, LA_ITEM_CAP);
+        items.resume = found > LA_ITEM_CAP ? misc[2] : -1;
+    }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), 512);
         tmem_relinquish();
@@ -208,13 +282,12 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_cons
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const uint32_t sbase = tmem_base + slot * SLOT_COLS;
-    const int total = nseq * LKB * kHeads;
 
     if (warp == 0 || warp == 10) {
         // ------------------------------------------------------ TMA producer --
         if (lane == 0) {
             SlotBlocks bl;
-            bl.start(slot, total, seq_start, seq_len);
+            bl.start(slot, total, seq_start, seq_len, items);
             int nq = 0;
             while (bl.has) {
                 if (bl.j == 0) {
@@ -253,8 +326,8 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_cons
             const uint32_t idesc_s = idesc_bf16_f32(LQ, KB);
             const uint32_t idesc_o = idesc_bf16_f32(LQ, kHeadDim) | (1u << 16);  // B (= V) MN-major
             SlotBlocks gs, gp;  // next block for S, next block for P V
-            gs.start(slot, total, seq_start, seq_len);
-            gp.start(slot, total, seq_start, seq_len);
+            gs.start(slot, total, seq_start, seq_len, items);
+            gp.start(slot, total, seq_start, seq_len, items);
             bool ok = true;
             uint32_t oph = 0;
             auto issue_s = [&]() -> bool {
@@ -322,7 +395,7 @@ attn_tc_long_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_cons
         uint32_t oph = 0;
         int b = 0;  // block counter of the slot (score buffer b & 1)
         SlotCursor cur;
-        cur.start();
+        cur.start(slot, items);
         LongItem it;
         bool ok = true;
         while (ok && cur.next(slot, total, seq_start, seq_len, it)) {
